@@ -1,0 +1,141 @@
+"""fp64 CPU oracle for the KDA forward pass -- TEST INFRASTRUCTURE ONLY.
+
+Only the test suite, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  It is the independent checker of the
+CUDA library: it shares no code with ``gated_delta_rule_139_b200`` and never
+imports it.
+
+The arithmetic lives in ``kda_oracle.c`` (plain C, fp64, pthreads), built by
+:func:`build` into ``libkda_oracle.so`` next to this file.  It follows the
+delta-rule state update of aiblin.ru, "Kimi K3 -- открытая модель, которая
+обошла закрытых лидеров рынка", section "Как хранить миллион токенов в памяти"
+(partial erase then write of a fixed d_k x d_v state, write strength beta,
+per-channel forget gate alpha clamped to [e^-5, 1]), read as
+
+    S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,
+    o_t = S_t^T q_t.
+
+:func:`recurrent` evaluates that definition token by token; :func:`chunked`
+evaluates the chunkwise reformulation of section "Как распараллелили
+последовательное обновление" of the same page.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "kda_oracle.c")
+_LIB = os.path.join(_HERE, "libkda_oracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile kda_oracle.c with gcc into libkda_oracle.so (in place)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-pthread", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        p, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+        lib.kda_oracle_recurrent.argtypes = [p, p, p, i32, p, p, p, p, i64, i64, i64, i64, i64,
+                                             p, i64, p, i32]
+        lib.kda_oracle_recurrent.restype = i32
+        lib.kda_oracle_chunked.argtypes = [p, p, p, i32, p, p, p, p, i64, i64, i64, i64, i64, i64,
+                                           p, i64, p, i32]
+        lib.kda_oracle_chunked.restype = i32
+        _lib = lib
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _prep(q, k, v, log_alpha, beta, initial_state, cu_seqlens):
+    """Flatten [B,T,H,d] / [T,H,d] inputs to the packed layout the C code reads.
+
+    q, k, v are float32 arrays (exact values) or uint16 arrays holding bf16 bits.
+    Returns (arrays..., cu int64, N, T, H, dk, dv, dtype_code, out_shape_prefix).
+    """
+    q = np.ascontiguousarray(q)
+    k = np.ascontiguousarray(k)
+    v = np.ascontiguousarray(v)
+    if q.dtype == np.float32:
+        code = 0
+    elif q.dtype == np.uint16:
+        code = 1
+    else:
+        raise TypeError("q/k/v must be float32 or uint16 (bf16 bits)")
+    if not (k.dtype == q.dtype and v.dtype == q.dtype):
+        raise TypeError("q, k, v must share one dtype")
+    lead = q.shape[:-2]
+    H, dk = q.shape[-2], q.shape[-1]
+    dv = v.shape[-1]
+    T = int(np.prod(lead))
+    if cu_seqlens is None:
+        if q.ndim == 4:
+            B, Tb = q.shape[0], q.shape[1]
+        else:
+            B, Tb = 1, q.shape[0]
+        cu = np.arange(B + 1, dtype=np.int64) * Tb
+    else:
+        cu = np.asarray(cu_seqlens, dtype=np.int64)
+    N = len(cu) - 1
+    la = np.ascontiguousarray(log_alpha, dtype=np.float32)
+    be = np.ascontiguousarray(beta, dtype=np.float32)
+    s0 = None if initial_state is None else np.ascontiguousarray(initial_state, dtype=np.float32)
+    if la.size != T * H * dk or be.size != T * H or v.size != T * H * dv or k.size != q.size:
+        raise ValueError("inconsistent shapes")
+    if s0 is not None and s0.size != N * H * dk * dv:
+        raise ValueError("initial_state must be [N,H,dk,dv]")
+    return q, k, v, la, be, s0, cu, N, T, H, dk, dv, code, lead
+
+
+def _run(fn_name, q, k, v, log_alpha, beta, initial_state, cu_seqlens, o_tokens, threads,
+         chunk=None):
+    q, k, v, la, be, s0, cu, N, T, H, dk, dv, code, lead = _prep(
+        q, k, v, log_alpha, beta, initial_state, cu_seqlens)
+    o_tokens = T if o_tokens is None else int(o_tokens)
+    o = np.empty((max(o_tokens, 0), H, dv), dtype=np.float64)
+    sf = np.empty((N, H, dk, dv), dtype=np.float64)
+    lib = _load()
+    args = [_ptr(q), _ptr(k), _ptr(v), code, _ptr(la), _ptr(be), _ptr(s0), _ptr(cu), N, T, H,
+            dk, dv]
+    if chunk is not None:
+        args.append(int(chunk))
+    args += [_ptr(o) if o_tokens > 0 else None, o_tokens, _ptr(sf), int(threads)]
+    rc = getattr(lib, fn_name)(*args)
+    if rc != 0:
+        raise ValueError(f"{fn_name} rejected its arguments (code {rc})")
+    if o_tokens == T and len(lead) == 2:
+        o = o.reshape(lead + (H, dv))
+    return o, sf
+
+
+def recurrent(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, o_tokens=None,
+              threads=0):
+    """Token-by-token fp64 evaluation of the KDA recurrence.
+
+    Returns (o, final_state): o is float64 [.., H, d_v] for the first ``o_tokens``
+    packed tokens (all by default), final_state float64 [N, H, d_k, d_v].
+    """
+    return _run("kda_oracle_recurrent", q, k, v, log_alpha, beta, initial_state, cu_seqlens,
+                o_tokens, threads)
+
+
+def chunked(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, chunk=64,
+            o_tokens=None, threads=0):
+    """Chunkwise fp64 reformulation (plain exp(+-g), any chunk size >= 1)."""
+    return _run("kda_oracle_chunked", q, k, v, log_alpha, beta, initial_state, cu_seqlens,
+                o_tokens, threads, chunk=chunk)
