@@ -1,0 +1,370 @@
+#!/usr/bin/env python
+"""Benchmark of the KDA chunked forward (libkda.so) on B200; prints ONE JSON line.
+
+    python bench.py [--gpus N --steps K --warmup W] [--workload prefill_1m]
+    python bench.py --impl reference ...      # the fp64 CPU oracle, timed on host cores
+
+A step is one kda_fwd call over the whole workload (default: the 1M-token
+prefill, B=1, H=8, T=2^20, d_k=d_v=128, bf16 q/k/v, fp32 gates, chunk 64).
+``value`` is Mtokens/s with inputs resident in HBM (tokens counted once, not per
+head); ``e2e`` is the same metric through the host-buffer entry point
+kda_fwd_host with the host->device copy of the inputs and the device->host copy
+of the outputs inside every timed step.  The workload's inputs (12.9 GB) are
+larger than the 126 MB L2, so no flush is needed between steps.
+
+With N GPUs (torchrun, one rank per GPU) every rank runs its own copy of the
+workload (independent problems, no data-path collective): weak scaling, value =
+N * tokens / max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from gated_delta_rule_139_b200.inputs import (WORKLOADS, algorithmic_bytes,  # noqa: E402
+                                              algorithmic_flops, make_inputs, workload)
+
+METRIC = "KDA chunked prefill Mtokens/s on 1 B200; % of bf16 tensor / HBM roofline"
+UNIT = "Mtokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_config(inp, n_gpus):
+    return {"workload": inp.name, "B": inp.B, "T": inp.T, "H": inp.H, "d_k": inp.dk,
+            "d_v": inp.dv, "chunk": inp.chunk, "num_seqs": inp.n_seqs,
+            "tokens_per_gpu": inp.tokens, "qkv_dtype": "bf16" if inp.bf16 else "f32",
+            "gates": "fp32 log_alpha, fp32 beta", "state": "fp32",
+            "l2": "inputs larger than L2 (%.1f GB per step vs 126 MB L2), no flush" %
+                  (algorithmic_bytes(inp) / 1e9),
+            "parallelism": f"dp{n_gpus} (independent problem per GPU)"}
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples (every 100 ms) of one GPU while the timed region runs."""
+
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.uuid = uuid
+        self.proc = None
+        self.path = os.path.join("/tmp", f"kda_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"],
+                    "samples": 0}
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            if self.uuid and self.uuid not in parts[0]:
+                continue
+            rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        loaded = [s for s in sm if mx and s > 0.5 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(
+                    (float(r[3]) for r in rows if r[3].replace(".", "").isdigit()), default=None)}
+
+
+# ------------------------------------------------------------------ oracle baseline
+def oracle_sample_rate(inp_name: str, target_s: float = 15.0, seed: int = 0):
+    """Time the fp64 oracle on a bounded prefix of the workload's recipe."""
+    import oracle
+    spec = dict(WORKLOADS[inp_name])
+    spec.pop("packed", None)
+    spec.pop("T", None)
+    H = spec["H"]
+    probe_T = 1024
+    x = make_inputs(T=probe_T, seed=seed, name=inp_name, **{k: v for k, v in spec.items()
+                                                              if k != "B"}, B=1)
+    t0 = time.perf_counter()
+    oracle.recurrent(x.q, x.k, x.v, x.log_alpha, x.beta, x.initial_state, None, o_tokens=0)
+    rate = probe_T / max(time.perf_counter() - t0, 1e-6)  # tokens/s (all heads)
+    T_s = int(max(probe_T, min(rate * target_s, 1 << 20)))
+    T_s = (T_s // 64) * 64
+    x = make_inputs(T=T_s, seed=seed, name=inp_name, **{k: v for k, v in spec.items()
+                                                          if k != "B"}, B=1)
+    threads = min(len(os.sched_getaffinity(0)), H)
+    t0 = time.perf_counter()
+    oracle.recurrent(x.q, x.k, x.v, x.log_alpha, x.beta, x.initial_state, None, o_tokens=0,
+                     threads=threads)
+    dt = time.perf_counter() - t0
+    return {"value": T_s / dt / 1e6, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"first {T_s} tokens x {H} heads of the {inp_name} recipe "
+                      f"(fp64 token recurrence, {dt:.1f} s)", "seconds": dt}
+
+
+def run_reference(args, rank, world):
+    """The oracle as it stands, on host cores: rank 0 only."""
+    if rank != 0:
+        return
+    import oracle
+    name = args.workload
+    spec = dict(WORKLOADS[name])
+    spec.pop("packed", None)
+    spec.pop("T", None)
+    spec.pop("B", None)
+    H = spec["H"]
+    threads = min(len(os.sched_getaffinity(0)), H)
+    # size each step to ~2 s of oracle work
+    probe = make_inputs(B=1, T=512, seed=0, name=name, **spec)
+    t0 = time.perf_counter()
+    oracle.recurrent(probe.q, probe.k, probe.v, probe.log_alpha, probe.beta, None, None,
+                     o_tokens=0, threads=threads)
+    rate = 512 / max(time.perf_counter() - t0, 1e-6)
+    T_s = max(64, int(rate * 2.0) // 64 * 64)
+    x = make_inputs(B=1, T=T_s, seed=0, name=name, **spec)
+    f = lambda: oracle.recurrent(x.q, x.k, x.v, x.log_alpha, x.beta, x.initial_state, None,
+                                 o_tokens=T_s, threads=threads)
+    for _ in range(args.warmup):
+        f()
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        f()
+        times.append(time.perf_counter() - t0)
+    step = sum(times) / len(times)
+    val = T_s / step / 1e6
+    full = workload_config(x, world)
+    full.update({"workload": name, "T": None, "sampled_T": T_s})
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": full,
+            "cpu_baseline": {"value": val, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": f"first {T_s} tokens x {H} heads of the {name} recipe "
+                                       "per step (fp64 token recurrence)"},
+            "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ traffic record
+def recorded_traffic(kernel_tag: str):
+    """DRAM bytes per launch from a committed ncu summary, if its kernel sources
+    are unchanged since the capture (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f).get(kernel_tag)
+    if not rec:
+        return None
+    h = hashlib.sha256()
+    for src in rec["sources"]:
+        with open(os.path.join(ROOT, src), "rb") as f:
+            h.update(f.read())
+    return rec["bytes_per_launch"] if h.hexdigest() == rec["sha256"] else None
+
+
+# ------------------------------------------------------------------ main arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="prefill_1m", choices=sorted(WORKLOADS))
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    args.warmup = max(args.warmup, 3)
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    import gated_delta_rule_139_b200 as kda
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+        pg = dist
+
+    inp = workload(args.workload, seed=rank)
+    tokens = inp.tokens
+    bf16 = inp.bf16
+
+    # pinned host copies (for e2e) and device-resident copies (for value)
+    def pinned(a):
+        t = torch.from_numpy(a)
+        if bf16 and a.dtype == np.uint16:
+            t = t.view(torch.bfloat16)
+        return t.pin_memory()
+
+    host = {k: (None if getattr(inp, k) is None else pinned(getattr(inp, k)))
+            for k in ("q", "k", "v", "log_alpha", "beta", "initial_state")}
+    alg_bytes = algorithmic_bytes(inp)
+    alg_flops = algorithmic_flops(inp)
+    v_shape = tuple(inp.v.shape)
+    for k_ in ("q", "k", "v", "log_alpha", "beta"):
+        setattr(inp, k_, None)  # the pinned copies are the host data from here on
+    cu_host = inp.cu_seqlens
+    stream = torch.cuda.Stream(dev)
+    with torch.cuda.stream(stream):
+        d = {k: (None if t is None else t.to(dev, non_blocking=True)) for k, t in host.items()}
+        cu_dev = None if cu_host is None else torch.from_numpy(cu_host).to(dev)
+        out = torch.empty(v_shape, dtype=d["q"].dtype, device=dev)
+        fs = torch.empty((inp.n_seqs, inp.H, inp.dk, inp.dv), dtype=torch.float32, device=dev)
+    stream.synchronize()
+
+    def step():
+        kda.kda_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["initial_state"],
+                    cu_dev, 64, out, fs, stream=stream)
+        return kda.last_launch_count()
+
+    for _ in range(args.warmup):
+        step()
+    stream.synchronize()
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    launches = 0
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(uuid) as clk:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            launches += step()
+        ev1.record(stream)
+        stream.synchronize()
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    clocks = clk.summary()
+    if pg:
+        t = torch.tensor([ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms = float(t.item())
+    value = world * tokens / (ms * 1e-3) / 1e6
+
+    # e2e: host buffers through kda_fwd_host, copies inside every step
+    out_h = torch.empty(v_shape, dtype=host["q"].dtype).pin_memory()
+    fs_h = torch.empty((inp.n_seqs, inp.H, inp.dk, inp.dv), dtype=torch.float32).pin_memory()
+    cu_arg = None if cu_host is None else np.ascontiguousarray(cu_host, dtype=np.int32)
+
+    def e2e_step():
+        kda.kda_fwd_host(host["q"], host["k"], host["v"], host["log_alpha"], host["beta"],
+                         host["initial_state"], cu_arg, 64, out_h, fs_h, stream=stream)
+
+    e2e_step()
+    if pg:
+        pg.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    stream.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+    if pg:
+        t = torch.tensor([e2e_ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    nbytes = lambda t: 0 if t is None else t.numel() * t.element_size()
+    h2d = sum(nbytes(t) for t in host.values()) + (0 if cu_arg is None else cu_arg.nbytes)
+    d2h = nbytes(out_h) + nbytes(fs_h)
+
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks, peak_src = load_peaks()
+    achieved = alg_bytes / (ms * 1e-3) / 1e9
+    t_roof = max(alg_bytes / (peaks["hbm_gbs"] * 1e9), alg_flops / (peaks["bf16_tflops"] * 1e12))
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32" if kda.last_path() == "ffma" else "bf16",
+        "data": "synthetic", "config": workload_config(inp, world),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                     "traffic": recorded_traffic(kda.last_path()),
+                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
+                     if peak_src == "measured" else "fallback 6.65 TB/s",
+                     "kernel": kda.last_path(),
+                     "algorithmic_bytes_per_launch": alg_bytes,
+                     "path_roofline_frac": t_roof / (ms * 1e-3)},
+        "e2e": {"value": world * tokens / (e2e_ms * 1e-3) / 1e6, "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms, "steps": args.e2e_steps},
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        cb = oracle_sample_rate(args.workload)
+        cb.pop("seconds", None)
+        line["cpu_baseline"] = cb
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

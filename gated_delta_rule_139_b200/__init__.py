@@ -1,0 +1,178 @@
+"""Python binding of libkda.so -- the KDA chunked forward pass on B200 (sm_100a).
+
+Thin ctypes marshalling around the C ABI of ``include/kda.h``; every step of the
+computation runs in the library's CUDA kernels.  PyTorch provides device memory
+and streams only.  If ``libkda.so`` has not been built this module raises on
+first use: there is no fallback implementation.
+
+    from gated_delta_rule_139_b200 import kda_fwd
+    out, final_state = kda_fwd(q, k, v, log_alpha, beta, initial_state, cu_seqlens)
+
+Shapes (row-major): q, k [B,T,H,d_k]; v [B,T,H,d_v]; log_alpha [B,T,H,d_k] fp32;
+beta [B,T,H] fp32; states [N,H,d_k,d_v] fp32; packed input passes [T,H,*]
+tensors (or B=1) with cu_seqlens int32 [N+1].
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = ["kda_fwd", "kda_fwd_host", "KDAError", "library_path", "load_library",
+           "last_launch_count", "last_path", "STATUS"]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_PKG, "libkda.so")
+
+STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED",
+          3: "KDA_ERR_MISALIGNED", 4: "KDA_ERR_ALIAS", 5: "KDA_ERR_CUDA",
+          6: "KDA_ERR_DEVICE_TIMEOUT"}
+KDA_F32, KDA_BF16 = 0, 1
+
+
+class KDAError(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        self.status = status
+        self.name = STATUS.get(status, f"status {status}")
+        super().__init__(f"{self.name}: {detail}")
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("T", ctypes.c_int32), ("H", ctypes.c_int32),
+                ("d_k", ctypes.c_int32), ("d_v", ctypes.c_int32), ("num_seqs", ctypes.c_int32),
+                ("qkv_dtype", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def load_library():
+    """Load libkda.so (raises if it is missing: build it with ``build.py``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(library_path):
+            raise ImportError(f"{library_path} is missing; run "
+                              "`python -m gated_delta_rule_139_b200.build` first")
+        lib = ctypes.CDLL(library_path)
+        p = ctypes.c_void_p
+        sig = [p, p, p, p, p, p, p, ctypes.c_int32, p, p, ctypes.POINTER(Dims), p]
+        for name in ("kda_fwd", "kda_fwd_host"):
+            fn = getattr(lib, name)
+            fn.argtypes = sig
+            fn.restype = ctypes.c_int
+        lib.kda_status_string.argtypes = [ctypes.c_int]
+        lib.kda_status_string.restype = ctypes.c_char_p
+        lib.kda_last_error.argtypes = []
+        lib.kda_last_error.restype = ctypes.c_char_p
+        lib.kda_last_launch_count.argtypes = []
+        lib.kda_last_launch_count.restype = ctypes.c_int32
+        lib.kda_last_path.argtypes = []
+        lib.kda_last_path.restype = ctypes.c_char_p
+        _lib = lib
+    return _lib
+
+
+def last_launch_count() -> int:
+    """Kernel launches issued by the last kda_fwd call on this thread."""
+    return int(load_library().kda_last_launch_count())
+
+
+def last_path() -> str:
+    """Kernel family of the last kda_fwd call on this thread ("ffma" or "tc")."""
+    return load_library().kda_last_path().decode()
+
+
+def _check(rc: int):
+    if rc != 0:
+        raise KDAError(rc, load_library().kda_last_error().decode())
+
+
+def _dims(q_shape, v_shape, T_override, cu_len, bf16):
+    if len(q_shape) == 4:
+        B, T, H, dk = q_shape
+    elif len(q_shape) == 3:
+        B, (T, H, dk) = 1, q_shape
+    else:
+        raise ValueError("q must be [B,T,H,d_k] or [T,H,d_k]")
+    return Dims(B, T, H, dk, v_shape[-1], max(cu_len - 1, 0) if cu_len else 0,
+                KDA_BF16 if bf16 else KDA_F32)
+
+
+def kda_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, chunk: int = 64,
+            out=None, final_state=None, stream=None, want_final: bool = True):
+    """KDA forward on CUDA tensors; returns (out, final_state or None).
+
+    q/k/v are bf16 or fp32 CUDA tensors; gates and states fp32.  ``stream`` is a
+    torch.cuda.Stream (default: the current stream).  Outputs are allocated when
+    not given.  Runs asynchronously on the stream.
+    """
+    import torch
+
+    lib = load_library()
+    bf16 = q.dtype == torch.bfloat16
+    if not bf16 and q.dtype != torch.float32:
+        raise TypeError("q/k/v must be bfloat16 or float32")
+    for t in (q, k, v, log_alpha, beta):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("inputs must be contiguous CUDA tensors")
+    d = _dims(tuple(q.shape), tuple(v.shape), None,
+              cu_seqlens.numel() if cu_seqlens is not None else 0, bf16)
+    N = d.num_seqs if cu_seqlens is not None else d.B
+    if out is None:
+        out = torch.empty(tuple(q.shape[:-1]) + (d.d_v,), dtype=q.dtype, device=q.device)
+    if final_state is None and want_final:
+        final_state = torch.empty((N, d.H, d.d_k, d.d_v), dtype=torch.float32, device=q.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    ptr = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
+    rc = lib.kda_fwd(ptr(q), ptr(k), ptr(v), ptr(log_alpha), ptr(beta), ptr(initial_state),
+                     ptr(cu_seqlens), int(chunk), ptr(out), ptr(final_state), ctypes.byref(d),
+                     ctypes.c_void_p(stream.cuda_stream))
+    _check(rc)
+    return out, final_state
+
+
+def kda_fwd_host(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
+                 chunk: int = 64, out=None, final_state=None, stream=None,
+                 want_final: bool = True):
+    """KDA forward on HOST numpy arrays (or CPU tensors; pinned memory copies
+    asynchronously).  The library copies inputs in, runs, copies results back
+    and synchronises.  bf16 data is passed as uint16 bit patterns (numpy) or
+    torch.bfloat16 CPU tensors.  Returns (out, final_state or None) on the host.
+    """
+    import numpy as np
+
+    lib = load_library()
+
+    def info(a):
+        if a is None:
+            return None, None, None
+        if isinstance(a, np.ndarray):
+            return a.ctypes.data, a.shape, a.dtype
+        return a.data_ptr(), tuple(a.shape), a.dtype  # torch CPU tensor
+
+    _, qs, qd = info(q)
+    _, vs, _ = info(v)
+    bf16 = str(qd) in ("uint16", "torch.bfloat16")
+    cu_len = 0 if cu_seqlens is None else len(cu_seqlens)
+    d = _dims(tuple(qs), tuple(vs), None, cu_len, bf16)
+    N = d.num_seqs if cu_seqlens is not None else d.B
+    if isinstance(q, np.ndarray):
+        if out is None:
+            out = np.empty(tuple(qs[:-1]) + (d.d_v,), dtype=q.dtype)
+        if final_state is None and want_final:
+            final_state = np.empty((N, d.H, d.d_k, d.d_v), dtype=np.float32)
+        if cu_seqlens is not None:
+            cu_seqlens = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    else:
+        import torch
+        if out is None:
+            out = torch.empty(tuple(qs[:-1]) + (d.d_v,), dtype=q.dtype, pin_memory=q.is_pinned())
+        if final_state is None and want_final:
+            final_state = torch.empty((N, d.H, d.d_k, d.d_v), dtype=torch.float32,
+                                      pin_memory=q.is_pinned())
+    h = lambda a: None if a is None else ctypes.c_void_p(info(a)[0])
+    s = None if stream is None else ctypes.c_void_p(stream.cuda_stream)
+    rc = lib.kda_fwd_host(h(q), h(k), h(v), h(log_alpha), h(beta), h(initial_state),
+                          h(cu_seqlens), int(chunk), h(out), h(final_state), ctypes.byref(d), s)
+    _check(rc)
+    return out, final_state

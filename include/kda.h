@@ -1,0 +1,130 @@
+/*
+ * kda.h -- C ABI of libkda.so: the Kimi Delta Attention (KDA) chunked forward
+ * pass on NVIDIA B200 (sm_100a).
+ *
+ * The operation (aiblin.ru, "Kimi K3 -- открытая модель, которая обошла
+ * закрытых лидеров рынка", section "Как хранить миллион токенов в памяти"):
+ * a fixed-size state S (d_k x d_v, fp32) replaces the KV cache and is rewritten
+ * at every token -- part of the old content is erased, then new content is
+ * written with strength beta in (0,1); a per-channel forget coefficient alpha,
+ * clamped to [e^-5, 1], decays the old content.  Read as
+ *
+ *     alpha_t = exp(clamp(log_alpha_t, -5, 0))                (d_k vector)
+ *     S_t     = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T
+ *     o_t     = S_t^T q_t
+ *
+ * The library evaluates it chunkwise (section "Как распараллелили
+ * последовательное обновление" of the same page): all tokens of a 64-token
+ * chunk in parallel, then the state passed from chunk to chunk; long sequences
+ * are additionally cut into segments whose state transitions (a local state
+ * plus a d_k x d_k transition matrix, S_out = M S_in + B) are computed in
+ * parallel on one GPU and chained by a scan.  No q scaling, no k
+ * normalisation, no beta or gate activation happens inside: the caller passes
+ * k, beta and log_alpha as the recurrence consumes them (log_alpha is clamped
+ * inside).
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return codes.  Every argument error is detected on the host before any
+ * launch; such a call writes nothing. */
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1,    /* null/negative/inconsistent argument, host pointer where a
+                                   device pointer is required, bad cu_seqlens length        */
+    KDA_ERR_UNSUPPORTED = 2,    /* valid but not implemented: d_k/d_v not in {64,128}, chunk != 64 */
+    KDA_ERR_MISALIGNED = 3,     /* a tensor pointer is not 16-byte aligned                   */
+    KDA_ERR_ALIAS = 4,          /* out or final_state overlaps an input (final_state ==
+                                   initial_state exactly is allowed)                         */
+    KDA_ERR_CUDA = 5,           /* a CUDA runtime call or kernel launch failed               */
+    KDA_ERR_DEVICE_TIMEOUT = 6  /* a bounded inter-block wait on the device gave up; the
+                                   outputs of that call are undefined                        */
+} kda_status;
+
+typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype;
+
+/* Shapes.  Without cu_seqlens: B sequences of T tokens each (N = B).
+ * With cu_seqlens: B must be 1, T is the packed token count and
+ * N = num_seqs sequences are given by cu_seqlens. */
+typedef struct {
+    int32_t B;          /* batch (>= 1; 1 when packed)                          */
+    int32_t T;          /* tokens per sequence, or packed total (>= 0)          */
+    int32_t H;          /* heads (>= 1)                                         */
+    int32_t d_k;        /* key/query channels: 64 or 128                        */
+    int32_t d_v;        /* value channels: 64 or 128                            */
+    int32_t num_seqs;   /* N when cu_seqlens != NULL (>= 1); ignored otherwise  */
+    int32_t qkv_dtype;  /* kda_dtype of q, k, v and out                          */
+} kda_dims;
+
+/*
+ * kda_fwd -- chunked KDA forward on device buffers, asynchronous on `stream`.
+ *
+ * All tensors are dense, row-major (last index fastest), 16-byte aligned,
+ * device-resident, owned by the caller:
+ *   q            [B, T, H, d_k]   qkv_dtype
+ *   k            [B, T, H, d_k]   qkv_dtype
+ *   v            [B, T, H, d_v]   qkv_dtype
+ *   log_alpha    [B, T, H, d_k]   fp32, clamped to [-5, 0] inside
+ *   beta         [B, T, H]        fp32, used as given
+ *   initial_state[N, H, d_k, d_v] fp32, or NULL for a zero state
+ *   cu_seqlens   [N + 1]          int32 on the device, or NULL (then N = B);
+ *                                 cu[0] = 0, non-decreasing, cu[N] = T.  The
+ *                                 library does not read it on the host: a
+ *                                 malformed table is undefined behaviour.
+ *   chunk        tokens per chunk; must be 64
+ *   out          [B, T, H, d_v]   qkv_dtype (bf16 rounded to nearest even)
+ *   final_state  [N, H, d_k, d_v] fp32, or NULL; may be the same pointer as
+ *                                 initial_state (read before written)
+ *   stream       a cudaStream_t (NULL = legacy default stream)
+ *
+ * The state restarts at every sequence start (from initial_state[n] or zero)
+ * and a chunk never straddles two sequences.  A zero-length sequence gives
+ * final_state[n] = initial_state[n].
+ *
+ * Temporary device memory (segment transitions for long sequences) is taken
+ * stream-ordered from the current device's default memory pool
+ * (cudaMallocAsync/cudaFreeAsync on `stream`); no state persists between calls
+ * apart from cached kernel attributes.  Errors: see kda_status; a kernel fault
+ * surfaces at the caller's next synchronisation, as with any CUDA launch.
+ */
+kda_status kda_fwd(const void* q, const void* k, const void* v, const float* log_alpha,
+                   const float* beta, const float* initial_state, const int32_t* cu_seqlens,
+                   int32_t chunk, void* out, float* final_state, const kda_dims* dims,
+                   void* stream);
+
+/*
+ * kda_fwd_host -- the same computation on HOST buffers (same shapes/layouts;
+ * cu_seqlens is a host array here).  Copies the inputs to the device (one
+ * cudaMemcpyAsync per tensor; pinned host memory makes them asynchronous),
+ * runs kda_fwd on `stream`, copies out/final_state back and synchronises the
+ * stream before returning.  Device buffers come from the stream-ordered pool.
+ */
+kda_status kda_fwd_host(const void* q, const void* k, const void* v, const float* log_alpha,
+                        const float* beta, const float* initial_state,
+                        const int32_t* cu_seqlens, int32_t chunk, void* out,
+                        float* final_state, const kda_dims* dims, void* stream);
+
+/* Static description of a status code. */
+const char* kda_status_string(kda_status s);
+
+/* Detail of the last error raised on the calling host thread ("" if none). */
+const char* kda_last_error(void);
+
+/* Number of kernel launches the last kda_fwd call on this host thread issued. */
+int32_t kda_last_launch_count(void);
+
+/* Kernel family the last kda_fwd call on this host thread used: "ffma" (fp32
+ * CUDA-core path), "tc" (tcgen05 tensor-core path) or "" (no launch). */
+const char* kda_last_path(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KDA_H_ */

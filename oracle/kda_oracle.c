@@ -85,36 +85,34 @@ static void run_recurrent(const job_t *J, int64_t n, int64_t h, double *S, doubl
     const int64_t dk = J->dk, dv = J->dv, H = J->H;
     for (int64_t t = J->cu[n]; t < J->cu[n + 1]; ++t) {
         const int64_t rk = (t * H + h) * dk, rv = (t * H + h) * dv;
-        /* forget: Diag(alpha_t) S_{t-1} scales row i (key channel i) */
-        for (int64_t i = 0; i < dk; ++i) {
-            double a = exp(clamp_log_alpha(J->log_alpha[rk + i]));
-            double *row = S + i * dv;
-            for (int64_t j = 0; j < dv; ++j) row[j] *= a;
-        }
-        /* p = (Diag(alpha) S_{t-1})^T k_t : what the state currently returns for k_t */
+        /* forget, row by row: Diag(alpha_t) S_{t-1} scales row i (key channel i);
+         * in the same pass p = (Diag(alpha_t) S_{t-1})^T k_t, what the decayed
+         * state returns for k_t */
         for (int64_t j = 0; j < dv; ++j) p[j] = 0.0;
         for (int64_t i = 0; i < dk; ++i) {
-            double ki = widen(J->k, J->qkv_dtype, rk + i);
-            const double *row = S + i * dv;
-            for (int64_t j = 0; j < dv; ++j) p[j] += row[j] * ki;
-        }
-        /* erase-then-write: S += beta k (v - p)^T
-         * == (I - beta k k^T) Diag(alpha) S_{t-1} + beta k v^T */
-        double b = (double)J->beta[t * H + h];
-        for (int64_t j = 0; j < dv; ++j) p[j] = b * (widen(J->v, J->qkv_dtype, rv + j) - p[j]);
-        for (int64_t i = 0; i < dk; ++i) {
+            double a = exp(clamp_log_alpha(J->log_alpha[rk + i]));
             double ki = widen(J->k, J->qkv_dtype, rk + i);
             double *row = S + i * dv;
-            for (int64_t j = 0; j < dv; ++j) row[j] += ki * p[j];
+            for (int64_t j = 0; j < dv; ++j) {
+                row[j] *= a;
+                p[j] += row[j] * ki;
+            }
         }
-        /* o_t = S_t^T q_t */
-        if (t < J->o_tokens) {
-            double *o = J->o + rv;
-            for (int64_t j = 0; j < dv; ++j) o[j] = 0.0;
-            for (int64_t i = 0; i < dk; ++i) {
-                double qi = widen(J->q, J->qkv_dtype, rk + i);
-                const double *row = S + i * dv;
-                for (int64_t j = 0; j < dv; ++j) o[j] += row[j] * qi;
+        /* erase-then-write: S += beta k (v - p)^T
+         * == (I - beta k k^T) Diag(alpha) S_{t-1} + beta k v^T;
+         * in the same pass o_t = S_t^T q_t (the UPDATED state) */
+        double b = (double)J->beta[t * H + h];
+        for (int64_t j = 0; j < dv; ++j) p[j] = b * (widen(J->v, J->qkv_dtype, rv + j) - p[j]);
+        const int want_o = t < J->o_tokens;
+        double *o = want_o ? J->o + rv : p + dv; /* scratch row when o is not kept */
+        for (int64_t j = 0; j < dv; ++j) o[j] = 0.0;
+        for (int64_t i = 0; i < dk; ++i) {
+            double ki = widen(J->k, J->qkv_dtype, rk + i);
+            double qi = widen(J->q, J->qkv_dtype, rk + i);
+            double *row = S + i * dv;
+            for (int64_t j = 0; j < dv; ++j) {
+                row[j] += ki * p[j];
+                o[j] += row[j] * qi;
             }
         }
     }
@@ -221,7 +219,7 @@ static void run_chunked(const job_t *J, int64_t n, int64_t h, double *S, double 
 static void *worker(void *arg) {
     job_t *J = (job_t *)arg;
     const int64_t dk = J->dk, dv = J->dv, C = J->chunk;
-    size_t ws_n = (size_t)(dk * dv + dv);
+    size_t ws_n = (size_t)(dk * dv + 2 * dv);
     if (J->mode == 1) ws_n += (size_t)(5 * C * dk + C * C + C * dv + dk * dv);
     double *S = (double *)malloc(ws_n * sizeof(double));
     if (!S) return (void *)1;

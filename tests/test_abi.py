@@ -1,0 +1,94 @@
+"""Host-side checks of libkda.so: it loads, exports every declared symbol, and
+rejects bad arguments before any launch (fake, never-dereferenced pointers)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gated_delta_rule_139_b200 as kda
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"^\s*(?:const\s+)?\w+\*?\s+\**(kda_\w+)\s*\(", src, flags=re.M)
+    return names
+
+
+def test_library_exports_every_declared_function():
+    lib = kda.load_library()
+    names = declared_functions()
+    assert {"kda_fwd", "kda_fwd_host", "kda_status_string", "kda_last_error"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings():
+    lib = kda.load_library()
+    for code, name in kda.STATUS.items():
+        assert lib.kda_status_string(code).decode() == name
+
+
+FAKE = 0x7F0000000000  # 16-byte aligned, never dereferenced
+
+
+def call(dims, q=FAKE, k=FAKE + (1 << 30), v=FAKE + (2 << 30), la=FAKE + (3 << 30),
+         be=FAKE + (4 << 30), s0=None, cu=None, chunk=64, out=FAKE + (5 << 30), sf=None):
+    lib = kda.load_library()
+    P = lambda x: None if x is None else ctypes.c_void_p(x)
+    rc = lib.kda_fwd(P(q), P(k), P(v), P(la), P(be), P(s0), P(cu), chunk, P(out), P(sf),
+                     ctypes.byref(dims), None)
+    return kda.STATUS[rc], lib.kda_last_error().decode()
+
+
+def D(B=1, T=128, H=2, dk=128, dv=128, N=0, dt=1):
+    return kda.Dims(B, T, H, dk, dv, N, dt)
+
+
+def test_rejects_unsupported_shapes_and_chunk():
+    assert call(D(dk=96))[0] == "KDA_ERR_UNSUPPORTED"
+    assert call(D(dv=32))[0] == "KDA_ERR_UNSUPPORTED"
+    assert call(D(), chunk=32)[0] == "KDA_ERR_UNSUPPORTED"
+
+
+def test_rejects_invalid_arguments():
+    assert call(D(B=0))[0] == "KDA_ERR_INVALID_ARG"
+    assert call(D(T=-1))[0] == "KDA_ERR_INVALID_ARG"
+    assert call(D(dt=7))[0] == "KDA_ERR_INVALID_ARG"
+    assert call(D(), q=None)[0] == "KDA_ERR_INVALID_ARG"
+    assert call(D(B=2, N=3), cu=FAKE + (7 << 30))[0] == "KDA_ERR_INVALID_ARG"  # packed needs B=1
+    assert call(D(N=0), cu=FAKE + (7 << 30))[0] == "KDA_ERR_INVALID_ARG"
+    lib = kda.load_library()
+    assert kda.STATUS[lib.kda_fwd(None, None, None, None, None, None, None, 64, None, None,
+                                  None, None)] == "KDA_ERR_INVALID_ARG"
+
+
+def test_rejects_misaligned_pointers():
+    st, msg = call(D(), k=FAKE + 8)
+    assert st == "KDA_ERR_MISALIGNED" and "k " in msg + " "
+
+
+def test_rejects_aliasing():
+    assert call(D(), out=FAKE + 64)[0] == "KDA_ERR_ALIAS"  # out inside q
+    s0 = FAKE + (6 << 30)
+    assert call(D(), s0=s0, sf=s0 + 16)[0] == "KDA_ERR_ALIAS"  # partial state overlap
+    assert call(D(), sf=FAKE + (4 << 30))[0] == "KDA_ERR_ALIAS"  # final_state over beta
+
+
+def test_state_in_place_passes_host_checks():
+    # final_state == initial_state is allowed; the call then fails only at the
+    # device-accessibility check (the fake pointers are not device memory)
+    s0 = FAKE + (6 << 30)
+    st, msg = call(D(), s0=s0, sf=s0)
+    assert st == "KDA_ERR_INVALID_ARG" and "device-accessible" in msg
+
+
+def test_zero_length_is_accepted_by_host_checks():
+    st, msg = call(D(T=0), q=None, k=None, v=None, la=None, be=None, out=None)
+    assert st in ("KDA_OK", "KDA_ERR_CUDA")  # no device needed for T=0 validation
