@@ -18,7 +18,7 @@ import ctypes
 import os
 
 __all__ = ["kda_fwd", "kda_fwd_host", "KDAError", "library_path", "load_library",
-           "last_launch_count", "last_path", "STATUS"]
+           "last_launch_count", "last_path", "check_device", "STATUS"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_PKG, "libkda.so")
@@ -67,6 +67,8 @@ def load_library():
         lib.kda_last_launch_count.restype = ctypes.c_int32
         lib.kda_last_path.argtypes = []
         lib.kda_last_path.restype = ctypes.c_char_p
+        lib.kda_check_device.argtypes = [ctypes.c_void_p]
+        lib.kda_check_device.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -79,6 +81,13 @@ def last_launch_count() -> int:
 def last_path() -> str:
     """Kernel family of the last kda_fwd call on this thread ("ffma" or "tc")."""
     return load_library().kda_last_path().decode()
+
+
+def check_device(stream=None) -> None:
+    """Synchronise ``stream`` and raise KDAError if a kernel recorded a device-side
+    error (a bounded wait that gave up, or a malformed cu_seqlens table)."""
+    s = None if stream is None else ctypes.c_void_p(stream.cuda_stream)
+    _check(load_library().kda_check_device(s))
 
 
 def _check(rc: int):

@@ -5,7 +5,12 @@
 #include <cuda_runtime.h>
 #include <stdarg.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
+
+#include <algorithm>
+#include <cmath>
+#include <mutex>
 
 #include "kda.h"
 #include "kda_internal.h"
@@ -125,13 +130,122 @@ kda_status validate(const void* q, const void* k, const void* v, const float* la
     return KDA_OK;
 }
 
-kda_status run(const kda::FwdArgs& a, cudaStream_t stream) {
-    int launches = 0;
-    g_last_path = "ffma";
-    cudaError_t e = kda::launch_ffma(a, stream, &launches);
-    g_last_launches = launches;
+// Library-owned stream-ordered pool per device.  Freed blocks stay reserved in
+// the pool (release threshold = max), so repeated calls do not re-map memory.
+cudaError_t get_pool(cudaMemPool_t* pool) {
+    static cudaMemPool_t pools[kda::kMaxDevices] = {};
+    static std::mutex mu;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= kda::kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!pools[dev]) {
+        cudaMemPoolProps props;
+        memset(&props, 0, sizeof props);
+        props.allocType = cudaMemAllocationTypePinned;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        e = cudaMemPoolCreate(&pools[dev], &props);
+        if (e != cudaSuccess) return e;
+        uint64_t thr = UINT64_MAX;
+        e = cudaMemPoolSetAttribute(pools[dev], cudaMemPoolAttrReleaseThreshold, &thr);
+        if (e != cudaSuccess) return e;
+    }
+    *pool = pools[dev];
+    return cudaSuccess;
+}
+
+cudaError_t pool_alloc(void** p, size_t bytes, cudaStream_t stream) {
+    cudaMemPool_t pool;
+    cudaError_t e = get_pool(&pool);
+    if (e != cudaSuccess) return e;
+    return cudaMallocFromPoolAsync(p, bytes, pool, stream);
+}
+
+int sm_count() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n;
+}
+
+// Segment plan: enough (segment, head) units for about two waves of CTAs.
+kda::TcPlan plan_segments(const kda::FwdArgs& a) {
+    constexpr int C = kda::kChunk;
+    const int64_t nch_seq_max = ((int64_t)a.T + C - 1) / C;  // chunks of the longest possible sequence
+    const int64_t nch_total = a.cu ? nch_seq_max + a.N : (int64_t)a.B * nch_seq_max;
+    const int64_t target = 2LL * sm_count();
+    int64_t seg;
+    if (!a.cu) {
+        const int64_t G = std::max<int64_t>(1, llround((double)target / ((double)a.B * a.H)));
+        seg = (nch_seq_max + G - 1) / G;
+    } else {
+        seg = (nch_total * a.H + target - 1) / target;
+    }
+    seg = std::max<int64_t>(seg, 8);
+    // test hook: force the segment length (in chunks)
+    if (const char* env = getenv("KDA_SEG_CHUNKS")) {
+        const long v = atol(env);
+        if (v > 0) seg = v;
+    }
+    kda::TcPlan p;
+    p.segmented = seg < nch_seq_max;
+    if (!p.segmented) seg = std::max<int64_t>(nch_seq_max, 1);
+    p.seg_chunks = (int)std::min<int64_t>(seg, 1 << 30);
+    p.max_units = (int)(p.segmented ? (nch_total + seg - 1) / seg + a.N : a.N);
+    return p;
+}
+
+kda_status run_tc(const kda::FwdArgs& a, cudaStream_t stream, int* launches) {
+    const kda::TcPlan p = plan_segments(a);
+    const size_t st = (size_t)128 * 128 * sizeof(float);
+    const size_t b_segs = ((size_t)p.max_units * sizeof(kda::SegEntry) + 255) & ~(size_t)255;
+    const size_t b_off = ((size_t)(a.N + 1) * 4 + 4 + 255) & ~(size_t)255;
+    const size_t b_trans = p.segmented ? (size_t)p.max_units * a.H * 2 * st : 0;
+    const size_t b_sin = p.segmented ? (size_t)p.max_units * a.H * st : 0;
+    char* ws = nullptr;
+    cudaError_t e = pool_alloc((void**)&ws, b_segs + b_off + b_trans + b_sin, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "workspace allocation");
+    kda::TcArgs t;
+    t.q = a.q;
+    t.k = a.k;
+    t.v = a.v;
+    t.log_alpha = a.log_alpha;
+    t.beta = a.beta;
+    t.s0 = a.s0;
+    t.cu = a.cu;
+    t.out = a.out;
+    t.s_final = a.s_final;
+    t.B = a.B;
+    t.T = a.T;
+    t.H = a.H;
+    t.N = a.N;
+    t.segs = (kda::SegEntry*)ws;
+    t.seg_off = (int32_t*)(ws + b_segs);
+    t.n_units = t.seg_off + a.N + 1;
+    t.trans = p.segmented ? (float*)(ws + b_segs + b_off) : nullptr;
+    t.sin = p.segmented ? (float*)(ws + b_segs + b_off + b_trans) : nullptr;
+    e = kda::launch_tc(t, p, stream, launches);
+    cudaFreeAsync(ws, stream);
     if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
     return KDA_OK;
+}
+
+kda_status run(const kda::FwdArgs& a, cudaStream_t stream) {
+    int launches = 0;
+    if ((int64_t)a.N * a.H == 0) return KDA_OK;
+    kda_status s = KDA_OK;
+    if (a.bf16 && a.dk == 128 && a.dv == 128) {
+        g_last_path = "tc";
+        s = run_tc(a, stream, &launches);
+    } else {
+        g_last_path = "ffma";
+        cudaError_t e = kda::launch_ffma(a, stream, &launches);
+        if (e != cudaSuccess) s = cuda_fail(e, "kernel launch");
+    }
+    g_last_launches = launches;
+    return s;
 }
 
 }  // namespace
@@ -180,8 +294,8 @@ kda_status kda_fwd_host(const void* q, const void* k, const void* v, const float
     char* base = nullptr;
     cudaError_t e = cudaSuccess;
     if (total) {
-        e = cudaMallocAsync((void**)&base, total, stream);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync");
+        e = pool_alloc((void**)&base, total, stream);
+        if (e != cudaSuccess) return cuda_fail(e, "device buffer allocation");
     }
     const void* src[] = {q, k, v, log_alpha, beta, initial_state, cu_seqlens};
     for (int i = 0; i < 7 && e == cudaSuccess; ++i)
@@ -233,5 +347,18 @@ const char* kda_last_error(void) { return g_last_error; }
 int32_t kda_last_launch_count(void) { return g_last_launches; }
 
 const char* kda_last_path(void) { return g_last_path; }
+
+kda_status kda_check_device(void* stream) {
+    g_last_error[0] = 0;
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+    int code = 0;
+    e = kda::tc_take_status(&code);
+    if (e != cudaSuccess) return cuda_fail(e, "device status read");
+    if (code == 1) return fail(KDA_ERR_DEVICE_TIMEOUT, "a bounded device wait gave up");
+    if (code == 2) return fail(KDA_ERR_INVALID_ARG, "segment table overflow: malformed cu_seqlens");
+    if (code) return fail(KDA_ERR_CUDA, "device status %d", code);
+    return KDA_OK;
+}
 
 }  // extern "C"

@@ -26,4 +26,45 @@ struct FwdArgs {
 // CUDA-core chunkwise path (exact fp32 arithmetic on fp32 or bf16 inputs).
 cudaError_t launch_ffma(const FwdArgs& a, cudaStream_t stream, int* launches);
 
+// One segment of one sequence: tokens [t_begin, t_end), whole chunks except
+// possibly the sequence's last.
+struct SegEntry {
+    int64_t t_begin, t_end;
+    int32_t n;     // sequence
+    int32_t j;     // segment index inside the sequence
+    int32_t last;  // 1 for the sequence's last segment
+    int32_t pad;
+};
+
+// Tensor-core path arguments: the validated forward arguments plus workspace.
+struct TcArgs {
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* log_alpha;
+    const float* beta;
+    const float* s0;
+    const int32_t* cu;
+    void* out;
+    float* s_final;
+    int32_t B, T, H, N;
+    SegEntry* segs;     // [max_units]
+    int32_t* seg_off;   // [N+1]: first unit of each sequence
+    int32_t* n_units;   // [1]
+    float* trans;       // [max_units, H, 2, 128, 128]: B^T then M^T of each segment
+    float* sin;         // [max_units, H, 128, 128]: S_in^T of each segment
+};
+
+struct TcPlan {
+    int seg_chunks;   // chunks per segment
+    int max_units;    // upper bound on the number of segments over all sequences
+    bool segmented;   // some sequence may have more than one segment
+};
+
+// bf16 q/k/v with d_k = d_v = 128: tcgen05 tensor-core path.
+cudaError_t launch_tc(const TcArgs& a, const TcPlan& p, cudaStream_t stream, int* launches);
+size_t tc_smem_bytes();
+// Reads and clears the current device's status word (0 = no device-side error).
+cudaError_t tc_take_status(int* code);
+
 }  // namespace kda

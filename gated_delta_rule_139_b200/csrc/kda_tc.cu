@@ -1,0 +1,762 @@
+// kda_tc.cu -- KDA chunked forward on the 5th-generation tensor cores (sm_100a).
+//
+// Source of the method: aiblin.ru, "Kimi K3 -- открытая модель, которая обошла
+// закрытых лидеров рынка".  Section "Как хранить миллион токенов в памяти":
+// the state S (d_k x d_v) is rewritten per token, erase-then-write with
+// strength beta and per-channel forget gate alpha clamped to [e^-5, 1].
+// Section "Как распараллелили последовательное обновление": (i) all tokens of a
+// chunk are processed in parallel and the state is then passed from chunk to
+// chunk; (ii) a long prefill is cut into segments whose state transitions are
+// computed in parallel on different SMs of one GPU and reassembled exactly,
+// each segment being described by a local state (its effect on a zero state)
+// and a token-dependent transition matrix: S_out = M S_in + B.
+//
+// Kernels (one launch each, all on the caller's stream):
+//   seg_setup   : segment table from cu_seqlens (or B x T) on the device.
+//   tc_kernel<SEG=true>  "pass 1": per (segment, head) the transition (B, M)
+//                 of every segment that has a successor, computed as the
+//                 chunk loop applied to the augmented state [B | M] from [0 | I].
+//   seg_scan    : S_in(j+1) = M_j S_in(j) + B_j, sequential over the segments
+//                 of a sequence, parallel over (sequence, head, 16-row block).
+//   tc_kernel<SEG=false> "pass 3": per (segment, head) the chunk loop from the
+//                 true incoming state, writing o and the final state.
+//
+// Per chunk of C = 64 tokens (g = in-chunk inclusive cumsum of the clamped
+// log-gates, per key channel), everything in the transposed orientation so
+// that every tensor-core product has M = 128 rows:
+//   A  = strict_lower(diag(beta) (K e^g)(K e^-g)^T),  P = lower_incl((Q e^g)(K e^-g)^T)
+//   T  = (I + A)^-1                                      (fp32, CUDA cores)
+//   W^T = (diag(beta) K e^g)^T T^T,   U'^T = (diag(beta) V)^T T^T
+//   U^T = U'^T - S^T W^T
+//   O^T = S^T (Q e^g)^T + U^T P^T
+//   S^T <- S^T Diag(e^{g_last}) + U^T (K e^{g_last - g})
+// The state S^T (d_v x d_k, fp32) stays in tensor memory for the whole
+// segment; it enters the products as a bf16 copy.  Gate factors are
+// referenced to the middle of each 32-token half (rho_a = g_15, rho_b = g_47)
+// so every factor handed to the tensor core lies in [e^-80, e^80], inside the
+// bf16/fp32 exponent range; the cross-half block of A and P is a separate
+// product whose factors are both <= 1 (underflow to 0 is the correct limit).
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "kda_internal.h"
+#include "tc_common.cuh"
+
+namespace kda {
+namespace {
+
+__device__ int g_tc_status = 0;  // first device-side error code of this device (0 = none)
+
+
+using namespace tc;
+
+constexpr int C = 64;     // tokens per chunk
+constexpr int D = 128;    // d_k = d_v
+constexpr int NT = 256;   // threads per CTA
+constexpr float LOG2E = 1.4426950408889634f;
+
+enum : int { ERR_WAIT_TIMEOUT = 1, ERR_SEG_OVERFLOW = 2 };
+
+// ---------------------------------------------------------------- shared memory map
+// Region R1 is reused across the phases of one chunk:
+//   phases 0-1: X1 (A operand, 128 x 128) and BT (B operand, 96 x 128)
+//   phase  2  : As, Ts (fp32 64 x 65) and Ys (fp32 3 x 16 x 17) for (I + A)^-1
+//   phases 3-8: SA (bf16 S^T), WB (W^T), UA (U^T), and OS (output staging) or,
+//               in pass 1, MA (bf16 M^T) and UMA (U_M^T)
+struct Lay {
+    static constexpr uint32_t X1 = 0, BT = 32768;
+    static constexpr uint32_t AS = 0, TS = 16640, YS = 33280;
+    static constexpr uint32_t SA = 0, WB = 32768, UA = 49152, OS = 65536, MA = 65536,
+                              UMA = 98304;
+    static constexpr uint32_t R1 = 114688;
+    static constexpr uint32_t QT = R1;               // 64 x 128, K-major
+    static constexpr uint32_t KB = QT + 16384;       // 64 x 128, MN-major
+    static constexpr uint32_t VB = KB + 16384;       // 64 x 128, MN-major
+    static constexpr uint32_t KD = VB + 16384;       // 64 x 128, MN-major
+    static constexpr uint32_t TB = KD + 16384;       // 64 x 64, K-major
+    static constexpr uint32_t PB = TB + 8192;        // 64 x 64, K-major
+    static constexpr uint32_t GSUM = PB + 8192;      // fp32 [8][128]
+    static constexpr uint32_t REFS = GSUM + 4096;    // fp32 [4][128]: rho_a, rho_m, rho_b, g_last
+    static constexpr uint32_t GAM = REFS + 2048;     // fp32 [128]
+    static constexpr uint32_t BETA = GAM + 512;      // fp32 [64]
+    static constexpr uint32_t BAR = BETA + 256;      // mbarrier
+    static constexpr uint32_t TMEMP = BAR + 16;      // TMEM base address
+    static constexpr uint32_t END = TMEMP + 16;
+    static constexpr uint32_t BYTES = END + 1024;    // + alignment slack
+};
+static_assert(Lay::OS + 16384 <= Lay::R1 && Lay::UMA + 16384 <= Lay::R1, "R1 overflow");
+static_assert(Lay::YS + 3 * 16 * 17 * 4 <= Lay::R1, "R1 overflow");
+
+// TMEM columns (512 allocated).  Pass 3: AP [0,96) W [96,160) U [160,224)
+// O [224,288) S [384,512).  Pass 1: AP/U_M [0,96) W U as above, B [256,384), M [384,512).
+constexpr uint32_t TM_AP = 0, TM_W = 96, TM_U = 160, TM_O = 224;
+constexpr uint32_t TM_B = 256, TM_S = 384, TM_M = 384;
+
+__device__ __forceinline__ float clamp_gate(float x) { return fminf(fmaxf(x, -5.f), 0.f); }
+__device__ __forceinline__ float ex2(float x) { return exp2f(x); }
+
+__device__ __forceinline__ void st8(uint8_t* base, uint32_t off, float a, float b, float c,
+                                    float d) {
+    uint2 v;
+    v.x = pack_bf16(a, b);
+    v.y = pack_bf16(c, d);
+    *reinterpret_cast<uint2*>(base + off) = v;
+}
+
+__device__ __forceinline__ void load_bf16x4(const __nv_bfloat16* p, float (&f)[4]) {
+    const uint2 raw = __ldg(reinterpret_cast<const uint2*>(p));
+    const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
+    const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
+    f[0] = __low2float(lo);
+    f[1] = __high2float(lo);
+    f[2] = __low2float(hi);
+    f[3] = __high2float(hi);
+}
+
+// Block-wide bounded wait on the MMA barrier; returns false (uniformly) if any
+// thread gave up.
+__device__ __forceinline__ bool wait_mma(void* bar, uint32_t& parity) {
+    const bool ok = mbar_wait(bar, parity, &g_tc_status, ERR_WAIT_TIMEOUT);
+    parity ^= 1u;
+    tc_fence_after();
+    return !__syncthreads_or(!ok);
+}
+
+// Copy 16 TMEM columns x this warp's 32 lanes into a bf16 K-major tile row
+// (chunks c8, c8+1 of row `row`), optionally scaling the TMEM copy by gam.
+__device__ __forceinline__ void stage_row16(uint32_t tm, uint8_t* tile, int R, int row, int col0,
+                                            const float* gam, bool scale_back) {
+    float v[16];
+    tmem_ld16(tm, v);
+    tmem_wait16(v);
+    const uint32_t base = smem_u32(tile);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int c8 = (col0 >> 3) + h;
+        st_shared_v4(base + kmajor_chunk_off(row, c8, R), pack_bf16(v[8 * h + 0], v[8 * h + 1]),
+                     pack_bf16(v[8 * h + 2], v[8 * h + 3]), pack_bf16(v[8 * h + 4], v[8 * h + 5]),
+                     pack_bf16(v[8 * h + 6], v[8 * h + 7]));
+    }
+    if (scale_back) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] *= gam[col0 + i];
+        tmem_st16(tm, v);
+    }
+}
+
+// ---------------------------------------------------------------- (I + A)^-1
+// As: strictly lower 64 x 64 (fp32, stride 65).  Writes T = (I + A)^-1 into Ts
+// (fp32, stride 65, zeros above the diagonal) by 16 x 16 blocks: diagonal
+// blocks by forward substitution, then T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ.
+__device__ void invert_unit_lower(const float* As, float* Ts, float* Ys, int tid) {
+    constexpr int S = 65;
+    if (tid < 64) {
+        const int b = tid >> 4, j = tid & 15, o = 16 * b;
+        float t[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            float v = (i == j) ? 1.f : 0.f;
+#pragma unroll
+            for (int m = 0; m < i; ++m) v = fmaf(-As[(o + i) * S + o + m], t[m], v);
+            t[i] = (i < j) ? 0.f : v;
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) Ts[(o + i) * S + o + j] = t[i];
+    }
+    // zero the strictly upper blocks
+    for (int x = tid; x < 6 * 256; x += NT) {
+        const int p = x >> 8, e = x & 255;
+        const int I = p < 3 ? 0 : p < 5 ? 1 : 2;
+        const int J = p < 3 ? p + 1 : p < 5 ? p - 1 : 3;
+        Ts[(16 * I + (e >> 4)) * S + 16 * J + (e & 15)] = 0.f;
+    }
+    __syncthreads();
+    // levels: distance 1 (3 blocks), 2 (2 blocks), 3 (1 block)
+#pragma unroll 1
+    for (int dist = 1; dist <= 3; ++dist) {
+        const int nblk = 4 - dist;
+        for (int x = tid; x < nblk * 256; x += NT) {
+            const int J = x >> 8, I = J + dist, i = (x >> 4) & 15, j = x & 15;
+            float y = 0.f;
+            for (int K = J; K < I; ++K)
+#pragma unroll
+                for (int m = 0; m < 16; ++m)
+                    y = fmaf(As[(16 * I + i) * S + 16 * K + m], Ts[(16 * K + m) * S + 16 * J + j], y);
+            Ys[(J * 16 + i) * 17 + j] = y;
+        }
+        __syncthreads();
+        for (int x = tid; x < nblk * 256; x += NT) {
+            const int J = x >> 8, I = J + dist, i = (x >> 4) & 15, j = x & 15;
+            float t = 0.f;
+#pragma unroll
+            for (int m = 0; m < 16; ++m)
+                t = fmaf(Ts[(16 * I + i) * S + 16 * I + m], Ys[(J * 16 + m) * 17 + j], t);
+            Ts[(16 * I + i) * S + 16 * J + j] = -t;
+        }
+        __syncthreads();
+    }
+}
+
+// ---------------------------------------------------------------- the chunk loop
+template <bool SEG>
+__global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int u = blockIdx.x, h = blockIdx.y, H = a.H;
+    if (u >= *a.n_units) return;
+    const SegEntry sg = a.segs[u];
+    if (SEG && sg.last) return;  // transitions only for segments with a successor
+
+    float* gsum = reinterpret_cast<float*>(sm + Lay::GSUM);
+    float* gam = reinterpret_cast<float*>(sm + Lay::GAM);
+    float* beta_s = reinterpret_cast<float*>(sm + Lay::BETA);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + Lay::BAR);
+    uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(sm + Lay::TMEMP);
+
+    if (warp == 0) {
+        tmem_alloc(tmem_ptr, 512);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_ptr;
+    const int quad = warp & 3;                       // TMEM lane quadrant of this warp
+    const int lrow = quad * 32 + lane;               // TMEM lane / tile row owned by this thread
+    const uint32_t tq = tmem + ((uint32_t)(quad * 32) << 16);
+    uint32_t parity = 0;
+
+    // ---- initial state
+    if (warp >= 4) {
+        const int e = lrow;
+        for (int c0 = 0; c0 < D; c0 += 16) {
+            float v[16];
+            if (SEG) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[i] = 0.f;  // B = 0
+            } else if (sg.j == 0 && sg.last) {  // single segment: read the caller's state
+                const float* s0 = a.s0 ? a.s0 + ((int64_t)sg.n * H + h) * D * D : nullptr;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[i] = s0 ? s0[(int64_t)(c0 + i) * D + e] : 0.f;
+            } else {
+                const float* sin = a.sin + ((int64_t)u * H + h) * D * D + (int64_t)e * D;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[i] = sin[c0 + i];
+            }
+            tmem_st16(tq + (SEG ? TM_B : TM_S) + c0, v);
+        }
+    } else if (SEG) {
+        const int i0 = lrow;  // M = I
+        for (int c0 = 0; c0 < D; c0 += 16) {
+            float v[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] = (c0 + i == i0) ? 1.f : 0.f;
+            tmem_st16(tq + TM_M + c0, v);
+        }
+    }
+    tmem_st_wait();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    bool ok = true;
+    for (int64_t t0 = sg.t_begin; t0 < sg.t_end && ok; t0 += C) {
+        const int Lc = (int)((sg.t_end - t0) < C ? (sg.t_end - t0) : C);
+
+        // ============ phase 0: gates, scaled operands
+        {
+            const int c4 = lane, tg = warp, c0 = 4 * c4;
+            float g[8][4];
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int r = 8 * tg + i;
+                float4 la = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (r < Lc)
+                    la = __ldg(reinterpret_cast<const float4*>(
+                        a.log_alpha + ((t0 + r) * H + h) * (int64_t)D + c0));
+                acc[0] += clamp_gate(la.x);
+                acc[1] += clamp_gate(la.y);
+                acc[2] += clamp_gate(la.z);
+                acc[3] += clamp_gate(la.w);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) g[i][c] = acc[c];
+            }
+            *reinterpret_cast<float4*>(gsum + tg * D + c0) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+            if (tid < C) beta_s[tid] = tid < Lc ? a.beta[(t0 + tid) * H + h] : 0.f;
+            __syncthreads();
+            float off[4] = {0.f, 0.f, 0.f, 0.f}, run[4] = {0.f, 0.f, 0.f, 0.f};
+            float ra[4], rb[4], gl[4];
+#pragma unroll
+            for (int t2 = 0; t2 < 8; ++t2) {
+                const float4 s = *reinterpret_cast<const float4*>(gsum + t2 * D + c0);
+                const float sv[4] = {s.x, s.y, s.z, s.w};
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    if (t2 < tg) off[c] += sv[c];
+                    run[c] += sv[c];
+                    if (t2 == 1) ra[c] = run[c];
+                    if (t2 == 5) rb[c] = run[c];
+                    if (t2 == 7) gl[c] = run[c];
+                }
+            }
+            // per-channel factors (log2 domain): E_h = e^{rho_h}, Dh = e^{g_last - rho_h},
+            // fba = e^{rho_b - rho_a}
+            float Eh[4], Dh[4], fba[4], rho[4];
+            const bool hb = tg >= 4;  // tokens 8tg.. lie in the second half
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                rho[c] = hb ? rb[c] : ra[c];
+                Eh[c] = ex2(rho[c] * LOG2E);
+                Dh[c] = ex2((gl[c] - rho[c]) * LOG2E);
+                fba[c] = ex2((rb[c] - ra[c]) * LOG2E);
+            }
+            if (tg == 0) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) gam[c0 + c] = ex2(gl[c] * LOG2E);
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int r = 8 * tg + i;
+                const bool valid = r < Lc;
+                const int64_t row = ((t0 + r) * H + h) * (int64_t)D + c0;
+                float kf[4] = {0.f, 0.f, 0.f, 0.f}, qf[4] = {0.f, 0.f, 0.f, 0.f},
+                      vf[4] = {0.f, 0.f, 0.f, 0.f};
+                if (valid) {
+                    load_bf16x4(reinterpret_cast<const __nv_bfloat16*>(a.k) + row, kf);
+                    load_bf16x4(reinterpret_cast<const __nv_bfloat16*>(a.v) + row, vf);
+                    if (!SEG) load_bf16x4(reinterpret_cast<const __nv_bfloat16*>(a.q) + row, qf);
+                }
+                const float br = beta_s[r];
+                float e1[4], e2[4];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const float d2 = (g[i][c] + off[c] - rho[c]) * LOG2E;
+                    e1[c] = ex2(d2);
+                    e2[c] = ex2(-d2);
+                }
+                st8(sm + Lay::X1, kmajor_off(r, c0, 128), kf[0] * e1[0], kf[1] * e1[1],
+                    kf[2] * e1[2], kf[3] * e1[3]);
+                if (!SEG)
+                    st8(sm + Lay::X1, kmajor_off(64 + r, c0, 128), qf[0] * e1[0], qf[1] * e1[1],
+                        qf[2] * e1[2], qf[3] * e1[3]);
+                st8(sm + Lay::BT, kmajor_off(r, c0, 96), kf[0] * e2[0], kf[1] * e2[1],
+                    kf[2] * e2[2], kf[3] * e2[3]);
+                if (r < 32)
+                    st8(sm + Lay::BT, kmajor_off(64 + r, c0, 96), kf[0] * e2[0] * fba[0],
+                        kf[1] * e2[1] * fba[1], kf[2] * e2[2] * fba[2], kf[3] * e2[3] * fba[3]);
+                if (!SEG)
+                    st8(sm + Lay::QT, kmajor_off(r, c0, 64), qf[0] * e1[0] * Eh[0],
+                        qf[1] * e1[1] * Eh[1], qf[2] * e1[2] * Eh[2], qf[3] * e1[3] * Eh[3]);
+                st8(sm + Lay::KB, mnmajor_off(r, c0, 64), br * kf[0] * e1[0] * Eh[0],
+                    br * kf[1] * e1[1] * Eh[1], br * kf[2] * e1[2] * Eh[2],
+                    br * kf[3] * e1[3] * Eh[3]);
+                st8(sm + Lay::VB, mnmajor_off(r, c0, 64), br * vf[0], br * vf[1], br * vf[2],
+                    br * vf[3]);
+                st8(sm + Lay::KD, mnmajor_off(r, c0, 64), kf[0] * e2[0] * Dh[0],
+                    kf[1] * e2[1] * Dh[1], kf[2] * e2[2] * Dh[2], kf[3] * e2[3] * Dh[3]);
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+
+        // ============ phase 1: [A;P] = X1 . BT^T   (M=128, N=96, K=128)
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t x1 = smem_u32(sm + Lay::X1), bt = smem_u32(sm + Lay::BT);
+            constexpr uint32_t id = idesc_bf16(128, 96, false, false);
+#pragma unroll
+            for (int s = 0; s < 8; ++s)
+                mma_bf16(tmem + TM_AP, kmajor_desc(x1, 128, s), kmajor_desc(bt, 96, s), id, s > 0);
+            mma_commit(bar);
+        }
+        if (!(ok = wait_mma(bar, parity))) break;
+
+        // ============ phase 2: masks, beta, (I + A)^-1, P
+        {
+            float* As = reinterpret_cast<float*>(sm + Lay::AS);
+            float* Ts = reinterpret_cast<float*>(sm + Lay::TS);
+            float* Ys = reinterpret_cast<float*>(sm + Lay::YS);
+            if (warp < 4 && (!SEG || warp < 2)) {
+                float v[96];
+#pragma unroll
+                for (int q = 0; q < 6; ++q) tmem_ld16(tq + TM_AP + 16 * q, *reinterpret_cast<float(*)[16]>(v + 16 * q));
+#pragma unroll
+                for (int q = 0; q < 6; ++q) tmem_wait16(*reinterpret_cast<float(*)[16]>(v + 16 * q));
+                const int r = lrow & 63;
+                const bool isP = lrow >= 64;
+                const float br = beta_s[r];
+                float x[64];
+#pragma unroll
+                for (int j = 0; j < 64; ++j) {
+                    float val;
+                    if (j < 32)
+                        val = r < 32 ? v[j] : v[64 + j];
+                    else
+                        val = r >= 32 ? v[j] : 0.f;
+                    x[j] = isP ? (j <= r ? val : 0.f) : (j < r ? br * val : 0.f);
+                }
+                if (!isP) {
+#pragma unroll
+                    for (int j = 0; j < 64; ++j) As[r * 65 + j] = x[j];
+                } else {
+                    const uint32_t pb = smem_u32(sm + Lay::PB);
+#pragma unroll
+                    for (int j8 = 0; j8 < 8; ++j8)
+                        st_shared_v4(pb + kmajor_chunk_off(r, j8, 64), pack_bf16(x[8 * j8], x[8 * j8 + 1]),
+                                     pack_bf16(x[8 * j8 + 2], x[8 * j8 + 3]),
+                                     pack_bf16(x[8 * j8 + 4], x[8 * j8 + 5]),
+                                     pack_bf16(x[8 * j8 + 6], x[8 * j8 + 7]));
+                }
+            }
+            __syncthreads();
+            invert_unit_lower(As, Ts, Ys, tid);
+            {  // T -> bf16 K-major [r][j]
+                const uint32_t tb = smem_u32(sm + Lay::TB);
+                const int r = tid >> 2;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int j8 = 2 * (tid & 3) + hh;
+                    const float* t = Ts + r * 65 + 8 * j8;
+                    st_shared_v4(tb + kmajor_chunk_off(r, j8, 64), pack_bf16(t[0], t[1]),
+                                 pack_bf16(t[2], t[3]), pack_bf16(t[4], t[5]), pack_bf16(t[6], t[7]));
+                }
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+
+        // ============ phase 3: W^T = (beta K e^g)^T T^T, U'^T = (beta V)^T T^T
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t kb = smem_u32(sm + Lay::KB), vb = smem_u32(sm + Lay::VB),
+                           tb = smem_u32(sm + Lay::TB);
+            constexpr uint32_t id = idesc_bf16(128, 64, true, false);
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                mma_bf16(tmem + TM_W, mnmajor_desc(kb, 64, s), kmajor_desc(tb, 64, s), id, s > 0);
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                mma_bf16(tmem + TM_U, mnmajor_desc(vb, 64, s), kmajor_desc(tb, 64, s), id, s > 0);
+            mma_commit(bar);
+        }
+        // meanwhile: bf16 copy of the state into SA (and MA), state scaled by gamma in TMEM
+        if (warp >= 4) {
+#pragma unroll 1
+            for (int c0 = 0; c0 < D; c0 += 16)
+                stage_row16(tq + (SEG ? TM_B : TM_S) + c0, sm + Lay::SA, 128, lrow, c0, gam, true);
+        } else if (SEG) {
+#pragma unroll 1
+            for (int c0 = 0; c0 < D; c0 += 16)
+                stage_row16(tq + TM_M + c0, sm + Lay::MA, 128, lrow, c0, gam, true);
+        }
+        tmem_st_wait();
+        if (!(ok = wait_mma(bar, parity))) break;
+        // W^T -> WB (MN-major B operand: K rows = c, MN = r)
+        if (warp < 4) {
+            const uint32_t wb = smem_u32(sm + Lay::WB);
+#pragma unroll 1
+            for (int q = 0; q < 4; ++q) {
+                float v[16];
+                tmem_ld16(tq + TM_W + 16 * q, v);
+                tmem_wait16(v);
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh)
+                    st_shared_v4(wb + mnmajor_chunk_off(lrow, 2 * q + hh, 128),
+                                 pack_bf16(v[8 * hh + 0], v[8 * hh + 1]),
+                                 pack_bf16(v[8 * hh + 2], v[8 * hh + 3]),
+                                 pack_bf16(v[8 * hh + 4], v[8 * hh + 5]),
+                                 pack_bf16(v[8 * hh + 6], v[8 * hh + 7]));
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+
+        // ============ phase 5: U^T -= S^T W^T ; O^T = S^T Q~^T  (pass 1: U_M^T = -M^T W^T)
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t sa = smem_u32(sm + Lay::SA), wb = smem_u32(sm + Lay::WB);
+            constexpr uint32_t id_neg = idesc_bf16(128, 64, false, true, true);
+#pragma unroll
+            for (int s = 0; s < 8; ++s)
+                mma_bf16(tmem + TM_U, kmajor_desc(sa, 128, s), mnmajor_desc(wb, 128, s), id_neg, 1);
+            if (!SEG) {
+                const uint32_t qt = smem_u32(sm + Lay::QT);
+                constexpr uint32_t id = idesc_bf16(128, 64, false, false);
+#pragma unroll
+                for (int s = 0; s < 8; ++s)
+                    mma_bf16(tmem + TM_O, kmajor_desc(sa, 128, s), kmajor_desc(qt, 64, s), id, s > 0);
+            } else {
+                const uint32_t ma = smem_u32(sm + Lay::MA);
+#pragma unroll
+                for (int s = 0; s < 8; ++s)
+                    mma_bf16(tmem + TM_AP, kmajor_desc(ma, 128, s), mnmajor_desc(wb, 128, s), id_neg,
+                             s > 0);
+            }
+            mma_commit(bar);
+        }
+        if (!(ok = wait_mma(bar, parity))) break;
+
+        // ============ phase 6: U^T -> UA (bf16, K-major, 128 x 64); pass 1 also U_M^T -> UMA
+        if (warp < 4) {
+#pragma unroll 1
+            for (int c0 = 0; c0 < C; c0 += 16)
+                stage_row16(tq + TM_U + c0, sm + Lay::UA, 128, lrow, c0, nullptr, false);
+        } else if (SEG) {
+#pragma unroll 1
+            for (int c0 = 0; c0 < C; c0 += 16)
+                stage_row16(tq + TM_AP + c0, sm + Lay::UMA, 128, lrow, c0, nullptr, false);
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+
+        // ============ phase 7: O^T += U^T P^T ; S^T += U^T Kdec  (pass 1: B, M updates)
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t ua = smem_u32(sm + Lay::UA), kd = smem_u32(sm + Lay::KD);
+            constexpr uint32_t id_s = idesc_bf16(128, 128, false, true);
+            if (!SEG) {
+                const uint32_t pb = smem_u32(sm + Lay::PB);
+                constexpr uint32_t id = idesc_bf16(128, 64, false, false);
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_bf16(tmem + TM_O, kmajor_desc(ua, 128, s), kmajor_desc(pb, 64, s), id, 1);
+            }
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                mma_bf16(tmem + (SEG ? TM_B : TM_S), kmajor_desc(ua, 128, s), mnmajor_desc(kd, 64, s),
+                         id_s, 1);
+            if (SEG) {
+                const uint32_t uma = smem_u32(sm + Lay::UMA);
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_bf16(tmem + TM_M, kmajor_desc(uma, 128, s), mnmajor_desc(kd, 64, s), id_s, 1);
+            }
+            mma_commit(bar);
+        }
+        if (!(ok = wait_mma(bar, parity))) break;
+
+        // ============ phase 8: O^T -> out (via shared memory, 16-byte global stores)
+        if (!SEG) {
+            __nv_bfloat16* os = reinterpret_cast<__nv_bfloat16*>(sm + Lay::OS);
+            if (warp < 4) {
+#pragma unroll 1
+                for (int q = 0; q < 4; ++q) {
+                    float v[16];
+                    tmem_ld16(tq + TM_O + 16 * q, v);
+                    tmem_wait16(v);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) os[(16 * q + i) * D + lrow] = __float2bfloat16_rn(v[i]);
+                }
+            }
+            tc_fence_before();
+            __syncthreads();
+            __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                const int idx = tid + NT * x, r = idx >> 4, cc = idx & 15;
+                if (r < Lc)
+                    *reinterpret_cast<uint4*>(out + ((t0 + r) * H + h) * (int64_t)D + 8 * cc) =
+                        *reinterpret_cast<const uint4*>(os + r * D + 8 * cc);
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    }
+
+    // ---- results of the segment
+    if (ok) {
+        if (SEG) {
+            float* dst = a.trans + ((int64_t)u * H + h) * 2 * D * D;
+            const uint32_t col = warp >= 4 ? TM_B : TM_M;
+            float* rowp = dst + (warp >= 4 ? 0 : D * D) + (int64_t)lrow * D;
+            for (int c0 = 0; c0 < D; c0 += 16) {
+                float v[16];
+                tmem_ld16(tq + col + c0, v);
+                tmem_wait16(v);
+#pragma unroll
+                for (int i = 0; i < 16; i += 4)
+                    *reinterpret_cast<float4*>(rowp + c0 + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+            }
+        } else if (sg.last && a.s_final && warp >= 4) {
+            float* sf = a.s_final + ((int64_t)sg.n * H + h) * D * D;
+            for (int c0 = 0; c0 < D; c0 += 16) {
+                float v[16];
+                tmem_ld16(tq + TM_S + c0, v);
+                tmem_wait16(v);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) sf[(int64_t)(c0 + i) * D + lrow] = v[i];
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+// ---------------------------------------------------------------- segment table
+// One CTA.  Sequence n has nch = ceil(len/64) chunks and G_n = max(1,
+// ceil(nch / seg_chunks)) segments; segment j covers chunks [j*seg_chunks,
+// min(nch, (j+1)*seg_chunks)).
+__global__ void __launch_bounds__(1024) seg_setup_kernel(const int32_t* cu, int N, int T,
+                                                         int seg_chunks, int max_units,
+                                                         SegEntry* segs, int32_t* seg_off,
+                                                         int32_t* n_units) {
+    __shared__ int32_t warp_sums[32];
+    __shared__ int32_t carry;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid == 0) carry = 0;
+    __syncthreads();
+    for (int base = 0; base < N; base += 1024) {
+        const int n = base + tid;
+        int64_t lo = 0, hi = 0;
+        if (n < N) {
+            lo = cu ? cu[n] : (int64_t)n * T;
+            hi = cu ? cu[n + 1] : lo + T;
+        }
+        const int64_t nch = hi > lo ? (hi - lo + C - 1) / C : 0;
+        int g = n < N ? (int)(nch > 0 ? (nch + seg_chunks - 1) / seg_chunks : 1) : 0;
+        // block-wide exclusive scan of g
+        int x = g;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane == 31) warp_sums[warp] = x;
+        __syncthreads();
+        if (warp == 0) {
+            int w = warp_sums[lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, w, o);
+                if (lane >= o) w += y;
+            }
+            warp_sums[lane] = w;
+        }
+        __syncthreads();
+        const int excl = carry + x - g + (warp > 0 ? warp_sums[warp - 1] : 0);
+        if (n < N) {
+            seg_off[n] = excl;
+            for (int j = 0; j < g; ++j) {
+                const int uidx = excl + j;
+                if (uidx >= max_units) {
+                    atomicCAS(&g_tc_status, 0, ERR_SEG_OVERFLOW);
+                    break;
+                }
+                SegEntry e;
+                e.n = n;
+                e.j = j;
+                e.t_begin = lo + (int64_t)j * seg_chunks * C;
+                const int64_t end = lo + (int64_t)(j + 1) * seg_chunks * C;
+                e.t_end = end < hi ? end : hi;
+                e.last = (j == g - 1) ? 1 : 0;
+                segs[uidx] = e;
+            }
+        }
+        __syncthreads();
+        if (tid == 1023) carry = excl + g;
+        __syncthreads();
+    }
+    if (tid == 0) {
+        seg_off[N] = carry;
+        *n_units = carry < max_units ? carry : max_units;
+    }
+}
+
+// ---------------------------------------------------------------- segment scan
+// S_in^T(j+1) = S_in^T(j) M_j^T + B_j^T for the 16 rows e in [16*blockIdx.z, +16)
+// of S^T, sequentially over the segments of sequence n, head h.
+__global__ void __launch_bounds__(256) seg_scan_kernel(TcArgs a) {
+    __shared__ float S[16][D];
+    const int n = blockIdx.x, h = blockIdx.y, e0 = 16 * blockIdx.z, H = a.H;
+    const int tid = threadIdx.x, el = tid >> 4, cg = tid & 15;
+    const int32_t u0 = a.seg_off[n], u1 = a.seg_off[n + 1];
+    if (u1 - u0 <= 1 || u0 >= *a.n_units) return;
+    // S_in of segment 0, also copied to the workspace so that pass 3 never reads
+    // initial_state while another segment may be writing final_state (they may
+    // be the same buffer)
+    for (int x = tid; x < 16 * D; x += 256) {
+        const int r = x / D, c = x % D;
+        const float v = a.s0 ? a.s0[(((int64_t)n * H + h) * D + c) * D + e0 + r] : 0.f;
+        S[r][c] = v;
+        a.sin[((int64_t)u0 * H + h) * D * D + (int64_t)(e0 + r) * D + c] = v;
+    }
+    __syncthreads();
+    for (int32_t uu = u0; uu + 1 < u1 && uu + 1 < *a.n_units; ++uu) {
+        const float* Bt = a.trans + ((int64_t)uu * H + h) * 2 * D * D;
+        const float* Mt = Bt + D * D;
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = Bt[(int64_t)(e0 + el) * D + cg + 16 * i];
+        for (int c = 0; c < D; ++c) {
+            const float s = S[el][c];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] = fmaf(s, __ldg(Mt + (int64_t)c * D + cg + 16 * i), acc[i]);
+        }
+        __syncthreads();
+        float* dst = a.sin + ((int64_t)(uu + 1) * H + h) * D * D + (int64_t)(e0 + el) * D;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            S[el][cg + 16 * i] = acc[i];
+            dst[cg + 16 * i] = acc[i];
+        }
+        __syncthreads();
+    }
+}
+
+}  // namespace
+
+size_t tc_smem_bytes() { return Lay::BYTES; }
+
+cudaError_t tc_take_status(int* code) {
+    int zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(code, g_tc_status, sizeof(int));
+    if (e == cudaSuccess && *code) e = cudaMemcpyToSymbol(g_tc_status, &zero, sizeof(int));
+    return e;
+}
+
+cudaError_t launch_tc(const TcArgs& a, const TcPlan& p, cudaStream_t stream, int* launches) {
+    static bool attr_set[kMaxDevices][2] = {};
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev >= kMaxDevices || !attr_set[dev][0]) {
+        err = cudaFuncSetAttribute(tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)Lay::BYTES);
+        if (err == cudaSuccess)
+            err = cudaFuncSetAttribute(tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)Lay::BYTES);
+        if (err != cudaSuccess) return err;
+        if (dev < kMaxDevices) attr_set[dev][0] = true;
+    }
+    seg_setup_kernel<<<1, 1024, 0, stream>>>(a.cu, a.N, a.T, p.seg_chunks, p.max_units, a.segs,
+                                             a.seg_off, a.n_units);
+    *launches += 1;
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    const dim3 grid((unsigned)p.max_units, (unsigned)a.H);
+    if (p.segmented) {
+        tc_kernel<true><<<grid, NT, Lay::BYTES, stream>>>(a);
+        *launches += 1;
+        if ((err = cudaGetLastError()) != cudaSuccess) return err;
+        seg_scan_kernel<<<dim3((unsigned)a.N, (unsigned)a.H, D / 16), 256, 0, stream>>>(a);
+        *launches += 1;
+        if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    }
+    tc_kernel<false><<<grid, NT, Lay::BYTES, stream>>>(a);
+    *launches += 1;
+    return cudaGetLastError();
+}
+
+}  // namespace kda

@@ -88,11 +88,14 @@ typedef struct {
  * and a chunk never straddles two sequences.  A zero-length sequence gives
  * final_state[n] = initial_state[n].
  *
- * Temporary device memory (segment transitions for long sequences) is taken
- * stream-ordered from the current device's default memory pool
- * (cudaMallocAsync/cudaFreeAsync on `stream`); no state persists between calls
- * apart from cached kernel attributes.  Errors: see kda_status; a kernel fault
- * surfaces at the caller's next synchronisation, as with any CUDA launch.
+ * Temporary device memory (segment table, segment transitions and incoming
+ * states for long sequences) is taken stream-ordered (cudaMallocFromPoolAsync /
+ * cudaFreeAsync on `stream`) from a memory pool the library creates once per
+ * device and keeps for the life of the process; freed blocks stay reserved in
+ * that pool for the next call.  Nothing else persists between calls apart from
+ * cached kernel attributes and the device status word (kda_check_device).
+ * Errors: see kda_status; a kernel fault surfaces at the caller's next
+ * synchronisation, as with any CUDA launch.
  */
 kda_status kda_fwd(const void* q, const void* k, const void* v, const float* log_alpha,
                    const float* beta, const float* initial_state, const int32_t* cu_seqlens,
@@ -123,6 +126,13 @@ int32_t kda_last_launch_count(void);
 /* Kernel family the last kda_fwd call on this host thread used: "ffma" (fp32
  * CUDA-core path), "tc" (tcgen05 tensor-core path) or "" (no launch). */
 const char* kda_last_path(void);
+
+/* Synchronises `stream`, then reads and clears the current device's status
+ * word, which kernels set when a bounded wait gives up (KDA_ERR_DEVICE_TIMEOUT)
+ * or the device-built segment table would overflow because cu_seqlens is
+ * malformed (KDA_ERR_INVALID_ARG).  KDA_OK when neither happened since the last
+ * check. */
+kda_status kda_check_device(void* stream);
 
 #ifdef __cplusplus
 }

@@ -74,7 +74,7 @@ __global__ void __launch_bounds__(128) gemm_kernel(const __nv_bfloat16* A, const
     for (int c0 = 0; c0 < N; c0 += 16) {
         float v[16];
         tmem_ld16(taddr(tm, warp * 32, c0), v);
-        tmem_ld_wait();
+        tmem_wait16(v);
         for (int j = 0; j < 16; ++j) D[(warp * 32 + lane) * N + c0 + j] = v[j];
     }
     tc_fence_before();

@@ -131,20 +131,56 @@ def test_packed_equals_separate_bitwise():
         assert torch.equal(on[0], o[sl]) and torch.equal(sn[0], s[n])
 
 
-def test_resume_from_final_state():
+def test_resume_from_final_state(monkeypatch):
+    """Split at a chunk boundary with final -> initial state: identical to one call
+    when neither call is cut into segments (same chunks, same arithmetic)."""
     import torch
     from gated_delta_rule_139_b200 import kda_fwd
+    monkeypatch.setenv("KDA_SEG_CHUNKS", "100000")
     inp = make_inputs(1, 640, 2, 128, 128, bf16=True, seed=26, state_sigma=0.05)
     d = to_device(inp)
     o, s = kda_fwd(**d)
-    T1 = 320  # on a chunk boundary: the split computes exactly the same chunks
-    cut = lambda x, sl: x[:, sl].contiguous()
-    a = {k_: cut(v_, slice(0, T1)) for k_, v_ in d.items() if k_ in ("q", "k", "v", "log_alpha", "beta")}
-    b = {k_: cut(v_, slice(T1, None)) for k_, v_ in d.items() if k_ in ("q", "k", "v", "log_alpha", "beta")}
+    T1 = 320
+    keys = ("q", "k", "v", "log_alpha", "beta")
+    a = {k_: d[k_][:, :T1].contiguous() for k_ in keys}
+    b = {k_: d[k_][:, T1:].contiguous() for k_ in keys}
     o1, s1 = kda_fwd(**a, initial_state=d["initial_state"])
     o2, s2 = kda_fwd(**b, initial_state=s1)
     torch.cuda.synchronize()
     assert torch.equal(torch.cat([o1, o2], 1), o) and torch.equal(s2, s)
+
+
+@pytest.mark.parametrize("seg_chunks", ["1", "2", "3", "5"])
+def test_segment_split_matches_oracle(monkeypatch, seg_chunks):
+    """Forced segment lengths: the segment transitions (local state + transition
+    matrix) and their scan reassemble the sequential result."""
+    monkeypatch.setenv("KDA_SEG_CHUNKS", seg_chunks)
+    lens = [64 * 7 + 5, 64, 0, 64 * 3, 31]
+    inp = make_inputs(1, 0, 3, 128, 128, bf16=True, seed=31, seq_lens=lens, state_sigma=0.05,
+                      gate_sigma=2.0)
+    _check(inp)
+    inp2 = make_inputs(2, 64 * 6 + 9, 2, 128, 128, bf16=True, seed=32, state_sigma=0.05)
+    _check(inp2)
+
+
+def test_segment_split_in_place_state(monkeypatch):
+    import torch
+    from gated_delta_rule_139_b200 import kda_fwd
+    monkeypatch.setenv("KDA_SEG_CHUNKS", "2")
+    inp = make_inputs(1, 64 * 9, 2, 128, 128, bf16=True, seed=33, state_sigma=0.05)
+    d = to_device(inp)
+    o, s = kda_fwd(**d)
+    st = d["initial_state"].clone()
+    o2, _ = kda_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], st, final_state=st)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o2) and torch.equal(s, st)
+
+
+def test_device_status_clean():
+    from gated_delta_rule_139_b200 import check_device
+    inp = make_inputs(1, 300, 2, 128, 128, bf16=True, seed=34)
+    run_gpu(inp)
+    check_device()
 
 
 def test_state_in_place():
