@@ -18,7 +18,8 @@ import ctypes
 import os
 
 __all__ = ["kda_fwd", "kda_fwd_host", "KDAError", "library_path", "load_library",
-           "last_launch_count", "last_path", "check_device", "STATUS"]
+           "last_launch_count", "last_path", "check_device", "profile_enable", "profile_read",
+           "STATUS"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_PKG, "libkda.so")
@@ -69,6 +70,12 @@ def load_library():
         lib.kda_last_path.restype = ctypes.c_char_p
         lib.kda_check_device.argtypes = [ctypes.c_void_p]
         lib.kda_check_device.restype = ctypes.c_int
+        lib.kda_profile_enable.argtypes = [ctypes.c_int32]
+        lib.kda_profile_enable.restype = None
+        lib.kda_profile_read.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32]
+        lib.kda_profile_read.restype = ctypes.c_int
+        lib.kda_profile_slot_name.argtypes = [ctypes.c_int32]
+        lib.kda_profile_slot_name.restype = ctypes.c_char_p
         _lib = lib
     return _lib
 
@@ -81,6 +88,21 @@ def last_launch_count() -> int:
 def last_path() -> str:
     """Kernel family of the last kda_fwd call on this thread ("ffma" or "tc")."""
     return load_library().kda_last_path().decode()
+
+
+def profile_enable(on: bool = True) -> None:
+    """Turn on/off CUDA-event timing of every internal kernel launch."""
+    load_library().kda_profile_enable(1 if on else 0)
+
+
+def profile_read() -> dict:
+    """{kernel name: (summed ms, launches)} since the previous read (synchronises)."""
+    lib = load_library()
+    n = 5
+    ms = (ctypes.c_double * n)()
+    cnt = (ctypes.c_int64 * n)()
+    _check(lib.kda_profile_read(ctypes.cast(ms, ctypes.c_void_p), ctypes.cast(cnt, ctypes.c_void_p), n))
+    return {lib.kda_profile_slot_name(i).decode(): (ms[i], cnt[i]) for i in range(n) if cnt[i]}
 
 
 def check_device(stream=None) -> None:

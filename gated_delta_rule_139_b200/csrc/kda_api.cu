@@ -9,8 +9,10 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <mutex>
+#include <vector>
 
 #include "kda.h"
 #include "kda_internal.h"
@@ -248,7 +250,52 @@ kda_status run(const kda::FwdArgs& a, cudaStream_t stream) {
     return s;
 }
 
+// ---------------------------------------------------------------- launch timing
+struct Profiler {
+    std::mutex mu;
+    std::atomic<bool> on{false};
+    struct Mark {
+        int slot;
+        cudaEvent_t a, b;
+    };
+    std::vector<Mark> pending;
+    std::vector<cudaEvent_t> free_events;
+    cudaEvent_t open_ev[kda::NUM_SLOTS] = {};
+    double total_ms[kda::NUM_SLOTS] = {};
+    int64_t count[kda::NUM_SLOTS] = {};
+
+    cudaEvent_t get_event() {
+        if (!free_events.empty()) {
+            cudaEvent_t e = free_events.back();
+            free_events.pop_back();
+            return e;
+        }
+        cudaEvent_t e = nullptr;
+        cudaEventCreate(&e);
+        return e;
+    }
+};
+Profiler& profiler() {
+    static Profiler p;
+    return p;
+}
+
 }  // namespace
+
+void kda::profile_mark(int slot, bool begin, cudaStream_t stream) {
+    Profiler& P = profiler();
+    if (!P.on.load(std::memory_order_relaxed)) return;
+    std::lock_guard<std::mutex> lock(P.mu);
+    cudaEvent_t e = P.get_event();
+    if (!e) return;
+    cudaEventRecord(e, stream);
+    if (begin) {
+        P.open_ev[slot] = e;
+    } else if (P.open_ev[slot]) {
+        P.pending.push_back({slot, P.open_ev[slot], e});
+        P.open_ev[slot] = nullptr;
+    }
+}
 
 extern "C" {
 
@@ -347,6 +394,40 @@ const char* kda_last_error(void) { return g_last_error; }
 int32_t kda_last_launch_count(void) { return g_last_launches; }
 
 const char* kda_last_path(void) { return g_last_path; }
+
+void kda_profile_enable(int32_t on) { profiler().on.store(on != 0); }
+
+kda_status kda_profile_read(double* total_ms, int64_t* launches, int32_t n) {
+    g_last_error[0] = 0;
+    Profiler& P = profiler();
+    std::lock_guard<std::mutex> lock(P.mu);
+    cudaError_t err = cudaSuccess;
+    for (const Profiler::Mark& m : P.pending) {
+        float ms = 0.f;
+        cudaError_t e = cudaEventSynchronize(m.b);
+        if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, m.a, m.b);
+        if (e != cudaSuccess) err = e;
+        P.total_ms[m.slot] += ms;
+        P.count[m.slot] += 1;
+        P.free_events.push_back(m.a);
+        P.free_events.push_back(m.b);
+    }
+    P.pending.clear();
+    for (int i = 0; i < kda::NUM_SLOTS && i < n; ++i) {
+        if (total_ms) total_ms[i] = P.total_ms[i];
+        if (launches) launches[i] = P.count[i];
+        P.total_ms[i] = 0.0;
+        P.count[i] = 0;
+    }
+    if (err != cudaSuccess) return cuda_fail(err, "profile event");
+    return KDA_OK;
+}
+
+const char* kda_profile_slot_name(int32_t slot) {
+    static const char* names[] = {"seg_setup", "tc_pass1_transitions", "seg_scan",
+                                  "tc_pass3_forward", "ffma_forward"};
+    return (slot >= 0 && slot < kda::NUM_SLOTS) ? names[slot] : "";
+}
 
 kda_status kda_check_device(void* stream) {
     g_last_error[0] = 0;

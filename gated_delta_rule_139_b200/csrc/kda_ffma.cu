@@ -291,7 +291,9 @@ cudaError_t launch_t(const FwdArgs& a, cudaStream_t stream) {
         if (dev < kMaxDevices) attr_set[dev] = true;
     }
     dim3 grid((unsigned)(a.N * a.H), (unsigned)(a.dv / DVB));
+    profile_mark(SLOT_FFMA, true, stream);
     kern<<<grid, NT, L::bytes, stream>>>(a);
+    profile_mark(SLOT_FFMA, false, stream);
     return cudaGetLastError();
 }
 

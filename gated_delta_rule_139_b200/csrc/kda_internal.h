@@ -8,6 +8,13 @@ namespace kda {
 constexpr int kChunk = 64;       // tokens per chunk
 constexpr int kMaxDevices = 64;  // size of per-device attribute caches
 
+// Kernel slots of the optional per-launch timing (kda_profile_*).
+enum KernelSlot : int { SLOT_SETUP = 0, SLOT_PASS1 = 1, SLOT_SCAN = 2, SLOT_PASS3 = 3, SLOT_FFMA = 4,
+                        NUM_SLOTS = 5 };
+// Records a CUDA event on `stream` before (begin=true) or after a launch of
+// `slot` when timing is enabled; no-op otherwise.
+void profile_mark(int slot, bool begin, cudaStream_t stream);
+
 // Everything a forward launch needs, already validated on the host.
 struct FwdArgs {
     const void* q;

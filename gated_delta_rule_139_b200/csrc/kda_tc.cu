@@ -741,20 +741,28 @@ cudaError_t launch_tc(const TcArgs& a, const TcPlan& p, cudaStream_t stream, int
         if (err != cudaSuccess) return err;
         if (dev < kMaxDevices) attr_set[dev][0] = true;
     }
+    profile_mark(SLOT_SETUP, true, stream);
     seg_setup_kernel<<<1, 1024, 0, stream>>>(a.cu, a.N, a.T, p.seg_chunks, p.max_units, a.segs,
                                              a.seg_off, a.n_units);
+    profile_mark(SLOT_SETUP, false, stream);
     *launches += 1;
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     const dim3 grid((unsigned)p.max_units, (unsigned)a.H);
     if (p.segmented) {
+        profile_mark(SLOT_PASS1, true, stream);
         tc_kernel<true><<<grid, NT, Lay::BYTES, stream>>>(a);
+        profile_mark(SLOT_PASS1, false, stream);
         *launches += 1;
         if ((err = cudaGetLastError()) != cudaSuccess) return err;
+        profile_mark(SLOT_SCAN, true, stream);
         seg_scan_kernel<<<dim3((unsigned)a.N, (unsigned)a.H, D / 16), 256, 0, stream>>>(a);
+        profile_mark(SLOT_SCAN, false, stream);
         *launches += 1;
         if ((err = cudaGetLastError()) != cudaSuccess) return err;
     }
+    profile_mark(SLOT_PASS3, true, stream);
     tc_kernel<false><<<grid, NT, Lay::BYTES, stream>>>(a);
+    profile_mark(SLOT_PASS3, false, stream);
     *launches += 1;
     return cudaGetLastError();
 }

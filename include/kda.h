@@ -134,6 +134,17 @@ const char* kda_last_path(void);
  * check. */
 kda_status kda_check_device(void* stream);
 
+/* Optional launch timing (off by default).  While enabled, every kda_fwd
+ * records a CUDA event on its stream before and after each internal kernel
+ * launch.  kda_profile_read synchronises those events, writes for each of the
+ * first n kernel slots the summed duration in milliseconds and the number of
+ * launches since the previous read, then resets the sums.  Slots: 0 segment
+ * table, 1 pass 1 (segment transitions), 2 segment scan, 3 pass 3 (forward),
+ * 4 CUDA-core forward; kda_profile_slot_name gives their names. */
+void kda_profile_enable(int32_t on);
+kda_status kda_profile_read(double* total_ms, int64_t* launches, int32_t n);
+const char* kda_profile_slot_name(int32_t slot);
+
 #ifdef __cplusplus
 }
 #endif
