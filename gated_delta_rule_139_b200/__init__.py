@@ -17,7 +17,7 @@ from __future__ import annotations
 import ctypes
 import os
 
-__all__ = ["kda_fwd", "kda_fwd_host", "KDAError", "library_path", "load_library",
+__all__ = ["kda_fwd", "kda_fwd_host", "kda_fwd_noalloc", "KDAError", "library_path", "load_library",
            "last_launch_count", "last_path", "check_device", "profile_enable", "profile_read",
            "STATUS"]
 
@@ -56,7 +56,7 @@ def load_library():
         lib = ctypes.CDLL(library_path)
         p = ctypes.c_void_p
         sig = [p, p, p, p, p, p, p, ctypes.c_int32, p, p, ctypes.POINTER(Dims), p]
-        for name in ("kda_fwd", "kda_fwd_host"):
+        for name in ("kda_fwd", "kda_fwd_host", "kda_fwd_noalloc"):
             fn = getattr(lib, name)
             fn.argtypes = sig
             fn.restype = ctypes.c_int
@@ -129,7 +129,8 @@ def _dims(q_shape, v_shape, T_override, cu_len, bf16):
 
 
 def kda_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, chunk: int = 64,
-            out=None, final_state=None, stream=None, want_final: bool = True):
+            out=None, final_state=None, stream=None, want_final: bool = True,
+            _entry: str = "kda_fwd"):
     """KDA forward on CUDA tensors; returns (out, final_state or None).
 
     q/k/v are bf16 or fp32 CUDA tensors; gates and states fp32.  ``stream`` is a
@@ -155,11 +156,27 @@ def kda_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, chunk
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
     ptr = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
-    rc = lib.kda_fwd(ptr(q), ptr(k), ptr(v), ptr(log_alpha), ptr(beta), ptr(initial_state),
-                     ptr(cu_seqlens), int(chunk), ptr(out), ptr(final_state), ctypes.byref(d),
-                     ctypes.c_void_p(stream.cuda_stream))
+    rc = getattr(lib, _entry)(ptr(q), ptr(k), ptr(v), ptr(log_alpha), ptr(beta),
+                              ptr(initial_state), ptr(cu_seqlens), int(chunk), ptr(out),
+                              ptr(final_state), ctypes.byref(d),
+                              ctypes.c_void_p(stream.cuda_stream))
     _check(rc)
     return out, final_state
+
+
+def kda_fwd_noalloc(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
+                    chunk: int = 64, out=None, final_state=None, stream=None,
+                    want_final: bool = True):
+    """kda_fwd through the entry point that allocates no device memory.
+
+    The library's temporaries come from its fixed 32 MiB device scratch array
+    instead of a memory pool (for callers that cannot allocate on the call
+    path).  ``out`` and ``final_state`` are allocated here when not given (by
+    torch, before the call); pass them in to keep the whole call free of
+    allocations.  Calls that overlap on the GPU share the array and race.
+    """
+    return kda_fwd(q, k, v, log_alpha, beta, initial_state, cu_seqlens, chunk, out,
+                   final_state, stream, want_final, _entry="kda_fwd_noalloc")
 
 
 def kda_fwd_host(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,

@@ -280,6 +280,44 @@ Profiler& profiler() {
     return p;
 }
 
+// ---------------------------------------------------------------- no-allocation scratch
+// Device scratch for kda_fwd_noalloc: a fixed array inside the library image.
+// The driver reserves it on every device the library is loaded on, for the
+// life of the process.  In host code `g_noalloc_scratch` only names the
+// symbol; its device address comes from cudaGetSymbolAddress, taken once per
+// device (with that device current) by noalloc_scratch().
+constexpr size_t kNoAllocScratchBytes = (size_t)32 << 20;  // 32 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+cudaError_t noalloc_scratch(char** ptr) {
+    static void* addr[kda::kMaxDevices] = {};
+    static std::mutex mu;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= kda::kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        addr[dev] = p;
+    }
+    *ptr = (char*)addr[dev];
+    return cudaSuccess;
+}
+
+// Bytes of scratch the tensor-core path needs for a segment plan.
+size_t tc_scratch_bytes(const kda::FwdArgs& a, const kda::TcPlan& p, size_t* b_segs,
+                        size_t* b_off, size_t* b_trans) {
+    const size_t st = (size_t)128 * 128 * sizeof(float);
+    *b_segs = ((size_t)p.max_units * sizeof(kda::SegEntry) + 255) & ~(size_t)255;
+    *b_off = ((size_t)(a.N + 1) * 4 + 4 + 255) & ~(size_t)255;
+    *b_trans = p.segmented ? (size_t)p.max_units * a.H * 2 * st : 0;
+    const size_t b_sin = p.segmented ? (size_t)p.max_units * a.H * st : 0;
+    return *b_segs + *b_off + *b_trans + b_sin;
+}
+
 }  // namespace
 
 void kda::profile_mark(int slot, bool begin, cudaStream_t stream) {
@@ -373,6 +411,78 @@ kda_status kda_fwd_host(const void* q, const void* k, const void* v, const float
     if (s != KDA_OK) return s;
     if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
     if (e2 != cudaSuccess) return cuda_fail(e2, "stream synchronize");
+    return KDA_OK;
+}
+
+kda_status kda_fwd_noalloc(const void* q, const void* k, const void* v, const float* log_alpha,
+                           const float* beta, const float* initial_state,
+                           const int32_t* cu_seqlens, int32_t chunk, void* out,
+                           float* final_state, const kda_dims* dims, void* stream_) {
+    g_last_error[0] = 0;
+    g_last_launches = 0;
+    g_last_path = "";
+    kda::FwdArgs a;
+    kda_status s = validate(q, k, v, log_alpha, beta, initial_state, cu_seqlens, chunk, out,
+                            final_state, dims, true, &a);
+    if (s != KDA_OK) return s;
+    cudaStream_t stream = (cudaStream_t)stream_;
+    if ((int64_t)a.N * a.H == 0) return KDA_OK;
+    int launches = 0;
+    if (!(a.bf16 && a.dk == 128 && a.dv == 128)) {
+        // the CUDA-core path keeps everything on chip: no scratch at all
+        g_last_path = "ffma";
+        cudaError_t e = kda::launch_ffma(a, stream, &launches);
+        g_last_launches = launches;
+        return e == cudaSuccess ? KDA_OK : cuda_fail(e, "kernel launch");
+    }
+    // Segment plan of kda_fwd, with longer segments until the scratch fits.
+    kda::TcPlan p = plan_segments(a);
+    size_t b_segs, b_off, b_trans;
+    size_t need = tc_scratch_bytes(a, p, &b_segs, &b_off, &b_trans);
+    while (need > kNoAllocScratchBytes && p.segmented) {
+        const int64_t nch_seq_max = ((int64_t)a.T + kda::kChunk - 1) / kda::kChunk;
+        const int64_t nch_total = a.cu ? nch_seq_max + a.N : (int64_t)a.B * nch_seq_max;
+        const int64_t seg = (int64_t)p.seg_chunks * 2;
+        p.segmented = seg < nch_seq_max;
+        p.seg_chunks = (int)std::min<int64_t>(p.segmented ? seg : std::max<int64_t>(nch_seq_max, 1),
+                                              1 << 30);
+        p.max_units = (int)(p.segmented ? (nch_total + p.seg_chunks - 1) / p.seg_chunks + a.N : a.N);
+        need = tc_scratch_bytes(a, p, &b_segs, &b_off, &b_trans);
+    }
+    if (need > kNoAllocScratchBytes)
+        return fail(KDA_ERR_UNSUPPORTED,
+                    "kda_fwd_noalloc: %d sequences need %zu bytes of scratch, more than the "
+                    "fixed %zu-byte array",
+                    a.N, need, kNoAllocScratchBytes);
+    char* ws = nullptr;
+    cudaError_t e = noalloc_scratch(&ws);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-allocation scratch)");
+    // Nothing in the scratch needs to start at zero: the segment-table kernel
+    // writes every entry that is read later, pass 1 writes every transition the
+    // scan reads, and the scan writes every incoming state pass 3 reads.
+    kda::TcArgs t;
+    t.q = a.q;
+    t.k = a.k;
+    t.v = a.v;
+    t.log_alpha = a.log_alpha;
+    t.beta = a.beta;
+    t.s0 = a.s0;
+    t.cu = a.cu;
+    t.out = a.out;
+    t.s_final = a.s_final;
+    t.B = a.B;
+    t.T = a.T;
+    t.H = a.H;
+    t.N = a.N;
+    t.segs = (kda::SegEntry*)ws;
+    t.seg_off = (int32_t*)(ws + b_segs);
+    t.n_units = t.seg_off + a.N + 1;
+    t.trans = p.segmented ? (float*)(ws + b_segs + b_off) : nullptr;
+    t.sin = p.segmented ? (float*)(ws + b_segs + b_off + b_trans) : nullptr;
+    g_last_path = "tc";
+    e = kda::launch_tc(t, p, stream, &launches);
+    g_last_launches = launches;
+    if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
     return KDA_OK;
 }
 

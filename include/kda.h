@@ -114,6 +114,36 @@ kda_status kda_fwd_host(const void* q, const void* k, const void* v, const float
                         const int32_t* cu_seqlens, int32_t chunk, void* out,
                         float* final_state, const kda_dims* dims, void* stream);
 
+/*
+ * kda_fwd_noalloc -- kda_fwd for callers that cannot allocate device memory.
+ *
+ * (The pages describe no such entry point; it is an addition of this library.)
+ * Some callers must not allocate on the call path: a serving loop whose device
+ * memory is reserved up front by another allocator, a process whose memory
+ * budget leaves nothing to grow a pool, or code that cannot afford the latency
+ * or implicit synchronisation an allocation may bring.  kda_fwd takes its
+ * temporaries from a stream-ordered pool; this entry point takes them instead
+ * from a fixed 32 MiB scratch array compiled into the library, which every GPU
+ * that loads the library holds until the process exits.  It calls no
+ * cudaMalloc, cudaFree or allocating library routine.
+ *
+ * Arguments, layouts, ownership and results are those of kda_fwd.  The segment
+ * split of long sequences is coarsened (longer segments) until its temporaries
+ * fit in the array; a call whose segment table alone does not fit (about a
+ * million sequences) returns KDA_ERR_UNSUPPORTED and launches nothing.
+ *
+ * Every call shares the one array, which keeps the previous call's contents
+ * (nothing in it has to start at zero).  Calls whose kernels overlap on the GPU
+ * -- on two streams, or from two host threads -- race on the array: order them
+ * on one stream or synchronise between them.  The first call on a device looks
+ * up the array's device address (cudaGetSymbolAddress, with that device
+ * current); make that first call before any stream capture on the device.
+ */
+kda_status kda_fwd_noalloc(const void* q, const void* k, const void* v, const float* log_alpha,
+                           const float* beta, const float* initial_state,
+                           const int32_t* cu_seqlens, int32_t chunk, void* out,
+                           float* final_state, const kda_dims* dims, void* stream);
+
 /* Static description of a status code. */
 const char* kda_status_string(kda_status s);
 
