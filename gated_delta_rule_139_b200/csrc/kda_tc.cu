@@ -60,12 +60,12 @@ enum : int { ERR_WAIT_TIMEOUT = 1, ERR_SEG_OVERFLOW = 2 };
 // ---------------------------------------------------------------- shared memory map
 // Region R1 is reused across the phases of one chunk:
 //   phases 0-1: X1 (A operand, 128 x 128) and BT (B operand, 96 x 128)
-//   phase  2  : As, Ts (fp32 64 x 65) and Ys (fp32 3 x 16 x 17) for (I + A)^-1
+//   phase  2  : As, Ts (fp32, strides 68 and 72) and Ys (fp32 32 x 40) for (I + A)^-1
 //   phases 3-8: SA (bf16 S^T), WB (W^T), UA (U^T), and OS (output staging) or,
 //               in pass 1, MA (bf16 M^T) and UMA (U_M^T)
 struct Lay {
     static constexpr uint32_t X1 = 0, BT = 32768;
-    static constexpr uint32_t AS = 0, TS = 16640, YS = 33280;
+    static constexpr uint32_t AS = 0, TS = 17408, YS = 35840;  // 64x68, 64x72, 32x40 fp32
     static constexpr uint32_t SA = 0, WB = 32768, UA = 49152, OS = 65536, MA = 65536,
                               UMA = 98304;
     static constexpr uint32_t R1 = 114688;
@@ -85,7 +85,7 @@ struct Lay {
     static constexpr uint32_t BYTES = END + 1024;    // + alignment slack
 };
 static_assert(Lay::OS + 16384 <= Lay::R1 && Lay::UMA + 16384 <= Lay::R1, "R1 overflow");
-static_assert(Lay::YS + 3 * 16 * 17 * 4 <= Lay::R1, "R1 overflow");
+static_assert(Lay::YS + 32 * 40 * 4 <= Lay::R1, "R1 overflow");
 
 // TMEM columns (512 allocated).  Pass 3: AP [0,96) W [96,160) U [160,224)
 // O [224,288) S [384,512).  Pass 1: AP/U_M [0,96) W U as above, B [256,384), M [384,512).
@@ -93,7 +93,13 @@ constexpr uint32_t TM_AP = 0, TM_W = 96, TM_U = 160, TM_O = 224;
 constexpr uint32_t TM_B = 256, TM_S = 384, TM_M = 384;
 
 __device__ __forceinline__ float clamp_gate(float x) { return fminf(fmaxf(x, -5.f), 0.f); }
-__device__ __forceinline__ float ex2(float x) { return exp2f(x); }
+// 2^x by the SFU instruction (relative error about 2^-22, flushes results
+// below 2^-126 to zero, which is harmless for the factors here)
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 __device__ __forceinline__ void st8(uint8_t* base, uint32_t off, float a, float b, float c,
                                     float d) {
@@ -103,8 +109,7 @@ __device__ __forceinline__ void st8(uint8_t* base, uint32_t off, float a, float 
     *reinterpret_cast<uint2*>(base + off) = v;
 }
 
-__device__ __forceinline__ void load_bf16x4(const __nv_bfloat16* p, float (&f)[4]) {
-    const uint2 raw = __ldg(reinterpret_cast<const uint2*>(p));
+__device__ __forceinline__ void unpack_bf16x4(const uint2 raw, float (&f)[4]) {
     const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
     const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
     f[0] = __low2float(lo);
@@ -122,79 +127,148 @@ __device__ __forceinline__ bool wait_mma(void* bar, uint32_t& parity) {
     return !__syncthreads_or(!ok);
 }
 
-// Copy 16 TMEM columns x this warp's 32 lanes into a bf16 K-major tile row
-// (chunks c8, c8+1 of row `row`), optionally scaling the TMEM copy by gam.
-__device__ __forceinline__ void stage_row16(uint32_t tm, uint8_t* tile, int R, int row, int col0,
-                                            const float* gam, bool scale_back) {
-    float v[16];
-    tmem_ld16(tm, v);
-    tmem_wait16(v);
+// Copy NB x 16 TMEM columns (starting at TMEM address tm, tile column col0) of
+// this thread's lane into row `row` of a bf16 tile (K-major with R rows, or
+// MN-major with R K-rows when MN is true); optionally scale the TMEM copy by
+// gam[col0 + i] in place.  All loads are issued before the first wait.
+template <int NB, bool MN = false>
+__device__ __forceinline__ void stage_cols(uint32_t tm, uint8_t* tile, int R, int row, int col0,
+                                           const float* gam, bool scale_back) {
+    float v[NB][16];
+#pragma unroll
+    for (int b = 0; b < NB; ++b) tmem_ld16(tm + 16 * b, v[b]);
+#pragma unroll
+    for (int b = 0; b < NB; ++b) tmem_wait16(v[b]);
     const uint32_t base = smem_u32(tile);
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const int c8 = (col0 >> 3) + h;
-        st_shared_v4(base + kmajor_chunk_off(row, c8, R), pack_bf16(v[8 * h + 0], v[8 * h + 1]),
-                     pack_bf16(v[8 * h + 2], v[8 * h + 3]), pack_bf16(v[8 * h + 4], v[8 * h + 5]),
-                     pack_bf16(v[8 * h + 6], v[8 * h + 7]));
-    }
+    for (int b = 0; b < NB; ++b)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const int c8 = ((col0 + 16 * b) >> 3) + hh;
+            const uint32_t off = MN ? mnmajor_chunk_off(row, c8, R) : kmajor_chunk_off(row, c8, R);
+            st_shared_v4(base + off, pack_bf16(v[b][8 * hh + 0], v[b][8 * hh + 1]),
+                         pack_bf16(v[b][8 * hh + 2], v[b][8 * hh + 3]),
+                         pack_bf16(v[b][8 * hh + 4], v[b][8 * hh + 5]),
+                         pack_bf16(v[b][8 * hh + 6], v[b][8 * hh + 7]));
+        }
     if (scale_back) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] *= gam[col0 + i];
-        tmem_st16(tm, v);
+        for (int b = 0; b < NB; ++b) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[b][i] *= gam[col0 + 16 * b + i];
+            tmem_st16(tm + 16 * b, v[b]);
+        }
     }
 }
 
 // ---------------------------------------------------------------- (I + A)^-1
-// As: strictly lower 64 x 64 (fp32, stride 65).  Writes T = (I + A)^-1 into Ts
-// (fp32, stride 65, zeros above the diagonal) by 16 x 16 blocks: diagonal
-// blocks by forward substitution, then T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ.
+constexpr int AS_LD = 68;  // row stride (floats) of As: A-fragment loads hit 32 banks
+constexpr int TS_LD = 72;  // row stride of Ts: B-fragment loads hit 32 banks
+constexpr int YS_LD = 40;  // row stride of the intermediate products
+
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+// d (16 x 8, fp32) += a (16 x 8) . b (8 x 8) on the warp's tensor core (tf32 in,
+// fp32 accumulate).  a: element (m, k) at a[m*lda + k]; b: (k, n) at b[k*ldb + n].
+// Fragments (PTX m16n8k8 .tf32): g = lane/4, t = lane%4; a: (g,t) (g+8,t)
+// (g,t+4) (g+8,t+4); b: (t,g) (t+4,g); d: (g,2t) (g,2t+1) (g+8,2t) (g+8,2t+1).
+__device__ __forceinline__ void warp_mma_tf32(float (&d)[4], const float* a, int lda,
+                                              const float* b, int ldb, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    const uint32_t a0 = to_tf32(a[g * lda + t]), a1 = to_tf32(a[(g + 8) * lda + t]);
+    const uint32_t a2 = to_tf32(a[g * lda + t + 4]), a3 = to_tf32(a[(g + 8) * lda + t + 4]);
+    const uint32_t b0 = to_tf32(b[t * ldb + g]), b1 = to_tf32(b[(t + 4) * ldb + g]);
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void warp_store16x8(float* dst, int ld, const float (&d)[4], float sgn,
+                                               int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    dst[g * ld + 2 * t] = sgn * d[0];
+    dst[g * ld + 2 * t + 1] = sgn * d[1];
+    dst[(g + 8) * ld + 2 * t] = sgn * d[2];
+    dst[(g + 8) * ld + 2 * t + 1] = sgn * d[3];
+}
+
+// As: strictly lower 64 x 64 (fp32, stride AS_LD).  Writes T = (I + A)^-1 into Ts
+// (fp32, stride TS_LD, zeros above the diagonal):
+//  1. the four 16 x 16 diagonal blocks by substitution (one thread per column,
+//     eliminating one known entry at a time so the dependency chain is 16 long);
+//  2. T_10 = -T_11 (A_10 T_00) and T_32 = -T_33 (A_32 T_22), completing the two
+//     32 x 32 diagonal inverses T_lo, T_hi;
+//  3. T[32:64, 0:32] = -T_hi (A[32:64, 0:32] T_lo).
+// The block products of steps 2 and 3 run as tf32 warp MMAs with fp32
+// accumulation (T then enters the chunk products as bf16).
 __device__ void invert_unit_lower(const float* As, float* Ts, float* Ys, int tid) {
-    constexpr int S = 65;
+    const int warp = tid >> 5, lane = tid & 31;
     if (tid < 64) {
         const int b = tid >> 4, j = tid & 15, o = 16 * b;
         float t[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            float v = (i == j) ? 1.f : 0.f;
+        for (int i = 0; i < 16; ++i) t[i] = (i == j) ? 1.f : 0.f;
 #pragma unroll
-            for (int m = 0; m < i; ++m) v = fmaf(-As[(o + i) * S + o + m], t[m], v);
-            t[i] = (i < j) ? 0.f : v;
+        for (int m = 0; m < 15; ++m)
+#pragma unroll
+            for (int i = m + 1; i < 16; ++i) t[i] = fmaf(-As[(o + i) * AS_LD + o + m], t[m], t[i]);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) Ts[(o + i) * TS_LD + o + j] = t[i];
+    } else {
+        // zero everything above the diagonal blocks
+        for (int x = tid - 64; x < 6 * 256; x += NT - 64) {
+            const int p = x >> 8, e = x & 255;
+            const int I = p < 3 ? 0 : p < 5 ? 1 : 2;
+            const int J = p < 3 ? p + 1 : p < 5 ? p - 1 : 3;
+            Ts[(16 * I + (e >> 4)) * TS_LD + 16 * J + (e & 15)] = 0.f;
         }
-#pragma unroll
-        for (int i = 0; i < 16; ++i) Ts[(o + i) * S + o + j] = t[i];
-    }
-    // zero the strictly upper blocks
-    for (int x = tid; x < 6 * 256; x += NT) {
-        const int p = x >> 8, e = x & 255;
-        const int I = p < 3 ? 0 : p < 5 ? 1 : 2;
-        const int J = p < 3 ? p + 1 : p < 5 ? p - 1 : 3;
-        Ts[(16 * I + (e >> 4)) * S + 16 * J + (e & 15)] = 0.f;
     }
     __syncthreads();
-    // levels: distance 1 (3 blocks), 2 (2 blocks), 3 (1 block)
-#pragma unroll 1
-    for (int dist = 1; dist <= 3; ++dist) {
-        const int nblk = 4 - dist;
-        for (int x = tid; x < nblk * 256; x += NT) {
-            const int J = x >> 8, I = J + dist, i = (x >> 4) & 15, j = x & 15;
-            float y = 0.f;
-            for (int K = J; K < I; ++K)
+    // 2. warps 0-3: (I = 1 or 3) x (8-column half nt)
+    if (warp < 4) {
+        const int I = warp < 2 ? 1 : 3, nt = warp & 1, ro = 16 * I, co = ro - 16;
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int m = 0; m < 16; ++m)
-                    y = fmaf(As[(16 * I + i) * S + 16 * K + m], Ts[(16 * K + m) * S + 16 * J + j], y);
-            Ys[(J * 16 + i) * 17 + j] = y;
-        }
-        __syncthreads();
-        for (int x = tid; x < nblk * 256; x += NT) {
-            const int J = x >> 8, I = J + dist, i = (x >> 4) & 15, j = x & 15;
-            float t = 0.f;
-#pragma unroll
-            for (int m = 0; m < 16; ++m)
-                t = fmaf(Ts[(16 * I + i) * S + 16 * I + m], Ys[(J * 16 + m) * 17 + j], t);
-            Ts[(16 * I + i) * S + 16 * J + j] = -t;
-        }
-        __syncthreads();
+        for (int k0 = 0; k0 < 16; k0 += 8)
+            warp_mma_tf32(d, As + ro * AS_LD + co + k0, AS_LD, Ts + (co + k0) * TS_LD + co + 8 * nt,
+                          TS_LD, lane);
+        warp_store16x8(Ys + (warp >> 1) * 16 * YS_LD + 8 * nt, YS_LD, d, 1.f, lane);
     }
+    __syncthreads();
+    if (warp < 4) {
+        const int I = warp < 2 ? 1 : 3, nt = warp & 1, ro = 16 * I, co = ro - 16;
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int k0 = 0; k0 < 16; k0 += 8)
+            warp_mma_tf32(d, Ts + ro * TS_LD + ro + k0, TS_LD,
+                          Ys + (warp >> 1) * 16 * YS_LD + k0 * YS_LD + 8 * nt, YS_LD, lane);
+        warp_store16x8(Ts + ro * TS_LD + co + 8 * nt, TS_LD, d, -1.f, lane);
+    }
+    __syncthreads();
+    // 3. all 8 warps: output tile (16-row mt, 8-column nt) of the 32 x 32 block
+    const int mt = warp >> 2, nt = warp & 3;
+    {
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int k0 = 0; k0 < 32; k0 += 8)
+            warp_mma_tf32(d, As + (32 + 16 * mt) * AS_LD + k0, AS_LD, Ts + k0 * TS_LD + 8 * nt,
+                          TS_LD, lane);
+        warp_store16x8(Ys + 16 * mt * YS_LD + 8 * nt, YS_LD, d, 1.f, lane);
+    }
+    __syncthreads();
+    {
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int k0 = 0; k0 < 32; k0 += 8)
+            warp_mma_tf32(d, Ts + (32 + 16 * mt) * TS_LD + 32 + k0, TS_LD, Ys + k0 * YS_LD + 8 * nt,
+                          YS_LD, lane);
+        warp_store16x8(Ts + (32 + 16 * mt) * TS_LD + 8 * nt, TS_LD, d, -1.f, lane);
+    }
+    __syncthreads();
 }
 
 // ---------------------------------------------------------------- the chunk loop
@@ -265,6 +339,36 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a) {
     __syncthreads();
     tc_fence_after();
 
+    // Global inputs of the next chunk are loaded into registers while the
+    // current chunk's state products run (phases 3-8), so a chunk's phase 0
+    // normally finds them already there.
+    float4 la[8];
+    uint2 kr[8], vr[8], qr[8];
+    float beta_ld;
+    auto prefetch = [&](int64_t tn) {
+        const int Ln = (int)((sg.t_end - tn) < C ? (sg.t_end - tn) : C);
+        const int c0 = 4 * lane;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int r = 8 * warp + i;
+            const int64_t row = ((tn + r) * H + h) * (int64_t)D + c0;
+            la[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+            kr[i] = vr[i] = qr[i] = make_uint2(0u, 0u);
+            if (r < Ln) {
+                la[i] = __ldg(reinterpret_cast<const float4*>(a.log_alpha + row));
+                kr[i] = __ldg(reinterpret_cast<const uint2*>(
+                    reinterpret_cast<const __nv_bfloat16*>(a.k) + row));
+                vr[i] = __ldg(reinterpret_cast<const uint2*>(
+                    reinterpret_cast<const __nv_bfloat16*>(a.v) + row));
+                if (!SEG)
+                    qr[i] = __ldg(reinterpret_cast<const uint2*>(
+                        reinterpret_cast<const __nv_bfloat16*>(a.q) + row));
+            }
+        }
+        beta_ld = (tid < Ln) ? __ldg(a.beta + (tn + tid) * H + h) : 0.f;
+    };
+    if (sg.t_begin < sg.t_end) prefetch(sg.t_begin);
+
     bool ok = true;
     for (int64_t t0 = sg.t_begin; t0 < sg.t_end && ok; t0 += C) {
         const int Lc = (int)((sg.t_end - t0) < C ? (sg.t_end - t0) : C);
@@ -276,20 +380,15 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a) {
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                const int r = 8 * tg + i;
-                float4 la = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (r < Lc)
-                    la = __ldg(reinterpret_cast<const float4*>(
-                        a.log_alpha + ((t0 + r) * H + h) * (int64_t)D + c0));
-                acc[0] += clamp_gate(la.x);
-                acc[1] += clamp_gate(la.y);
-                acc[2] += clamp_gate(la.z);
-                acc[3] += clamp_gate(la.w);
+                acc[0] += clamp_gate(la[i].x);
+                acc[1] += clamp_gate(la[i].y);
+                acc[2] += clamp_gate(la[i].z);
+                acc[3] += clamp_gate(la[i].w);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) g[i][c] = acc[c];
             }
             *reinterpret_cast<float4*>(gsum + tg * D + c0) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-            if (tid < C) beta_s[tid] = tid < Lc ? a.beta[(t0 + tid) * H + h] : 0.f;
+            if (tid < C) beta_s[tid] = beta_ld;
             __syncthreads();
             float off[4] = {0.f, 0.f, 0.f, 0.f}, run[4] = {0.f, 0.f, 0.f, 0.f};
             float ra[4], rb[4], gl[4];
@@ -324,15 +423,10 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a) {
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const int r = 8 * tg + i;
-                const bool valid = r < Lc;
-                const int64_t row = ((t0 + r) * H + h) * (int64_t)D + c0;
-                float kf[4] = {0.f, 0.f, 0.f, 0.f}, qf[4] = {0.f, 0.f, 0.f, 0.f},
-                      vf[4] = {0.f, 0.f, 0.f, 0.f};
-                if (valid) {
-                    load_bf16x4(reinterpret_cast<const __nv_bfloat16*>(a.k) + row, kf);
-                    load_bf16x4(reinterpret_cast<const __nv_bfloat16*>(a.v) + row, vf);
-                    if (!SEG) load_bf16x4(reinterpret_cast<const __nv_bfloat16*>(a.q) + row, qf);
-                }
+                float kf[4], qf[4], vf[4];
+                unpack_bf16x4(kr[i], kf);
+                unpack_bf16x4(vr[i], vf);
+                unpack_bf16x4(qr[i], qf);
                 const float br = beta_s[r];
                 float e1[4], e2[4];
 #pragma unroll
@@ -405,7 +499,7 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a) {
                 }
                 if (!isP) {
 #pragma unroll
-                    for (int j = 0; j < 64; ++j) As[r * 65 + j] = x[j];
+                    for (int j = 0; j < 64; ++j) As[r * AS_LD + j] = x[j];
                 } else {
                     const uint32_t pb = smem_u32(sm + Lay::PB);
 #pragma unroll
@@ -424,7 +518,7 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a) {
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     const int j8 = 2 * (tid & 3) + hh;
-                    const float* t = Ts + r * 65 + 8 * j8;
+                    const float* t = Ts + r * TS_LD + 8 * j8;
                     st_shared_v4(tb + kmajor_chunk_off(r, j8, 64), pack_bf16(t[0], t[1]),
                                  pack_bf16(t[2], t[3]), pack_bf16(t[4], t[5]), pack_bf16(t[6], t[7]));
                 }
@@ -448,35 +542,24 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a) {
                 mma_bf16(tmem + TM_U, mnmajor_desc(vb, 64, s), kmajor_desc(tb, 64, s), id, s > 0);
             mma_commit(bar);
         }
-        // meanwhile: bf16 copy of the state into SA (and MA), state scaled by gamma in TMEM
-        if (warp >= 4) {
-#pragma unroll 1
-            for (int c0 = 0; c0 < D; c0 += 16)
-                stage_row16(tq + (SEG ? TM_B : TM_S) + c0, sm + Lay::SA, 128, lrow, c0, gam, true);
-        } else if (SEG) {
-#pragma unroll 1
-            for (int c0 = 0; c0 < D; c0 += 16)
-                stage_row16(tq + TM_M + c0, sm + Lay::MA, 128, lrow, c0, gam, true);
+        // meanwhile: bf16 copy of the state into SA (and MA), state scaled by gamma in
+        // TMEM.  Pass 3: warps 4-7 take columns 0-63, warps 0-3 columns 64-127 of the
+        // same lanes.  Pass 1: warps 4-7 take B, warps 0-3 take M.
+        if (!SEG) {
+            const int c0 = warp >= 4 ? 0 : 64;
+            stage_cols<4>(tq + TM_S + c0, sm + Lay::SA, 128, lrow, c0, gam, true);
+        } else {
+            const uint32_t col = warp >= 4 ? TM_B : TM_M;
+            uint8_t* tile = sm + (warp >= 4 ? Lay::SA : Lay::MA);
+            stage_cols<4>(tq + col, tile, 128, lrow, 0, gam, true);
+            stage_cols<4>(tq + col + 64, tile, 128, lrow, 64, gam, true);
         }
         tmem_st_wait();
         if (!(ok = wait_mma(bar, parity))) break;
-        // W^T -> WB (MN-major B operand: K rows = c, MN = r)
-        if (warp < 4) {
-            const uint32_t wb = smem_u32(sm + Lay::WB);
-#pragma unroll 1
-            for (int q = 0; q < 4; ++q) {
-                float v[16];
-                tmem_ld16(tq + TM_W + 16 * q, v);
-                tmem_wait16(v);
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh)
-                    st_shared_v4(wb + mnmajor_chunk_off(lrow, 2 * q + hh, 128),
-                                 pack_bf16(v[8 * hh + 0], v[8 * hh + 1]),
-                                 pack_bf16(v[8 * hh + 2], v[8 * hh + 3]),
-                                 pack_bf16(v[8 * hh + 4], v[8 * hh + 5]),
-                                 pack_bf16(v[8 * hh + 6], v[8 * hh + 7]));
-            }
-        }
+        // W^T -> WB (MN-major B operand: K rows = c, MN = r); warps 0-3 columns 0-31,
+        // warps 4-7 columns 32-63
+        stage_cols<2, true>(tq + TM_W + (warp >= 4 ? 32 : 0), sm + Lay::WB, 128, lrow,
+                            warp >= 4 ? 32 : 0, nullptr, false);
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
@@ -504,17 +587,17 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a) {
             }
             mma_commit(bar);
         }
+        if (t0 + C < sg.t_end) prefetch(t0 + C);
         if (!(ok = wait_mma(bar, parity))) break;
 
         // ============ phase 6: U^T -> UA (bf16, K-major, 128 x 64); pass 1 also U_M^T -> UMA
-        if (warp < 4) {
-#pragma unroll 1
-            for (int c0 = 0; c0 < C; c0 += 16)
-                stage_row16(tq + TM_U + c0, sm + Lay::UA, 128, lrow, c0, nullptr, false);
-        } else if (SEG) {
-#pragma unroll 1
-            for (int c0 = 0; c0 < C; c0 += 16)
-                stage_row16(tq + TM_AP + c0, sm + Lay::UMA, 128, lrow, c0, nullptr, false);
+        if (!SEG) {
+            const int c0 = warp >= 4 ? 32 : 0;
+            stage_cols<2>(tq + TM_U + c0, sm + Lay::UA, 128, lrow, c0, nullptr, false);
+        } else if (warp < 4) {
+            stage_cols<4>(tq + TM_U, sm + Lay::UA, 128, lrow, 0, nullptr, false);
+        } else {
+            stage_cols<4>(tq + TM_AP, sm + Lay::UMA, 128, lrow, 0, nullptr, false);
         }
         fence_async_smem();
         tc_fence_before();
@@ -549,15 +632,18 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a) {
         // ============ phase 8: O^T -> out (via shared memory, 16-byte global stores)
         if (!SEG) {
             __nv_bfloat16* os = reinterpret_cast<__nv_bfloat16*>(sm + Lay::OS);
-            if (warp < 4) {
-#pragma unroll 1
-                for (int q = 0; q < 4; ++q) {
-                    float v[16];
-                    tmem_ld16(tq + TM_O + 16 * q, v);
-                    tmem_wait16(v);
+            {  // warps 0-3 rows r = 0-31, warps 4-7 rows 32-63 of this thread's column e
+                const int r0 = warp >= 4 ? 32 : 0;
+                float v[2][16];
+                tmem_ld16(tq + TM_O + r0, v[0]);
+                tmem_ld16(tq + TM_O + r0 + 16, v[1]);
+                tmem_wait16(v[0]);
+                tmem_wait16(v[1]);
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) os[(16 * q + i) * D + lrow] = __float2bfloat16_rn(v[i]);
-                }
+                for (int b = 0; b < 2; ++b)
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        os[(r0 + 16 * b + i) * D + lrow] = __float2bfloat16_rn(v[b][i]);
             }
             tc_fence_before();
             __syncthreads();
@@ -677,41 +763,68 @@ __global__ void __launch_bounds__(1024) seg_setup_kernel(const int32_t* cu, int 
 
 // ---------------------------------------------------------------- segment scan
 // S_in^T(j+1) = S_in^T(j) M_j^T + B_j^T for the 16 rows e in [16*blockIdx.z, +16)
-// of S^T, sequentially over the segments of sequence n, head h.
+// of S^T, sequentially over the segments of sequence n, head h.  M_j^T (64 KB)
+// is staged in shared memory; the next one is loaded into registers while the
+// current product runs.
+constexpr int SCAN_SMEM = 2 * D * D * 4 + 16 * D * 4;
+
 __global__ void __launch_bounds__(256) seg_scan_kernel(TcArgs a) {
-    __shared__ float S[16][D];
+    extern __shared__ float4 scan_smem4[];
+    float* Ms = reinterpret_cast<float*>(scan_smem4);  // [2][128][128]
+    float* S = Ms + 2 * D * D;                        // [16][128]
     const int n = blockIdx.x, h = blockIdx.y, e0 = 16 * blockIdx.z, H = a.H;
     const int tid = threadIdx.x, el = tid >> 4, cg = tid & 15;
     const int32_t u0 = a.seg_off[n], u1 = a.seg_off[n + 1];
-    if (u1 - u0 <= 1 || u0 >= *a.n_units) return;
+    const int32_t nu = *a.n_units;
+    if (u1 - u0 <= 1 || u0 >= nu) return;
+    const int32_t last = (u1 < nu ? u1 : nu) - 1;  // segments u0 .. last; transitions u0 .. last-1
     // S_in of segment 0, also copied to the workspace so that pass 3 never reads
     // initial_state while another segment may be writing final_state (they may
     // be the same buffer)
     for (int x = tid; x < 16 * D; x += 256) {
         const int r = x / D, c = x % D;
         const float v = a.s0 ? a.s0[(((int64_t)n * H + h) * D + c) * D + e0 + r] : 0.f;
-        S[r][c] = v;
+        S[r * D + c] = v;
         a.sin[((int64_t)u0 * H + h) * D * D + (int64_t)(e0 + r) * D + c] = v;
     }
+    float4 pre[16];
+    auto load_m = [&](int32_t uu) {
+        const float4* Mt = reinterpret_cast<const float4*>(a.trans + ((int64_t)uu * H + h) * 2 * D * D + D * D);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pre[i] = __ldg(Mt + tid + 256 * i);
+    };
+    auto store_m = [&](int buf) {
+        float4* dst = reinterpret_cast<float4*>(Ms + buf * D * D);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) dst[tid + 256 * i] = pre[i];
+    };
+    if (u0 < last) {
+        load_m(u0);
+        store_m(0);
+    }
     __syncthreads();
-    for (int32_t uu = u0; uu + 1 < u1 && uu + 1 < *a.n_units; ++uu) {
+    for (int32_t uu = u0; uu < last; ++uu) {
+        const int buf = (uu - u0) & 1;
+        if (uu + 1 < last) load_m(uu + 1);
         const float* Bt = a.trans + ((int64_t)uu * H + h) * 2 * D * D;
-        const float* Mt = Bt + D * D;
         float acc[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = Bt[(int64_t)(e0 + el) * D + cg + 16 * i];
+        for (int i = 0; i < 8; ++i) acc[i] = __ldg(Bt + (int64_t)(e0 + el) * D + cg + 16 * i);
+        const float* M = Ms + buf * D * D;
+#pragma unroll 4
         for (int c = 0; c < D; ++c) {
-            const float s = S[el][c];
+            const float sv = S[el * D + c];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) acc[i] = fmaf(s, __ldg(Mt + (int64_t)c * D + cg + 16 * i), acc[i]);
+            for (int i = 0; i < 8; ++i) acc[i] = fmaf(sv, M[c * D + cg + 16 * i], acc[i]);
         }
-        __syncthreads();
+        __syncthreads();  // everyone is done reading S and M[buf]
         float* dst = a.sin + ((int64_t)(uu + 1) * H + h) * D * D + (int64_t)(e0 + el) * D;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            S[el][cg + 16 * i] = acc[i];
+            S[el * D + cg + 16 * i] = acc[i];
             dst[cg + 16 * i] = acc[i];
         }
+        if (uu + 1 < last) store_m(buf ^ 1);
         __syncthreads();
     }
 }
@@ -736,6 +849,9 @@ cudaError_t launch_tc(const TcArgs& a, const TcPlan& p, cudaStream_t stream, int
         err = cudaFuncSetAttribute(tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    (int)Lay::BYTES);
         if (err == cudaSuccess)
+            err = cudaFuncSetAttribute(seg_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       SCAN_SMEM);
+        if (err == cudaSuccess)
             err = cudaFuncSetAttribute(tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)Lay::BYTES);
         if (err != cudaSuccess) return err;
@@ -755,7 +871,7 @@ cudaError_t launch_tc(const TcArgs& a, const TcPlan& p, cudaStream_t stream, int
         *launches += 1;
         if ((err = cudaGetLastError()) != cudaSuccess) return err;
         profile_mark(SLOT_SCAN, true, stream);
-        seg_scan_kernel<<<dim3((unsigned)a.N, (unsigned)a.H, D / 16), 256, 0, stream>>>(a);
+        seg_scan_kernel<<<dim3((unsigned)a.N, (unsigned)a.H, D / 16), 256, SCAN_SMEM, stream>>>(a);
         profile_mark(SLOT_SCAN, false, stream);
         *launches += 1;
         if ((err = cudaGetLastError()) != cudaSuccess) return err;
