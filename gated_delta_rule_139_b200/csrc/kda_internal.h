@@ -1,5 +1,6 @@
 // Internal declarations shared by the C-ABI layer and the kernels of libkda.so.
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -60,6 +61,12 @@ struct TcArgs {
     int32_t* n_units;   // [1]
     float* trans;       // [max_units, H, 2, 128, 128]: B^T then M^T of each segment
     float* sin;         // [max_units, H, 128, 128]: S_in^T of each segment
+};
+
+// TMA descriptors of the q, k, v (bf16) and log_alpha (fp32) tensors, viewed
+// as [T, H, 128] with a (128, 1, 64) tile box; passed as a grid constant.
+struct TcMaps {
+    CUtensorMap q, k, v, la;
 };
 
 struct TcPlan {

@@ -38,6 +38,9 @@
 // product whose factors are both <= 1 (underflow to 0 is the correct limit).
 #include <cuda_bf16.h>
 #include <stdint.h>
+#include <string.h>
+
+#include <mutex>
 
 #include "kda_internal.h"
 #include "tc_common.cuh"
@@ -59,33 +62,49 @@ enum : int { ERR_WAIT_TIMEOUT = 1, ERR_SEG_OVERFLOW = 2 };
 
 // ---------------------------------------------------------------- shared memory map
 // Region R1 is reused across the phases of one chunk:
-//   phases 0-1: X1 (A operand, 128 x 128) and BT (B operand, 96 x 128)
-//   phase  2  : As, Ts (fp32, strides 68 and 72) and Ys (fp32 32 x 40) for (I + A)^-1
-//   phases 3-8: SA (bf16 S^T), WB (W^T), UA (U^T), and OS (output staging) or,
-//               in pass 1, MA (bf16 M^T) and UMA (U_M^T)
-struct Lay {
+//   phases 0-3: X1 (A operand, 128 x 128, K-major: rows 0-63 k e^{g-rho}, rows
+//               64-127 q e^{g-rho}); its k rows (bytes [0,8K) and [16K,24K)) are read
+//               again by the phase-3 W products, as an MN-major operand.
+//               BT (B operand, 96 x 128) until the phase-1 product completes.
+//   phase  2  : As, Ts (fp32, strides 68 and 72) in BT's place, Ys in a q-row hole,
+//               then TB (bf16 T diag(beta)) in the other q-row hole
+//   phases 3-8: SA (bf16 S^T) over As/Ts, WB (W^T) and UA (U^T) over X1;
+//               pass 1 adds MA (bf16 M^T) after Ts
+// RAW holds the next chunk's k, log alpha (and q) tiles, written by TMA while
+// the current chunk is processed; RV0/RV1 alternate as the chunk's v tile, which
+// TMA writes directly in the 128-byte-swizzled MN-major operand layout.
+template <bool SEG>
+struct LayT {
     static constexpr uint32_t X1 = 0, BT = 32768;
-    static constexpr uint32_t AS = 0, TS = 17408, YS = 35840;  // 64x68, 64x72, 32x40 fp32
-    static constexpr uint32_t SA = 0, WB = 32768, UA = 49152, OS = 65536, MA = 65536,
-                              UMA = 98304;
-    static constexpr uint32_t R1 = 114688;
-    static constexpr uint32_t QT = R1;               // 64 x 128, K-major
-    static constexpr uint32_t KB = QT + 16384;       // 64 x 128, MN-major
-    static constexpr uint32_t VB = KB + 16384;       // 64 x 128, MN-major
-    static constexpr uint32_t KD = VB + 16384;       // 64 x 128, MN-major
-    static constexpr uint32_t TB = KD + 16384;       // 64 x 64, K-major
-    static constexpr uint32_t PB = TB + 8192;        // 64 x 64, K-major
-    static constexpr uint32_t GSUM = PB + 8192;      // fp32 [8][128]
-    static constexpr uint32_t REFS = GSUM + 4096;    // fp32 [4][128]: rho_a, rho_m, rho_b, g_last
-    static constexpr uint32_t GAM = REFS + 2048;     // fp32 [128]
-    static constexpr uint32_t BETA = GAM + 512;      // fp32 [64]
-    static constexpr uint32_t BAR = BETA + 256;      // mbarrier
-    static constexpr uint32_t TMEMP = BAR + 16;      // TMEM base address
+    static constexpr uint32_t AS = 32768, TS = AS + 17408, YS = 24576, TB = 8192;
+    static constexpr uint32_t SA = 32768, WB = 0, UA = 16384, MA = 69632;
+    static constexpr uint32_t R1 = SEG ? 102400 : 69632;
+    static constexpr uint32_t QT = R1;                            // pass 3: 64 x 128, K-major
+    static constexpr uint32_t OS = QT;                            // output staging (QT is dead)
+    static constexpr uint32_t KD = SEG ? R1 : QT + 16384;         // 64 x 128, MN-major
+    static constexpr uint32_t UMA = KD + 16384;                   // pass 1: 128 x 64, K-major
+    static constexpr uint32_t PB = KD + 16384;                    // pass 3: 64 x 64, K-major
+    static constexpr uint32_t RAW = SEG ? UMA + 16384 : PB + 8192;
+    static constexpr uint32_t RK = RAW, RL = RAW + 16384;
+    static constexpr uint32_t RQ = RAW + 49152;                   // pass 3 only
+    static constexpr uint32_t RV = RAW + (SEG ? 49152 : 65536);   // two 16 KB buffers
+    static constexpr uint32_t RAW_TX = SEG ? 65536 : 81920;       // TMA bytes per chunk
+    static constexpr uint32_t GSUM = RV + 32768;                  // fp32 [8][128]
+    static constexpr uint32_t GAM = GSUM + 4096;                  // fp32 [128] e^{g_last}
+    static constexpr uint32_t EHA = GAM + 512;                    // fp32 [128] e^{rho_a}
+    static constexpr uint32_t EHB = EHA + 512;                    // fp32 [128] e^{rho_b}
+    static constexpr uint32_t BETA = EHB + 512;                   // fp32 [64]
+    static constexpr uint32_t BAR = BETA + 256;                   // 2 mbarriers: MMA, TMA
+    static constexpr uint32_t TMEMP = BAR + 16;                   // TMEM base address
     static constexpr uint32_t END = TMEMP + 16;
-    static constexpr uint32_t BYTES = END + 1024;    // + alignment slack
+    static constexpr uint32_t BYTES = END + 1024;                 // + alignment slack
 };
-static_assert(Lay::OS + 16384 <= Lay::R1 && Lay::UMA + 16384 <= Lay::R1, "R1 overflow");
-static_assert(Lay::YS + 32 * 40 * 4 <= Lay::R1, "R1 overflow");
+static_assert(LayT<false>::TS + 64 * 72 * 4 <= LayT<false>::R1, "As/Ts overflow");
+static_assert(LayT<false>::YS + 32 * 40 * 4 <= 32768 && LayT<false>::TB + 8192 <= 16384,
+              "Ys/TB must sit in the q-row holes of X1");
+static_assert(LayT<false>::SA + 32768 <= LayT<false>::R1, "SA overflow");
+static_assert(LayT<true>::MA + 32768 <= LayT<true>::R1, "MA overflow");
+static_assert(LayT<false>::BYTES <= 232448 && LayT<true>::BYTES <= 232448, "shared memory");
 
 // TMEM columns (512 allocated).  Pass 3: AP [0,96) W [96,160) U [160,224)
 // O [224,288) S [384,512).  Pass 1: AP/U_M [0,96) W U as above, B [256,384), M [384,512).
@@ -159,6 +178,23 @@ __device__ __forceinline__ void stage_cols(uint32_t tm, uint8_t* tile, int R, in
             tmem_st16(tm + 16 * b, v[b]);
         }
     }
+}
+
+// ---------------------------------------------------------------- TMA
+__device__ __forceinline__ void mbar_expect_tx(void* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+// one [64 tokens][box width] tile of a [T, H, 128] tensor at (x, h, t0); rows
+// past the tensor's end are filled with zeros
+__device__ __forceinline__ void tma_tile(void* dst, const CUtensorMap* map, int x, int h, int t0,
+                                         void* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(h), "r"(t0), "r"(smem_u32(bar))
+        : "memory");
 }
 
 // ---------------------------------------------------------------- (I + A)^-1
@@ -273,7 +309,8 @@ __device__ void invert_unit_lower(const float* As, float* Ts, float* Ys, int tid
 
 // ---------------------------------------------------------------- the chunk loop
 template <bool SEG>
-__global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a) {
+__global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_constant__ TcMaps maps) {
+    using Lay = LayT<SEG>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -285,8 +322,11 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a) {
 
     float* gsum = reinterpret_cast<float*>(sm + Lay::GSUM);
     float* gam = reinterpret_cast<float*>(sm + Lay::GAM);
+    float* eha = reinterpret_cast<float*>(sm + Lay::EHA);
+    float* ehb = reinterpret_cast<float*>(sm + Lay::EHB);
     float* beta_s = reinterpret_cast<float*>(sm + Lay::BETA);
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + Lay::BAR);
+    uint64_t* bar_raw = bar + 1;
     uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(sm + Lay::TMEMP);
 
     if (warp == 0) {
@@ -295,6 +335,7 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a) {
     }
     if (tid == 0) {
         mbar_init(bar, 1);
+        mbar_init(bar_raw, 1);
         fence_mbar_init();
     }
     tc_fence_before();
@@ -339,43 +380,52 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a) {
     __syncthreads();
     tc_fence_after();
 
-    // Global inputs of the next chunk are loaded into registers while the
-    // current chunk's state products run (phases 3-8), so a chunk's phase 0
-    // normally finds them already there.
-    float4 la[8];
-    uint2 kr[8], vr[8], qr[8];
-    float beta_ld;
-    auto prefetch = [&](int64_t tn) {
-        const int Ln = (int)((sg.t_end - tn) < C ? (sg.t_end - tn) : C);
-        const int c0 = 4 * lane;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int r = 8 * warp + i;
-            const int64_t row = ((tn + r) * H + h) * (int64_t)D + c0;
-            la[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-            kr[i] = vr[i] = qr[i] = make_uint2(0u, 0u);
-            if (r < Ln) {
-                la[i] = __ldg(reinterpret_cast<const float4*>(a.log_alpha + row));
-                kr[i] = __ldg(reinterpret_cast<const uint2*>(
-                    reinterpret_cast<const __nv_bfloat16*>(a.k) + row));
-                vr[i] = __ldg(reinterpret_cast<const uint2*>(
-                    reinterpret_cast<const __nv_bfloat16*>(a.v) + row));
-                if (!SEG)
-                    qr[i] = __ldg(reinterpret_cast<const uint2*>(
-                        reinterpret_cast<const __nv_bfloat16*>(a.q) + row));
-            }
-        }
-        beta_ld = (tid < Ln) ? __ldg(a.beta + (tn + tid) * H + h) : 0.f;
+    // The next chunk's q, k, v and log alpha tiles are copied by TMA into RAW
+    // while the current chunk is processed (issued once every thread has read
+    // the current tiles into registers); beta goes through registers.
+    auto issue_raw = [&](int64_t tn, int vbuf) {
+        mbar_expect_tx(bar_raw, Lay::RAW_TX);
+        tma_tile(sm + Lay::RK, &maps.k, 0, h, (int)tn, bar_raw);
+        tma_tile(sm + Lay::RL, &maps.la, 0, h, (int)tn, bar_raw);
+        if (!SEG) tma_tile(sm + Lay::RQ, &maps.q, 0, h, (int)tn, bar_raw);
+        uint8_t* rv = sm + Lay::RV + vbuf * 16384;  // two 64-channel swizzled halves
+        tma_tile(rv, &maps.v, 0, h, (int)tn, bar_raw);
+        tma_tile(rv + 8192, &maps.v, 64, h, (int)tn, bar_raw);
     };
-    if (sg.t_begin < sg.t_end) prefetch(sg.t_begin);
+    uint32_t raw_parity = 0;
+    float beta_ld = 0.f;
+    if (sg.t_begin < sg.t_end) {
+        if (tid == 0) issue_raw(sg.t_begin, 0);
+        if (tid < C && sg.t_begin + tid < sg.t_end) beta_ld = __ldg(a.beta + (sg.t_begin + tid) * H + h);
+    }
 
     bool ok = true;
-    for (int64_t t0 = sg.t_begin; t0 < sg.t_end && ok; t0 += C) {
+    int vbuf = 0;  // RV buffer of the current chunk
+    for (int64_t t0 = sg.t_begin; t0 < sg.t_end && ok; t0 += C, vbuf ^= 1) {
         const int Lc = (int)((sg.t_end - t0) < C ? (sg.t_end - t0) : C);
 
         // ============ phase 0: gates, scaled operands
         {
             const int c4 = lane, tg = warp, c0 = 4 * c4;
+            float4 la[8];
+            uint2 kr[8], qr[8];
+            if (!(ok = !__syncthreads_or(!mbar_wait(bar_raw, raw_parity, &g_tc_status,
+                                                    ERR_WAIT_TIMEOUT)))) break;
+            raw_parity ^= 1u;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {  // rows past the segment end act as identity steps
+                const int r = 8 * tg + i;
+                la[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+                kr[i] = qr[i] = make_uint2(0u, 0u);
+                if (r < Lc) {
+                    la[i] = *reinterpret_cast<const float4*>(sm + Lay::RL + (r * D + c0) * 4);
+                    kr[i] = *reinterpret_cast<const uint2*>(sm + Lay::RK + (r * D + c0) * 2);
+                    if (!SEG) qr[i] = *reinterpret_cast<const uint2*>(sm + Lay::RQ + (r * D + c0) * 2);
+                } else {  // the v tile is an operand as TMA wrote it: clear rows past the end
+                    *reinterpret_cast<uint2*>(sm + Lay::RV + vbuf * 16384 + mnmajor_off(r, c0, 64)) =
+                        make_uint2(0u, 0u);
+                }
+            }
             float g[8][4];
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -390,6 +440,11 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a) {
             *reinterpret_cast<float4*>(gsum + tg * D + c0) = make_float4(acc[0], acc[1], acc[2], acc[3]);
             if (tid < C) beta_s[tid] = beta_ld;
             __syncthreads();
+            // every thread holds its raw inputs: RAW may now receive the next chunk
+            if (t0 + C < sg.t_end) {
+                if (tid == 0) issue_raw(t0 + C, vbuf ^ 1);
+                beta_ld = (tid < C && t0 + C + tid < sg.t_end) ? __ldg(a.beta + (t0 + C + tid) * H + h) : 0.f;
+            }
             float off[4] = {0.f, 0.f, 0.f, 0.f}, run[4] = {0.f, 0.f, 0.f, 0.f};
             float ra[4], rb[4], gl[4];
 #pragma unroll
@@ -418,16 +473,18 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a) {
             }
             if (tg == 0) {
 #pragma unroll
-                for (int c = 0; c < 4; ++c) gam[c0 + c] = ex2(gl[c] * LOG2E);
+                for (int c = 0; c < 4; ++c) {
+                    gam[c0 + c] = ex2(gl[c] * LOG2E);
+                    eha[c0 + c] = ex2(ra[c] * LOG2E);
+                    ehb[c0 + c] = ex2(rb[c] * LOG2E);
+                }
             }
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const int r = 8 * tg + i;
-                float kf[4], qf[4], vf[4];
+                float kf[4], qf[4];
                 unpack_bf16x4(kr[i], kf);
-                unpack_bf16x4(vr[i], vf);
                 unpack_bf16x4(qr[i], qf);
-                const float br = beta_s[r];
                 float e1[4], e2[4];
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
@@ -448,11 +505,6 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a) {
                 if (!SEG)
                     st8(sm + Lay::QT, kmajor_off(r, c0, 64), qf[0] * e1[0] * Eh[0],
                         qf[1] * e1[1] * Eh[1], qf[2] * e1[2] * Eh[2], qf[3] * e1[3] * Eh[3]);
-                st8(sm + Lay::KB, mnmajor_off(r, c0, 64), br * kf[0] * e1[0] * Eh[0],
-                    br * kf[1] * e1[1] * Eh[1], br * kf[2] * e1[2] * Eh[2],
-                    br * kf[3] * e1[3] * Eh[3]);
-                st8(sm + Lay::VB, mnmajor_off(r, c0, 64), br * vf[0], br * vf[1], br * vf[2],
-                    br * vf[3]);
                 st8(sm + Lay::KD, mnmajor_off(r, c0, 64), kf[0] * e2[0] * Dh[0],
                     kf[1] * e2[1] * Dh[1], kf[2] * e2[2] * Dh[2], kf[3] * e2[3] * Dh[3]);
             }
@@ -519,8 +571,11 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a) {
                 for (int hh = 0; hh < 2; ++hh) {
                     const int j8 = 2 * (tid & 3) + hh;
                     const float* t = Ts + r * TS_LD + 8 * j8;
-                    st_shared_v4(tb + kmajor_chunk_off(r, j8, 64), pack_bf16(t[0], t[1]),
-                                 pack_bf16(t[2], t[3]), pack_bf16(t[4], t[5]), pack_bf16(t[6], t[7]));
+                    const float* bj = beta_s + 8 * j8;
+                    st_shared_v4(tb + kmajor_chunk_off(r, j8, 64), pack_bf16(t[0] * bj[0], t[1] * bj[1]),
+                                 pack_bf16(t[2] * bj[2], t[3] * bj[3]),
+                                 pack_bf16(t[4] * bj[4], t[5] * bj[5]),
+                                 pack_bf16(t[6] * bj[6], t[7] * bj[7]));
                 }
             }
         }
@@ -528,18 +583,27 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a) {
         tc_fence_before();
         __syncthreads();
 
-        // ============ phase 3: W^T = (beta K e^g)^T T^T, U'^T = (beta V)^T T^T
+        // ============ phase 3: with TB = T diag(beta) and the per-half factors e^{rho_h}:
+        //   W^T  = e^{rho_a} (X1k_a)^T TB_a^T + e^{rho_b} (X1k_b)^T TB_b^T  (combined at staging)
+        //   U'^T = V^T TB^T
+        // X1's k rows serve as an MN-major operand (K rows = tokens, MN blocks 16 KB apart);
+        // the v tile is used as TMA wrote it.
         if (tid == 0) {
             tc_fence_after();
-            const uint32_t kb = smem_u32(sm + Lay::KB), vb = smem_u32(sm + Lay::VB),
-                           tb = smem_u32(sm + Lay::TB);
+            const uint32_t x1 = smem_u32(sm + Lay::X1), tb = smem_u32(sm + Lay::TB),
+                           rv = smem_u32(sm + Lay::RV + vbuf * 16384);
             constexpr uint32_t id = idesc_bf16(128, 64, true, false);
 #pragma unroll
-            for (int s = 0; s < 4; ++s)
-                mma_bf16(tmem + TM_W, mnmajor_desc(kb, 64, s), kmajor_desc(tb, 64, s), id, s > 0);
+            for (int s = 0; s < 2; ++s)
+                mma_bf16(tmem + TM_W, sdesc(x1 + s * 2048, 16384, 1024), kmajor_desc(tb, 64, s), id,
+                         s > 0);
+#pragma unroll
+            for (int s = 0; s < 2; ++s)
+                mma_bf16(tmem + TM_AP, sdesc(x1 + 4096 + s * 2048, 16384, 1024),
+                         kmajor_desc(tb, 64, s + 2), id, s > 0);
 #pragma unroll
             for (int s = 0; s < 4; ++s)
-                mma_bf16(tmem + TM_U, mnmajor_desc(vb, 64, s), kmajor_desc(tb, 64, s), id, s > 0);
+                mma_bf16(tmem + TM_U, mnmajor_desc(rv, 64, s), kmajor_desc(tb, 64, s), id, s > 0);
             mma_commit(bar);
         }
         // meanwhile: bf16 copy of the state into SA (and MA), state scaled by gamma in
@@ -556,10 +620,34 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a) {
         }
         tmem_st_wait();
         if (!(ok = wait_mma(bar, parity))) break;
-        // W^T -> WB (MN-major B operand: K rows = c, MN = r); warps 0-3 columns 0-31,
-        // warps 4-7 columns 32-63
-        stage_cols<2, true>(tq + TM_W + (warp >= 4 ? 32 : 0), sm + Lay::WB, 128, lrow,
-                            warp >= 4 ? 32 : 0, nullptr, false);
+        // W^T = e^{rho_a} Wa^T + e^{rho_b} Wb^T (lane = channel c) -> WB (MN-major B
+        // operand: K rows = c, MN = token r); warps 0-3 tokens 0-31, warps 4-7 tokens 32-63
+        {
+            const int r0 = warp >= 4 ? 32 : 0;
+            float wa[2][16], wbv[2][16];
+            tmem_ld16(tq + TM_W + r0, wa[0]);
+            tmem_ld16(tq + TM_W + r0 + 16, wa[1]);
+            tmem_ld16(tq + TM_AP + r0, wbv[0]);
+            tmem_ld16(tq + TM_AP + r0 + 16, wbv[1]);
+            tmem_wait16(wa[0]);
+            tmem_wait16(wa[1]);
+            tmem_wait16(wbv[0]);
+            tmem_wait16(wbv[1]);
+            const float ea = eha[lrow], eb = ehb[lrow];
+            const uint32_t wbs = smem_u32(sm + Lay::WB);
+#pragma unroll
+            for (int b = 0; b < 2; ++b)
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    float w[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        w[i] = fmaf(ea, wa[b][8 * hh + i], eb * wbv[b][8 * hh + i]);
+                    st_shared_v4(wbs + mnmajor_chunk_off(lrow, ((r0 + 16 * b) >> 3) + hh, 128),
+                                 pack_bf16(w[0], w[1]), pack_bf16(w[2], w[3]),
+                                 pack_bf16(w[4], w[5]), pack_bf16(w[6], w[7]));
+                }
+        }
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
@@ -587,7 +675,6 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a) {
             }
             mma_commit(bar);
         }
-        if (t0 + C < sg.t_end) prefetch(t0 + C);
         if (!(ok = wait_mma(bar, parity))) break;
 
         // ============ phase 6: U^T -> UA (bf16, K-major, 128 x 64); pass 1 also U_M^T -> UMA
@@ -831,7 +918,47 @@ __global__ void __launch_bounds__(256) seg_scan_kernel(TcArgs a) {
 
 }  // namespace
 
-size_t tc_smem_bytes() { return Lay::BYTES; }
+size_t tc_smem_bytes() { return LayT<false>::BYTES; }
+
+namespace {
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// [T, H, 128] tensor, tile box (128 channels, 1 head, 64 tokens) without swizzle,
+// or (64 channels, 1 head, 64 tokens) with the 128-byte swizzle of the MMA operand
+// layouts; zero fill past the end.
+cudaError_t tile_map(CUtensorMap* m, const void* base, bool f32, int H, int64_t T, bool sw128) {
+    EncodeTiledFn fn = encode_tiled();
+    if (!fn) return cudaErrorNotSupported;
+    const cuuint64_t e = f32 ? 4 : 2;
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T};
+    const cuuint64_t strides[2] = {(cuuint64_t)D * e, (cuuint64_t)H * D * e};
+    const cuuint32_t box[3] = {(cuuint32_t)(sw128 ? 64 : D), 1, (cuuint32_t)C};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r =
+        fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+           const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+           sw128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+}  // namespace
 
 cudaError_t tc_take_status(int* code) {
     int zero = 0;
@@ -847,15 +974,25 @@ cudaError_t launch_tc(const TcArgs& a, const TcPlan& p, cudaStream_t stream, int
     if (err != cudaSuccess) return err;
     if (dev >= kMaxDevices || !attr_set[dev][0]) {
         err = cudaFuncSetAttribute(tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)Lay::BYTES);
+                                   (int)LayT<false>::BYTES);
         if (err == cudaSuccess)
             err = cudaFuncSetAttribute(seg_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        SCAN_SMEM);
         if (err == cudaSuccess)
             err = cudaFuncSetAttribute(tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)Lay::BYTES);
+                                       (int)LayT<true>::BYTES);
         if (err != cudaSuccess) return err;
         if (dev < kMaxDevices) attr_set[dev][0] = true;
+    }
+    TcMaps maps;
+    memset(&maps, 0, sizeof maps);
+    const int64_t tokens = (int64_t)a.B * a.T;
+    if (tokens > 0) {
+        if ((err = tile_map(&maps.q, a.q, false, a.H, tokens, false)) != cudaSuccess ||
+            (err = tile_map(&maps.k, a.k, false, a.H, tokens, false)) != cudaSuccess ||
+            (err = tile_map(&maps.v, a.v, false, a.H, tokens, true)) != cudaSuccess ||
+            (err = tile_map(&maps.la, a.log_alpha, true, a.H, tokens, false)) != cudaSuccess)
+            return err;
     }
     profile_mark(SLOT_SETUP, true, stream);
     seg_setup_kernel<<<1, 1024, 0, stream>>>(a.cu, a.N, a.T, p.seg_chunks, p.max_units, a.segs,
@@ -866,7 +1003,7 @@ cudaError_t launch_tc(const TcArgs& a, const TcPlan& p, cudaStream_t stream, int
     const dim3 grid((unsigned)p.max_units, (unsigned)a.H);
     if (p.segmented) {
         profile_mark(SLOT_PASS1, true, stream);
-        tc_kernel<true><<<grid, NT, Lay::BYTES, stream>>>(a);
+        tc_kernel<true><<<grid, NT, LayT<true>::BYTES, stream>>>(a, maps);
         profile_mark(SLOT_PASS1, false, stream);
         *launches += 1;
         if ((err = cudaGetLastError()) != cudaSuccess) return err;
@@ -877,7 +1014,7 @@ cudaError_t launch_tc(const TcArgs& a, const TcPlan& p, cudaStream_t stream, int
         if ((err = cudaGetLastError()) != cudaSuccess) return err;
     }
     profile_mark(SLOT_PASS3, true, stream);
-    tc_kernel<false><<<grid, NT, Lay::BYTES, stream>>>(a);
+    tc_kernel<false><<<grid, NT, LayT<false>::BYTES, stream>>>(a, maps);
     profile_mark(SLOT_PASS3, false, stream);
     *launches += 1;
     return cudaGetLastError();
