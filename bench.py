@@ -60,6 +60,23 @@ def workload_config(inp, n_gpus):
             "parallelism": f"dp{n_gpus} (independent problem per GPU)"}
 
 
+# ------------------------------------------------------------------ multi-rank helpers
+def max_over_ranks(ms: float, dist_mod=None, device=None) -> float:
+    """Slowest rank's time (every rank calls this at the same point)."""
+    if dist_mod is None or not dist_mod.is_initialized() or dist_mod.get_world_size() == 1:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist_mod.all_reduce(t, op=dist_mod.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, tokens_per_rank: int, ms: float) -> float:
+    """Whole-job Mtokens/s: every rank processes its own problem of tokens_per_rank
+    tokens; the job takes as long as its slowest rank."""
+    return world * tokens_per_rank / (ms * 1e-3) / 1e6
+
+
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
     """nvidia-smi samples (every 100 ms) of one GPU while the timed region runs."""
@@ -340,13 +357,9 @@ def main():
     if pg:
         pg.barrier()
     torch.cuda.synchronize()
-    ms = ev0.elapsed_time(ev1) / args.steps
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, pg, dev)
     clocks = clk.summary()
-    if pg:
-        t = torch.tensor([ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms = float(t.item())
-    value = world * tokens / (ms * 1e-3) / 1e6
+    value = job_throughput(world, tokens, ms)
 
     # e2e: host buffers through kda_fwd_host, copies inside every step
     nbytes = lambda t: 0 if t is None else t.numel() * t.element_size()
@@ -369,14 +382,10 @@ def main():
             e2e_step()
         e1.record(stream)
         stream.synchronize()
-        e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
-        if pg:
-            t = torch.tensor([e2e_ms], device=dev)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, pg, dev)
         h2d = sum(nbytes(t) for t in host.values()) + (0 if cu_arg is None else cu_arg.nbytes)
         d2h = nbytes(out_h) + nbytes(fs_h)
-        e2e = {"value": world * tokens / (e2e_ms * 1e-3) / 1e6, "unit": UNIT,
+        e2e = {"value": job_throughput(world, tokens, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                "steps": args.e2e_steps}
 
