@@ -55,7 +55,7 @@ using namespace tc;
 
 constexpr int C = 64;     // tokens per chunk
 constexpr int D = 128;    // d_k = d_v
-constexpr int NT = 256;   // threads per CTA
+constexpr int NT = 512;   // threads per CTA: 16 warps, 4 per TMEM lane quadrant
 constexpr float LOG2E = 1.4426950408889634f;
 
 enum : int { ERR_WAIT_TIMEOUT = 1, ERR_SEG_OVERFLOW = 2 };
@@ -80,7 +80,6 @@ struct LayT {
     static constexpr uint32_t SA = 32768, WB = 0, UA = 16384, MA = 69632;
     static constexpr uint32_t R1 = SEG ? 102400 : 69632;
     static constexpr uint32_t QT = R1;                            // pass 3: 64 x 128, K-major
-    static constexpr uint32_t OS = QT;                            // output staging (QT is dead)
     static constexpr uint32_t KD = SEG ? R1 : QT + 16384;         // 64 x 128, MN-major
     static constexpr uint32_t UMA = KD + 16384;                   // pass 1: 128 x 64, K-major
     static constexpr uint32_t PB = KD + 16384;                    // pass 3: 64 x 64, K-major
@@ -89,11 +88,12 @@ struct LayT {
     static constexpr uint32_t RQ = RAW + 49152;                   // pass 3 only
     static constexpr uint32_t RV = RAW + (SEG ? 49152 : 65536);   // two 16 KB buffers
     static constexpr uint32_t RAW_TX = SEG ? 65536 : 81920;       // TMA bytes per chunk
-    static constexpr uint32_t GSUM = RV + 32768;                  // fp32 [8][128]
-    static constexpr uint32_t GAM = GSUM + 4096;                  // fp32 [128] e^{g_last}
+    static constexpr uint32_t GSUM = RV + 32768;                  // fp32 [16][128]
+    static constexpr uint32_t GAM = GSUM + 8192;                  // fp32 [128] e^{g_last}
     static constexpr uint32_t EHA = GAM + 512;                    // fp32 [128] e^{rho_a}
     static constexpr uint32_t EHB = EHA + 512;                    // fp32 [128] e^{rho_b}
-    static constexpr uint32_t BETA = EHB + 512;                   // fp32 [64]
+    static constexpr uint32_t FAC = EHB + 512;                    // fp32 [5][128] gate factors
+    static constexpr uint32_t BETA = FAC + 2560;                  // fp32 [64]
     static constexpr uint32_t BAR = BETA + 256;                   // 2 mbarriers: MMA, TMA
     static constexpr uint32_t TMEMP = BAR + 16;                   // TMEM base address
     static constexpr uint32_t END = TMEMP + 16;
@@ -107,8 +107,8 @@ static_assert(LayT<true>::MA + 32768 <= LayT<true>::R1, "MA overflow");
 static_assert(LayT<false>::BYTES <= 232448 && LayT<true>::BYTES <= 232448, "shared memory");
 
 // TMEM columns (512 allocated).  Pass 3: AP [0,96) W [96,160) U [160,224)
-// O [224,288) S [384,512).  Pass 1: AP/U_M [0,96) W U as above, B [256,384), M [384,512).
-constexpr uint32_t TM_AP = 0, TM_W = 96, TM_U = 160, TM_O = 224;
+// O [224,288) and [288,352) for alternate chunks, S [384,512).  Pass 1: AP/U_M [0,96) W U as above, B [256,384), M [384,512).
+constexpr uint32_t TM_AP = 0, TM_W = 96, TM_U = 160, TM_O = 224;  // pass 3: O at 224 or 288
 constexpr uint32_t TM_B = 256, TM_S = 384, TM_M = 384;
 
 __device__ __forceinline__ float clamp_gate(float x) { return fminf(fmaxf(x, -5.f), 0.f); }
@@ -285,9 +285,9 @@ __device__ void invert_unit_lower(const float* As, float* Ts, float* Ys, int tid
         warp_store16x8(Ts + ro * TS_LD + co + 8 * nt, TS_LD, d, -1.f, lane);
     }
     __syncthreads();
-    // 3. all 8 warps: output tile (16-row mt, 8-column nt) of the 32 x 32 block
-    const int mt = warp >> 2, nt = warp & 3;
-    {
+    // 3. warps 0-7: output tile (16-row mt, 8-column nt) of the 32 x 32 block
+    const int mt = (warp >> 2) & 1, nt = warp & 3;
+    if (warp < 8) {
         float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int k0 = 0; k0 < 32; k0 += 8)
@@ -296,7 +296,7 @@ __device__ void invert_unit_lower(const float* As, float* Ts, float* Ys, int tid
         warp_store16x8(Ys + 16 * mt * YS_LD + 8 * nt, YS_LD, d, 1.f, lane);
     }
     __syncthreads();
-    {
+    if (warp < 8) {
         float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int k0 = 0; k0 < 32; k0 += 8)
@@ -343,19 +343,18 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
     tc_fence_after();
     const uint32_t tmem = *tmem_ptr;
     const int quad = warp & 3;                       // TMEM lane quadrant of this warp
+    const int wg = warp >> 2;                        // column slice within the quadrant (0-3)
     const int lrow = quad * 32 + lane;               // TMEM lane / tile row owned by this thread
     const uint32_t tq = tmem + ((uint32_t)(quad * 32) << 16);
     uint32_t parity = 0;
 
-    // ---- initial state
-    if (warp >= 4) {
-        const int e = lrow;
-        for (int c0 = 0; c0 < D; c0 += 16) {
+    // ---- initial state (pass 3: each column slice wg writes 32 columns of S^T;
+    // pass 1: wg 0-1 write B = 0, wg 2-3 write M = I, 64 columns each)
+    if (!SEG) {
+        const int e = lrow, cb = 32 * wg;
+        for (int c0 = cb; c0 < cb + 32; c0 += 16) {
             float v[16];
-            if (SEG) {
-#pragma unroll
-                for (int i = 0; i < 16; ++i) v[i] = 0.f;  // B = 0
-            } else if (sg.j == 0 && sg.last) {  // single segment: read the caller's state
+            if (sg.j == 0 && sg.last) {  // single segment: read the caller's state
                 const float* s0 = a.s0 ? a.s0 + ((int64_t)sg.n * H + h) * D * D : nullptr;
 #pragma unroll
                 for (int i = 0; i < 16; ++i) v[i] = s0 ? s0[(int64_t)(c0 + i) * D + e] : 0.f;
@@ -364,15 +363,16 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
 #pragma unroll
                 for (int i = 0; i < 16; ++i) v[i] = sin[c0 + i];
             }
-            tmem_st16(tq + (SEG ? TM_B : TM_S) + c0, v);
+            tmem_st16(tq + TM_S + c0, v);
         }
-    } else if (SEG) {
-        const int i0 = lrow;  // M = I
-        for (int c0 = 0; c0 < D; c0 += 16) {
+    } else {
+        const int cb = 64 * (wg & 1);
+        const bool is_m = wg >= 2;
+        for (int c0 = cb; c0 < cb + 64; c0 += 16) {
             float v[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] = (c0 + i == i0) ? 1.f : 0.f;
-            tmem_st16(tq + TM_M + c0, v);
+            for (int i = 0; i < 16; ++i) v[i] = (is_m && c0 + i == lrow) ? 1.f : 0.f;
+            tmem_st16(tq + (is_m ? TM_M : TM_B) + c0, v);
         }
     }
     tmem_st_wait();
@@ -399,22 +399,37 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
         if (tid < C && sg.t_begin + tid < sg.t_end) beta_ld = __ldg(a.beta + (sg.t_begin + tid) * H + h);
     }
 
+    // O^T of a finished chunk sits in TMEM (two buffers, alternating by chunk);
+    // each thread stores its channel e for 16 tokens straight to global memory.
+    int64_t prev_t0 = -1;
+    int prev_L = 0;
+    auto store_out = [&](int buf) {
+        const int r0 = 16 * wg;
+        float v[16];
+        tmem_ld16(tq + TM_O + 64 * buf + r0, v);
+        tmem_wait16(v);
+        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out) + (int64_t)h * D + lrow;
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            if (r0 + i < prev_L) out[(prev_t0 + r0 + i) * H * (int64_t)D] = __float2bfloat16_rn(v[i]);
+    };
+
     bool ok = true;
-    int vbuf = 0;  // RV buffer of the current chunk
+    int vbuf = 0;  // RV buffer and O buffer of the current chunk
     for (int64_t t0 = sg.t_begin; t0 < sg.t_end && ok; t0 += C, vbuf ^= 1) {
         const int Lc = (int)((sg.t_end - t0) < C ? (sg.t_end - t0) : C);
 
         // ============ phase 0: gates, scaled operands
         {
-            const int c4 = lane, tg = warp, c0 = 4 * c4;
-            float4 la[8];
-            uint2 kr[8], qr[8];
+            const int c4 = lane, tg = warp, c0 = 4 * c4;  // tokens 4tg..4tg+3, channels c0..c0+3
+            float4 la[4];
+            uint2 kr[4], qr[4];
             if (!(ok = !__syncthreads_or(!mbar_wait(bar_raw, raw_parity, &g_tc_status,
                                                     ERR_WAIT_TIMEOUT)))) break;
             raw_parity ^= 1u;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {  // rows past the segment end act as identity steps
-                const int r = 8 * tg + i;
+            for (int i = 0; i < 4; ++i) {  // rows past the segment end act as identity steps
+                const int r = 4 * tg + i;
                 la[i] = make_float4(0.f, 0.f, 0.f, 0.f);
                 kr[i] = qr[i] = make_uint2(0u, 0u);
                 if (r < Lc) {
@@ -426,10 +441,10 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
                         make_uint2(0u, 0u);
                 }
             }
-            float g[8][4];
+            float g[4][4];
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
+            for (int i = 0; i < 4; ++i) {
                 acc[0] += clamp_gate(la[i].x);
                 acc[1] += clamp_gate(la[i].y);
                 acc[2] += clamp_gate(la[i].z);
@@ -445,50 +460,53 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
                 if (tid == 0) issue_raw(t0 + C, vbuf ^ 1);
                 beta_ld = (tid < C && t0 + C + tid < sg.t_end) ? __ldg(a.beta + (t0 + C + tid) * H + h) : 0.f;
             }
-            float off[4] = {0.f, 0.f, 0.f, 0.f}, run[4] = {0.f, 0.f, 0.f, 0.f};
-            float ra[4], rb[4], gl[4];
+            // one thread per channel: exclusive prefix of the 16 token groups (in place),
+            // references rho_a = g_15, rho_b = g_47, g_last = g_63 and the factors
+            //   FAC[0] rho_a, FAC[1] rho_b (log2 units), FAC[2] e^{g_last - rho_a},
+            //   FAC[3] e^{g_last - rho_b}, FAC[4] e^{rho_b - rho_a}
+            float* fac = reinterpret_cast<float*>(sm + Lay::FAC);
+            if (tid < D) {
+                const int c = tid;
+                float run = 0.f, ra = 0.f, rb = 0.f;
 #pragma unroll
-            for (int t2 = 0; t2 < 8; ++t2) {
-                const float4 s = *reinterpret_cast<const float4*>(gsum + t2 * D + c0);
-                const float sv[4] = {s.x, s.y, s.z, s.w};
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    if (t2 < tg) off[c] += sv[c];
-                    run[c] += sv[c];
-                    if (t2 == 1) ra[c] = run[c];
-                    if (t2 == 5) rb[c] = run[c];
-                    if (t2 == 7) gl[c] = run[c];
+                for (int t2 = 0; t2 < 16; ++t2) {
+                    const float x = gsum[t2 * D + c];
+                    gsum[t2 * D + c] = run;
+                    run += x;
+                    if (t2 == 3) ra = run;
+                    if (t2 == 11) rb = run;
                 }
+                fac[c] = ra * LOG2E;
+                fac[D + c] = rb * LOG2E;
+                fac[2 * D + c] = ex2((run - ra) * LOG2E);
+                fac[3 * D + c] = ex2((run - rb) * LOG2E);
+                fac[4 * D + c] = ex2((rb - ra) * LOG2E);
+                gam[c] = ex2(run * LOG2E);
+                eha[c] = ex2(ra * LOG2E);
+                ehb[c] = ex2(rb * LOG2E);
             }
-            // per-channel factors (log2 domain): E_h = e^{rho_h}, Dh = e^{g_last - rho_h},
-            // fba = e^{rho_b - rho_a}
-            float Eh[4], Dh[4], fba[4], rho[4];
-            const bool hb = tg >= 4;  // tokens 8tg.. lie in the second half
+            __syncthreads();
+            const bool hb = tg >= 8;  // tokens 4tg.. lie in the second half
+            const float4 off4 = *reinterpret_cast<const float4*>(gsum + tg * D + c0);
+            const float4 rho4 = *reinterpret_cast<const float4*>(fac + (hb ? D : 0) + c0);
+            const float4 eh4 = *reinterpret_cast<const float4*>((hb ? ehb : eha) + c0);
+            const float4 dh4 = *reinterpret_cast<const float4*>(fac + (hb ? 3 : 2) * D + c0);
+            const float4 fba4 = *reinterpret_cast<const float4*>(fac + 4 * D + c0);
+            const float off[4] = {off4.x, off4.y, off4.z, off4.w};
+            const float rho2[4] = {rho4.x, rho4.y, rho4.z, rho4.w};  // log2 units
+            const float Eh[4] = {eh4.x, eh4.y, eh4.z, eh4.w};
+            const float Dh[4] = {dh4.x, dh4.y, dh4.z, dh4.w};
+            const float fba[4] = {fba4.x, fba4.y, fba4.z, fba4.w};
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                rho[c] = hb ? rb[c] : ra[c];
-                Eh[c] = ex2(rho[c] * LOG2E);
-                Dh[c] = ex2((gl[c] - rho[c]) * LOG2E);
-                fba[c] = ex2((rb[c] - ra[c]) * LOG2E);
-            }
-            if (tg == 0) {
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    gam[c0 + c] = ex2(gl[c] * LOG2E);
-                    eha[c0 + c] = ex2(ra[c] * LOG2E);
-                    ehb[c0 + c] = ex2(rb[c] * LOG2E);
-                }
-            }
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int r = 8 * tg + i;
+            for (int i = 0; i < 4; ++i) {
+                const int r = 4 * tg + i;
                 float kf[4], qf[4];
                 unpack_bf16x4(kr[i], kf);
                 unpack_bf16x4(qr[i], qf);
                 float e1[4], e2[4];
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    const float d2 = (g[i][c] + off[c] - rho[c]) * LOG2E;
+                    const float d2 = fmaf(g[i][c] + off[c], LOG2E, -rho2[c]);
                     e1[c] = ex2(d2);
                     e2[c] = ex2(-d2);
                 }
@@ -523,6 +541,7 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
                 mma_bf16(tmem + TM_AP, kmajor_desc(x1, 128, s), kmajor_desc(bt, 96, s), id, s > 0);
             mma_commit(bar);
         }
+        if (!SEG && prev_t0 >= 0) store_out(vbuf ^ 1);  // previous chunk's output, meanwhile
         if (!(ok = wait_mma(bar, parity))) break;
 
         // ============ phase 2: masks, beta, (I + A)^-1, P
@@ -530,46 +549,50 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
             float* As = reinterpret_cast<float*>(sm + Lay::AS);
             float* Ts = reinterpret_cast<float*>(sm + Lay::TS);
             float* Ys = reinterpret_cast<float*>(sm + Lay::YS);
-            if (warp < 4 && (!SEG || warp < 2)) {
-                float v[96];
-#pragma unroll
-                for (int q = 0; q < 6; ++q) tmem_ld16(tq + TM_AP + 16 * q, *reinterpret_cast<float(*)[16]>(v + 16 * q));
-#pragma unroll
-                for (int q = 0; q < 6; ++q) tmem_wait16(*reinterpret_cast<float(*)[16]>(v + 16 * q));
+            // rows r of A (lanes 0-63) and P (lanes 64-127); warp slice wg handles the 16
+            // columns j in [16wg, 16wg+16).  Columns j < 32 of rows r >= 32 come from the
+            // cross-half product (TMEM columns 64 + j).
+            if (!SEG || quad < 2) {
                 const int r = lrow & 63;
-                const bool isP = lrow >= 64;
-                const float br = beta_s[r];
-                float x[64];
+                const bool isP = quad >= 2;
+                const bool lower_half = r < 32;  // warp-uniform
+                const int j0 = 16 * wg;
+                float x[16];
+                if (j0 >= 32 && lower_half) {
 #pragma unroll
-                for (int j = 0; j < 64; ++j) {
-                    float val;
-                    if (j < 32)
-                        val = r < 32 ? v[j] : v[64 + j];
-                    else
-                        val = r >= 32 ? v[j] : 0.f;
-                    x[j] = isP ? (j <= r ? val : 0.f) : (j < r ? br * val : 0.f);
+                    for (int i = 0; i < 16; ++i) x[i] = 0.f;
+                } else {
+                    float v[16];
+                    tmem_ld16(tq + TM_AP + (j0 < 32 && !lower_half ? 64 + j0 : j0), v);
+                    tmem_wait16(v);
+                    const float br = beta_s[r];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int j = j0 + i;
+                        x[i] = isP ? (j <= r ? v[i] : 0.f) : (j < r ? br * v[i] : 0.f);
+                    }
                 }
                 if (!isP) {
 #pragma unroll
-                    for (int j = 0; j < 64; ++j) As[r * AS_LD + j] = x[j];
+                    for (int i = 0; i < 16; ++i) As[r * AS_LD + j0 + i] = x[i];
                 } else {
                     const uint32_t pb = smem_u32(sm + Lay::PB);
 #pragma unroll
-                    for (int j8 = 0; j8 < 8; ++j8)
-                        st_shared_v4(pb + kmajor_chunk_off(r, j8, 64), pack_bf16(x[8 * j8], x[8 * j8 + 1]),
-                                     pack_bf16(x[8 * j8 + 2], x[8 * j8 + 3]),
-                                     pack_bf16(x[8 * j8 + 4], x[8 * j8 + 5]),
-                                     pack_bf16(x[8 * j8 + 6], x[8 * j8 + 7]));
+                    for (int hh = 0; hh < 2; ++hh)
+                        st_shared_v4(pb + kmajor_chunk_off(r, 2 * wg + hh, 64),
+                                     pack_bf16(x[8 * hh], x[8 * hh + 1]),
+                                     pack_bf16(x[8 * hh + 2], x[8 * hh + 3]),
+                                     pack_bf16(x[8 * hh + 4], x[8 * hh + 5]),
+                                     pack_bf16(x[8 * hh + 6], x[8 * hh + 7]));
                 }
             }
             __syncthreads();
             invert_unit_lower(As, Ts, Ys, tid);
-            {  // T -> bf16 K-major [r][j]
+            {  // T diag(beta) -> bf16 K-major [r][j]: one 8-column chunk per thread
                 const uint32_t tb = smem_u32(sm + Lay::TB);
-                const int r = tid >> 2;
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const int j8 = 2 * (tid & 3) + hh;
+                const int r = tid >> 3;
+                {
+                    const int j8 = tid & 7;
                     const float* t = Ts + r * TS_LD + 8 * j8;
                     const float* bj = beta_s + 8 * j8;
                     st_shared_v4(tb + kmajor_chunk_off(r, j8, 64), pack_bf16(t[0] * bj[0], t[1] * bj[1]),
@@ -607,46 +630,39 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
             mma_commit(bar);
         }
         // meanwhile: bf16 copy of the state into SA (and MA), state scaled by gamma in
-        // TMEM.  Pass 3: warps 4-7 take columns 0-63, warps 0-3 columns 64-127 of the
-        // same lanes.  Pass 1: warps 4-7 take B, warps 0-3 take M.
+        // TMEM.  Pass 3: slice wg takes columns 32wg..32wg+31.  Pass 1: slices 0-1 take
+        // B, slices 2-3 take M, 64 columns each.
         if (!SEG) {
-            const int c0 = warp >= 4 ? 0 : 64;
-            stage_cols<4>(tq + TM_S + c0, sm + Lay::SA, 128, lrow, c0, gam, true);
+            const int c0 = 32 * wg;
+            stage_cols<2>(tq + TM_S + c0, sm + Lay::SA, 128, lrow, c0, gam, true);
         } else {
-            const uint32_t col = warp >= 4 ? TM_B : TM_M;
-            uint8_t* tile = sm + (warp >= 4 ? Lay::SA : Lay::MA);
-            stage_cols<4>(tq + col, tile, 128, lrow, 0, gam, true);
-            stage_cols<4>(tq + col + 64, tile, 128, lrow, 64, gam, true);
+            const bool is_m = wg >= 2;
+            const int c0 = 64 * (wg & 1);
+            stage_cols<4>(tq + (is_m ? TM_M : TM_B) + c0, sm + (is_m ? Lay::MA : Lay::SA), 128, lrow,
+                          c0, gam, true);
         }
         tmem_st_wait();
         if (!(ok = wait_mma(bar, parity))) break;
         // W^T = e^{rho_a} Wa^T + e^{rho_b} Wb^T (lane = channel c) -> WB (MN-major B
-        // operand: K rows = c, MN = token r); warps 0-3 tokens 0-31, warps 4-7 tokens 32-63
+        // operand: K rows = c, MN = token r)
         {
-            const int r0 = warp >= 4 ? 32 : 0;
-            float wa[2][16], wbv[2][16];
-            tmem_ld16(tq + TM_W + r0, wa[0]);
-            tmem_ld16(tq + TM_W + r0 + 16, wa[1]);
-            tmem_ld16(tq + TM_AP + r0, wbv[0]);
-            tmem_ld16(tq + TM_AP + r0 + 16, wbv[1]);
-            tmem_wait16(wa[0]);
-            tmem_wait16(wa[1]);
-            tmem_wait16(wbv[0]);
-            tmem_wait16(wbv[1]);
+            const int r0 = 16 * wg;  // tokens r0..r0+15 of this thread's channel row
+            float wa[16], wbv[16];
+            tmem_ld16(tq + TM_W + r0, wa);
+            tmem_ld16(tq + TM_AP + r0, wbv);
+            tmem_wait16(wa);
+            tmem_wait16(wbv);
             const float ea = eha[lrow], eb = ehb[lrow];
             const uint32_t wbs = smem_u32(sm + Lay::WB);
 #pragma unroll
-            for (int b = 0; b < 2; ++b)
+            for (int hh = 0; hh < 2; ++hh) {
+                float w[8];
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    float w[8];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        w[i] = fmaf(ea, wa[b][8 * hh + i], eb * wbv[b][8 * hh + i]);
-                    st_shared_v4(wbs + mnmajor_chunk_off(lrow, ((r0 + 16 * b) >> 3) + hh, 128),
-                                 pack_bf16(w[0], w[1]), pack_bf16(w[2], w[3]),
-                                 pack_bf16(w[4], w[5]), pack_bf16(w[6], w[7]));
-                }
+                for (int i = 0; i < 8; ++i) w[i] = fmaf(ea, wa[8 * hh + i], eb * wbv[8 * hh + i]);
+                st_shared_v4(wbs + mnmajor_chunk_off(lrow, (r0 >> 3) + hh, 128),
+                             pack_bf16(w[0], w[1]), pack_bf16(w[2], w[3]), pack_bf16(w[4], w[5]),
+                             pack_bf16(w[6], w[7]));
+            }
         }
         fence_async_smem();
         tc_fence_before();
@@ -665,7 +681,8 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
                 constexpr uint32_t id = idesc_bf16(128, 64, false, false);
 #pragma unroll
                 for (int s = 0; s < 8; ++s)
-                    mma_bf16(tmem + TM_O, kmajor_desc(sa, 128, s), kmajor_desc(qt, 64, s), id, s > 0);
+                    mma_bf16(tmem + TM_O + 64 * vbuf, kmajor_desc(sa, 128, s), kmajor_desc(qt, 64, s),
+                             id, s > 0);
             } else {
                 const uint32_t ma = smem_u32(sm + Lay::MA);
 #pragma unroll
@@ -679,12 +696,13 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
 
         // ============ phase 6: U^T -> UA (bf16, K-major, 128 x 64); pass 1 also U_M^T -> UMA
         if (!SEG) {
-            const int c0 = warp >= 4 ? 32 : 0;
-            stage_cols<2>(tq + TM_U + c0, sm + Lay::UA, 128, lrow, c0, nullptr, false);
-        } else if (warp < 4) {
-            stage_cols<4>(tq + TM_U, sm + Lay::UA, 128, lrow, 0, nullptr, false);
+            const int c0 = 16 * wg;
+            stage_cols<1>(tq + TM_U + c0, sm + Lay::UA, 128, lrow, c0, nullptr, false);
         } else {
-            stage_cols<4>(tq + TM_AP, sm + Lay::UMA, 128, lrow, 0, nullptr, false);
+            const bool is_m = wg >= 2;
+            const int c0 = 32 * (wg & 1);
+            stage_cols<2>(tq + (is_m ? TM_AP : TM_U) + c0, sm + (is_m ? Lay::UMA : Lay::UA), 128,
+                          lrow, c0, nullptr, false);
         }
         fence_async_smem();
         tc_fence_before();
@@ -700,7 +718,8 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
                 constexpr uint32_t id = idesc_bf16(128, 64, false, false);
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
-                    mma_bf16(tmem + TM_O, kmajor_desc(ua, 128, s), kmajor_desc(pb, 64, s), id, 1);
+                    mma_bf16(tmem + TM_O + 64 * vbuf, kmajor_desc(ua, 128, s), kmajor_desc(pb, 64, s),
+                             id, 1);
             }
 #pragma unroll
             for (int s = 0; s < 4; ++s)
@@ -716,32 +735,9 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
         }
         if (!(ok = wait_mma(bar, parity))) break;
 
-        // ============ phase 8: O^T -> out (via shared memory, 16-byte global stores)
-        if (!SEG) {
-            __nv_bfloat16* os = reinterpret_cast<__nv_bfloat16*>(sm + Lay::OS);
-            {  // warps 0-3 rows r = 0-31, warps 4-7 rows 32-63 of this thread's column e
-                const int r0 = warp >= 4 ? 32 : 0;
-                float v[2][16];
-                tmem_ld16(tq + TM_O + r0, v[0]);
-                tmem_ld16(tq + TM_O + r0 + 16, v[1]);
-                tmem_wait16(v[0]);
-                tmem_wait16(v[1]);
-#pragma unroll
-                for (int b = 0; b < 2; ++b)
-#pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        os[(r0 + 16 * b + i) * D + lrow] = __float2bfloat16_rn(v[b][i]);
-            }
-            tc_fence_before();
-            __syncthreads();
-            __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
-#pragma unroll
-            for (int x = 0; x < 4; ++x) {
-                const int idx = tid + NT * x, r = idx >> 4, cc = idx & 15;
-                if (r < Lc)
-                    *reinterpret_cast<uint4*>(out + ((t0 + r) * H + h) * (int64_t)D + 8 * cc) =
-                        *reinterpret_cast<const uint4*>(os + r * D + 8 * cc);
-            }
+        if (!SEG) {  // this chunk's output is stored during the next chunk's first product
+            prev_t0 = t0;
+            prev_L = Lc;
         }
         tc_fence_before();
         __syncthreads();
@@ -749,22 +745,24 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
     }
 
     // ---- results of the segment
+    if (ok && !SEG && prev_t0 >= 0) store_out(vbuf ^ 1);
     if (ok) {
-        if (SEG) {
-            float* dst = a.trans + ((int64_t)u * H + h) * 2 * D * D;
-            const uint32_t col = warp >= 4 ? TM_B : TM_M;
-            float* rowp = dst + (warp >= 4 ? 0 : D * D) + (int64_t)lrow * D;
-            for (int c0 = 0; c0 < D; c0 += 16) {
+        if (SEG) {  // slices 0-1: B^T, slices 2-3: M^T, 64 columns each
+            const bool is_m = wg >= 2;
+            const int cb = 64 * (wg & 1);
+            float* rowp = a.trans + ((int64_t)u * H + h) * 2 * D * D + (is_m ? D * D : 0) +
+                          (int64_t)lrow * D;
+            for (int c0 = cb; c0 < cb + 64; c0 += 16) {
                 float v[16];
-                tmem_ld16(tq + col + c0, v);
+                tmem_ld16(tq + (is_m ? TM_M : TM_B) + c0, v);
                 tmem_wait16(v);
 #pragma unroll
                 for (int i = 0; i < 16; i += 4)
                     *reinterpret_cast<float4*>(rowp + c0 + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
             }
-        } else if (sg.last && a.s_final && warp >= 4) {
+        } else if (sg.last && a.s_final) {  // slice wg: columns 32wg..32wg+31 of S^T
             float* sf = a.s_final + ((int64_t)sg.n * H + h) * D * D;
-            for (int c0 = 0; c0 < D; c0 += 16) {
+            for (int c0 = 32 * wg; c0 < 32 * wg + 32; c0 += 16) {
                 float v[16];
                 tmem_ld16(tq + TM_S + c0, v);
                 tmem_wait16(v);
