@@ -63,10 +63,10 @@ struct TcArgs {
     float* sin;         // [max_units, H, 128, 128]: S_in^T of each segment
 };
 
-// TMA descriptors of the q, k, v (bf16) and log_alpha (fp32) tensors, viewed
-// as [T, H, 128] with a (128, 1, 64) tile box; passed as a grid constant.
+// TMA descriptors of the q, k, v, out (bf16) and log_alpha (fp32) tensors,
+// viewed as [T, H, 128]; passed as a grid constant.
 struct TcMaps {
-    CUtensorMap q, k, v, la;
+    CUtensorMap q, k, v, la, out;
 };
 
 struct TcPlan {

@@ -107,8 +107,9 @@ static_assert(LayT<true>::MA + 32768 <= LayT<true>::R1, "MA overflow");
 static_assert(LayT<false>::BYTES <= 232448 && LayT<true>::BYTES <= 232448, "shared memory");
 
 // TMEM columns (512 allocated).  Pass 3: AP [0,96) W [96,160) U [160,224)
-// O [224,288) and [288,352) for alternate chunks, S [384,512).  Pass 1: AP/U_M [0,96) W U as above, B [256,384), M [384,512).
-constexpr uint32_t TM_AP = 0, TM_W = 96, TM_U = 160, TM_O = 224;  // pass 3: O at 224 or 288
+// O [224,288) bf16 S^T [288,352) bf16 U^T [352,384) S [384,512).  Pass 1: AP/U_M [0,96) W U as above, B [256,384), M [384,512).
+constexpr uint32_t TM_AP = 0, TM_W = 96, TM_U = 160, TM_O = 224;
+constexpr uint32_t TM_SB = 288, TM_UB = 352;  // pass 3: bf16 copies of S^T and U^T (A operands)
 constexpr uint32_t TM_B = 256, TM_S = 384, TM_M = 384;
 
 __device__ __forceinline__ float clamp_gate(float x) { return fminf(fmaxf(x, -5.f), 0.f); }
@@ -180,6 +181,34 @@ __device__ __forceinline__ void stage_cols(uint32_t tm, uint8_t* tile, int R, in
     }
 }
 
+// Copy 16 x NB fp32 TMEM columns at tm (tile columns col0..) of this thread's
+// lane into NB x 8 packed-bf16 columns at tb (for an A operand read from TMEM);
+// optionally scale the fp32 copy by gam[col0 + i] in place.
+template <int NB>
+__device__ __forceinline__ void stage_cols_tmem(uint32_t tm, uint32_t tb, int col0, const float* gam,
+                                                bool scale_back) {
+    float v[NB][16];
+#pragma unroll
+    for (int b = 0; b < NB; ++b) tmem_ld16(tm + 16 * b, v[b]);
+#pragma unroll
+    for (int b = 0; b < NB; ++b) tmem_wait16(v[b]);
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+        uint32_t u[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) u[i] = pack_bf16(v[b][2 * i], v[b][2 * i + 1]);
+        tmem_st8(tb + 8 * b, u);
+    }
+    if (scale_back) {
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[b][i] *= gam[col0 + 16 * b + i];
+            tmem_st16(tm + 16 * b, v[b]);
+        }
+    }
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void mbar_expect_tx(void* bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
@@ -195,6 +224,26 @@ __device__ __forceinline__ void tma_tile(void* dst, const CUtensorMap* map, int 
         " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(h), "r"(t0), "r"(smem_u32(bar))
         : "memory");
+}
+
+// shared [64 tokens][128 channels] tile -> global tile at (0, h, t0) of a [T, H, 128] tensor
+__device__ __forceinline__ void tma_store_tile(const CUtensorMap* map, const void* src, int h, int t0) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(0), "r"(h), "r"(t0), "r"(smem_u32(src))
+        : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// the issuing thread's bulk stores have finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// ... and have completed
+__device__ __forceinline__ void bulk_wait_all() {
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 // ---------------------------------------------------------------- (I + A)^-1
@@ -232,60 +281,91 @@ __device__ __forceinline__ void warp_store16x8(float* dst, int ld, const float (
     dst[(g + 8) * ld + 2 * t + 1] = sgn * d[3];
 }
 
-// As: strictly lower 64 x 64 (fp32, stride AS_LD).  Writes T = (I + A)^-1 into Ts
-// (fp32, stride TS_LD, zeros above the diagonal):
-//  1. the four 16 x 16 diagonal blocks by substitution (one thread per column,
-//     eliminating one known entry at a time so the dependency chain is 16 long);
-//  2. T_10 = -T_11 (A_10 T_00) and T_32 = -T_33 (A_32 T_22), completing the two
-//     32 x 32 diagonal inverses T_lo, T_hi;
-//  3. T[32:64, 0:32] = -T_hi (A[32:64, 0:32] T_lo).
-// The block products of steps 2 and 3 run as tf32 warp MMAs with fp32
-// accumulation (T then enters the chunk products as bf16).
-__device__ void invert_unit_lower(const float* As, float* Ts, float* Ys, int tid) {
+// As: strictly lower 64 x 64 (fp32, stride AS_LD).  Writes TB = T diag(beta) as
+// the bf16 K-major [r][j] tile tbp, where T = (I + A)^-1, using Ts (fp32, stride
+// TS_LD) and Ys as scratch:
+//  1. warp h (h = 0, 1) alone builds the 32 x 32 diagonal half h of T: its two
+//     16 x 16 diagonal blocks by substitution (one lane per column, eliminating one
+//     known entry at a time), then T_21 = -T_22 (A_21 T_11) inside the half with
+//     tf32 warp MMAs -- warp-level synchronisation only;  the other warps zero the
+//     upper-right 32 x 32 block of TB;
+//  2. Z = A[32:64, 0:32] T_lo (8 warps, one 16 x 8 tile each);
+//  3. T[32:64, 0:32] = -T_hi Z, written straight into TB.
+// The block products are tf32 warp MMAs with fp32 accumulation (T then enters
+// the chunk products as bf16).
+__device__ void invert_to_tb(const float* As, float* Ts, float* Ys, const float* beta,
+                             uint32_t tbp, int tid) {
     const int warp = tid >> 5, lane = tid & 31;
-    if (tid < 64) {
-        const int b = tid >> 4, j = tid & 15, o = 16 * b;
-        float t[16];
+    const int g = lane >> 2, t4 = lane & 3;
+    if (warp < 2) {
+        const int o = 32 * warp;
+        {  // 1a. diagonal blocks o (lanes 0-15) and o+16 (lanes 16-31): lane i holds
+           // row i of its block; T_i = e_i - sum_{m<i} A_im T_m, rows finished in order
+           // and broadcast to the 16 lanes of the block by shuffles
+            const int i = lane & 15, ob = o + 16 * (lane >> 4), src0 = lane & 16;
+            float arow[16], trow[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) t[i] = (i == j) ? 1.f : 0.f;
+            for (int m = 0; m < 16; ++m) {
+                arow[m] = m < i ? As[(ob + i) * AS_LD + ob + m] : 0.f;
+                trow[m] = m == i ? 1.f : 0.f;
+            }
 #pragma unroll
-        for (int m = 0; m < 15; ++m)
+            for (int m = 0; m < 15; ++m) {
+                const float am = arow[m];
 #pragma unroll
-            for (int i = m + 1; i < 16; ++i) t[i] = fmaf(-As[(o + i) * AS_LD + o + m], t[m], t[i]);
+                for (int c = 0; c <= m; ++c) {  // row m has entries in columns 0..m only
+                    const float tmc = __shfl_sync(0xffffffffu, trow[c], src0 + m);
+                    trow[c] = fmaf(-am, tmc, trow[c]);
+                }
+            }
 #pragma unroll
-        for (int i = 0; i < 16; ++i) Ts[(o + i) * TS_LD + o + j] = t[i];
-    } else {
-        // zero everything above the diagonal blocks
-        for (int x = tid - 64; x < 6 * 256; x += NT - 64) {
-            const int p = x >> 8, e = x & 255;
-            const int I = p < 3 ? 0 : p < 5 ? 1 : 2;
-            const int J = p < 3 ? p + 1 : p < 5 ? p - 1 : 3;
-            Ts[(16 * I + (e >> 4)) * TS_LD + 16 * J + (e & 15)] = 0.f;
+            for (int c = 0; c < 16; ++c) Ts[(ob + i) * TS_LD + ob + c] = trow[c];
+            // zero the upper-right 16 x 16 block of this half (rows o..o+15, cols o+16..o+31)
+#pragma unroll
+            for (int x = 0; x < 8; ++x) {
+                const int e = lane + 32 * x;
+                Ts[(o + (e >> 4)) * TS_LD + o + 16 + (e & 15)] = 0.f;
+            }
         }
-    }
-    __syncthreads();
-    // 2. warps 0-3: (I = 1 or 3) x (8-column half nt)
-    if (warp < 4) {
-        const int I = warp < 2 ? 1 : 3, nt = warp & 1, ro = 16 * I, co = ro - 16;
-        float d[4] = {0.f, 0.f, 0.f, 0.f};
+        __syncwarp();
+        // 1b. Y = A_21 T_11 (16 x 16 x 16), then T_21 = -T_22 Y, within the half
+        float* Yh = Ys + warp * 16 * YS_LD;
 #pragma unroll
-        for (int k0 = 0; k0 < 16; k0 += 8)
-            warp_mma_tf32(d, As + ro * AS_LD + co + k0, AS_LD, Ts + (co + k0) * TS_LD + co + 8 * nt,
-                          TS_LD, lane);
-        warp_store16x8(Ys + (warp >> 1) * 16 * YS_LD + 8 * nt, YS_LD, d, 1.f, lane);
-    }
-    __syncthreads();
-    if (warp < 4) {
-        const int I = warp < 2 ? 1 : 3, nt = warp & 1, ro = 16 * I, co = ro - 16;
-        float d[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int nt = 0; nt < 2; ++nt) {
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int k0 = 0; k0 < 16; k0 += 8)
-            warp_mma_tf32(d, Ts + ro * TS_LD + ro + k0, TS_LD,
-                          Ys + (warp >> 1) * 16 * YS_LD + k0 * YS_LD + 8 * nt, YS_LD, lane);
-        warp_store16x8(Ts + ro * TS_LD + co + 8 * nt, TS_LD, d, -1.f, lane);
+            for (int k0 = 0; k0 < 16; k0 += 8)
+                warp_mma_tf32(d, As + (o + 16) * AS_LD + o + k0, AS_LD,
+                              Ts + (o + k0) * TS_LD + o + 8 * nt, TS_LD, lane);
+            warp_store16x8(Yh + 8 * nt, YS_LD, d, 1.f, lane);
+        }
+        __syncwarp();
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int k0 = 0; k0 < 16; k0 += 8)
+                warp_mma_tf32(d, Ts + (o + 16) * TS_LD + o + 16 + k0, TS_LD, Yh + k0 * YS_LD + 8 * nt,
+                              YS_LD, lane);
+            warp_store16x8(Ts + (o + 16) * TS_LD + o + 8 * nt, TS_LD, d, -1.f, lane);
+        }
+        __syncwarp();
+        // 1c. TB for the half: 32 rows x 4 chunks of 8 columns
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            const int id = lane + 32 * x, r = o + (id >> 2), j8 = (o >> 3) + (id & 3);
+            const float* tr = Ts + r * TS_LD + 8 * j8;
+            const float* bj = beta + 8 * j8;
+            st_shared_v4(tbp + kmajor_chunk_off(r, j8, 64), pack_bf16(tr[0] * bj[0], tr[1] * bj[1]),
+                         pack_bf16(tr[2] * bj[2], tr[3] * bj[3]), pack_bf16(tr[4] * bj[4], tr[5] * bj[5]),
+                         pack_bf16(tr[6] * bj[6], tr[7] * bj[7]));
+        }
+    } else if (warp < 6) {  // zero TB rows 0..31, columns 32..63: 128 chunks
+        const int id = tid - 64, r = id >> 2, j8 = 4 + (id & 3);
+        st_shared_v4(tbp + kmajor_chunk_off(r, j8, 64), 0u, 0u, 0u, 0u);
     }
     __syncthreads();
-    // 3. warps 0-7: output tile (16-row mt, 8-column nt) of the 32 x 32 block
+    // 2. Z = A[32:64, 0:32] T_lo: warp (mt, nt) for warps 0-7
     const int mt = (warp >> 2) & 1, nt = warp & 3;
     if (warp < 8) {
         float d[4] = {0.f, 0.f, 0.f, 0.f};
@@ -296,15 +376,20 @@ __device__ void invert_unit_lower(const float* As, float* Ts, float* Ys, int tid
         warp_store16x8(Ys + 16 * mt * YS_LD + 8 * nt, YS_LD, d, 1.f, lane);
     }
     __syncthreads();
+    // 3. T[32:64, 0:32] = -T_hi Z, scaled by beta_j, straight into TB
     if (warp < 8) {
         float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int k0 = 0; k0 < 32; k0 += 8)
             warp_mma_tf32(d, Ts + (32 + 16 * mt) * TS_LD + 32 + k0, TS_LD, Ys + k0 * YS_LD + 8 * nt,
                           YS_LD, lane);
-        warp_store16x8(Ts + (32 + 16 * mt) * TS_LD + 8 * nt, TS_LD, d, -1.f, lane);
+        const int r = 32 + 16 * mt + g, j = 8 * nt + 2 * t4;
+        const float b0 = beta[j], b1 = beta[j + 1];
+        asm volatile("st.shared.b32 [%0], %1;" ::"r"(tbp + kmajor_off(r, j, 64)),
+                     "r"(pack_bf16(-d[0] * b0, -d[1] * b1)));
+        asm volatile("st.shared.b32 [%0], %1;" ::"r"(tbp + kmajor_off(r + 8, j, 64)),
+                     "r"(pack_bf16(-d[2] * b0, -d[3] * b1)));
     }
-    __syncthreads();
 }
 
 // ---------------------------------------------------------------- the chunk loop
@@ -399,21 +484,6 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
         if (tid < C && sg.t_begin + tid < sg.t_end) beta_ld = __ldg(a.beta + (sg.t_begin + tid) * H + h);
     }
 
-    // O^T of a finished chunk sits in TMEM (two buffers, alternating by chunk);
-    // each thread stores its channel e for 16 tokens straight to global memory.
-    int64_t prev_t0 = -1;
-    int prev_L = 0;
-    auto store_out = [&](int buf) {
-        const int r0 = 16 * wg;
-        float v[16];
-        tmem_ld16(tq + TM_O + 64 * buf + r0, v);
-        tmem_wait16(v);
-        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out) + (int64_t)h * D + lrow;
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-            if (r0 + i < prev_L) out[(prev_t0 + r0 + i) * H * (int64_t)D] = __float2bfloat16_rn(v[i]);
-    };
-
     bool ok = true;
     int vbuf = 0;  // RV buffer and O buffer of the current chunk
     for (int64_t t0 = sg.t_begin; t0 < sg.t_end && ok; t0 += C, vbuf ^= 1) {
@@ -457,7 +527,10 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
             __syncthreads();
             // every thread holds its raw inputs: RAW may now receive the next chunk
             if (t0 + C < sg.t_end) {
-                if (tid == 0) issue_raw(t0 + C, vbuf ^ 1);
+                if (tid == 0) {
+                    if (!SEG) bulk_wait_read();  // the v buffer may still be feeding an output store
+                    issue_raw(t0 + C, vbuf ^ 1);
+                }
                 beta_ld = (tid < C && t0 + C + tid < sg.t_end) ? __ldg(a.beta + (t0 + C + tid) * H + h) : 0.f;
             }
             // one thread per channel: exclusive prefix of the 16 token groups (in place),
@@ -541,7 +614,6 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
                 mma_bf16(tmem + TM_AP, kmajor_desc(x1, 128, s), kmajor_desc(bt, 96, s), id, s > 0);
             mma_commit(bar);
         }
-        if (!SEG && prev_t0 >= 0) store_out(vbuf ^ 1);  // previous chunk's output, meanwhile
         if (!(ok = wait_mma(bar, parity))) break;
 
         // ============ phase 2: masks, beta, (I + A)^-1, P
@@ -587,20 +659,7 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
                 }
             }
             __syncthreads();
-            invert_unit_lower(As, Ts, Ys, tid);
-            {  // T diag(beta) -> bf16 K-major [r][j]: one 8-column chunk per thread
-                const uint32_t tb = smem_u32(sm + Lay::TB);
-                const int r = tid >> 3;
-                {
-                    const int j8 = tid & 7;
-                    const float* t = Ts + r * TS_LD + 8 * j8;
-                    const float* bj = beta_s + 8 * j8;
-                    st_shared_v4(tb + kmajor_chunk_off(r, j8, 64), pack_bf16(t[0] * bj[0], t[1] * bj[1]),
-                                 pack_bf16(t[2] * bj[2], t[3] * bj[3]),
-                                 pack_bf16(t[4] * bj[4], t[5] * bj[5]),
-                                 pack_bf16(t[6] * bj[6], t[7] * bj[7]));
-                }
-            }
+            invert_to_tb(As, Ts, Ys, beta_s, smem_u32(sm + Lay::TB), tid);
         }
         fence_async_smem();
         tc_fence_before();
@@ -634,14 +693,15 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
         // B, slices 2-3 take M, 64 columns each.
         if (!SEG) {
             const int c0 = 32 * wg;
-            stage_cols<2>(tq + TM_S + c0, sm + Lay::SA, 128, lrow, c0, gam, true);
+            stage_cols_tmem<2>(tq + TM_S + c0, tq + TM_SB + c0 / 2, c0, gam, true);
+            tmem_st_wait();
         } else {
             const bool is_m = wg >= 2;
             const int c0 = 64 * (wg & 1);
             stage_cols<4>(tq + (is_m ? TM_M : TM_B) + c0, sm + (is_m ? Lay::MA : Lay::SA), 128, lrow,
                           c0, gam, true);
+            tmem_st_wait();
         }
-        tmem_st_wait();
         if (!(ok = wait_mma(bar, parity))) break;
         // W^T = e^{rho_a} Wa^T + e^{rho_b} Wb^T (lane = channel c) -> WB (MN-major B
         // operand: K rows = c, MN = token r)
@@ -673,18 +733,20 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
             tc_fence_after();
             const uint32_t sa = smem_u32(sm + Lay::SA), wb = smem_u32(sm + Lay::WB);
             constexpr uint32_t id_neg = idesc_bf16(128, 64, false, true, true);
-#pragma unroll
-            for (int s = 0; s < 8; ++s)
-                mma_bf16(tmem + TM_U, kmajor_desc(sa, 128, s), mnmajor_desc(wb, 128, s), id_neg, 1);
-            if (!SEG) {
+            if (!SEG) {  // A = bf16 S^T from TMEM
                 const uint32_t qt = smem_u32(sm + Lay::QT);
                 constexpr uint32_t id = idesc_bf16(128, 64, false, false);
 #pragma unroll
                 for (int s = 0; s < 8; ++s)
-                    mma_bf16(tmem + TM_O + 64 * vbuf, kmajor_desc(sa, 128, s), kmajor_desc(qt, 64, s),
-                             id, s > 0);
+                    mma_bf16_ts(tmem + TM_U, tmem + TM_SB + 8 * s, mnmajor_desc(wb, 128, s), id_neg, 1);
+#pragma unroll
+                for (int s = 0; s < 8; ++s)
+                    mma_bf16_ts(tmem + TM_O, tmem + TM_SB + 8 * s, kmajor_desc(qt, 64, s), id, s > 0);
             } else {
                 const uint32_t ma = smem_u32(sm + Lay::MA);
+#pragma unroll
+                for (int s = 0; s < 8; ++s)
+                    mma_bf16(tmem + TM_U, kmajor_desc(sa, 128, s), mnmajor_desc(wb, 128, s), id_neg, 1);
 #pragma unroll
                 for (int s = 0; s < 8; ++s)
                     mma_bf16(tmem + TM_AP, kmajor_desc(ma, 128, s), mnmajor_desc(wb, 128, s), id_neg,
@@ -697,7 +759,8 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
         // ============ phase 6: U^T -> UA (bf16, K-major, 128 x 64); pass 1 also U_M^T -> UMA
         if (!SEG) {
             const int c0 = 16 * wg;
-            stage_cols<1>(tq + TM_U + c0, sm + Lay::UA, 128, lrow, c0, nullptr, false);
+            stage_cols_tmem<1>(tq + TM_U + c0, tq + TM_UB + c0 / 2, c0, nullptr, false);
+            tmem_st_wait();
         } else {
             const bool is_m = wg >= 2;
             const int c0 = 32 * (wg & 1);
@@ -713,20 +776,20 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
             tc_fence_after();
             const uint32_t ua = smem_u32(sm + Lay::UA), kd = smem_u32(sm + Lay::KD);
             constexpr uint32_t id_s = idesc_bf16(128, 128, false, true);
-            if (!SEG) {
+            if (!SEG) {  // A = bf16 U^T from TMEM
                 const uint32_t pb = smem_u32(sm + Lay::PB);
                 constexpr uint32_t id = idesc_bf16(128, 64, false, false);
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
-                    mma_bf16(tmem + TM_O + 64 * vbuf, kmajor_desc(ua, 128, s), kmajor_desc(pb, 64, s),
-                             id, 1);
-            }
+                    mma_bf16_ts(tmem + TM_O, tmem + TM_UB + 8 * s, kmajor_desc(pb, 64, s), id, 1);
 #pragma unroll
-            for (int s = 0; s < 4; ++s)
-                mma_bf16(tmem + (SEG ? TM_B : TM_S), kmajor_desc(ua, 128, s), mnmajor_desc(kd, 64, s),
-                         id_s, 1);
-            if (SEG) {
+                for (int s = 0; s < 4; ++s)
+                    mma_bf16_ts(tmem + TM_S, tmem + TM_UB + 8 * s, mnmajor_desc(kd, 64, s), id_s, 1);
+            } else {
                 const uint32_t uma = smem_u32(sm + Lay::UMA);
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_bf16(tmem + TM_B, kmajor_desc(ua, 128, s), mnmajor_desc(kd, 64, s), id_s, 1);
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
                     mma_bf16(tmem + TM_M, kmajor_desc(uma, 128, s), mnmajor_desc(kd, 64, s), id_s, 1);
@@ -735,9 +798,30 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
         }
         if (!(ok = wait_mma(bar, parity))) break;
 
-        if (!SEG) {  // this chunk's output is stored during the next chunk's first product
-            prev_t0 = t0;
-            prev_L = Lc;
+        if (!SEG) {
+            // O^T -> out.  A full chunk is staged as a [64][128] bf16 tile in this chunk's
+            // v buffer (dead since phase 3) and written by one TMA store; a partial last
+            // chunk is stored from registers, row by row.
+            const int r0 = 16 * wg;
+            float v[16];
+            tmem_ld16(tq + TM_O + r0, v);
+            tmem_wait16(v);
+            if (Lc == C) {
+                __nv_bfloat16* os = reinterpret_cast<__nv_bfloat16*>(sm + Lay::RV + vbuf * 16384);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) os[(r0 + i) * D + lrow] = __float2bfloat16_rn(v[i]);
+                fence_async_smem();
+                __syncthreads();
+                if (tid == 0) {
+                    tma_store_tile(&maps.out, sm + Lay::RV + vbuf * 16384, h, (int)t0);
+                    bulk_commit();
+                }
+            } else {
+                __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out) + (int64_t)h * D + lrow;
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    if (r0 + i < Lc) out[(t0 + r0 + i) * H * (int64_t)D] = __float2bfloat16_rn(v[i]);
+            }
         }
         tc_fence_before();
         __syncthreads();
@@ -745,7 +829,7 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
     }
 
     // ---- results of the segment
-    if (ok && !SEG && prev_t0 >= 0) store_out(vbuf ^ 1);
+    if (!SEG && tid == 0) bulk_wait_all();  // output stores have left shared memory
     if (ok) {
         if (SEG) {  // slices 0-1: B^T, slices 2-3: M^T, 64 columns each
             const bool is_m = wg >= 2;
@@ -989,7 +1073,8 @@ cudaError_t launch_tc(const TcArgs& a, const TcPlan& p, cudaStream_t stream, int
         if ((err = tile_map(&maps.q, a.q, false, a.H, tokens, false)) != cudaSuccess ||
             (err = tile_map(&maps.k, a.k, false, a.H, tokens, false)) != cudaSuccess ||
             (err = tile_map(&maps.v, a.v, false, a.H, tokens, true)) != cudaSuccess ||
-            (err = tile_map(&maps.la, a.log_alpha, true, a.H, tokens, false)) != cudaSuccess)
+            (err = tile_map(&maps.la, a.log_alpha, true, a.H, tokens, false)) != cudaSuccess ||
+            (err = tile_map(&maps.out, a.out, false, a.H, tokens, false)) != cudaSuccess)
             return err;
     }
     profile_mark(SLOT_SETUP, true, stream);

@@ -39,6 +39,11 @@ CASES = [  # M, N, K, a_mn, b_mn, neg, init
     (128, 128, 64, 1, 1, 0, 0),
     (128, 64, 128, 0, 1, 1, 1),
     (128, 128, 64, 0, 0, 0, 1),
+    # A read from TMEM (packed bf16 pairs)
+    (128, 64, 128, 2, 1, 0, 0),
+    (128, 128, 64, 2, 1, 0, 0),
+    (128, 64, 64, 2, 0, 0, 0),
+    (128, 64, 128, 2, 1, 1, 1),
 ]
 
 
