@@ -12,6 +12,12 @@ kda_fwd_host with the host->device copy of the inputs and the device->host copy
 of the outputs inside every timed step.  The workload's inputs (12.9 GB) are
 larger than the 126 MB L2, so no flush is needed between steps.
 
+``--workload decode_1024x1`` / ``verify_512x4`` time instead one decode /
+multi-token verify step (kda_decode) over 1024 sequences x 1 token or 512
+sequences x 4 tokens whose states (8 heads x 64 KiB each) stay resident and are
+updated in place; there ``e2e`` copies the step's tokens up and its outputs back
+through the Python binding while the states stay on the device.
+
 With N GPUs (torchrun, one rank per GPU) every rank runs its own copy of the
 workload (independent problems, no data-path collective): weak scaling, value =
 N * tokens / max-over-ranks time.
@@ -34,9 +40,11 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from gated_delta_rule_139_b200.inputs import (WORKLOADS, algorithmic_bytes,  # noqa: E402
-                                              algorithmic_flops, make_inputs, workload)
+                                              algorithmic_flops, is_decode, make_inputs,
+                                              workload)
 
 METRIC = "KDA chunked prefill Mtokens/s on 1 B200; % of bf16 tensor / HBM roofline"
+METRIC_DECODE = "KDA decode/verify step Mtokens/s on 1 B200 (resident states); % of HBM roofline"
 UNIT = "Mtokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -57,6 +65,17 @@ def workload_config(inp, n_gpus):
             "gates": "fp32 log_alpha, fp32 beta", "state": "fp32",
             "l2": "inputs larger than L2 (%.1f GB per step vs 126 MB L2), no flush" %
                   (algorithmic_bytes(inp) / 1e9),
+            "parallelism": f"dp{n_gpus} (independent problem per GPU)"}
+
+
+def decode_config(inp, n_gpus):
+    st = inp.n_seqs * inp.H * inp.dk * inp.dv * 4
+    return {"workload": inp.name, "step": "decode/verify on resident states (kda_decode)",
+            "sequences": inp.B, "new_tokens_per_seq": inp.T, "H": inp.H, "d_k": inp.dk,
+            "d_v": inp.dv, "tokens_per_gpu": inp.tokens,
+            "qkv_dtype": "bf16" if inp.bf16 else "f32", "gates": "fp32 log_alpha, fp32 beta",
+            "state": "fp32, updated in place",
+            "l2": "states larger than L2 (%.0f MB vs 126 MB L2), no flush" % (st / 1e6),
             "parallelism": f"dp{n_gpus} (independent problem per GPU)"}
 
 
@@ -137,9 +156,36 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ oracle baseline
+def decode_sample(name: str, target_s: float, seed: int = 0):
+    """Sequences of a decode workload's recipe that take the oracle about
+    target_s seconds (whole workload at most): (inputs, threads)."""
+    import oracle
+    spec = dict(WORKLOADS[name])
+    spec.pop("step")
+    B = spec.pop("B")
+    threads = min(len(os.sched_getaffinity(0)), spec["H"])
+    probe = make_inputs(B=min(B, 32), seed=seed, name=name, **spec)
+    t0 = time.perf_counter()
+    oracle.recurrent(probe.q, probe.k, probe.v, probe.log_alpha, probe.beta,
+                     probe.initial_state, None, threads=threads)
+    per_seq = max(time.perf_counter() - t0, 1e-6) / probe.B
+    n = int(max(1, min(B, target_s / per_seq)))
+    return make_inputs(B=n, seed=seed, name=name, **spec), threads
+
+
 def oracle_sample_rate(inp_name: str, target_s: float = 15.0, seed: int = 0):
     """Time the fp64 oracle on a bounded prefix of the workload's recipe."""
     import oracle
+    if is_decode(inp_name):
+        x, threads = decode_sample(inp_name, target_s, seed)
+        t0 = time.perf_counter()
+        oracle.recurrent(x.q, x.k, x.v, x.log_alpha, x.beta, x.initial_state, None,
+                         threads=threads)
+        dt = time.perf_counter() - t0
+        return {"value": x.tokens / dt / 1e6, "unit": UNIT, "cores": threads, "kind": "oracle",
+                "sample": f"{x.B} of the sequences x {x.T} tokens x {x.H} heads of the "
+                          f"{inp_name} recipe (fp64 token recurrence, {dt:.1f} s)",
+                "seconds": dt}
     spec = dict(WORKLOADS[inp_name])
     spec.pop("packed", None)
     spec.pop("T", None)
@@ -170,6 +216,8 @@ def run_reference(args, rank, world):
         return
     import oracle
     name = args.workload
+    if is_decode(name):
+        return run_reference_decode(args, world)
     spec = dict(WORKLOADS[name])
     spec.pop("packed", None)
     spec.pop("T", None)
@@ -204,6 +252,35 @@ def run_reference(args, rank, world):
             "cpu_baseline": {"value": val, "unit": UNIT, "cores": threads, "kind": "oracle",
                              "sample": f"first {T_s} tokens x {H} heads of the {name} recipe "
                                        "per step (fp64 token recurrence)"},
+            "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_reference_decode(args, world):
+    import oracle
+    x, threads = decode_sample(args.workload, 2.0)
+    f = lambda: oracle.recurrent(x.q, x.k, x.v, x.log_alpha, x.beta, x.initial_state, None,
+                                 threads=threads)
+    for _ in range(args.warmup):
+        f()
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        f()
+        times.append(time.perf_counter() - t0)
+    step = sum(times) / len(times)
+    val = x.tokens / step / 1e6
+    cfg = decode_config(x, world)
+    cfg["sampled_sequences"] = x.B
+    sample = (f"{x.B} of the sequences x {x.T} tokens x {x.H} heads of the {args.workload} "
+              "recipe per step (fp64 token recurrence)")
+    line = {"impl": "reference", "metric": METRIC_DECODE, "value": val, "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": step * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg,
+            "cpu_baseline": {"value": val, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": sample},
             "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -313,7 +390,9 @@ def main():
     host = {k: (None if getattr(inp, k) is None else pinned(getattr(inp, k)))
             for k in ("q", "k", "v", "log_alpha", "beta", "initial_state")}
     alg_bytes = algorithmic_bytes(inp)
-    alg_flops = algorithmic_flops(inp)
+    # a decode token costs 7 flops per state element (decay; S^T k; rank-1 update; S^T q)
+    alg_flops = (7.0 * inp.tokens * inp.H * inp.dk * inp.dv if is_decode(args.workload)
+                 else algorithmic_flops(inp))
     v_shape = tuple(inp.v.shape)
     for k_ in ("q", "k", "v", "log_alpha", "beta"):
         setattr(inp, k_, None)  # the pinned copies are the host data from here on
@@ -326,9 +405,15 @@ def main():
         fs = torch.empty((inp.n_seqs, inp.H, inp.dk, inp.dv), dtype=torch.float32, device=dev)
     stream.synchronize()
 
+    decode = is_decode(args.workload)
+
     def step():
-        kda.kda_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["initial_state"],
-                    cu_dev, 64, out, fs, stream=stream)
+        if decode:  # the state is updated in place, step after step
+            kda.kda_decode(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"],
+                           d["initial_state"], out=out, stream=stream)
+        else:
+            kda.kda_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["initial_state"],
+                        cu_dev, 64, out, fs, stream=stream)
         return kda.last_launch_count()
 
     for _ in range(args.warmup):
@@ -369,9 +454,21 @@ def main():
         fs_h = torch.empty((inp.n_seqs, inp.H, inp.dk, inp.dv), dtype=torch.float32).pin_memory()
         cu_arg = None if cu_host is None else np.ascontiguousarray(cu_host, dtype=np.int32)
 
+        tok_keys = ("q", "k", "v", "log_alpha", "beta")
+
         def e2e_step():
-            kda.kda_fwd_host(host["q"], host["k"], host["v"], host["log_alpha"], host["beta"],
-                             host["initial_state"], cu_arg, 64, out_h, fs_h, stream=stream)
+            if decode:
+                # a serving step: this step's tokens go up, the outputs come back,
+                # the states stay resident on the device
+                with torch.cuda.stream(stream):
+                    x = {k_: host[k_].to(dev, non_blocking=True) for k_ in tok_keys}
+                    o, _ = kda.kda_decode(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"],
+                                          d["initial_state"], stream=stream)
+                    out_h.copy_(o, non_blocking=True)
+            else:
+                kda.kda_fwd_host(host["q"], host["k"], host["v"], host["log_alpha"],
+                                 host["beta"], host["initial_state"], cu_arg, 64, out_h, fs_h,
+                                 stream=stream)
 
         e2e_step()
         if pg:
@@ -383,8 +480,12 @@ def main():
         e1.record(stream)
         stream.synchronize()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, pg, dev)
-        h2d = sum(nbytes(t) for t in host.values()) + (0 if cu_arg is None else cu_arg.nbytes)
-        d2h = nbytes(out_h) + nbytes(fs_h)
+        if decode:
+            h2d = sum(nbytes(host[k_]) for k_ in tok_keys)
+            d2h = nbytes(out_h)
+        else:
+            h2d = sum(nbytes(t) for t in host.values()) + (0 if cu_arg is None else cu_arg.nbytes)
+            d2h = nbytes(out_h) + nbytes(fs_h)
         e2e = {"value": job_throughput(world, tokens, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                "steps": args.e2e_steps}
@@ -403,10 +504,12 @@ def main():
     achieved = dom_bytes / (kernels[dom]["ms_per_launch"] * 1e-3) / 1e9
     t_roof = max(alg_bytes / (peaks["hbm_gbs"] * 1e9), alg_flops / (peaks["bf16_tflops"] * 1e12))
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32" if kda.last_path() == "ffma" else "bf16",
-        "data": "synthetic", "config": workload_config(inp, world),
+        "metric": METRIC_DECODE if decode else METRIC, "value": value, "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32" if kda.last_path() in ("ffma", "decode") else "bf16",
+        "data": "synthetic",
+        "config": decode_config(inp, world) if decode else workload_config(inp, world),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
                      "traffic": recorded_traffic(dom),

@@ -17,7 +17,7 @@ from __future__ import annotations
 import ctypes
 import os
 
-__all__ = ["kda_fwd", "kda_fwd_host", "kda_fwd_noalloc", "KDAError", "library_path", "load_library",
+__all__ = ["kda_fwd", "kda_fwd_host", "kda_fwd_noalloc", "kda_decode", "KDAError", "library_path", "load_library",
            "last_launch_count", "last_path", "check_device", "profile_enable", "profile_read",
            "STATUS"]
 
@@ -43,6 +43,12 @@ class Dims(ctypes.Structure):
                 ("qkv_dtype", ctypes.c_int32)]
 
 
+class DecodeDims(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int32), ("T", ctypes.c_int32), ("H", ctypes.c_int32),
+                ("d_k", ctypes.c_int32), ("d_v", ctypes.c_int32), ("num_slots", ctypes.c_int32),
+                ("qkv_dtype", ctypes.c_int32)]
+
+
 _lib = None
 
 
@@ -60,6 +66,8 @@ def load_library():
             fn = getattr(lib, name)
             fn.argtypes = sig
             fn.restype = ctypes.c_int
+        lib.kda_decode.argtypes = [p, p, p, p, p, p, p, p, p, ctypes.POINTER(DecodeDims), p]
+        lib.kda_decode.restype = ctypes.c_int
         lib.kda_status_string.argtypes = [ctypes.c_int]
         lib.kda_status_string.restype = ctypes.c_char_p
         lib.kda_last_error.argtypes = []
@@ -86,7 +94,7 @@ def last_launch_count() -> int:
 
 
 def last_path() -> str:
-    """Kernel family of the last kda_fwd call on this thread ("ffma" or "tc")."""
+    """Kernel family of the last call on this thread ("ffma", "tc" or "decode")."""
     return load_library().kda_last_path().decode()
 
 
@@ -98,7 +106,7 @@ def profile_enable(on: bool = True) -> None:
 def profile_read() -> dict:
     """{kernel name: (summed ms, launches)} since the previous read (synchronises)."""
     lib = load_library()
-    n = 5
+    n = 6
     ms = (ctypes.c_double * n)()
     cnt = (ctypes.c_int64 * n)()
     _check(lib.kda_profile_read(ctypes.cast(ms, ctypes.c_void_p), ctypes.cast(cnt, ctypes.c_void_p), n))
@@ -224,3 +232,43 @@ def kda_fwd_host(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
                           h(cu_seqlens), int(chunk), h(out), h(final_state), ctypes.byref(d), s)
     _check(rc)
     return out, final_state
+
+
+def kda_decode(q, k, v, log_alpha, beta, state, slots=None, out=None, token_states=None,
+               want_token_states: bool = False, stream=None):
+    """Decode / multi-token verify step: T new tokens per sequence on a resident
+    state, which is updated IN PLACE.  Returns (out, token_states or None).
+
+    q, k [N,T,H,d_k]; v [N,T,H,d_v] (bf16 or fp32); log_alpha [N,T,H,d_k] and
+    beta [N,T,H] fp32; state [S,H,d_k,d_v] fp32 where S = N, or the pool size
+    when ``slots`` (int32 [N] on the device; -1 = padding entry) maps sequences
+    to pool rows.  ``token_states`` [N,T,H,d_k,d_v] receives the state after
+    every token (allocated here when ``want_token_states``).
+    """
+    import torch
+
+    lib = load_library()
+    bf16 = q.dtype == torch.bfloat16
+    if not bf16 and q.dtype != torch.float32:
+        raise TypeError("q/k/v must be bfloat16 or float32")
+    for t in (q, k, v, log_alpha, beta, state):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("inputs must be contiguous CUDA tensors")
+    if q.dim() != 4:
+        raise ValueError("q must be [N,T,H,d_k]")
+    N, T, H, dk = q.shape
+    dv = v.shape[-1]
+    d = DecodeDims(N, T, H, dk, dv, state.shape[0] if slots is not None else N,
+                   KDA_BF16 if bf16 else KDA_F32)
+    if out is None:
+        out = torch.empty((N, T, H, dv), dtype=q.dtype, device=q.device)
+    if token_states is None and want_token_states:
+        token_states = torch.empty((N, T, H, dk, dv), dtype=torch.float32, device=q.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    ptr = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
+    rc = lib.kda_decode(ptr(q), ptr(k), ptr(v), ptr(log_alpha), ptr(beta), ptr(state), ptr(slots),
+                        ptr(out), ptr(token_states), ctypes.byref(d),
+                        ctypes.c_void_p(stream.cuda_stream))
+    _check(rc)
+    return out, token_states

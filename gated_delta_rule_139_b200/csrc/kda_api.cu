@@ -486,6 +486,85 @@ kda_status kda_fwd_noalloc(const void* q, const void* k, const void* v, const fl
     return KDA_OK;
 }
 
+kda_status kda_decode(const void* q, const void* k, const void* v, const float* log_alpha,
+                      const float* beta, float* state, const int32_t* slots, void* out,
+                      float* token_states, const kda_decode_dims* d, void* stream) {
+    g_last_error[0] = 0;
+    g_last_launches = 0;
+    g_last_path = "";
+    if (!d) return fail(KDA_ERR_INVALID_ARG, "dims is NULL");
+    if (d->N < 0 || d->T < 0 || d->H < 1)
+        return fail(KDA_ERR_INVALID_ARG, "need N >= 0, T >= 0, H >= 1 (got N=%d T=%d H=%d)", d->N,
+                    d->T, d->H);
+    if (d->qkv_dtype != KDA_F32 && d->qkv_dtype != KDA_BF16)
+        return fail(KDA_ERR_INVALID_ARG, "qkv_dtype must be KDA_F32 or KDA_BF16");
+    if ((d->d_k != 64 && d->d_k != 128) || (d->d_v != 64 && d->d_v != 128))
+        return fail(KDA_ERR_UNSUPPORTED, "d_k and d_v must be 64 or 128 (got %d, %d)", d->d_k,
+                    d->d_v);
+    if (slots && d->num_slots < 1)
+        return fail(KDA_ERR_INVALID_ARG, "num_slots must be >= 1 with a slot table");
+    const int64_t S = slots ? d->num_slots : d->N;
+    const int64_t tokens = (int64_t)d->N * d->T;
+    const int64_t e_in = d->qkv_dtype == KDA_BF16 ? 2 : 4;
+    const int64_t nqk = tokens * d->H * d->d_k, nv = tokens * d->H * d->d_v;
+    const int64_t dd = (int64_t)d->d_k * d->d_v;
+    if ((int64_t)d->N * d->H == 0) return KDA_OK;
+    if ((int64_t)d->N * d->H > INT32_MAX)
+        return fail(KDA_ERR_UNSUPPORTED, "N * H = %lld exceeds 2^31 - 1",
+                    (long long)d->N * d->H);
+    if (!state) return fail(KDA_ERR_INVALID_ARG, "state must be non-NULL");
+    if (tokens > 0 && (!q || !k || !v || !log_alpha || !beta || !out))
+        return fail(KDA_ERR_INVALID_ARG, "q, k, v, log_alpha, beta and out must be non-NULL");
+    const void* ptrs[] = {q, k, v, log_alpha, beta, state, slots, out, token_states};
+    const char* names[] = {"q", "k", "v", "log_alpha", "beta", "state", "slots", "out",
+                           "token_states"};
+    for (int i = 0; i < 9; ++i) {
+        if (ptrs[i] && ((uintptr_t)ptrs[i] & 15u) && i != 6)
+            return fail(KDA_ERR_MISALIGNED, "%s is not 16-byte aligned", names[i]);
+        if (i == 6 && ptrs[i] && ((uintptr_t)ptrs[i] & 3u))
+            return fail(KDA_ERR_MISALIGNED, "slots is not 4-byte aligned");
+    }
+    const int64_t bytes[] = {nqk * e_in, nqk * e_in, nv * e_in, nqk * 4, tokens * d->H * 4,
+                             S * d->H * dd * 4, (int64_t)d->N * 4, nv * e_in,
+                             tokens * d->H * dd * 4};
+    Range r[9];
+    for (int i = 0; i < 9; ++i)
+        r[i] = {(uintptr_t)ptrs[i], (uintptr_t)ptrs[i] + (ptrs[i] ? bytes[i] : 0), names[i]};
+    // written buffers (state, out, token_states) overlap nothing else
+    for (int w : {5, 7, 8})
+        for (int i = 0; i < 9; ++i)
+            if (i != w && overlaps(r[w], r[i]))
+                return fail(KDA_ERR_ALIAS, "%s overlaps %s", names[w], names[i]);
+    for (int i = 0; i < 9; ++i)
+        if (ptrs[i] && !device_accessible(ptrs[i]))
+            return fail(KDA_ERR_INVALID_ARG, "%s is not device-accessible memory", names[i]);
+    kda::DecodeArgs a;
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.log_alpha = log_alpha;
+    a.beta = beta;
+    a.state = state;
+    a.slots = slots;
+    a.out = out;
+    a.token_states = token_states;
+    a.N = d->N;
+    a.T = d->T;
+    a.H = d->H;
+    a.dk = d->d_k;
+    a.dv = d->d_v;
+    a.num_slots = (int32_t)S;
+    a.bf16 = d->qkv_dtype == KDA_BF16;
+    cudaError_t e = kda::status_word(&a.status);
+    if (e != cudaSuccess) return cuda_fail(e, "device status word");
+    int launches = 0;
+    g_last_path = "decode";
+    e = kda::launch_decode(a, (cudaStream_t)stream, &launches);
+    g_last_launches = launches;
+    if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+    return KDA_OK;
+}
+
 const char* kda_status_string(kda_status s) {
     switch (s) {
         case KDA_OK: return "KDA_OK";
@@ -535,7 +614,7 @@ kda_status kda_profile_read(double* total_ms, int64_t* launches, int32_t n) {
 
 const char* kda_profile_slot_name(int32_t slot) {
     static const char* names[] = {"seg_setup", "tc_pass1_transitions", "seg_scan",
-                                  "tc_pass3_forward", "ffma_forward"};
+                                  "tc_pass3_forward", "ffma_forward", "decode_step"};
     return (slot >= 0 && slot < kda::NUM_SLOTS) ? names[slot] : "";
 }
 
@@ -546,8 +625,11 @@ kda_status kda_check_device(void* stream) {
     int code = 0;
     e = kda::tc_take_status(&code);
     if (e != cudaSuccess) return cuda_fail(e, "device status read");
-    if (code == 1) return fail(KDA_ERR_DEVICE_TIMEOUT, "a bounded device wait gave up");
-    if (code == 2) return fail(KDA_ERR_INVALID_ARG, "segment table overflow: malformed cu_seqlens");
+    if (code == kda::ERR_WAIT_TIMEOUT) return fail(KDA_ERR_DEVICE_TIMEOUT, "a bounded device wait gave up");
+    if (code == kda::ERR_SEG_OVERFLOW)
+        return fail(KDA_ERR_INVALID_ARG, "segment table overflow: malformed cu_seqlens");
+    if (code == kda::ERR_BAD_SLOT)
+        return fail(KDA_ERR_INVALID_ARG, "a decode slot index lies outside the state pool");
     if (code) return fail(KDA_ERR_CUDA, "device status %d", code);
     return KDA_OK;
 }

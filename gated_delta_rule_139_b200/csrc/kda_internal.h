@@ -11,7 +11,12 @@ constexpr int kMaxDevices = 64;  // size of per-device attribute caches
 
 // Kernel slots of the optional per-launch timing (kda_profile_*).
 enum KernelSlot : int { SLOT_SETUP = 0, SLOT_PASS1 = 1, SLOT_SCAN = 2, SLOT_PASS3 = 3, SLOT_FFMA = 4,
-                        NUM_SLOTS = 5 };
+                        SLOT_DECODE = 5, NUM_SLOTS = 6 };
+
+// Device status codes (first error wins; read and cleared by kda_check_device).
+enum DeviceStatus : int { ERR_WAIT_TIMEOUT = 1, ERR_SEG_OVERFLOW = 2, ERR_BAD_SLOT = 3 };
+// Device address of the current device's status word.
+cudaError_t status_word(int** p);
 // Records a CUDA event on `stream` before (begin=true) or after a launch of
 // `slot` when timing is enabled; no-op otherwise.
 void profile_mark(int slot, bool begin, cudaStream_t stream);
@@ -80,5 +85,22 @@ cudaError_t launch_tc(const TcArgs& a, const TcPlan& p, cudaStream_t stream, int
 size_t tc_smem_bytes();
 // Reads and clears the current device's status word (0 = no device-side error).
 cudaError_t tc_take_status(int* code);
+
+// Decode / multi-token verify step on a resident state (validated on the host).
+struct DecodeArgs {
+    const void* q;             // [N, T, H, dk]
+    const void* k;             // [N, T, H, dk]
+    const void* v;             // [N, T, H, dv]
+    const float* log_alpha;    // [N, T, H, dk]
+    const float* beta;         // [N, T, H]
+    float* state;              // [num_slots, H, dk, dv], read and written in place
+    const int32_t* slots;      // [N] state row of each sequence (-1 = skip), or nullptr
+    void* out;                 // [N, T, H, dv]
+    float* token_states;       // [N, T, H, dk, dv] or nullptr
+    int* status;               // device status word
+    int32_t N, T, H, dk, dv, num_slots;
+    int32_t bf16;
+};
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream, int* launches);
 
 }  // namespace kda

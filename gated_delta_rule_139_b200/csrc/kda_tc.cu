@@ -58,7 +58,6 @@ constexpr int D = 128;    // d_k = d_v
 constexpr int NT = 512;   // threads per CTA: 16 warps, 4 per TMEM lane quadrant
 constexpr float LOG2E = 1.4426950408889634f;
 
-enum : int { ERR_WAIT_TIMEOUT = 1, ERR_SEG_OVERFLOW = 2 };
 
 // ---------------------------------------------------------------- shared memory map
 // Region R1 is reused across the phases of one chunk:
@@ -1041,6 +1040,24 @@ cudaError_t tile_map(CUtensorMap* m, const void* base, bool f32, int H, int64_t 
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 }  // namespace
+
+cudaError_t status_word(int** p) {
+    static int* addr[kMaxDevices] = {};
+    static std::mutex mu;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void* a = nullptr;
+        e = cudaGetSymbolAddress(&a, g_tc_status);
+        if (e != cudaSuccess) return e;
+        addr[dev] = (int*)a;
+    }
+    *p = addr[dev];
+    return cudaSuccess;
+}
 
 cudaError_t tc_take_status(int* code) {
     int zero = 0;

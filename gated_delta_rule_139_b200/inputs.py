@@ -4,7 +4,7 @@ This module only draws random numbers and shapes them; it holds none of the
 recurrence's arithmetic.  It serves both the CUDA library's tests/benchmark and
 the fp64 oracle, which receive the same arrays.
 
-Recipes (the five workloads the library is measured and checked on):
+Recipes (the five forward workloads the library is measured and checked on):
 
   ``tiny_fp32``   B=1, H=1, T=256, d_k=d_v=64, fp32 q/k/v; q,k ~ N(0,1) then
                   L2-normalised per (token, head); v ~ N(0,1);
@@ -20,6 +20,13 @@ Recipes (the five workloads the library is measured and checked on):
                   one random initial state ~ N(0,0.02) per sequence.
   ``prefill_1m``  B=1, H=8, T=2^20, d=128, bf16; log_alpha = -softplus(N(-1,1))
                   clamped; zero initial state.
+
+Two more recipes time the decode / multi-token verify step on resident states:
+
+  ``decode_1024x1``  1024 sequences x 1 new token, H=8, d=128, bf16; gates of
+                     ``prefill_1m``; states ~ N(0,0.3) (a state after a long
+                     prefill holds O(1) entries).
+  ``verify_512x4``   512 sequences x 4 drafted tokens, otherwise the same.
 
 N(mu, sigma) means mean and standard deviation.  Every workload uses seed 0;
 each tensor draws from its own child of ``np.random.SeedSequence(seed)`` in the
@@ -224,12 +231,25 @@ WORKLOADS = {
                       state_sigma=0.02, packed=(16, 1024, 32768)),
     "prefill_1m": dict(B=1, T=1 << 20, H=8, dk=128, dv=128, bf16=True, gate_mu=-1.0,
                        gate_sigma=1.0, state_sigma=None),
+    # decode / multi-token verify steps on resident states (kda_decode): B
+    # sequences of T new tokens each; the states (B x 8 heads x 64 KiB) are
+    # larger than the 126 MB L2.
+    "decode_1024x1": dict(B=1024, T=1, H=8, dk=128, dv=128, bf16=True, gate_mu=-1.0,
+                          gate_sigma=1.0, state_sigma=0.3, step="decode"),
+    "verify_512x4": dict(B=512, T=4, H=8, dk=128, dv=128, bf16=True, gate_mu=-1.0,
+                         gate_sigma=1.0, state_sigma=0.3, step="decode"),
 }
+
+
+def is_decode(name: str) -> bool:
+    """True for the workloads that time a decode / verify step (kda_decode)."""
+    return WORKLOADS[name].get("step") == "decode"
 
 
 def workload(name: str, seed: int = 0) -> KDAInputs:
     """Build one of the five named workloads (see the module docstring)."""
     spec = dict(WORKLOADS[name])
+    spec.pop("step", None)
     packed = spec.pop("packed", None)
     if packed is not None:
         lens = packed_lengths(*packed, seed=seed)
@@ -266,5 +286,5 @@ def algorithmic_flops(inp: KDAInputs, chunk: int = 64) -> float:
     return per_token * inp.tokens * inp.H
 
 
-__all__ = ["KDAInputs", "make_inputs", "workload", "WORKLOADS", "f32_to_bf16", "bf16_to_f32",
+__all__ = ["KDAInputs", "make_inputs", "workload", "WORKLOADS", "is_decode", "f32_to_bf16", "bf16_to_f32",
            "packed_lengths", "algorithmic_bytes", "algorithmic_flops"]

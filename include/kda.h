@@ -144,33 +144,88 @@ kda_status kda_fwd_noalloc(const void* q, const void* k, const void* v, const fl
                            const int32_t* cu_seqlens, int32_t chunk, void* out,
                            float* final_state, const kda_dims* dims, void* stream);
 
+/* Shapes of a decode / verify step. */
+typedef struct {
+    int32_t N;          /* sequences in the step (>= 0)                             */
+    int32_t T;          /* new tokens per sequence (>= 0; meant for 1..16)          */
+    int32_t H;          /* heads (>= 1)                                             */
+    int32_t d_k;        /* 64 or 128                                                */
+    int32_t d_v;        /* 64 or 128                                                */
+    int32_t num_slots;  /* rows of the state pool when slots != NULL (>= 1); else N */
+    int32_t qkv_dtype;  /* kda_dtype of q, k, v and out                             */
+} kda_decode_dims;
+
+/*
+ * kda_decode -- a few new tokens per sequence on a resident state, in place.
+ *
+ * The same recurrence as kda_fwd (section "Как хранить миллион токенов в
+ * памяти" of the page named at the top), evaluated token by token as in
+ * generation: a decoder passes T = 1; a speculative-decoding verifier passes
+ * the T drafted tokens at once (the same page, in its account of the training
+ * pipeline, describes an auxiliary draft model whose proposed tokens the main
+ * model confirms in batches).  Equal to
+ * kda_fwd on the same tokens with initial_state = final_state = state, but
+ * without a 64-token chunk per call: the work is one read and one write of the
+ * state (64 KiB of fp32 per head at d_k = d_v = 128) plus the tokens.
+ *
+ * Tensors are dense, row-major, 16-byte aligned, device-resident, owned by
+ * the caller:
+ *   q, k         [N, T, H, d_k]   qkv_dtype
+ *   v            [N, T, H, d_v]   qkv_dtype
+ *   log_alpha    [N, T, H, d_k]   fp32, clamped to [-5, 0] inside
+ *   beta         [N, T, H]        fp32, used as given
+ *   state        [S, H, d_k, d_v] fp32 (S = num_slots with slots, else N):
+ *                                 read, then overwritten with the state after
+ *                                 the T tokens
+ *   slots        [N] int32 on the device, or NULL (sequence n uses state row
+ *                n).  Row slots[n] of the pool holds sequence n's state; -1
+ *                marks a padding entry, which reads and writes nothing (its
+ *                out rows are left as they were).  Other values outside
+ *                [0, num_slots) skip the sequence the same way and set the
+ *                device status word (kda_check_device: KDA_ERR_INVALID_ARG).
+ *                Two sequences must not name the same slot.
+ *   out          [N, T, H, d_v]   qkv_dtype (bf16 rounded to nearest even)
+ *   token_states [N, T, H, d_k, d_v] fp32, or NULL: the state after each of
+ *                the T tokens, so that a verifier that accepts only the first
+ *                m tokens can continue from token_states[n][m-1]
+ *
+ * No buffer may overlap another.  Allocates nothing; one kernel launch.
+ */
+kda_status kda_decode(const void* q, const void* k, const void* v, const float* log_alpha,
+                      const float* beta, float* state, const int32_t* slots, void* out,
+                      float* token_states, const kda_decode_dims* dims, void* stream);
+
 /* Static description of a status code. */
 const char* kda_status_string(kda_status s);
 
 /* Detail of the last error raised on the calling host thread ("" if none). */
 const char* kda_last_error(void);
 
-/* Number of kernel launches the last kda_fwd call on this host thread issued. */
+/* Number of kernel launches the last kda_fwd / kda_decode call on this host
+ * thread issued. */
 int32_t kda_last_launch_count(void);
 
-/* Kernel family the last kda_fwd call on this host thread used: "ffma" (fp32
- * CUDA-core path), "tc" (tcgen05 tensor-core path) or "" (no launch). */
+/* Kernel family the last kda_fwd / kda_decode call on this host thread used:
+ * "ffma" (fp32 CUDA-core path), "tc" (tcgen05 tensor-core path), "decode"
+ * (kda_decode) or "" (no launch). */
 const char* kda_last_path(void);
 
 /* Synchronises `stream`, then reads and clears the current device's status
  * word, which kernels set when a bounded wait gives up (KDA_ERR_DEVICE_TIMEOUT)
- * or the device-built segment table would overflow because cu_seqlens is
- * malformed (KDA_ERR_INVALID_ARG).  KDA_OK when neither happened since the last
+ * (KDA_ERR_DEVICE_TIMEOUT), the device-built segment table would overflow
+ * because cu_seqlens is malformed, or a kda_decode slot index lay outside the
+ * state pool (both KDA_ERR_INVALID_ARG).  KDA_OK when neither happened since the last
  * check. */
 kda_status kda_check_device(void* stream);
 
-/* Optional launch timing (off by default).  While enabled, every kda_fwd
- * records a CUDA event on its stream before and after each internal kernel
- * launch.  kda_profile_read synchronises those events, writes for each of the
+/* Optional launch timing (off by default).  While enabled, every kda_fwd and
+ * kda_decode call records a CUDA event on its stream before and after each
+ * internal kernel launch.  kda_profile_read synchronises those events, writes for each of the
  * first n kernel slots the summed duration in milliseconds and the number of
  * launches since the previous read, then resets the sums.  Slots: 0 segment
  * table, 1 pass 1 (segment transitions), 2 segment scan, 3 pass 3 (forward),
- * 4 CUDA-core forward; kda_profile_slot_name gives their names. */
+ * 4 CUDA-core forward, 5 decode step; kda_profile_slot_name gives their
+ * names. */
 void kda_profile_enable(int32_t on);
 kda_status kda_profile_read(double* total_ms, int64_t* launches, int32_t n);
 const char* kda_profile_slot_name(int32_t slot);

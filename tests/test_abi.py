@@ -92,3 +92,49 @@ def test_state_in_place_passes_host_checks():
 def test_zero_length_is_accepted_by_host_checks():
     st, msg = call(D(T=0), q=None, k=None, v=None, la=None, be=None, out=None)
     assert st in ("KDA_OK", "KDA_ERR_CUDA")  # no device needed for T=0 validation
+
+
+# ---------------------------------------------------------------- kda_decode arguments
+def call_decode(dims, q=FAKE, k=FAKE + (1 << 30), v=FAKE + (2 << 30), la=FAKE + (3 << 30),
+                be=FAKE + (4 << 30), st=FAKE + (6 << 30), slots=None, out=FAKE + (5 << 30),
+                ts=None):
+    lib = kda.load_library()
+    P = lambda x: None if x is None else ctypes.c_void_p(x)
+    rc = lib.kda_decode(P(q), P(k), P(v), P(la), P(be), P(st), P(slots), P(out), P(ts),
+                        ctypes.byref(dims), None)
+    return kda.STATUS[rc], lib.kda_last_error().decode()
+
+
+def DD(N=4, T=2, H=2, dk=128, dv=128, S=0, dt=1):
+    return kda.DecodeDims(N, T, H, dk, dv, S, dt)
+
+
+def test_decode_rejects_bad_arguments():
+    assert call_decode(DD(N=-1))[0] == "KDA_ERR_INVALID_ARG"
+    assert call_decode(DD(T=-1))[0] == "KDA_ERR_INVALID_ARG"
+    assert call_decode(DD(H=0))[0] == "KDA_ERR_INVALID_ARG"
+    assert call_decode(DD(dt=3))[0] == "KDA_ERR_INVALID_ARG"
+    assert call_decode(DD(dk=32))[0] == "KDA_ERR_UNSUPPORTED"
+    assert call_decode(DD(), st=None)[0] == "KDA_ERR_INVALID_ARG"
+    assert call_decode(DD(), v=None)[0] == "KDA_ERR_INVALID_ARG"
+    assert call_decode(DD(S=0), slots=FAKE + (7 << 30))[0] == "KDA_ERR_INVALID_ARG"
+    assert call_decode(DD(), out=FAKE + (5 << 30) + 4)[0] == "KDA_ERR_MISALIGNED"
+    assert call_decode(DD(S=8), slots=FAKE + (7 << 30) + 2)[0] == "KDA_ERR_MISALIGNED"
+    lib = kda.load_library()
+    assert kda.STATUS[lib.kda_decode(None, None, None, None, None, None, None, None, None, None,
+                                     None)] == "KDA_ERR_INVALID_ARG"
+
+
+def test_decode_rejects_aliasing():
+    # out inside v; state inside k; token_states overlapping the state
+    assert call_decode(DD(), out=FAKE + (2 << 30) + 256)[0] == "KDA_ERR_ALIAS"
+    assert call_decode(DD(), st=FAKE + (1 << 30) + 256)[0] == "KDA_ERR_ALIAS"
+    st, msg = call_decode(DD(), ts=FAKE + (6 << 30) + 4096)
+    assert st == "KDA_ERR_ALIAS" and "token_states" in msg
+
+
+def test_decode_empty_batch_is_a_no_op():
+    # nothing to do: no pointer is looked at, no launch
+    assert call_decode(DD(N=0), q=None, k=None, v=None, la=None, be=None, st=None,
+                       out=None)[0] == "KDA_OK"
+    assert kda.last_launch_count() == 0
