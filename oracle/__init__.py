@@ -102,8 +102,16 @@ def _prep(q, k, v, log_alpha, beta, initial_state, cu_seqlens):
     return q, k, v, la, be, s0, cu, N, T, H, dk, dv, code, lead
 
 
+def _widen(a):
+    """Exact fp64 copy of an fp32 array or of bf16 bit patterns (uint16)."""
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return a.astype(np.float64)
+
+
 def _run(fn_name, q, k, v, log_alpha, beta, initial_state, cu_seqlens, o_tokens, threads,
-         chunk=None):
+         chunk=None, out_gate=None):
     q, k, v, la, be, s0, cu, N, T, H, dk, dv, code, lead = _prep(
         q, k, v, log_alpha, beta, initial_state, cu_seqlens)
     o_tokens = T if o_tokens is None else int(o_tokens)
@@ -118,24 +126,33 @@ def _run(fn_name, q, k, v, log_alpha, beta, initial_state, cu_seqlens, o_tokens,
     rc = getattr(lib, fn_name)(*args)
     if rc != 0:
         raise ValueError(f"{fn_name} rejected its arguments (code {rc})")
+    if out_gate is not None and o_tokens > 0:
+        # the output gate of a KDA block (aiblin.ru page, description of the layer
+        # stack): a share of each output element passes on, o * gate, after the
+        # attention and outside the recurrence
+        g = _widen(out_gate)
+        if g.size != T * H * dv:
+            raise ValueError("out_gate must have the shape of the output")
+        o *= g.reshape(T, H, dv)[:o_tokens]
     if o_tokens == T and len(lead) == 2:
         o = o.reshape(lead + (H, dv))
     return o, sf
 
 
 def recurrent(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, o_tokens=None,
-              threads=0):
+              threads=0, out_gate=None):
     """Token-by-token fp64 evaluation of the KDA recurrence.
 
     Returns (o, final_state): o is float64 [.., H, d_v] for the first ``o_tokens``
-    packed tokens (all by default), final_state float64 [N, H, d_k, d_v].
+    packed tokens (all by default), final_state float64 [N, H, d_k, d_v].  With
+    ``out_gate`` (shape of the output; fp32 or bf16 bits) o is multiplied by it.
     """
     return _run("kda_oracle_recurrent", q, k, v, log_alpha, beta, initial_state, cu_seqlens,
-                o_tokens, threads)
+                o_tokens, threads, out_gate=out_gate)
 
 
 def chunked(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, chunk=64,
-            o_tokens=None, threads=0):
+            o_tokens=None, threads=0, out_gate=None):
     """Chunkwise fp64 reformulation (plain exp(+-g), any chunk size >= 1)."""
     return _run("kda_oracle_chunked", q, k, v, log_alpha, beta, initial_state, cu_seqlens,
-                o_tokens, threads, chunk=chunk)
+                o_tokens, threads, chunk=chunk, out_gate=out_gate)

@@ -298,3 +298,54 @@ def test_bf16_rounding_is_nearest_even():
                                                np.float32(2.9916e38)], np.float32)[:5].tolist()
                                   + [r[5]])
     assert abs(r[5] - 3.0e38) / 3.0e38 < 2**-8
+
+
+# ---------------------------------------------------------------- output gate
+# The gate that follows the attention passes a share of each output element on
+# (aiblin.ru page, description of the layer stack).  Pins: it acts on the output
+# only (never on the state), element by element, multiplicatively.
+def test_gate_of_ones_is_the_ungated_output():
+    x = _case(70, 2, 8, 6, seed=40)
+    o, s = oracle.recurrent(x.q, x.k, x.v, x.log_alpha, x.beta, x.initial_state)
+    og, sg = oracle.recurrent(x.q, x.k, x.v, x.log_alpha, x.beta, x.initial_state,
+                              out_gate=np.ones_like(x.v))
+    np.testing.assert_array_equal(o, og)
+    np.testing.assert_array_equal(s, sg)
+
+
+def test_gate_acts_on_one_element_only():
+    """Zeroing the gate at one (token, head, channel) zeroes exactly that output
+    element; other outputs and the final state are untouched, so the gate is
+    outside the recurrence and indexed like the output (d_k != d_v)."""
+    x = _case(50, 3, 8, 6, seed=41)
+    g = np.ones_like(x.v)
+    g[0, 17, 2, 4] = 0.0
+    o, s = oracle.recurrent(x.q, x.k, x.v, x.log_alpha, x.beta, x.initial_state)
+    og, sg = oracle.recurrent(x.q, x.k, x.v, x.log_alpha, x.beta, x.initial_state, out_gate=g)
+    assert og[0, 17, 2, 4] == 0.0 and o[0, 17, 2, 4] != 0.0
+    mask = np.ones(o.shape, bool)
+    mask[0, 17, 2, 4] = False
+    np.testing.assert_array_equal(og[mask], o[mask])
+    np.testing.assert_array_equal(sg, s)
+
+
+def test_gate_scales_each_output_exactly():
+    """A power-of-two gate scales the output exactly; random gates act as the
+    elementwise product (chunked form as well)."""
+    x = _case(90, 2, 8, 6, seed=42)
+    o, _ = oracle.recurrent(x.q, x.k, x.v, x.log_alpha, x.beta, x.initial_state)
+    og, _ = oracle.recurrent(x.q, x.k, x.v, x.log_alpha, x.beta, x.initial_state,
+                             out_gate=np.full_like(x.v, 0.25))
+    np.testing.assert_array_equal(og, 0.25 * o)
+    g = RNG.uniform(0, 1, x.v.shape).astype(np.float32)
+    oc, _ = oracle.chunked(x.q, x.k, x.v, x.log_alpha, x.beta, x.initial_state, chunk=16,
+                           out_gate=g)
+    assert _rel(oc, o * g.astype(np.float64)) < 1e-12
+
+
+def test_gate_bf16_bits_match_widened_fp32():
+    x = make_inputs(1, 40, 2, 8, 8, bf16=True, seed=43)
+    g = f32_to_bf16(RNG.uniform(0, 1, (1, 40, 2, 8)).astype(np.float32))
+    o1, _ = oracle.recurrent(x.q, x.k, x.v, x.log_alpha, x.beta, out_gate=g)
+    o2, _ = oracle.recurrent(x.q, x.k, x.v, x.log_alpha, x.beta, out_gate=bf16_to_f32(g))
+    np.testing.assert_array_equal(o1, o2)
