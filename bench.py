@@ -354,6 +354,12 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer measurement")
+    ap.add_argument("--out-gate", action="store_true",
+                    help="fuse an output gate (random values in (0, 1), dtype of q) into the "
+                         "step (kda_fwd_ex / kda_decode)")
+    ap.add_argument("--snap-interval", type=int, default=0,
+                    help="forward workloads: also write a prefix-cache state snapshot every "
+                         "this many tokens (kda_fwd_snap), each to its own pool row")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -406,14 +412,39 @@ def main():
     stream.synchronize()
 
     decode = is_decode(args.workload)
+    snap = None
+    if args.snap_interval and not decode:
+        lens = [int(x) for x in inp.seq_lens]
+        max_snaps = max(1, max(lens) // args.snap_interval)
+        n_snaps = sum(L // args.snap_interval for L in lens)
+        with torch.cuda.stream(stream):
+            slots = torch.arange(inp.n_seqs * max_snaps, dtype=torch.int32,
+                                 device=dev).reshape(inp.n_seqs, max_snaps)
+            pool = torch.empty((inp.n_seqs * max_snaps, inp.H, inp.dk, inp.dv),
+                               dtype=torch.float32, device=dev)
+        snap = {"slots": slots, "pool": pool, "count": n_snaps}
+        alg_bytes += n_snaps * inp.H * inp.dk * inp.dv * 4
+
+    gate = None
+    if args.out_gate:
+        with torch.cuda.stream(stream):
+            g = torch.Generator(device=dev)
+            g.manual_seed(1000 + rank)
+            gate = torch.rand(v_shape, generator=g, device=dev).to(d["q"].dtype)
+        alg_bytes += gate.numel() * gate.element_size()
 
     def step():
         if decode:  # the state is updated in place, step after step
             kda.kda_decode(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"],
-                           d["initial_state"], out=out, stream=stream)
+                           d["initial_state"], out=out, stream=stream, out_gate=gate)
+        elif snap is not None:
+            kda.kda_fwd_snap(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"],
+                             d["initial_state"], cu_dev, snap_interval=args.snap_interval,
+                             snap_slots=snap["slots"], snap_pool=snap["pool"], out=out,
+                             final_state=fs, stream=stream, out_gate=gate)
         else:
             kda.kda_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["initial_state"],
-                        cu_dev, 64, out, fs, stream=stream)
+                        cu_dev, 64, out, fs, stream=stream, out_gate=gate)
         return kda.last_launch_count()
 
     for _ in range(args.warmup):
@@ -449,7 +480,7 @@ def main():
     # e2e: host buffers through kda_fwd_host, copies inside every step
     nbytes = lambda t: 0 if t is None else t.numel() * t.element_size()
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and snap is None and gate is None:
         out_h = torch.empty(v_shape, dtype=host["q"].dtype).pin_memory()
         fs_h = torch.empty((inp.n_seqs, inp.H, inp.dk, inp.dv), dtype=torch.float32).pin_memory()
         cu_arg = None if cu_host is None else np.ascontiguousarray(cu_host, dtype=np.int32)
@@ -497,6 +528,13 @@ def main():
         return
 
     peaks, peak_src = load_peaks()
+    cfg = decode_config(inp, world) if decode else workload_config(inp, world)
+    if gate is not None:
+        cfg["out_gate"] = "fused output gate, %s, shape of out" % str(gate.dtype).split(".")[-1]
+    if snap is not None:
+        cfg["snapshots"] = {"interval_tokens": args.snap_interval, "count": snap["count"],
+                            "bytes": snap["count"] * inp.H * inp.dk * inp.dv * 4,
+                            "entry": "kda_fwd_snap"}
     kernels = {name: {"ms_per_launch": tot / n, "launches": n, "share": tot / (ms * args.steps)}
                for name, (tot, n) in per_kernel.items()}
     dom = max(kernels, key=lambda k_: kernels[k_]["ms_per_launch"] * kernels[k_]["launches"])
@@ -509,7 +547,7 @@ def main():
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32" if kda.last_path() in ("ffma", "decode") else "bf16",
         "data": "synthetic",
-        "config": decode_config(inp, world) if decode else workload_config(inp, world),
+        "config": cfg,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
                      "traffic": recorded_traffic(dom),

@@ -17,7 +17,7 @@ from __future__ import annotations
 import ctypes
 import os
 
-__all__ = ["kda_fwd", "kda_fwd_host", "kda_fwd_noalloc", "kda_decode", "KDAError", "library_path", "load_library",
+__all__ = ["kda_fwd", "kda_fwd_host", "kda_fwd_noalloc", "kda_fwd_snap", "kda_decode", "KDAError", "library_path", "load_library",
            "last_launch_count", "last_path", "check_device", "profile_enable", "profile_read",
            "STATUS"]
 
@@ -43,6 +43,16 @@ class Dims(ctypes.Structure):
                 ("qkv_dtype", ctypes.c_int32)]
 
 
+class SnapSpec(ctypes.Structure):
+    _fields_ = [("interval", ctypes.c_int32), ("max_snaps", ctypes.c_int32),
+                ("num_slots", ctypes.c_int32)]
+
+
+class FwdOpts(ctypes.Structure):
+    _fields_ = [("out_gate", ctypes.c_void_p), ("snap", ctypes.POINTER(SnapSpec)),
+                ("snap_slots", ctypes.c_void_p), ("snap_pool", ctypes.c_void_p)]
+
+
 class DecodeDims(ctypes.Structure):
     _fields_ = [("N", ctypes.c_int32), ("T", ctypes.c_int32), ("H", ctypes.c_int32),
                 ("d_k", ctypes.c_int32), ("d_v", ctypes.c_int32), ("num_slots", ctypes.c_int32),
@@ -66,7 +76,11 @@ def load_library():
             fn = getattr(lib, name)
             fn.argtypes = sig
             fn.restype = ctypes.c_int
-        lib.kda_decode.argtypes = [p, p, p, p, p, p, p, p, p, ctypes.POINTER(DecodeDims), p]
+        lib.kda_fwd_snap.argtypes = sig[:-1] + [ctypes.POINTER(SnapSpec), p, p, p]
+        lib.kda_fwd_snap.restype = ctypes.c_int
+        lib.kda_fwd_ex.argtypes = sig[:-1] + [ctypes.POINTER(FwdOpts), p]
+        lib.kda_fwd_ex.restype = ctypes.c_int
+        lib.kda_decode.argtypes = [p, p, p, p, p, p, p, p, p, p, ctypes.POINTER(DecodeDims), p]
         lib.kda_decode.restype = ctypes.c_int
         lib.kda_status_string.argtypes = [ctypes.c_int]
         lib.kda_status_string.restype = ctypes.c_char_p
@@ -138,12 +152,13 @@ def _dims(q_shape, v_shape, T_override, cu_len, bf16):
 
 def kda_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, chunk: int = 64,
             out=None, final_state=None, stream=None, want_final: bool = True,
-            _entry: str = "kda_fwd"):
+            out_gate=None, _entry: str = "kda_fwd", _snap=None):
     """KDA forward on CUDA tensors; returns (out, final_state or None).
 
     q/k/v are bf16 or fp32 CUDA tensors; gates and states fp32.  ``stream`` is a
     torch.cuda.Stream (default: the current stream).  Outputs are allocated when
-    not given.  Runs asynchronously on the stream.
+    not given.  Runs asynchronously on the stream.  ``out_gate`` (same shape and
+    dtype as out) multiplies the output before it is stored (kda_fwd_ex).
     """
     import torch
 
@@ -164,12 +179,52 @@ def kda_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, chunk
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
     ptr = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
-    rc = getattr(lib, _entry)(ptr(q), ptr(k), ptr(v), ptr(log_alpha), ptr(beta),
-                              ptr(initial_state), ptr(cu_seqlens), int(chunk), ptr(out),
-                              ptr(final_state), ctypes.byref(d),
-                              ctypes.c_void_p(stream.cuda_stream))
+    args = (ptr(q), ptr(k), ptr(v), ptr(log_alpha), ptr(beta), ptr(initial_state),
+            ptr(cu_seqlens), int(chunk), ptr(out), ptr(final_state), ctypes.byref(d))
+    if out_gate is not None or _snap is not None:
+        if _entry != "kda_fwd":
+            raise ValueError(f"{_entry} takes no output gate or snapshots")
+        if out_gate is not None:
+            if not out_gate.is_cuda or not out_gate.is_contiguous() or out_gate.dtype != q.dtype \
+                    or tuple(out_gate.shape) != tuple(out.shape):
+                raise ValueError("out_gate must be a contiguous CUDA tensor shaped and typed as out")
+        opts = FwdOpts(None if out_gate is None else out_gate.data_ptr(), None, None, None)
+        if _snap is not None:
+            spec, slots, pool = _snap
+            opts.snap = ctypes.pointer(spec)
+            opts.snap_slots = slots.data_ptr()
+            opts.snap_pool = pool.data_ptr()
+        rc = lib.kda_fwd_ex(*args, ctypes.byref(opts), ctypes.c_void_p(stream.cuda_stream))
+    else:
+        rc = getattr(lib, _entry)(*args, ctypes.c_void_p(stream.cuda_stream))
     _check(rc)
     return out, final_state
+
+
+def kda_fwd_snap(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, *,
+                 snap_interval: int, snap_slots, snap_pool, chunk: int = 64, out=None,
+                 final_state=None, stream=None, want_final: bool = True, out_gate=None):
+    """kda_fwd that also writes prefix-cache state snapshots.
+
+    Snapshot j of sequence n -- the state after its first (j+1)*snap_interval
+    tokens (snap_interval a multiple of 64) -- goes to row snap_slots[n, j] of
+    ``snap_pool`` [num_slots,H,d_k,d_v] fp32 when that entry is >= 0.
+    ``snap_slots`` is an int32 CUDA tensor [N, max_snaps].  Returns (out,
+    final_state or None); the pool is written in place.
+    """
+    import torch
+
+    for t in (snap_slots, snap_pool):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("snap_slots and snap_pool must be contiguous CUDA tensors")
+    if snap_slots.dtype != torch.int32 or snap_slots.dim() != 2:
+        raise ValueError("snap_slots must be an int32 [N, max_snaps] tensor")
+    n_seqs = (cu_seqlens.numel() - 1) if cu_seqlens is not None else q.shape[0]
+    if snap_slots.shape[0] != n_seqs:
+        raise ValueError(f"snap_slots has {snap_slots.shape[0]} rows for {n_seqs} sequences")
+    spec = SnapSpec(int(snap_interval), snap_slots.shape[1], snap_pool.shape[0])
+    return kda_fwd(q, k, v, log_alpha, beta, initial_state, cu_seqlens, chunk, out, final_state,
+                   stream, want_final, out_gate=out_gate, _snap=(spec, snap_slots, snap_pool))
 
 
 def kda_fwd_noalloc(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
@@ -235,7 +290,7 @@ def kda_fwd_host(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
 
 
 def kda_decode(q, k, v, log_alpha, beta, state, slots=None, out=None, token_states=None,
-               want_token_states: bool = False, stream=None):
+               want_token_states: bool = False, stream=None, out_gate=None):
     """Decode / multi-token verify step: T new tokens per sequence on a resident
     state, which is updated IN PLACE.  Returns (out, token_states or None).
 
@@ -243,7 +298,8 @@ def kda_decode(q, k, v, log_alpha, beta, state, slots=None, out=None, token_stat
     beta [N,T,H] fp32; state [S,H,d_k,d_v] fp32 where S = N, or the pool size
     when ``slots`` (int32 [N] on the device; -1 = padding entry) maps sequences
     to pool rows.  ``token_states`` [N,T,H,d_k,d_v] receives the state after
-    every token (allocated here when ``want_token_states``).
+    every token (allocated here when ``want_token_states``).  ``out_gate``
+    [N,T,H,d_v] (dtype of q) multiplies the output before it is stored.
     """
     import torch
 
@@ -267,8 +323,12 @@ def kda_decode(q, k, v, log_alpha, beta, state, slots=None, out=None, token_stat
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
     ptr = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
+    if out_gate is not None and (not out_gate.is_cuda or not out_gate.is_contiguous()
+                                 or out_gate.dtype != q.dtype
+                                 or tuple(out_gate.shape) != tuple(out.shape)):
+        raise ValueError("out_gate must be a contiguous CUDA tensor shaped and typed as out")
     rc = lib.kda_decode(ptr(q), ptr(k), ptr(v), ptr(log_alpha), ptr(beta), ptr(state), ptr(slots),
-                        ptr(out), ptr(token_states), ctypes.byref(d),
+                        ptr(out), ptr(out_gate), ptr(token_states), ctypes.byref(d),
                         ctypes.c_void_p(stream.cuda_stream))
     _check(rc)
     return out, token_states

@@ -55,6 +55,13 @@ bool device_accessible(const void* p) {
            (at.type == cudaMemoryTypeHost && at.devicePointer != nullptr);
 }
 
+kda_status check_accessible(const void* const* ptrs, const char* const* names, int n) {
+    for (int i = 0; i < n; ++i)
+        if (ptrs[i] && !device_accessible(ptrs[i]))
+            return fail(KDA_ERR_INVALID_ARG, "%s is not device-accessible memory", names[i]);
+    return KDA_OK;
+}
+
 kda_status validate(const void* q, const void* k, const void* v, const float* la,
                     const float* beta, const float* s0, const int32_t* cu, int32_t chunk,
                     const void* out, const float* sf, const kda_dims* d, bool device_ptrs,
@@ -109,9 +116,8 @@ kda_status validate(const void* q, const void* k, const void* v, const float* la
     }
     if (overlaps(ro, rs)) return fail(KDA_ERR_ALIAS, "out overlaps final_state");
     if (device_ptrs) {
-        for (int i = 0; i < 9; ++i)
-            if (ptrs[i] && !device_accessible(ptrs[i]))
-                return fail(KDA_ERR_INVALID_ARG, "%s is not device-accessible memory", names[i]);
+        kda_status st = check_accessible(ptrs, names, 9);
+        if (st != KDA_OK) return st;
     }
     a->q = q;
     a->k = k;
@@ -219,6 +225,12 @@ kda_status run_tc(const kda::FwdArgs& a, cudaStream_t stream, int* launches) {
     t.cu = a.cu;
     t.out = a.out;
     t.s_final = a.s_final;
+    t.gate = a.gate;
+    t.snap_slots = a.snap_slots;
+    t.snap_pool = a.snap_pool;
+    t.snap_interval = a.snap_interval;
+    t.snap_max = a.snap_max;
+    t.snap_num_slots = a.snap_num_slots;
     t.B = a.B;
     t.T = a.T;
     t.H = a.H;
@@ -351,6 +363,108 @@ kda_status kda_fwd(const void* q, const void* k, const void* v, const float* log
     return run(a, (cudaStream_t)stream);
 }
 
+kda_status kda_fwd_ex(const void* q, const void* k, const void* v, const float* log_alpha,
+                      const float* beta, const float* initial_state, const int32_t* cu_seqlens,
+                      int32_t chunk, void* out, float* final_state, const kda_dims* dims,
+                      const kda_fwd_opts* opts, void* stream) {
+    g_last_error[0] = 0;
+    g_last_launches = 0;
+    g_last_path = "";
+    kda::FwdArgs a;
+    // argument checks first, then (as in kda_fwd) whether the pointers are device memory
+    kda_status s = validate(q, k, v, log_alpha, beta, initial_state, cu_seqlens, chunk, out,
+                            final_state, dims, false, &a);
+    if (s != KDA_OK) return s;
+    const kda_fwd_opts none = {nullptr, nullptr, nullptr, nullptr};
+    if (!opts) opts = &none;
+    const kda_snap_spec* snap = opts->snap;
+    if (snap) {
+        if (snap->interval <= 0 || snap->interval % kda::kChunk)
+            return fail(KDA_ERR_INVALID_ARG, "snapshot interval must be a positive multiple of %d "
+                        "(got %d)", kda::kChunk, snap->interval);
+        if (snap->max_snaps < 0 || snap->num_slots < 0)
+            return fail(KDA_ERR_INVALID_ARG, "max_snaps and num_slots must be >= 0");
+        if (snap->max_snaps == 0 || snap->num_slots == 0) snap = nullptr;  // nothing requested
+    }
+    const void* gate = opts->out_gate;
+    const int32_t* snap_slots = snap ? opts->snap_slots : nullptr;
+    float* snap_pool = snap ? opts->snap_pool : nullptr;
+    if (snap && (!snap_slots || !snap_pool))
+        return fail(KDA_ERR_INVALID_ARG, "snap_slots and snap_pool must be non-NULL");
+    if (gate && ((uintptr_t)gate & 15u)) return fail(KDA_ERR_MISALIGNED, "out_gate is not 16-byte aligned");
+    if (snap_slots && ((uintptr_t)snap_slots & 3u))
+        return fail(KDA_ERR_MISALIGNED, "snap_slots is not 4-byte aligned");
+    if (snap_pool && ((uintptr_t)snap_pool & 15u))
+        return fail(KDA_ERR_MISALIGNED, "snap_pool is not 16-byte aligned");
+    const int64_t tokens = (int64_t)a.B * a.T, e_in = a.bf16 ? 2 : 4;
+    const int64_t dd = (int64_t)a.dk * a.dv, nst = (int64_t)a.N * a.H * dd * 4;
+    const Range r_gate = {(uintptr_t)gate, (uintptr_t)gate + (gate ? tokens * a.H * a.dv * e_in : 0),
+                          "out_gate"};
+    const Range r_pool = {(uintptr_t)snap_pool,
+                          (uintptr_t)snap_pool + (snap_pool ? (uintptr_t)snap->num_slots * a.H * dd * 4 : 0),
+                          "snap_pool"};
+    const Range r_slots = {(uintptr_t)snap_slots,
+                           (uintptr_t)snap_slots + (snap_slots ? (uintptr_t)a.N * snap->max_snaps * 4 : 0),
+                           "snap_slots"};
+    const Range r_out = {(uintptr_t)out, (uintptr_t)out + (out ? tokens * a.H * a.dv * e_in : 0), "out"};
+    const Range r_fin = {(uintptr_t)final_state, (uintptr_t)final_state + (final_state ? nst : 0),
+                         "final_state"};
+    const Range inputs[] = {
+        {(uintptr_t)q, (uintptr_t)q + (q ? tokens * a.H * a.dk * e_in : 0), "q"},
+        {(uintptr_t)k, (uintptr_t)k + (k ? tokens * a.H * a.dk * e_in : 0), "k"},
+        {(uintptr_t)v, (uintptr_t)v + (v ? tokens * a.H * a.dv * e_in : 0), "v"},
+        {(uintptr_t)log_alpha, (uintptr_t)log_alpha + (log_alpha ? tokens * a.H * a.dk * 4 : 0),
+         "log_alpha"},
+        {(uintptr_t)beta, (uintptr_t)beta + (beta ? tokens * a.H * 4 : 0), "beta"},
+        {(uintptr_t)initial_state, (uintptr_t)initial_state + (initial_state ? nst : 0),
+         "initial_state"},
+        {(uintptr_t)cu_seqlens, (uintptr_t)cu_seqlens + (cu_seqlens ? (a.N + 1) * 4 : 0),
+         "cu_seqlens"},
+        r_gate, r_slots,
+    };
+    // the written buffers (out, final_state: checked by validate; snap_pool) overlap no input
+    for (const Range& r : inputs) {
+        if (overlaps(r_pool, r)) return fail(KDA_ERR_ALIAS, "snap_pool overlaps %s", r.name);
+        if (&r >= &inputs[7] && (overlaps(r_out, r) || overlaps(r_fin, r)))
+            return fail(KDA_ERR_ALIAS, "%s overlaps an output", r.name);
+    }
+    if (overlaps(r_pool, r_out) || overlaps(r_pool, r_fin))
+        return fail(KDA_ERR_ALIAS, "snap_pool overlaps an output");
+    const void* ptrs[] = {q, k, v, log_alpha, beta, initial_state, cu_seqlens, out, final_state,
+                          gate, snap_slots, snap_pool};
+    const char* names[] = {"q", "k", "v", "log_alpha", "beta", "initial_state", "cu_seqlens",
+                           "out", "final_state", "out_gate", "snap_slots", "snap_pool"};
+    s = check_accessible(ptrs, names, 12);
+    if (s != KDA_OK) return s;
+    a.gate = gate;
+    if (snap) {
+        a.snap_slots = snap_slots;
+        a.snap_pool = snap_pool;
+        a.snap_interval = snap->interval;
+        a.snap_max = snap->max_snaps;
+        a.snap_num_slots = snap->num_slots;
+        cudaError_t e = kda::status_word(&a.status);
+        if (e != cudaSuccess) return cuda_fail(e, "device status word");
+    }
+    return run(a, (cudaStream_t)stream);
+}
+
+kda_status kda_fwd_snap(const void* q, const void* k, const void* v, const float* log_alpha,
+                        const float* beta, const float* initial_state,
+                        const int32_t* cu_seqlens, int32_t chunk, void* out, float* final_state,
+                        const kda_dims* dims, const kda_snap_spec* snap,
+                        const int32_t* snap_slots, float* snap_pool, void* stream) {
+    if (!snap) {
+        g_last_error[0] = 0;
+        g_last_launches = 0;
+        g_last_path = "";
+        return fail(KDA_ERR_INVALID_ARG, "snap is NULL");
+    }
+    const kda_fwd_opts o = {nullptr, snap, snap_slots, snap_pool};
+    return kda_fwd_ex(q, k, v, log_alpha, beta, initial_state, cu_seqlens, chunk, out, final_state,
+                      dims, &o, stream);
+}
+
 kda_status kda_fwd_host(const void* q, const void* k, const void* v, const float* log_alpha,
                         const float* beta, const float* initial_state,
                         const int32_t* cu_seqlens, int32_t chunk, void* out,
@@ -470,6 +584,12 @@ kda_status kda_fwd_noalloc(const void* q, const void* k, const void* v, const fl
     t.cu = a.cu;
     t.out = a.out;
     t.s_final = a.s_final;
+    t.gate = a.gate;
+    t.snap_slots = a.snap_slots;
+    t.snap_pool = a.snap_pool;
+    t.snap_interval = a.snap_interval;
+    t.snap_max = a.snap_max;
+    t.snap_num_slots = a.snap_num_slots;
     t.B = a.B;
     t.T = a.T;
     t.H = a.H;
@@ -488,7 +608,8 @@ kda_status kda_fwd_noalloc(const void* q, const void* k, const void* v, const fl
 
 kda_status kda_decode(const void* q, const void* k, const void* v, const float* log_alpha,
                       const float* beta, float* state, const int32_t* slots, void* out,
-                      float* token_states, const kda_decode_dims* d, void* stream) {
+                      const void* out_gate, float* token_states, const kda_decode_dims* d,
+                      void* stream) {
     g_last_error[0] = 0;
     g_last_launches = 0;
     g_last_path = "";
@@ -515,10 +636,10 @@ kda_status kda_decode(const void* q, const void* k, const void* v, const float* 
     if (!state) return fail(KDA_ERR_INVALID_ARG, "state must be non-NULL");
     if (tokens > 0 && (!q || !k || !v || !log_alpha || !beta || !out))
         return fail(KDA_ERR_INVALID_ARG, "q, k, v, log_alpha, beta and out must be non-NULL");
-    const void* ptrs[] = {q, k, v, log_alpha, beta, state, slots, out, token_states};
+    const void* ptrs[] = {q, k, v, log_alpha, beta, state, slots, out, token_states, out_gate};
     const char* names[] = {"q", "k", "v", "log_alpha", "beta", "state", "slots", "out",
-                           "token_states"};
-    for (int i = 0; i < 9; ++i) {
+                           "token_states", "out_gate"};
+    for (int i = 0; i < 10; ++i) {
         if (ptrs[i] && ((uintptr_t)ptrs[i] & 15u) && i != 6)
             return fail(KDA_ERR_MISALIGNED, "%s is not 16-byte aligned", names[i]);
         if (i == 6 && ptrs[i] && ((uintptr_t)ptrs[i] & 3u))
@@ -526,18 +647,17 @@ kda_status kda_decode(const void* q, const void* k, const void* v, const float* 
     }
     const int64_t bytes[] = {nqk * e_in, nqk * e_in, nv * e_in, nqk * 4, tokens * d->H * 4,
                              S * d->H * dd * 4, (int64_t)d->N * 4, nv * e_in,
-                             tokens * d->H * dd * 4};
-    Range r[9];
-    for (int i = 0; i < 9; ++i)
+                             tokens * d->H * dd * 4, nv * e_in};
+    Range r[10];
+    for (int i = 0; i < 10; ++i)
         r[i] = {(uintptr_t)ptrs[i], (uintptr_t)ptrs[i] + (ptrs[i] ? bytes[i] : 0), names[i]};
     // written buffers (state, out, token_states) overlap nothing else
     for (int w : {5, 7, 8})
-        for (int i = 0; i < 9; ++i)
+        for (int i = 0; i < 10; ++i)
             if (i != w && overlaps(r[w], r[i]))
                 return fail(KDA_ERR_ALIAS, "%s overlaps %s", names[w], names[i]);
-    for (int i = 0; i < 9; ++i)
-        if (ptrs[i] && !device_accessible(ptrs[i]))
-            return fail(KDA_ERR_INVALID_ARG, "%s is not device-accessible memory", names[i]);
+    kda_status st = check_accessible(ptrs, names, 10);
+    if (st != KDA_OK) return st;
     kda::DecodeArgs a;
     a.q = q;
     a.k = k;
@@ -547,6 +667,7 @@ kda_status kda_decode(const void* q, const void* k, const void* v, const float* 
     a.state = state;
     a.slots = slots;
     a.out = out;
+    a.gate = out_gate;
     a.token_states = token_states;
     a.N = d->N;
     a.T = d->T;

@@ -17,9 +17,10 @@
 // state as one contiguous block.  Per token, each thread reads its rows'
 // (alpha, k, q) as broadcast float4s from shared memory; the two reductions
 // over d_k (S^T k and S^T q) combine per-row-group partial sums through shared
-// memory.  The token inputs arrive by cp.async, 4 tokens per block and two
-// blocks in flight, issued before the state loads so that both latencies
-// overlap.
+// memory.  An optional output gate (precomputed by the caller) multiplies o
+// before it is stored.  The token inputs arrive by cp.async, 4 tokens per
+// block (2 for fp32 inputs) and two blocks in flight, issued before the state
+// loads so that both latencies overlap.
 // Optionally the state after every token is written out (a verifier that
 // accepts only a prefix of the drafted tokens rolls back to one of them), and
 // sequences may address their state through a slot table into a state pool.
@@ -61,24 +62,26 @@ __device__ __forceinline__ float raw_x(const unsigned char* p, int i) {
         return reinterpret_cast<const float*>(p)[i];
 }
 
-template <int DK, int DV>
+template <bool BF16, int DK, int DV>
 struct DecodeShape {
-    static constexpr int CW = DV / 4;            // lanes across one state row (4 columns each)
-    static constexpr int RGS = DK / 8;           // row groups of 8 rows
-    static constexpr int NTH = RGS * CW;         // threads: d_k * d_v / 32
-    static constexpr int TB = 4;                 // tokens per staged block
+    static constexpr int CW = DV / 4;     // lanes across one state row (4 columns each)
+    static constexpr int RGS = DK / 8;    // row groups of 8 rows
+    static constexpr int NTH = RGS * CW;  // threads: d_k * d_v / 32
+    static constexpr int TB = BF16 ? 4 : 2;  // tokens per staged block (static shared memory)
 };
 
 template <bool BF16, int DK, int DV>
-__global__ void __launch_bounds__(DecodeShape<DK, DV>::NTH, 1024 / DecodeShape<DK, DV>::NTH)
+__global__ void __launch_bounds__(DecodeShape<BF16, DK, DV>::NTH,
+                                  1024 / DecodeShape<BF16, DK, DV>::NTH)
     decode_kernel(DecodeArgs a) {
-    using Sh = DecodeShape<DK, DV>;
+    using Sh = DecodeShape<BF16, DK, DV>;
     constexpr int CW = Sh::CW, RGS = Sh::RGS, NTH = Sh::NTH, TB = Sh::TB;
     constexpr int ES = BF16 ? 2 : 4;  // bytes per q/k/v element
-    // raw bytes of one token as it arrives: k | q | v | log_alpha, in 16-byte chunks
+    // raw bytes of one token as it arrives: k | q | v | log_alpha [| gate], in
+    // 16-byte chunks
     constexpr int CK = DK * ES / 16, CV = DV * ES / 16, CL = DK * 4 / 16;
     constexpr int CH = 2 * CK + CV + CL;
-    constexpr int RAWB = CH * 16;
+    constexpr int RAWB = (CH + CV) * 16;
     // Raw token blocks arrive by cp.async, two blocks in flight; each block is
     // then widened to fp32: tok[t][r] = {alpha_r, k_r, q_r, 0} with
     // alpha = exp(clamp(log_alpha)), read by a warp as one broadcast float4.
@@ -86,6 +89,7 @@ __global__ void __launch_bounds__(DecodeShape<DK, DV>::NTH, 1024 / DecodeShape<D
     __shared__ float raw_beta[2][TB];
     __shared__ __align__(16) float4 tok[TB][DK];
     __shared__ float vs[TB][DV];
+    __shared__ float gs[TB][DV];  // output gate (when given)
     __shared__ float bs[TB];
     __shared__ __align__(16) float red[2][RGS][DV];  // per-row-group partial sums
     __shared__ __align__(16) float us[DV];          // u = beta (v - S^T k) of the token
@@ -102,11 +106,12 @@ __global__ void __launch_bounds__(DecodeShape<DK, DV>::NTH, 1024 / DecodeShape<D
         }
     }
     const int nblk = (T + TB - 1) / TB;
+    const int ch = CH + (a.gate ? CV : 0);  // chunks per token
     // issue the raw copies of token block b into buffer b & 1 (one commit group)
     auto issue = [&](int b) {
         const int t0 = b * TB, nt = min(TB, T - t0);
-        for (int x = tid; x < nt * CH; x += NTH) {
-            const int t = x / CH, c = x - t * CH;
+        for (int x = tid; x < nt * ch; x += NTH) {
+            const int t = x / ch, c = x - t * ch;
             const int64_t row = ((int64_t)n * T + t0 + t) * H + h;
             const unsigned char* src;
             if (c < CK)
@@ -115,8 +120,10 @@ __global__ void __launch_bounds__(DecodeShape<DK, DV>::NTH, 1024 / DecodeShape<D
                 src = (const unsigned char*)a.q + (row * DK) * ES + (c - CK) * 16;
             else if (c < 2 * CK + CV)
                 src = (const unsigned char*)a.v + (row * DV) * ES + (c - 2 * CK) * 16;
-            else
+            else if (c < CH)
                 src = (const unsigned char*)(a.log_alpha + row * DK) + (c - 2 * CK - CV) * 16;
+            else
+                src = (const unsigned char*)a.gate + (row * DV) * ES + (c - CH) * 16;
             cp_async16(&raw[b & 1][t][c * 16], src);
         }
         if (tid < nt) cp_async4(&raw_beta[b & 1][tid], a.beta + ((int64_t)n * T + t0 + tid) * H + h);
@@ -136,15 +143,18 @@ __global__ void __launch_bounds__(DecodeShape<DK, DV>::NTH, 1024 / DecodeShape<D
         const int t0 = b * TB, nt = min(TB, T - t0), buf = b & 1;
         cp_async_wait_1();  // block b has landed (block b+1 may still be in flight)
         __syncthreads();
-        for (int x = tid; x < nt * (DK + DV); x += NTH) {
-            const int t = x / (DK + DV), e = x - t * (DK + DV);
+        const int per_tok = DK + (a.gate ? 2 : 1) * DV;
+        for (int x = tid; x < nt * per_tok; x += NTH) {
+            const int t = x / per_tok, e = x - t * per_tok;
             const unsigned char* r = raw[buf][t];
             if (e < DK) {
                 const float la = reinterpret_cast<const float*>(r + (2 * CK + CV) * 16)[e];
                 tok[t][e] = make_float4(expf(fminf(fmaxf(la, -5.f), 0.f)), raw_x<BF16>(r, e),
                                         raw_x<BF16>(r + CK * 16, e), 0.f);
-            } else {
+            } else if (e < DK + DV) {
                 vs[t][e - DK] = raw_x<BF16>(r + 2 * CK * 16, e - DK);
+            } else {
+                gs[t][e - DK - DV] = raw_x<BF16>(r + CH * 16, e - DK - DV);
             }
         }
         if (tid < nt) bs[tid] = raw_beta[buf][tid];
@@ -203,7 +213,9 @@ __global__ void __launch_bounds__(DecodeShape<DK, DV>::NTH, 1024 / DecodeShape<D
                 float acc = 0.f;
 #pragma unroll
                 for (int g = 0; g < RGS; ++g) acc += red[1][g][tid];
-                st_x<BF16>(a.out, (((int64_t)n * T + t0 + t) * H + h) * DV + tid, acc);
+                const int64_t oi = (((int64_t)n * T + t0 + t) * H + h) * DV + tid;
+                if (a.gate) acc *= gs[t][tid];  // output gate
+                st_x<BF16>(a.out, oi, acc);
             }
             // red[1] is next written after the next token's first barrier, red[0]
             // and us after its second: no barrier needed here
@@ -216,7 +228,8 @@ __global__ void __launch_bounds__(DecodeShape<DK, DV>::NTH, 1024 / DecodeShape<D
 template <bool BF16, int DK, int DV>
 cudaError_t launch_t(const DecodeArgs& a, cudaStream_t stream) {
     profile_mark(SLOT_DECODE, true, stream);
-    decode_kernel<BF16, DK, DV><<<(unsigned)(a.N * a.H), DecodeShape<DK, DV>::NTH, 0, stream>>>(a);
+    decode_kernel<BF16, DK, DV>
+        <<<(unsigned)(a.N * a.H), DecodeShape<BF16, DK, DV>::NTH, 0, stream>>>(a);
     profile_mark(SLOT_DECODE, false, stream);
     return cudaGetLastError();
 }

@@ -226,7 +226,9 @@ __device__ __forceinline__ void chunk_step(const FwdArgs& a, float* sm, int64_t 
         float acc = 0.f;
         for (int c = 0; c < DK; ++c) acc = fmaf(Qt[r * KS + c], S[c * DVB + e], acc);
         for (int j = 0; j <= r; ++j) acc = fmaf(P[r * AS + j], X[j * XS + DK + e], acc);
-        st_out<BF16>(a.out, ((t0 + r) * H + h) * (int64_t)DV + dv0 + e, acc);
+        const int64_t oi = ((t0 + r) * H + h) * (int64_t)DV + dv0 + e;
+        if (a.gate) acc *= ld_in<BF16>(a.gate, oi);  // output gate
+        st_out<BF16>(a.out, oi, acc);
     }
     __syncthreads();
 
@@ -268,6 +270,19 @@ __global__ void __launch_bounds__(NT, 1) kda_ffma_kernel(FwdArgs a) {
     for (int64_t t0 = lo; t0 < hi; t0 += C) {
         const int Lc = (int)(hi - t0 < C ? hi - t0 : C);
         chunk_step<BF16, DK>(a, sm, t0, Lc, h, dv0);
+        const int64_t pos = t0 + Lc - lo;  // tokens of the sequence done so far
+        if (a.snap_pool && pos % a.snap_interval == 0 && pos / a.snap_interval <= a.snap_max) {
+            const int slot = a.snap_slots[(int64_t)n * a.snap_max + pos / a.snap_interval - 1];
+            if (slot >= a.snap_num_slots) {
+                if (tid == 0) atomicCAS(a.status, 0, ERR_BAD_SLOT);
+            } else if (slot >= 0) {
+                float* sp = a.snap_pool + ((int64_t)slot * H + h) * DK * (int64_t)DV + dv0;
+                for (int i = tid; i < DK * DVB; i += NT) {
+                    const int c = i / DVB, e = i % DVB;
+                    sp[(int64_t)c * DV + e] = S[i];
+                }
+            }
+        }
     }
     if (a.s_final) {
         for (int i = tid; i < DK * DVB; i += NT) {

@@ -34,6 +34,14 @@ struct FwdArgs {
     float* s_final;          // [N,H,dk,dv] or nullptr
     int32_t B, T, H, dk, dv, N;
     int32_t bf16;            // q/k/v/out are bf16 (else fp32)
+    const void* gate = nullptr;  // optional output gate [B, T, H, dv] (dtype of out): out = o * gate
+    // optional state snapshots (kda_fwd_snap): snapshot j of sequence n, the
+    // state after its first (j+1)*snap_interval tokens, goes to pool row
+    // snap_slots[n*snap_max + j] when that entry is >= 0
+    const int32_t* snap_slots = nullptr;  // [N, snap_max] device
+    float* snap_pool = nullptr;           // [snap_num_slots, H, dk, dv]
+    int32_t snap_interval = 0, snap_max = 0, snap_num_slots = 0;
+    int* status = nullptr;                // device status word (set when snapshots are on)
 };
 
 // CUDA-core chunkwise path (exact fp32 arithmetic on fp32 or bf16 inputs).
@@ -66,12 +74,17 @@ struct TcArgs {
     int32_t* n_units;   // [1]
     float* trans;       // [max_units, H, 2, 128, 128]: B^T then M^T of each segment
     float* sin;         // [max_units, H, 128, 128]: S_in^T of each segment
+    const void* gate = nullptr;  // optional output gate, as in FwdArgs
+    // optional state snapshots, as in FwdArgs
+    const int32_t* snap_slots = nullptr;
+    float* snap_pool = nullptr;
+    int32_t snap_interval = 0, snap_max = 0, snap_num_slots = 0;
 };
 
-// TMA descriptors of the q, k, v, out (bf16) and log_alpha (fp32) tensors,
-// viewed as [T, H, 128]; passed as a grid constant.
+// TMA descriptors of the q, k, v, out, gate (bf16) and log_alpha (fp32)
+// tensors, viewed as [T, H, 128]; passed as a grid constant.
 struct TcMaps {
-    CUtensorMap q, k, v, la, out;
+    CUtensorMap q, k, v, la, out, gate;
 };
 
 struct TcPlan {
@@ -96,6 +109,7 @@ struct DecodeArgs {
     float* state;              // [num_slots, H, dk, dv], read and written in place
     const int32_t* slots;      // [N] state row of each sequence (-1 = skip), or nullptr
     void* out;                 // [N, T, H, dv]
+    const void* gate;          // [N, T, H, dv] output gate (dtype of out), or nullptr
     float* token_states;       // [N, T, H, dk, dv] or nullptr
     int* status;               // device status word
     int32_t N, T, H, dk, dv, num_slots;

@@ -93,8 +93,8 @@ struct LayT {
     static constexpr uint32_t EHB = EHA + 512;                    // fp32 [128] e^{rho_b}
     static constexpr uint32_t FAC = EHB + 512;                    // fp32 [5][128] gate factors
     static constexpr uint32_t BETA = FAC + 2560;                  // fp32 [64]
-    static constexpr uint32_t BAR = BETA + 256;                   // 2 mbarriers: MMA, TMA
-    static constexpr uint32_t TMEMP = BAR + 16;                   // TMEM base address
+    static constexpr uint32_t BAR = BETA + 256;                   // mbarriers: MMA, TMA, gate
+    static constexpr uint32_t TMEMP = BAR + 32;                   // TMEM base address
     static constexpr uint32_t END = TMEMP + 16;
     static constexpr uint32_t BYTES = END + 1024;                 // + alignment slack
 };
@@ -403,6 +403,10 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
     if (u >= *a.n_units) return;
     const SegEntry sg = a.segs[u];
     if (SEG && sg.last) return;  // transitions only for segments with a successor
+    const bool snap_on = !SEG && a.snap_pool != nullptr;
+    const bool gate_on = !SEG && a.gate != nullptr;
+    uint32_t gate_parity = 0;
+    const int64_t seq_lo = snap_on ? (a.cu ? (int64_t)a.cu[sg.n] : (int64_t)sg.n * a.T) : 0;
 
     float* gsum = reinterpret_cast<float*>(sm + Lay::GSUM);
     float* gam = reinterpret_cast<float*>(sm + Lay::GAM);
@@ -411,6 +415,7 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
     float* beta_s = reinterpret_cast<float*>(sm + Lay::BETA);
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + Lay::BAR);
     uint64_t* bar_raw = bar + 1;
+    uint64_t* bar_gate = bar + 2;  // output-gate tile (pass 3 with a gate)
     uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(sm + Lay::TMEMP);
 
     if (warp == 0) {
@@ -420,6 +425,7 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
     if (tid == 0) {
         mbar_init(bar, 1);
         mbar_init(bar_raw, 1);
+        mbar_init(bar_gate, 1);
         fence_mbar_init();
     }
     tc_fence_before();
@@ -702,6 +708,12 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
             tmem_st_wait();
         }
         if (!(ok = wait_mma(bar, parity))) break;
+        // The v tile is consumed: the output gate's [64][128] tile (if any) goes into
+        // its buffer now, for the epilogue.
+        if (gate_on && tid == 0) {
+            mbar_expect_tx(bar_gate, 16384);
+            tma_tile(sm + Lay::RV + vbuf * 16384, &maps.gate, 0, h, (int)t0, bar_gate);
+        }
         // W^T = e^{rho_a} Wa^T + e^{rho_b} Wb^T (lane = channel c) -> WB (MN-major B
         // operand: K rows = c, MN = token r)
         {
@@ -800,13 +812,21 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
         if (!SEG) {
             // O^T -> out.  A full chunk is staged as a [64][128] bf16 tile in this chunk's
             // v buffer (dead since phase 3) and written by one TMA store; a partial last
-            // chunk is stored from registers, row by row.
+            // chunk is stored from registers, row by row.  With an output gate, the
+            // buffer holds the gate tile, and each element is gated in place.
             const int r0 = 16 * wg;
             float v[16];
             tmem_ld16(tq + TM_O + r0, v);
             tmem_wait16(v);
+            __nv_bfloat16* os = reinterpret_cast<__nv_bfloat16*>(sm + Lay::RV + vbuf * 16384);
+            if (gate_on) {
+                if (!(ok = !__syncthreads_or(!mbar_wait(bar_gate, gate_parity, &g_tc_status,
+                                                        ERR_WAIT_TIMEOUT)))) break;
+                gate_parity ^= 1u;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[i] *= __bfloat162float(os[(r0 + i) * D + lrow]);
+            }
             if (Lc == C) {
-                __nv_bfloat16* os = reinterpret_cast<__nv_bfloat16*>(sm + Lay::RV + vbuf * 16384);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) os[(r0 + i) * D + lrow] = __float2bfloat16_rn(v[i]);
                 fence_async_smem();
@@ -820,6 +840,24 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
                     if (r0 + i < Lc) out[(t0 + r0 + i) * H * (int64_t)D] = __float2bfloat16_rn(v[i]);
+            }
+        }
+        if (!SEG && snap_on) {  // state snapshot at this chunk end, if one is requested
+            const int64_t pos = t0 + Lc - seq_lo;
+            if (pos % a.snap_interval == 0 && pos / a.snap_interval <= a.snap_max) {
+                const int slot = a.snap_slots[(int64_t)sg.n * a.snap_max + pos / a.snap_interval - 1];
+                if (slot >= a.snap_num_slots) {
+                    if (tid == 0) atomicCAS(&g_tc_status, 0, ERR_BAD_SLOT);
+                } else if (slot >= 0) {  // slice wg: columns 32wg..32wg+31 of S^T
+                    float* sp = a.snap_pool + ((int64_t)slot * H + h) * D * D;
+                    for (int c0 = 32 * wg; c0 < 32 * wg + 32; c0 += 16) {
+                        float v[16];
+                        tmem_ld16(tq + TM_S + c0, v);
+                        tmem_wait16(v);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) sp[(int64_t)(c0 + i) * D + lrow] = v[i];
+                    }
+                }
             }
         }
         tc_fence_before();
@@ -1091,7 +1129,9 @@ cudaError_t launch_tc(const TcArgs& a, const TcPlan& p, cudaStream_t stream, int
             (err = tile_map(&maps.k, a.k, false, a.H, tokens, false)) != cudaSuccess ||
             (err = tile_map(&maps.v, a.v, false, a.H, tokens, true)) != cudaSuccess ||
             (err = tile_map(&maps.la, a.log_alpha, true, a.H, tokens, false)) != cudaSuccess ||
-            (err = tile_map(&maps.out, a.out, false, a.H, tokens, false)) != cudaSuccess)
+            (err = tile_map(&maps.out, a.out, false, a.H, tokens, false)) != cudaSuccess ||
+            (err = tile_map(&maps.gate, a.gate ? a.gate : a.out, false, a.H, tokens, false)) !=
+                cudaSuccess)
             return err;
     }
     profile_mark(SLOT_SETUP, true, stream);

@@ -102,6 +102,79 @@ kda_status kda_fwd(const void* q, const void* k, const void* v, const float* log
                    int32_t chunk, void* out, float* final_state, const kda_dims* dims,
                    void* stream);
 
+/* Where kda_fwd_snap / kda_fwd_ex write state snapshots. */
+typedef struct {
+    int32_t interval;   /* tokens between snapshots: a positive multiple of 64 (chunk) */
+    int32_t max_snaps;  /* snapshots per sequence the slot table has room for (>= 0)  */
+    int32_t num_slots;  /* rows of the snapshot pool (>= 0)                           */
+} kda_snap_spec;
+
+/*
+ * kda_fwd_snap -- kda_fwd that also writes the state at chunk boundaries, for
+ * a prefix cache.
+ *
+ * KDA places new demands on prefix caching, and its authors released an
+ * implementation of it for a public serving engine (habr.com article 1063882
+ * on the Kimi K3 technical report, the paragraph on KDA and AttnRes).  A
+ * cached prefix of a linear-attention layer is a state, not a list of keys and
+ * values, so a request that shares a prefix resumes from the state at its end.
+ * This call writes such states while it runs the forward pass.
+ *
+ * Arguments and results of kda_fwd, plus:
+ *   snap        interval, max_snaps, num_slots (above)
+ *   snap_slots  [N, max_snaps] int32 on the device: snapshot j of sequence n,
+ *               the state after its first (j+1)*interval tokens (so only for
+ *               (j+1)*interval <= length of the sequence), is written to row
+ *               snap_slots[n*max_snaps + j] of snap_pool when that entry is
+ *               >= 0; entries < 0 request nothing.  An entry >= num_slots
+ *               skips that snapshot and sets the device status word
+ *               (kda_check_device: KDA_ERR_INVALID_ARG).  Two requested
+ *               snapshots must not name the same row.
+ *   snap_pool   [num_slots, H, d_k, d_v] fp32 on the device, 16-byte
+ *               aligned; rows not named are left as they were.  It may not
+ *               overlap any other buffer.
+ * A snapshot is the state after those tokens: the final_state kda_fwd
+ * returns for the sequence cut there (bit for bit when neither call splits
+ * the sequence into segments, else up to rounding), and kda_fwd continued
+ * from it reproduces the rest of the sequence.  Writing snapshots changes no
+ * other result.  max_snaps == 0 or num_slots == 0 is a plain kda_fwd.
+ * Temporary memory: as kda_fwd.
+ */
+kda_status kda_fwd_snap(const void* q, const void* k, const void* v, const float* log_alpha,
+                        const float* beta, const float* initial_state,
+                        const int32_t* cu_seqlens, int32_t chunk, void* out, float* final_state,
+                        const kda_dims* dims, const kda_snap_spec* snap,
+                        const int32_t* snap_slots, float* snap_pool, void* stream);
+
+/* Optional parts of a forward call (kda_fwd_ex). */
+typedef struct {
+    const void* out_gate;         /* [B, T, H, d_v] qkv_dtype, or NULL              */
+    const kda_snap_spec* snap;    /* NULL: no snapshots                             */
+    const int32_t* snap_slots;    /* as in kda_fwd_snap (used when snap != NULL)    */
+    float* snap_pool;             /* as in kda_fwd_snap (used when snap != NULL)    */
+} kda_fwd_opts;
+
+/*
+ * kda_fwd_ex -- kda_fwd with the optional parts of a KDA layer's forward.
+ *
+ * out_gate: the gate that follows the attention in KDA blocks (aiblin.ru page
+ * named at the top, in its description of the layer stack: after the
+ * attention a further filter decides which share of the retrieved information
+ * passes on to the model's main stream, in the Gated MLA blocks and in the
+ * KDA blocks alike).  The caller computes the gate (its projection and
+ * activation are outside this library) and passes its values; the library
+ * multiplies them into the output before the single rounding to qkv_dtype:
+ *     out[t, h, c] = o[t, h, c] * out_gate[t, h, c]
+ * Same layout as out, 16-byte aligned, device memory; it may not overlap out
+ * or final_state.  The gate does not enter the state.
+ * snap, snap_slots, snap_pool: prefix-cache snapshots exactly as in
+ * kda_fwd_snap.  opts == NULL (or all members NULL) is a plain kda_fwd.
+ */
+kda_status kda_fwd_ex(const void* q, const void* k, const void* v, const float* log_alpha,
+                      const float* beta, const float* initial_state, const int32_t* cu_seqlens,
+                      int32_t chunk, void* out, float* final_state, const kda_dims* dims,
+                      const kda_fwd_opts* opts, void* stream);
+
 /*
  * kda_fwd_host -- the same computation on HOST buffers (same shapes/layouts;
  * cu_seqlens is a host array here).  Copies the inputs to the device (one
@@ -185,6 +258,8 @@ typedef struct {
  *                device status word (kda_check_device: KDA_ERR_INVALID_ARG).
  *                Two sequences must not name the same slot.
  *   out          [N, T, H, d_v]   qkv_dtype (bf16 rounded to nearest even)
+ *   out_gate     [N, T, H, d_v]   qkv_dtype, or NULL: output gate, as in
+ *                                 kda_fwd_ex (out = o * out_gate)
  *   token_states [N, T, H, d_k, d_v] fp32, or NULL: the state after each of
  *                the T tokens, so that a verifier that accepts only the first
  *                m tokens can continue from token_states[n][m-1]
@@ -193,7 +268,8 @@ typedef struct {
  */
 kda_status kda_decode(const void* q, const void* k, const void* v, const float* log_alpha,
                       const float* beta, float* state, const int32_t* slots, void* out,
-                      float* token_states, const kda_decode_dims* dims, void* stream);
+                      const void* out_gate, float* token_states, const kda_decode_dims* dims,
+                      void* stream);
 
 /* Static description of a status code. */
 const char* kda_status_string(kda_status s);

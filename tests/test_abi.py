@@ -97,10 +97,10 @@ def test_zero_length_is_accepted_by_host_checks():
 # ---------------------------------------------------------------- kda_decode arguments
 def call_decode(dims, q=FAKE, k=FAKE + (1 << 30), v=FAKE + (2 << 30), la=FAKE + (3 << 30),
                 be=FAKE + (4 << 30), st=FAKE + (6 << 30), slots=None, out=FAKE + (5 << 30),
-                ts=None):
+                ts=None, gate=None):
     lib = kda.load_library()
     P = lambda x: None if x is None else ctypes.c_void_p(x)
-    rc = lib.kda_decode(P(q), P(k), P(v), P(la), P(be), P(st), P(slots), P(out), P(ts),
+    rc = lib.kda_decode(P(q), P(k), P(v), P(la), P(be), P(st), P(slots), P(out), P(gate), P(ts),
                         ctypes.byref(dims), None)
     return kda.STATUS[rc], lib.kda_last_error().decode()
 
@@ -122,7 +122,7 @@ def test_decode_rejects_bad_arguments():
     assert call_decode(DD(S=8), slots=FAKE + (7 << 30) + 2)[0] == "KDA_ERR_MISALIGNED"
     lib = kda.load_library()
     assert kda.STATUS[lib.kda_decode(None, None, None, None, None, None, None, None, None, None,
-                                     None)] == "KDA_ERR_INVALID_ARG"
+                                     None, None)] == "KDA_ERR_INVALID_ARG"
 
 
 def test_decode_rejects_aliasing():
@@ -131,6 +131,8 @@ def test_decode_rejects_aliasing():
     assert call_decode(DD(), st=FAKE + (1 << 30) + 256)[0] == "KDA_ERR_ALIAS"
     st, msg = call_decode(DD(), ts=FAKE + (6 << 30) + 4096)
     assert st == "KDA_ERR_ALIAS" and "token_states" in msg
+    assert call_decode(DD(), gate=FAKE + (5 << 30) + 32)[0] == "KDA_ERR_ALIAS"  # gate inside out
+    assert call_decode(DD(), gate=FAKE + (7 << 30) + 8)[0] == "KDA_ERR_MISALIGNED"
 
 
 def test_decode_empty_batch_is_a_no_op():
@@ -138,3 +140,54 @@ def test_decode_empty_batch_is_a_no_op():
     assert call_decode(DD(N=0), q=None, k=None, v=None, la=None, be=None, st=None,
                        out=None)[0] == "KDA_OK"
     assert kda.last_launch_count() == 0
+
+
+# ---------------------------------------------------------------- kda_fwd_snap arguments
+def call_snap(spec, slots=FAKE + (8 << 30), pool=FAKE + (9 << 30), dims=None, out=FAKE + (5 << 30)):
+    lib = kda.load_library()
+    P = lambda x: None if x is None else ctypes.c_void_p(x)
+    d = dims or D()
+    rc = lib.kda_fwd_snap(P(FAKE), P(FAKE + (1 << 30)), P(FAKE + (2 << 30)), P(FAKE + (3 << 30)),
+                          P(FAKE + (4 << 30)), None, None, 64, P(out), None, ctypes.byref(d),
+                          None if spec is None else ctypes.byref(spec), P(slots), P(pool), None)
+    return kda.STATUS[rc], lib.kda_last_error().decode()
+
+
+def test_snap_rejects_bad_arguments():
+    S = kda.SnapSpec
+    assert call_snap(None)[0] == "KDA_ERR_INVALID_ARG"
+    assert call_snap(S(0, 2, 4))[0] == "KDA_ERR_INVALID_ARG"
+    assert call_snap(S(96, 2, 4))[0] == "KDA_ERR_INVALID_ARG"  # not a multiple of the chunk
+    assert call_snap(S(64, -1, 4))[0] == "KDA_ERR_INVALID_ARG"
+    assert call_snap(S(64, 2, 4), slots=None)[0] == "KDA_ERR_INVALID_ARG"
+    assert call_snap(S(64, 2, 4), pool=FAKE + (9 << 30) + 4)[0] == "KDA_ERR_MISALIGNED"
+    assert call_snap(S(64, 2, 4), slots=FAKE + (8 << 30) + 2)[0] == "KDA_ERR_MISALIGNED"
+    # the forward's own checks still come first
+    assert call_snap(S(64, 2, 4), dims=D(dk=96))[0] == "KDA_ERR_UNSUPPORTED"
+
+
+def test_snap_rejects_aliasing():
+    S = kda.SnapSpec
+    st, msg = call_snap(S(64, 2, 4), pool=FAKE + (5 << 30))  # pool == out
+    assert st == "KDA_ERR_ALIAS" and "snap_pool" in msg
+    st, msg = call_snap(S(64, 2, 4), slots=FAKE + (5 << 30) + 64)  # slot table inside out
+    assert st == "KDA_ERR_ALIAS"
+
+
+# ---------------------------------------------------------------- kda_fwd_ex (output gate)
+def call_ex(gate, out=FAKE + (5 << 30), dims=None):
+    lib = kda.load_library()
+    P = lambda x: None if x is None else ctypes.c_void_p(x)
+    opts = kda.FwdOpts(gate, None, None, None)
+    d = dims or D()
+    rc = lib.kda_fwd_ex(P(FAKE), P(FAKE + (1 << 30)), P(FAKE + (2 << 30)), P(FAKE + (3 << 30)),
+                        P(FAKE + (4 << 30)), None, None, 64, P(out), None, ctypes.byref(d),
+                        ctypes.byref(opts), None)
+    return kda.STATUS[rc], lib.kda_last_error().decode()
+
+
+def test_gate_rejects_bad_pointers():
+    assert call_ex(FAKE + (7 << 30) + 2)[0] == "KDA_ERR_MISALIGNED"
+    st, msg = call_ex(FAKE + (5 << 30) + 64)  # gate inside out
+    assert st == "KDA_ERR_ALIAS" and "out_gate" in msg
+    assert call_ex(FAKE + (7 << 30), dims=D(dv=48))[0] == "KDA_ERR_UNSUPPORTED"
