@@ -343,6 +343,71 @@ def recorded_traffic(kernel_tag: str):
     return rec["bytes_per_launch"] if h.hexdigest() == rec["sha256"] else None
 
 
+# ------------------------------------------------------------------ context parallel, emulated
+def run_cp_emulation(args):
+    """Each of W virtual ranks owns T/W tokens of every sequence.  Rank r runs
+    kda_transition on its span, kda_apply_transitions on the transitions of
+    ranks < r (the all-gather's result), then kda_fwd from that state.  On one
+    GPU the ranks run one after another; each rank's work is timed with CUDA
+    events, and a W-GPU run would take the slowest rank's time plus one
+    all-gather of W x B x H x 128 KiB (estimated here at the measured 770 GB/s
+    NVLink peer bandwidth, never timed)."""
+    import torch
+    import gated_delta_rule_139_b200 as kda
+
+    W = args.cp_emulate
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    inp = workload(args.workload, seed=0)
+    if inp.cu_seqlens is not None or inp.T % W or not inp.bf16 or inp.dk != 128:
+        raise SystemExit("--cp-emulate needs an unpacked bf16 d=128 workload with T divisible by W")
+    span = inp.T // W
+    t = lambda a: torch.from_numpy(a).view(torch.bfloat16) if a.dtype == np.uint16 else \
+        torch.from_numpy(a)
+    full = {k_: t(getattr(inp, k_)).to(dev) for k_ in ("q", "k", "v", "log_alpha", "beta")}
+    s0 = None if inp.initial_state is None else torch.from_numpy(inp.initial_state).to(dev)
+    spans = [{k_: full[k_][:, r * span:(r + 1) * span].contiguous() for k_ in full}
+             for r in range(W)]
+    del full
+    stream = torch.cuda.current_stream(dev)
+    trans = [kda.kda_transition(s["k"], s["v"], s["log_alpha"], s["beta"]) for s in spans]
+    gathered = torch.stack(trans)
+
+    def rank_step(r):
+        s = spans[r]
+        kda.kda_transition(s["k"], s["v"], s["log_alpha"], s["beta"], out=trans[r])
+        s_in = kda.kda_apply_transitions(gathered[:r], s0)
+        return kda.kda_fwd(**s, initial_state=s_in)
+
+    per_rank = []
+    for r in range(W):
+        for _ in range(args.warmup):
+            rank_step(r)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.steps):
+            rank_step(r)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        per_rank.append(e0.elapsed_time(e1) / args.steps)
+    gather_bytes = W * inp.B * inp.H * 2 * 128 * 128 * 4
+    gather_ms = gather_bytes / 770e9 * 1e3
+    proj_ms = max(per_rank) + gather_ms
+    tokens = inp.tokens
+    line = {"metric": METRIC + " -- context parallel, emulated", "value": tokens / (proj_ms * 1e-3) / 1e6,
+            "unit": UNIT, "n_gpus": 1, "emulated_ranks": W, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": proj_ms, "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": dict(workload_config(inp, 1), parallelism=f"cp{W} emulated on 1 GPU",
+                           span_tokens=span),
+            "per_rank_ms": per_rank, "sum_of_ranks_ms": sum(per_rank),
+            "allgather": {"bytes": gather_bytes, "ms_estimate": gather_ms,
+                          "basis": "770 GB/s measured NVLink peer copy; not timed"},
+            "note": "ms_per_step = slowest emulated rank + all-gather estimate"}
+    print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------------------ main arm
 def main():
     ap = argparse.ArgumentParser()
@@ -357,6 +422,10 @@ def main():
     ap.add_argument("--out-gate", action="store_true",
                     help="fuse an output gate (random values in (0, 1), dtype of q) into the "
                          "step (kda_fwd_ex / kda_decode)")
+    ap.add_argument("--cp-emulate", type=int, default=0, metavar="W",
+                    help="context-parallel prefill of the workload over W ranks, emulated on "
+                         "one GPU: the ranks' span work runs one after another and is timed "
+                         "per rank (not a multi-GPU measurement)")
     ap.add_argument("--snap-interval", type=int, default=0,
                     help="forward workloads: also write a prefix-cache state snapshot every "
                          "this many tokens (kda_fwd_snap), each to its own pool row")
@@ -367,6 +436,9 @@ def main():
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.cp_emulate:
+        run_cp_emulation(args)
         return
 
     import torch

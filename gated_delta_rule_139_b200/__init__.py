@@ -17,7 +17,8 @@ from __future__ import annotations
 import ctypes
 import os
 
-__all__ = ["kda_fwd", "kda_fwd_host", "kda_fwd_noalloc", "kda_fwd_snap", "kda_decode", "KDAError", "library_path", "load_library",
+__all__ = ["kda_fwd", "kda_fwd_host", "kda_fwd_noalloc", "kda_fwd_snap", "kda_decode",
+           "kda_transition", "kda_apply_transitions", "KDAError", "library_path", "load_library",
            "last_launch_count", "last_path", "check_device", "profile_enable", "profile_read",
            "STATUS"]
 
@@ -81,6 +82,11 @@ def load_library():
         lib.kda_fwd_ex.argtypes = sig[:-1] + [ctypes.POINTER(FwdOpts), p]
         lib.kda_fwd_ex.restype = ctypes.c_int
         lib.kda_decode.argtypes = [p, p, p, p, p, p, p, p, p, p, ctypes.POINTER(DecodeDims), p]
+        lib.kda_transition.argtypes = [p, p, p, p, ctypes.POINTER(Dims), p, p]
+        lib.kda_transition.restype = ctypes.c_int
+        lib.kda_apply_transitions.argtypes = [p, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                              p, p, p]
+        lib.kda_apply_transitions.restype = ctypes.c_int
         lib.kda_decode.restype = ctypes.c_int
         lib.kda_status_string.argtypes = [ctypes.c_int]
         lib.kda_status_string.restype = ctypes.c_char_p
@@ -120,7 +126,7 @@ def profile_enable(on: bool = True) -> None:
 def profile_read() -> dict:
     """{kernel name: (summed ms, launches)} since the previous read (synchronises)."""
     lib = load_library()
-    n = 6
+    n = 7
     ms = (ctypes.c_double * n)()
     cnt = (ctypes.c_int64 * n)()
     _check(lib.kda_profile_read(ctypes.cast(ms, ctypes.c_void_p), ctypes.cast(cnt, ctypes.c_void_p), n))
@@ -332,3 +338,47 @@ def kda_decode(q, k, v, log_alpha, beta, state, slots=None, out=None, token_stat
                         ctypes.c_void_p(stream.cuda_stream))
     _check(rc)
     return out, token_states
+
+
+def kda_transition(k, v, log_alpha, beta, out=None, stream=None):
+    """Affine map S_out = M S_in + B of each of the B sequences of [B,T,H,128]
+    bf16 k, v (fp32 log_alpha, beta): returns trans [B,H,2,128,128] fp32 with
+    trans[b,h,0] = B^T and trans[b,h,1] = M^T."""
+    import torch
+
+    lib = load_library()
+    for t in (k, v, log_alpha, beta):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("inputs must be contiguous CUDA tensors")
+    if k.dim() != 4:
+        raise ValueError("k must be [B,T,H,128]")
+    B, T, H, dk = k.shape
+    d = Dims(B, T, H, dk, v.shape[-1], 0, KDA_BF16 if k.dtype == torch.bfloat16 else KDA_F32)
+    if out is None:
+        out = torch.empty((B, H, 2, 128, 128), dtype=torch.float32, device=k.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(k.device)
+    ptr = lambda t: ctypes.c_void_p(t.data_ptr())
+    _check(lib.kda_transition(ptr(k), ptr(v), ptr(log_alpha), ptr(beta), ctypes.byref(d),
+                              ptr(out), ctypes.c_void_p(stream.cuda_stream)))
+    return out
+
+
+def kda_apply_transitions(trans, initial_state=None, out=None, stream=None):
+    """State after a chain of spans: trans [count,B,H,2,128,128] (span 0 first),
+    initial_state [B,H,128,128] or None (zero).  Returns [B,H,128,128] fp32."""
+    import torch
+
+    lib = load_library()
+    if trans.dim() != 6 or not trans.is_cuda or not trans.is_contiguous():
+        raise ValueError("trans must be a contiguous CUDA tensor [count,B,H,2,128,128]")
+    count, B, H = trans.shape[:3]
+    if out is None:
+        out = torch.empty((B, H, 128, 128), dtype=torch.float32, device=trans.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(trans.device)
+    ptr = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
+    _check(lib.kda_apply_transitions(ptr(trans) if count else None, count, B, H,
+                                     ptr(initial_state), ptr(out),
+                                     ctypes.c_void_p(stream.cuda_stream)))
+    return out

@@ -606,6 +606,131 @@ kda_status kda_fwd_noalloc(const void* q, const void* k, const void* v, const fl
     return KDA_OK;
 }
 
+kda_status kda_transition(const void* k, const void* v, const float* log_alpha,
+                          const float* beta, const kda_dims* d, float* trans, void* stream) {
+    g_last_error[0] = 0;
+    g_last_launches = 0;
+    g_last_path = "";
+    if (!d) return fail(KDA_ERR_INVALID_ARG, "dims is NULL");
+    if (d->B < 1 || d->T < 0 || d->H < 1)
+        return fail(KDA_ERR_INVALID_ARG, "need B >= 1, T >= 0, H >= 1 (got B=%d T=%d H=%d)",
+                    d->B, d->T, d->H);
+    if (d->qkv_dtype != KDA_F32 && d->qkv_dtype != KDA_BF16)
+        return fail(KDA_ERR_INVALID_ARG, "qkv_dtype must be KDA_F32 or KDA_BF16");
+    if (d->d_k != 128 || d->d_v != 128 || d->qkv_dtype != KDA_BF16)
+        return fail(KDA_ERR_UNSUPPORTED, "kda_transition needs bf16 k/v with d_k = d_v = 128");
+    const int64_t tokens = (int64_t)d->B * d->T;
+    if (!trans) return fail(KDA_ERR_INVALID_ARG, "trans must be non-NULL");
+    if (tokens > 0 && (!k || !v || !log_alpha || !beta))
+        return fail(KDA_ERR_INVALID_ARG, "k, v, log_alpha and beta must be non-NULL");
+    const void* ptrs[] = {k, v, log_alpha, beta, trans};
+    const char* names[] = {"k", "v", "log_alpha", "beta", "trans"};
+    for (int i = 0; i < 5; ++i)
+        if (ptrs[i] && ((uintptr_t)ptrs[i] & 15u))
+            return fail(KDA_ERR_MISALIGNED, "%s is not 16-byte aligned", names[i]);
+    const int64_t n = tokens * d->H * 128;
+    const Range in[] = {{(uintptr_t)k, (uintptr_t)k + (k ? n * 2 : 0), "k"},
+                        {(uintptr_t)v, (uintptr_t)v + (v ? n * 2 : 0), "v"},
+                        {(uintptr_t)log_alpha, (uintptr_t)log_alpha + (log_alpha ? n * 4 : 0),
+                         "log_alpha"},
+                        {(uintptr_t)beta, (uintptr_t)beta + (beta ? tokens * d->H * 4 : 0), "beta"}};
+    const Range rt = {(uintptr_t)trans, (uintptr_t)trans + (uintptr_t)d->B * d->H * 2 * 128 * 128 * 4,
+                      "trans"};
+    for (const Range& r : in)
+        if (overlaps(rt, r)) return fail(KDA_ERR_ALIAS, "trans overlaps %s", r.name);
+    kda_status st = check_accessible(ptrs, names, 5);
+    if (st != KDA_OK) return st;
+    kda::FwdArgs a;
+    a.q = nullptr;
+    a.k = k;
+    a.v = v;
+    a.log_alpha = log_alpha;
+    a.beta = beta;
+    a.s0 = nullptr;
+    a.cu = nullptr;
+    a.out = nullptr;
+    a.s_final = nullptr;
+    a.B = d->B;
+    a.T = d->T;
+    a.H = d->H;
+    a.dk = 128;
+    a.dv = 128;
+    a.N = d->B;
+    a.bf16 = 1;
+    const kda::TcPlan p = plan_segments(a);
+    const size_t b_segs = ((size_t)p.max_units * sizeof(kda::SegEntry) + 255) & ~(size_t)255;
+    const size_t b_off = ((size_t)(a.N + 1) * 4 + 4 + 255) & ~(size_t)255;
+    const size_t b_trans = (size_t)p.max_units * a.H * 2 * 128 * 128 * sizeof(float);
+    cudaStream_t cs = (cudaStream_t)stream;
+    char* ws = nullptr;
+    cudaError_t e = pool_alloc((void**)&ws, b_segs + b_off + b_trans, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "workspace allocation");
+    kda::TcArgs t{};
+    t.k = k;
+    t.v = v;
+    t.log_alpha = log_alpha;
+    t.beta = beta;
+    t.B = a.B;
+    t.T = a.T;
+    t.H = a.H;
+    t.N = a.N;
+    t.segs = (kda::SegEntry*)ws;
+    t.seg_off = (int32_t*)(ws + b_segs);
+    t.n_units = t.seg_off + a.N + 1;
+    t.trans = (float*)(ws + b_segs + b_off);
+    int launches = 0;
+    g_last_path = "tc";
+    e = kda::launch_transition(t, p, trans, cs, &launches);
+    cudaFreeAsync(ws, cs);
+    g_last_launches = launches;
+    if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+    return KDA_OK;
+}
+
+kda_status kda_apply_transitions(const float* trans, int32_t count, int32_t B, int32_t H,
+                                 const float* initial_state, float* state_out, void* stream) {
+    g_last_error[0] = 0;
+    g_last_launches = 0;
+    g_last_path = "";
+    if (count < 0 || B < 1 || H < 1)
+        return fail(KDA_ERR_INVALID_ARG, "need count >= 0, B >= 1, H >= 1 (got %d, %d, %d)",
+                    count, B, H);
+    if (!state_out) return fail(KDA_ERR_INVALID_ARG, "state_out must be non-NULL");
+    if (count > 0 && !trans) return fail(KDA_ERR_INVALID_ARG, "trans must be non-NULL");
+    const void* ptrs[] = {trans, initial_state, state_out};
+    const char* names[] = {"trans", "initial_state", "state_out"};
+    for (int i = 0; i < 3; ++i)
+        if (ptrs[i] && ((uintptr_t)ptrs[i] & 15u))
+            return fail(KDA_ERR_MISALIGNED, "%s is not 16-byte aligned", names[i]);
+    const uintptr_t st_bytes = (uintptr_t)B * H * 128 * 128 * 4;
+    const Range rt = {(uintptr_t)trans, (uintptr_t)trans + (trans ? (uintptr_t)count * 2 * st_bytes : 0),
+                      "trans"};
+    const Range r0 = {(uintptr_t)initial_state, (uintptr_t)initial_state + (initial_state ? st_bytes : 0),
+                      "initial_state"};
+    const Range ro = {(uintptr_t)state_out, (uintptr_t)state_out + st_bytes, "state_out"};
+    if (overlaps(ro, rt)) return fail(KDA_ERR_ALIAS, "state_out overlaps trans");
+    if (overlaps(ro, r0) && !(ro.lo == r0.lo))
+        return fail(KDA_ERR_ALIAS, "state_out partly overlaps initial_state");
+    kda_status st = check_accessible(ptrs, names, 3);
+    if (st != KDA_OK) return st;
+    kda::ChainArgs c;
+    c.trans = trans;
+    c.off = nullptr;
+    c.n_units = nullptr;
+    c.count = count;
+    c.B = B;
+    c.H = H;
+    c.s0 = initial_state;
+    c.out = state_out;
+    c.compose = 0;
+    int launches = 0;
+    g_last_path = "chain";
+    cudaError_t e = kda::launch_chain(c, (cudaStream_t)stream, &launches);
+    g_last_launches = launches;
+    if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+    return KDA_OK;
+}
+
 kda_status kda_decode(const void* q, const void* k, const void* v, const float* log_alpha,
                       const float* beta, float* state, const int32_t* slots, void* out,
                       const void* out_gate, float* token_states, const kda_decode_dims* d,
@@ -735,7 +860,8 @@ kda_status kda_profile_read(double* total_ms, int64_t* launches, int32_t n) {
 
 const char* kda_profile_slot_name(int32_t slot) {
     static const char* names[] = {"seg_setup", "tc_pass1_transitions", "seg_scan",
-                                  "tc_pass3_forward", "ffma_forward", "decode_step"};
+                                  "tc_pass3_forward", "ffma_forward", "decode_step",
+                                  "transition_chain"};
     return (slot >= 0 && slot < kda::NUM_SLOTS) ? names[slot] : "";
 }
 

@@ -11,7 +11,7 @@ constexpr int kMaxDevices = 64;  // size of per-device attribute caches
 
 // Kernel slots of the optional per-launch timing (kda_profile_*).
 enum KernelSlot : int { SLOT_SETUP = 0, SLOT_PASS1 = 1, SLOT_SCAN = 2, SLOT_PASS3 = 3, SLOT_FFMA = 4,
-                        SLOT_DECODE = 5, NUM_SLOTS = 6 };
+                        SLOT_DECODE = 5, SLOT_CHAIN = 6, NUM_SLOTS = 7 };
 
 // Device status codes (first error wins; read and cleared by kda_check_device).
 enum DeviceStatus : int { ERR_WAIT_TIMEOUT = 1, ERR_SEG_OVERFLOW = 2, ERR_BAD_SLOT = 3 };
@@ -75,6 +75,7 @@ struct TcArgs {
     float* trans;       // [max_units, H, 2, 128, 128]: B^T then M^T of each segment
     float* sin;         // [max_units, H, 128, 128]: S_in^T of each segment
     const void* gate = nullptr;  // optional output gate, as in FwdArgs
+    int32_t trans_all = 0;       // pass 1 also for each sequence's last segment
     // optional state snapshots, as in FwdArgs
     const int32_t* snap_slots = nullptr;
     float* snap_pool = nullptr;
@@ -95,6 +96,34 @@ struct TcPlan {
 
 // bf16 q/k/v with d_k = d_v = 128: tcgen05 tensor-core path.
 cudaError_t launch_tc(const TcArgs& a, const TcPlan& p, cudaStream_t stream, int* launches);
+
+// Chain of affine state maps S -> M S + B, in the transposed layout of the
+// library's transitions (entry [2][128][128]: B^T, then M^T; S^T_out = S^T_in M^T
+// + B^T), evaluated on fp32 CUDA cores.
+//   compose = 1: for each sequence b, compose its units off[b] .. off[b+1]-1 of
+//                `trans` ([units][H][2][128][128]) into one transition, written to
+//                out[b][h] in the same layout.
+//   compose = 0: apply the first `count` transitions of `trans`
+//                ([count][B][H][2][128][128]) to s0 ([B][H][128][128], or zero),
+//                writing the resulting state to out ([B][H][128][128], natural
+//                d_k x d_v layout).
+struct ChainArgs {
+    const float* trans;
+    const int32_t* off;      // compose: [B+1] first unit of each sequence
+    const int32_t* n_units;  // compose: number of valid units
+    int32_t count;           // apply: transitions to apply
+    int32_t B, H;
+    const float* s0;         // apply: initial state or nullptr
+    float* out;
+    int32_t compose;
+};
+cudaError_t launch_chain(const ChainArgs& c, cudaStream_t stream, int* launches);
+
+// Transition of every sequence (S_out = M S_in + B over all its tokens): the
+// segment table, pass 1 over all segments, then their composition into out
+// ([N][H][2][128][128]: B^T, M^T).  Uses a.trans as the per-segment workspace.
+cudaError_t launch_transition(const TcArgs& a, const TcPlan& p, float* out, cudaStream_t stream,
+                              int* launches);
 size_t tc_smem_bytes();
 // Reads and clears the current device's status word (0 = no device-side error).
 cudaError_t tc_take_status(int* code);

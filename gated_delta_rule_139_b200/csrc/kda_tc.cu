@@ -402,7 +402,8 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
     const int u = blockIdx.x, h = blockIdx.y, H = a.H;
     if (u >= *a.n_units) return;
     const SegEntry sg = a.segs[u];
-    if (SEG && sg.last) return;  // transitions only for segments with a successor
+    // transitions only for segments with a successor, unless all are asked for
+    if (SEG && sg.last && !a.trans_all) return;
     const bool snap_on = !SEG && a.snap_pool != nullptr;
     const bool gate_on = !SEG && a.gate != nullptr;
     uint32_t gate_parity = 0;
@@ -1158,6 +1159,55 @@ cudaError_t launch_tc(const TcArgs& a, const TcPlan& p, cudaStream_t stream, int
     profile_mark(SLOT_PASS3, false, stream);
     *launches += 1;
     return cudaGetLastError();
+}
+
+cudaError_t launch_transition(const TcArgs& a_in, const TcPlan& p, float* out, cudaStream_t stream,
+                              int* launches) {
+    TcArgs a = a_in;
+    a.trans_all = 1;
+    static bool attr_set[kMaxDevices] = {};
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev >= kMaxDevices || !attr_set[dev]) {
+        err = cudaFuncSetAttribute(tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)LayT<true>::BYTES);
+        if (err != cudaSuccess) return err;
+        if (dev < kMaxDevices) attr_set[dev] = true;
+    }
+    TcMaps maps;
+    memset(&maps, 0, sizeof maps);
+    const int64_t tokens = (int64_t)a.B * a.T;
+    if (tokens > 0) {
+        if ((err = tile_map(&maps.k, a.k, false, a.H, tokens, false)) != cudaSuccess ||
+            (err = tile_map(&maps.v, a.v, false, a.H, tokens, true)) != cudaSuccess ||
+            (err = tile_map(&maps.la, a.log_alpha, true, a.H, tokens, false)) != cudaSuccess)
+            return err;
+    }
+    profile_mark(SLOT_SETUP, true, stream);
+    seg_setup_kernel<<<1, 1024, 0, stream>>>(a.cu, a.N, a.T, p.seg_chunks, p.max_units, a.segs,
+                                             a.seg_off, a.n_units);
+    profile_mark(SLOT_SETUP, false, stream);
+    *launches += 1;
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    profile_mark(SLOT_PASS1, true, stream);
+    tc_kernel<true><<<dim3((unsigned)p.max_units, (unsigned)a.H), NT, LayT<true>::BYTES, stream>>>(
+        a, maps);
+    profile_mark(SLOT_PASS1, false, stream);
+    *launches += 1;
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    // compose each sequence's segment transitions into one
+    ChainArgs c;
+    c.trans = a.trans;
+    c.off = a.seg_off;
+    c.n_units = a.n_units;
+    c.count = 0;
+    c.B = a.N;
+    c.H = a.H;
+    c.s0 = nullptr;
+    c.out = out;
+    c.compose = 1;
+    return launch_chain(c, stream, launches);
 }
 
 }  // namespace kda

@@ -271,6 +271,46 @@ kda_status kda_decode(const void* q, const void* k, const void* v, const float* 
                       const void* out_gate, float* token_states, const kda_decode_dims* dims,
                       void* stream);
 
+/*
+ * kda_transition -- the affine map each sequence applies to its state.
+ *
+ * The chunk-parallel section of the page named at the top: a span of tokens
+ * acts on the state that enters it as S_out = M S_in + B, with B the span's
+ * local state (from a zero incoming state) and M a token-dependent d_k x d_k
+ * transition matrix, so spans can be processed independently and chained
+ * afterwards.  This entry point returns (M, B) for each of the B sequences of
+ * [B, T, H, *] k, v, log_alpha, beta (no cu_seqlens; q is not needed); with
+ * kda_apply_transitions it is the exchange step of context parallelism, where
+ * each GPU holds one span of a long sequence.
+ *
+ *   k, v       [B, T, H, 128] bf16;  log_alpha [B, T, H, 128] fp32;  beta [B, T, H]
+ *   trans      [B, H, 2, 128, 128] fp32, written: trans[b][h][0] = B^T (d_v x d_k),
+ *              trans[b][h][1] = M^T (d_k x d_k), i.e. S_out^T = S_in^T M^T + B^T
+ * Only bf16 with d_k = d_v = 128 (KDA_ERR_UNSUPPORTED otherwise).  Long spans
+ * are cut into segments whose transitions are computed in parallel and then
+ * composed in fp32.  Temporary memory as kda_fwd.  trans may not overlap an
+ * input.
+ */
+kda_status kda_transition(const void* k, const void* v, const float* log_alpha,
+                          const float* beta, const kda_dims* dims, float* trans, void* stream);
+
+/*
+ * kda_apply_transitions -- the state after a chain of spans.
+ *
+ *   trans          [count, B, H, 2, 128, 128] fp32: transitions of consecutive
+ *                  spans (as kda_transition writes them), span 0 first
+ *   initial_state  [B, H, 128, 128] fp32 (d_k x d_v), or NULL for zero
+ *   state_out      [B, H, 128, 128] fp32, written with the state after the
+ *                  `count` spans: S <- M_j S + B_j for j = 0 .. count-1 (fp32).
+ *                  count = 0 copies initial_state (or writes zero).  It may be
+ *                  the same buffer as initial_state, not otherwise overlap it,
+ *                  and may not overlap trans.
+ * With the spans of a sequence spread over ranks, rank r passes the gathered
+ * transitions of ranks 0 .. r-1 and gets its incoming state.
+ */
+kda_status kda_apply_transitions(const float* trans, int32_t count, int32_t B, int32_t H,
+                                 const float* initial_state, float* state_out, void* stream);
+
 /* Static description of a status code. */
 const char* kda_status_string(kda_status s);
 
@@ -281,9 +321,9 @@ const char* kda_last_error(void);
  * thread issued. */
 int32_t kda_last_launch_count(void);
 
-/* Kernel family the last kda_fwd / kda_decode call on this host thread used:
- * "ffma" (fp32 CUDA-core path), "tc" (tcgen05 tensor-core path), "decode"
- * (kda_decode) or "" (no launch). */
+/* Kernel family the last call on this host thread used: "ffma" (fp32
+ * CUDA-core path), "tc" (tcgen05 tensor-core path), "decode" (kda_decode),
+ * "chain" (kda_apply_transitions) or "" (no launch). */
 const char* kda_last_path(void);
 
 /* Synchronises `stream`, then reads and clears the current device's status
@@ -300,8 +340,8 @@ kda_status kda_check_device(void* stream);
  * first n kernel slots the summed duration in milliseconds and the number of
  * launches since the previous read, then resets the sums.  Slots: 0 segment
  * table, 1 pass 1 (segment transitions), 2 segment scan, 3 pass 3 (forward),
- * 4 CUDA-core forward, 5 decode step; kda_profile_slot_name gives their
- * names. */
+ * 4 CUDA-core forward, 5 decode step, 6 transition chain;
+ * kda_profile_slot_name gives their names. */
 void kda_profile_enable(int32_t on);
 kda_status kda_profile_read(double* total_ms, int64_t* launches, int32_t n);
 const char* kda_profile_slot_name(int32_t slot);

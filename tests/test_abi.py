@@ -191,3 +191,38 @@ def test_gate_rejects_bad_pointers():
     st, msg = call_ex(FAKE + (5 << 30) + 64)  # gate inside out
     assert st == "KDA_ERR_ALIAS" and "out_gate" in msg
     assert call_ex(FAKE + (7 << 30), dims=D(dv=48))[0] == "KDA_ERR_UNSUPPORTED"
+
+
+# ---------------------------------------------------------------- transitions (context parallel)
+def test_transition_rejects_bad_arguments():
+    lib = kda.load_library()
+    P = lambda x: None if x is None else ctypes.c_void_p(x)
+
+    def call(d, k=FAKE, v=FAKE + (1 << 30), la=FAKE + (2 << 30), be=FAKE + (3 << 30),
+             tr=FAKE + (4 << 30)):
+        rc = lib.kda_transition(P(k), P(v), P(la), P(be), ctypes.byref(d), P(tr), None)
+        return kda.STATUS[rc]
+
+    assert call(D(dk=64, dv=64)) == "KDA_ERR_UNSUPPORTED"
+    assert call(D(dt=0)) == "KDA_ERR_UNSUPPORTED"  # fp32 inputs
+    assert call(D(B=0)) == "KDA_ERR_INVALID_ARG"
+    assert call(D(), tr=None) == "KDA_ERR_INVALID_ARG"
+    assert call(D(), v=None) == "KDA_ERR_INVALID_ARG"
+    assert call(D(), tr=FAKE + (4 << 30) + 8) == "KDA_ERR_MISALIGNED"
+    assert call(D(), tr=FAKE + (1 << 30) + 1024) == "KDA_ERR_ALIAS"  # trans inside v
+
+
+def test_apply_transitions_rejects_bad_arguments():
+    lib = kda.load_library()
+    P = lambda x: None if x is None else ctypes.c_void_p(x)
+
+    def call(count=2, B=1, H=2, tr=FAKE, s0=FAKE + (1 << 30), out=FAKE + (2 << 30)):
+        return kda.STATUS[lib.kda_apply_transitions(P(tr), count, B, H, P(s0), P(out), None)]
+
+    assert call(count=-1) == "KDA_ERR_INVALID_ARG"
+    assert call(H=0) == "KDA_ERR_INVALID_ARG"
+    assert call(tr=None) == "KDA_ERR_INVALID_ARG"
+    assert call(out=None) == "KDA_ERR_INVALID_ARG"
+    assert call(out=FAKE + (2 << 30) + 4) == "KDA_ERR_MISALIGNED"
+    assert call(out=FAKE + 4096) == "KDA_ERR_ALIAS"  # state_out inside trans
+    assert call(out=FAKE + (1 << 30) + 4096) == "KDA_ERR_ALIAS"  # partial overlap with s0

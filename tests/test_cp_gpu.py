@@ -1,0 +1,132 @@
+"""GPU parity of the context-parallel pieces: span transitions
+(kda_transition), chains of them (kda_apply_transitions), and the whole
+context-parallel prefill emulated on one GPU -- the virtual ranks run one after
+another, the all-gather is a stack of their transitions -- against the fp64
+oracle.  The real collective path runs with a one-rank NCCL group.
+
+Tolerance: relative Frobenius error per (sequence, head) <= 2e-2 (bf16 inputs).
+"""
+import numpy as np
+import pytest
+
+import oracle
+from gated_delta_rule_139_b200.inputs import make_inputs
+from kda_testlib import TOL_BF16_REL_FRO, out_to_f64, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+def _rel(a, b):
+    return np.linalg.norm(a - b) / np.linalg.norm(b)
+
+
+def _worst_state_err(got, ref):
+    return max(_rel(got[n, h], ref[n, h]) for n in range(ref.shape[0]) for h in range(ref.shape[1]))
+
+
+@pytest.mark.parametrize("seg_chunks", [None, "2", "3"])
+def test_transition_is_the_spans_affine_map(monkeypatch, seg_chunks):
+    """B = the state reached from zero; M S + B = the state reached from S."""
+    import torch
+    from gated_delta_rule_139_b200 import kda_apply_transitions, kda_transition
+    if seg_chunks:
+        monkeypatch.setenv("KDA_SEG_CHUNKS", seg_chunks)
+    inp = make_inputs(2, 64 * 9 + 13, 2, 128, 128, bf16=True, seed=400, state_sigma=0.1,
+                      gate_sigma=2.0)
+    d = to_device(inp)
+    trans = kda_transition(d["k"], d["v"], d["log_alpha"], d["beta"])
+    from_zero = kda_apply_transitions(trans[None])
+    from_s = kda_apply_transitions(trans[None], d["initial_state"])
+    torch.cuda.synchronize()
+    _, b_ref = oracle.recurrent(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, None, o_tokens=0)
+    _, s_ref = oracle.recurrent(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.initial_state,
+                                o_tokens=0)
+    bt = trans[:, :, 0].transpose(-1, -2).cpu().numpy().astype(np.float64)
+    assert _worst_state_err(bt, b_ref) <= TOL_BF16_REL_FRO
+    assert _worst_state_err(from_zero.cpu().numpy().astype(np.float64), b_ref) <= TOL_BF16_REL_FRO
+    assert _worst_state_err(from_s.cpu().numpy().astype(np.float64), s_ref) <= TOL_BF16_REL_FRO
+
+
+def test_empty_span_is_the_identity_map():
+    import torch
+    from gated_delta_rule_139_b200 import kda_apply_transitions, kda_transition
+    inp = make_inputs(1, 0, 2, 128, 128, bf16=True, seed=401, state_sigma=0.1)
+    d = to_device(inp)
+    e = torch.empty(1, 0, 2, 128, dtype=torch.bfloat16, device="cuda")
+    trans = kda_transition(e, e, torch.empty(1, 0, 2, 128, device="cuda"),
+                           torch.empty(1, 0, 2, device="cuda"))
+    out = kda_apply_transitions(trans[None], d["initial_state"])
+    torch.cuda.synchronize()
+    assert torch.equal(trans[:, :, 0], torch.zeros_like(trans[:, :, 0]))
+    assert torch.equal(trans[:, :, 1], torch.eye(128, device="cuda").expand_as(trans[:, :, 1]))
+    assert torch.equal(out, d["initial_state"])
+
+
+def test_apply_zero_transitions_copies_and_works_in_place():
+    import torch
+    from gated_delta_rule_139_b200 import kda_apply_transitions, kda_transition
+    inp = make_inputs(2, 300, 2, 128, 128, bf16=True, seed=402, state_sigma=0.1)
+    d = to_device(inp)
+    s0 = d["initial_state"]
+    none = torch.empty(0, 2, 2, 2, 128, 128, device="cuda")
+    assert torch.equal(kda_apply_transitions(none, s0), s0)
+    assert torch.equal(kda_apply_transitions(none), torch.zeros_like(s0))
+    trans = kda_transition(d["k"], d["v"], d["log_alpha"], d["beta"])
+    ref = kda_apply_transitions(trans[None], s0)
+    st = s0.clone()
+    kda_apply_transitions(trans[None], st, out=st)
+    torch.cuda.synchronize()
+    assert torch.equal(st, ref)
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_context_parallel_prefill_emulated_on_one_gpu(world):
+    """Virtual ranks one after another on one GPU: their concatenated outputs
+    and the last rank's state match the oracle over the whole sequences."""
+    import torch
+    from gated_delta_rule_139_b200 import kda_apply_transitions, kda_fwd, kda_transition
+    span = 64 * 5 + 7
+    inp = make_inputs(2, span * world, 2, 128, 128, bf16=True, seed=403 + world,
+                      state_sigma=0.05, gate_sigma=2.0)
+    d = to_device(inp)
+    keys = ("q", "k", "v", "log_alpha", "beta")
+    spans = [{k_: d[k_][:, r * span:(r + 1) * span].contiguous() for k_ in keys}
+             for r in range(world)]
+    trans = [kda_transition(s["k"], s["v"], s["log_alpha"], s["beta"]) for s in spans]
+    gathered = torch.stack(trans)  # what the all-gather delivers
+    outs, finals = [], []
+    for r, s in enumerate(spans):
+        s_in = kda_apply_transitions(gathered[:r], d["initial_state"])
+        o, f = kda_fwd(**s, initial_state=s_in)
+        outs.append(o)
+        finals.append(f)
+    torch.cuda.synchronize()
+    o_ref, s_ref = oracle.recurrent(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta,
+                                    inp.initial_state)
+    o_cp = out_to_f64(torch.cat(outs, 1))
+    for n in range(2):
+        for h in range(2):
+            assert _rel(o_cp[n, :, h], o_ref[n, :, h]) <= TOL_BF16_REL_FRO
+    assert _worst_state_err(finals[-1].cpu().numpy().astype(np.float64), s_ref) <= TOL_BF16_REL_FRO
+
+
+def test_cp_prefill_through_a_one_rank_nccl_group():
+    """The collective code path with real kernels: one rank, so it must equal
+    kda_fwd bit for bit."""
+    import torch
+    import torch.distributed as dist
+    from gated_delta_rule_139_b200 import kda_fwd
+    from gated_delta_rule_139_b200.cp import cp_prefill
+    inp = make_inputs(1, 64 * 4 + 5, 2, 128, 128, bf16=True, seed=410, state_sigma=0.05)
+    d = to_device(inp)
+    store = dist.HashStore()
+    dist.init_process_group("nccl", store=store, rank=0, world_size=1,
+                            device_id=torch.device("cuda", 0))
+    try:
+        o, f = cp_prefill(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["initial_state"])
+        o_ref, f_ref = kda_fwd(**{k_: d[k_] for k_ in ("q", "k", "v", "log_alpha", "beta")},
+                               initial_state=d["initial_state"])
+        torch.cuda.synchronize()
+        assert torch.equal(o, o_ref) and torch.equal(f, f_ref)
+    finally:
+        dist.destroy_process_group()
