@@ -93,9 +93,11 @@ struct LayT {
     static constexpr uint32_t EHB = EHA + 512;                    // fp32 [128] e^{rho_b}
     static constexpr uint32_t FAC = EHB + 512;                    // fp32 [5][128] gate factors
     static constexpr uint32_t BETA = FAC + 2560;                  // fp32 [64]
-    static constexpr uint32_t BAR = BETA + 256;                   // mbarriers: MMA, TMA, gate
+    static constexpr uint32_t BAR = BETA + 256;                   // mbarriers: MMA, TMA, gate, TB
     static constexpr uint32_t TMEMP = BAR + 32;                   // TMEM base address
-    static constexpr uint32_t END = TMEMP + 16;
+    // pass 3: T diag(beta) of the chunk as pass 1 stored it (bf16 64 x 64, K-major)
+    static constexpr uint32_t TBX = SEG ? TMEMP + 16 : (TMEMP + 16 + 1023) / 1024 * 1024;
+    static constexpr uint32_t END = SEG ? TMEMP + 16 : TBX + 8192;
     static constexpr uint32_t BYTES = END + 1024;                 // + alignment slack
 };
 static_assert(LayT<false>::TS + 64 * 72 * 4 <= LayT<false>::R1, "As/Ts overflow");
@@ -233,6 +235,20 @@ __device__ __forceinline__ void tma_store_tile(const CUtensorMap* map, const voi
         "r"(0), "r"(h), "r"(t0), "r"(smem_u32(src))
         : "memory");
 }
+// plain bulk copies (8 KB T tiles): shared -> global (bulk group), global -> shared (mbarrier)
+__device__ __forceinline__ void bulk_store(void* gdst, const void* ssrc, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst),
+                 "r"(smem_u32(ssrc)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_load(void* sdst, const void* gsrc, uint32_t bytes, void* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(sdst)),
+        "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit() {
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
@@ -407,6 +423,13 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
     const bool snap_on = !SEG && a.snap_pool != nullptr;
     const bool gate_on = !SEG && a.gate != nullptr;
     uint32_t gate_parity = 0;
+    // T cache: pass 1 stores each chunk's T diag(beta) tile, pass 3 loads it instead of
+    // inverting again.  Tile of chunk t of unit u at tbs + ((u H + h) seg_chunks + chunk) 8 KB.
+    const bool tb_cache = a.tbs != nullptr;
+    uint32_t tb_parity = 0;
+    auto tb_tile = [&](int64_t tt) {
+        return a.tbs + ((((int64_t)u * H + h) * a.seg_chunks + (tt - sg.t_begin) / C) << 13);
+    };
     const int64_t seq_lo = snap_on ? (a.cu ? (int64_t)a.cu[sg.n] : (int64_t)sg.n * a.T) : 0;
 
     float* gsum = reinterpret_cast<float*>(sm + Lay::GSUM);
@@ -417,6 +440,7 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + Lay::BAR);
     uint64_t* bar_raw = bar + 1;
     uint64_t* bar_gate = bar + 2;  // output-gate tile (pass 3 with a gate)
+    uint64_t* bar_tb = bar + 3;    // T tile stored by pass 1 (pass 3 with a T cache)
     uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(sm + Lay::TMEMP);
 
     if (warp == 0) {
@@ -427,6 +451,7 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
         mbar_init(bar, 1);
         mbar_init(bar_raw, 1);
         mbar_init(bar_gate, 1);
+        mbar_init(bar_tb, 1);
         fence_mbar_init();
     }
     tc_fence_before();
@@ -487,6 +512,10 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
     float beta_ld = 0.f;
     if (sg.t_begin < sg.t_end) {
         if (tid == 0) issue_raw(sg.t_begin, 0);
+        if (!SEG && tb_cache && tid == 0) {
+            mbar_expect_tx(bar_tb, 8192);
+            bulk_load(sm + Lay::TBX, tb_tile(sg.t_begin), 8192, bar_tb);
+        }
         if (tid < C && sg.t_begin + tid < sg.t_end) beta_ld = __ldg(a.beta + (sg.t_begin + tid) * H + h);
     }
 
@@ -500,6 +529,7 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
             const int c4 = lane, tg = warp, c0 = 4 * c4;  // tokens 4tg..4tg+3, channels c0..c0+3
             float4 la[4];
             uint2 kr[4], qr[4];
+            if (SEG && tb_cache && tid == 0) bulk_wait_read();  // last chunk's T tile has left TB
             if (!(ok = !__syncthreads_or(!mbar_wait(bar_raw, raw_parity, &g_tc_status,
                                                     ERR_WAIT_TIMEOUT)))) break;
             raw_parity ^= 1u;
@@ -630,7 +660,8 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
             // rows r of A (lanes 0-63) and P (lanes 64-127); warp slice wg handles the 16
             // columns j in [16wg, 16wg+16).  Columns j < 32 of rows r >= 32 come from the
             // cross-half product (TMEM columns 64 + j).
-            if (!SEG || quad < 2) {
+            const bool need_a = SEG || !tb_cache;  // A only feeds the inversion
+            if ((!SEG || quad < 2) && (quad >= 2 || need_a)) {
                 const int r = lrow & 63;
                 const bool isP = quad >= 2;
                 const bool lower_half = r < 32;  // warp-uniform
@@ -665,20 +696,30 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
                 }
             }
             __syncthreads();
-            invert_to_tb(As, Ts, Ys, beta_s, smem_u32(sm + Lay::TB), tid);
+            if (need_a) invert_to_tb(As, Ts, Ys, beta_s, smem_u32(sm + Lay::TB), tid);
         }
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
+        if (SEG && tb_cache && tid == 0) {  // keep T diag(beta) for pass 3
+            bulk_store(tb_tile(t0), sm + Lay::TB, 8192);
+            bulk_commit();
+        }
 
         // ============ phase 3: with TB = T diag(beta) and the per-half factors e^{rho_h}:
         //   W^T  = e^{rho_a} (X1k_a)^T TB_a^T + e^{rho_b} (X1k_b)^T TB_b^T  (combined at staging)
         //   U'^T = V^T TB^T
         // X1's k rows serve as an MN-major operand (K rows = tokens, MN blocks 16 KB apart);
         // the v tile is used as TMA wrote it.
-        if (tid == 0) {
+        bool tb_ok = true;
+        if (!SEG && tb_cache && tid == 0) {
+            tb_ok = mbar_wait(bar_tb, tb_parity, &g_tc_status, ERR_WAIT_TIMEOUT);
+            tb_parity ^= 1u;
+        }
+        if (tid == 0 && tb_ok) {
             tc_fence_after();
-            const uint32_t x1 = smem_u32(sm + Lay::X1), tb = smem_u32(sm + Lay::TB),
+            const uint32_t x1 = smem_u32(sm + Lay::X1),
+                           tb = smem_u32(sm + ((!SEG && tb_cache) ? Lay::TBX : Lay::TB)),
                            rv = smem_u32(sm + Lay::RV + vbuf * 16384);
             constexpr uint32_t id = idesc_bf16(128, 64, true, false);
 #pragma unroll
@@ -709,6 +750,11 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
             tmem_st_wait();
         }
         if (!(ok = wait_mma(bar, parity))) break;
+        // TBX is consumed: the next chunk's T tile may come in
+        if (!SEG && tb_cache && tid == 0 && t0 + C < sg.t_end) {
+            mbar_expect_tx(bar_tb, 8192);
+            bulk_load(sm + Lay::TBX, tb_tile(t0 + C), 8192, bar_tb);
+        }
         // The v tile is consumed: the output gate's [64][128] tile (if any) goes into
         // its buffer now, for the epilogue.
         if (gate_on && tid == 0) {
@@ -867,7 +913,7 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
     }
 
     // ---- results of the segment
-    if (!SEG && tid == 0) bulk_wait_all();  // output stores have left shared memory
+    if (tid == 0 && (!SEG || tb_cache)) bulk_wait_all();  // output / T stores are complete
     if (ok) {
         if (SEG) {  // slices 0-1: B^T, slices 2-3: M^T, 64 columns each
             const bool is_m = wg >= 2;
