@@ -212,10 +212,10 @@ kda_status run_tc(const kda::FwdArgs& a, cudaStream_t stream, int* launches) {
     const size_t b_off = ((size_t)(a.N + 1) * 4 + 4 + 255) & ~(size_t)255;
     const size_t b_trans = p.segmented ? (size_t)p.max_units * a.H * 2 * st : 0;
     const size_t b_sin = p.segmented ? (size_t)p.max_units * a.H * st : 0;
-    // T cache of the segmented plan: one 8 KB tile per chunk of every unit
-    const size_t b_tbs = p.segmented ? (size_t)p.max_units * a.H * p.seg_chunks * 8192 : 0;
+    // W/U' cache of the segmented plan: 32 KB per chunk of every unit
+    const size_t b_wu = p.segmented ? (size_t)p.max_units * a.H * p.seg_chunks * 32768 : 0;
     char* ws = nullptr;
-    cudaError_t e = pool_alloc((void**)&ws, b_segs + b_off + b_trans + b_sin + b_tbs, stream);
+    cudaError_t e = pool_alloc((void**)&ws, b_segs + b_off + b_trans + b_sin + b_wu, stream);
     if (e != cudaSuccess) return cuda_fail(e, "workspace allocation");
     kda::TcArgs t;
     t.q = a.q;
@@ -242,8 +242,8 @@ kda_status run_tc(const kda::FwdArgs& a, cudaStream_t stream, int* launches) {
     t.n_units = t.seg_off + a.N + 1;
     t.trans = p.segmented ? (float*)(ws + b_segs + b_off) : nullptr;
     t.sin = p.segmented ? (float*)(ws + b_segs + b_off + b_trans) : nullptr;
-    if (p.segmented) {  // pass 1 runs over every segment and keeps its T tiles for pass 3
-        t.tbs = (uint8_t*)(ws + b_segs + b_off + b_trans + b_sin);
+    if (p.segmented) {  // pass 1 runs over every segment and keeps W^T, U'^T for pass 3
+        t.wu = (uint8_t*)(ws + b_segs + b_off + b_trans + b_sin);
         t.seg_chunks = p.seg_chunks;
         t.trans_all = 1;
     }

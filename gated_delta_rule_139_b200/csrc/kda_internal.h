@@ -76,8 +76,8 @@ struct TcArgs {
     float* sin;         // [max_units, H, 128, 128]: S_in^T of each segment
     const void* gate = nullptr;  // optional output gate, as in FwdArgs
     int32_t trans_all = 0;       // pass 1 also for each sequence's last segment
-    uint8_t* tbs = nullptr;      // T cache: [max_units][H][seg_chunks][8 KB] (pass 1 writes, pass 3 reads)
-    int32_t seg_chunks = 0;      // chunks per segment (T cache stride)
+    uint8_t* wu = nullptr;       // W/U' cache: [max_units][H][seg_chunks][32 KB] (pass 1 writes, pass 3 reads)
+    int32_t seg_chunks = 0;      // chunks per segment (cache stride)
     // optional state snapshots, as in FwdArgs
     const int32_t* snap_slots = nullptr;
     float* snap_pool = nullptr;

@@ -93,11 +93,9 @@ struct LayT {
     static constexpr uint32_t EHB = EHA + 512;                    // fp32 [128] e^{rho_b}
     static constexpr uint32_t FAC = EHB + 512;                    // fp32 [5][128] gate factors
     static constexpr uint32_t BETA = FAC + 2560;                  // fp32 [64]
-    static constexpr uint32_t BAR = BETA + 256;                   // mbarriers: MMA, TMA, gate, TB
+    static constexpr uint32_t BAR = BETA + 256;                   // mbarriers: MMA, TMA, gate, W
     static constexpr uint32_t TMEMP = BAR + 32;                   // TMEM base address
-    // pass 3: T diag(beta) of the chunk as pass 1 stored it (bf16 64 x 64, K-major)
-    static constexpr uint32_t TBX = SEG ? TMEMP + 16 : (TMEMP + 16 + 1023) / 1024 * 1024;
-    static constexpr uint32_t END = SEG ? TMEMP + 16 : TBX + 8192;
+    static constexpr uint32_t END = TMEMP + 16;
     static constexpr uint32_t BYTES = END + 1024;                 // + alignment slack
 };
 static_assert(LayT<false>::TS + 64 * 72 * 4 <= LayT<false>::R1, "As/Ts overflow");
@@ -408,8 +406,11 @@ __device__ void invert_to_tb(const float* As, float* Ts, float* Ys, const float*
 }
 
 // ---------------------------------------------------------------- the chunk loop
-template <bool SEG>
+// MODE 0: pass 3 (forward from the true incoming state); MODE 1: pass 1 (segment
+// transitions); MODE 2: pass 3 that takes each chunk's W and U' from pass 1's cache.
+template <int MODE>
 __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_constant__ TcMaps maps) {
+    constexpr bool SEG = MODE == 1, FAST = MODE == 2;
     using Lay = LayT<SEG>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -423,12 +424,14 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
     const bool snap_on = !SEG && a.snap_pool != nullptr;
     const bool gate_on = !SEG && a.gate != nullptr;
     uint32_t gate_parity = 0;
-    // T cache: pass 1 stores each chunk's T diag(beta) tile, pass 3 loads it instead of
-    // inverting again.  Tile of chunk t of unit u at tbs + ((u H + h) seg_chunks + chunk) 8 KB.
-    const bool tb_cache = a.tbs != nullptr;
-    uint32_t tb_parity = 0;
-    auto tb_tile = [&](int64_t tt) {
-        return a.tbs + ((((int64_t)u * H + h) * a.seg_chunks + (tt - sg.t_begin) / C) << 13);
+    // W/U' cache: pass 1 stores each chunk's W^T (the 16 KB bf16 MN-major B operand of
+    // phase 5) and U'^T (bf16 [128][64], 16-byte pieces of row e XOR-swizzled by e & 7);
+    // MODE 2 loads them instead of building A, T, W and U' again.  Entry of chunk t of
+    // unit u: wu + ((u H + h) seg_chunks + chunk) * 32 KB, W^T first.
+    const bool wu_cache = a.wu != nullptr;
+    uint32_t w_parity = 0;
+    auto wu_tile = [&](int64_t tt) {
+        return a.wu + ((((int64_t)u * H + h) * a.seg_chunks + (tt - sg.t_begin) / C) << 15);
     };
     const int64_t seq_lo = snap_on ? (a.cu ? (int64_t)a.cu[sg.n] : (int64_t)sg.n * a.T) : 0;
 
@@ -440,8 +443,15 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + Lay::BAR);
     uint64_t* bar_raw = bar + 1;
     uint64_t* bar_gate = bar + 2;  // output-gate tile (pass 3 with a gate)
-    uint64_t* bar_tb = bar + 3;    // T tile stored by pass 1 (pass 3 with a T cache)
+    uint64_t* bar_w = bar + 3;     // W^T tile from the cache (MODE 2)
     uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(sm + Lay::TMEMP);
+    // MODE 2 keeps q~ in rows 0-63 of X1; rows 64-127 hold W^T in two 8 KB pieces
+    // (K steps 0-3 and 4-7 of the MN-major operand)
+    auto load_w = [&](int64_t tt) {
+        mbar_expect_tx(bar_w, 16384);
+        bulk_load(sm + Lay::X1 + 8192, wu_tile(tt), 8192, bar_w);
+        bulk_load(sm + Lay::X1 + 24576, wu_tile(tt) + 8192, 8192, bar_w);
+    };
 
     if (warp == 0) {
         tmem_alloc(tmem_ptr, 512);
@@ -451,7 +461,7 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
         mbar_init(bar, 1);
         mbar_init(bar_raw, 1);
         mbar_init(bar_gate, 1);
-        mbar_init(bar_tb, 1);
+        mbar_init(bar_w, 1);
         fence_mbar_init();
     }
     tc_fence_before();
@@ -504,18 +514,19 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
         tma_tile(sm + Lay::RK, &maps.k, 0, h, (int)tn, bar_raw);
         tma_tile(sm + Lay::RL, &maps.la, 0, h, (int)tn, bar_raw);
         if (!SEG) tma_tile(sm + Lay::RQ, &maps.q, 0, h, (int)tn, bar_raw);
-        uint8_t* rv = sm + Lay::RV + vbuf * 16384;  // two 64-channel swizzled halves
-        tma_tile(rv, &maps.v, 0, h, (int)tn, bar_raw);
-        tma_tile(rv + 8192, &maps.v, 64, h, (int)tn, bar_raw);
+        uint8_t* rv = sm + Lay::RV + vbuf * 16384;
+        if (FAST) {  // U'^T from the cache instead of v
+            bulk_load(rv, wu_tile(tn) + 16384, 16384, bar_raw);
+        } else {     // two 64-channel swizzled halves
+            tma_tile(rv, &maps.v, 0, h, (int)tn, bar_raw);
+            tma_tile(rv + 8192, &maps.v, 64, h, (int)tn, bar_raw);
+        }
     };
     uint32_t raw_parity = 0;
     float beta_ld = 0.f;
     if (sg.t_begin < sg.t_end) {
         if (tid == 0) issue_raw(sg.t_begin, 0);
-        if (!SEG && tb_cache && tid == 0) {
-            mbar_expect_tx(bar_tb, 8192);
-            bulk_load(sm + Lay::TBX, tb_tile(sg.t_begin), 8192, bar_tb);
-        }
+        if (FAST && tid == 0) load_w(sg.t_begin);
         if (tid < C && sg.t_begin + tid < sg.t_end) beta_ld = __ldg(a.beta + (sg.t_begin + tid) * H + h);
     }
 
@@ -529,7 +540,7 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
             const int c4 = lane, tg = warp, c0 = 4 * c4;  // tokens 4tg..4tg+3, channels c0..c0+3
             float4 la[4];
             uint2 kr[4], qr[4];
-            if (SEG && tb_cache && tid == 0) bulk_wait_read();  // last chunk's T tile has left TB
+            if (SEG && wu_cache && tid == 0) bulk_wait_read();  // last chunk's W^T has left WB
             if (!(ok = !__syncthreads_or(!mbar_wait(bar_raw, raw_parity, &g_tc_status,
                                                     ERR_WAIT_TIMEOUT)))) break;
             raw_parity ^= 1u;
@@ -542,7 +553,7 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
                     la[i] = *reinterpret_cast<const float4*>(sm + Lay::RL + (r * D + c0) * 4);
                     kr[i] = *reinterpret_cast<const uint2*>(sm + Lay::RK + (r * D + c0) * 2);
                     if (!SEG) qr[i] = *reinterpret_cast<const uint2*>(sm + Lay::RQ + (r * D + c0) * 2);
-                } else {  // the v tile is an operand as TMA wrote it: clear rows past the end
+                } else if (!FAST) {  // the v tile is an operand as TMA wrote it: clear rows past the end
                     *reinterpret_cast<uint2*>(sm + Lay::RV + vbuf * 16384 + mnmajor_off(r, c0, 64)) =
                         make_uint2(0u, 0u);
                 }
@@ -619,11 +630,12 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
                     e1[c] = ex2(d2);
                     e2[c] = ex2(-d2);
                 }
-                st8(sm + Lay::X1, kmajor_off(r, c0, 128), kf[0] * e1[0], kf[1] * e1[1],
-                    kf[2] * e1[2], kf[3] * e1[3]);
+                if (!FAST)
+                    st8(sm + Lay::X1, kmajor_off(r, c0, 128), kf[0] * e1[0], kf[1] * e1[1],
+                        kf[2] * e1[2], kf[3] * e1[3]);
                 if (!SEG)
-                    st8(sm + Lay::X1, kmajor_off(64 + r, c0, 128), qf[0] * e1[0], qf[1] * e1[1],
-                        qf[2] * e1[2], qf[3] * e1[3]);
+                    st8(sm + Lay::X1, kmajor_off(FAST ? r : 64 + r, c0, 128), qf[0] * e1[0],
+                        qf[1] * e1[1], qf[2] * e1[2], qf[3] * e1[3]);
                 st8(sm + Lay::BT, kmajor_off(r, c0, 96), kf[0] * e2[0], kf[1] * e2[1],
                     kf[2] * e2[2], kf[3] * e2[3]);
                 if (r < 32)
@@ -650,6 +662,28 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
                 mma_bf16(tmem + TM_AP, kmajor_desc(x1, 128, s), kmajor_desc(bt, 96, s), id, s > 0);
             mma_commit(bar);
         }
+        if (FAST) {
+            // meanwhile: bf16 copy of the state (S^T scaled by gamma in TMEM afterwards), and
+            // the chunk's U'^T from the cache into the U accumulator
+            const int c0 = 32 * wg, r0 = 16 * wg;
+            stage_cols_tmem<2>(tq + TM_S + c0, tq + TM_SB + c0 / 2, c0, gam, true);
+            const uint8_t* ru = sm + Lay::RV + vbuf * 16384 + lrow * 128;
+            float v[16];
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const uint4 x = *reinterpret_cast<const uint4*>(ru + ((((r0 >> 3) + hh) ^ (lrow & 7)) << 4));
+                float lo4[4], hi4[4];
+                unpack_bf16x4(make_uint2(x.x, x.y), lo4);
+                unpack_bf16x4(make_uint2(x.z, x.w), hi4);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    v[8 * hh + i] = lo4[i];
+                    v[8 * hh + 4 + i] = hi4[i];
+                }
+            }
+            tmem_st16(tq + TM_U + r0, v);
+            tmem_st_wait();
+        }
         if (!(ok = wait_mma(bar, parity))) break;
 
         // ============ phase 2: masks, beta, (I + A)^-1, P
@@ -660,10 +694,11 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
             // rows r of A (lanes 0-63) and P (lanes 64-127); warp slice wg handles the 16
             // columns j in [16wg, 16wg+16).  Columns j < 32 of rows r >= 32 come from the
             // cross-half product (TMEM columns 64 + j).
-            const bool need_a = SEG || !tb_cache;  // A only feeds the inversion
-            if ((!SEG || quad < 2) && (quad >= 2 || need_a)) {
+            // MODE 2 needs only P, which it finds in rows 0-63 (q~ sits there in X1)
+            const bool need_a = !FAST;
+            if (FAST ? quad < 2 : (!SEG || quad < 2)) {
                 const int r = lrow & 63;
-                const bool isP = quad >= 2;
+                const bool isP = FAST || quad >= 2;
                 const bool lower_half = r < 32;  // warp-uniform
                 const int j0 = 16 * wg;
                 float x[16];
@@ -701,9 +736,10 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
-        if (SEG && tb_cache && tid == 0) {  // keep T diag(beta) for pass 3
-            bulk_store(tb_tile(t0), sm + Lay::TB, 8192);
-            bulk_commit();
+        // MODE 2: U'^T has gone to TMEM, so its buffer may receive the output gate's tile
+        if (FAST && gate_on && tid == 0) {
+            mbar_expect_tx(bar_gate, 16384);
+            tma_tile(sm + Lay::RV + vbuf * 16384, &maps.gate, 0, h, (int)t0, bar_gate);
         }
 
         // ============ phase 3: with TB = T diag(beta) and the per-half factors e^{rho_h}:
@@ -711,15 +747,10 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
         //   U'^T = V^T TB^T
         // X1's k rows serve as an MN-major operand (K rows = tokens, MN blocks 16 KB apart);
         // the v tile is used as TMA wrote it.
-        bool tb_ok = true;
-        if (!SEG && tb_cache && tid == 0) {
-            tb_ok = mbar_wait(bar_tb, tb_parity, &g_tc_status, ERR_WAIT_TIMEOUT);
-            tb_parity ^= 1u;
-        }
-        if (tid == 0 && tb_ok) {
+        if (!FAST) {  // MODE 2 has W^T and U'^T from the cache
+        if (tid == 0) {
             tc_fence_after();
-            const uint32_t x1 = smem_u32(sm + Lay::X1),
-                           tb = smem_u32(sm + ((!SEG && tb_cache) ? Lay::TBX : Lay::TB)),
+            const uint32_t x1 = smem_u32(sm + Lay::X1), tb = smem_u32(sm + Lay::TB),
                            rv = smem_u32(sm + Lay::RV + vbuf * 16384);
             constexpr uint32_t id = idesc_bf16(128, 64, true, false);
 #pragma unroll
@@ -750,11 +781,6 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
             tmem_st_wait();
         }
         if (!(ok = wait_mma(bar, parity))) break;
-        // TBX is consumed: the next chunk's T tile may come in
-        if (!SEG && tb_cache && tid == 0 && t0 + C < sg.t_end) {
-            mbar_expect_tx(bar_tb, 8192);
-            bulk_load(sm + Lay::TBX, tb_tile(t0 + C), 8192, bar_tb);
-        }
         // The v tile is consumed: the output gate's [64][128] tile (if any) goes into
         // its buffer now, for the epilogue.
         if (gate_on && tid == 0) {
@@ -765,9 +791,10 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
         // operand: K rows = c, MN = token r)
         {
             const int r0 = 16 * wg;  // tokens r0..r0+15 of this thread's channel row
-            float wa[16], wbv[16];
+            float wa[16], wbv[16], up[16];
             tmem_ld16(tq + TM_W + r0, wa);
             tmem_ld16(tq + TM_AP + r0, wbv);
+            if (SEG && wu_cache) tmem_ld16(tq + TM_U + r0, up);  // U' (before phase 5 changes it)
             tmem_wait16(wa);
             tmem_wait16(wbv);
             const float ea = eha[lrow], eb = ehb[lrow];
@@ -781,22 +808,48 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
                              pack_bf16(w[0], w[1]), pack_bf16(w[2], w[3]), pack_bf16(w[4], w[5]),
                              pack_bf16(w[6], w[7]));
             }
+            if (SEG && wu_cache) {  // U'^T, bf16, straight to the cache (row lrow = e)
+                tmem_wait16(up);
+                uint8_t* gu = wu_tile(t0) + 16384 + lrow * 128;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh)
+                    *reinterpret_cast<uint4*>(gu + ((((r0 >> 3) + hh) ^ (lrow & 7)) << 4)) =
+                        make_uint4(pack_bf16(up[8 * hh], up[8 * hh + 1]),
+                                   pack_bf16(up[8 * hh + 2], up[8 * hh + 3]),
+                                   pack_bf16(up[8 * hh + 4], up[8 * hh + 5]),
+                                   pack_bf16(up[8 * hh + 6], up[8 * hh + 7]));
+            }
         }
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
+        if (SEG && wu_cache && tid == 0) {  // keep W^T of the chunk for pass 3
+            bulk_store(wu_tile(t0), sm + Lay::WB, 16384);
+            bulk_commit();
+        }
+        }  // !FAST
 
         // ============ phase 5: U^T -= S^T W^T ; O^T = S^T Q~^T  (pass 1: U_M^T = -M^T W^T)
-        if (tid == 0) {
+        bool w_ok = true;
+        if (FAST && tid == 0) {  // this chunk's W^T from the cache
+            w_ok = mbar_wait(bar_w, w_parity, &g_tc_status, ERR_WAIT_TIMEOUT);
+            w_parity ^= 1u;
+        }
+        if (tid == 0 && w_ok) {
             tc_fence_after();
             const uint32_t sa = smem_u32(sm + Lay::SA), wb = smem_u32(sm + Lay::WB);
             constexpr uint32_t id_neg = idesc_bf16(128, 64, false, true, true);
             if (!SEG) {  // A = bf16 S^T from TMEM
                 const uint32_t qt = smem_u32(sm + Lay::QT);
                 constexpr uint32_t id = idesc_bf16(128, 64, false, false);
+                const uint32_t x1 = smem_u32(sm + Lay::X1);
 #pragma unroll
-                for (int s = 0; s < 8; ++s)
-                    mma_bf16_ts(tmem + TM_U, tmem + TM_SB + 8 * s, mnmajor_desc(wb, 128, s), id_neg, 1);
+                for (int s = 0; s < 8; ++s) {
+                    // MODE 2: K steps 0-3 at X1 + 8 KB, 4-7 at X1 + 24 KB (the cache's pieces)
+                    const uint64_t wd = FAST ? sdesc(x1 + (s < 4 ? 8192 : 24576) + 2048 * (s & 3), 128 * 128, 1024)
+                                             : mnmajor_desc(wb, 128, s);
+                    mma_bf16_ts(tmem + TM_U, tmem + TM_SB + 8 * s, wd, id_neg, 1);
+                }
 #pragma unroll
                 for (int s = 0; s < 8; ++s)
                     mma_bf16_ts(tmem + TM_O, tmem + TM_SB + 8 * s, kmajor_desc(qt, 64, s), id, s > 0);
@@ -813,6 +866,7 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
             mma_commit(bar);
         }
         if (!(ok = wait_mma(bar, parity))) break;
+        if (FAST && tid == 0 && t0 + C < sg.t_end) load_w(t0 + C);  // W^T consumed: the next one
 
         // ============ phase 6: U^T -> UA (bf16, K-major, 128 x 64); pass 1 also U_M^T -> UMA
         if (!SEG) {
@@ -913,7 +967,7 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
     }
 
     // ---- results of the segment
-    if (tid == 0 && (!SEG || tb_cache)) bulk_wait_all();  // output / T stores are complete
+    if (tid == 0 && (!SEG || wu_cache)) bulk_wait_all();  // output / cache stores are complete
     if (ok) {
         if (SEG) {  // slices 0-1: B^T, slices 2-3: M^T, 64 columns each
             const bool is_m = wg >= 2;
@@ -1157,13 +1211,16 @@ cudaError_t launch_tc(const TcArgs& a, const TcPlan& p, cudaStream_t stream, int
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
     if (dev >= kMaxDevices || !attr_set[dev][0]) {
-        err = cudaFuncSetAttribute(tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        err = cudaFuncSetAttribute(tc_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    (int)LayT<false>::BYTES);
+        if (err == cudaSuccess)
+            err = cudaFuncSetAttribute(tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)LayT<false>::BYTES);
         if (err == cudaSuccess)
             err = cudaFuncSetAttribute(seg_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        SCAN_SMEM);
         if (err == cudaSuccess)
-            err = cudaFuncSetAttribute(tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            err = cudaFuncSetAttribute(tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)LayT<true>::BYTES);
         if (err != cudaSuccess) return err;
         if (dev < kMaxDevices) attr_set[dev][0] = true;
@@ -1190,7 +1247,7 @@ cudaError_t launch_tc(const TcArgs& a, const TcPlan& p, cudaStream_t stream, int
     const dim3 grid((unsigned)p.max_units, (unsigned)a.H);
     if (p.segmented) {
         profile_mark(SLOT_PASS1, true, stream);
-        tc_kernel<true><<<grid, NT, LayT<true>::BYTES, stream>>>(a, maps);
+        tc_kernel<1><<<grid, NT, LayT<true>::BYTES, stream>>>(a, maps);
         profile_mark(SLOT_PASS1, false, stream);
         *launches += 1;
         if ((err = cudaGetLastError()) != cudaSuccess) return err;
@@ -1201,7 +1258,10 @@ cudaError_t launch_tc(const TcArgs& a, const TcPlan& p, cudaStream_t stream, int
         if ((err = cudaGetLastError()) != cudaSuccess) return err;
     }
     profile_mark(SLOT_PASS3, true, stream);
-    tc_kernel<false><<<grid, NT, LayT<false>::BYTES, stream>>>(a, maps);
+    if (a.wu)
+        tc_kernel<2><<<grid, NT, LayT<false>::BYTES, stream>>>(a, maps);
+    else
+        tc_kernel<0><<<grid, NT, LayT<false>::BYTES, stream>>>(a, maps);
     profile_mark(SLOT_PASS3, false, stream);
     *launches += 1;
     return cudaGetLastError();
@@ -1216,7 +1276,7 @@ cudaError_t launch_transition(const TcArgs& a_in, const TcPlan& p, float* out, c
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
     if (dev >= kMaxDevices || !attr_set[dev]) {
-        err = cudaFuncSetAttribute(tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        err = cudaFuncSetAttribute(tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    (int)LayT<true>::BYTES);
         if (err != cudaSuccess) return err;
         if (dev < kMaxDevices) attr_set[dev] = true;
@@ -1237,7 +1297,7 @@ cudaError_t launch_transition(const TcArgs& a_in, const TcPlan& p, float* out, c
     *launches += 1;
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     profile_mark(SLOT_PASS1, true, stream);
-    tc_kernel<true><<<dim3((unsigned)p.max_units, (unsigned)a.H), NT, LayT<true>::BYTES, stream>>>(
+    tc_kernel<1><<<dim3((unsigned)p.max_units, (unsigned)a.H), NT, LayT<true>::BYTES, stream>>>(
         a, maps);
     profile_mark(SLOT_PASS1, false, stream);
     *launches += 1;
