@@ -102,6 +102,7 @@ static_assert(LayT<false>::TS + 64 * 72 * 4 <= LayT<false>::R1, "As/Ts overflow"
 static_assert(LayT<false>::YS + 32 * 40 * 4 <= 32768 && LayT<false>::TB + 8192 <= 16384,
               "Ys/TB must sit in the q-row holes of X1");
 static_assert(LayT<false>::SA + 32768 <= LayT<false>::R1, "SA overflow");
+static_assert(LayT<true>::WB + 16384 == LayT<true>::UA, "pass 1 stores W^T and U'^T as one 32 KB copy");
 static_assert(LayT<true>::MA + 32768 <= LayT<true>::R1, "MA overflow");
 static_assert(LayT<false>::BYTES <= 232448 && LayT<true>::BYTES <= 232448, "shared memory");
 
@@ -808,23 +809,23 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
                              pack_bf16(w[0], w[1]), pack_bf16(w[2], w[3]), pack_bf16(w[4], w[5]),
                              pack_bf16(w[6], w[7]));
             }
-            if (SEG && wu_cache) {  // U'^T, bf16, straight to the cache (row lrow = e)
+            if (SEG && wu_cache) {  // U'^T (before phase 5 changes it), bf16, next to W^T in UA
                 tmem_wait16(up);
-                uint8_t* gu = wu_tile(t0) + 16384 + lrow * 128;
+                const uint32_t ru = smem_u32(sm + Lay::UA + lrow * 128);
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh)
-                    *reinterpret_cast<uint4*>(gu + ((((r0 >> 3) + hh) ^ (lrow & 7)) << 4)) =
-                        make_uint4(pack_bf16(up[8 * hh], up[8 * hh + 1]),
-                                   pack_bf16(up[8 * hh + 2], up[8 * hh + 3]),
-                                   pack_bf16(up[8 * hh + 4], up[8 * hh + 5]),
-                                   pack_bf16(up[8 * hh + 6], up[8 * hh + 7]));
+                    st_shared_v4(ru + ((((r0 >> 3) + hh) ^ (lrow & 7)) << 4),
+                                 pack_bf16(up[8 * hh], up[8 * hh + 1]),
+                                 pack_bf16(up[8 * hh + 2], up[8 * hh + 3]),
+                                 pack_bf16(up[8 * hh + 4], up[8 * hh + 5]),
+                                 pack_bf16(up[8 * hh + 6], up[8 * hh + 7]));
             }
         }
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
-        if (SEG && wu_cache && tid == 0) {  // keep W^T of the chunk for pass 3
-            bulk_store(wu_tile(t0), sm + Lay::WB, 16384);
+        if (SEG && wu_cache && tid == 0) {  // keep W^T and U'^T (WB, UA: 32 KB) for pass 3
+            bulk_store(wu_tile(t0), sm + Lay::WB, 32768);
             bulk_commit();
         }
         }  // !FAST
@@ -868,6 +869,10 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
         if (!(ok = wait_mma(bar, parity))) break;
         if (FAST && tid == 0 && t0 + C < sg.t_end) load_w(t0 + C);  // W^T consumed: the next one
 
+        if (SEG && wu_cache) {  // UA is about to be rewritten: the cache copy must have left it
+            if (tid == 0) bulk_wait_read();
+            __syncthreads();
+        }
         // ============ phase 6: U^T -> UA (bf16, K-major, 128 x 64); pass 1 also U_M^T -> UMA
         if (!SEG) {
             const int c0 = 16 * wg;
