@@ -307,8 +307,11 @@ __device__ __forceinline__ void warp_store16x8(float* dst, int ld, const float (
 //  3. T[32:64, 0:32] = -T_hi Z, written straight into TB.
 // The block products are tf32 warp MMAs with fp32 accumulation (T then enters
 // the chunk products as bf16).
+// `side(warp)` runs on warps 8-15 while warps 0-1 invert the diagonal blocks
+// (work that does not touch As, Ts, Ys or TB).
+template <typename Side>
 __device__ void invert_to_tb(const float* As, float* Ts, float* Ys, const float* beta,
-                             uint32_t tbp, int tid) {
+                             uint32_t tbp, int tid, Side side) {
     const int warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t4 = lane & 3;
     if (warp < 2) {
@@ -364,21 +367,23 @@ __device__ void invert_to_tb(const float* As, float* Ts, float* Ys, const float*
             warp_store16x8(Ts + (o + 16) * TS_LD + o + 8 * nt, TS_LD, d, -1.f, lane);
         }
         __syncwarp();
-        // 1c. TB for the half: 32 rows x 4 chunks of 8 columns
-#pragma unroll
-        for (int x = 0; x < 4; ++x) {
-            const int id = lane + 32 * x, r = o + (id >> 2), j8 = (o >> 3) + (id & 3);
-            const float* tr = Ts + r * TS_LD + 8 * j8;
-            const float* bj = beta + 8 * j8;
-            st_shared_v4(tbp + kmajor_chunk_off(r, j8, 64), pack_bf16(tr[0] * bj[0], tr[1] * bj[1]),
-                         pack_bf16(tr[2] * bj[2], tr[3] * bj[3]), pack_bf16(tr[4] * bj[4], tr[5] * bj[5]),
-                         pack_bf16(tr[6] * bj[6], tr[7] * bj[7]));
-        }
     } else if (warp < 6) {  // zero TB rows 0..31, columns 32..63: 128 chunks
         const int id = tid - 64, r = id >> 2, j8 = 4 + (id & 3);
         st_shared_v4(tbp + kmajor_chunk_off(r, j8, 64), 0u, 0u, 0u, 0u);
+    } else if (warp >= 8) {
+        side(warp);
     }
     __syncthreads();
+    // 1c (warps 8-15, beside step 2). TB of the two diagonal halves: 2 x 32 rows x 4
+    // chunks of 8 columns, one chunk per thread
+    if (warp >= 8) {
+        const int id = tid - 256, hf = id >> 7, r = 32 * hf + ((id >> 2) & 31), j8 = 4 * hf + (id & 3);
+        const float* tr = Ts + r * TS_LD + 8 * j8;
+        const float* bj = beta + 8 * j8;
+        st_shared_v4(tbp + kmajor_chunk_off(r, j8, 64), pack_bf16(tr[0] * bj[0], tr[1] * bj[1]),
+                     pack_bf16(tr[2] * bj[2], tr[3] * bj[3]), pack_bf16(tr[4] * bj[4], tr[5] * bj[5]),
+                     pack_bf16(tr[6] * bj[6], tr[7] * bj[7]));
+    }
     // 2. Z = A[32:64, 0:32] T_lo: warp (mt, nt) for warps 0-7
     const int mt = (warp >> 2) & 1, nt = warp & 3;
     if (warp < 8) {
@@ -732,7 +737,17 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
                 }
             }
             __syncthreads();
-            if (need_a) invert_to_tb(As, Ts, Ys, beta_s, smem_u32(sm + Lay::TB), tid);
+            if (need_a) {
+                // beside the diagonal inversions: pass 1 stages M (bf16 M^T -> MA, M scaled by
+                // gamma in TMEM) on warps 8-15, which own two 64-column slices per quadrant
+                invert_to_tb(As, Ts, Ys, beta_s, smem_u32(sm + Lay::TB), tid, [&](int w) {
+                    if (SEG) {
+                        const int c0 = 64 * ((w >> 2) - 2);
+                        stage_cols<4>(tq + TM_M + c0, sm + Lay::MA, 128, lrow, c0, gam, true);
+                        tmem_st_wait();
+                    }
+                });
+            }
         }
         fence_async_smem();
         tc_fence_before();
@@ -767,18 +782,15 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
                 mma_bf16(tmem + TM_U, mnmajor_desc(rv, 64, s), kmajor_desc(tb, 64, s), id, s > 0);
             mma_commit(bar);
         }
-        // meanwhile: bf16 copy of the state into SA (and MA), state scaled by gamma in
-        // TMEM.  Pass 3: slice wg takes columns 32wg..32wg+31.  Pass 1: slices 0-1 take
-        // B, slices 2-3 take M, 64 columns each.
+        // meanwhile: bf16 copy of the state, state scaled by gamma in TMEM.  Slice wg
+        // takes columns 32wg..32wg+31 (pass 3: S^T into TMEM; pass 1: B^T into SA).
         if (!SEG) {
             const int c0 = 32 * wg;
             stage_cols_tmem<2>(tq + TM_S + c0, tq + TM_SB + c0 / 2, c0, gam, true);
             tmem_st_wait();
-        } else {
-            const bool is_m = wg >= 2;
-            const int c0 = 64 * (wg & 1);
-            stage_cols<4>(tq + (is_m ? TM_M : TM_B) + c0, sm + (is_m ? Lay::MA : Lay::SA), 128, lrow,
-                          c0, gam, true);
+        } else {  // pass 1: B (M was staged beside the inversion)
+            const int c0 = 32 * wg;
+            stage_cols<2>(tq + TM_B + c0, sm + Lay::SA, 128, lrow, c0, gam, true);
             tmem_st_wait();
         }
         if (!(ok = wait_mma(bar, parity))) break;
