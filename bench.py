@@ -304,25 +304,25 @@ def segment_plan(inp, sms=148):
 
 
 def kernel_algorithmic_bytes(name, inp, path_bytes):
-    """Minimum bytes one launch of kernel `name` must move.
+    """Minimum bytes one launch of kernel `name` must move for what it computes.
 
     pass 3 (forward) reads every input once and writes o and the states: the
-    whole path's algorithmic bytes.  Pass 1 (segment transitions) reads k, v,
-    log alpha and beta of every token in a segment that has a successor and
-    writes one (B, M) pair (2 x 128 x 128 fp32) per such segment and head."""
+    whole path's algorithmic bytes.  Pass 1 (segment transitions) runs over
+    every segment when sequences are cut (it also leaves each chunk's W and U'
+    for pass 3): it reads k, v, log alpha and beta of every token and writes
+    one (B, M) pair (2 x 128 x 128 fp32) per segment and head.  The W/U' cache
+    (512 B per token-head each way) is implementation traffic, not counted."""
     if name != "tc_pass1_transitions":
         return path_bytes
     seg, cut = segment_plan(inp)
     if not cut:
         return 0
     per_tok = inp.H * (inp.dk * 2 + inp.dv * 2 + inp.dk * 4 + 4)
-    toks, segs = 0, 0
+    segs = 0
     for L in inp.seq_lens:
         nch = (int(L) + 63) // 64
-        G = max(1, (nch + seg - 1) // seg)
-        toks += min(int(L), (G - 1) * seg * 64)
-        segs += G - 1
-    return toks * per_tok + segs * inp.H * 2 * inp.dk * inp.dv * 4
+        segs += max(1, (nch + seg - 1) // seg)
+    return inp.tokens * per_tok + segs * inp.H * 2 * inp.dk * inp.dv * 4
 
 
 # ------------------------------------------------------------------ traffic record
