@@ -346,8 +346,9 @@ def recorded_traffic(kernel_tag: str):
 # ------------------------------------------------------------------ context parallel, emulated
 def run_cp_emulation(args):
     """Each of W virtual ranks owns T/W tokens of every sequence.  Rank r runs
-    kda_transition on its span, kda_apply_transitions on the transitions of
-    ranks < r (the all-gather's result), then kda_fwd from that state.  On one
+    kda_span_transition on its span, kda_apply_transitions on the transitions of
+    ranks < r (the all-gather's result), then kda_span_forward from that state
+    (which reuses the transition's per-segment work).  On one
     GPU the ranks run one after another; each rank's work is timed with CUDA
     events, and a W-GPU run would take the slowest rank's time plus one
     all-gather of W x B x H x 128 KiB (estimated here at the measured 770 GB/s
@@ -370,14 +371,16 @@ def run_cp_emulation(args):
              for r in range(W)]
     del full
     stream = torch.cuda.current_stream(dev)
-    trans = [kda.kda_transition(s["k"], s["v"], s["log_alpha"], s["beta"]) for s in spans]
+    ws = [kda.span_workspace(s["k"]) for s in spans]
+    trans = [kda.kda_span_transition(s["k"], s["v"], s["log_alpha"], s["beta"], w)
+             for s, w in zip(spans, ws)]
     gathered = torch.stack(trans)
 
-    def rank_step(r):
+    def rank_step(r):  # transition (kept work in ws[r]), incoming state, forward
         s = spans[r]
-        kda.kda_transition(s["k"], s["v"], s["log_alpha"], s["beta"], out=trans[r])
+        kda.kda_span_transition(s["k"], s["v"], s["log_alpha"], s["beta"], ws[r], out=trans[r])
         s_in = kda.kda_apply_transitions(gathered[:r], s0)
-        return kda.kda_fwd(**s, initial_state=s_in)
+        return kda.kda_span_forward(s["q"], s["k"], s["v"], s["log_alpha"], s["beta"], ws[r], s_in)
 
     per_rank = []
     for r in range(W):

@@ -18,7 +18,8 @@ import ctypes
 import os
 
 __all__ = ["kda_fwd", "kda_fwd_host", "kda_fwd_noalloc", "kda_fwd_snap", "kda_decode",
-           "kda_transition", "kda_apply_transitions", "KDAError", "library_path", "load_library",
+           "kda_transition", "kda_apply_transitions", "span_workspace", "kda_span_transition",
+           "kda_span_forward", "KDAError", "library_path", "load_library",
            "last_launch_count", "last_path", "check_device", "profile_enable", "profile_read",
            "STATUS"]
 
@@ -87,6 +88,13 @@ def load_library():
         lib.kda_apply_transitions.argtypes = [p, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                               p, p, p]
         lib.kda_apply_transitions.restype = ctypes.c_int
+        lib.kda_span_workspace_bytes.argtypes = [ctypes.POINTER(Dims)]
+        lib.kda_span_workspace_bytes.restype = ctypes.c_size_t
+        lib.kda_span_transition.argtypes = [p, p, p, p, ctypes.POINTER(Dims), p, ctypes.c_size_t, p, p]
+        lib.kda_span_transition.restype = ctypes.c_int
+        lib.kda_span_forward.argtypes = [p, p, p, p, p, p, p, p, ctypes.POINTER(Dims), p,
+                                         ctypes.c_size_t, p]
+        lib.kda_span_forward.restype = ctypes.c_int
         lib.kda_decode.restype = ctypes.c_int
         lib.kda_status_string.argtypes = [ctypes.c_int]
         lib.kda_status_string.restype = ctypes.c_char_p
@@ -382,3 +390,57 @@ def kda_apply_transitions(trans, initial_state=None, out=None, stream=None):
                                      ptr(initial_state), ptr(out),
                                      ctypes.c_void_p(stream.cuda_stream)))
     return out
+
+
+def _span_dims(k):
+    import torch
+    if k.dim() != 4:
+        raise ValueError("k must be [B,T,H,128]")
+    B, T, H, dk = k.shape
+    return Dims(B, T, H, dk, dk, 0, KDA_BF16 if k.dtype == torch.bfloat16 else KDA_F32)
+
+
+def span_workspace(k):
+    """A device buffer for kda_span_transition / kda_span_forward on spans shaped like k."""
+    import torch
+    n = int(load_library().kda_span_workspace_bytes(ctypes.byref(_span_dims(k))))
+    if n == 0:
+        raise ValueError("invalid span dims")
+    return torch.empty(n, dtype=torch.uint8, device=k.device)
+
+
+def kda_span_transition(k, v, log_alpha, beta, workspace, out=None, stream=None):
+    """kda_transition that also leaves the span's segment transitions and W/U' in
+    ``workspace`` (from :func:`span_workspace`) for :func:`kda_span_forward`."""
+    import torch
+    lib = load_library()
+    d = _span_dims(k)
+    if out is None:
+        out = torch.empty((d.B, d.H, 2, 128, 128), dtype=torch.float32, device=k.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(k.device)
+    ptr = lambda t: ctypes.c_void_p(t.data_ptr())
+    _check(lib.kda_span_transition(ptr(k), ptr(v), ptr(log_alpha), ptr(beta), ctypes.byref(d),
+                                   ptr(workspace), workspace.numel(), ptr(out),
+                                   ctypes.c_void_p(stream.cuda_stream)))
+    return out
+
+
+def kda_span_forward(q, k, v, log_alpha, beta, workspace, initial_state=None, out=None,
+                     final_state=None, stream=None, want_final: bool = True):
+    """kda_fwd on a span whose kda_span_transition filled ``workspace``."""
+    import torch
+    lib = load_library()
+    d = _dims(tuple(q.shape), tuple(v.shape), None, 0, q.dtype == torch.bfloat16)
+    if out is None:
+        out = torch.empty(tuple(q.shape[:-1]) + (d.d_v,), dtype=q.dtype, device=q.device)
+    if final_state is None and want_final:
+        final_state = torch.empty((d.B, d.H, d.d_k, d.d_v), dtype=torch.float32, device=q.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    ptr = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
+    _check(lib.kda_span_forward(ptr(q), ptr(k), ptr(v), ptr(log_alpha), ptr(beta),
+                                ptr(initial_state), ptr(out), ptr(final_state), ctypes.byref(d),
+                                ptr(workspace), workspace.numel(),
+                                ctypes.c_void_p(stream.cuda_stream)))
+    return out, final_state

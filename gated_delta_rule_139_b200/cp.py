@@ -17,9 +17,10 @@ rank).  Every rank passes the same ``initial_state`` (the state entering span
 its span; on the last rank that is the sequences' final state.
 
 The collective is a plain ``torch.distributed.all_gather`` (NCCL between GPUs);
-the kernels are the library's: :func:`kda_transition`, then
+the kernels are the library's: :func:`kda_span_transition`, then
 :func:`kda_apply_transitions` on the gathered maps of the ranks before this
-one, then :func:`kda_fwd` from that state.
+one, then :func:`kda_span_forward` from that state, which reuses the
+transition step's per-segment work.
 """
 from __future__ import annotations
 
@@ -29,21 +30,33 @@ from typing import Callable
 
 @dataclass
 class SpanOps:
-    """The three per-rank steps.  ``transition`` returns one opaque tensor per
-    rank (all ranks the same shape); ``apply`` takes the stack of the earlier
-    ranks' tensors ([r, ...], r may be 0) and the initial state."""
+    """The three per-rank steps.  ``transition(k, v, log_alpha, beta)`` returns
+    (one tensor to exchange, all ranks the same shape; a context the forward
+    step may reuse); ``apply(prior, initial_state)`` takes the stack of the
+    earlier ranks' tensors ([r, ...], r may be 0); ``forward(q, k, v,
+    log_alpha, beta, s_in, out_gate, context)`` returns (out, end state)."""
     transition: Callable
     apply: Callable
     forward: Callable
 
 
 def library_ops() -> SpanOps:
-    from . import kda_apply_transitions, kda_fwd, kda_transition
+    """The library's kernels.  The transition step keeps its segment transitions
+    and per-chunk W, U' in a workspace, so the forward step does not compute
+    them again (kda_span_transition / kda_span_forward)."""
+    from . import (kda_apply_transitions, kda_fwd, kda_span_forward, kda_span_transition,
+                   span_workspace)
 
-    def forward(q, k, v, log_alpha, beta, s_in, out_gate):
-        return kda_fwd(q, k, v, log_alpha, beta, s_in, out_gate=out_gate)
+    def transition(k, v, log_alpha, beta):
+        ws = span_workspace(k)
+        return kda_span_transition(k, v, log_alpha, beta, ws), ws
 
-    return SpanOps(transition=lambda k, v, la, be: kda_transition(k, v, la, be),
+    def forward(q, k, v, log_alpha, beta, s_in, out_gate, ws):
+        if out_gate is not None:  # the gated epilogue lives in the full forward
+            return kda_fwd(q, k, v, log_alpha, beta, s_in, out_gate=out_gate)
+        return kda_span_forward(q, k, v, log_alpha, beta, ws, s_in)
+
+    return SpanOps(transition=transition,
                    apply=lambda prior, s0: kda_apply_transitions(prior, s0),
                    forward=forward)
 
@@ -57,9 +70,9 @@ def cp_prefill(q, k, v, log_alpha, beta, initial_state=None, group=None, out_gat
     ops = ops or library_ops()
     rank = dist.get_rank(group)
     world = dist.get_world_size(group)
-    trans = ops.transition(k, v, log_alpha, beta)
+    trans, ctx = ops.transition(k, v, log_alpha, beta)
     gathered = [torch.empty_like(trans) for _ in range(world)]
     dist.all_gather(gathered, trans.contiguous(), group=group)
     prior = torch.stack(gathered[:rank]) if rank else trans.new_empty((0,) + tuple(trans.shape))
     s_in = ops.apply(prior, initial_state)
-    return ops.forward(q, k, v, log_alpha, beta, s_in, out_gate)
+    return ops.forward(q, k, v, log_alpha, beta, s_in, out_gate, ctx)

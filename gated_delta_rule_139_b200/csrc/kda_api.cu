@@ -337,6 +337,111 @@ size_t tc_scratch_bytes(const kda::FwdArgs& a, const kda::TcPlan& p, size_t* b_s
     return *b_segs + *b_off + *b_trans + b_sin;
 }
 
+// Workspace of a span (segment table, per-segment transitions and incoming
+// states, W/U' cache) for the segment plan of the dims: offsets into one buffer.
+struct SpanWs {
+    kda::TcPlan p;
+    size_t segs, off, trans, sin, wu, total;
+};
+
+SpanWs span_layout(const kda::FwdArgs& a) {
+    SpanWs w;
+    w.p = plan_segments(a);
+    const size_t st = (size_t)128 * 128 * sizeof(float);
+    size_t o = 0;
+    auto take = [&](size_t b) {
+        const size_t at = o;
+        o += (b + 255) & ~(size_t)255;
+        return at;
+    };
+    w.segs = take((size_t)w.p.max_units * sizeof(kda::SegEntry));
+    w.off = take((size_t)(a.N + 1) * 4 + 4);
+    w.trans = take((size_t)w.p.max_units * a.H * 2 * st);
+    w.sin = take((size_t)w.p.max_units * a.H * st);
+    w.wu = take((size_t)w.p.max_units * a.H * w.p.seg_chunks * 32768);
+    w.total = o;
+    return w;
+}
+
+kda::TcArgs span_args(const kda::FwdArgs& a, const SpanWs& w, char* ws) {
+    kda::TcArgs t{};
+    t.k = a.k;
+    t.v = a.v;
+    t.log_alpha = a.log_alpha;
+    t.beta = a.beta;
+    t.B = a.B;
+    t.T = a.T;
+    t.H = a.H;
+    t.N = a.N;
+    t.segs = (kda::SegEntry*)(ws + w.segs);
+    t.seg_off = (int32_t*)(ws + w.off);
+    t.n_units = t.seg_off + a.N + 1;
+    t.trans = (float*)(ws + w.trans);
+    t.sin = (float*)(ws + w.sin);
+    t.wu = (uint8_t*)(ws + w.wu);
+    t.seg_chunks = w.p.seg_chunks;
+    t.trans_all = 1;
+    return t;
+}
+
+kda_status check_workspace(const void* ws, size_t bytes, size_t need) {
+    if (!ws) return fail(KDA_ERR_INVALID_ARG, "workspace is NULL");
+    if ((uintptr_t)ws & 255u) return fail(KDA_ERR_MISALIGNED, "workspace is not 256-byte aligned");
+    if (bytes < need)
+        return fail(KDA_ERR_INVALID_ARG, "workspace holds %zu bytes, the span needs %zu", bytes, need);
+    return KDA_OK;
+}
+
+// Arguments of a span transition (k, v, log_alpha, beta; bf16, d = 128, no cu_seqlens).
+kda_status validate_span_inputs(const void* k, const void* v, const float* log_alpha,
+                                const float* beta, const kda_dims* d, const float* trans,
+                                kda::FwdArgs* a) {
+    if (!d) return fail(KDA_ERR_INVALID_ARG, "dims is NULL");
+    if (d->B < 1 || d->T < 0 || d->H < 1)
+        return fail(KDA_ERR_INVALID_ARG, "need B >= 1, T >= 0, H >= 1 (got B=%d T=%d H=%d)",
+                    d->B, d->T, d->H);
+    if (d->qkv_dtype != KDA_F32 && d->qkv_dtype != KDA_BF16)
+        return fail(KDA_ERR_INVALID_ARG, "qkv_dtype must be KDA_F32 or KDA_BF16");
+    if (d->d_k != 128 || d->d_v != 128 || d->qkv_dtype != KDA_BF16)
+        return fail(KDA_ERR_UNSUPPORTED, "span transitions need bf16 k/v with d_k = d_v = 128");
+    const int64_t tokens = (int64_t)d->B * d->T;
+    if (!trans) return fail(KDA_ERR_INVALID_ARG, "trans must be non-NULL");
+    if (tokens > 0 && (!k || !v || !log_alpha || !beta))
+        return fail(KDA_ERR_INVALID_ARG, "k, v, log_alpha and beta must be non-NULL");
+    const void* ptrs[] = {k, v, log_alpha, beta, trans};
+    const char* names[] = {"k", "v", "log_alpha", "beta", "trans"};
+    for (int i = 0; i < 5; ++i)
+        if (ptrs[i] && ((uintptr_t)ptrs[i] & 15u))
+            return fail(KDA_ERR_MISALIGNED, "%s is not 16-byte aligned", names[i]);
+    const int64_t n = tokens * d->H * 128;
+    const Range in[] = {{(uintptr_t)k, (uintptr_t)k + (k ? n * 2 : 0), "k"},
+                        {(uintptr_t)v, (uintptr_t)v + (v ? n * 2 : 0), "v"},
+                        {(uintptr_t)log_alpha, (uintptr_t)log_alpha + (log_alpha ? n * 4 : 0),
+                         "log_alpha"},
+                        {(uintptr_t)beta, (uintptr_t)beta + (beta ? tokens * d->H * 4 : 0), "beta"}};
+    const Range rt = {(uintptr_t)trans, (uintptr_t)trans + (uintptr_t)d->B * d->H * 2 * 128 * 128 * 4,
+                      "trans"};
+    for (const Range& r : in)
+        if (overlaps(rt, r)) return fail(KDA_ERR_ALIAS, "trans overlaps %s", r.name);
+    a->q = nullptr;
+    a->k = k;
+    a->v = v;
+    a->log_alpha = log_alpha;
+    a->beta = beta;
+    a->s0 = nullptr;
+    a->cu = nullptr;
+    a->out = nullptr;
+    a->s_final = nullptr;
+    a->B = d->B;
+    a->T = d->T;
+    a->H = d->H;
+    a->dk = 128;
+    a->dv = 128;
+    a->N = d->B;
+    a->bf16 = 1;
+    return KDA_OK;
+}
+
 }  // namespace
 
 void kda::profile_mark(int slot, bool begin, cudaStream_t stream) {
@@ -689,6 +794,96 @@ kda_status kda_transition(const void* k, const void* v, const float* log_alpha,
     g_last_path = "tc";
     e = kda::launch_transition(t, p, trans, cs, &launches);
     cudaFreeAsync(ws, cs);
+    g_last_launches = launches;
+    if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+    return KDA_OK;
+}
+
+size_t kda_span_workspace_bytes(const kda_dims* d) {
+    if (!d || d->B < 1 || d->T < 0 || d->H < 1) return 0;
+    kda::FwdArgs a;
+    a.B = d->B;
+    a.T = d->T;
+    a.H = d->H;
+    a.dk = a.dv = 128;
+    a.N = d->B;
+    a.cu = nullptr;
+    return span_layout(a).total;
+}
+
+kda_status kda_span_transition(const void* k, const void* v, const float* log_alpha,
+                               const float* beta, const kda_dims* d, void* workspace,
+                               size_t workspace_bytes, float* trans, void* stream) {
+    g_last_error[0] = 0;
+    g_last_launches = 0;
+    g_last_path = "";
+    kda::FwdArgs a;
+    kda_status st = validate_span_inputs(k, v, log_alpha, beta, d, trans, &a);
+    if (st != KDA_OK) return st;
+    const SpanWs w = span_layout(a);
+    st = check_workspace(workspace, workspace_bytes, w.total);
+    if (st != KDA_OK) return st;
+    const int64_t tokens = (int64_t)a.B * a.T, n = tokens * a.H * 128;
+    const Range rw = {(uintptr_t)workspace, (uintptr_t)workspace + w.total, "workspace"};
+    const Range other[] = {{(uintptr_t)k, (uintptr_t)k + (k ? n * 2 : 0), "k"},
+                           {(uintptr_t)v, (uintptr_t)v + (v ? n * 2 : 0), "v"},
+                           {(uintptr_t)log_alpha, (uintptr_t)log_alpha + (log_alpha ? n * 4 : 0),
+                            "log_alpha"},
+                           {(uintptr_t)beta, (uintptr_t)beta + (beta ? tokens * a.H * 4 : 0), "beta"},
+                           {(uintptr_t)trans, (uintptr_t)trans + (uintptr_t)a.B * a.H * 2 * 128 * 128 * 4,
+                            "trans"}};
+    for (const Range& r : other)
+        if (overlaps(rw, r)) return fail(KDA_ERR_ALIAS, "workspace overlaps %s", r.name);
+    const void* wp[] = {k, v, log_alpha, beta, trans, workspace};
+    const char* wn[] = {"k", "v", "log_alpha", "beta", "trans", "workspace"};
+    st = check_accessible(wp, wn, 6);
+    if (st != KDA_OK) return st;
+    kda::TcArgs t = span_args(a, w, (char*)workspace);
+    int launches = 0;
+    g_last_path = "tc";
+    cudaError_t e = kda::launch_transition(t, w.p, trans, (cudaStream_t)stream, &launches);
+    g_last_launches = launches;
+    if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+    return KDA_OK;
+}
+
+kda_status kda_span_forward(const void* q, const void* k, const void* v, const float* log_alpha,
+                            const float* beta, const float* initial_state, void* out,
+                            float* final_state, const kda_dims* d, const void* workspace,
+                            size_t workspace_bytes, void* stream) {
+    g_last_error[0] = 0;
+    g_last_launches = 0;
+    g_last_path = "";
+    kda::FwdArgs a;
+    kda_status st = validate(q, k, v, log_alpha, beta, initial_state, nullptr, kda::kChunk, out,
+                             final_state, d, true, &a);
+    if (st != KDA_OK) return st;
+    if (!(a.bf16 && a.dk == 128 && a.dv == 128))
+        return fail(KDA_ERR_UNSUPPORTED, "kda_span_forward needs bf16 q/k/v with d_k = d_v = 128");
+    const SpanWs w = span_layout(a);
+    st = check_workspace(workspace, workspace_bytes, w.total);
+    if (st != KDA_OK) return st;
+    const int64_t tokens = (int64_t)a.B * a.T;
+    const Range rw = {(uintptr_t)workspace, (uintptr_t)workspace + w.total, "workspace"};
+    const Range outs[] = {{(uintptr_t)out, (uintptr_t)out + (out ? tokens * a.H * a.dv * 2 : 0), "out"},
+                          {(uintptr_t)final_state,
+                           (uintptr_t)final_state + (final_state ? (uintptr_t)a.N * a.H * 128 * 128 * 4 : 0),
+                           "final_state"}};
+    for (const Range& r : outs)
+        if (overlaps(rw, r)) return fail(KDA_ERR_ALIAS, "workspace overlaps %s", r.name);
+    const void* wp[] = {workspace};
+    const char* wn[] = {"workspace"};
+    st = check_accessible(wp, wn, 1);
+    if (st != KDA_OK) return st;
+    if ((int64_t)a.N * a.H == 0) return KDA_OK;
+    kda::TcArgs t = span_args(a, w, (char*)workspace);
+    t.q = q;
+    t.s0 = initial_state;
+    t.out = out;
+    t.s_final = final_state;
+    int launches = 0;
+    g_last_path = "tc";
+    cudaError_t e = kda::launch_tc(t, w.p, (cudaStream_t)stream, &launches, /*from_cache=*/true);
     g_last_launches = launches;
     if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
     return KDA_OK;

@@ -96,8 +96,11 @@ struct TcPlan {
     bool segmented;   // some sequence may have more than one segment
 };
 
-// bf16 q/k/v with d_k = d_v = 128: tcgen05 tensor-core path.
-cudaError_t launch_tc(const TcArgs& a, const TcPlan& p, cudaStream_t stream, int* launches);
+// bf16 q/k/v with d_k = d_v = 128: tcgen05 tensor-core path.  from_cache: the
+// segment table, the transitions and the W/U' cache of this plan are already in
+// a's workspace (left by launch_transition), so only the scan and pass 3 run.
+cudaError_t launch_tc(const TcArgs& a, const TcPlan& p, cudaStream_t stream, int* launches,
+                      bool from_cache = false);
 
 // Chain of affine state maps S -> M S + B, in the transposed layout of the
 // library's transitions (entry [2][128][128]: B^T, then M^T; S^T_out = S^T_in M^T

@@ -1222,7 +1222,8 @@ cudaError_t tc_take_status(int* code) {
     return e;
 }
 
-cudaError_t launch_tc(const TcArgs& a, const TcPlan& p, cudaStream_t stream, int* launches) {
+cudaError_t launch_tc(const TcArgs& a, const TcPlan& p, cudaStream_t stream, int* launches,
+                      bool from_cache) {
     static bool attr_set[kMaxDevices][2] = {};
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
@@ -1255,19 +1256,23 @@ cudaError_t launch_tc(const TcArgs& a, const TcPlan& p, cudaStream_t stream, int
                 cudaSuccess)
             return err;
     }
-    profile_mark(SLOT_SETUP, true, stream);
-    seg_setup_kernel<<<1, 1024, 0, stream>>>(a.cu, a.N, a.T, p.seg_chunks, p.max_units, a.segs,
-                                             a.seg_off, a.n_units);
-    profile_mark(SLOT_SETUP, false, stream);
-    *launches += 1;
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
     const dim3 grid((unsigned)p.max_units, (unsigned)a.H);
-    if (p.segmented) {
-        profile_mark(SLOT_PASS1, true, stream);
-        tc_kernel<1><<<grid, NT, LayT<true>::BYTES, stream>>>(a, maps);
-        profile_mark(SLOT_PASS1, false, stream);
+    if (!from_cache) {  // else the segment table, transitions and W/U' cache are in place
+        profile_mark(SLOT_SETUP, true, stream);
+        seg_setup_kernel<<<1, 1024, 0, stream>>>(a.cu, a.N, a.T, p.seg_chunks, p.max_units, a.segs,
+                                                 a.seg_off, a.n_units);
+        profile_mark(SLOT_SETUP, false, stream);
         *launches += 1;
         if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    }
+    if (p.segmented) {
+        if (!from_cache) {
+            profile_mark(SLOT_PASS1, true, stream);
+            tc_kernel<1><<<grid, NT, LayT<true>::BYTES, stream>>>(a, maps);
+            profile_mark(SLOT_PASS1, false, stream);
+            *launches += 1;
+            if ((err = cudaGetLastError()) != cudaSuccess) return err;
+        }
         profile_mark(SLOT_SCAN, true, stream);
         seg_scan_kernel<<<dim3((unsigned)a.N, (unsigned)a.H, D / 16), 256, SCAN_SMEM, stream>>>(a);
         profile_mark(SLOT_SCAN, false, stream);

@@ -311,6 +311,35 @@ kda_status kda_transition(const void* k, const void* v, const float* log_alpha,
 kda_status kda_apply_transitions(const float* trans, int32_t count, int32_t B, int32_t H,
                                  const float* initial_state, float* state_out, void* stream);
 
+/*
+ * Context-parallel spans with shared work.  A rank that holds one span of B
+ * sequences first computes the span's transition (to exchange), then -- once it
+ * knows its incoming state -- the span's forward pass.  Both need the same
+ * per-segment transitions and per-chunk W, U' (see kda_fwd_ex), so the
+ * transition call can leave them in a caller-owned workspace for the forward
+ * call, which then runs only the segment scan and the output pass.
+ *
+ * kda_span_workspace_bytes: bytes of that workspace for these dims (B, T, H;
+ *   d_k = d_v = 128, bf16, no cu_seqlens); 0 for invalid dims.
+ * kda_span_transition: kda_transition that also fills `workspace` (device,
+ *   256-byte aligned, at least kda_span_workspace_bytes, not overlapping any
+ *   argument).
+ * kda_span_forward: kda_fwd on the same span (same k, v, log_alpha, beta and
+ *   dims; q, initial_state, out, final_state as in kda_fwd) that takes the
+ *   workspace's contents instead of recomputing them.  Results equal kda_fwd's
+ *   bit for bit.  If the workspace was not filled by kda_span_transition on the
+ *   same inputs the results are undefined.  It reads the workspace only, so one
+ *   transition may serve several forward calls (e.g. retries).
+ */
+size_t kda_span_workspace_bytes(const kda_dims* dims);
+kda_status kda_span_transition(const void* k, const void* v, const float* log_alpha,
+                               const float* beta, const kda_dims* dims, void* workspace,
+                               size_t workspace_bytes, float* trans, void* stream);
+kda_status kda_span_forward(const void* q, const void* k, const void* v, const float* log_alpha,
+                            const float* beta, const float* initial_state, void* out,
+                            float* final_state, const kda_dims* dims, const void* workspace,
+                            size_t workspace_bytes, void* stream);
+
 /* Static description of a status code. */
 const char* kda_status_string(kda_status s);
 

@@ -226,3 +226,34 @@ def test_apply_transitions_rejects_bad_arguments():
     assert call(out=FAKE + (2 << 30) + 4) == "KDA_ERR_MISALIGNED"
     assert call(out=FAKE + 4096) == "KDA_ERR_ALIAS"  # state_out inside trans
     assert call(out=FAKE + (1 << 30) + 4096) == "KDA_ERR_ALIAS"  # partial overlap with s0
+
+
+# ---------------------------------------------------------------- span workspace (context parallel)
+def test_span_workspace_size_and_bad_arguments():
+    lib = kda.load_library()
+    P = lambda x: None if x is None else ctypes.c_void_p(x)
+    n = lib.kda_span_workspace_bytes(ctypes.byref(D(B=1, T=1 << 16, H=8)))
+    assert n > 0 and n % 256 == 0
+    assert lib.kda_span_workspace_bytes(ctypes.byref(D(B=0))) == 0
+    assert lib.kda_span_workspace_bytes(None) == 0
+
+    def trans_call(ws=FAKE + (8 << 30), nbytes=n, d=None):
+        rc = lib.kda_span_transition(P(FAKE), P(FAKE + (1 << 30)), P(FAKE + (2 << 30)),
+                                     P(FAKE + (3 << 30)), ctypes.byref(d or D(T=1 << 16, H=8)),
+                                     P(ws), nbytes, P(FAKE + (4 << 30)), None)
+        return kda.STATUS[rc]
+
+    assert trans_call(ws=None) == "KDA_ERR_INVALID_ARG"
+    assert trans_call(ws=FAKE + (8 << 30) + 16) == "KDA_ERR_MISALIGNED"
+    assert trans_call(nbytes=n - 256) == "KDA_ERR_INVALID_ARG"
+    assert trans_call(ws=FAKE + (1 << 30)) == "KDA_ERR_ALIAS"  # workspace over v
+    assert trans_call(d=D(T=1 << 16, H=8, dk=64, dv=64)) == "KDA_ERR_UNSUPPORTED"
+
+    def fwd_call(ws=FAKE + (8 << 30), nbytes=n, d=None):
+        rc = lib.kda_span_forward(P(FAKE), P(FAKE + (1 << 30)), P(FAKE + (2 << 30)),
+                                  P(FAKE + (3 << 30)), P(FAKE + (4 << 30)), None,
+                                  P(FAKE + (5 << 30)), None, ctypes.byref(d or D(T=1 << 16, H=8)),
+                                  P(ws), nbytes, None)
+        return kda.STATUS[rc]
+
+    assert fwd_call(d=D(T=1 << 16, H=8, dt=0)) in ("KDA_ERR_UNSUPPORTED", "KDA_ERR_INVALID_ARG")

@@ -48,7 +48,7 @@ def _oracle_ops():
             e[:, :, i, 0] = 1.0
             _, s = oracle.recurrent(initial_state=e, **kw)
             m[:, :, :, i] = s[:, :, :, 0] - b[:, :, :, 0]
-        return torch.from_numpy(np.concatenate([m, b], axis=3))  # [B,H,dk,dk+dv] = [M | B]
+        return torch.from_numpy(np.concatenate([m, b], axis=3)), None  # [B,H,dk,dk+dv] = [M | B]
 
     def apply(prior, s0):
         s = np.zeros((B, H, DK, DV)) if s0 is None else s0.numpy().astype(np.float64)
@@ -57,7 +57,7 @@ def _oracle_ops():
             s = np.einsum("bhij,bhjv->bhiv", m, s) + b
         return s
 
-    def forward(q, k, v, la, be, s_in, gate):
+    def forward(q, k, v, la, be, s_in, gate, ctx):
         o, s = oracle.recurrent(npy(q), npy(k), npy(v), npy(la), npy(be),
                                 s_in.astype(np.float32), o_tokens=None)
         return torch.from_numpy(o), torch.from_numpy(s)

@@ -84,7 +84,8 @@ def test_context_parallel_prefill_emulated_on_one_gpu(world):
     """Virtual ranks one after another on one GPU: their concatenated outputs
     and the last rank's state match the oracle over the whole sequences."""
     import torch
-    from gated_delta_rule_139_b200 import kda_apply_transitions, kda_fwd, kda_transition
+    from gated_delta_rule_139_b200 import (kda_apply_transitions, kda_span_forward,
+                                           kda_span_transition, span_workspace)
     span = 64 * 5 + 7
     inp = make_inputs(2, span * world, 2, 128, 128, bf16=True, seed=403 + world,
                       state_sigma=0.05, gate_sigma=2.0)
@@ -92,12 +93,14 @@ def test_context_parallel_prefill_emulated_on_one_gpu(world):
     keys = ("q", "k", "v", "log_alpha", "beta")
     spans = [{k_: d[k_][:, r * span:(r + 1) * span].contiguous() for k_ in keys}
              for r in range(world)]
-    trans = [kda_transition(s["k"], s["v"], s["log_alpha"], s["beta"]) for s in spans]
+    ws = [span_workspace(s["k"]) for s in spans]
+    trans = [kda_span_transition(s["k"], s["v"], s["log_alpha"], s["beta"], w)
+             for s, w in zip(spans, ws)]
     gathered = torch.stack(trans)  # what the all-gather delivers
     outs, finals = [], []
     for r, s in enumerate(spans):
         s_in = kda_apply_transitions(gathered[:r], d["initial_state"])
-        o, f = kda_fwd(**s, initial_state=s_in)
+        o, f = kda_span_forward(s["q"], s["k"], s["v"], s["log_alpha"], s["beta"], ws[r], s_in)
         outs.append(o)
         finals.append(f)
     torch.cuda.synchronize()
@@ -110,13 +113,49 @@ def test_context_parallel_prefill_emulated_on_one_gpu(world):
     assert _worst_state_err(finals[-1].cpu().numpy().astype(np.float64), s_ref) <= TOL_BF16_REL_FRO
 
 
-def test_cp_prefill_through_a_one_rank_nccl_group():
-    """The collective code path with real kernels: one rank, so it must equal
+@pytest.mark.parametrize("seg_chunks", [None, "2"])
+def test_span_transition_and_forward_share_the_work(monkeypatch, seg_chunks):
+    """kda_span_transition fills the workspace; kda_span_forward from it gives
+    kda_fwd's results (bit for bit when the span is cut into segments, where
+    kda_fwd takes the same cached path; within tolerance otherwise) and the
+    transition equals kda_transition's."""
+    import torch
+    from gated_delta_rule_139_b200 import (kda_fwd, kda_span_forward, kda_span_transition,
+                                           kda_transition, span_workspace)
+    if seg_chunks:
+        monkeypatch.setenv("KDA_SEG_CHUNKS", seg_chunks)
+    inp = make_inputs(2, 64 * 7 + 11, 2, 128, 128, bf16=True, seed=420, state_sigma=0.05,
+                      gate_sigma=2.0)
+    d = to_device(inp)
+    keys = ("q", "k", "v", "log_alpha", "beta")
+    ws = span_workspace(d["k"])
+    trans = kda_span_transition(d["k"], d["v"], d["log_alpha"], d["beta"], ws)
+    trans_ref = kda_transition(d["k"], d["v"], d["log_alpha"], d["beta"])
+    o, f = kda_span_forward(*(d[k_] for k_ in keys), ws, d["initial_state"])
+    o2, f2 = kda_span_forward(*(d[k_] for k_ in keys), ws, d["initial_state"])  # reusable
+    o_ref, f_ref = kda_fwd(**{k_: d[k_] for k_ in keys}, initial_state=d["initial_state"])
+    torch.cuda.synchronize()
+    assert torch.equal(trans, trans_ref)
+    assert torch.equal(o, o2) and torch.equal(f, f2)
+    if seg_chunks:
+        assert torch.equal(o, o_ref) and torch.equal(f, f_ref)
+    o_or, s_or = oracle.recurrent(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.initial_state)
+    o_g = out_to_f64(o)
+    for n in range(2):
+        for h in range(2):
+            assert _rel(o_g[n, :, h], o_or[n, :, h]) <= TOL_BF16_REL_FRO
+    assert _worst_state_err(f.cpu().numpy().astype(np.float64), s_or) <= TOL_BF16_REL_FRO
+
+
+def test_cp_prefill_through_a_one_rank_nccl_group(monkeypatch):
+    """The collective code path with real kernels: one rank, with the span cut
+    into segments (so kda_fwd takes the same cached path), so it must equal
     kda_fwd bit for bit."""
     import torch
     import torch.distributed as dist
     from gated_delta_rule_139_b200 import kda_fwd
     from gated_delta_rule_139_b200.cp import cp_prefill
+    monkeypatch.setenv("KDA_SEG_CHUNKS", "2")
     inp = make_inputs(1, 64 * 4 + 5, 2, 128, 128, bf16=True, seed=410, state_sigma=0.05)
     d = to_device(inp)
     store = dist.HashStore()
