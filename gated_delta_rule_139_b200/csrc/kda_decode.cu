@@ -10,11 +10,10 @@
 // The state is read once and written once; the path is bound by that traffic
 // (64 KB of fp32 state per head and direction at d = 128).
 //
-// One CTA per (sequence, head) with d_k * d_v / 32 threads; each thread keeps
-// an 8-row x 4-column tile of the state in registers for all the tokens.  The
-// lanes of a warp lie across whole 512-byte state rows, so every state access
-// is a fully coalesced float4 per lane, and the CTA reads and writes its head's
-// state as one contiguous block.  Per token, each thread reads its rows'
+// One CTA per (sequence, head, 64 state columns) with d_k * 64 / 32 threads;
+// each thread keeps an 8-row x 4-column tile of the state in registers for all
+// the tokens.  The lanes of a warp lie across 256-byte row pieces, so every
+// state access is a coalesced float4 per lane.  Per token, each thread reads its rows'
 // (alpha, k, q) as broadcast float4s from shared memory; the two reductions
 // over d_k (S^T k and S^T q) combine per-row-group partial sums through shared
 // memory.  An optional output gate (precomputed by the caller) multiplies o
@@ -62,24 +61,27 @@ __device__ __forceinline__ float raw_x(const unsigned char* p, int i) {
         return reinterpret_cast<const float*>(p)[i];
 }
 
-template <bool BF16, int DK, int DV>
+// A CTA owns DVC = 64 columns of one head's state (grid.y = d_v / 64): half a
+// d_v = 128 state, so that four CTAs fit an SM and one's memory phases overlap
+// another's arithmetic.
+template <bool BF16, int DK, int DVC>
 struct DecodeShape {
-    static constexpr int CW = DV / 4;     // lanes across one state row (4 columns each)
+    static constexpr int CW = DVC / 4;    // lanes across the CTA's columns of one row (4 each)
     static constexpr int RGS = DK / 8;    // row groups of 8 rows
     static constexpr int NTH = RGS * CW;  // threads: d_k * d_v / 32
     static constexpr int TB = BF16 ? 4 : 2;  // tokens per staged block (static shared memory)
 };
 
-template <bool BF16, int DK, int DV>
-__global__ void __launch_bounds__(DecodeShape<BF16, DK, DV>::NTH,
-                                  1024 / DecodeShape<BF16, DK, DV>::NTH)
+template <bool BF16, int DK, int DVC>
+__global__ void __launch_bounds__(DecodeShape<BF16, DK, DVC>::NTH,
+                                  1024 / DecodeShape<BF16, DK, DVC>::NTH)
     decode_kernel(DecodeArgs a) {
-    using Sh = DecodeShape<BF16, DK, DV>;
+    using Sh = DecodeShape<BF16, DK, DVC>;
     constexpr int CW = Sh::CW, RGS = Sh::RGS, NTH = Sh::NTH, TB = Sh::TB;
     constexpr int ES = BF16 ? 2 : 4;  // bytes per q/k/v element
     // raw bytes of one token as it arrives: k | q | v | log_alpha [| gate], in
     // 16-byte chunks
-    constexpr int CK = DK * ES / 16, CV = DV * ES / 16, CL = DK * 4 / 16;
+    constexpr int CK = DK * ES / 16, CV = DVC * ES / 16, CL = DK * 4 / 16;
     constexpr int CH = 2 * CK + CV + CL;
     constexpr int RAWB = (CH + CV) * 16;
     // Raw token blocks arrive by cp.async, two blocks in flight; each block is
@@ -88,14 +90,15 @@ __global__ void __launch_bounds__(DecodeShape<BF16, DK, DV>::NTH,
     __shared__ __align__(16) unsigned char raw[2][TB][RAWB];
     __shared__ float raw_beta[2][TB];
     __shared__ __align__(16) float4 tok[TB][DK];
-    __shared__ float vs[TB][DV];
-    __shared__ float gs[TB][DV];  // output gate (when given)
+    __shared__ float vs[TB][DVC];
+    __shared__ float gs[TB][DVC];  // output gate (when given)
     __shared__ float bs[TB];
-    __shared__ __align__(16) float red[2][RGS][DV];  // per-row-group partial sums
-    __shared__ __align__(16) float us[DV];          // u = beta (v - S^T k) of the token
+    __shared__ __align__(16) float red[2][RGS][DVC];  // per-row-group partial sums
+    __shared__ __align__(16) float us[DVC];          // u = beta (v - S^T k) of the token
     const int tid = threadIdx.x;
     const int rgrp = tid / CW, cq = tid % CW;  // rows 8 rgrp .. +7, columns 4 cq .. +3
     const int nh = blockIdx.x, n = nh / a.H, h = nh % a.H, H = a.H, T = a.T;
+    const int DV = a.dv, c_off = DVC * blockIdx.y;  // row length; this CTA's first column
     int slot = n;
     if (a.slots) {
         slot = a.slots[n];
@@ -119,11 +122,11 @@ __global__ void __launch_bounds__(DecodeShape<BF16, DK, DV>::NTH,
             else if (c < 2 * CK)
                 src = (const unsigned char*)a.q + (row * DK) * ES + (c - CK) * 16;
             else if (c < 2 * CK + CV)
-                src = (const unsigned char*)a.v + (row * DV) * ES + (c - 2 * CK) * 16;
+                src = (const unsigned char*)a.v + (row * DV + c_off) * ES + (c - 2 * CK) * 16;
             else if (c < CH)
                 src = (const unsigned char*)(a.log_alpha + row * DK) + (c - 2 * CK - CV) * 16;
             else
-                src = (const unsigned char*)a.gate + (row * DV) * ES + (c - CH) * 16;
+                src = (const unsigned char*)a.gate + (row * DV + c_off) * ES + (c - CH) * 16;
             cp_async16(&raw[b & 1][t][c * 16], src);
         }
         if (tid < nt) cp_async4(&raw_beta[b & 1][tid], a.beta + ((int64_t)n * T + t0 + tid) * H + h);
@@ -134,7 +137,7 @@ __global__ void __launch_bounds__(DecodeShape<BF16, DK, DV>::NTH,
     cp_async_commit();
 
     // the thread's 8 x 4 tile of the state; a warp covers whole 512-byte rows
-    float* st = a.state + ((int64_t)slot * H + h) * DK * DV + (int64_t)(8 * rgrp) * DV + 4 * cq;
+    float* st = a.state + ((int64_t)slot * H + h) * DK * DV + (int64_t)(8 * rgrp) * DV + c_off + 4 * cq;
     float4 s[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) s[i] = *reinterpret_cast<const float4*>(st + i * DV);
@@ -143,7 +146,7 @@ __global__ void __launch_bounds__(DecodeShape<BF16, DK, DV>::NTH,
         const int t0 = b * TB, nt = min(TB, T - t0), buf = b & 1;
         cp_async_wait_1();  // block b has landed (block b+1 may still be in flight)
         __syncthreads();
-        const int per_tok = DK + (a.gate ? 2 : 1) * DV;
+        const int per_tok = DK + (a.gate ? 2 : 1) * DVC;
         for (int x = tid; x < nt * per_tok; x += NTH) {
             const int t = x / per_tok, e = x - t * per_tok;
             const unsigned char* r = raw[buf][t];
@@ -151,19 +154,19 @@ __global__ void __launch_bounds__(DecodeShape<BF16, DK, DV>::NTH,
                 const float la = reinterpret_cast<const float*>(r + (2 * CK + CV) * 16)[e];
                 tok[t][e] = make_float4(expf(fminf(fmaxf(la, -5.f), 0.f)), raw_x<BF16>(r, e),
                                         raw_x<BF16>(r + CK * 16, e), 0.f);
-            } else if (e < DK + DV) {
+            } else if (e < DK + DVC) {
                 vs[t][e - DK] = raw_x<BF16>(r + 2 * CK * 16, e - DK);
             } else {
-                gs[t][e - DK - DV] = raw_x<BF16>(r + CH * 16, e - DK - DV);
+                gs[t][e - DK - DVC] = raw_x<BF16>(r + CH * 16, e - DK - DVC);
             }
         }
         if (tid < nt) bs[tid] = raw_beta[buf][tid];
         __syncthreads();  // raw[buf] consumed; tok/vs/bs ready
         if (b + 2 < nblk) issue(b + 2);
         cp_async_commit();
-        for (int t = 0; t < nt; ++t) {
+        // decay of token t, then its partial p = S^T k over the thread's 8 rows -> red[0]
+        auto decay_p = [&](int t) {
             const float4* tk = tok[t] + 8 * rgrp;
-            // decay, then partial p = S^T k over the thread's 8 rows
             float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
@@ -178,15 +181,31 @@ __global__ void __launch_bounds__(DecodeShape<BF16, DK, DV>::NTH,
                 p.w = fmaf(s[i].w, x.y, p.w);
             }
             *reinterpret_cast<float4*>(&red[0][rgrp][4 * cq]) = p;
-            __syncthreads();
-            if (tid < DV) {
+        };
+        // o of token t from the row-group partials in red[1] (threads tid < d_v)
+        auto out_o = [&](int t) {
+            float acc = 0.f;
+#pragma unroll
+            for (int g = 0; g < RGS; ++g) acc += red[1][g][tid];
+            const int64_t oi = (((int64_t)n * T + t0 + t) * H + h) * DV + c_off + tid;
+            if (a.gate) acc *= gs[t][tid];  // output gate
+            st_x<BF16>(a.out, oi, acc);
+        };
+        // Two barriers per token: token t's rank-1 update and partial o share a phase
+        // with token t+1's decay and partial p, and o(t) is reduced beside u(t+1).
+        decay_p(0);
+        for (int t = 0; t < nt; ++t) {
+            __syncthreads();  // red[0] (p of t) and red[1] (o of t-1) complete
+            if (tid < DVC) {
                 float acc = 0.f;
 #pragma unroll
                 for (int g = 0; g < RGS; ++g) acc += red[0][g][tid];
                 us[tid] = bs[t] * (vs[t][tid] - acc);
+                if (t > 0) out_o(t - 1);
             }
-            __syncthreads();
-            // rank-1 update, then partial o = S^T q
+            __syncthreads();  // us complete; red[0], red[1] consumed
+            // rank-1 update, then partial o = S^T q -> red[1]
+            const float4* tk = tok[t] + 8 * rgrp;
             const float4 u = *reinterpret_cast<const float4*>(&us[4 * cq]);
             float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
@@ -204,41 +223,33 @@ __global__ void __launch_bounds__(DecodeShape<BF16, DK, DV>::NTH,
             *reinterpret_cast<float4*>(&red[1][rgrp][4 * cq]) = o;
             if (a.token_states) {  // the state after token t0 + t
                 float* ts = a.token_states + (((int64_t)n * T + t0 + t) * H + h) * DK * DV +
-                            (int64_t)(8 * rgrp) * DV + 4 * cq;
+                            (int64_t)(8 * rgrp) * DV + c_off + 4 * cq;
 #pragma unroll
                 for (int i = 0; i < 8; ++i) *reinterpret_cast<float4*>(ts + i * DV) = s[i];
             }
-            __syncthreads();
-            if (tid < DV) {
-                float acc = 0.f;
-#pragma unroll
-                for (int g = 0; g < RGS; ++g) acc += red[1][g][tid];
-                const int64_t oi = (((int64_t)n * T + t0 + t) * H + h) * DV + tid;
-                if (a.gate) acc *= gs[t][tid];  // output gate
-                st_x<BF16>(a.out, oi, acc);
-            }
-            // red[1] is next written after the next token's first barrier, red[0]
-            // and us after its second: no barrier needed here
+            if (t + 1 < nt) decay_p(t + 1);
         }
+        __syncthreads();  // red[1] holds the partials of the block's last token
+        if (tid < DVC) out_o(nt - 1);
+        // the next block's staging begins with a barrier, after which red, us and the
+        // staged vectors may be rewritten
     }
 #pragma unroll
     for (int i = 0; i < 8; ++i) *reinterpret_cast<float4*>(st + i * DV) = s[i];
 }
 
-template <bool BF16, int DK, int DV>
+template <bool BF16, int DK>
 cudaError_t launch_t(const DecodeArgs& a, cudaStream_t stream) {
     profile_mark(SLOT_DECODE, true, stream);
-    decode_kernel<BF16, DK, DV>
-        <<<(unsigned)(a.N * a.H), DecodeShape<BF16, DK, DV>::NTH, 0, stream>>>(a);
+    decode_kernel<BF16, DK, 64><<<dim3((unsigned)(a.N * a.H), (unsigned)(a.dv / 64)),
+                                  DecodeShape<BF16, DK, 64>::NTH, 0, stream>>>(a);
     profile_mark(SLOT_DECODE, false, stream);
     return cudaGetLastError();
 }
 
 template <bool BF16>
 cudaError_t launch_dims(const DecodeArgs& a, cudaStream_t stream) {
-    if (a.dk == 128)
-        return a.dv == 128 ? launch_t<BF16, 128, 128>(a, stream) : launch_t<BF16, 128, 64>(a, stream);
-    return a.dv == 128 ? launch_t<BF16, 64, 128>(a, stream) : launch_t<BF16, 64, 64>(a, stream);
+    return a.dk == 128 ? launch_t<BF16, 128>(a, stream) : launch_t<BF16, 64>(a, stream);
 }
 
 }  // namespace
