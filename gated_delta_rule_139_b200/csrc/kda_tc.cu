@@ -13,13 +13,18 @@
 //
 // Kernels (one launch each, all on the caller's stream):
 //   seg_setup   : segment table from cu_seqlens (or B x T) on the device.
-//   tc_kernel<SEG=true>  "pass 1": per (segment, head) the transition (B, M)
-//                 of every segment that has a successor, computed as the
-//                 chunk loop applied to the augmented state [B | M] from [0 | I].
+//   tc_kernel<1> "pass 1": per (segment, head) the transition (B, M) of the
+//                 segment, computed as the chunk loop applied to the augmented
+//                 state [B | M] from [0 | I].  When sequences are cut into
+//                 segments it runs over every segment and also keeps each
+//                 chunk's W^T and U'^T (bf16) in a cache for pass 3.
 //   seg_scan    : S_in(j+1) = M_j S_in(j) + B_j, sequential over the segments
 //                 of a sequence, parallel over (sequence, head, 16-row block).
-//   tc_kernel<SEG=false> "pass 3": per (segment, head) the chunk loop from the
-//                 true incoming state, writing o and the final state.
+//   tc_kernel<2> "pass 3" with the cache: per (segment, head) the chunk loop
+//                 from the true incoming state, taking W^T and U'^T from the
+//                 cache (only P, the state products and the output remain).
+//   tc_kernel<0> "pass 3" without a cache (one segment per sequence): the full
+//                 chunk loop, writing o and the final state.
 //
 // Per chunk of C = 64 tokens (g = in-chunk inclusive cumsum of the clamped
 // log-gates, per key channel), everything in the transposed orientation so
