@@ -79,7 +79,7 @@ def _rank(rank, world, port, q):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("world", [2, 3, 4])
 def test_cp_prefill_on_gloo_ranks_matches_the_whole_sequence(world):
     import oracle
     ctx = mp.get_context("spawn")

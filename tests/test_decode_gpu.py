@@ -171,3 +171,37 @@ def test_decode_launch_count_and_path():
     inp = make_inputs(2, 1, 2, 128, 128, bf16=True, seed=116, state_sigma=0.3)
     _decode(to_device(inp))
     assert last_launch_count() == 1 and last_path() == "decode"
+
+
+def test_decode_fp32_slots_token_states_and_gate_together():
+    """Every option at once on the fp32 path: results match the oracle, the
+    per-token states are the prefix states, padding entries touch nothing."""
+    import torch
+    from gated_delta_rule_139_b200 import kda_decode
+    inp = make_inputs(3, 5, 2, 64, 128, bf16=False, seed=117, state_sigma=0.3, gate_sigma=2.0)
+    d = to_device(inp)
+    gate = torch.from_numpy(np.random.default_rng(5).uniform(0, 1, inp.v.shape).astype(np.float32)).cuda()
+    pool = torch.zeros(6, 2, 64, 128, device="cuda")
+    slot_of = [4, -1, 1]
+    for n, sl in enumerate(slot_of):
+        if sl >= 0:
+            pool[sl] = d["initial_state"][n]
+    slots = torch.tensor(slot_of, dtype=torch.int32, device="cuda")
+    out = torch.full((3, 5, 2, 128), 9.0, device="cuda")
+    _, ts = kda_decode(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], pool, slots=slots, out=out,
+                       out_gate=gate, want_token_states=True)
+    torch.cuda.synchronize()
+    o_r, s_r = oracle.recurrent(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.initial_state,
+                                out_gate=gate.cpu().numpy())
+    for n, sl in enumerate(slot_of):
+        if sl < 0:
+            assert (out[n] == 9.0).all()
+            continue
+        assert np.abs(out[n].cpu().numpy() - o_r[n]).max() <= TOL_F32_MAX_ABS
+        assert np.abs(pool[sl].cpu().numpy() - s_r[n]).max() <= TOL_F32_MAX_ABS
+        assert torch.equal(ts[n, -1], pool[sl])
+        for t in range(5):
+            sub = lambda a: np.ascontiguousarray(a[n:n + 1, :t + 1])
+            _, s_t = oracle.recurrent(sub(inp.q), sub(inp.k), sub(inp.v), sub(inp.log_alpha),
+                                      sub(inp.beta), inp.initial_state[n:n + 1], o_tokens=0)
+            assert np.abs(ts[n, t].cpu().numpy() - s_t[0]).max() <= TOL_F32_MAX_ABS

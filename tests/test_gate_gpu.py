@@ -109,3 +109,44 @@ def test_gate_with_snapshots():
     o_ref, _ = kda_fwd(**d, out_gate=gate)
     torch.cuda.synchronize()
     assert torch.equal(pool_g, pool) and torch.equal(o_g, o_ref)
+
+
+def test_fwd_ex_without_options_is_kda_fwd_bitwise():
+    import ctypes
+    import torch
+    import gated_delta_rule_139_b200 as kda
+    inp = make_inputs(1, 64 * 3 + 9, 2, 128, 128, bf16=True, seed=304, state_sigma=0.05)
+    d = to_device(inp)
+    o_ref, s_ref = kda.kda_fwd(**d)
+    o = torch.empty_like(o_ref)
+    s = torch.empty_like(s_ref)
+    dims = kda.Dims(1, inp.T, 2, 128, 128, 0, 1)
+    P = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
+    rc = kda.load_library().kda_fwd_ex(P(d["q"]), P(d["k"]), P(d["v"]), P(d["log_alpha"]),
+                                       P(d["beta"]), P(d["initial_state"]), None, 64, P(o), P(s),
+                                       ctypes.byref(dims), None,
+                                       ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    torch.cuda.synchronize()
+    assert kda.STATUS[rc] == "KDA_OK"
+    assert torch.equal(o, o_ref) and torch.equal(s, s_ref)
+
+
+def test_snapshots_and_gate_on_the_cuda_core_path():
+    import torch
+    from gated_delta_rule_139_b200 import kda_fwd_snap
+    inp = make_inputs(2, 64 * 2 + 30, 2, 64, 64, bf16=False, seed=305, state_sigma=0.05)
+    d = to_device(inp)
+    gate = _gate(inp, 6)
+    slots = torch.tensor([[0, 1], [2, 3]], dtype=torch.int32, device="cuda")
+    pool = torch.zeros(4, 2, 64, 64, device="cuda")
+    o, s = kda_fwd_snap(**d, snap_interval=64, snap_slots=slots, snap_pool=pool,
+                        out_gate=_dev(gate, False))
+    torch.cuda.synchronize()
+    _check(inp, o, s, gate)
+    for n in range(2):
+        for j in range(2):
+            L = 64 * (j + 1)
+            sub = lambda a: np.ascontiguousarray(a[n:n + 1, :L])
+            _, s_ref = oracle.recurrent(sub(inp.q), sub(inp.k), sub(inp.v), sub(inp.log_alpha),
+                                        sub(inp.beta), inp.initial_state[n:n + 1], o_tokens=0)
+            assert np.abs(pool[2 * n + j].cpu().numpy() - s_ref[0]).max() <= TOL_F32_MAX_ABS
