@@ -723,52 +723,13 @@ kda_status kda_transition(const void* k, const void* v, const float* log_alpha,
     g_last_error[0] = 0;
     g_last_launches = 0;
     g_last_path = "";
-    if (!d) return fail(KDA_ERR_INVALID_ARG, "dims is NULL");
-    if (d->B < 1 || d->T < 0 || d->H < 1)
-        return fail(KDA_ERR_INVALID_ARG, "need B >= 1, T >= 0, H >= 1 (got B=%d T=%d H=%d)",
-                    d->B, d->T, d->H);
-    if (d->qkv_dtype != KDA_F32 && d->qkv_dtype != KDA_BF16)
-        return fail(KDA_ERR_INVALID_ARG, "qkv_dtype must be KDA_F32 or KDA_BF16");
-    if (d->d_k != 128 || d->d_v != 128 || d->qkv_dtype != KDA_BF16)
-        return fail(KDA_ERR_UNSUPPORTED, "kda_transition needs bf16 k/v with d_k = d_v = 128");
-    const int64_t tokens = (int64_t)d->B * d->T;
-    if (!trans) return fail(KDA_ERR_INVALID_ARG, "trans must be non-NULL");
-    if (tokens > 0 && (!k || !v || !log_alpha || !beta))
-        return fail(KDA_ERR_INVALID_ARG, "k, v, log_alpha and beta must be non-NULL");
+    kda::FwdArgs a;
+    kda_status st = validate_span_inputs(k, v, log_alpha, beta, d, trans, &a);
+    if (st != KDA_OK) return st;
     const void* ptrs[] = {k, v, log_alpha, beta, trans};
     const char* names[] = {"k", "v", "log_alpha", "beta", "trans"};
-    for (int i = 0; i < 5; ++i)
-        if (ptrs[i] && ((uintptr_t)ptrs[i] & 15u))
-            return fail(KDA_ERR_MISALIGNED, "%s is not 16-byte aligned", names[i]);
-    const int64_t n = tokens * d->H * 128;
-    const Range in[] = {{(uintptr_t)k, (uintptr_t)k + (k ? n * 2 : 0), "k"},
-                        {(uintptr_t)v, (uintptr_t)v + (v ? n * 2 : 0), "v"},
-                        {(uintptr_t)log_alpha, (uintptr_t)log_alpha + (log_alpha ? n * 4 : 0),
-                         "log_alpha"},
-                        {(uintptr_t)beta, (uintptr_t)beta + (beta ? tokens * d->H * 4 : 0), "beta"}};
-    const Range rt = {(uintptr_t)trans, (uintptr_t)trans + (uintptr_t)d->B * d->H * 2 * 128 * 128 * 4,
-                      "trans"};
-    for (const Range& r : in)
-        if (overlaps(rt, r)) return fail(KDA_ERR_ALIAS, "trans overlaps %s", r.name);
-    kda_status st = check_accessible(ptrs, names, 5);
+    st = check_accessible(ptrs, names, 5);
     if (st != KDA_OK) return st;
-    kda::FwdArgs a;
-    a.q = nullptr;
-    a.k = k;
-    a.v = v;
-    a.log_alpha = log_alpha;
-    a.beta = beta;
-    a.s0 = nullptr;
-    a.cu = nullptr;
-    a.out = nullptr;
-    a.s_final = nullptr;
-    a.B = d->B;
-    a.T = d->T;
-    a.H = d->H;
-    a.dk = 128;
-    a.dv = 128;
-    a.N = d->B;
-    a.bf16 = 1;
     const kda::TcPlan p = plan_segments(a);
     const size_t b_segs = ((size_t)p.max_units * sizeof(kda::SegEntry) + 255) & ~(size_t)255;
     const size_t b_off = ((size_t)(a.N + 1) * 4 + 4 + 255) & ~(size_t)255;
