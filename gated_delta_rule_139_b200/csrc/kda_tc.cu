@@ -313,10 +313,15 @@ __device__ __forceinline__ void warp_store16x8(float* dst, int ld, const float (
 // The block products are tf32 warp MMAs with fp32 accumulation (T then enters
 // the chunk products as bf16).
 // `side(warp)` runs on warps 8-15 while warps 0-1 invert the diagonal blocks
-// (work that does not touch As, Ts, Ys or TB).
-template <typename Side>
-__device__ void invert_to_tb(const float* As, float* Ts, float* Ys, const float* beta,
-                             uint32_t tbp, int tid, Side side) {
+// (work that does not touch As, Ts, Ys or TB).  OWN_A: As has not been
+// extracted; warps 0-1 (TMEM lanes 0-63 = rows of A, tq = their lane quadrant)
+// read their rows of A from the product in TMEM, scale by beta, mask, and write
+// the parts of As the later steps read (rows 0-31: columns 0-31; rows 32-63:
+// columns 0-63), keeping their diagonal blocks in registers, so the inversion
+// starts as soon as the product is complete.
+template <bool OWN_A, typename Side>
+__device__ void invert_to_tb(float* As, float* Ts, float* Ys, const float* beta, uint32_t tbp,
+                             int tid, uint32_t tq, Side side) {
     const int warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t4 = lane & 3;
     if (warp < 2) {
@@ -326,11 +331,31 @@ __device__ void invert_to_tb(const float* As, float* Ts, float* Ys, const float*
            // and broadcast to the 16 lanes of the block by shuffles
             const int i = lane & 15, ob = o + 16 * (lane >> 4), src0 = lane & 16;
             float arow[16], trow[16];
+            if (OWN_A) {
+                const int r = o + lane;  // this lane's row of A
+                const float br = beta[r];
 #pragma unroll
-            for (int m = 0; m < 16; ++m) {
-                arow[m] = m < i ? As[(ob + i) * AS_LD + ob + m] : 0.f;
-                trow[m] = m == i ? 1.f : 0.f;
+                for (int cc = 0; cc < 4; ++cc) {
+                    const int j0 = 16 * cc;
+                    if (warp == 0 && j0 >= 32) break;  // rows 0-31 need columns 0-31 only
+                    float v[16];
+                    // columns j < 32 of rows >= 32 are the cross-half product (TMEM 64 + j)
+                    tmem_ld16(tq + TM_AP + (warp == 1 && j0 < 32 ? 64 + j0 : j0), v);
+                    tmem_wait16(v);
+#pragma unroll
+                    for (int m = 0; m < 16; ++m) {
+                        const float x = j0 + m < r ? br * v[m] : 0.f;
+                        As[r * AS_LD + j0 + m] = x;
+                        if (j0 == ob) arow[m] = x;
+                    }
+                }
+                __syncwarp();
+            } else {
+#pragma unroll
+                for (int m = 0; m < 16; ++m) arow[m] = m < i ? As[(ob + i) * AS_LD + ob + m] : 0.f;
             }
+#pragma unroll
+            for (int m = 0; m < 16; ++m) trow[m] = m == i ? 1.f : 0.f;
 #pragma unroll
             for (int m = 0; m < 15; ++m) {
                 const float am = arow[m];
@@ -707,7 +732,7 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
             // cross-half product (TMEM columns 64 + j).
             // MODE 2 needs only P, which it finds in rows 0-63 (q~ sits there in X1)
             const bool need_a = !FAST;
-            if (FAST ? quad < 2 : (!SEG || quad < 2)) {
+            if (!SEG && (!FAST || quad < 2)) {  // pass 1 extracts A inside the inversion
                 const int r = lrow & 63;
                 const bool isP = FAST || quad >= 2;
                 const bool lower_half = r < 32;  // warp-uniform
@@ -741,11 +766,11 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
                                      pack_bf16(x[8 * hh + 6], x[8 * hh + 7]));
                 }
             }
-            __syncthreads();
+            if (!SEG) __syncthreads();
             if (need_a) {
                 // beside the diagonal inversions: pass 1 stages M (bf16 M^T -> MA, M scaled by
                 // gamma in TMEM) on warps 8-15, which own two 64-column slices per quadrant
-                invert_to_tb(As, Ts, Ys, beta_s, smem_u32(sm + Lay::TB), tid, [&](int w) {
+                invert_to_tb<SEG>(As, Ts, Ys, beta_s, smem_u32(sm + Lay::TB), tid, tq, [&](int w) {
                     if (SEG) {
                         const int c0 = 64 * ((w >> 2) - 2);
                         stage_cols<4>(tq + TM_M + c0, sm + Lay::MA, 128, lrow, c0, gam, true);
