@@ -112,10 +112,12 @@ static_assert(LayT<true>::MA + 32768 <= LayT<true>::R1, "MA overflow");
 static_assert(LayT<false>::BYTES <= 232448 && LayT<true>::BYTES <= 232448, "shared memory");
 
 // TMEM columns (512 allocated).  Pass 3: AP [0,96) W [96,160) U [160,224)
-// O [224,288) bf16 S^T [288,352) bf16 U^T [352,384) S [384,512).  Pass 1: AP/U_M [0,96) W U as above, B [256,384), M [384,512).
+// O [224,288) bf16 S^T [288,352) bf16 U^T [352,384) S [384,512).  Pass 1: AP/U_M [0,96) W U as
+// above (W's columns later hold bf16 U_B^T [96,128) and U_M^T [128,160)), B [256,384), M [384,512).
 constexpr uint32_t TM_AP = 0, TM_W = 96, TM_U = 160, TM_O = 224;
 constexpr uint32_t TM_SB = 288, TM_UB = 352;  // pass 3: bf16 copies of S^T and U^T (A operands)
 constexpr uint32_t TM_B = 256, TM_S = 384, TM_M = 384;
+constexpr uint32_t TM_UBB = 96, TM_UBM = 128;  // pass 1: bf16 U_B^T, U_M^T (A operands) in the W columns
 
 __device__ __forceinline__ float clamp_gate(float x) { return fminf(fmaxf(x, -5.f), 0.f); }
 // 2^x by the SFU instruction (relative error about 2^-22, flushes results
@@ -911,11 +913,8 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
         if (!(ok = wait_mma(bar, parity))) break;
         if (FAST && tid == 0 && t0 + C < sg.t_end) load_w(t0 + C);  // W^T consumed: the next one
 
-        if (SEG && wu_cache) {  // UA is about to be rewritten: the cache copy must have left it
-            if (tid == 0) bulk_wait_read();
-            __syncthreads();
-        }
-        // ============ phase 6: U^T -> UA (bf16, K-major, 128 x 64); pass 1 also U_M^T -> UMA
+        // ============ phase 6: bf16 U^T into TMEM as the next products' A operand (pass 1:
+        // U_B^T and U_M^T, in the W columns, which W staging has emptied)
         if (!SEG) {
             const int c0 = 16 * wg;
             stage_cols_tmem<1>(tq + TM_U + c0, tq + TM_UB + c0 / 2, c0, nullptr, false);
@@ -923,8 +922,9 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
         } else {
             const bool is_m = wg >= 2;
             const int c0 = 32 * (wg & 1);
-            stage_cols<2>(tq + (is_m ? TM_AP : TM_U) + c0, sm + (is_m ? Lay::UMA : Lay::UA), 128,
-                          lrow, c0, nullptr, false);
+            stage_cols_tmem<2>(tq + (is_m ? TM_AP : TM_U) + c0, tq + (is_m ? TM_UBM : TM_UBB) + c0 / 2,
+                               c0, nullptr, false);
+            tmem_st_wait();
         }
         fence_async_smem();
         tc_fence_before();
@@ -933,7 +933,7 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
         // ============ phase 7: O^T += U^T P^T ; S^T += U^T Kdec  (pass 1: B, M updates)
         if (tid == 0) {
             tc_fence_after();
-            const uint32_t ua = smem_u32(sm + Lay::UA), kd = smem_u32(sm + Lay::KD);
+            const uint32_t kd = smem_u32(sm + Lay::KD);
             constexpr uint32_t id_s = idesc_bf16(128, 128, false, true);
             if (!SEG) {  // A = bf16 U^T from TMEM
                 const uint32_t pb = smem_u32(sm + Lay::PB);
@@ -944,14 +944,13 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
                     mma_bf16_ts(tmem + TM_S, tmem + TM_UB + 8 * s, mnmajor_desc(kd, 64, s), id_s, 1);
-            } else {
-                const uint32_t uma = smem_u32(sm + Lay::UMA);
+            } else {  // A = bf16 U_B^T, U_M^T from TMEM
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
-                    mma_bf16(tmem + TM_B, kmajor_desc(ua, 128, s), mnmajor_desc(kd, 64, s), id_s, 1);
+                    mma_bf16_ts(tmem + TM_B, tmem + TM_UBB + 8 * s, mnmajor_desc(kd, 64, s), id_s, 1);
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
-                    mma_bf16(tmem + TM_M, kmajor_desc(uma, 128, s), mnmajor_desc(kd, 64, s), id_s, 1);
+                    mma_bf16_ts(tmem + TM_M, tmem + TM_UBM + 8 * s, mnmajor_desc(kd, 64, s), id_s, 1);
             }
             mma_commit(bar);
         }
