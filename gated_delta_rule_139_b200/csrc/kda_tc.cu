@@ -72,16 +72,21 @@ constexpr float LOG2E = 1.4426950408889634f;
 //               BT (B operand, 96 x 128) until the phase-1 product completes.
 //   phase  2  : As, Ts (fp32, strides 68 and 72) in BT's place, Ys in a q-row hole,
 //               then TB (bf16 T diag(beta)) in the other q-row hole
-//   phases 3-8: SA (bf16 S^T) over As/Ts, WB (W^T) and UA (U^T) over X1;
-//               pass 1 adds MA (bf16 M^T) after Ts
+//   phases 3-8: WB (W^T) over X1; pass 1 also UA (U'^T, kept with W^T for pass 3)
+//               over X1 and MA (bf16 M^T) after Ts.  The bf16 copies of S^T, B^T,
+//               U^T, U_B^T and U_M^T that the state products take as A operands
+//               live in tensor memory.
+//   MODE 2 (pass 3 with the W/U' cache): q~ in X1's rows 0-63, W^T in its rows
+//               64-127; no As/Ts/TB.
 // RAW holds the next chunk's k, log alpha (and q) tiles, written by TMA while
 // the current chunk is processed; RV0/RV1 alternate as the chunk's v tile, which
-// TMA writes directly in the 128-byte-swizzled MN-major operand layout.
+// TMA writes directly in the 128-byte-swizzled MN-major operand layout (MODE 2:
+// the chunk's U'^T from the cache).
 template <bool SEG>
 struct LayT {
     static constexpr uint32_t X1 = 0, BT = 32768;
     static constexpr uint32_t AS = 32768, TS = AS + 17408, YS = 24576, TB = 8192;
-    static constexpr uint32_t SA = 32768, WB = 0, UA = 16384, MA = 69632;
+    static constexpr uint32_t WB = 0, UA = 16384, MA = 69632;
     static constexpr uint32_t R1 = SEG ? 102400 : 69632;
     static constexpr uint32_t QT = R1;                            // pass 3: 64 x 128, K-major
     static constexpr uint32_t KD = SEG ? R1 : QT + 16384;         // 64 x 128, MN-major
@@ -106,7 +111,6 @@ struct LayT {
 static_assert(LayT<false>::TS + 64 * 72 * 4 <= LayT<false>::R1, "As/Ts overflow");
 static_assert(LayT<false>::YS + 32 * 40 * 4 <= 32768 && LayT<false>::TB + 8192 <= 16384,
               "Ys/TB must sit in the q-row holes of X1");
-static_assert(LayT<false>::SA + 32768 <= LayT<false>::R1, "SA overflow");
 static_assert(LayT<true>::WB + 16384 == LayT<true>::UA, "pass 1 stores W^T and U'^T as one 32 KB copy");
 static_assert(LayT<true>::MA + 32768 <= LayT<true>::R1, "MA overflow");
 static_assert(LayT<false>::BYTES <= 232448 && LayT<true>::BYTES <= 232448, "shared memory");
@@ -118,6 +122,9 @@ constexpr uint32_t TM_AP = 0, TM_W = 96, TM_U = 160, TM_O = 224;
 constexpr uint32_t TM_SB = 288, TM_UB = 352;  // pass 3: bf16 copies of S^T and U^T (A operands)
 constexpr uint32_t TM_B = 256, TM_S = 384, TM_M = 384;
 constexpr uint32_t TM_UBB = 96, TM_UBM = 128;  // pass 1: bf16 U_B^T, U_M^T (A operands) in the W columns
+// pass 1: bf16 B^T (A operand of U_B -= B W): K steps 0-3 (channels 0-63) in [64,96), which the
+// cross-half block of A has left, and K steps 4-7 in [224,256), unused in pass 1
+__device__ __forceinline__ uint32_t sbb_col(int s) { return s < 4 ? 64 + 8 * s : 224 + 8 * (s - 4); }
 
 __device__ __forceinline__ float clamp_gate(float x) { return fminf(fmaxf(x, -5.f), 0.f); }
 // 2^x by the SFU instruction (relative error about 2^-22, flushes results
@@ -820,9 +827,10 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
             const int c0 = 32 * wg;
             stage_cols_tmem<2>(tq + TM_S + c0, tq + TM_SB + c0 / 2, c0, gam, true);
             tmem_st_wait();
-        } else {  // pass 1: B (M was staged beside the inversion)
+        } else {  // pass 1: bf16 B^T into two free 32-column TMEM ranges (M was staged
+                  // beside the inversion)
             const int c0 = 32 * wg;
-            stage_cols<2>(tq + TM_B + c0, sm + Lay::SA, 128, lrow, c0, gam, true);
+            stage_cols_tmem<2>(tq + TM_B + c0, tq + sbb_col(c0 >> 4), c0, gam, true);
             tmem_st_wait();
         }
         if (!(ok = wait_mma(bar, parity))) break;
@@ -882,7 +890,7 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
         }
         if (tid == 0 && w_ok) {
             tc_fence_after();
-            const uint32_t sa = smem_u32(sm + Lay::SA), wb = smem_u32(sm + Lay::WB);
+            const uint32_t wb = smem_u32(sm + Lay::WB);
             constexpr uint32_t id_neg = idesc_bf16(128, 64, false, true, true);
             if (!SEG) {  // A = bf16 S^T from TMEM
                 const uint32_t qt = smem_u32(sm + Lay::QT);
@@ -902,7 +910,7 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
                 const uint32_t ma = smem_u32(sm + Lay::MA);
 #pragma unroll
                 for (int s = 0; s < 8; ++s)
-                    mma_bf16(tmem + TM_U, kmajor_desc(sa, 128, s), mnmajor_desc(wb, 128, s), id_neg, 1);
+                    mma_bf16_ts(tmem + TM_U, tmem + sbb_col(s), mnmajor_desc(wb, 128, s), id_neg, 1);
 #pragma unroll
                 for (int s = 0; s < 8; ++s)
                     mma_bf16(tmem + TM_AP, kmajor_desc(ma, 128, s), mnmajor_desc(wb, 128, s), id_neg,
