@@ -169,3 +169,28 @@ def test_cp_prefill_through_a_one_rank_nccl_group(monkeypatch):
         assert torch.equal(o, o_ref) and torch.equal(f, f_ref)
     finally:
         dist.destroy_process_group()
+
+
+def test_cp_prefill_with_output_gate(monkeypatch):
+    """The gated forward through the collective path: one rank, segmented span,
+    so it must equal kda_fwd with the same gate bit for bit."""
+    import torch
+    import torch.distributed as dist
+    from gated_delta_rule_139_b200 import kda_fwd
+    from gated_delta_rule_139_b200.cp import cp_prefill
+    monkeypatch.setenv("KDA_SEG_CHUNKS", "2")
+    inp = make_inputs(1, 64 * 5 + 3, 2, 128, 128, bf16=True, seed=411, state_sigma=0.05)
+    d = to_device(inp)
+    gate = torch.rand(inp.v.shape, device="cuda").to(torch.bfloat16)
+    store = dist.HashStore()
+    dist.init_process_group("nccl", store=store, rank=0, world_size=1,
+                            device_id=torch.device("cuda", 0))
+    try:
+        keys = ("q", "k", "v", "log_alpha", "beta")
+        o, f = cp_prefill(*(d[k_] for k_ in keys), d["initial_state"], out_gate=gate)
+        o_ref, f_ref = kda_fwd(**{k_: d[k_] for k_ in keys}, initial_state=d["initial_state"],
+                               out_gate=gate)
+        torch.cuda.synchronize()
+        assert torch.equal(o, o_ref) and torch.equal(f, f_ref)
+    finally:
+        dist.destroy_process_group()
