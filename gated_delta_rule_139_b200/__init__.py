@@ -95,6 +95,9 @@ def load_library():
         lib.kda_span_forward.argtypes = [p, p, p, p, p, p, p, p, ctypes.POINTER(Dims), p,
                                          ctypes.c_size_t, p]
         lib.kda_span_forward.restype = ctypes.c_int
+        lib.kda_span_forward_ex.argtypes = lib.kda_span_forward.argtypes[:-1] + \
+            [ctypes.POINTER(FwdOpts), p]
+        lib.kda_span_forward_ex.restype = ctypes.c_int
         lib.kda_decode.restype = ctypes.c_int
         lib.kda_status_string.argtypes = [ctypes.c_int]
         lib.kda_status_string.restype = ctypes.c_char_p
@@ -215,6 +218,18 @@ def kda_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, chunk
     return out, final_state
 
 
+def _snap_spec(snap_interval, snap_slots, snap_pool, n_seqs):
+    import torch
+    for t in (snap_slots, snap_pool):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("snap_slots and snap_pool must be contiguous CUDA tensors")
+    if snap_slots.dtype != torch.int32 or snap_slots.dim() != 2:
+        raise ValueError("snap_slots must be an int32 [N, max_snaps] tensor")
+    if snap_slots.shape[0] != n_seqs:
+        raise ValueError(f"snap_slots has {snap_slots.shape[0]} rows for {n_seqs} sequences")
+    return SnapSpec(int(snap_interval), snap_slots.shape[1], snap_pool.shape[0])
+
+
 def kda_fwd_snap(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, *,
                  snap_interval: int, snap_slots, snap_pool, chunk: int = 64, out=None,
                  final_state=None, stream=None, want_final: bool = True, out_gate=None):
@@ -226,17 +241,8 @@ def kda_fwd_snap(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, 
     ``snap_slots`` is an int32 CUDA tensor [N, max_snaps].  Returns (out,
     final_state or None); the pool is written in place.
     """
-    import torch
-
-    for t in (snap_slots, snap_pool):
-        if not t.is_cuda or not t.is_contiguous():
-            raise ValueError("snap_slots and snap_pool must be contiguous CUDA tensors")
-    if snap_slots.dtype != torch.int32 or snap_slots.dim() != 2:
-        raise ValueError("snap_slots must be an int32 [N, max_snaps] tensor")
     n_seqs = (cu_seqlens.numel() - 1) if cu_seqlens is not None else q.shape[0]
-    if snap_slots.shape[0] != n_seqs:
-        raise ValueError(f"snap_slots has {snap_slots.shape[0]} rows for {n_seqs} sequences")
-    spec = SnapSpec(int(snap_interval), snap_slots.shape[1], snap_pool.shape[0])
+    spec = _snap_spec(snap_interval, snap_slots, snap_pool, n_seqs)
     return kda_fwd(q, k, v, log_alpha, beta, initial_state, cu_seqlens, chunk, out, final_state,
                    stream, want_final, out_gate=out_gate, _snap=(spec, snap_slots, snap_pool))
 
@@ -427,8 +433,12 @@ def kda_span_transition(k, v, log_alpha, beta, workspace, out=None, stream=None)
 
 
 def kda_span_forward(q, k, v, log_alpha, beta, workspace, initial_state=None, out=None,
-                     final_state=None, stream=None, want_final: bool = True):
-    """kda_fwd on a span whose kda_span_transition filled ``workspace``."""
+                     final_state=None, stream=None, want_final: bool = True, out_gate=None, *,
+                     snap_interval=None, snap_slots=None, snap_pool=None):
+    """kda_fwd on a span whose kda_span_transition filled ``workspace``.
+    ``out_gate`` as in :func:`kda_fwd`; the snapshot arguments as in
+    :func:`kda_fwd_snap`, with positions counted from the span's start
+    (kda_span_forward_ex)."""
     import torch
     lib = load_library()
     d = _dims(tuple(q.shape), tuple(v.shape), None, 0, q.dtype == torch.bfloat16)
@@ -439,8 +449,21 @@ def kda_span_forward(q, k, v, log_alpha, beta, workspace, initial_state=None, ou
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
     ptr = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
-    _check(lib.kda_span_forward(ptr(q), ptr(k), ptr(v), ptr(log_alpha), ptr(beta),
-                                ptr(initial_state), ptr(out), ptr(final_state), ctypes.byref(d),
-                                ptr(workspace), workspace.numel(),
-                                ctypes.c_void_p(stream.cuda_stream)))
+    args = (ptr(q), ptr(k), ptr(v), ptr(log_alpha), ptr(beta), ptr(initial_state), ptr(out),
+            ptr(final_state), ctypes.byref(d), ptr(workspace), workspace.numel())
+    if out_gate is None and snap_interval is None:
+        _check(lib.kda_span_forward(*args, ctypes.c_void_p(stream.cuda_stream)))
+        return out, final_state
+    opts = FwdOpts(None, None, None, None)
+    if out_gate is not None:
+        if not out_gate.is_cuda or not out_gate.is_contiguous() or out_gate.dtype != q.dtype \
+                or tuple(out_gate.shape) != tuple(out.shape):
+            raise ValueError("out_gate must be a contiguous CUDA tensor shaped and typed as out")
+        opts.out_gate = out_gate.data_ptr()
+    if snap_interval is not None:
+        spec = _snap_spec(snap_interval, snap_slots, snap_pool, q.shape[0])
+        opts.snap = ctypes.pointer(spec)
+        opts.snap_slots = snap_slots.data_ptr()
+        opts.snap_pool = snap_pool.data_ptr()
+    _check(lib.kda_span_forward_ex(*args, ctypes.byref(opts), ctypes.c_void_p(stream.cuda_stream)))
     return out, final_state

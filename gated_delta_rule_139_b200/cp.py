@@ -44,17 +44,14 @@ def library_ops() -> SpanOps:
     """The library's kernels.  The transition step keeps its segment transitions
     and per-chunk W, U' in a workspace, so the forward step does not compute
     them again (kda_span_transition / kda_span_forward)."""
-    from . import (kda_apply_transitions, kda_fwd, kda_span_forward, kda_span_transition,
-                   span_workspace)
+    from . import kda_apply_transitions, kda_span_forward, kda_span_transition, span_workspace
 
     def transition(k, v, log_alpha, beta):
         ws = span_workspace(k)
         return kda_span_transition(k, v, log_alpha, beta, ws), ws
 
     def forward(q, k, v, log_alpha, beta, s_in, out_gate, ws):
-        if out_gate is not None:  # the gated epilogue lives in the full forward
-            return kda_fwd(q, k, v, log_alpha, beta, s_in, out_gate=out_gate)
-        return kda_span_forward(q, k, v, log_alpha, beta, ws, s_in)
+        return kda_span_forward(q, k, v, log_alpha, beta, ws, s_in, out_gate=out_gate)
 
     return SpanOps(transition=transition,
                    apply=lambda prior, s0: kda_apply_transitions(prior, s0),

@@ -475,18 +475,14 @@ kda_status kda_fwd(const void* q, const void* k, const void* v, const float* log
     return run(a, (cudaStream_t)stream);
 }
 
-kda_status kda_fwd_ex(const void* q, const void* k, const void* v, const float* log_alpha,
-                      const float* beta, const float* initial_state, const int32_t* cu_seqlens,
-                      int32_t chunk, void* out, float* final_state, const kda_dims* dims,
-                      const kda_fwd_opts* opts, void* stream) {
-    g_last_error[0] = 0;
-    g_last_launches = 0;
-    g_last_path = "";
-    kda::FwdArgs a;
-    // argument checks first, then (as in kda_fwd) whether the pointers are device memory
-    kda_status s = validate(q, k, v, log_alpha, beta, initial_state, cu_seqlens, chunk, out,
-                            final_state, dims, false, &a);
-    if (s != KDA_OK) return s;
+// Checks the optional parts of a forward call against the validated dims and
+// the call's other buffers, and records them in `a`.  Argument checks first,
+// then whether every pointer is device memory (as in kda_fwd).
+static kda_status apply_opts(const kda_fwd_opts* opts, const void* q, const void* k, const void* v,
+                             const float* log_alpha, const float* beta, const float* initial_state,
+                             const int32_t* cu_seqlens, const void* out, const float* final_state,
+                             kda::FwdArgs* pa) {
+    kda::FwdArgs& a = *pa;
     const kda_fwd_opts none = {nullptr, nullptr, nullptr, nullptr};
     if (!opts) opts = &none;
     const kda_snap_spec* snap = opts->snap;
@@ -546,7 +542,7 @@ kda_status kda_fwd_ex(const void* q, const void* k, const void* v, const float* 
                           gate, snap_slots, snap_pool};
     const char* names[] = {"q", "k", "v", "log_alpha", "beta", "initial_state", "cu_seqlens",
                            "out", "final_state", "out_gate", "snap_slots", "snap_pool"};
-    s = check_accessible(ptrs, names, 12);
+    kda_status s = check_accessible(ptrs, names, 12);
     if (s != KDA_OK) return s;
     a.gate = gate;
     if (snap) {
@@ -558,6 +554,22 @@ kda_status kda_fwd_ex(const void* q, const void* k, const void* v, const float* 
         cudaError_t e = kda::status_word(&a.status);
         if (e != cudaSuccess) return cuda_fail(e, "device status word");
     }
+    return KDA_OK;
+}
+
+kda_status kda_fwd_ex(const void* q, const void* k, const void* v, const float* log_alpha,
+                      const float* beta, const float* initial_state, const int32_t* cu_seqlens,
+                      int32_t chunk, void* out, float* final_state, const kda_dims* dims,
+                      const kda_fwd_opts* opts, void* stream) {
+    g_last_error[0] = 0;
+    g_last_launches = 0;
+    g_last_path = "";
+    kda::FwdArgs a;
+    kda_status s = validate(q, k, v, log_alpha, beta, initial_state, cu_seqlens, chunk, out,
+                            final_state, dims, false, &a);
+    if (s != KDA_OK) return s;
+    s = apply_opts(opts, q, k, v, log_alpha, beta, initial_state, cu_seqlens, out, final_state, &a);
+    if (s != KDA_OK) return s;
     return run(a, (cudaStream_t)stream);
 }
 
@@ -808,16 +820,17 @@ kda_status kda_span_transition(const void* k, const void* v, const float* log_al
     return KDA_OK;
 }
 
-kda_status kda_span_forward(const void* q, const void* k, const void* v, const float* log_alpha,
-                            const float* beta, const float* initial_state, void* out,
-                            float* final_state, const kda_dims* d, const void* workspace,
-                            size_t workspace_bytes, void* stream) {
+kda_status kda_span_forward_ex(const void* q, const void* k, const void* v,
+                               const float* log_alpha, const float* beta,
+                               const float* initial_state, void* out, float* final_state,
+                               const kda_dims* d, const void* workspace, size_t workspace_bytes,
+                               const kda_fwd_opts* opts, void* stream) {
     g_last_error[0] = 0;
     g_last_launches = 0;
     g_last_path = "";
     kda::FwdArgs a;
     kda_status st = validate(q, k, v, log_alpha, beta, initial_state, nullptr, kda::kChunk, out,
-                             final_state, d, true, &a);
+                             final_state, d, false, &a);
     if (st != KDA_OK) return st;
     if (!(a.bf16 && a.dk == 128 && a.dv == 128))
         return fail(KDA_ERR_UNSUPPORTED, "kda_span_forward needs bf16 q/k/v with d_k = d_v = 128");
@@ -832,6 +845,16 @@ kda_status kda_span_forward(const void* q, const void* k, const void* v, const f
                            "final_state"}};
     for (const Range& r : outs)
         if (overlaps(rw, r)) return fail(KDA_ERR_ALIAS, "workspace overlaps %s", r.name);
+    if (opts && opts->snap && opts->snap_pool) {
+        const kda_snap_spec* sp = opts->snap;
+        const Range rp = {(uintptr_t)opts->snap_pool,
+                          (uintptr_t)opts->snap_pool + (uintptr_t)std::max(sp->num_slots, 0) * a.H * 128 * 128 * 4,
+                          "snap_pool"};
+        if (overlaps(rw, rp)) return fail(KDA_ERR_ALIAS, "workspace overlaps snap_pool");
+    }
+    // option checks and the device-memory check of every caller buffer
+    st = apply_opts(opts, q, k, v, log_alpha, beta, initial_state, nullptr, out, final_state, &a);
+    if (st != KDA_OK) return st;
     const void* wp[] = {workspace};
     const char* wn[] = {"workspace"};
     st = check_accessible(wp, wn, 1);
@@ -842,12 +865,26 @@ kda_status kda_span_forward(const void* q, const void* k, const void* v, const f
     t.s0 = initial_state;
     t.out = out;
     t.s_final = final_state;
+    t.gate = a.gate;
+    t.snap_slots = a.snap_slots;
+    t.snap_pool = a.snap_pool;
+    t.snap_interval = a.snap_interval;
+    t.snap_max = a.snap_max;
+    t.snap_num_slots = a.snap_num_slots;
     int launches = 0;
     g_last_path = "tc";
     cudaError_t e = kda::launch_tc(t, w.p, (cudaStream_t)stream, &launches, /*from_cache=*/true);
     g_last_launches = launches;
     if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
     return KDA_OK;
+}
+
+kda_status kda_span_forward(const void* q, const void* k, const void* v, const float* log_alpha,
+                            const float* beta, const float* initial_state, void* out,
+                            float* final_state, const kda_dims* d, const void* workspace,
+                            size_t workspace_bytes, void* stream) {
+    return kda_span_forward_ex(q, k, v, log_alpha, beta, initial_state, out, final_state, d,
+                               workspace, workspace_bytes, nullptr, stream);
 }
 
 kda_status kda_apply_transitions(const float* trans, int32_t count, int32_t B, int32_t H,

@@ -326,10 +326,18 @@ kda_status kda_apply_transitions(const float* trans, int32_t count, int32_t B, i
  *   argument).
  * kda_span_forward: kda_fwd on the same span (same k, v, log_alpha, beta and
  *   dims; q, initial_state, out, final_state as in kda_fwd) that takes the
- *   workspace's contents instead of recomputing them.  Results equal kda_fwd's
- *   bit for bit.  If the workspace was not filled by kda_span_transition on the
- *   same inputs the results are undefined.  It reads the workspace only, so one
- *   transition may serve several forward calls (e.g. retries).
+ *   workspace's contents instead of recomputing them.  Where kda_fwd cuts the
+ *   span into segments (long spans) it computes the same way, and the results
+ *   are equal bit for bit; otherwise they agree within kda_fwd's tolerance.
+ *   If the workspace was not filled by kda_span_transition on the same inputs
+ *   the results are undefined.  It reads the workspace only, so one transition
+ *   may serve several forward calls (e.g. retries).
+ * kda_span_forward_ex: kda_span_forward with the options of kda_fwd_ex (output
+ *   gate, prefix-cache snapshots), checked as there; the workspace may not
+ *   overlap snap_pool either.  Snapshot positions count tokens from the start
+ *   of the span, so a rank whose span starts at a multiple of the interval
+ *   takes snapshots at the same sequence positions as a whole-sequence call.
+ *   opts == NULL is kda_span_forward.
  */
 size_t kda_span_workspace_bytes(const kda_dims* dims);
 kda_status kda_span_transition(const void* k, const void* v, const float* log_alpha,
@@ -339,6 +347,11 @@ kda_status kda_span_forward(const void* q, const void* k, const void* v, const f
                             const float* beta, const float* initial_state, void* out,
                             float* final_state, const kda_dims* dims, const void* workspace,
                             size_t workspace_bytes, void* stream);
+kda_status kda_span_forward_ex(const void* q, const void* k, const void* v,
+                               const float* log_alpha, const float* beta,
+                               const float* initial_state, void* out, float* final_state,
+                               const kda_dims* dims, const void* workspace, size_t workspace_bytes,
+                               const kda_fwd_opts* opts, void* stream);
 
 /* Static description of a status code. */
 const char* kda_status_string(kda_status s);

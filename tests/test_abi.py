@@ -257,3 +257,34 @@ def test_span_workspace_size_and_bad_arguments():
         return kda.STATUS[rc]
 
     assert fwd_call(d=D(T=1 << 16, H=8, dt=0)) in ("KDA_ERR_UNSUPPORTED", "KDA_ERR_INVALID_ARG")
+
+    assert fwd_call(ws=FAKE + (8 << 30) + 16) == "KDA_ERR_MISALIGNED"
+    assert fwd_call(nbytes=n - 256) == "KDA_ERR_INVALID_ARG"
+    assert fwd_call(ws=FAKE + (5 << 30)) == "KDA_ERR_ALIAS"  # workspace over out
+
+
+def test_span_forward_ex_checks_its_options():
+    lib = kda.load_library()
+    P = lambda x: None if x is None else ctypes.c_void_p(x)
+    d = D(T=1 << 16, H=8)
+    n = lib.kda_span_workspace_bytes(ctypes.byref(d))
+
+    def call_ex(opts, ws=FAKE + (8 << 30)):
+        rc = lib.kda_span_forward_ex(P(FAKE), P(FAKE + (1 << 30)), P(FAKE + (2 << 30)),
+                                     P(FAKE + (3 << 30)), P(FAKE + (4 << 30)), None,
+                                     P(FAKE + (5 << 30)), None, ctypes.byref(d), P(ws), n,
+                                     None if opts is None else ctypes.byref(opts), None)
+        return kda.STATUS[rc]
+
+    gate = FAKE + (6 << 30)
+    assert call_ex(kda.FwdOpts(gate + 8, None, None, None)) == "KDA_ERR_MISALIGNED"
+    assert call_ex(kda.FwdOpts(FAKE + (5 << 30), None, None, None)) == "KDA_ERR_ALIAS"  # gate = out
+    spec = kda.SnapSpec(100, 4, 8)  # interval not a multiple of 64
+    assert call_ex(kda.FwdOpts(None, ctypes.pointer(spec), FAKE + (7 << 30),
+                               FAKE + (9 << 30))) == "KDA_ERR_INVALID_ARG"
+    spec = kda.SnapSpec(128, 4, 8)
+    assert call_ex(kda.FwdOpts(None, ctypes.pointer(spec), FAKE + (7 << 30), None)) \
+        == "KDA_ERR_INVALID_ARG"  # pool missing
+    # workspace placed over the snapshot pool
+    assert call_ex(kda.FwdOpts(None, ctypes.pointer(spec), FAKE + (7 << 30), FAKE + (8 << 30)),
+                   ws=FAKE + (8 << 30)) == "KDA_ERR_ALIAS"

@@ -194,3 +194,64 @@ def test_cp_prefill_with_output_gate(monkeypatch):
         assert torch.equal(o, o_ref) and torch.equal(f, f_ref)
     finally:
         dist.destroy_process_group()
+
+
+def test_span_forward_with_gate_and_snapshots_equals_kda_fwd(monkeypatch):
+    """kda_span_forward_ex from the workspace: with the span cut into segments it
+    takes kda_fwd's cached path, so output, state and snapshots equal
+    kda_fwd_snap's with the same gate bit for bit."""
+    import torch
+    from gated_delta_rule_139_b200 import (kda_fwd_snap, kda_span_forward, kda_span_transition,
+                                           span_workspace)
+    monkeypatch.setenv("KDA_SEG_CHUNKS", "2")
+    inp = make_inputs(2, 64 * 7 + 11, 2, 128, 128, bf16=True, seed=421, state_sigma=0.05,
+                      gate_sigma=2.0)
+    d = to_device(inp)
+    keys = ("q", "k", "v", "log_alpha", "beta")
+    gate = torch.rand(inp.v.shape, device="cuda").to(torch.bfloat16)
+    slots = torch.tensor([[0, -1, 1], [2, 3, 4]], dtype=torch.int32, device="cuda")
+    pools = [torch.full((6, 2, 128, 128), 3.0, device="cuda") for _ in range(2)]
+    ws = span_workspace(d["k"])
+    kda_span_transition(d["k"], d["v"], d["log_alpha"], d["beta"], ws)
+    o, f = kda_span_forward(*(d[k_] for k_ in keys), ws, d["initial_state"], out_gate=gate,
+                            snap_interval=128, snap_slots=slots, snap_pool=pools[0])
+    o_ref, f_ref = kda_fwd_snap(**{k_: d[k_] for k_ in keys}, initial_state=d["initial_state"],
+                                snap_interval=128, snap_slots=slots, snap_pool=pools[1],
+                                out_gate=gate)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o_ref) and torch.equal(f, f_ref)
+    assert torch.equal(pools[0], pools[1])
+    assert (pools[0][5] == 3.0).all()  # unused slot untouched
+
+
+def test_cp_snapshots_at_span_aligned_positions(monkeypatch):
+    """Two virtual ranks whose spans start at multiples of the interval: each
+    rank's snapshots (positions counted from its span's start) are the oracle's
+    prefix states at the matching whole-sequence positions."""
+    import torch
+    from gated_delta_rule_139_b200 import (kda_apply_transitions, kda_span_forward,
+                                           kda_span_transition, span_workspace)
+    monkeypatch.setenv("KDA_SEG_CHUNKS", "2")
+    span, interval = 64 * 4, 128
+    inp = make_inputs(1, 2 * span, 2, 128, 128, bf16=True, seed=422, state_sigma=0.05,
+                      gate_sigma=2.0)
+    d = to_device(inp)
+    keys = ("q", "k", "v", "log_alpha", "beta")
+    spans = [{k_: d[k_][:, r * span:(r + 1) * span].contiguous() for k_ in keys} for r in range(2)]
+    ws = [span_workspace(s["k"]) for s in spans]
+    trans = torch.stack([kda_span_transition(s["k"], s["v"], s["log_alpha"], s["beta"], w)
+                         for s, w in zip(spans, ws)])
+    pool = torch.zeros(4, 2, 128, 128, device="cuda")
+    for r, s in enumerate(spans):
+        s_in = kda_apply_transitions(trans[:r], d["initial_state"])
+        sl = torch.tensor([[2 * r, 2 * r + 1]], dtype=torch.int32, device="cuda")
+        kda_span_forward(*(s[k_] for k_ in keys), ws[r], s_in, snap_interval=interval,
+                         snap_slots=sl, snap_pool=pool)
+    torch.cuda.synchronize()
+    got = pool.cpu().numpy().astype(np.float64)
+    for j in range(4):  # whole-sequence positions 128, 256, 384, 512
+        L = (j + 1) * interval
+        _, ref = oracle.recurrent(inp.q[:, :L], inp.k[:, :L], inp.v[:, :L], inp.log_alpha[:, :L],
+                                  inp.beta[:, :L], inp.initial_state, o_tokens=0)
+        for h in range(2):
+            assert _rel(got[j, h], ref[0, h]) <= TOL_BF16_REL_FRO, (j, h)
