@@ -372,13 +372,14 @@ def run_cp_emulation(args):
     del full
     stream = torch.cuda.current_stream(dev)
     ws = [kda.span_workspace(s["k"]) for s in spans]
-    trans = [kda.kda_span_transition(s["k"], s["v"], s["log_alpha"], s["beta"], w)
+    trans = [kda.kda_span_transition(s["q"], s["k"], s["v"], s["log_alpha"], s["beta"], w)
              for s, w in zip(spans, ws)]
     gathered = torch.stack(trans)
 
     def rank_step(r):  # transition (kept work in ws[r]), incoming state, forward
         s = spans[r]
-        kda.kda_span_transition(s["k"], s["v"], s["log_alpha"], s["beta"], ws[r], out=trans[r])
+        kda.kda_span_transition(s["q"], s["k"], s["v"], s["log_alpha"], s["beta"], ws[r],
+                                out=trans[r])
         s_in = kda.kda_apply_transitions(gathered[:r], s0)
         return kda.kda_span_forward(s["q"], s["k"], s["v"], s["log_alpha"], s["beta"], ws[r], s_in)
 

@@ -90,7 +90,8 @@ def load_library():
         lib.kda_apply_transitions.restype = ctypes.c_int
         lib.kda_span_workspace_bytes.argtypes = [ctypes.POINTER(Dims)]
         lib.kda_span_workspace_bytes.restype = ctypes.c_size_t
-        lib.kda_span_transition.argtypes = [p, p, p, p, ctypes.POINTER(Dims), p, ctypes.c_size_t, p, p]
+        lib.kda_span_transition.argtypes = [p, p, p, p, p, ctypes.POINTER(Dims), p, ctypes.c_size_t, p,
+                                            p]
         lib.kda_span_transition.restype = ctypes.c_int
         lib.kda_span_forward.argtypes = [p, p, p, p, p, p, p, p, ctypes.POINTER(Dims), p,
                                          ctypes.c_size_t, p]
@@ -415,9 +416,10 @@ def span_workspace(k):
     return torch.empty(n, dtype=torch.uint8, device=k.device)
 
 
-def kda_span_transition(k, v, log_alpha, beta, workspace, out=None, stream=None):
-    """kda_transition that also leaves the span's segment transitions and W/U' in
-    ``workspace`` (from :func:`span_workspace`) for :func:`kda_span_forward`."""
+def kda_span_transition(q, k, v, log_alpha, beta, workspace, out=None, stream=None):
+    """kda_transition that also leaves the span's segment transitions and every
+    chunk's output-pass operands (hence q) in ``workspace`` (from
+    :func:`span_workspace`) for :func:`kda_span_forward`."""
     import torch
     lib = load_library()
     d = _span_dims(k)
@@ -426,7 +428,7 @@ def kda_span_transition(k, v, log_alpha, beta, workspace, out=None, stream=None)
     if stream is None:
         stream = torch.cuda.current_stream(k.device)
     ptr = lambda t: ctypes.c_void_p(t.data_ptr())
-    _check(lib.kda_span_transition(ptr(k), ptr(v), ptr(log_alpha), ptr(beta), ctypes.byref(d),
+    _check(lib.kda_span_transition(ptr(q), ptr(k), ptr(v), ptr(log_alpha), ptr(beta), ctypes.byref(d),
                                    ptr(workspace), workspace.numel(), ptr(out),
                                    ctypes.c_void_p(stream.cuda_stream)))
     return out

@@ -30,7 +30,7 @@ from typing import Callable
 
 @dataclass
 class SpanOps:
-    """The three per-rank steps.  ``transition(k, v, log_alpha, beta)`` returns
+    """The three per-rank steps.  ``transition(q, k, v, log_alpha, beta)`` returns
     (one tensor to exchange, all ranks the same shape; a context the forward
     step may reuse); ``apply(prior, initial_state)`` takes the stack of the
     earlier ranks' tensors ([r, ...], r may be 0); ``forward(q, k, v,
@@ -42,13 +42,13 @@ class SpanOps:
 
 def library_ops() -> SpanOps:
     """The library's kernels.  The transition step keeps its segment transitions
-    and per-chunk W, U' in a workspace, so the forward step does not compute
-    them again (kda_span_transition / kda_span_forward)."""
+    and every chunk's output-pass operands in a workspace, so the forward step
+    does not compute them again (kda_span_transition / kda_span_forward)."""
     from . import kda_apply_transitions, kda_span_forward, kda_span_transition, span_workspace
 
-    def transition(k, v, log_alpha, beta):
+    def transition(q, k, v, log_alpha, beta):
         ws = span_workspace(k)
-        return kda_span_transition(k, v, log_alpha, beta, ws), ws
+        return kda_span_transition(q, k, v, log_alpha, beta, ws), ws
 
     def forward(q, k, v, log_alpha, beta, s_in, out_gate, ws):
         return kda_span_forward(q, k, v, log_alpha, beta, ws, s_in, out_gate=out_gate)
@@ -67,7 +67,7 @@ def cp_prefill(q, k, v, log_alpha, beta, initial_state=None, group=None, out_gat
     ops = ops or library_ops()
     rank = dist.get_rank(group)
     world = dist.get_world_size(group)
-    trans, ctx = ops.transition(k, v, log_alpha, beta)
+    trans, ctx = ops.transition(q, k, v, log_alpha, beta)
     gathered = [torch.empty_like(trans) for _ in range(world)]
     dist.all_gather(gathered, trans.contiguous(), group=group)
     prior = torch.stack(gathered[:rank]) if rank else trans.new_empty((0,) + tuple(trans.shape))

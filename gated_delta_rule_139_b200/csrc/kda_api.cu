@@ -213,7 +213,7 @@ kda_status run_tc(const kda::FwdArgs& a, cudaStream_t stream, int* launches) {
     const size_t b_trans = p.segmented ? (size_t)p.max_units * a.H * 2 * st : 0;
     const size_t b_sin = p.segmented ? (size_t)p.max_units * a.H * st : 0;
     // W/U' cache of the segmented plan: 32 KB per chunk of every unit
-    const size_t b_wu = p.segmented ? (size_t)p.max_units * a.H * p.seg_chunks * 32768 : 0;
+    const size_t b_wu = p.segmented ? (size_t)p.max_units * a.H * p.seg_chunks * kda::kChunkImageBytes : 0;
     char* ws = nullptr;
     cudaError_t e = pool_alloc((void**)&ws, b_segs + b_off + b_trans + b_sin + b_wu, stream);
     if (e != cudaSuccess) return cuda_fail(e, "workspace allocation");
@@ -358,13 +358,14 @@ SpanWs span_layout(const kda::FwdArgs& a) {
     w.off = take((size_t)(a.N + 1) * 4 + 4);
     w.trans = take((size_t)w.p.max_units * a.H * 2 * st);
     w.sin = take((size_t)w.p.max_units * a.H * st);
-    w.wu = take((size_t)w.p.max_units * a.H * w.p.seg_chunks * 32768);
+    w.wu = take((size_t)w.p.max_units * a.H * w.p.seg_chunks * kda::kChunkImageBytes);
     w.total = o;
     return w;
 }
 
 kda::TcArgs span_args(const kda::FwdArgs& a, const SpanWs& w, char* ws) {
     kda::TcArgs t{};
+    t.q = a.q;
     t.k = a.k;
     t.v = a.v;
     t.log_alpha = a.log_alpha;
@@ -392,10 +393,11 @@ kda_status check_workspace(const void* ws, size_t bytes, size_t need) {
     return KDA_OK;
 }
 
-// Arguments of a span transition (k, v, log_alpha, beta; bf16, d = 128, no cu_seqlens).
-kda_status validate_span_inputs(const void* k, const void* v, const float* log_alpha,
+// Arguments of a span transition (k, v, log_alpha, beta; bf16, d = 128, no cu_seqlens);
+// need_q: q too (the transition that fills a span workspace prepares the output pass).
+kda_status validate_span_inputs(const void* q, const void* k, const void* v, const float* log_alpha,
                                 const float* beta, const kda_dims* d, const float* trans,
-                                kda::FwdArgs* a) {
+                                bool need_q, kda::FwdArgs* a) {
     if (!d) return fail(KDA_ERR_INVALID_ARG, "dims is NULL");
     if (d->B < 1 || d->T < 0 || d->H < 1)
         return fail(KDA_ERR_INVALID_ARG, "need B >= 1, T >= 0, H >= 1 (got B=%d T=%d H=%d)",
@@ -406,15 +408,18 @@ kda_status validate_span_inputs(const void* k, const void* v, const float* log_a
         return fail(KDA_ERR_UNSUPPORTED, "span transitions need bf16 k/v with d_k = d_v = 128");
     const int64_t tokens = (int64_t)d->B * d->T;
     if (!trans) return fail(KDA_ERR_INVALID_ARG, "trans must be non-NULL");
-    if (tokens > 0 && (!k || !v || !log_alpha || !beta))
-        return fail(KDA_ERR_INVALID_ARG, "k, v, log_alpha and beta must be non-NULL");
-    const void* ptrs[] = {k, v, log_alpha, beta, trans};
-    const char* names[] = {"k", "v", "log_alpha", "beta", "trans"};
-    for (int i = 0; i < 5; ++i)
+    if (tokens > 0 && (!k || !v || !log_alpha || !beta || (need_q && !q)))
+        return fail(KDA_ERR_INVALID_ARG, need_q ? "q, k, v, log_alpha and beta must be non-NULL"
+                                                : "k, v, log_alpha and beta must be non-NULL");
+    if (!need_q) q = nullptr;
+    const void* ptrs[] = {q, k, v, log_alpha, beta, trans};
+    const char* names[] = {"q", "k", "v", "log_alpha", "beta", "trans"};
+    for (int i = 0; i < 6; ++i)
         if (ptrs[i] && ((uintptr_t)ptrs[i] & 15u))
             return fail(KDA_ERR_MISALIGNED, "%s is not 16-byte aligned", names[i]);
     const int64_t n = tokens * d->H * 128;
-    const Range in[] = {{(uintptr_t)k, (uintptr_t)k + (k ? n * 2 : 0), "k"},
+    const Range in[] = {{(uintptr_t)q, (uintptr_t)q + (q ? n * 2 : 0), "q"},
+                        {(uintptr_t)k, (uintptr_t)k + (k ? n * 2 : 0), "k"},
                         {(uintptr_t)v, (uintptr_t)v + (v ? n * 2 : 0), "v"},
                         {(uintptr_t)log_alpha, (uintptr_t)log_alpha + (log_alpha ? n * 4 : 0),
                          "log_alpha"},
@@ -423,7 +428,7 @@ kda_status validate_span_inputs(const void* k, const void* v, const float* log_a
                       "trans"};
     for (const Range& r : in)
         if (overlaps(rt, r)) return fail(KDA_ERR_ALIAS, "trans overlaps %s", r.name);
-    a->q = nullptr;
+    a->q = q;
     a->k = k;
     a->v = v;
     a->log_alpha = log_alpha;
@@ -736,7 +741,7 @@ kda_status kda_transition(const void* k, const void* v, const float* log_alpha,
     g_last_launches = 0;
     g_last_path = "";
     kda::FwdArgs a;
-    kda_status st = validate_span_inputs(k, v, log_alpha, beta, d, trans, &a);
+    kda_status st = validate_span_inputs(nullptr, k, v, log_alpha, beta, d, trans, false, &a);
     if (st != KDA_OK) return st;
     const void* ptrs[] = {k, v, log_alpha, beta, trans};
     const char* names[] = {"k", "v", "log_alpha", "beta", "trans"};
@@ -784,21 +789,22 @@ size_t kda_span_workspace_bytes(const kda_dims* d) {
     return span_layout(a).total;
 }
 
-kda_status kda_span_transition(const void* k, const void* v, const float* log_alpha,
+kda_status kda_span_transition(const void* q, const void* k, const void* v, const float* log_alpha,
                                const float* beta, const kda_dims* d, void* workspace,
                                size_t workspace_bytes, float* trans, void* stream) {
     g_last_error[0] = 0;
     g_last_launches = 0;
     g_last_path = "";
     kda::FwdArgs a;
-    kda_status st = validate_span_inputs(k, v, log_alpha, beta, d, trans, &a);
+    kda_status st = validate_span_inputs(q, k, v, log_alpha, beta, d, trans, true, &a);
     if (st != KDA_OK) return st;
     const SpanWs w = span_layout(a);
     st = check_workspace(workspace, workspace_bytes, w.total);
     if (st != KDA_OK) return st;
     const int64_t tokens = (int64_t)a.B * a.T, n = tokens * a.H * 128;
     const Range rw = {(uintptr_t)workspace, (uintptr_t)workspace + w.total, "workspace"};
-    const Range other[] = {{(uintptr_t)k, (uintptr_t)k + (k ? n * 2 : 0), "k"},
+    const Range other[] = {{(uintptr_t)q, (uintptr_t)q + (q ? n * 2 : 0), "q"},
+                           {(uintptr_t)k, (uintptr_t)k + (k ? n * 2 : 0), "k"},
                            {(uintptr_t)v, (uintptr_t)v + (v ? n * 2 : 0), "v"},
                            {(uintptr_t)log_alpha, (uintptr_t)log_alpha + (log_alpha ? n * 4 : 0),
                             "log_alpha"},
@@ -807,9 +813,9 @@ kda_status kda_span_transition(const void* k, const void* v, const float* log_al
                             "trans"}};
     for (const Range& r : other)
         if (overlaps(rw, r)) return fail(KDA_ERR_ALIAS, "workspace overlaps %s", r.name);
-    const void* wp[] = {k, v, log_alpha, beta, trans, workspace};
-    const char* wn[] = {"k", "v", "log_alpha", "beta", "trans", "workspace"};
-    st = check_accessible(wp, wn, 6);
+    const void* wp[] = {q, k, v, log_alpha, beta, trans, workspace};
+    const char* wn[] = {"q", "k", "v", "log_alpha", "beta", "trans", "workspace"};
+    st = check_accessible(wp, wn, 7);
     if (st != KDA_OK) return st;
     kda::TcArgs t = span_args(a, w, (char*)workspace);
     int launches = 0;

@@ -76,7 +76,7 @@ struct TcArgs {
     float* sin;         // [max_units, H, 128, 128]: S_in^T of each segment
     const void* gate = nullptr;  // optional output gate, as in FwdArgs
     int32_t trans_all = 0;       // pass 1 also for each sequence's last segment
-    uint8_t* wu = nullptr;       // W/U' cache: [max_units][H][seg_chunks][32 KB] (pass 1 writes, pass 3 reads)
+    uint8_t* wu = nullptr;       // chunk cache: [max_units][H][seg_chunks][kChunkImageBytes] (pass 1 writes, pass 3 reads)
     int32_t seg_chunks = 0;      // chunks per segment (cache stride)
     // optional state snapshots, as in FwdArgs
     const int32_t* snap_slots = nullptr;
@@ -86,6 +86,11 @@ struct TcArgs {
 
 // TMA descriptors of the q, k, v, out, gate (bf16) and log_alpha (fp32)
 // tensors, viewed as [T, H, 128]; passed as a grid constant.
+// Bytes of one chunk's entry in the chunk cache that pass 1 leaves for pass 3:
+// the bf16 operand images of W^T, U'^T, K_dec, Q~ (16 KB each), P (8 KB) and
+// the fp32 chunk decay gamma (512 B).
+constexpr size_t kChunkImageBytes = 74240;
+
 struct TcMaps {
     CUtensorMap q, k, v, la, out, gate;
 };

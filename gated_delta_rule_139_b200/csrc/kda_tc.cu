@@ -16,13 +16,15 @@
 //   tc_kernel<1> "pass 1": per (segment, head) the transition (B, M) of the
 //                 segment, computed as the chunk loop applied to the augmented
 //                 state [B | M] from [0 | I].  When sequences are cut into
-//                 segments it runs over every segment and also keeps each
-//                 chunk's W^T and U'^T (bf16) in a cache for pass 3.
+//                 segments it runs over every segment and also leaves in a
+//                 chunk cache, for every chunk, the operand images pass 3
+//                 needs: W^T, U'^T, K_dec, Q~ and P (bf16) and gamma.
 //   seg_scan    : S_in(j+1) = M_j S_in(j) + B_j, sequential over the segments
 //                 of a sequence, parallel over (sequence, head, 16-row block).
-//   tc_kernel<2> "pass 3" with the cache: per (segment, head) the chunk loop
-//                 from the true incoming state, taking W^T and U'^T from the
-//                 cache (only P, the state products and the output remain).
+//   cached_kernel "pass 3" with the cache: per (segment, head) the state chain
+//                 from the true incoming state and the output, every chunk's
+//                 operands bulk-loaded from the cache (double-buffered), so
+//                 only the four state/output products remain per chunk.
 //   tc_kernel<0> "pass 3" without a cache (one segment per sequence): the full
 //                 chunk loop, writing o and the final state.
 //
@@ -76,12 +78,11 @@ constexpr float LOG2E = 1.4426950408889634f;
 //               over X1 and MA (bf16 M^T) after Ts.  The bf16 copies of S^T, B^T,
 //               U^T, U_B^T and U_M^T that the state products take as A operands
 //               live in tensor memory.
-//   MODE 2 (pass 3 with the W/U' cache): q~ in X1's rows 0-63, W^T in its rows
-//               64-127; no As/Ts/TB.
+//   pass 1 with the chunk cache also builds q~ in X1's rows 64-127 (so the phase-1
+//               product yields P in TMEM lanes 64-127) and P's bf16 image in GSUM.
 // RAW holds the next chunk's k, log alpha (and q) tiles, written by TMA while
 // the current chunk is processed; RV0/RV1 alternate as the chunk's v tile, which
-// TMA writes directly in the 128-byte-swizzled MN-major operand layout (MODE 2:
-// the chunk's U'^T from the cache).
+// TMA writes directly in the 128-byte-swizzled MN-major operand layout.
 template <bool SEG>
 struct LayT {
     static constexpr uint32_t X1 = 0, BT = 32768;
@@ -90,13 +91,11 @@ struct LayT {
     static constexpr uint32_t R1 = SEG ? 102400 : 69632;
     static constexpr uint32_t QT = R1;                            // pass 3: 64 x 128, K-major
     static constexpr uint32_t KD = SEG ? R1 : QT + 16384;         // 64 x 128, MN-major
-    static constexpr uint32_t UMA = KD + 16384;                   // pass 1: 128 x 64, K-major
     static constexpr uint32_t PB = KD + 16384;                    // pass 3: 64 x 64, K-major
-    static constexpr uint32_t RAW = SEG ? UMA + 16384 : PB + 8192;
+    static constexpr uint32_t RAW = SEG ? KD + 32768 : PB + 8192;
     static constexpr uint32_t RK = RAW, RL = RAW + 16384;
-    static constexpr uint32_t RQ = RAW + 49152;                   // pass 3 only
+    static constexpr uint32_t RQ = SEG ? KD + 16384 : RAW + 49152;  // pass 1: only with the cache
     static constexpr uint32_t RV = RAW + (SEG ? 49152 : 65536);   // two 16 KB buffers
-    static constexpr uint32_t RAW_TX = SEG ? 65536 : 81920;       // TMA bytes per chunk
     static constexpr uint32_t GSUM = RV + 32768;                  // fp32 [16][128]
     static constexpr uint32_t GAM = GSUM + 8192;                  // fp32 [128] e^{g_last}
     static constexpr uint32_t EHA = GAM + 512;                    // fp32 [128] e^{rho_a}
@@ -113,6 +112,7 @@ static_assert(LayT<false>::YS + 32 * 40 * 4 <= 32768 && LayT<false>::TB + 8192 <
               "Ys/TB must sit in the q-row holes of X1");
 static_assert(LayT<true>::WB + 16384 == LayT<true>::UA, "pass 1 stores W^T and U'^T as one 32 KB copy");
 static_assert(LayT<true>::MA + 32768 <= LayT<true>::R1, "MA overflow");
+static_assert(LayT<true>::RQ + 16384 <= LayT<true>::RAW, "pass 1 q tile");
 static_assert(LayT<false>::BYTES <= 232448 && LayT<true>::BYTES <= 232448, "shared memory");
 
 // TMEM columns (512 allocated).  Pass 3: AP [0,96) W [96,160) U [160,224)
@@ -125,6 +125,17 @@ constexpr uint32_t TM_UBB = 96, TM_UBM = 128;  // pass 1: bf16 U_B^T, U_M^T (A o
 // pass 1: bf16 B^T (A operand of U_B -= B W): K steps 0-3 (channels 0-63) in [64,96), which the
 // cross-half block of A has left, and K steps 4-7 in [224,256), unused in pass 1
 __device__ __forceinline__ uint32_t sbb_col(int s) { return s < 4 ? 64 + 8 * s : 224 + 8 * (s - 4); }
+
+// Chunk cache entry (kChunkImageBytes per chunk and head): the bf16 operand images as
+// they sit in shared memory, in 1024-byte aligned pieces (a bulk copy into a 1024-byte
+// aligned buffer keeps their 128-byte swizzle), then gamma.
+constexpr uint32_t CI_W = 0;        // W^T: MN-major, K rows = channels, MN = tokens
+constexpr uint32_t CI_U = 16384;    // U'^T: [128][64], 16-byte pieces of row e XOR-swizzled by e & 7
+constexpr uint32_t CI_KD = 32768;   // K_dec: MN-major, K rows = tokens, MN = channels
+constexpr uint32_t CI_QT = 49152;   // Q~ (q e^{g - rho} e^{rho}): K-major, 64 rows x 128
+constexpr uint32_t CI_PB = 65536;   // P: K-major, 64 x 64
+constexpr uint32_t CI_GAM = 73728;  // fp32 [128] e^{g_last}
+static_assert(CI_GAM + 512 == kChunkImageBytes, "chunk cache entry");
 
 __device__ __forceinline__ float clamp_gate(float x) { return fminf(fmaxf(x, -5.f), 0.f); }
 // 2^x by the SFU instruction (relative error about 2^-22, flushes results
@@ -321,7 +332,7 @@ __device__ __forceinline__ void warp_store16x8(float* dst, int ld, const float (
 //  3. T[32:64, 0:32] = -T_hi Z, written straight into TB.
 // The block products are tf32 warp MMAs with fp32 accumulation (T then enters
 // the chunk products as bf16).
-// `side(warp)` runs on warps 8-15 while warps 0-1 invert the diagonal blocks
+// `side(warp)` runs on warps 2-15 while warps 0-1 invert the diagonal blocks
 // (work that does not touch As, Ts, Ys or TB).  OWN_A: As has not been
 // extracted; warps 0-1 (TMEM lanes 0-63 = rows of A, tq = their lane quadrant)
 // read their rows of A from the product in TMEM, scale by beta, mask, and write
@@ -406,10 +417,11 @@ __device__ void invert_to_tb(float* As, float* Ts, float* Ys, const float* beta,
             warp_store16x8(Ts + (o + 16) * TS_LD + o + 8 * nt, TS_LD, d, -1.f, lane);
         }
         __syncwarp();
-    } else if (warp < 6) {  // zero TB rows 0..31, columns 32..63: 128 chunks
-        const int id = tid - 64, r = id >> 2, j8 = 4 + (id & 3);
-        st_shared_v4(tbp + kmajor_chunk_off(r, j8, 64), 0u, 0u, 0u, 0u);
-    } else if (warp >= 8) {
+    } else {
+        if (warp < 6) {  // zero TB rows 0..31, columns 32..63: 128 chunks
+            const int id = tid - 64, r = id >> 2, j8 = 4 + (id & 3);
+            st_shared_v4(tbp + kmajor_chunk_off(r, j8, 64), 0u, 0u, 0u, 0u);
+        }
         side(warp);
     }
     __syncthreads();
@@ -450,12 +462,36 @@ __device__ void invert_to_tb(float* As, float* Ts, float* Ys, const float* beta,
     }
 }
 
+// Row r (0-63) of P, columns j0..j0+15 (j0 a multiple of 16), from the [A;P] product
+// in TMEM (P's rows in lanes 64-127; tq = the calling warp's lane quadrant): the
+// lower-inclusive mask, bf16, into the K-major 64 x 64 image at pb.  Columns j < 32
+// of rows r >= 32 are the cross-half product (TMEM columns 64 + j); rows r < 32 have
+// nothing in columns j >= 32.  Warp-uniform: r < 32 for the whole quadrant or none.
+__device__ __forceinline__ void extract_p16(uint32_t tq, int r, int j0, uint32_t pb) {
+    float x[16];
+    if (j0 >= 32 && r < 32) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) x[i] = 0.f;
+    } else {
+        float v[16];
+        tmem_ld16(tq + TM_AP + (j0 < 32 && r >= 32 ? 64 + j0 : j0), v);
+        tmem_wait16(v);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) x[i] = j0 + i <= r ? v[i] : 0.f;
+    }
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh)
+        st_shared_v4(pb + kmajor_chunk_off(r, (j0 >> 3) + hh, 64), pack_bf16(x[8 * hh], x[8 * hh + 1]),
+                     pack_bf16(x[8 * hh + 2], x[8 * hh + 3]), pack_bf16(x[8 * hh + 4], x[8 * hh + 5]),
+                     pack_bf16(x[8 * hh + 6], x[8 * hh + 7]));
+}
+
 // ---------------------------------------------------------------- the chunk loop
-// MODE 0: pass 3 (forward from the true incoming state); MODE 1: pass 1 (segment
-// transitions); MODE 2: pass 3 that takes each chunk's W and U' from pass 1's cache.
+// MODE 0: pass 3 without a cache (forward from the true incoming state); MODE 1:
+// pass 1 (segment transitions; with a.wu set, also the chunk cache for pass 3).
 template <int MODE>
 __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_constant__ TcMaps maps) {
-    constexpr bool SEG = MODE == 1, FAST = MODE == 2;
+    constexpr bool SEG = MODE == 1;
     using Lay = LayT<SEG>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -469,14 +505,12 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
     const bool snap_on = !SEG && a.snap_pool != nullptr;
     const bool gate_on = !SEG && a.gate != nullptr;
     uint32_t gate_parity = 0;
-    // W/U' cache: pass 1 stores each chunk's W^T (the 16 KB bf16 MN-major B operand of
-    // phase 5) and U'^T (bf16 [128][64], 16-byte pieces of row e XOR-swizzled by e & 7);
-    // MODE 2 loads them instead of building A, T, W and U' again.  Entry of chunk t of
-    // unit u: wu + ((u H + h) seg_chunks + chunk) * 32 KB, W^T first.
-    const bool wu_cache = a.wu != nullptr;
-    uint32_t w_parity = 0;
+    // Chunk cache (pass 1): entry of chunk t of unit u at
+    // wu + ((u H + h) seg_chunks + chunk) * kChunkImageBytes, pieces at the CI_* offsets.
+    const bool wu_cache = SEG && a.wu != nullptr;
     auto wu_tile = [&](int64_t tt) {
-        return a.wu + ((((int64_t)u * H + h) * a.seg_chunks + (tt - sg.t_begin) / C) << 15);
+        return a.wu + (((int64_t)u * H + h) * a.seg_chunks + (tt - sg.t_begin) / C) *
+                          (int64_t)kChunkImageBytes;
     };
     const int64_t seq_lo = snap_on ? (a.cu ? (int64_t)a.cu[sg.n] : (int64_t)sg.n * a.T) : 0;
 
@@ -488,15 +522,7 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + Lay::BAR);
     uint64_t* bar_raw = bar + 1;
     uint64_t* bar_gate = bar + 2;  // output-gate tile (pass 3 with a gate)
-    uint64_t* bar_w = bar + 3;     // W^T tile from the cache (MODE 2)
     uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(sm + Lay::TMEMP);
-    // MODE 2 keeps q~ in rows 0-63 of X1; rows 64-127 hold W^T in two 8 KB pieces
-    // (K steps 0-3 and 4-7 of the MN-major operand)
-    auto load_w = [&](int64_t tt) {
-        mbar_expect_tx(bar_w, 16384);
-        bulk_load(sm + Lay::X1 + 8192, wu_tile(tt), 8192, bar_w);
-        bulk_load(sm + Lay::X1 + 24576, wu_tile(tt) + 8192, 8192, bar_w);
-    };
 
     if (warp == 0) {
         tmem_alloc(tmem_ptr, 512);
@@ -506,7 +532,6 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
         mbar_init(bar, 1);
         mbar_init(bar_raw, 1);
         mbar_init(bar_gate, 1);
-        mbar_init(bar_w, 1);
         fence_mbar_init();
     }
     tc_fence_before();
@@ -554,24 +579,22 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
     // The next chunk's q, k, v and log alpha tiles are copied by TMA into RAW
     // while the current chunk is processed (issued once every thread has read
     // the current tiles into registers); beta goes through registers.
+    const bool with_q = !SEG || wu_cache;  // pass 1 needs q only to fill the chunk cache
+    bool raw_pending = false, gate_pending = false;  // thread 0: TMA loads in flight
     auto issue_raw = [&](int64_t tn, int vbuf) {
-        mbar_expect_tx(bar_raw, Lay::RAW_TX);
+        raw_pending = true;
+        mbar_expect_tx(bar_raw, with_q ? 81920u : 65536u);  // k, log alpha, v (, q)
         tma_tile(sm + Lay::RK, &maps.k, 0, h, (int)tn, bar_raw);
         tma_tile(sm + Lay::RL, &maps.la, 0, h, (int)tn, bar_raw);
-        if (!SEG) tma_tile(sm + Lay::RQ, &maps.q, 0, h, (int)tn, bar_raw);
-        uint8_t* rv = sm + Lay::RV + vbuf * 16384;
-        if (FAST) {  // U'^T from the cache instead of v
-            bulk_load(rv, wu_tile(tn) + 16384, 16384, bar_raw);
-        } else {     // two 64-channel swizzled halves
-            tma_tile(rv, &maps.v, 0, h, (int)tn, bar_raw);
-            tma_tile(rv + 8192, &maps.v, 64, h, (int)tn, bar_raw);
-        }
+        if (with_q) tma_tile(sm + Lay::RQ, &maps.q, 0, h, (int)tn, bar_raw);
+        uint8_t* rv = sm + Lay::RV + vbuf * 16384;  // two 64-channel swizzled halves
+        tma_tile(rv, &maps.v, 0, h, (int)tn, bar_raw);
+        tma_tile(rv + 8192, &maps.v, 64, h, (int)tn, bar_raw);
     };
     uint32_t raw_parity = 0;
     float beta_ld = 0.f;
     if (sg.t_begin < sg.t_end) {
         if (tid == 0) issue_raw(sg.t_begin, 0);
-        if (FAST && tid == 0) load_w(sg.t_begin);
         if (tid < C && sg.t_begin + tid < sg.t_end) beta_ld = __ldg(a.beta + (sg.t_begin + tid) * H + h);
     }
 
@@ -585,10 +608,12 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
             const int c4 = lane, tg = warp, c0 = 4 * c4;  // tokens 4tg..4tg+3, channels c0..c0+3
             float4 la[4];
             uint2 kr[4], qr[4];
-            if (SEG && wu_cache && tid == 0) bulk_wait_read();  // last chunk's W^T has left WB
+            // the last chunk's cache stores have read WB, UA, KD, GSUM and GAM
+            if (wu_cache && tid == 0) bulk_wait_read();
             if (!(ok = !__syncthreads_or(!mbar_wait(bar_raw, raw_parity, &g_tc_status,
                                                     ERR_WAIT_TIMEOUT)))) break;
             raw_parity ^= 1u;
+            raw_pending = false;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {  // rows past the segment end act as identity steps
                 const int r = 4 * tg + i;
@@ -597,8 +622,8 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
                 if (r < Lc) {
                     la[i] = *reinterpret_cast<const float4*>(sm + Lay::RL + (r * D + c0) * 4);
                     kr[i] = *reinterpret_cast<const uint2*>(sm + Lay::RK + (r * D + c0) * 2);
-                    if (!SEG) qr[i] = *reinterpret_cast<const uint2*>(sm + Lay::RQ + (r * D + c0) * 2);
-                } else if (!FAST) {  // the v tile is an operand as TMA wrote it: clear rows past the end
+                    if (with_q) qr[i] = *reinterpret_cast<const uint2*>(sm + Lay::RQ + (r * D + c0) * 2);
+                } else {  // the v tile is an operand as TMA wrote it: clear rows past the end
                     *reinterpret_cast<uint2*>(sm + Lay::RV + vbuf * 16384 + mnmajor_off(r, c0, 64)) =
                         make_uint2(0u, 0u);
                 }
@@ -675,11 +700,10 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
                     e1[c] = ex2(d2);
                     e2[c] = ex2(-d2);
                 }
-                if (!FAST)
-                    st8(sm + Lay::X1, kmajor_off(r, c0, 128), kf[0] * e1[0], kf[1] * e1[1],
-                        kf[2] * e1[2], kf[3] * e1[3]);
-                if (!SEG)
-                    st8(sm + Lay::X1, kmajor_off(FAST ? r : 64 + r, c0, 128), qf[0] * e1[0],
+                st8(sm + Lay::X1, kmajor_off(r, c0, 128), kf[0] * e1[0], kf[1] * e1[1],
+                    kf[2] * e1[2], kf[3] * e1[3]);
+                if (with_q)
+                    st8(sm + Lay::X1, kmajor_off(64 + r, c0, 128), qf[0] * e1[0],
                         qf[1] * e1[1], qf[2] * e1[2], qf[3] * e1[3]);
                 st8(sm + Lay::BT, kmajor_off(r, c0, 96), kf[0] * e2[0], kf[1] * e2[1],
                     kf[2] * e2[2], kf[3] * e2[3]);
@@ -688,6 +712,10 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
                         kf[1] * e2[1] * fba[1], kf[2] * e2[2] * fba[2], kf[3] * e2[3] * fba[3]);
                 if (!SEG)
                     st8(sm + Lay::QT, kmajor_off(r, c0, 64), qf[0] * e1[0] * Eh[0],
+                        qf[1] * e1[1] * Eh[1], qf[2] * e1[2] * Eh[2], qf[3] * e1[3] * Eh[3]);
+                else if (wu_cache)  // Q~'s image straight into the cache: each warp row is
+                                    // two contiguous 128-byte pieces
+                    st8(wu_tile(t0) + CI_QT, kmajor_off(r, c0, 64), qf[0] * e1[0] * Eh[0],
                         qf[1] * e1[1] * Eh[1], qf[2] * e1[2] * Eh[2], qf[3] * e1[3] * Eh[3]);
                 st8(sm + Lay::KD, mnmajor_off(r, c0, 64), kf[0] * e2[0] * Dh[0],
                     kf[1] * e2[1] * Dh[1], kf[2] * e2[2] * Dh[2], kf[3] * e2[3] * Dh[3]);
@@ -706,28 +734,11 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
             for (int s = 0; s < 8; ++s)
                 mma_bf16(tmem + TM_AP, kmajor_desc(x1, 128, s), kmajor_desc(bt, 96, s), id, s > 0);
             mma_commit(bar);
-        }
-        if (FAST) {
-            // meanwhile: bf16 copy of the state (S^T scaled by gamma in TMEM afterwards), and
-            // the chunk's U'^T from the cache into the U accumulator
-            const int c0 = 32 * wg, r0 = 16 * wg;
-            stage_cols_tmem<2>(tq + TM_S + c0, tq + TM_SB + c0 / 2, c0, gam, true);
-            const uint8_t* ru = sm + Lay::RV + vbuf * 16384 + lrow * 128;
-            float v[16];
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const uint4 x = *reinterpret_cast<const uint4*>(ru + ((((r0 >> 3) + hh) ^ (lrow & 7)) << 4));
-                float lo4[4], hi4[4];
-                unpack_bf16x4(make_uint2(x.x, x.y), lo4);
-                unpack_bf16x4(make_uint2(x.z, x.w), hi4);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    v[8 * hh + i] = lo4[i];
-                    v[8 * hh + 4 + i] = hi4[i];
-                }
+            if (wu_cache) {  // K_dec and gamma are final: into the chunk cache
+                bulk_store(wu_tile(t0) + CI_KD, sm + Lay::KD, 16384);
+                bulk_store(wu_tile(t0) + CI_GAM, sm + Lay::GAM, 512);
+                bulk_commit();
             }
-            tmem_st16(tq + TM_U + r0, v);
-            tmem_st_wait();
         }
         if (!(ok = wait_mma(bar, parity))) break;
 
@@ -736,73 +747,56 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
             float* As = reinterpret_cast<float*>(sm + Lay::AS);
             float* Ts = reinterpret_cast<float*>(sm + Lay::TS);
             float* Ys = reinterpret_cast<float*>(sm + Lay::YS);
-            // rows r of A (lanes 0-63) and P (lanes 64-127); warp slice wg handles the 16
-            // columns j in [16wg, 16wg+16).  Columns j < 32 of rows r >= 32 come from the
-            // cross-half product (TMEM columns 64 + j).
-            // MODE 2 needs only P, which it finds in rows 0-63 (q~ sits there in X1)
-            const bool need_a = !FAST;
-            if (!SEG && (!FAST || quad < 2)) {  // pass 1 extracts A inside the inversion
-                const int r = lrow & 63;
-                const bool isP = FAST || quad >= 2;
-                const bool lower_half = r < 32;  // warp-uniform
-                const int j0 = 16 * wg;
-                float x[16];
-                if (j0 >= 32 && lower_half) {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) x[i] = 0.f;
+            // MODE 0: rows r of A (lanes 0-63) into As and of P (lanes 64-127) into PB; warp
+            // slice wg handles the 16 columns j in [16wg, 16wg+16).  Pass 1 extracts A
+            // inside the inversion (and, with the cache, P beside it).
+            if (!SEG) {
+                const int r = lrow & 63, j0 = 16 * wg;
+                if (quad >= 2) {
+                    extract_p16(tq, r, j0, smem_u32(sm + Lay::PB));
                 } else {
-                    float v[16];
-                    tmem_ld16(tq + TM_AP + (j0 < 32 && !lower_half ? 64 + j0 : j0), v);
-                    tmem_wait16(v);
-                    const float br = beta_s[r];
+                    float x[16];
+                    if (j0 >= 32 && r < 32) {  // warp-uniform
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int j = j0 + i;
-                        x[i] = isP ? (j <= r ? v[i] : 0.f) : (j < r ? br * v[i] : 0.f);
+                        for (int i = 0; i < 16; ++i) x[i] = 0.f;
+                    } else {  // columns j < 32 of rows r >= 32: the cross-half product
+                        float v[16];
+                        tmem_ld16(tq + TM_AP + (j0 < 32 && r >= 32 ? 64 + j0 : j0), v);
+                        tmem_wait16(v);
+                        const float br = beta_s[r];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) x[i] = j0 + i < r ? br * v[i] : 0.f;
                     }
-                }
-                if (!isP) {
 #pragma unroll
                     for (int i = 0; i < 16; ++i) As[r * AS_LD + j0 + i] = x[i];
-                } else {
-                    const uint32_t pb = smem_u32(sm + Lay::PB);
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh)
-                        st_shared_v4(pb + kmajor_chunk_off(r, 2 * wg + hh, 64),
-                                     pack_bf16(x[8 * hh], x[8 * hh + 1]),
-                                     pack_bf16(x[8 * hh + 2], x[8 * hh + 3]),
-                                     pack_bf16(x[8 * hh + 4], x[8 * hh + 5]),
-                                     pack_bf16(x[8 * hh + 6], x[8 * hh + 7]));
                 }
+                __syncthreads();
             }
-            if (!SEG) __syncthreads();
-            if (need_a) {
-                // beside the diagonal inversions: pass 1 stages M (bf16 M^T -> MA, M scaled by
-                // gamma in TMEM) on warps 8-15, which own two 64-column slices per quadrant
-                invert_to_tb<SEG>(As, Ts, Ys, beta_s, smem_u32(sm + Lay::TB), tid, tq, [&](int w) {
-                    if (SEG) {
-                        const int c0 = 64 * ((w >> 2) - 2);
-                        stage_cols<4>(tq + TM_M + c0, sm + Lay::MA, 128, lrow, c0, gam, true);
-                        tmem_st_wait();
-                    }
-                });
-            }
+            // beside the diagonal inversions, pass 1 stages M (bf16 M^T -> MA, M scaled by
+            // gamma in TMEM) on warps 8-15, which own two 64-column slices per quadrant, and
+            // with the cache puts P (TMEM lanes 64-127) into GSUM on warps 2, 3, 6, 7
+            invert_to_tb<SEG>(As, Ts, Ys, beta_s, smem_u32(sm + Lay::TB), tid, tq, [&](int w) {
+                if (!SEG) return;
+                if (w >= 8) {
+                    const int c0 = 64 * ((w >> 2) - 2);
+                    stage_cols<4>(tq + TM_M + c0, sm + Lay::MA, 128, lrow, c0, gam, true);
+                    tmem_st_wait();
+                } else if (wu_cache && (w & 3) >= 2) {
+                    const int j0 = 32 * (w >> 2);  // warps 2, 3: columns 0-31; 6, 7: 32-63
+                    extract_p16(tq, lrow - 64, j0, smem_u32(sm + Lay::GSUM));
+                    extract_p16(tq, lrow - 64, j0 + 16, smem_u32(sm + Lay::GSUM));
+                }
+            });
         }
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
-        // MODE 2: U'^T has gone to TMEM, so its buffer may receive the output gate's tile
-        if (FAST && gate_on && tid == 0) {
-            mbar_expect_tx(bar_gate, 16384);
-            tma_tile(sm + Lay::RV + vbuf * 16384, &maps.gate, 0, h, (int)t0, bar_gate);
-        }
 
         // ============ phase 3: with TB = T diag(beta) and the per-half factors e^{rho_h}:
         //   W^T  = e^{rho_a} (X1k_a)^T TB_a^T + e^{rho_b} (X1k_b)^T TB_b^T  (combined at staging)
         //   U'^T = V^T TB^T
         // X1's k rows serve as an MN-major operand (K rows = tokens, MN blocks 16 KB apart);
         // the v tile is used as TMA wrote it.
-        if (!FAST) {  // MODE 2 has W^T and U'^T from the cache
         if (tid == 0) {
             tc_fence_after();
             const uint32_t x1 = smem_u32(sm + Lay::X1), tb = smem_u32(sm + Lay::TB),
@@ -837,6 +831,7 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
         // The v tile is consumed: the output gate's [64][128] tile (if any) goes into
         // its buffer now, for the epilogue.
         if (gate_on && tid == 0) {
+            gate_pending = true;
             mbar_expect_tx(bar_gate, 16384);
             tma_tile(sm + Lay::RV + vbuf * 16384, &maps.gate, 0, h, (int)t0, bar_gate);
         }
@@ -876,33 +871,23 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
-        if (SEG && wu_cache && tid == 0) {  // keep W^T and U'^T (WB, UA: 32 KB) for pass 3
-            bulk_store(wu_tile(t0), sm + Lay::WB, 32768);
+        if (wu_cache && tid == 0) {  // W^T, U'^T (WB, UA: 32 KB) and P (GSUM) into the chunk cache
+            bulk_store(wu_tile(t0) + CI_W, sm + Lay::WB, 32768);
+            bulk_store(wu_tile(t0) + CI_PB, sm + Lay::GSUM, 8192);
             bulk_commit();
         }
-        }  // !FAST
 
         // ============ phase 5: U^T -= S^T W^T ; O^T = S^T Q~^T  (pass 1: U_M^T = -M^T W^T)
-        bool w_ok = true;
-        if (FAST && tid == 0) {  // this chunk's W^T from the cache
-            w_ok = mbar_wait(bar_w, w_parity, &g_tc_status, ERR_WAIT_TIMEOUT);
-            w_parity ^= 1u;
-        }
-        if (tid == 0 && w_ok) {
+        if (tid == 0) {
             tc_fence_after();
             const uint32_t wb = smem_u32(sm + Lay::WB);
             constexpr uint32_t id_neg = idesc_bf16(128, 64, false, true, true);
             if (!SEG) {  // A = bf16 S^T from TMEM
                 const uint32_t qt = smem_u32(sm + Lay::QT);
                 constexpr uint32_t id = idesc_bf16(128, 64, false, false);
-                const uint32_t x1 = smem_u32(sm + Lay::X1);
 #pragma unroll
-                for (int s = 0; s < 8; ++s) {
-                    // MODE 2: K steps 0-3 at X1 + 8 KB, 4-7 at X1 + 24 KB (the cache's pieces)
-                    const uint64_t wd = FAST ? sdesc(x1 + (s < 4 ? 8192 : 24576) + 2048 * (s & 3), 128 * 128, 1024)
-                                             : mnmajor_desc(wb, 128, s);
-                    mma_bf16_ts(tmem + TM_U, tmem + TM_SB + 8 * s, wd, id_neg, 1);
-                }
+                for (int s = 0; s < 8; ++s)
+                    mma_bf16_ts(tmem + TM_U, tmem + TM_SB + 8 * s, mnmajor_desc(wb, 128, s), id_neg, 1);
 #pragma unroll
                 for (int s = 0; s < 8; ++s)
                     mma_bf16_ts(tmem + TM_O, tmem + TM_SB + 8 * s, kmajor_desc(qt, 64, s), id, s > 0);
@@ -919,7 +904,6 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
             mma_commit(bar);
         }
         if (!(ok = wait_mma(bar, parity))) break;
-        if (FAST && tid == 0 && t0 + C < sg.t_end) load_w(t0 + C);  // W^T consumed: the next one
 
         // ============ phase 6: bf16 U^T into TMEM as the next products' A operand (pass 1:
         // U_B^T and U_M^T, in the W columns, which W staging has emptied)
@@ -978,6 +962,7 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
                 if (!(ok = !__syncthreads_or(!mbar_wait(bar_gate, gate_parity, &g_tc_status,
                                                         ERR_WAIT_TIMEOUT)))) break;
                 gate_parity ^= 1u;
+                gate_pending = false;
 #pragma unroll
                 for (int i = 0; i < 16; ++i) v[i] *= __bfloat162float(os[(r0 + i) * D + lrow]);
             }
@@ -1021,6 +1006,11 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
     }
 
     // ---- results of the segment
+    if (!ok && tid == 0) {  // after a timeout: bounded waits for what may still be in flight
+        mbar_wait(bar, parity ^ 1u, &g_tc_status, ERR_WAIT_TIMEOUT);
+        if (raw_pending) mbar_wait(bar_raw, raw_parity, &g_tc_status, ERR_WAIT_TIMEOUT);
+        if (gate_pending) mbar_wait(bar_gate, gate_parity, &g_tc_status, ERR_WAIT_TIMEOUT);
+    }
     if (tid == 0 && (!SEG || wu_cache)) bulk_wait_all();  // output / cache stores are complete
     if (ok) {
         if (SEG) {  // slices 0-1: B^T, slices 2-3: M^T, 64 columns each
@@ -1045,6 +1035,262 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
 #pragma unroll
                 for (int i = 0; i < 16; ++i) sf[(int64_t)(c0 + i) * D + lrow] = v[i];
             }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+// ---------------------------------------------------------------- pass 3 from the chunk cache
+// Shared memory: two chunk images (the cache entry as pass 1 wrote it, 1024-byte
+// aligned), the output tile and the output gate's tile.
+struct LayC {
+    static constexpr uint32_t IMG = 0, IMG_STRIDE = 75776;  // kChunkImageBytes rounded to 1 KB
+    static constexpr uint32_t OUT = 2 * IMG_STRIDE;         // bf16 [64][128]
+    static constexpr uint32_t GATE = OUT + 16384;           // bf16 [64][128]
+    static constexpr uint32_t BAR = GATE + 16384;           // mbarriers: MMA, image 0, image 1, gate
+    static constexpr uint32_t TMEMP = BAR + 32;
+    static constexpr uint32_t BYTES = TMEMP + 16 + 1024;    // + alignment slack
+};
+static_assert(LayC::IMG_STRIDE >= kChunkImageBytes && LayC::IMG_STRIDE % 1024 == 0, "image stride");
+static_assert(LayC::BYTES <= 232448, "shared memory");
+
+// Per (segment, head): the state chain from the true incoming state and the output.
+// Per chunk, with its image in shared memory (loaded two chunks ahead):
+//   bf16 S^T -> TMEM, S^T *= gamma, U'^T -> the U accumulator        (all threads)
+//   U^T -= S^T W^T ;  O^T = S^T Q~^T                                   (one thread)
+//   bf16 U^T -> TMEM                                                   (all threads)
+//   O^T += U^T P^T ;  S^T += U^T K_dec                                 (one thread)
+//   O^T (x gate) -> bf16 tile -> TMA store                             (all threads)
+// TMEM columns as in tc_kernel's pass 3.  The same products in the same precision
+// as tc_kernel<0>, so the two paths differ only in where W, U', Q~, K_dec, P and
+// gamma come from.
+__global__ void __launch_bounds__(NT, 1) cached_kernel(TcArgs a, const __grid_constant__ TcMaps maps) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int u = blockIdx.x, h = blockIdx.y, H = a.H;
+    if (u >= *a.n_units) return;
+    const SegEntry sg = a.segs[u];
+    const bool snap_on = a.snap_pool != nullptr;
+    const bool gate_on = a.gate != nullptr;
+    const int64_t seq_lo = snap_on ? (a.cu ? (int64_t)a.cu[sg.n] : (int64_t)sg.n * a.T) : 0;
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + LayC::BAR);  // MMA completion
+    uint64_t* bar_img = bar + 1;                                  // [2] image loads
+    uint64_t* bar_gate = bar + 3;                                 // output-gate tile
+    uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(sm + LayC::TMEMP);
+    auto entry = [&](int64_t tt) {
+        return a.wu + (((int64_t)u * H + h) * a.seg_chunks + (tt - sg.t_begin) / C) *
+                          (int64_t)kChunkImageBytes;
+    };
+    uint32_t pending = 0;  // thread 0: bit b = a load into image b in flight; bit 2 = gate tile
+    auto load_img = [&](int64_t tt, int b) {
+        pending |= 1u << b;
+        mbar_expect_tx(bar_img + b, (uint32_t)kChunkImageBytes);
+        bulk_load(sm + LayC::IMG + b * LayC::IMG_STRIDE, entry(tt), (uint32_t)kChunkImageBytes,
+                  bar_img + b);
+    };
+    auto load_gate = [&](int64_t tt) {
+        pending |= 4u;
+        mbar_expect_tx(bar_gate, 16384);
+        tma_tile(sm + LayC::GATE, &maps.gate, 0, h, (int)tt, bar_gate);
+    };
+
+    if (warp == 0) {
+        tmem_alloc(tmem_ptr, 512);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        mbar_init(bar_img, 1);
+        mbar_init(bar_img + 1, 1);
+        mbar_init(bar_gate, 1);
+        fence_mbar_init();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_ptr;
+    const int quad = warp & 3, wg = warp >> 2, lrow = quad * 32 + lane;
+    const uint32_t tq = tmem + ((uint32_t)(quad * 32) << 16);
+    if (tid == 0 && sg.t_begin < sg.t_end) {  // the first two chunks' images
+        load_img(sg.t_begin, 0);
+        if (sg.t_begin + C < sg.t_end) load_img(sg.t_begin + C, 1);
+        if (gate_on) load_gate(sg.t_begin);
+    }
+    // initial state: slice wg writes columns 32wg..32wg+31 of S^T
+    {
+        const int e = lrow, cb = 32 * wg;
+        for (int c0 = cb; c0 < cb + 32; c0 += 16) {
+            float v[16];
+            if (sg.j == 0 && sg.last) {  // single segment: the caller's state
+                const float* s0 = a.s0 ? a.s0 + ((int64_t)sg.n * H + h) * D * D : nullptr;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[i] = s0 ? s0[(int64_t)(c0 + i) * D + e] : 0.f;
+            } else {
+                const float* sin = a.sin + ((int64_t)u * H + h) * D * D + (int64_t)e * D;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[i] = sin[c0 + i];
+            }
+            tmem_st16(tq + TM_S + c0, v);
+        }
+    }
+    tmem_st_wait();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    uint32_t parity = 0, img_parity = 0, gate_parity = 0;  // img_parity: bit b for image b
+    bool ok = true;
+    int b = 0;
+    for (int64_t t0 = sg.t_begin; t0 < sg.t_end && ok; t0 += C, b ^= 1) {
+        const int Lc = (int)((sg.t_end - t0) < C ? (sg.t_end - t0) : C);
+        uint8_t* img = sm + LayC::IMG + b * LayC::IMG_STRIDE;
+        if (!(ok = !__syncthreads_or(!mbar_wait(bar_img + b, (img_parity >> b) & 1u, &g_tc_status,
+                                                ERR_WAIT_TIMEOUT)))) break;
+        img_parity ^= 1u << b;
+        pending &= ~(1u << b);
+        // bf16 S^T into TMEM (A operand), S^T *= gamma in place; U'^T into the U accumulator
+        {
+            const float* gam = reinterpret_cast<const float*>(img + CI_GAM);
+            const int c0 = 32 * wg, r0 = 16 * wg;
+            stage_cols_tmem<2>(tq + TM_S + c0, tq + TM_SB + c0 / 2, c0, gam, true);
+            const uint8_t* ru = img + CI_U + lrow * 128;
+            float v[16];
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const uint4 x = *reinterpret_cast<const uint4*>(ru + ((((r0 >> 3) + hh) ^ (lrow & 7)) << 4));
+                float lo4[4], hi4[4];
+                unpack_bf16x4(make_uint2(x.x, x.y), lo4);
+                unpack_bf16x4(make_uint2(x.z, x.w), hi4);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    v[8 * hh + i] = lo4[i];
+                    v[8 * hh + 4 + i] = hi4[i];
+                }
+            }
+            tmem_st16(tq + TM_U + r0, v);
+            tmem_st_wait();
+        }
+        tc_fence_before();
+        __syncthreads();
+        // U^T -= S^T W^T ; O^T = S^T Q~^T
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t wb = smem_u32(img + CI_W), qt = smem_u32(img + CI_QT);
+            constexpr uint32_t id_neg = idesc_bf16(128, 64, false, true, true);
+            constexpr uint32_t id = idesc_bf16(128, 64, false, false);
+#pragma unroll
+            for (int s = 0; s < 8; ++s)
+                mma_bf16_ts(tmem + TM_U, tmem + TM_SB + 8 * s, mnmajor_desc(wb, 128, s), id_neg, 1);
+#pragma unroll
+            for (int s = 0; s < 8; ++s)
+                mma_bf16_ts(tmem + TM_O, tmem + TM_SB + 8 * s, kmajor_desc(qt, 64, s), id, s > 0);
+            mma_commit(bar);
+        }
+        if (!(ok = wait_mma(bar, parity))) break;
+        // bf16 U^T into TMEM; the last output store has left OUT by the next barrier
+        {
+            const int c0 = 16 * wg;
+            stage_cols_tmem<1>(tq + TM_U + c0, tq + TM_UB + c0 / 2, c0, nullptr, false);
+            tmem_st_wait();
+        }
+        if (tid == 0) bulk_wait_read();
+        tc_fence_before();
+        __syncthreads();
+        // O^T += U^T P^T ; S^T += U^T K_dec
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t pb = smem_u32(img + CI_PB), kd = smem_u32(img + CI_KD);
+            constexpr uint32_t id = idesc_bf16(128, 64, false, false);
+            constexpr uint32_t id_s = idesc_bf16(128, 128, false, true);
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                mma_bf16_ts(tmem + TM_O, tmem + TM_UB + 8 * s, kmajor_desc(pb, 64, s), id, 1);
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                mma_bf16_ts(tmem + TM_S, tmem + TM_UB + 8 * s, mnmajor_desc(kd, 64, s), id_s, 1);
+            mma_commit(bar);
+        }
+        if (!(ok = wait_mma(bar, parity))) break;
+        // this image is consumed: the chunk after next may load into it
+        if (tid == 0 && t0 + 2 * C < sg.t_end) load_img(t0 + 2 * C, b);
+
+        // O^T -> out: a full chunk as one [64][128] bf16 tile by TMA, a partial last chunk
+        // row by row from registers; with an output gate, each element gated first
+        {
+            const int r0 = 16 * wg;
+            float v[16];
+            tmem_ld16(tq + TM_O + r0, v);
+            tmem_wait16(v);
+            __nv_bfloat16* os = reinterpret_cast<__nv_bfloat16*>(sm + LayC::OUT);
+            if (gate_on) {
+                const __nv_bfloat16* gs = reinterpret_cast<const __nv_bfloat16*>(sm + LayC::GATE);
+                if (!(ok = !__syncthreads_or(!mbar_wait(bar_gate, gate_parity, &g_tc_status,
+                                                        ERR_WAIT_TIMEOUT)))) break;
+                gate_parity ^= 1u;
+                pending &= ~4u;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[i] *= __bfloat162float(gs[(r0 + i) * D + lrow]);
+            }
+            if (Lc == C) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) os[(r0 + i) * D + lrow] = __float2bfloat16_rn(v[i]);
+                fence_async_smem();
+                __syncthreads();
+                if (tid == 0) {
+                    tma_store_tile(&maps.out, sm + LayC::OUT, h, (int)t0);
+                    bulk_commit();
+                    if (gate_on && t0 + C < sg.t_end) load_gate(t0 + C);  // GATE has been read
+                }
+            } else {
+                __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out) + (int64_t)h * D + lrow;
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    if (r0 + i < Lc) out[(t0 + r0 + i) * H * (int64_t)D] = __float2bfloat16_rn(v[i]);
+            }
+        }
+        if (snap_on) {  // state snapshot at this chunk end, if one is requested
+            const int64_t pos = t0 + Lc - seq_lo;
+            if (pos % a.snap_interval == 0 && pos / a.snap_interval <= a.snap_max) {
+                const int slot = a.snap_slots[(int64_t)sg.n * a.snap_max + pos / a.snap_interval - 1];
+                if (slot >= a.snap_num_slots) {
+                    if (tid == 0) atomicCAS(&g_tc_status, 0, ERR_BAD_SLOT);
+                } else if (slot >= 0) {  // slice wg: columns 32wg..32wg+31 of S^T
+                    float* sp = a.snap_pool + ((int64_t)slot * H + h) * D * D;
+                    for (int c0 = 32 * wg; c0 < 32 * wg + 32; c0 += 16) {
+                        float v[16];
+                        tmem_ld16(tq + TM_S + c0, v);
+                        tmem_wait16(v);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) sp[(int64_t)(c0 + i) * D + lrow] = v[i];
+                    }
+                }
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    }
+
+    if (!ok && tid == 0) {  // after a timeout: bounded waits for what may still be in flight
+        mbar_wait(bar, parity ^ 1u, &g_tc_status, ERR_WAIT_TIMEOUT);
+        for (int bb = 0; bb < 2; ++bb)
+            if (pending & (1u << bb))
+                mbar_wait(bar_img + bb, (img_parity >> bb) & 1u, &g_tc_status, ERR_WAIT_TIMEOUT);
+        if (pending & 4u) mbar_wait(bar_gate, gate_parity, &g_tc_status, ERR_WAIT_TIMEOUT);
+    }
+    if (tid == 0) bulk_wait_all();  // output stores are complete
+    if (ok && sg.last && a.s_final) {  // slice wg: columns 32wg..32wg+31 of S^T
+        float* sf = a.s_final + ((int64_t)sg.n * H + h) * D * D;
+        for (int c0 = 32 * wg; c0 < 32 * wg + 32; c0 += 16) {
+            float v[16];
+            tmem_ld16(tq + TM_S + c0, v);
+            tmem_wait16(v);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) sf[(int64_t)(c0 + i) * D + lrow] = v[i];
         }
     }
     tc_fence_before();
@@ -1269,8 +1515,8 @@ cudaError_t launch_tc(const TcArgs& a, const TcPlan& p, cudaStream_t stream, int
         err = cudaFuncSetAttribute(tc_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    (int)LayT<false>::BYTES);
         if (err == cudaSuccess)
-            err = cudaFuncSetAttribute(tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)LayT<false>::BYTES);
+            err = cudaFuncSetAttribute(cached_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)LayC::BYTES);
         if (err == cudaSuccess)
             err = cudaFuncSetAttribute(seg_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        SCAN_SMEM);
@@ -1318,7 +1564,7 @@ cudaError_t launch_tc(const TcArgs& a, const TcPlan& p, cudaStream_t stream, int
     }
     profile_mark(SLOT_PASS3, true, stream);
     if (a.wu)
-        tc_kernel<2><<<grid, NT, LayT<false>::BYTES, stream>>>(a, maps);
+        cached_kernel<<<grid, NT, LayC::BYTES, stream>>>(a, maps);
     else
         tc_kernel<0><<<grid, NT, LayT<false>::BYTES, stream>>>(a, maps);
     profile_mark(SLOT_PASS3, false, stream);
@@ -1346,7 +1592,8 @@ cudaError_t launch_transition(const TcArgs& a_in, const TcPlan& p, float* out, c
     if (tokens > 0) {
         if ((err = tile_map(&maps.k, a.k, false, a.H, tokens, false)) != cudaSuccess ||
             (err = tile_map(&maps.v, a.v, false, a.H, tokens, true)) != cudaSuccess ||
-            (err = tile_map(&maps.la, a.log_alpha, true, a.H, tokens, false)) != cudaSuccess)
+            (err = tile_map(&maps.la, a.log_alpha, true, a.H, tokens, false)) != cudaSuccess ||
+            (a.wu && (err = tile_map(&maps.q, a.q, false, a.H, tokens, false)) != cudaSuccess))
             return err;
     }
     profile_mark(SLOT_SETUP, true, stream);

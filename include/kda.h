@@ -89,7 +89,9 @@ typedef struct {
  * final_state[n] = initial_state[n].
  *
  * Temporary device memory (segment table, segment transitions and incoming
- * states for long sequences) is taken stream-ordered (cudaMallocFromPoolAsync /
+ * states for long sequences, and for those also a cache of every chunk's
+ * operands of the output pass, which the transition pass prepares: about 290
+ * bytes per token and head) is taken stream-ordered (cudaMallocFromPoolAsync /
  * cudaFreeAsync on `stream`) from a memory pool the library creates once per
  * device and keeps for the life of the process; freed blocks stay reserved in
  * that pool for the next call.  Nothing else persists between calls apart from
@@ -323,7 +325,11 @@ kda_status kda_apply_transitions(const float* trans, int32_t count, int32_t B, i
  *   d_k = d_v = 128, bf16, no cu_seqlens); 0 for invalid dims.
  * kda_span_transition: kda_transition that also fills `workspace` (device,
  *   256-byte aligned, at least kda_span_workspace_bytes, not overlapping any
- *   argument).
+ *   argument).  It takes the span's q as well (same layout as k): besides the
+ *   segment transitions it leaves every chunk's operands of the output pass
+ *   (W, U', the decayed keys, the gated queries, the intra-chunk query-key
+ *   matrix and the chunk decay) in the workspace, about 290 bytes per token
+ *   and head.
  * kda_span_forward: kda_fwd on the same span (same k, v, log_alpha, beta and
  *   dims; q, initial_state, out, final_state as in kda_fwd) that takes the
  *   workspace's contents instead of recomputing them.  Where kda_fwd cuts the
@@ -340,9 +346,9 @@ kda_status kda_apply_transitions(const float* trans, int32_t count, int32_t B, i
  *   opts == NULL is kda_span_forward.
  */
 size_t kda_span_workspace_bytes(const kda_dims* dims);
-kda_status kda_span_transition(const void* k, const void* v, const float* log_alpha,
-                               const float* beta, const kda_dims* dims, void* workspace,
-                               size_t workspace_bytes, float* trans, void* stream);
+kda_status kda_span_transition(const void* q, const void* k, const void* v,
+                               const float* log_alpha, const float* beta, const kda_dims* dims,
+                               void* workspace, size_t workspace_bytes, float* trans, void* stream);
 kda_status kda_span_forward(const void* q, const void* k, const void* v, const float* log_alpha,
                             const float* beta, const float* initial_state, void* out,
                             float* final_state, const kda_dims* dims, const void* workspace,

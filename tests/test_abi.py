@@ -237,11 +237,15 @@ def test_span_workspace_size_and_bad_arguments():
     assert lib.kda_span_workspace_bytes(ctypes.byref(D(B=0))) == 0
     assert lib.kda_span_workspace_bytes(None) == 0
 
-    def trans_call(ws=FAKE + (8 << 30), nbytes=n, d=None):
-        rc = lib.kda_span_transition(P(FAKE), P(FAKE + (1 << 30)), P(FAKE + (2 << 30)),
+    def trans_call(ws=FAKE + (8 << 30), nbytes=n, d=None, q=FAKE + (9 << 30)):
+        rc = lib.kda_span_transition(P(q), P(FAKE), P(FAKE + (1 << 30)), P(FAKE + (2 << 30)),
                                      P(FAKE + (3 << 30)), ctypes.byref(d or D(T=1 << 16, H=8)),
                                      P(ws), nbytes, P(FAKE + (4 << 30)), None)
         return kda.STATUS[rc]
+
+    assert trans_call(q=None) == "KDA_ERR_INVALID_ARG"  # the workspace needs q
+    assert trans_call(q=FAKE + (9 << 30) + 8) == "KDA_ERR_MISALIGNED"
+    assert trans_call(ws=FAKE + (9 << 30)) == "KDA_ERR_ALIAS"  # workspace over q
 
     assert trans_call(ws=None) == "KDA_ERR_INVALID_ARG"
     assert trans_call(ws=FAKE + (8 << 30) + 16) == "KDA_ERR_MISALIGNED"

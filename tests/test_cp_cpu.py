@@ -39,7 +39,7 @@ def _oracle_ops():
 
     npy = lambda t: t.numpy()
 
-    def transition(k, v, la, be):
+    def transition(q, k, v, la, be):
         kw = dict(q=npy(k), k=npy(k), v=npy(v), log_alpha=npy(la), beta=npy(be), o_tokens=0)
         _, b = oracle.recurrent(initial_state=None, **kw)
         m = np.empty((B, H, DK, DK))

@@ -94,7 +94,7 @@ def test_context_parallel_prefill_emulated_on_one_gpu(world):
     spans = [{k_: d[k_][:, r * span:(r + 1) * span].contiguous() for k_ in keys}
              for r in range(world)]
     ws = [span_workspace(s["k"]) for s in spans]
-    trans = [kda_span_transition(s["k"], s["v"], s["log_alpha"], s["beta"], w)
+    trans = [kda_span_transition(s["q"], s["k"], s["v"], s["log_alpha"], s["beta"], w)
              for s, w in zip(spans, ws)]
     gathered = torch.stack(trans)  # what the all-gather delivers
     outs, finals = [], []
@@ -129,7 +129,7 @@ def test_span_transition_and_forward_share_the_work(monkeypatch, seg_chunks):
     d = to_device(inp)
     keys = ("q", "k", "v", "log_alpha", "beta")
     ws = span_workspace(d["k"])
-    trans = kda_span_transition(d["k"], d["v"], d["log_alpha"], d["beta"], ws)
+    trans = kda_span_transition(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], ws)
     trans_ref = kda_transition(d["k"], d["v"], d["log_alpha"], d["beta"])
     o, f = kda_span_forward(*(d[k_] for k_ in keys), ws, d["initial_state"])
     o2, f2 = kda_span_forward(*(d[k_] for k_ in keys), ws, d["initial_state"])  # reusable
@@ -212,7 +212,7 @@ def test_span_forward_with_gate_and_snapshots_equals_kda_fwd(monkeypatch):
     slots = torch.tensor([[0, -1, 1], [2, 3, 4]], dtype=torch.int32, device="cuda")
     pools = [torch.full((6, 2, 128, 128), 3.0, device="cuda") for _ in range(2)]
     ws = span_workspace(d["k"])
-    kda_span_transition(d["k"], d["v"], d["log_alpha"], d["beta"], ws)
+    kda_span_transition(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], ws)
     o, f = kda_span_forward(*(d[k_] for k_ in keys), ws, d["initial_state"], out_gate=gate,
                             snap_interval=128, snap_slots=slots, snap_pool=pools[0])
     o_ref, f_ref = kda_fwd_snap(**{k_: d[k_] for k_ in keys}, initial_state=d["initial_state"],
@@ -239,7 +239,7 @@ def test_cp_snapshots_at_span_aligned_positions(monkeypatch):
     keys = ("q", "k", "v", "log_alpha", "beta")
     spans = [{k_: d[k_][:, r * span:(r + 1) * span].contiguous() for k_ in keys} for r in range(2)]
     ws = [span_workspace(s["k"]) for s in spans]
-    trans = torch.stack([kda_span_transition(s["k"], s["v"], s["log_alpha"], s["beta"], w)
+    trans = torch.stack([kda_span_transition(s["q"], s["k"], s["v"], s["log_alpha"], s["beta"], w)
                          for s, w in zip(spans, ws)])
     pool = torch.zeros(4, 2, 128, 128, device="cuda")
     for r, s in enumerate(spans):
