@@ -306,18 +306,19 @@ def segment_plan(inp, sms=148):
 def kernel_algorithmic_bytes(name, inp, path_bytes):
     """Minimum bytes one launch of kernel `name` must move for what it computes.
 
-    pass 3 (forward) reads every input once and writes o and the states: the
-    whole path's algorithmic bytes.  Pass 1 (segment transitions) runs over
-    every segment when sequences are cut (it also leaves each chunk's W and U'
-    for pass 3): it reads k, v, log alpha and beta of every token and writes
-    one (B, M) pair (2 x 128 x 128 fp32) per segment and head.  The W/U' cache
-    (512 B per token-head each way) is implementation traffic, not counted."""
+    pass 3 (forward) delivers the path's results from its inputs: the whole
+    path's algorithmic bytes.  Pass 1 (segment transitions) runs over every
+    segment when sequences are cut, and also prepares every chunk's operands
+    of the output pass: it reads q, k, v, log alpha and beta of every token
+    and writes one (B, M) pair (2 x 128 x 128 fp32) per segment and head.  The
+    chunk cache (about 1160 B per token-head, written by pass 1 and read by
+    pass 3) is implementation traffic, not counted."""
     if name != "tc_pass1_transitions":
         return path_bytes
     seg, cut = segment_plan(inp)
     if not cut:
         return 0
-    per_tok = inp.H * (inp.dk * 2 + inp.dv * 2 + inp.dk * 4 + 4)
+    per_tok = inp.H * (2 * inp.dk * 2 + inp.dv * 2 + inp.dk * 4 + 4)
     segs = 0
     for L in inp.seq_lens:
         nch = (int(L) + 63) // 64
