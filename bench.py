@@ -327,15 +327,15 @@ def kernel_algorithmic_bytes(name, inp, path_bytes):
 
 
 # ------------------------------------------------------------------ traffic record
-def recorded_traffic(kernel_tag: str):
-    """DRAM bytes per launch from a committed ncu summary, if its kernel sources
-    are unchanged since the capture (else None)."""
+def recorded_traffic(kernel_tag: str, workload_name: str):
+    """DRAM bytes per launch from a committed ncu summary, if it is for this
+    workload and its kernel sources are unchanged since the capture (else None)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         rec = json.load(f).get(kernel_tag)
-    if not rec:
+    if not rec or rec.get("workload") != workload_name:
         return None
     h = hashlib.sha256()
     for src in rec["sources"]:
@@ -627,7 +627,7 @@ def main():
         "config": cfg,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                     "traffic": recorded_traffic(dom),
+                     "traffic": recorded_traffic(dom, inp.name),
                      "kernel": dom,
                      "algorithmic_bytes_per_launch": dom_bytes,
                      "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)"

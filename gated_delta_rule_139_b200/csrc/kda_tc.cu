@@ -119,6 +119,7 @@ static_assert(LayT<false>::BYTES <= 232448 && LayT<true>::BYTES <= 232448, "shar
 // O [224,288) bf16 S^T [288,352) bf16 U^T [352,384) S [384,512).  Pass 1: AP/U_M [0,96) W U as
 // above (W's columns later hold bf16 U_B^T [96,128) and U_M^T [128,160)), B [256,384), M [384,512).
 constexpr uint32_t TM_AP = 0, TM_W = 96, TM_U = 160, TM_O = 224;
+constexpr uint32_t TM_O2 = 0;  // cached_kernel: the second O accumulator (TM_AP's columns, unused there)
 constexpr uint32_t TM_SB = 288, TM_UB = 352;  // pass 3: bf16 copies of S^T and U^T (A operands)
 constexpr uint32_t TM_B = 256, TM_S = 384, TM_M = 384;
 constexpr uint32_t TM_UBB = 96, TM_UBM = 128;  // pass 1: bf16 U_B^T, U_M^T (A operands) in the W columns
@@ -580,7 +581,12 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
     // while the current chunk is processed (issued once every thread has read
     // the current tiles into registers); beta goes through registers.
     const bool with_q = !SEG || wu_cache;  // pass 1 needs q only to fill the chunk cache
-    bool raw_pending = false, gate_pending = false;  // thread 0: TMA loads in flight
+    // The raw tiles' tensor copies take long to issue: pass 1 issues them from warp 8,
+    // which has no part in the per-channel prefix that follows; pass 3 from thread 0, which
+    // must first see its output store leave the v buffer.  raw_pending (on that thread) /
+    // gate_pending (thread 0): copies in flight.
+    const int raw_tid = SEG ? 256 : 0;
+    bool raw_pending = false, gate_pending = false;
     auto issue_raw = [&](int64_t tn, int vbuf) {
         raw_pending = true;
         mbar_expect_tx(bar_raw, with_q ? 81920u : 65536u);  // k, log alpha, v (, q)
@@ -594,7 +600,7 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
     uint32_t raw_parity = 0;
     float beta_ld = 0.f;
     if (sg.t_begin < sg.t_end) {
-        if (tid == 0) issue_raw(sg.t_begin, 0);
+        if (tid == raw_tid) issue_raw(sg.t_begin, 0);
         if (tid < C && sg.t_begin + tid < sg.t_end) beta_ld = __ldg(a.beta + (sg.t_begin + tid) * H + h);
     }
 
@@ -644,7 +650,7 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
             __syncthreads();
             // every thread holds its raw inputs: RAW may now receive the next chunk
             if (t0 + C < sg.t_end) {
-                if (tid == 0) {
+                if (tid == raw_tid) {
                     if (!SEG) bulk_wait_read();  // the v buffer may still be feeding an output store
                     issue_raw(t0 + C, vbuf ^ 1);
                 }
@@ -1006,10 +1012,12 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
     }
 
     // ---- results of the segment
-    if (!ok && tid == 0) {  // after a timeout: bounded waits for what may still be in flight
-        mbar_wait(bar, parity ^ 1u, &g_tc_status, ERR_WAIT_TIMEOUT);
-        if (raw_pending) mbar_wait(bar_raw, raw_parity, &g_tc_status, ERR_WAIT_TIMEOUT);
-        if (gate_pending) mbar_wait(bar_gate, gate_parity, &g_tc_status, ERR_WAIT_TIMEOUT);
+    if (!ok) {  // after a timeout: bounded waits for what may still be in flight
+        if (tid == 0) {
+            mbar_wait(bar, parity ^ 1u, &g_tc_status, ERR_WAIT_TIMEOUT);
+            if (gate_pending) mbar_wait(bar_gate, gate_parity, &g_tc_status, ERR_WAIT_TIMEOUT);
+        }
+        if (tid == raw_tid && raw_pending) mbar_wait(bar_raw, raw_parity, &g_tc_status, ERR_WAIT_TIMEOUT);
     }
     if (tid == 0 && (!SEG || wu_cache)) bulk_wait_all();  // output / cache stores are complete
     if (ok) {
@@ -1143,11 +1151,56 @@ __global__ void __launch_bounds__(NT, 1) cached_kernel(TcArgs a, const __grid_co
     tc_fence_after();
 
     uint32_t parity = 0, img_parity = 0, gate_parity = 0;  // img_parity: bit b for image b
+    bool mma_out = false;  // thread 0: a commit not yet waited for, on phase mma_par
+    uint32_t mma_par = 0;
+    // O^T of the chunk at tt (Lcc tokens) from the O accumulator at tm_o -> out: a full chunk
+    // as one [64][128] bf16 tile by TMA, a partial last chunk row by row from registers; with
+    // an output gate, each element gated first (then the next chunk's gate tile is loaded).
+    // Called by all threads; false if a wait gave up.
+    auto emit = [&](int64_t tt, int Lcc, uint32_t tm_o) -> bool {
+        const int r0 = 16 * wg;
+        float v[16];
+        tmem_ld16(tq + tm_o + r0, v);
+        tmem_wait16(v);
+        __nv_bfloat16* os = reinterpret_cast<__nv_bfloat16*>(sm + LayC::OUT);
+        if (gate_on) {
+            const __nv_bfloat16* gs = reinterpret_cast<const __nv_bfloat16*>(sm + LayC::GATE);
+            if (__syncthreads_or(!mbar_wait(bar_gate, gate_parity, &g_tc_status, ERR_WAIT_TIMEOUT)))
+                return false;
+            gate_parity ^= 1u;
+            pending &= ~4u;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] *= __bfloat162float(gs[(r0 + i) * D + lrow]);
+        }
+        if (Lcc == C) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) os[(r0 + i) * D + lrow] = __float2bfloat16_rn(v[i]);
+            fence_async_smem();
+            __syncthreads();
+            if (tid == 0) {
+                tma_store_tile(&maps.out, sm + LayC::OUT, h, (int)tt);
+                bulk_commit();
+                if (gate_on && tt + C < sg.t_end) load_gate(tt + C);  // GATE has been read
+            }
+        } else {
+            __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out) + (int64_t)h * D + lrow;
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                if (r0 + i < Lcc) out[(tt + r0 + i) * H * (int64_t)D] = __float2bfloat16_rn(v[i]);
+        }
+        return true;
+    };
     bool ok = true;
     int b = 0;
+    int64_t last_t0 = sg.t_begin;  // the chunk whose output is still in TMEM
+    int last_Lc = 0;
+    uint32_t last_o = TM_O;
     for (int64_t t0 = sg.t_begin; t0 < sg.t_end && ok; t0 += C, b ^= 1) {
         const int Lc = (int)((sg.t_end - t0) < C ? (sg.t_end - t0) : C);
         uint8_t* img = sm + LayC::IMG + b * LayC::IMG_STRIDE;
+        // O accumulators alternate between chunks, so a chunk's output leaves TMEM while
+        // the next chunk's first products run
+        const uint32_t tm_o = (((t0 - sg.t_begin) / C) & 1) ? TM_O2 : TM_O;
         if (!(ok = !__syncthreads_or(!mbar_wait(bar_img + b, (img_parity >> b) & 1u, &g_tc_status,
                                                 ERR_WAIT_TIMEOUT)))) break;
         img_parity ^= 1u << b;
@@ -1187,10 +1240,15 @@ __global__ void __launch_bounds__(NT, 1) cached_kernel(TcArgs a, const __grid_co
                 mma_bf16_ts(tmem + TM_U, tmem + TM_SB + 8 * s, mnmajor_desc(wb, 128, s), id_neg, 1);
 #pragma unroll
             for (int s = 0; s < 8; ++s)
-                mma_bf16_ts(tmem + TM_O, tmem + TM_SB + 8 * s, kmajor_desc(qt, 64, s), id, s > 0);
+                mma_bf16_ts(tmem + tm_o, tmem + TM_SB + 8 * s, kmajor_desc(qt, 64, s), id, s > 0);
             mma_commit(bar);
+            mma_out = true;
+            mma_par = parity;
         }
+        // meanwhile: the previous chunk's output (a full chunk: only a segment's last is partial)
+        if (t0 > sg.t_begin && !(ok = emit(t0 - C, C, last_o))) break;
         if (!(ok = wait_mma(bar, parity))) break;
+        mma_out = false;
         // bf16 U^T into TMEM; the last output store has left OUT by the next barrier
         {
             const int c0 = 16 * wg;
@@ -1208,50 +1266,21 @@ __global__ void __launch_bounds__(NT, 1) cached_kernel(TcArgs a, const __grid_co
             constexpr uint32_t id_s = idesc_bf16(128, 128, false, true);
 #pragma unroll
             for (int s = 0; s < 4; ++s)
-                mma_bf16_ts(tmem + TM_O, tmem + TM_UB + 8 * s, kmajor_desc(pb, 64, s), id, 1);
+                mma_bf16_ts(tmem + tm_o, tmem + TM_UB + 8 * s, kmajor_desc(pb, 64, s), id, 1);
 #pragma unroll
             for (int s = 0; s < 4; ++s)
                 mma_bf16_ts(tmem + TM_S, tmem + TM_UB + 8 * s, mnmajor_desc(kd, 64, s), id_s, 1);
             mma_commit(bar);
+            mma_out = true;
+            mma_par = parity;
         }
         if (!(ok = wait_mma(bar, parity))) break;
+        mma_out = false;
         // this image is consumed: the chunk after next may load into it
         if (tid == 0 && t0 + 2 * C < sg.t_end) load_img(t0 + 2 * C, b);
-
-        // O^T -> out: a full chunk as one [64][128] bf16 tile by TMA, a partial last chunk
-        // row by row from registers; with an output gate, each element gated first
-        {
-            const int r0 = 16 * wg;
-            float v[16];
-            tmem_ld16(tq + TM_O + r0, v);
-            tmem_wait16(v);
-            __nv_bfloat16* os = reinterpret_cast<__nv_bfloat16*>(sm + LayC::OUT);
-            if (gate_on) {
-                const __nv_bfloat16* gs = reinterpret_cast<const __nv_bfloat16*>(sm + LayC::GATE);
-                if (!(ok = !__syncthreads_or(!mbar_wait(bar_gate, gate_parity, &g_tc_status,
-                                                        ERR_WAIT_TIMEOUT)))) break;
-                gate_parity ^= 1u;
-                pending &= ~4u;
-#pragma unroll
-                for (int i = 0; i < 16; ++i) v[i] *= __bfloat162float(gs[(r0 + i) * D + lrow]);
-            }
-            if (Lc == C) {
-#pragma unroll
-                for (int i = 0; i < 16; ++i) os[(r0 + i) * D + lrow] = __float2bfloat16_rn(v[i]);
-                fence_async_smem();
-                __syncthreads();
-                if (tid == 0) {
-                    tma_store_tile(&maps.out, sm + LayC::OUT, h, (int)t0);
-                    bulk_commit();
-                    if (gate_on && t0 + C < sg.t_end) load_gate(t0 + C);  // GATE has been read
-                }
-            } else {
-                __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out) + (int64_t)h * D + lrow;
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    if (r0 + i < Lc) out[(t0 + r0 + i) * H * (int64_t)D] = __float2bfloat16_rn(v[i]);
-            }
-        }
+        last_t0 = t0;
+        last_Lc = Lc;
+        last_o = tm_o;
         if (snap_on) {  // state snapshot at this chunk end, if one is requested
             const int64_t pos = t0 + Lc - seq_lo;
             if (pos % a.snap_interval == 0 && pos / a.snap_interval <= a.snap_max) {
@@ -1275,8 +1304,9 @@ __global__ void __launch_bounds__(NT, 1) cached_kernel(TcArgs a, const __grid_co
         tc_fence_after();
     }
 
+    if (ok && last_Lc > 0) ok = emit(last_t0, last_Lc, last_o);  // the last chunk's output
     if (!ok && tid == 0) {  // after a timeout: bounded waits for what may still be in flight
-        mbar_wait(bar, parity ^ 1u, &g_tc_status, ERR_WAIT_TIMEOUT);
+        if (mma_out) mbar_wait(bar, mma_par, &g_tc_status, ERR_WAIT_TIMEOUT);
         for (int bb = 0; bb < 2; ++bb)
             if (pending & (1u << bb))
                 mbar_wait(bar_img + bb, (img_parity >> bb) & 1u, &g_tc_status, ERR_WAIT_TIMEOUT);
