@@ -212,7 +212,7 @@ kda_status run_tc(const kda::FwdArgs& a, cudaStream_t stream, int* launches) {
     const size_t b_off = ((size_t)(a.N + 1) * 4 + 4 + 255) & ~(size_t)255;
     const size_t b_trans = p.segmented ? (size_t)p.max_units * a.H * 2 * st : 0;
     const size_t b_sin = p.segmented ? (size_t)p.max_units * a.H * st : 0;
-    // W/U' cache of the segmented plan: 32 KB per chunk of every unit
+    // chunk cache of the segmented plan: kChunkImageBytes per chunk of every unit
     const size_t b_wu = p.segmented ? (size_t)p.max_units * a.H * p.seg_chunks * kda::kChunkImageBytes : 0;
     char* ws = nullptr;
     cudaError_t e = pool_alloc((void**)&ws, b_segs + b_off + b_trans + b_sin + b_wu, stream);
@@ -338,7 +338,7 @@ size_t tc_scratch_bytes(const kda::FwdArgs& a, const kda::TcPlan& p, size_t* b_s
 }
 
 // Workspace of a span (segment table, per-segment transitions and incoming
-// states, W/U' cache) for the segment plan of the dims: offsets into one buffer.
+// states, chunk cache) for the segment plan of the dims: offsets into one buffer.
 struct SpanWs {
     kda::TcPlan p;
     size_t segs, off, trans, sin, wu, total;

@@ -102,7 +102,7 @@ struct TcPlan {
 };
 
 // bf16 q/k/v with d_k = d_v = 128: tcgen05 tensor-core path.  from_cache: the
-// segment table, the transitions and the W/U' cache of this plan are already in
+// segment table, the transitions and the chunk cache of this plan are already in
 // a's workspace (left by launch_transition), so only the scan and pass 3 run.
 cudaError_t launch_tc(const TcArgs& a, const TcPlan& p, cudaStream_t stream, int* launches,
                       bool from_cache = false);
