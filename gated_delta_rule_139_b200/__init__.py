@@ -268,8 +268,10 @@ def kda_fwd_host(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None,
                  want_final: bool = True):
     """KDA forward on HOST numpy arrays (or CPU tensors; pinned memory copies
     asynchronously).  The library copies inputs in, runs, copies results back
-    and synchronises.  bf16 data is passed as uint16 bit patterns (numpy) or
-    torch.bfloat16 CPU tensors.  Returns (out, final_state or None) on the host.
+    and synchronises; one long sequence (B = 1, no cu_seqlens) runs as a
+    pipeline of spans so that the two copy directions overlap (kda_fwd_host).
+    bf16 data is passed as uint16 bit patterns (numpy) or torch.bfloat16 CPU
+    tensors.  Returns (out, final_state or None) on the host.
     """
     import numpy as np
 

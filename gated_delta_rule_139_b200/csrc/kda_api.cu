@@ -594,6 +594,19 @@ kda_status kda_fwd_snap(const void* q, const void* k, const void* v, const float
                       dims, &o, stream);
 }
 
+// Tokens per span of kda_fwd_host's pipelined path, or 0 for the one-call path: one
+// sequence (B = 1, no cu_seqlens) longer than one span is cut into spans of whole chunks.
+int64_t host_span_tokens(const kda::FwdArgs& a) {
+    if (a.cu || a.B != 1) return 0;
+    int64_t span = 131072;
+    if (const char* env = getenv("KDA_HOST_SPAN_TOKENS")) {  // test hook
+        const long v = atol(env);
+        if (v > 0) span = v;
+    }
+    span = (span + kda::kChunk - 1) / kda::kChunk * kda::kChunk;
+    return a.T > span ? span : 0;
+}
+
 kda_status kda_fwd_host(const void* q, const void* k, const void* v, const float* log_alpha,
                         const float* beta, const float* initial_state,
                         const int32_t* cu_seqlens, int32_t chunk, void* out,
@@ -611,11 +624,13 @@ kda_status kda_fwd_host(const void* q, const void* k, const void* v, const float
     const size_t bqk = (size_t)(tokens * a.H * a.dk * e_in), bv = (size_t)(tokens * a.H * a.dv * e_in);
     const size_t bla = (size_t)(tokens * a.H * a.dk * 4), bbe = (size_t)(tokens * a.H * 4);
     const size_t bst = (size_t)a.N * a.H * a.dk * a.dv * 4, bcu = cu_seqlens ? (size_t)(a.N + 1) * 4 : 0;
-    // one pool allocation carved into 16-byte aligned pieces
+    const int64_t span = host_span_tokens(a);
+    // one pool allocation carved into 256-byte aligned pieces (the last: the state passed
+    // between spans)
     const size_t sizes[] = {bqk, bqk, bv, bla, bbe, initial_state ? bst : 0, bcu, bv,
-                            final_state ? bst : 0};
-    size_t off[9], total = 0;
-    for (int i = 0; i < 9; ++i) {
+                            final_state ? bst : 0, span ? bst : 0};
+    size_t off[10], total = 0;
+    for (int i = 0; i < 10; ++i) {
         off[i] = total;
         total += (sizes[i] + 255) & ~(size_t)255;
     }
@@ -624,14 +639,6 @@ kda_status kda_fwd_host(const void* q, const void* k, const void* v, const float
     if (total) {
         e = pool_alloc((void**)&base, total, stream);
         if (e != cudaSuccess) return cuda_fail(e, "device buffer allocation");
-    }
-    const void* src[] = {q, k, v, log_alpha, beta, initial_state, cu_seqlens};
-    for (int i = 0; i < 7 && e == cudaSuccess; ++i)
-        if (sizes[i] && src[i])
-            e = cudaMemcpyAsync(base + off[i], src[i], sizes[i], cudaMemcpyHostToDevice, stream);
-    if (e != cudaSuccess) {
-        cudaFreeAsync(base, stream);
-        return cuda_fail(e, "host-to-device copy");
     }
     kda::FwdArgs d = a;
     d.q = base + off[0];
@@ -643,16 +650,102 @@ kda_status kda_fwd_host(const void* q, const void* k, const void* v, const float
     d.cu = cu_seqlens ? (const int32_t*)(base + off[6]) : nullptr;
     d.out = base + off[7];
     d.s_final = final_state ? (float*)(base + off[8]) : nullptr;
-    s = run(d, stream);
-    if (s == KDA_OK) {
-        if (sizes[7]) e = cudaMemcpyAsync(out, d.out, sizes[7], cudaMemcpyDeviceToHost, stream);
-        if (e == cudaSuccess && final_state)
-            e = cudaMemcpyAsync(final_state, d.s_final, sizes[8], cudaMemcpyDeviceToHost, stream);
+    const void* src[] = {q, k, v, log_alpha, beta, initial_state, cu_seqlens};
+    if (!span) {  // copy in, one forward call, copy out, all on the caller's stream
+        for (int i = 0; i < 7 && e == cudaSuccess; ++i)
+            if (sizes[i] && src[i])
+                e = cudaMemcpyAsync(base + off[i], src[i], sizes[i], cudaMemcpyHostToDevice, stream);
+        if (e != cudaSuccess) {
+            cudaFreeAsync(base, stream);
+            return cuda_fail(e, "host-to-device copy");
+        }
+        s = run(d, stream);
+        if (s == KDA_OK) {
+            if (sizes[7]) e = cudaMemcpyAsync(out, d.out, sizes[7], cudaMemcpyDeviceToHost, stream);
+            if (e == cudaSuccess && final_state)
+                e = cudaMemcpyAsync(final_state, d.s_final, sizes[8], cudaMemcpyDeviceToHost, stream);
+        }
+    } else {
+        // The sequence in spans: span r's inputs come in on `cin` while earlier spans are
+        // computed on `cmp` (one forward call per span, each starting from the state the
+        // previous one ended with, held in one buffer that every call reads before it
+        // writes it) and earlier outputs go back on `cout`, so the two copy directions
+        // overlap.  The caller's stream waits for all three at the end.
+        const int64_t n_spans = (a.T + span - 1) / span;
+        const int64_t row_in = a.H * a.dk * e_in, row_v = a.H * a.dv * e_in;
+        const int64_t row_la = a.H * a.dk * 4, row_be = a.H * 4;
+        float* st = (float*)(base + off[9]);
+        cudaStream_t cin = nullptr, cmp = nullptr, cout_ = nullptr;
+        cudaEvent_t ev_start = nullptr, ev_end = nullptr;
+        e = cudaStreamCreateWithFlags(&cin, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&cmp, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&cout_, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_start, cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_end, cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventRecord(ev_start, stream);  // after the allocation
+        for (cudaStream_t x : {cin, cmp, cout_})
+            if (e == cudaSuccess) e = cudaStreamWaitEvent(x, ev_start, 0);
+        if (e == cudaSuccess && initial_state)
+            e = cudaMemcpyAsync(base + off[5], initial_state, bst, cudaMemcpyHostToDevice, cin);
+        int launches = 0;
+        for (int64_t r = 0; r < n_spans && e == cudaSuccess && s == KDA_OK; ++r) {
+            const int64_t t0 = r * span, L = std::min<int64_t>(span, a.T - t0);
+            const size_t pieces[5][2] = {{off[0] + t0 * row_in, (size_t)(L * row_in)},
+                                         {off[1] + t0 * row_in, (size_t)(L * row_in)},
+                                         {off[2] + t0 * row_v, (size_t)(L * row_v)},
+                                         {off[3] + t0 * row_la, (size_t)(L * row_la)},
+                                         {off[4] + t0 * row_be, (size_t)(L * row_be)}};
+            const int64_t src_off[5] = {t0 * row_in, t0 * row_in, t0 * row_v, t0 * row_la, t0 * row_be};
+            for (int i = 0; i < 5 && e == cudaSuccess; ++i)
+                e = cudaMemcpyAsync(base + pieces[i][0], (const char*)src[i] + src_off[i], pieces[i][1],
+                                    cudaMemcpyHostToDevice, cin);
+            cudaEvent_t ev_in = nullptr, ev_done = nullptr;
+            if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_in, cudaEventDisableTiming);
+            if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_done, cudaEventDisableTiming);
+            if (e == cudaSuccess) e = cudaEventRecord(ev_in, cin);
+            if (e == cudaSuccess) e = cudaStreamWaitEvent(cmp, ev_in, 0);
+            if (e == cudaSuccess) {
+                kda::FwdArgs dr = d;
+                dr.T = (int32_t)L;
+                dr.q = base + pieces[0][0];
+                dr.k = base + pieces[1][0];
+                dr.v = base + pieces[2][0];
+                dr.log_alpha = (const float*)(base + pieces[3][0]);
+                dr.beta = (const float*)(base + pieces[4][0]);
+                dr.out = base + off[7] + t0 * row_v;
+                dr.s0 = r == 0 ? d.s0 : st;
+                dr.s_final = (r == n_spans - 1 && d.s_final) ? d.s_final : st;
+                s = run(dr, cmp);
+                launches += g_last_launches;
+            }
+            if (e == cudaSuccess && s == KDA_OK) e = cudaEventRecord(ev_done, cmp);
+            if (e == cudaSuccess && s == KDA_OK) e = cudaStreamWaitEvent(cout_, ev_done, 0);
+            if (e == cudaSuccess && s == KDA_OK)
+                e = cudaMemcpyAsync((char*)out + t0 * row_v, base + off[7] + t0 * row_v, (size_t)(L * row_v),
+                                    cudaMemcpyDeviceToHost, cout_);
+            if (ev_in) cudaEventDestroy(ev_in);  // released once the work recorded on it is done
+            if (ev_done) cudaEventDestroy(ev_done);
+        }
+        if (e == cudaSuccess && s == KDA_OK && final_state)
+            e = cudaMemcpyAsync(final_state, d.s_final, bst, cudaMemcpyDeviceToHost, cout_);
+        // join: the caller's stream waits for every stream that ran (copies in flight on a
+        // failed path are drained by the synchronisations below)
+        for (cudaStream_t x : {cin, cmp, cout_}) {
+            if (!x) continue;
+            if (ev_end && cudaEventRecord(ev_end, x) == cudaSuccess) cudaStreamWaitEvent(stream, ev_end, 0);
+            cudaStreamSynchronize(x);
+        }
+        for (cudaStream_t x : {cin, cmp, cout_})
+            if (x) cudaStreamDestroy(x);
+        if (ev_start) cudaEventDestroy(ev_start);
+        if (ev_end) cudaEventDestroy(ev_end);
+        g_last_path = a.bf16 && a.dk == 128 && a.dv == 128 ? "tc" : "ffma";
+        g_last_launches = launches;
     }
     if (base) cudaFreeAsync(base, stream);
     cudaError_t e2 = cudaStreamSynchronize(stream);
     if (s != KDA_OK) return s;
-    if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
+    if (e != cudaSuccess) return cuda_fail(e, "copy or stream operation");
     if (e2 != cudaSuccess) return cuda_fail(e2, "stream synchronize");
     return KDA_OK;
 }

@@ -183,6 +183,16 @@ kda_status kda_fwd_ex(const void* q, const void* k, const void* v, const float* 
  * cudaMemcpyAsync per tensor; pinned host memory makes them asynchronous),
  * runs kda_fwd on `stream`, copies out/final_state back and synchronises the
  * stream before returning.  Device buffers come from the stream-ordered pool.
+ *
+ * One sequence longer than 131 072 tokens (B = 1, cu_seqlens NULL) is run as
+ * a pipeline of spans of that many tokens: the state after span r is exact
+ * (fp32) and depends on spans 0..r only, so span r's outputs are copied back
+ * while later spans are still being copied in.  The call creates three
+ * streams for this (copy in, compute, copy out), which wait for `stream`
+ * first and which `stream` waits for at the end.  Results are those of
+ * kda_fwd called span by span with the state carried between the calls; they
+ * agree with one kda_fwd over the whole sequence within rounding (the spans
+ * change where the tensor-core path cuts the sequence into segments).
  */
 kda_status kda_fwd_host(const void* q, const void* k, const void* v, const float* log_alpha,
                         const float* beta, const float* initial_state,

@@ -231,3 +231,38 @@ def test_host_pointer_is_rejected():
     rc = kda.load_library().kda_fwd(P(inp.q), P(inp.k), P(inp.v), P(inp.log_alpha), P(inp.beta),
                                     None, None, 64, P(out), None, ctypes.byref(d), None)
     assert kda.STATUS[rc] == "KDA_ERR_INVALID_ARG"
+
+
+@pytest.mark.parametrize("bf16,d", [(True, 128), (False, 64)])
+def test_host_entry_point_pipelines_long_sequences_in_spans(monkeypatch, bf16, d):
+    """One long sequence through kda_fwd_host runs as spans (here 512 tokens): the
+    result is bit for bit kda_fwd called span after span with the state carried,
+    and matches the oracle over the whole sequence."""
+    import torch
+    from gated_delta_rule_139_b200 import kda_fwd, kda_fwd_host, last_launch_count
+    monkeypatch.setenv("KDA_HOST_SPAN_TOKENS", "512")
+    T = 64 * 37 + 21  # four full spans and a ragged fifth
+    inp = make_inputs(1, T, 2, d, d, bf16=bf16, seed=31, state_sigma=0.05, gate_sigma=2.0)
+    o_h, s_h = kda_fwd_host(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.initial_state)
+    assert last_launch_count() >= 5
+    dd = to_device(inp)
+    state = dd["initial_state"]
+    outs = []
+    for t0 in range(0, T, 512):
+        sl = {k_: dd[k_][:, t0:t0 + 512].contiguous() for k_ in ("q", "k", "v", "log_alpha", "beta")}
+        o, state = kda_fwd(**sl, initial_state=state)
+        outs.append(o)
+    torch.cuda.synchronize()
+    o_d = torch.cat(outs, 1)
+    o_d = o_d.view(torch.int16).cpu().numpy().view(np.uint16) if bf16 else o_d.cpu().numpy()
+    np.testing.assert_array_equal(o_h, o_d)
+    np.testing.assert_array_equal(s_h, state.cpu().numpy())
+    o_r, s_r = oracle.recurrent(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.initial_state)
+    og = out_to_f64(torch.from_numpy(o_h.view(np.int16)).view(torch.bfloat16) if bf16
+                    else torch.from_numpy(o_h))
+    if bf16:
+        eo, es = rel_fro_per_head(og, o_r, s_h.astype(np.float64), s_r, inp)
+        assert eo <= TOL_BF16_REL_FRO and es <= TOL_BF16_REL_FRO, (eo, es)
+    else:
+        assert np.abs(og.reshape(o_r.shape) - o_r).max() <= TOL_F32_MAX_ABS
+        assert np.abs(s_h - s_r).max() <= TOL_F32_MAX_ABS
