@@ -1399,18 +1399,20 @@ __global__ void __launch_bounds__(1024) seg_setup_kernel(const int32_t* cu, int 
 }
 
 // ---------------------------------------------------------------- segment scan
-// S_in^T(j+1) = S_in^T(j) M_j^T + B_j^T for the 16 rows e in [16*blockIdx.z, +16)
-// of S^T, sequentially over the segments of sequence n, head h.  M_j^T (64 KB)
-// is staged in shared memory; the next one is loaded into registers while the
-// current product runs.
-constexpr int SCAN_SMEM = 2 * D * D * 4 + 16 * D * 4;
-
+// S_in^T(j+1) = S_in^T(j) M_j^T + B_j^T for the 8 rows e in [8*blockIdx.z, +8) of S^T,
+// sequentially over the segments of sequence n, head h (rows of S^T are independent, so
+// the CTAs of one head need nothing from each other).  M_j^T (64 KB) sits in shared
+// memory; the next one, and the next B_j^T rows, are loaded into registers while the
+// current product runs.  Thread (el, cg) owns row el and columns 4cg..4cg+3; each output
+// is B + sum over c of S[c] M[c][col] in order of c.
+constexpr int SCAN_ROWS = 8;
+constexpr int SCAN_SMEM = D * D * 4 + SCAN_ROWS * D * 4;
 __global__ void __launch_bounds__(256) seg_scan_kernel(TcArgs a) {
     extern __shared__ float4 scan_smem4[];
-    float* Ms = reinterpret_cast<float*>(scan_smem4);  // [2][128][128]
-    float* S = Ms + 2 * D * D;                        // [16][128]
-    const int n = blockIdx.x, h = blockIdx.y, e0 = 16 * blockIdx.z, H = a.H;
-    const int tid = threadIdx.x, el = tid >> 4, cg = tid & 15;
+    float* Ms = reinterpret_cast<float*>(scan_smem4);  // [128][128]
+    float* S = Ms + D * D;                            // [SCAN_ROWS][128]
+    const int n = blockIdx.x, h = blockIdx.y, e0 = SCAN_ROWS * blockIdx.z, H = a.H;
+    const int tid = threadIdx.x, el = tid >> 5, cg = tid & 31;
     const int32_t u0 = a.seg_off[n], u1 = a.seg_off[n + 1];
     const int32_t nu = *a.n_units;
     if (u1 - u0 <= 1 || u0 >= nu) return;
@@ -1418,50 +1420,46 @@ __global__ void __launch_bounds__(256) seg_scan_kernel(TcArgs a) {
     // S_in of segment 0, also copied to the workspace so that pass 3 never reads
     // initial_state while another segment may be writing final_state (they may
     // be the same buffer)
-    for (int x = tid; x < 16 * D; x += 256) {
+    for (int x = tid; x < SCAN_ROWS * D; x += 256) {
         const int r = x / D, c = x % D;
         const float v = a.s0 ? a.s0[(((int64_t)n * H + h) * D + c) * D + e0 + r] : 0.f;
         S[r * D + c] = v;
         a.sin[((int64_t)u0 * H + h) * D * D + (int64_t)(e0 + r) * D + c] = v;
     }
-    float4 pre[16];
-    auto load_m = [&](int32_t uu) {
-        const float4* Mt = reinterpret_cast<const float4*>(a.trans + ((int64_t)uu * H + h) * 2 * D * D + D * D);
+    float4 pre[16], bpre;
+    auto load_next = [&](int32_t uu) {  // M_uu^T and this thread's four entries of B_uu^T
+        const float4* T = reinterpret_cast<const float4*>(a.trans + ((int64_t)uu * H + h) * 2 * D * D);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) pre[i] = __ldg(Mt + tid + 256 * i);
+        for (int i = 0; i < 16; ++i) pre[i] = __ldg(T + D * D / 4 + tid + 256 * i);
+        bpre = __ldg(T + ((e0 + el) * D + 4 * cg) / 4);
     };
-    auto store_m = [&](int buf) {
-        float4* dst = reinterpret_cast<float4*>(Ms + buf * D * D);
+    auto store_m = [&]() {
+        float4* dst = reinterpret_cast<float4*>(Ms);
 #pragma unroll
         for (int i = 0; i < 16; ++i) dst[tid + 256 * i] = pre[i];
     };
     if (u0 < last) {
-        load_m(u0);
-        store_m(0);
+        load_next(u0);
+        store_m();
     }
     __syncthreads();
     for (int32_t uu = u0; uu < last; ++uu) {
-        const int buf = (uu - u0) & 1;
-        if (uu + 1 < last) load_m(uu + 1);
-        const float* Bt = a.trans + ((int64_t)uu * H + h) * 2 * D * D;
-        float acc[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = __ldg(Bt + (int64_t)(e0 + el) * D + cg + 16 * i);
-        const float* M = Ms + buf * D * D;
-#pragma unroll 4
+        float acc[4] = {bpre.x, bpre.y, bpre.z, bpre.w};
+        if (uu + 1 < last) load_next(uu + 1);
+#pragma unroll 8
         for (int c = 0; c < D; ++c) {
             const float sv = S[el * D + c];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) acc[i] = fmaf(sv, M[c * D + cg + 16 * i], acc[i]);
+            const float4 m = *reinterpret_cast<const float4*>(Ms + c * D + 4 * cg);
+            acc[0] = fmaf(sv, m.x, acc[0]);
+            acc[1] = fmaf(sv, m.y, acc[1]);
+            acc[2] = fmaf(sv, m.z, acc[2]);
+            acc[3] = fmaf(sv, m.w, acc[3]);
         }
-        __syncthreads();  // everyone is done reading S and M[buf]
-        float* dst = a.sin + ((int64_t)(uu + 1) * H + h) * D * D + (int64_t)(e0 + el) * D;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            S[el * D + cg + 16 * i] = acc[i];
-            dst[cg + 16 * i] = acc[i];
-        }
-        if (uu + 1 < last) store_m(buf ^ 1);
+        __syncthreads();  // everyone is done reading S and M_uu
+        *reinterpret_cast<float4*>(S + el * D + 4 * cg) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        *reinterpret_cast<float4*>(a.sin + ((int64_t)(uu + 1) * H + h) * D * D + (int64_t)(e0 + el) * D +
+                                   4 * cg) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        if (uu + 1 < last) store_m();
         __syncthreads();
     }
 }
@@ -1587,7 +1585,7 @@ cudaError_t launch_tc(const TcArgs& a, const TcPlan& p, cudaStream_t stream, int
             if ((err = cudaGetLastError()) != cudaSuccess) return err;
         }
         profile_mark(SLOT_SCAN, true, stream);
-        seg_scan_kernel<<<dim3((unsigned)a.N, (unsigned)a.H, D / 16), 256, SCAN_SMEM, stream>>>(a);
+        seg_scan_kernel<<<dim3((unsigned)a.N, (unsigned)a.H, D / SCAN_ROWS), 256, SCAN_SMEM, stream>>>(a);
         profile_mark(SLOT_SCAN, false, stream);
         *launches += 1;
         if ((err = cudaGetLastError()) != cudaSuccess) return err;
