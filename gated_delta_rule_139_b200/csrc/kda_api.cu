@@ -202,6 +202,7 @@ kda::TcPlan plan_segments(const kda::FwdArgs& a) {
     if (!p.segmented) seg = std::max<int64_t>(nch_seq_max, 1);
     p.seg_chunks = (int)std::min<int64_t>(seg, 1 << 30);
     p.max_units = (int)(p.segmented ? (nch_total + seg - 1) / seg + a.N : a.N);
+    p.total_chunks = nch_total;
     return p;
 }
 
@@ -212,8 +213,8 @@ kda_status run_tc(const kda::FwdArgs& a, cudaStream_t stream, int* launches) {
     const size_t b_off = ((size_t)(a.N + 1) * 4 + 4 + 255) & ~(size_t)255;
     const size_t b_trans = p.segmented ? (size_t)p.max_units * a.H * 2 * st : 0;
     const size_t b_sin = p.segmented ? (size_t)p.max_units * a.H * st : 0;
-    // chunk cache of the segmented plan: kChunkImageBytes per chunk of every unit
-    const size_t b_wu = p.segmented ? (size_t)p.max_units * a.H * p.seg_chunks * kda::kChunkImageBytes : 0;
+    // chunk cache of the segmented plan: kChunkImageBytes per chunk and head
+    const size_t b_wu = p.segmented ? (size_t)p.total_chunks * a.H * kda::kChunkImageBytes : 0;
     char* ws = nullptr;
     cudaError_t e = pool_alloc((void**)&ws, b_segs + b_off + b_trans + b_sin + b_wu, stream);
     if (e != cudaSuccess) return cuda_fail(e, "workspace allocation");
@@ -244,6 +245,7 @@ kda_status run_tc(const kda::FwdArgs& a, cudaStream_t stream, int* launches) {
     t.sin = p.segmented ? (float*)(ws + b_segs + b_off + b_trans) : nullptr;
     if (p.segmented) {  // pass 1 runs over every segment and keeps W^T, U'^T for pass 3
         t.wu = (uint8_t*)(ws + b_segs + b_off + b_trans + b_sin);
+        t.total_chunks = p.total_chunks;
         t.seg_chunks = p.seg_chunks;
         t.trans_all = 1;
     }
@@ -358,7 +360,7 @@ SpanWs span_layout(const kda::FwdArgs& a) {
     w.off = take((size_t)(a.N + 1) * 4 + 4);
     w.trans = take((size_t)w.p.max_units * a.H * 2 * st);
     w.sin = take((size_t)w.p.max_units * a.H * st);
-    w.wu = take((size_t)w.p.max_units * a.H * w.p.seg_chunks * kda::kChunkImageBytes);
+    w.wu = take((size_t)w.p.total_chunks * a.H * kda::kChunkImageBytes);
     w.total = o;
     return w;
 }
@@ -380,6 +382,7 @@ kda::TcArgs span_args(const kda::FwdArgs& a, const SpanWs& w, char* ws) {
     t.trans = (float*)(ws + w.trans);
     t.sin = (float*)(ws + w.sin);
     t.wu = (uint8_t*)(ws + w.wu);
+    t.total_chunks = w.p.total_chunks;
     t.seg_chunks = w.p.seg_chunks;
     t.trans_all = 1;
     return t;

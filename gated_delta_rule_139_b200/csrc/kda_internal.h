@@ -51,10 +51,11 @@ cudaError_t launch_ffma(const FwdArgs& a, cudaStream_t stream, int* launches);
 // possibly the sequence's last.
 struct SegEntry {
     int64_t t_begin, t_end;
-    int32_t n;     // sequence
-    int32_t j;     // segment index inside the sequence
-    int32_t last;  // 1 for the sequence's last segment
+    int32_t n;       // sequence
+    int32_t j;       // segment index inside the sequence
+    int32_t last;    // 1 for the sequence's last segment
     int32_t pad;
+    int64_t c_base;  // index of the segment's first chunk among all chunks of all sequences
 };
 
 // Tensor-core path arguments: the validated forward arguments plus workspace.
@@ -76,7 +77,8 @@ struct TcArgs {
     float* sin;         // [max_units, H, 128, 128]: S_in^T of each segment
     const void* gate = nullptr;  // optional output gate, as in FwdArgs
     int32_t trans_all = 0;       // pass 1 also for each sequence's last segment
-    uint8_t* wu = nullptr;       // chunk cache: [max_units][H][seg_chunks][kChunkImageBytes] (pass 1 writes, pass 3 reads)
+    uint8_t* wu = nullptr;       // chunk cache: [total_chunks][H][kChunkImageBytes] (pass 1 writes, pass 3 reads)
+    int64_t total_chunks = 0;    // chunks the cache holds per head (an upper bound on all sequences' chunks)
     int32_t seg_chunks = 0;      // chunks per segment (cache stride)
     // optional state snapshots, as in FwdArgs
     const int32_t* snap_slots = nullptr;
@@ -96,9 +98,10 @@ struct TcMaps {
 };
 
 struct TcPlan {
-    int seg_chunks;   // chunks per segment
-    int max_units;    // upper bound on the number of segments over all sequences
-    bool segmented;   // some sequence may have more than one segment
+    int seg_chunks;        // chunks per segment
+    int max_units;         // upper bound on the number of segments over all sequences
+    bool segmented;        // some sequence may have more than one segment
+    int64_t total_chunks;  // upper bound on the chunks of all sequences (ceil(T/64) + N packed)
 };
 
 // bf16 q/k/v with d_k = d_v = 128: tcgen05 tensor-core path.  from_cache: the

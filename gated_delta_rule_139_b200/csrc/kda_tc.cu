@@ -506,12 +506,16 @@ __global__ void __launch_bounds__(NT, 1) tc_kernel(TcArgs a, const __grid_consta
     const bool snap_on = !SEG && a.snap_pool != nullptr;
     const bool gate_on = !SEG && a.gate != nullptr;
     uint32_t gate_parity = 0;
-    // Chunk cache (pass 1): entry of chunk t of unit u at
-    // wu + ((u H + h) seg_chunks + chunk) * kChunkImageBytes, pieces at the CI_* offsets.
+    // Chunk cache (pass 1): the entry of the chunk at tt (the unit's chunk (tt - t_begin)/C,
+    // chunk c_base + that among all chunks) and head h at
+    // wu + ((c_base + (tt - t_begin)/C) H + h) * kChunkImageBytes, pieces at the CI_* offsets.
     const bool wu_cache = SEG && a.wu != nullptr;
+    if (wu_cache && (sg.c_base < 0 || sg.c_base + (sg.t_end - sg.t_begin + C - 1) / C > a.total_chunks)) {
+        if (tid == 0) atomicCAS(&g_tc_status, 0, ERR_SEG_OVERFLOW);  // malformed cu_seqlens
+        return;
+    }
     auto wu_tile = [&](int64_t tt) {
-        return a.wu + (((int64_t)u * H + h) * a.seg_chunks + (tt - sg.t_begin) / C) *
-                          (int64_t)kChunkImageBytes;
+        return a.wu + ((sg.c_base + (tt - sg.t_begin) / C) * H + h) * (int64_t)kChunkImageBytes;
     };
     const int64_t seq_lo = snap_on ? (a.cu ? (int64_t)a.cu[sg.n] : (int64_t)sg.n * a.T) : 0;
 
@@ -1089,9 +1093,12 @@ __global__ void __launch_bounds__(NT, 1) cached_kernel(TcArgs a, const __grid_co
     uint64_t* bar_img = bar + 1;                                  // [2] image loads
     uint64_t* bar_gate = bar + 3;                                 // output-gate tile
     uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(sm + LayC::TMEMP);
-    auto entry = [&](int64_t tt) {
-        return a.wu + (((int64_t)u * H + h) * a.seg_chunks + (tt - sg.t_begin) / C) *
-                          (int64_t)kChunkImageBytes;
+    if (sg.c_base < 0 || sg.c_base + (sg.t_end - sg.t_begin + C - 1) / C > a.total_chunks) {
+        if (tid == 0) atomicCAS(&g_tc_status, 0, ERR_SEG_OVERFLOW);  // malformed cu_seqlens
+        return;
+    }
+    auto entry = [&](int64_t tt) {  // the chunk cache entry of the chunk at tt, head h
+        return a.wu + ((sg.c_base + (tt - sg.t_begin) / C) * H + h) * (int64_t)kChunkImageBytes;
     };
     uint32_t pending = 0;  // thread 0: bit b = a load into image b in flight; bit 2 = gate tile
     auto load_img = [&](int64_t tt, int b) {
@@ -1337,9 +1344,14 @@ __global__ void __launch_bounds__(1024) seg_setup_kernel(const int32_t* cu, int 
                                                          SegEntry* segs, int32_t* seg_off,
                                                          int32_t* n_units) {
     __shared__ int32_t warp_sums[32];
+    __shared__ int64_t warp_csums[32];
     __shared__ int32_t carry;
+    __shared__ int64_t carry_c;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    if (tid == 0) carry = 0;
+    if (tid == 0) {
+        carry = 0;
+        carry_c = 0;
+    }
     __syncthreads();
     for (int base = 0; base < N; base += 1024) {
         const int n = base + tid;
@@ -1350,26 +1362,41 @@ __global__ void __launch_bounds__(1024) seg_setup_kernel(const int32_t* cu, int 
         }
         const int64_t nch = hi > lo ? (hi - lo + C - 1) / C : 0;
         int g = n < N ? (int)(nch > 0 ? (nch + seg_chunks - 1) / seg_chunks : 1) : 0;
-        // block-wide exclusive scan of g
+        // block-wide exclusive scans of g (segments) and nch (chunks)
         int x = g;
+        long long xc = nch;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int y = __shfl_up_sync(0xffffffffu, x, o);
-            if (lane >= o) x += y;
+            const long long yc = __shfl_up_sync(0xffffffffu, xc, o);
+            if (lane >= o) {
+                x += y;
+                xc += yc;
+            }
         }
-        if (lane == 31) warp_sums[warp] = x;
+        if (lane == 31) {
+            warp_sums[warp] = x;
+            warp_csums[warp] = xc;
+        }
         __syncthreads();
         if (warp == 0) {
             int w = warp_sums[lane];
+            long long wc = warp_csums[lane];
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const int y = __shfl_up_sync(0xffffffffu, w, o);
-                if (lane >= o) w += y;
+                const long long yc = __shfl_up_sync(0xffffffffu, wc, o);
+                if (lane >= o) {
+                    w += y;
+                    wc += yc;
+                }
             }
             warp_sums[lane] = w;
+            warp_csums[lane] = wc;
         }
         __syncthreads();
         const int excl = carry + x - g + (warp > 0 ? warp_sums[warp - 1] : 0);
+        const int64_t cexcl = carry_c + xc - nch + (warp > 0 ? warp_csums[warp - 1] : 0);
         if (n < N) {
             seg_off[n] = excl;
             for (int j = 0; j < g; ++j) {
@@ -1385,11 +1412,16 @@ __global__ void __launch_bounds__(1024) seg_setup_kernel(const int32_t* cu, int 
                 const int64_t end = lo + (int64_t)(j + 1) * seg_chunks * C;
                 e.t_end = end < hi ? end : hi;
                 e.last = (j == g - 1) ? 1 : 0;
+                e.pad = 0;
+                e.c_base = cexcl + (int64_t)j * seg_chunks;
                 segs[uidx] = e;
             }
         }
         __syncthreads();
-        if (tid == 1023) carry = excl + g;
+        if (tid == 1023) {
+            carry = excl + g;
+            carry_c = cexcl + nch;
+        }
         __syncthreads();
     }
     if (tid == 0) {

@@ -266,3 +266,14 @@ def test_host_entry_point_pipelines_long_sequences_in_spans(monkeypatch, bf16, d
     else:
         assert np.abs(og.reshape(o_r.shape) - o_r).max() <= TOL_F32_MAX_ABS
         assert np.abs(s_h - s_r).max() <= TOL_F32_MAX_ABS
+
+
+def test_packed_one_long_and_many_short_sequences(monkeypatch):
+    """One long sequence cut into segments beside 300 short ones: the chunk cache is
+    indexed by each segment's first chunk among all chunks (the short sequences' units
+    take one entry each), and every output and final state matches the oracle."""
+    monkeypatch.setenv("KDA_SEG_CHUNKS", "4")
+    lens = [64 * 40 + 7] + [1 + (37 * i) % 150 for i in range(300)]
+    inp = make_inputs(1, 0, 2, 128, 128, bf16=True, seed=33, seq_lens=lens, state_sigma=0.05,
+                      gate_sigma=2.0)
+    _check(inp)
