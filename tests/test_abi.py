@@ -292,3 +292,26 @@ def test_span_forward_ex_checks_its_options():
     # workspace placed over the snapshot pool
     assert call_ex(kda.FwdOpts(None, ctypes.pointer(spec), FAKE + (7 << 30), FAKE + (8 << 30)),
                    ws=FAKE + (8 << 30)) == "KDA_ERR_ALIAS"
+
+
+# ---------------------------------------------------------------- host and no-allocation entry points
+@pytest.mark.parametrize("entry", ["kda_fwd_host", "kda_fwd_noalloc"])
+def test_host_and_noalloc_entry_points_reject_bad_arguments(entry):
+    """The argument checks of kda_fwd hold for these entry points too, before any CUDA
+    call (the pointers are never dereferenced)."""
+    lib = kda.load_library()
+    fn = getattr(lib, entry)
+    P = lambda x: None if x is None else ctypes.c_void_p(x)
+
+    def call(d=None, q=FAKE, out=FAKE + (5 << 30), chunk=64, sf=None):
+        rc = fn(P(q), P(FAKE + (1 << 30)), P(FAKE + (2 << 30)), P(FAKE + (3 << 30)), P(FAKE + (4 << 30)),
+                None, None, chunk, P(out), P(sf), ctypes.byref(d or D()), None)
+        return kda.STATUS[rc]
+
+    assert call(d=D(dk=96)) == "KDA_ERR_UNSUPPORTED"
+    assert call(chunk=32) == "KDA_ERR_UNSUPPORTED"
+    assert call(d=D(B=0)) == "KDA_ERR_INVALID_ARG"
+    assert call(q=None) == "KDA_ERR_INVALID_ARG"
+    assert call(q=FAKE + 8) == "KDA_ERR_MISALIGNED"
+    assert call(out=FAKE + (1 << 30)) == "KDA_ERR_ALIAS"  # out over k
+    assert call(sf=FAKE + (4 << 30)) == "KDA_ERR_ALIAS"   # final_state over beta
