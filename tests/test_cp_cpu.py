@@ -59,13 +59,18 @@ def _oracle_ops():
 
     def forward(q, k, v, la, be, s_in, gate, ctx):
         o, s = oracle.recurrent(npy(q), npy(k), npy(v), npy(la), npy(be),
-                                s_in.astype(np.float32), o_tokens=None)
+                                s_in.astype(np.float32), o_tokens=None,
+                                out_gate=None if gate is None else npy(gate))
         return torch.from_numpy(o), torch.from_numpy(s)
 
     return SpanOps(transition, apply, forward)
 
 
-def _rank(rank, world, port, q):
+def _gate(world):
+    return np.random.default_rng(600 + world).uniform(0, 1, (B, SPAN * world, H, DV)).astype(np.float32)
+
+
+def _rank(rank, world, port, q, gated=False):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     from gated_delta_rule_139_b200.cp import cp_prefill
     dist.init_process_group("gloo", rank=rank, world_size=world)
@@ -73,19 +78,20 @@ def _rank(rank, world, port, q):
         x = _inputs(world)
         sl = lambda a: torch.from_numpy(np.ascontiguousarray(a[:, rank * SPAN:(rank + 1) * SPAN]))
         o, s = cp_prefill(sl(x.q), sl(x.k), sl(x.v), sl(x.log_alpha), sl(x.beta),
-                          torch.from_numpy(x.initial_state), ops=_oracle_ops())
+                          torch.from_numpy(x.initial_state), ops=_oracle_ops(),
+                          out_gate=sl(_gate(world)) if gated else None)
         q.put((rank, o.numpy(), s.numpy()))
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 3, 4])
-def test_cp_prefill_on_gloo_ranks_matches_the_whole_sequence(world):
+@pytest.mark.parametrize("world,gated", [(2, False), (3, False), (4, False), (2, True)])
+def test_cp_prefill_on_gloo_ranks_matches_the_whole_sequence(world, gated):
     import oracle
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank, args=(r, world, port, q)) for r in range(world)]
+    procs = [ctx.Process(target=_rank, args=(r, world, port, q, gated)) for r in range(world)]
     for p in procs:
         p.start()
     got = {}
@@ -96,7 +102,8 @@ def test_cp_prefill_on_gloo_ranks_matches_the_whole_sequence(world):
         p.join(60)
         assert p.exitcode == 0
     x = _inputs(world)
-    o_ref, s_ref = oracle.recurrent(x.q, x.k, x.v, x.log_alpha, x.beta, x.initial_state)
+    o_ref, s_ref = oracle.recurrent(x.q, x.k, x.v, x.log_alpha, x.beta, x.initial_state,
+                                    out_gate=_gate(world) if gated else None)
     o_cp = np.concatenate([got[r][0] for r in range(world)], axis=1)
     # the oracle takes its initial state in fp32, so the recovered state enters each
     # span rounded to fp32 (relative 2^-24); a structural mistake would be O(1)
