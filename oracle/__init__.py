@@ -156,3 +156,67 @@ def chunked(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, chunk
     """Chunkwise fp64 reformulation (plain exp(+-g), any chunk size >= 1)."""
     return _run("kda_oracle_chunked", q, k, v, log_alpha, beta, initial_state, cu_seqlens,
                 o_tokens, threads, chunk=chunk, out_gate=out_gate)
+
+
+def chunk_operands(q, k, v, log_alpha, beta, chunk=64):
+    """Per-chunk operands of the chunkwise form, fp64, for ONE sequence.
+
+    Same page and section as :func:`chunked` ("Как распараллелили последовательное
+    обновление": all tokens of a chunk are processed together, then the state is handed
+    on), with plain exp(+-g).  Inputs [T, H, *] or [1, T, H, *] (bf16 as uint16 bits).
+    For chunk c (tokens c*chunk ..) of head h -- a ragged last chunk padded with tokens
+    whose k, q, v, beta and log alpha are zero, which act as identity steps:
+
+        g      in-chunk inclusive cumsum of clamp(log alpha, -5, 0)        [C, d_k]
+        A      strict_lower(diag(beta) (K e^g)(K e^-g)^T)                  [C, C]
+        T      (I + A)^-1, by forward substitution                         [C, C]
+        W      T diag(beta) (K e^g)                                        [C, d_k]
+        U      T diag(beta) V                                              [C, d_v]
+        P      lower_incl((Q e^g)(K e^-g)^T)                               [C, C]
+        Qt     Q e^g                                                       [C, d_k]
+        Kdec   K e^(g_last - g)                                            [C, d_k]
+        gamma  e^(g_last)                                                  [d_k]
+
+    returned as a dict of arrays [n_chunks, H, ...].  From the incoming state S
+    (d_k x d_v) the chunk's outputs are Qt S + P (U - W S) and its outgoing state
+    diag(gamma) S + Kdec^T (U - W S).
+    """
+    q, k, v, la, be = (_widen(x) for x in (q, k, v, log_alpha, beta))
+    if q.ndim == 4:
+        if q.shape[0] != 1:
+            raise ValueError("chunk_operands takes one sequence")
+        q, k, v, la, be = q[0], k[0], v[0], la[0], be[0]
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    C = int(chunk)
+    n = (T + C - 1) // C
+    pad = n * C - T
+
+    def padded(a):
+        return np.concatenate([a, np.zeros((pad,) + a.shape[1:])], axis=0) if pad else a
+
+    q, k, v, la, be = (padded(x) for x in (q, k, v, la, be))
+    out = {name: np.empty((n, H) + shape) for name, shape in
+           (("g", (C, dk)), ("A", (C, C)), ("T", (C, C)), ("W", (C, dk)), ("U", (C, dv)),
+            ("P", (C, C)), ("Qt", (C, dk)), ("Kdec", (C, dk)), ("gamma", (dk,)))}
+    for c in range(n):
+        sl = slice(c * C, (c + 1) * C)
+        for h in range(H):
+            g = np.cumsum(np.clip(la[sl, h], -5.0, 0.0), axis=0)
+            K, Q, V, b = k[sl, h], q[sl, h], v[sl, h], be[sl, h]
+            Ke, Kh, Qe = K * np.exp(g), K * np.exp(-g), Q * np.exp(g)
+            A = np.tril(b[:, None] * (Ke @ Kh.T), -1)
+            Tm = np.zeros((C, C))
+            for i in range(C):  # row i of T from the rows before it: (I + A) T = I
+                Tm[i] = -A[i, :i] @ Tm[:i]
+                Tm[i, i] = 1.0
+            out["g"][c, h] = g
+            out["A"][c, h] = A
+            out["T"][c, h] = Tm
+            out["W"][c, h] = Tm @ (b[:, None] * Ke)
+            out["U"][c, h] = Tm @ (b[:, None] * V)
+            out["P"][c, h] = np.tril(Qe @ Kh.T)
+            out["Qt"][c, h] = Qe
+            out["Kdec"][c, h] = K * np.exp(g[-1] - g)
+            out["gamma"][c, h] = np.exp(g[-1])
+    return out

@@ -255,3 +255,91 @@ def test_cp_snapshots_at_span_aligned_positions(monkeypatch):
                                   inp.beta[:, :L], inp.initial_state, o_tokens=0)
         for h in range(2):
             assert _rel(got[j, h], ref[0, h]) <= TOL_BF16_REL_FRO, (j, h)
+
+
+# ---------------------------------------------------------------- the chunk cache's contents
+# One chunk-cache entry (74 240 bytes per chunk and head) holds bf16 operand images as they sit
+# in shared memory, with the 128-byte swizzle of the tensor-core operand layouts:
+#   K-major (rows r, K index k):  (k // 64) R 128 + (r // 8) 1024 + (r % 8) 128
+#                                 + (((k % 64) // 8) ^ (r % 8)) 16 + (k % 8) 2
+#   MN-major (K rows k, MN index m): the same with (r, k) -> (k, m) and R -> K rows
+# at offsets W^T 0 (MN-major, K rows = channels), U'^T 16K ([128][64], 16-byte pieces of
+# row e XOR-swizzled by e % 8), K_dec 32K (MN-major, K rows = tokens), Q~ 48K (K-major),
+# P 64K (K-major 64 x 64), gamma 72K (fp32 [128]).
+_CI = {"W": 0, "U": 16384, "Kdec": 32768, "Qt": 49152, "P": 65536, "gamma": 73728}
+_ENTRY = 74240
+
+
+def _swz(r, k, R):
+    return (k // 64) * R * 128 + (r // 8) * 1024 + (r % 8) * 128 + (((k % 64) // 8) ^ (r % 8)) * 16 + \
+        (k % 8) * 2
+
+
+def _offsets():
+    """Byte offsets of each piece's elements, as [rows, cols] of the operand (tokens first)."""
+    t = np.arange(64)[:, None]
+    c = np.arange(128)[None, :]
+    s = np.arange(64)[None, :]
+    return {"W": _CI["W"] + _swz(c, t, 128),               # W[t][c] = W^T[c][t], MN-major
+            "U": _CI["U"] + c * 128 + (((t // 8) ^ (c % 8)) << 4) + (t % 8) * 2,  # U'[t][e]
+            "Kdec": _CI["Kdec"] + _swz(t, c, 64),          # K_dec[t][c], MN-major (K rows = t)
+            "Qt": _CI["Qt"] + _swz(t, c, 64),              # Q~[t][c], K-major
+            "P": _CI["P"] + _swz(t, s, 64)}                # P[t][s], K-major
+
+
+def _bf16_round(x):
+    u = np.asarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    return (u.astype(np.uint32) << 16).view(np.float32)
+
+
+def _decode_entry(entry):
+    """{name: float32 array} of one cache entry (uint8 [74240])."""
+    out = {}
+    for name, off in _offsets().items():
+        lo, hi = entry[off].astype(np.uint32), entry[off + 1].astype(np.uint32)
+        out[name] = ((hi << 24) | (lo << 16)).view(np.float32)
+    out["gamma"] = entry[_CI["gamma"]:_CI["gamma"] + 512].view(np.float32).copy()
+    return out
+
+
+def _encode_entry(ops):
+    """The inverse of _decode_entry (bf16 rounding to nearest even), for checking it."""
+    entry = np.zeros(_ENTRY, dtype=np.uint8)
+    for name, off in _offsets().items():
+        bits = _bf16_round(ops[name]).view(np.uint32) >> 16
+        entry[off] = (bits & 0xFF).astype(np.uint8)
+        entry[off + 1] = (bits >> 8).astype(np.uint8)
+    entry[_CI["gamma"]:_CI["gamma"] + 512] = np.asarray(ops["gamma"], np.float32).view(np.uint8)
+    return entry
+
+
+def test_chunk_cache_holds_the_chunkwise_operands():
+    """kda_span_transition leaves every chunk's W, U', K_dec, Q~, P and gamma in the span
+    workspace; decoded from their operand images they match the fp64 chunkwise operands of
+    the oracle (one unsegmented span of 3 full chunks and a ragged one, two heads; bf16
+    operands: relative Frobenius error per chunk and head <= 2e-2; gamma within 1e-4)."""
+    import torch
+    from gated_delta_rule_139_b200 import kda_span_transition, span_workspace
+    T, H = 64 * 3 + 5, 2
+    inp = make_inputs(1, T, H, 128, 128, bf16=True, seed=430, gate_sigma=2.0)
+    d = to_device(inp)
+    ws = span_workspace(d["k"])
+    # workspace of one unit: segment table 256 B, offsets 256 B, transitions and incoming
+    # states of 2 heads (393 216 B), then the cache of 4 chunks x 2 heads
+    base = 512 + H * 3 * 65536
+    assert ws.numel() == base + 4 * H * _ENTRY
+    kda_span_transition(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], ws)
+    torch.cuda.synchronize()
+    raw = ws.cpu().numpy()
+    ref = oracle.chunk_operands(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, 64)
+    for c in range(4):
+        for h in range(H):
+            got = _decode_entry(raw[base + (c * H + h) * _ENTRY: base + (c * H + h + 1) * _ENTRY])
+            for name in ("W", "U", "Kdec", "Qt", "P"):
+                g, r = got[name].astype(np.float64), ref[name][c, h]
+                assert np.isfinite(g).all(), (c, h, name)
+                assert _rel(g, r) <= TOL_BF16_REL_FRO, (c, h, name, _rel(g, r))
+            # gamma = e^{g_last} in fp32 (the sum of up to 64 fp32 gates; strong decay may
+            # fall below fp32's normal range and flush to zero, which is the right limit)
+            np.testing.assert_allclose(got["gamma"], ref["gamma"][c, h], rtol=1e-4, atol=1e-6)

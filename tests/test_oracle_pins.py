@@ -349,3 +349,41 @@ def test_gate_bf16_bits_match_widened_fp32():
     o1, _ = oracle.recurrent(x.q, x.k, x.v, x.log_alpha, x.beta, out_gate=g)
     o2, _ = oracle.recurrent(x.q, x.k, x.v, x.log_alpha, x.beta, out_gate=bf16_to_f32(g))
     np.testing.assert_array_equal(o1, o2)
+
+
+# ---------------------------------------------------------------- per-chunk operands
+@pytest.mark.parametrize("chunk", [1, 8, 16, 64])
+def test_chunk_operands_rebuild_the_recurrence(chunk):
+    """The per-chunk operands, chained from a random state over a ragged sequence, give
+    the token recurrence's outputs and final state; T inverts I + A."""
+    x = make_inputs(1, 77, 2, 6, 5, bf16=False, seed=44, state_sigma=0.3, gate_sigma=2.0)
+    o_ref, s_ref = oracle.recurrent(x.q, x.k, x.v, x.log_alpha, x.beta, x.initial_state)
+    ops = oracle.chunk_operands(x.q, x.k, x.v, x.log_alpha, x.beta, chunk)
+    n = ops["W"].shape[0]
+    S = x.initial_state[0].astype(np.float64).copy()  # [H, dk, dv]
+    outs = []
+    for c in range(n):
+        o_c = np.empty((chunk, 2, 5))
+        for h in range(2):
+            u = ops["U"][c, h] - ops["W"][c, h] @ S[h]
+            o_c[:, h] = ops["Qt"][c, h] @ S[h] + ops["P"][c, h] @ u
+            S[h] = ops["gamma"][c, h][:, None] * S[h] + ops["Kdec"][c, h].T @ u
+            np.testing.assert_allclose((np.eye(chunk) + ops["A"][c, h]) @ ops["T"][c, h],
+                                       np.eye(chunk), atol=1e-9)
+        outs.append(o_c)
+    o = np.concatenate(outs)[:77]
+    assert _rel(o, o_ref.reshape(77, 2, 5)) < 1e-12
+    assert _rel(S, s_ref[0]) < 1e-12
+
+
+def test_chunk_operands_of_padding_rows_are_identity_steps():
+    """Rows past a ragged end: zero W, U, P, Kdec rows, T's identity there, gamma from
+    the last real token."""
+    x = make_inputs(1, 20, 1, 4, 3, bf16=False, seed=45, gate_sigma=2.0)
+    ops = oracle.chunk_operands(x.q, x.k, x.v, x.log_alpha, x.beta, 32)
+    for name in ("W", "U", "Kdec", "Qt"):
+        assert not ops[name][0, 0, 20:].any(), name
+    assert not ops["P"][0, 0, 20:].any() and not ops["A"][0, 0, 20:].any()
+    np.testing.assert_array_equal(ops["T"][0, 0, 20:, 20:], np.eye(12))
+    g_last = np.cumsum(np.clip(x.log_alpha[0, :, 0].astype(np.float64), -5, 0), axis=0)[-1]
+    np.testing.assert_allclose(ops["gamma"][0, 0], np.exp(g_last), rtol=1e-15)
