@@ -19,7 +19,7 @@ import os
 
 __all__ = ["kda_fwd", "kda_fwd_host", "kda_fwd_noalloc", "kda_fwd_snap", "kda_decode",
            "kda_transition", "kda_apply_transitions", "span_workspace", "kda_span_transition",
-           "kda_span_forward", "KDAError", "library_path", "load_library",
+           "kda_span_forward", "kda_chunk_operands", "KDAError", "library_path", "load_library",
            "last_launch_count", "last_path", "check_device", "profile_enable", "profile_read",
            "STATUS"]
 
@@ -99,6 +99,8 @@ def load_library():
         lib.kda_span_forward_ex.argtypes = lib.kda_span_forward.argtypes[:-1] + \
             [ctypes.POINTER(FwdOpts), p]
         lib.kda_span_forward_ex.restype = ctypes.c_int
+        lib.kda_chunk_operands.argtypes = [p, p, p, p, p, ctypes.POINTER(Dims), p, p]
+        lib.kda_chunk_operands.restype = ctypes.c_int
         lib.kda_decode.restype = ctypes.c_int
         lib.kda_status_string.argtypes = [ctypes.c_int]
         lib.kda_status_string.restype = ctypes.c_char_p
@@ -419,9 +421,9 @@ def span_workspace(k):
 
 
 def kda_span_transition(q, k, v, log_alpha, beta, workspace, out=None, stream=None):
-    """kda_transition that also leaves the span's segment transitions and every
-    chunk's output-pass operands (hence q) in ``workspace`` (from
-    :func:`span_workspace`) for :func:`kda_span_forward`."""
+    """kda_transition that also leaves the span's segment table and segment
+    transitions in ``workspace`` (from :func:`span_workspace`) for
+    :func:`kda_span_forward`.  ``q`` is not used (it may be None)."""
     import torch
     lib = load_library()
     d = _span_dims(k)
@@ -430,7 +432,8 @@ def kda_span_transition(q, k, v, log_alpha, beta, workspace, out=None, stream=No
     if stream is None:
         stream = torch.cuda.current_stream(k.device)
     ptr = lambda t: ctypes.c_void_p(t.data_ptr())
-    _check(lib.kda_span_transition(ptr(q), ptr(k), ptr(v), ptr(log_alpha), ptr(beta), ctypes.byref(d),
+    _check(lib.kda_span_transition(None if q is None else ptr(q), ptr(k), ptr(v), ptr(log_alpha),
+                                   ptr(beta), ctypes.byref(d),
                                    ptr(workspace), workspace.numel(), ptr(out),
                                    ctypes.c_void_p(stream.cuda_stream)))
     return out
@@ -471,3 +474,24 @@ def kda_span_forward(q, k, v, log_alpha, beta, workspace, initial_state=None, ou
         opts.snap_pool = snap_pool.data_ptr()
     _check(lib.kda_span_forward_ex(*args, ctypes.byref(opts), ctypes.c_void_p(stream.cuda_stream)))
     return out, final_state
+
+
+CHUNK_IMAGE_BYTES = 74240
+
+
+def kda_chunk_operands(q, k, v, log_alpha, beta, out=None, stream=None):
+    """Every chunk's operand images as the forward pass computes them
+    (kda_chunk_operands): a uint8 tensor [B * ceil(T/64) * H, 74240], entry
+    (b * ceil(T/64) + c) * H + h for chunk c of sequence b and head h."""
+    import torch
+    lib = load_library()
+    d = _span_dims(k)
+    nch = (d.T + 63) // 64
+    if out is None:
+        out = torch.empty((d.B * nch * d.H, CHUNK_IMAGE_BYTES), dtype=torch.uint8, device=k.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(k.device)
+    ptr = lambda t: ctypes.c_void_p(t.data_ptr())
+    _check(lib.kda_chunk_operands(ptr(q), ptr(k), ptr(v), ptr(log_alpha), ptr(beta), ctypes.byref(d),
+                                  ptr(out), ctypes.c_void_p(stream.cuda_stream)))
+    return out

@@ -213,12 +213,10 @@ kda_status run_tc(const kda::FwdArgs& a, cudaStream_t stream, int* launches) {
     const size_t b_off = ((size_t)(a.N + 1) * 4 + 4 + 255) & ~(size_t)255;
     const size_t b_trans = p.segmented ? (size_t)p.max_units * a.H * 2 * st : 0;
     const size_t b_sin = p.segmented ? (size_t)p.max_units * a.H * st : 0;
-    // chunk cache of the segmented plan: kChunkImageBytes per chunk and head
-    const size_t b_wu = p.segmented ? (size_t)p.total_chunks * a.H * kda::kChunkImageBytes : 0;
     char* ws = nullptr;
-    cudaError_t e = pool_alloc((void**)&ws, b_segs + b_off + b_trans + b_sin + b_wu, stream);
+    cudaError_t e = pool_alloc((void**)&ws, b_segs + b_off + b_trans + b_sin, stream);
     if (e != cudaSuccess) return cuda_fail(e, "workspace allocation");
-    kda::TcArgs t;
+    kda::TcArgs t{};
     t.q = a.q;
     t.k = a.k;
     t.v = a.v;
@@ -243,12 +241,6 @@ kda_status run_tc(const kda::FwdArgs& a, cudaStream_t stream, int* launches) {
     t.n_units = t.seg_off + a.N + 1;
     t.trans = p.segmented ? (float*)(ws + b_segs + b_off) : nullptr;
     t.sin = p.segmented ? (float*)(ws + b_segs + b_off + b_trans) : nullptr;
-    if (p.segmented) {  // pass 1 runs over every segment and keeps W^T, U'^T for pass 3
-        t.wu = (uint8_t*)(ws + b_segs + b_off + b_trans + b_sin);
-        t.total_chunks = p.total_chunks;
-        t.seg_chunks = p.seg_chunks;
-        t.trans_all = 1;
-    }
     e = kda::launch_tc(t, p, stream, launches);
     cudaFreeAsync(ws, stream);
     if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
@@ -340,10 +332,10 @@ size_t tc_scratch_bytes(const kda::FwdArgs& a, const kda::TcPlan& p, size_t* b_s
 }
 
 // Workspace of a span (segment table, per-segment transitions and incoming
-// states, chunk cache) for the segment plan of the dims: offsets into one buffer.
+// states) for the segment plan of the dims: offsets into one buffer.
 struct SpanWs {
     kda::TcPlan p;
-    size_t segs, off, trans, sin, wu, total;
+    size_t segs, off, trans, sin, total;
 };
 
 SpanWs span_layout(const kda::FwdArgs& a) {
@@ -360,7 +352,6 @@ SpanWs span_layout(const kda::FwdArgs& a) {
     w.off = take((size_t)(a.N + 1) * 4 + 4);
     w.trans = take((size_t)w.p.max_units * a.H * 2 * st);
     w.sin = take((size_t)w.p.max_units * a.H * st);
-    w.wu = take((size_t)w.p.total_chunks * a.H * kda::kChunkImageBytes);
     w.total = o;
     return w;
 }
@@ -381,9 +372,6 @@ kda::TcArgs span_args(const kda::FwdArgs& a, const SpanWs& w, char* ws) {
     t.n_units = t.seg_off + a.N + 1;
     t.trans = (float*)(ws + w.trans);
     t.sin = (float*)(ws + w.sin);
-    t.wu = (uint8_t*)(ws + w.wu);
-    t.total_chunks = w.p.total_chunks;
-    t.seg_chunks = w.p.seg_chunks;
     t.trans_all = 1;
     return t;
 }
@@ -397,10 +385,11 @@ kda_status check_workspace(const void* ws, size_t bytes, size_t need) {
 }
 
 // Arguments of a span transition (k, v, log_alpha, beta; bf16, d = 128, no cu_seqlens);
-// need_q: q too (the transition that fills a span workspace prepares the output pass).
+// need_q: q too (checked like the other inputs).
 kda_status validate_span_inputs(const void* q, const void* k, const void* v, const float* log_alpha,
                                 const float* beta, const kda_dims* d, const float* trans,
-                                bool need_q, kda::FwdArgs* a) {
+                                bool need_q, kda::FwdArgs* a, size_t trans_bytes = 0,
+                                const char* trans_name = "trans") {
     if (!d) return fail(KDA_ERR_INVALID_ARG, "dims is NULL");
     if (d->B < 1 || d->T < 0 || d->H < 1)
         return fail(KDA_ERR_INVALID_ARG, "need B >= 1, T >= 0, H >= 1 (got B=%d T=%d H=%d)",
@@ -410,13 +399,13 @@ kda_status validate_span_inputs(const void* q, const void* k, const void* v, con
     if (d->d_k != 128 || d->d_v != 128 || d->qkv_dtype != KDA_BF16)
         return fail(KDA_ERR_UNSUPPORTED, "span transitions need bf16 k/v with d_k = d_v = 128");
     const int64_t tokens = (int64_t)d->B * d->T;
-    if (!trans) return fail(KDA_ERR_INVALID_ARG, "trans must be non-NULL");
+    if (!trans) return fail(KDA_ERR_INVALID_ARG, "%s must be non-NULL", trans_name);
     if (tokens > 0 && (!k || !v || !log_alpha || !beta || (need_q && !q)))
         return fail(KDA_ERR_INVALID_ARG, need_q ? "q, k, v, log_alpha and beta must be non-NULL"
                                                 : "k, v, log_alpha and beta must be non-NULL");
     if (!need_q) q = nullptr;
     const void* ptrs[] = {q, k, v, log_alpha, beta, trans};
-    const char* names[] = {"q", "k", "v", "log_alpha", "beta", "trans"};
+    const char* names[] = {"q", "k", "v", "log_alpha", "beta", trans_name};
     for (int i = 0; i < 6; ++i)
         if (ptrs[i] && ((uintptr_t)ptrs[i] & 15u))
             return fail(KDA_ERR_MISALIGNED, "%s is not 16-byte aligned", names[i]);
@@ -427,10 +416,10 @@ kda_status validate_span_inputs(const void* q, const void* k, const void* v, con
                         {(uintptr_t)log_alpha, (uintptr_t)log_alpha + (log_alpha ? n * 4 : 0),
                          "log_alpha"},
                         {(uintptr_t)beta, (uintptr_t)beta + (beta ? tokens * d->H * 4 : 0), "beta"}};
-    const Range rt = {(uintptr_t)trans, (uintptr_t)trans + (uintptr_t)d->B * d->H * 2 * 128 * 128 * 4,
-                      "trans"};
+    if (!trans_bytes) trans_bytes = (size_t)d->B * d->H * 2 * 128 * 128 * 4;
+    const Range rt = {(uintptr_t)trans, (uintptr_t)trans + trans_bytes, trans_name};
     for (const Range& r : in)
-        if (overlaps(rt, r)) return fail(KDA_ERR_ALIAS, "trans overlaps %s", r.name);
+        if (overlaps(rt, r)) return fail(KDA_ERR_ALIAS, "%s overlaps %s", trans_name, r.name);
     a->q = q;
     a->k = k;
     a->v = v;
@@ -799,7 +788,7 @@ kda_status kda_fwd_noalloc(const void* q, const void* k, const void* v, const fl
     // Nothing in the scratch needs to start at zero: the segment-table kernel
     // writes every entry that is read later, pass 1 writes every transition the
     // scan reads, and the scan writes every incoming state pass 3 reads.
-    kda::TcArgs t;
+    kda::TcArgs t{};
     t.q = a.q;
     t.k = a.k;
     t.v = a.v;
@@ -892,15 +881,15 @@ kda_status kda_span_transition(const void* q, const void* k, const void* v, cons
     g_last_launches = 0;
     g_last_path = "";
     kda::FwdArgs a;
-    kda_status st = validate_span_inputs(q, k, v, log_alpha, beta, d, trans, true, &a);
+    kda_status st = validate_span_inputs(nullptr, k, v, log_alpha, beta, d, trans, false, &a);
     if (st != KDA_OK) return st;
+    (void)q;  // not needed: the forward call recomputes every chunk's operands
     const SpanWs w = span_layout(a);
     st = check_workspace(workspace, workspace_bytes, w.total);
     if (st != KDA_OK) return st;
     const int64_t tokens = (int64_t)a.B * a.T, n = tokens * a.H * 128;
     const Range rw = {(uintptr_t)workspace, (uintptr_t)workspace + w.total, "workspace"};
-    const Range other[] = {{(uintptr_t)q, (uintptr_t)q + (q ? n * 2 : 0), "q"},
-                           {(uintptr_t)k, (uintptr_t)k + (k ? n * 2 : 0), "k"},
+    const Range other[] = {{(uintptr_t)k, (uintptr_t)k + (k ? n * 2 : 0), "k"},
                            {(uintptr_t)v, (uintptr_t)v + (v ? n * 2 : 0), "v"},
                            {(uintptr_t)log_alpha, (uintptr_t)log_alpha + (log_alpha ? n * 4 : 0),
                             "log_alpha"},
@@ -909,9 +898,9 @@ kda_status kda_span_transition(const void* q, const void* k, const void* v, cons
                             "trans"}};
     for (const Range& r : other)
         if (overlaps(rw, r)) return fail(KDA_ERR_ALIAS, "workspace overlaps %s", r.name);
-    const void* wp[] = {q, k, v, log_alpha, beta, trans, workspace};
-    const char* wn[] = {"q", "k", "v", "log_alpha", "beta", "trans", "workspace"};
-    st = check_accessible(wp, wn, 7);
+    const void* wp[] = {k, v, log_alpha, beta, trans, workspace};
+    const char* wn[] = {"k", "v", "log_alpha", "beta", "trans", "workspace"};
+    st = check_accessible(wp, wn, 6);
     if (st != KDA_OK) return st;
     kda::TcArgs t = span_args(a, w, (char*)workspace);
     int launches = 0;
@@ -975,7 +964,7 @@ kda_status kda_span_forward_ex(const void* q, const void* k, const void* v,
     t.snap_num_slots = a.snap_num_slots;
     int launches = 0;
     g_last_path = "tc";
-    cudaError_t e = kda::launch_tc(t, w.p, (cudaStream_t)stream, &launches, /*from_cache=*/true);
+    cudaError_t e = kda::launch_tc(t, w.p, (cudaStream_t)stream, &launches, /*from_span=*/true);
     g_last_launches = launches;
     if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
     return KDA_OK;
@@ -987,6 +976,60 @@ kda_status kda_span_forward(const void* q, const void* k, const void* v, const f
                             size_t workspace_bytes, void* stream) {
     return kda_span_forward_ex(q, k, v, log_alpha, beta, initial_state, out, final_state, d,
                                workspace, workspace_bytes, nullptr, stream);
+}
+
+kda_status kda_chunk_operands(const void* q, const void* k, const void* v, const float* log_alpha,
+                              const float* beta, const kda_dims* d, void* images, void* stream) {
+    g_last_error[0] = 0;
+    g_last_launches = 0;
+    g_last_path = "";
+    if (!d) return fail(KDA_ERR_INVALID_ARG, "dims is NULL");
+    const int64_t nch = d->T > 0 ? ((int64_t)d->T + kda::kChunk - 1) / kda::kChunk : 0;
+    const size_t bytes = (size_t)std::max<int64_t>(d->B, 0) * nch * std::max(d->H, 0) *
+                         kda::kChunkImageBytes;
+    kda::FwdArgs a;
+    kda_status st = validate_span_inputs(q, k, v, log_alpha, beta, d, (const float*)images, true, &a,
+                                         std::max<size_t>(bytes, 1), "images");
+    if (st != KDA_OK) return st;
+    const void* wp[] = {q, k, v, log_alpha, beta, images};
+    const char* wn[] = {"q", "k", "v", "log_alpha", "beta", "images"};
+    st = check_accessible(wp, wn, 6);
+    if (st != KDA_OK) return st;
+    if (nch == 0) return KDA_OK;
+    // one segment per sequence: chunk c of sequence b is entry b * nch + c
+    kda::TcPlan p;
+    p.seg_chunks = (int)std::min<int64_t>(nch, 1 << 30);
+    p.segmented = false;
+    p.max_units = a.N;
+    p.total_chunks = (int64_t)a.B * nch;
+    const size_t b_segs = ((size_t)p.max_units * sizeof(kda::SegEntry) + 255) & ~(size_t)255;
+    const size_t b_off = ((size_t)(a.N + 1) * 4 + 4 + 255) & ~(size_t)255;
+    cudaStream_t cs = (cudaStream_t)stream;
+    char* ws = nullptr;
+    cudaError_t e = pool_alloc((void**)&ws, b_segs + b_off, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "workspace allocation");
+    kda::TcArgs t{};
+    t.q = q;
+    t.k = k;
+    t.v = v;
+    t.log_alpha = log_alpha;
+    t.beta = beta;
+    t.B = a.B;
+    t.T = a.T;
+    t.H = a.H;
+    t.N = a.N;
+    t.segs = (kda::SegEntry*)ws;
+    t.seg_off = (int32_t*)(ws + b_segs);
+    t.n_units = t.seg_off + a.N + 1;
+    t.dump = (uint8_t*)images;
+    t.total_chunks = p.total_chunks;
+    int launches = 0;
+    g_last_path = "tc";
+    e = kda::launch_dump(t, p, cs, &launches);
+    cudaFreeAsync(ws, cs);
+    g_last_launches = launches;
+    if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+    return KDA_OK;
 }
 
 kda_status kda_apply_transitions(const float* trans, int32_t count, int32_t B, int32_t H,

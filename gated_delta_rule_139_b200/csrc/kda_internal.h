@@ -77,22 +77,21 @@ struct TcArgs {
     float* sin;         // [max_units, H, 128, 128]: S_in^T of each segment
     const void* gate = nullptr;  // optional output gate, as in FwdArgs
     int32_t trans_all = 0;       // pass 1 also for each sequence's last segment
-    uint8_t* wu = nullptr;       // chunk cache: [total_chunks][H][kChunkImageBytes] (pass 1 writes, pass 3 reads)
-    int64_t total_chunks = 0;    // chunks the cache holds per head (an upper bound on all sequences' chunks)
-    int32_t seg_chunks = 0;      // chunks per segment (cache stride)
+    uint8_t* dump = nullptr;     // operand dump: [total_chunks][H][kChunkImageBytes] (launch_dump)
+    int64_t total_chunks = 0;    // chunks the dump holds per head
     // optional state snapshots, as in FwdArgs
     const int32_t* snap_slots = nullptr;
     float* snap_pool = nullptr;
     int32_t snap_interval = 0, snap_max = 0, snap_num_slots = 0;
 };
 
-// TMA descriptors of the q, k, v, out, gate (bf16) and log_alpha (fp32)
-// tensors, viewed as [T, H, 128]; passed as a grid constant.
-// Bytes of one chunk's entry in the chunk cache that pass 1 leaves for pass 3:
-// the bf16 operand images of W^T, U'^T, K_dec, Q~ (16 KB each), P (8 KB) and
+// Bytes of one chunk's operand images as the operand dump writes them (per chunk
+// and head): the bf16 images of W^T, U'^T, K_dec, Q~ (16 KB each), P (8 KB) and
 // the fp32 chunk decay gamma (512 B).
 constexpr size_t kChunkImageBytes = 74240;
 
+// TMA descriptors of the q, k, v, out, gate (bf16) and log_alpha (fp32)
+// tensors, viewed as [T, H, 128]; passed as a grid constant.
 struct TcMaps {
     CUtensorMap q, k, v, la, out, gate;
 };
@@ -104,11 +103,14 @@ struct TcPlan {
     int64_t total_chunks;  // upper bound on the chunks of all sequences (ceil(T/64) + N packed)
 };
 
-// bf16 q/k/v with d_k = d_v = 128: tcgen05 tensor-core path.  from_cache: the
-// segment table, the transitions and the chunk cache of this plan are already in
-// a's workspace (left by launch_transition), so only the scan and pass 3 run.
+// bf16 q/k/v with d_k = d_v = 128: tcgen05 tensor-core path.  from_span: the
+// segment table and the transitions of this plan are already in a's workspace
+// (left by launch_transition), so only the scan and pass 3 run.
 cudaError_t launch_tc(const TcArgs& a, const TcPlan& p, cudaStream_t stream, int* launches,
-                      bool from_cache = false);
+                      bool from_span = false);
+// Every chunk's operand images (kChunkImageBytes each) into a.dump: the segment
+// table, then the forward pass's chunk-local work with a chain that only copies.
+cudaError_t launch_dump(const TcArgs& a, const TcPlan& p, cudaStream_t stream, int* launches);
 
 // Chain of affine state maps S -> M S + B, in the transposed layout of the
 // library's transitions (entry [2][128][128]: B^T, then M^T; S^T_out = S^T_in M^T

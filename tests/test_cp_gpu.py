@@ -117,8 +117,8 @@ def test_context_parallel_prefill_emulated_on_one_gpu(world):
 def test_span_transition_and_forward_share_the_work(monkeypatch, seg_chunks):
     """kda_span_transition fills the workspace; kda_span_forward from it gives
     kda_fwd's results (bit for bit when the span is cut into segments, where
-    kda_fwd takes the same cached path; within tolerance otherwise) and the
-    transition equals kda_transition's."""
+    kda_fwd runs the same scan and forward pass; within tolerance otherwise) and
+    the transition equals kda_transition's."""
     import torch
     from gated_delta_rule_139_b200 import (kda_fwd, kda_span_forward, kda_span_transition,
                                            kda_transition, span_workspace)
@@ -149,7 +149,7 @@ def test_span_transition_and_forward_share_the_work(monkeypatch, seg_chunks):
 
 def test_cp_prefill_through_a_one_rank_nccl_group(monkeypatch):
     """The collective code path with real kernels: one rank, with the span cut
-    into segments (so kda_fwd takes the same cached path), so it must equal
+    into segments (so kda_fwd takes the same segmented path), so it must equal
     kda_fwd bit for bit."""
     import torch
     import torch.distributed as dist
@@ -198,7 +198,7 @@ def test_cp_prefill_with_output_gate(monkeypatch):
 
 def test_span_forward_with_gate_and_snapshots_equals_kda_fwd(monkeypatch):
     """kda_span_forward_ex from the workspace: with the span cut into segments it
-    takes kda_fwd's cached path, so output, state and snapshots equal
+    takes kda_fwd's segmented path, so output, state and snapshots equal
     kda_fwd_snap's with the same gate bit for bit."""
     import torch
     from gated_delta_rule_139_b200 import (kda_fwd_snap, kda_span_forward, kda_span_transition,
@@ -257,9 +257,9 @@ def test_cp_snapshots_at_span_aligned_positions(monkeypatch):
             assert _rel(got[j, h], ref[0, h]) <= TOL_BF16_REL_FRO, (j, h)
 
 
-# ---------------------------------------------------------------- the chunk cache's contents
-# One chunk-cache entry (74 240 bytes per chunk and head) holds bf16 operand images as they sit
-# in shared memory, with the 128-byte swizzle of the tensor-core operand layouts:
+# ---------------------------------------------------------------- the chunkwise operands
+# kda_chunk_operands writes, per chunk and head, one 74 240-byte entry of bf16 operand images
+# as they sit in shared memory, with the 128-byte swizzle of the tensor-core operand layouts:
 #   K-major (rows r, K index k):  (k // 64) R 128 + (r // 8) 1024 + (r % 8) 128
 #                                 + (((k % 64) // 8) ^ (r % 8)) 16 + (k % 8) 2
 #   MN-major (K rows k, MN index m): the same with (r, k) -> (k, m) and R -> K rows
@@ -287,14 +287,8 @@ def _offsets():
             "P": _CI["P"] + _swz(t, s, 64)}                # P[t][s], K-major
 
 
-def _bf16_round(x):
-    u = np.asarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
-    u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
-    return (u.astype(np.uint32) << 16).view(np.float32)
-
-
 def _decode_entry(entry):
-    """{name: float32 array} of one cache entry (uint8 [74240])."""
+    """{name: float32 array} of one entry (uint8 [74240])."""
     out = {}
     for name, off in _offsets().items():
         lo, hi = entry[off].astype(np.uint32), entry[off + 1].astype(np.uint32)
@@ -303,43 +297,38 @@ def _decode_entry(entry):
     return out
 
 
-def _encode_entry(ops):
-    """The inverse of _decode_entry (bf16 rounding to nearest even), for checking it."""
-    entry = np.zeros(_ENTRY, dtype=np.uint8)
-    for name, off in _offsets().items():
-        bits = _bf16_round(ops[name]).view(np.uint32) >> 16
-        entry[off] = (bits & 0xFF).astype(np.uint8)
-        entry[off + 1] = (bits >> 8).astype(np.uint8)
-    entry[_CI["gamma"]:_CI["gamma"] + 512] = np.asarray(ops["gamma"], np.float32).view(np.uint8)
-    return entry
-
-
-def test_chunk_cache_holds_the_chunkwise_operands():
-    """kda_span_transition leaves every chunk's W, U', K_dec, Q~, P and gamma in the span
-    workspace; decoded from their operand images they match the fp64 chunkwise operands of
-    the oracle (one unsegmented span of 3 full chunks and a ragged one, two heads; bf16
-    operands: relative Frobenius error per chunk and head <= 2e-2; gamma within 1e-4)."""
+@pytest.mark.parametrize("gate_sigma,pin", [(2.0, None), (1.0, "floor"), (1.0, "mixed")])
+def test_chunk_operands_match_the_oracle(gate_sigma, pin):
+    """kda_chunk_operands gives every chunk's W, U', K_dec, Q~, P and gamma as the forward
+    pass hands them to its state products; decoded from their operand images they match the
+    fp64 chunkwise operands of the oracle (two sequences of 3 full chunks and a ragged one,
+    two heads; bf16 operands: relative Frobenius error per chunk and head <= 2e-2; gamma
+    within 1e-4).  pin="floor": every gate at the clamp floor (the in-chunk decay reaches
+    e^-315); pin="mixed": half the channels at the floor, half at log alpha = 0."""
     import torch
-    from gated_delta_rule_139_b200 import kda_span_transition, span_workspace
-    T, H = 64 * 3 + 5, 2
-    inp = make_inputs(1, T, H, 128, 128, bf16=True, seed=430, gate_sigma=2.0)
+    from gated_delta_rule_139_b200 import kda_chunk_operands
+    T, H, B = 64 * 3 + 5, 2, 2
+    inp = make_inputs(B, T, H, 128, 128, bf16=True, seed=430, gate_sigma=gate_sigma)
+    if pin == "floor":
+        inp.log_alpha[...] = -5.0
+    elif pin == "mixed":
+        inp.log_alpha[..., 0::2] = -5.0
+        inp.log_alpha[..., 1::2] = 0.0
     d = to_device(inp)
-    ws = span_workspace(d["k"])
-    # workspace of one unit: segment table 256 B, offsets 256 B, transitions and incoming
-    # states of 2 heads (393 216 B), then the cache of 4 chunks x 2 heads
-    base = 512 + H * 3 * 65536
-    assert ws.numel() == base + 4 * H * _ENTRY
-    kda_span_transition(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], ws)
+    raw = kda_chunk_operands(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"]).cpu().numpy()
     torch.cuda.synchronize()
-    raw = ws.cpu().numpy()
-    ref = oracle.chunk_operands(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, 64)
-    for c in range(4):
-        for h in range(H):
-            got = _decode_entry(raw[base + (c * H + h) * _ENTRY: base + (c * H + h + 1) * _ENTRY])
-            for name in ("W", "U", "Kdec", "Qt", "P"):
-                g, r = got[name].astype(np.float64), ref[name][c, h]
-                assert np.isfinite(g).all(), (c, h, name)
-                assert _rel(g, r) <= TOL_BF16_REL_FRO, (c, h, name, _rel(g, r))
-            # gamma = e^{g_last} in fp32 (the sum of up to 64 fp32 gates; strong decay may
-            # fall below fp32's normal range and flush to zero, which is the right limit)
-            np.testing.assert_allclose(got["gamma"], ref["gamma"][c, h], rtol=1e-4, atol=1e-6)
+    nch = 4
+    assert raw.shape == (B * nch * H, _ENTRY)
+    for b in range(B):
+        ref = oracle.chunk_operands(inp.q[b:b + 1], inp.k[b:b + 1], inp.v[b:b + 1],
+                                    inp.log_alpha[b:b + 1], inp.beta[b:b + 1], 64)
+        for c in range(nch):
+            for h in range(H):
+                got = _decode_entry(raw[(b * nch + c) * H + h])
+                for name in ("W", "U", "Kdec", "Qt", "P"):
+                    g, r = got[name].astype(np.float64), ref[name][c, h]
+                    assert np.isfinite(g).all(), (b, c, h, name)
+                    assert _rel(g, r) <= TOL_BF16_REL_FRO, (b, c, h, name, _rel(g, r))
+                # gamma = e^{g_last} in fp32 (the sum of up to 64 fp32 gates; strong decay may
+                # fall below fp32's normal range and flush to zero, which is the right limit)
+                np.testing.assert_allclose(got["gamma"], ref["gamma"][c, h], rtol=1e-4, atol=1e-6)
