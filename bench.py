@@ -308,22 +308,23 @@ def kernel_algorithmic_bytes(name, inp, path_bytes):
 
     pass 3 (forward) delivers the path's results from its inputs: the whole
     path's algorithmic bytes.  Pass 1 (segment transitions) runs over every
-    segment when sequences are cut, and also prepares every chunk's operands
-    of the output pass: it reads q, k, v, log alpha and beta of every token
-    and writes one (B, M) pair (2 x 128 x 128 fp32) per segment and head.  The
-    chunk cache (about 1160 B per token-head, written by pass 1 and read by
-    pass 3) is implementation traffic, not counted."""
+    segment that has a successor: it reads k, v, log alpha and beta of those
+    segments' tokens and writes one (B, M) pair (2 x 128 x 128 fp32) per such
+    segment and head."""
     if name != "tc_pass1_transitions":
         return path_bytes
     seg, cut = segment_plan(inp)
     if not cut:
         return 0
-    per_tok = inp.H * (2 * inp.dk * 2 + inp.dv * 2 + inp.dk * 4 + 4)
-    segs = 0
+    per_tok = inp.H * (inp.dk * 2 + inp.dv * 2 + inp.dk * 4 + 4)
+    toks = segs = 0
     for L in inp.seq_lens:
-        nch = (int(L) + 63) // 64
-        segs += max(1, (nch + seg - 1) // seg)
-    return inp.tokens * per_tok + segs * inp.H * 2 * inp.dk * inp.dv * 4
+        L = int(L)
+        nch = (L + 63) // 64
+        g = max(1, (nch + seg - 1) // seg)
+        segs += g - 1
+        toks += min(L, (g - 1) * seg * 64)
+    return toks * per_tok + segs * inp.H * 2 * inp.dk * inp.dv * 4
 
 
 # ------------------------------------------------------------------ traffic record
@@ -537,20 +538,33 @@ def main():
         pass
     launches = 0
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    kda.profile_read()  # discard warm-up records
-    kda.profile_enable(True)
+    # the headline: K steps with no per-launch instrumentation
     with ClockSampler(uuid) as clk:
         ev0.record(stream)
         for _ in range(args.steps):
             launches += step()
         ev1.record(stream)
         stream.synchronize()
-    kda.profile_enable(False)
-    per_kernel = kda.profile_read()
     if pg:
         pg.barrier()
     torch.cuda.synchronize()
     ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, pg, dev)
+    # a second, separate loop with CUDA events around every internal launch (on the
+    # stream the kernels run on) for the per-kernel times and shares
+    kda.profile_read()  # discard earlier records
+    kda.profile_enable(True)
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    p0.record(stream)
+    for _ in range(args.steps):
+        step()
+    p1.record(stream)
+    stream.synchronize()
+    kda.profile_enable(False)
+    per_kernel = kda.profile_read()
+    prof_ms = p0.elapsed_time(p1) / args.steps
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
     clocks = clk.summary()
     value = job_throughput(world, tokens, ms)
 
@@ -612,7 +626,8 @@ def main():
         cfg["snapshots"] = {"interval_tokens": args.snap_interval, "count": snap["count"],
                             "bytes": snap["count"] * inp.H * inp.dk * inp.dv * 4,
                             "entry": "kda_fwd_snap"}
-    kernels = {name: {"ms_per_launch": tot / n, "launches": n, "share": tot / (ms * args.steps)}
+    kernels = {name: {"ms_per_launch": tot / n, "launches": n,
+                      "share": tot / (prof_ms * args.steps)}
                for name, (tot, n) in per_kernel.items()}
     dom = max(kernels, key=lambda k_: kernels[k_]["ms_per_launch"] * kernels[k_]["launches"])
     dom_bytes = kernel_algorithmic_bytes(dom, inp, alg_bytes)

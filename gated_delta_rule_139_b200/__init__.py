@@ -24,7 +24,8 @@ __all__ = ["kda_fwd", "kda_fwd_host", "kda_fwd_noalloc", "kda_fwd_snap", "kda_de
            "STATUS"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-library_path = os.path.join(_PKG, "libkda.so")
+# KDA_LIBRARY selects another build of the same library (e.g. the phase-trace build)
+library_path = os.environ.get("KDA_LIBRARY") or os.path.join(_PKG, "libkda.so")
 
 STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED",
           3: "KDA_ERR_MISALIGNED", 4: "KDA_ERR_ALIAS", 5: "KDA_ERR_CUDA",
@@ -101,6 +102,8 @@ def load_library():
         lib.kda_span_forward_ex.restype = ctypes.c_int
         lib.kda_chunk_operands.argtypes = [p, p, p, p, p, ctypes.POINTER(Dims), p, p]
         lib.kda_chunk_operands.restype = ctypes.c_int
+        lib.kda_selftest_wait.argtypes = [ctypes.c_uint64, ctypes.c_int32, p]
+        lib.kda_selftest_wait.restype = ctypes.c_int
         lib.kda_decode.restype = ctypes.c_int
         lib.kda_status_string.argtypes = [ctypes.c_int]
         lib.kda_status_string.restype = ctypes.c_char_p

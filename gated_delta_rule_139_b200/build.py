@@ -1,11 +1,16 @@
 """Build libkda.so in place with nvcc for sm_100a (B200).
 
-    python -m gated_delta_rule_139_b200.build [--force]
+    python -m gated_delta_rule_139_b200.build [--force] [--trace]
 
 Each ``csrc/*.cu`` file is compiled to an object in ``_build/`` (in parallel),
 then linked into ``gated_delta_rule_139_b200/libkda.so``.  Objects are rebuilt
 when their source, any ``csrc/*.h`` / ``include/*.h`` header, or this script is
 newer.
+
+``--trace`` builds a separate diagnostic library, ``_build/trace/libkda.so``,
+compiled with ``-DKDA_PHASE_TRACE``: the tensor-core kernels record the SM clock
+at their phase boundaries for the first CTA, readable with ``kda_trace_read``.
+Load it by setting ``KDA_LIBRARY`` to its path before importing the package.
 """
 from __future__ import annotations
 
@@ -32,19 +37,22 @@ def _newest(paths):
     return max((os.path.getmtime(p) for p in paths), default=0.0)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, trace: bool = False) -> str:
+    build_dir = os.path.join(BUILD, "trace") if trace else BUILD
+    lib_path = os.path.join(build_dir, "libkda.so") if trace else LIB
+    cflags = CFLAGS + (["-DKDA_PHASE_TRACE"] if trace else [])
+    os.makedirs(build_dir, exist_ok=True)
     sources = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     headers = glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.cuh")) + \
         glob.glob(os.path.join(INCLUDE, "*.h")) + [os.path.abspath(__file__)]
     hdr_time = _newest(headers)
     objs, jobs = [], []
     for src in sources:
-        obj = os.path.join(BUILD, os.path.basename(src) + ".o")
+        obj = os.path.join(build_dir, os.path.basename(src) + ".o")
         objs.append(obj)
         if force or not os.path.exists(obj) or os.path.getmtime(obj) < max(
                 os.path.getmtime(src), hdr_time):
-            jobs.append([NVCC] + CFLAGS + ["-c", src, "-o", obj])
+            jobs.append([NVCC] + cflags + ["-c", src, "-o", obj])
 
     def run(cmd):
         if verbose:
@@ -57,12 +65,12 @@ def build(force: bool = False, verbose: bool = False) -> str:
 
     with ThreadPoolExecutor(max(1, min(len(jobs), os.cpu_count() or 1))) as ex:
         list(ex.map(run, jobs))
-    if force or jobs or not os.path.exists(LIB) or os.path.getmtime(LIB) < _newest(objs):
-        tmp = LIB + f".tmp{os.getpid()}"
+    if force or jobs or not os.path.exists(lib_path) or os.path.getmtime(lib_path) < _newest(objs):
+        tmp = lib_path + f".tmp{os.getpid()}"
         run([NVCC] + ARCH + ["-shared", "-o", tmp] + objs + ["-lcudart"])
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib_path)
+    return lib_path
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose=True))
+    print(build(force="--force" in sys.argv, verbose=True, trace="--trace" in sys.argv))

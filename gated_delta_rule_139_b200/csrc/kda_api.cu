@@ -1210,6 +1210,19 @@ const char* kda_profile_slot_name(int32_t slot) {
     return (slot >= 0 && slot < kda::NUM_SLOTS) ? names[slot] : "";
 }
 
+kda_status kda_selftest_wait(uint64_t timeout_ns, int32_t arrive, void* stream) {
+    g_last_error[0] = 0;
+    g_last_launches = 0;
+    g_last_path = "";
+    if (timeout_ns < 1000 || timeout_ns > 100000000ull)
+        return fail(KDA_ERR_INVALID_ARG, "timeout_ns must lie in [1e3, 1e8] (got %llu)",
+                    (unsigned long long)timeout_ns);
+    cudaError_t e = kda::launch_wait_probe(timeout_ns, arrive != 0, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+    g_last_launches = 1;
+    return KDA_OK;
+}
+
 kda_status kda_check_device(void* stream) {
     g_last_error[0] = 0;
     cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);

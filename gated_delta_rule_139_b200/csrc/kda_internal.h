@@ -140,6 +140,8 @@ cudaError_t launch_chain(const ChainArgs& c, cudaStream_t stream, int* launches)
 cudaError_t launch_transition(const TcArgs& a, const TcPlan& p, float* out, cudaStream_t stream,
                               int* launches);
 size_t tc_smem_bytes();
+// The bounded-wait self-test kernel (kda_selftest_wait).
+cudaError_t launch_wait_probe(uint64_t timeout_ns, int arrive, cudaStream_t stream);
 // Reads and clears the current device's status word (0 = no device-side error).
 cudaError_t tc_take_status(int* code);
 

@@ -39,12 +39,12 @@
 // (<= 1) for the first half's keys.  The state-side operands K e^g, Q e^g and
 // K e^{g_last - g} are products of factors whose exact value is <= 1.
 //
-// Warp roles inside each CTA (one CTA per SM, 12 warps):
+// Warp roles inside each CTA (one CTA per SM, 16 warps):
 //   warps 0-7 ("prep"): the chunk-local work of chunk c+1 -- raw inputs by
 //     128-bit loads one chunk ahead, gates, operand images, [A;P] product,
 //     inversion, W and U' products -- into a two-slot shared-memory ring
 //     (W, Q~, K_dec, P, gamma) and the U accumulator in tensor memory;
-//   warps 8-11 ("chain"): the state chain of chunk c -- bf16 copy of S,
+//   warps 8-15 ("chain"): the state chain of chunk c -- bf16 copy of S,
 //     U -= S W, S += U K_dec, O = S Q~ + U P and the output epilogue; for the
 //     transitions the same two products on B and then on M.
 // The chain waits only on the ring, so one chunk's chunk-local work overlaps
@@ -63,12 +63,29 @@ namespace {
 
 __device__ int g_tc_status = 0;  // first device-side error code of this device (0 = none)
 
+// Phase trace (builds with -DKDA_PHASE_TRACE only): the SM clock at the phase
+// boundaries of the first kTraceChunks chunks of CTA (0, 0), per warp group
+// (0 prep, 1 chain), read back by kda_trace_read.
+#ifdef KDA_PHASE_TRACE
+constexpr int kTraceChunks = 64, kTraceStamps = 16;
+__device__ unsigned long long g_trace[2][kTraceChunks][kTraceStamps];
+#define TRACE(grp, chunk, k)                                                                    \
+    do {                                                                                        \
+        if (blockIdx.x == 0 && blockIdx.y == 0 && (chunk) < kTraceChunks)                       \
+            g_trace[grp][chunk][k] = clock64();                                                 \
+    } while (0)
+#else
+#define TRACE(grp, chunk, k) \
+    do {                     \
+    } while (0)
+#endif
+
 using namespace tc;
 
 constexpr int C = 64;              // tokens per chunk
 constexpr int D = 128;             // d_k = d_v
 constexpr int NPREP = 256;         // prep threads (warps 0-7)
-constexpr int NCHAIN = 128;        // chain threads (warps 8-11, one per TMEM lane quadrant)
+constexpr int NCHAIN = 256;        // chain threads (warps 8-15, two per TMEM lane quadrant)
 constexpr int NT = NPREP + NCHAIN;
 constexpr int BAR_PREP = 1, BAR_CHAIN = 2;  // named barriers of the two groups
 constexpr float LOG2E = 1.4426950408889634f;
@@ -76,13 +93,17 @@ constexpr float LOG2E = 1.4426950408889634f;
 enum Mode : int { FWD = 0, TRANS = 1, DUMP = 2 };
 
 // ---------------------------------------------------------------- shared memory map
-// Ring slot (two of them), 1024-byte aligned pieces:
-//   S_W   W^T, MN-major (K rows = channels, MN = tokens); after the chain's U
-//         product it holds the chunk's output-gate tile and then its bf16 output
-//         tile [64][128] for the TMA store (forward pass)
-//   S_KD  K_dec = K e^{g_last - g}, MN-major (K rows = tokens)
-//   S_QT  Q~ = Q e^g, K-major [64][128]            (forward pass)
-//   S_PB  P, K-major [64][64]                      (forward pass)
+// Ring slot (two of them; chunk c uses slot c % 2), 1024-byte aligned pieces.  Each
+// piece first receives one of the chunk's raw tiles by TMA, which the prep reads before
+// it writes the piece's operand image over it:
+//   S_W   v tile (two 64-channel boxes, 128-byte swizzle: the A operand of U'^T), then
+//         W^T, MN-major (K rows = channels, MN = tokens); after the chain's U product
+//         the chunk's output-gate tile, then its bf16 output tile [64][128] for the TMA
+//         store (forward pass)
+//   S_KD  k tile [64][128] bf16, then K_dec = K e^{g_last - g}, MN-major (K rows = tokens)
+//   S_QT  q tile, then Q~ = Q e^g, K-major [64][128]          (forward pass)
+//   S_PB  the eight warps' gate sums (fp32 [8][128]), then P, K-major [64][64]
+//                                                             (forward pass)
 //   S_GAM gamma = e^{g_last}, fp32 [128]
 // Prep scratch:
 //   X1    [A;P] A operand, K-major 128 x 128: rows 0-63 k e^{g-rho}, rows 64-127
@@ -92,7 +113,8 @@ enum Mode : int { FWD = 0, TRANS = 1, DUMP = 2 };
 //   after the [A;P] product X1 and BT hold As, Ts, Ys (the inversion's fp32
 //   scratch) and TB = T diag(beta) (bf16, K-major [r][s])
 //   KG    K e^g, MN-major (K rows = tokens): A operand of W^T
-//   V     the chunk's v tile as TMA wrote it: A operand of U'^T
+//   LA    the next chunk's log alpha tile [64][128] fp32 (TMA)
+//   GSUM  the gate sums when the slot has no P piece (transitions)
 template <int MODE>
 struct Lay {
     static constexpr bool Q = MODE != TRANS;
@@ -102,10 +124,10 @@ struct Lay {
     static constexpr uint32_t X1 = 2 * SLOT;
     static constexpr uint32_t BT = X1 + 32768;
     static constexpr uint32_t KG = BT + 24576;
-    static constexpr uint32_t V = KG + 16384;
+    static constexpr uint32_t LA = KG + 16384;
     static constexpr uint32_t AS = X1, TS = AS + 17408, YS = TS + 18432, TB = YS + 5120;
-    static constexpr uint32_t GSUM = V + 16384;   // fp32 [8][128] per-warp gate sums
-    static constexpr uint32_t BETA = GSUM + 4096;  // fp32 [64]
+    static constexpr uint32_t GSUM = LA + 32768;   // fp32 [8][128] (transitions only)
+    static constexpr uint32_t BETA = GSUM + (Q ? 0 : 4096);  // fp32 [64]
     static constexpr uint32_t BAR = BETA + 256;    // mbarriers
     static constexpr uint32_t TMEMP = BAR + 256;   // TMEM base address
     static constexpr uint32_t BYTES = TMEMP + 16 + 1024;  // + alignment slack
@@ -119,7 +141,7 @@ static_assert(Lay<FWD>::BYTES <= 232448 && Lay<TRANS>::BYTES <= 232448, "shared 
 enum Bars : int {
     B_AP = 0,      // prep: [A;P] product done
     B_WU = 1,      // prep: W and U' products done
-    B_V = 2,       // prep: v tile landed (TMA)
+    B_V = 2,       // prep: a chunk's v tile landed in its slot (TMA; one per chunk, in order)
     B_FULL = 3,    // [2] ring slot filled (prep -> chain)
     B_EMPTY = 5,   // [2] the chain's products have read the slot (MMA commit)
     B_WFREE = 7,   // [2] the slot's W area is free again (output tile stored)
@@ -128,7 +150,9 @@ enum Bars : int {
     B_S = 11,      // chain: state update done
     B_O = 12,      // [2] chain: output products of O buffer 0/1 done
     B_GATE = 14,   // chain: output-gate tile landed (TMA)
-    NBARS = 15
+    B_LA = 15,     // prep: a chunk's log alpha tile landed (TMA; one per chunk)
+    B_KQ = 16,     // prep: a chunk's k (and q) tiles landed in its slot (TMA; one per chunk)
+    NBARS = 17
 };
 
 // TMEM columns (512 allocated).
@@ -160,36 +184,9 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-__device__ __forceinline__ void st8(uint8_t* base, uint32_t off, float a, float b, float c,
-                                    float d) {
-    uint2 v;
-    v.x = pack_bf16(a, b);
-    v.y = pack_bf16(c, d);
-    *reinterpret_cast<uint2*>(base + off) = v;
-}
 
-__device__ __forceinline__ void unpack_bf16x4(const uint2 raw, float (&f)[4]) {
-    const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
-    const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
-    f[0] = __low2float(lo);
-    f[1] = __high2float(lo);
-    f[2] = __low2float(hi);
-    f[3] = __high2float(hi);
-}
 
-// read-only global loads that stay in flight until first use
-__device__ __forceinline__ float4 ld_nc_f4(const float* p) {
-    float4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.f32 {%0,%1,%2,%3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "l"(p));
-    return v;
-}
-__device__ __forceinline__ uint2 ld_nc_u2(const void* p) {
-    uint2 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
-    return v;
-}
+// read-only global load
 __device__ __forceinline__ float ld_nc_f1(const float* p) {
     float v;
     asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(v) : "l"(p));
@@ -343,19 +340,25 @@ __device__ void invert_to_tb(float* As, float* Ts, float* Ys, const float* beta,
             float arow[16], trow[16];
             const int r = o + lane;  // this lane's row of A
             const float br = beta[r];
+            // the row's TMEM loads in 32-column batches, one wait each: rows 0-31 need
+            // columns 0-31; columns j < 32 of rows >= 32 are the cross-half product (TMEM
+            // 64 + j), columns 32-63 of those rows the second half's block
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                const int j0 = 16 * cc;
-                if (warp == 0 && j0 >= 32) break;  // rows 0-31 need columns 0-31 only
-                float v[16];
-                // columns j < 32 of rows >= 32 are the cross-half product (TMEM 64 + j)
-                tmem_ld16(tq + TM_AP + (warp == 1 && j0 < 32 ? 64 + j0 : j0), v);
-                tmem_wait16(v);
+            for (int bb = 0; bb < 2; ++bb) {
+                if (warp == 0 && bb == 1) break;
+                const int j0 = 32 * bb;  // tile columns j0 .. j0+31
+                const uint32_t src = tq + TM_AP + (warp == 1 && bb == 0 ? 64 : j0);
+                float v0[16], v1[16];
+                tmem_ld16(src, v0);
+                tmem_ld16(src + 16, v1);
+                tmem_wait16(v0);
+                tmem_wait16(v1);
 #pragma unroll
-                for (int m = 0; m < 16; ++m) {
-                    const float x = j0 + m < r ? br * v[m] : 0.f;
+                for (int m = 0; m < 32; ++m) {
+                    const float vm = m < 16 ? v0[m] : v1[m - 16];
+                    const float x = j0 + m < r ? br * vm : 0.f;
                     As[r * AS_LD + j0 + m] = x;
-                    if (j0 == ob) arow[m] = x;
+                    if (j0 + (m & ~15) == ob) arow[m & 15] = x;
                 }
             }
             __syncwarp();
@@ -480,195 +483,247 @@ struct Ctx {
 };
 
 // ---------------------------------------------------------------- prep (warps 0-7)
-// Raw inputs of one chunk held by a prep thread: tokens 8w..8w+7 (w = warp),
-// channels 4l..4l+3 (l = lane); beta of token tid on threads 0-63.
-struct Raw {
-    float4 la[8];
-    uint2 k[8];
-    uint2 q[8];
-    float beta;
-};
-
-template <bool Q>
-__device__ __forceinline__ void load_raw(Raw& r, const TcArgs& a, int h, int64_t t0, int64_t t_end,
-                                         int tid) {
-    const int w = tid >> 5, lane = tid & 31, H = a.H;
+__device__ __forceinline__ void unpack_bf16x8(const uint4 raw, float (&f)[8]) {
+    const uint32_t u[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int64_t t = t0 + 8 * w + i;
-        if (t < t_end) {  // warp-uniform
-            const int64_t off = (t * H + h) * D + 4 * lane;
-            r.la[i] = ld_nc_f4(a.log_alpha + off);
-            r.k[i] = ld_nc_u2(reinterpret_cast<const __nv_bfloat16*>(a.k) + off);
-            if (Q) r.q[i] = ld_nc_u2(reinterpret_cast<const __nv_bfloat16*>(a.q) + off);
-        } else {  // rows past the segment end are identity steps
-            r.la[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-            r.k[i] = make_uint2(0u, 0u);
-            if (Q) r.q[i] = make_uint2(0u, 0u);
-        }
-    }
-    if (tid < C) {
-        const int64_t t = t0 + tid;
-        r.beta = t < t_end ? ld_nc_f1(a.beta + t * H + h) : 0.f;
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(u[i] << 16);
+        f[2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u);
     }
 }
+// 8 products a[i] * b[i], bf16, as one 16-byte shared store
+__device__ __forceinline__ void st_prod8(uint32_t addr, const float (&a)[8], const float (&b)[8]) {
+    st_shared_v4(addr, pack_bf16(a[0] * b[0], a[1] * b[1]), pack_bf16(a[2] * b[2], a[3] * b[3]),
+                 pack_bf16(a[4] * b[4], a[5] * b[5]), pack_bf16(a[6] * b[6], a[7] * b[7]));
+}
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
 
+// The prep warps' TMA issues for chunk index cc (tokens t0 = t_begin + 64 cc of head h):
+// its log alpha tile into LA, its k (and q) tiles into its slot's K_dec (and Q~)
+// pieces, its v tile into its slot's W piece, each on its own mbarrier; and the L2
+// prefetch of a later chunk's tiles.
+template <int MODE>
+__device__ __forceinline__ void tma_la(uint8_t* sm, uint64_t* bar, const TcMaps& maps, int h, int t0) {
+    using L = Lay<MODE>;
+    mbar_expect_tx(bar + B_LA, 32768);
+    tma_tile(sm + L::LA, &maps.la, 0, h, t0, bar + B_LA);
+}
+template <int MODE>
+__device__ __forceinline__ void tma_kq(uint8_t* slot, uint64_t* bar, const TcMaps& maps, int h, int t0) {
+    using L = Lay<MODE>;
+    mbar_expect_tx(bar + B_KQ, L::Q ? 32768 : 16384);
+    tma_tile(slot + L::S_KD, &maps.k, 0, h, t0, bar + B_KQ);
+    if (L::Q) tma_tile(slot + L::S_QT, &maps.q, 0, h, t0, bar + B_KQ);
+}
+__device__ __forceinline__ void tma_v(uint8_t* slot, uint64_t* bar, const TcMaps& maps, int h, int t0) {
+    mbar_expect_tx(bar + B_V, 16384);
+    tma_tile(slot, &maps.v, 0, h, t0, bar + B_V);  // the W piece is at offset 0
+    tma_tile(slot + 8192, &maps.v, 64, h, t0, bar + B_V);
+}
+template <bool Q>
+__device__ __forceinline__ void prefetch_chunk(const TcMaps& maps, int h, int t0) {
+    tma_prefetch(&maps.la, 0, h, t0);
+    tma_prefetch(&maps.k, 0, h, t0);
+    if (Q) tma_prefetch(&maps.q, 0, h, t0);
+    tma_prefetch(&maps.v, 0, h, t0);
+    tma_prefetch(&maps.v, 64, h, t0);
+}
+
+// Prep warps: for every chunk of the unit, in order, the chunk-local work into the
+// chunk's ring slot (and U' into the U accumulator).  Thread mapping for the
+// elementwise phases: warp w, lane l = 16 hl + cg holds tokens 8w + 4hl + i (i < 4)
+// and channels 8cg .. 8cg + 7.
 template <int MODE>
 __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int tid) {
     using L = Lay<MODE>;
     constexpr bool Q = L::Q;
     uint8_t* sm = x.sm;
     uint64_t* bar = x.bar;
-    const int w = tid >> 5, lane = tid & 31, h = x.h;
-    const int c0 = 4 * lane;
+    const int w = tid >> 5, lane = tid & 31, h = x.h, H = a.H;
+    const int hl = lane >> 4, cg = lane & 15, c0 = 8 * cg;
     const bool half_b = w >= 4;  // this warp's tokens lie in the chunk's second half
     const uint32_t tq = x.tmem + ((uint32_t)((w & 3) * 32) << 16);
-    float* gsum = reinterpret_cast<float*>(sm + L::GSUM);
     float* beta_s = reinterpret_cast<float*>(sm + L::BETA);
     const int64_t tb = x.sg.t_begin, te = x.sg.t_end;
+    // Shared addresses of this thread's 16-byte piece of each operand image row: every
+    // image stores row r = 8w + 4hl + i, channels c0..c0+7 at base + (r & 7) 128 +
+    // (((c0 / 8) % 8) ^ (r & 7)) 16 (128-byte swizzle); the bases differ by the image's
+    // row count (K-major R rows, or MN-major with K = 64 token rows).
+    const uint32_t blk = (uint32_t)w * 1024u;
+    const uint32_t a_x1 = smem_u32(sm + L::X1) + (uint32_t)(cg >> 3) * 16384u + blk;
+    const uint32_t a_bt = smem_u32(sm + L::BT) + (uint32_t)(cg >> 3) * 12288u + blk;
+    const uint32_t a_kg = smem_u32(sm + L::KG) + (uint32_t)(cg >> 3) * 8192u + blk;
+    const uint32_t a_r64 = (uint32_t)(cg >> 3) * 8192u + blk;  // slot images, 64 rows
+    // this thread's row of the raw [64][128] tiles: token 8w + 4hl + i, channels c0..
+    const uint32_t raw_row0 = (uint32_t)(8 * w + 4 * hl) * 128u + (uint32_t)c0;
 
-    Raw raw;
-    // thread 0: operations in flight (a timeout must wait for them before returning)
-    bool ap_out = false, wu_out = false, v_out = false;
-    uint32_t ap_par = 0, wu_par = 0, v_par = 0;
-    if (x.nc > 0) {
-        load_raw<Q>(raw, a, h, tb, te, tid);
-        if (tid == 0) {
-            v_out = true;
-            v_par = 0;
-            mbar_expect_tx(bar + B_V, 16384);
-            tma_tile(sm + L::V, &maps.v, 0, h, (int)tb, bar + B_V);
-            tma_tile(sm + L::V + 8192, &maps.v, 64, h, (int)tb, bar + B_V);
-        }
-        if (tid == 32 && x.nc > 1) {  // the next chunk's tiles into L2
-            tma_prefetch(&maps.la, 0, h, (int)(tb + C));
-            tma_prefetch(&maps.k, 0, h, (int)(tb + C));
-            if (Q) tma_prefetch(&maps.q, 0, h, (int)(tb + C));
-            tma_prefetch(&maps.v, 0, h, (int)(tb + C));
-            tma_prefetch(&maps.v, 64, h, (int)(tb + C));
-        }
+    // thread 0: TMA loads and products in flight, for the waits after a timeout
+    bool ap_out = false, wu_out = false, v_out = false, la_out = false, kq_out = false;
+    uint32_t ap_par = 0, wu_par = 0, v_par = 0, la_par = 0, kq_par = 0;
+    if (x.nc > 0 && tid == 0) {  // chunk 0's tiles (slot 0 is free)
+        tma_la<MODE>(sm, bar, maps, h, (int)tb);
+        tma_kq<MODE>(sm, bar, maps, h, (int)tb);
+        tma_v(sm, bar, maps, h, (int)tb);
+        la_out = kq_out = v_out = true;
+    }
+    if (tid == 32) {
+        if (x.nc > 1) prefetch_chunk<Q>(maps, h, (int)(tb + C));
+        if (x.nc > 2) prefetch_chunk<Q>(maps, h, (int)(tb + 2 * C));
     }
     bool ok = true;
     for (int64_t c = 0; c < x.nc; ++c) {
         const int64_t t0 = tb + c * C;
+        const int Lc = (int)((te - t0) < C ? (te - t0) : C);
         const int s = (int)(c & 1);
         const uint32_t use = (uint32_t)((c >> 1) & 1);  // phase of this slot use
         uint8_t* slot = sm + s * L::SLOT;
+        float* gsum = reinterpret_cast<float*>(Q ? slot + L::S_PB : sm + L::GSUM);
+        if (tid == 0) TRACE(0, c, 0);
 
-        // ============ gates: in-chunk inclusive cumsum of the clamped log-gates
-        float g[8][4];
+        // ============ raw tiles of this chunk -> registers; gates
+        float g[4][8];
+        uint4 kr[4], qr[4];
         {
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            const bool lok = wait_bar(bar + B_LA, (uint32_t)(c & 1)) &&
+                             wait_bar(bar + B_KQ, (uint32_t)(c & 1));
+            if (lok && tid == 0) la_out = kq_out = false;
+            const float* la_t = reinterpret_cast<const float*>(sm + L::LA);
+            const uint32_t kt = smem_u32(slot + L::S_KD), qt = smem_u32(slot + L::S_QT);
+            float acc[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                acc[0] += clamp_gate(raw.la[i].x);
-                acc[1] += clamp_gate(raw.la[i].y);
-                acc[2] += clamp_gate(raw.la[i].z);
-                acc[3] += clamp_gate(raw.la[i].w);
+            for (int j = 0; j < 8; ++j) acc[j] = 0.f;
 #pragma unroll
-                for (int j = 0; j < 4; ++j) g[i][j] = acc[j];
+            for (int i = 0; i < 4; ++i) {
+                const bool live = 8 * w + 4 * hl + i < Lc;  // rows past the segment end:
+                const uint32_t ro = raw_row0 + (uint32_t)i * 128u;  // identity steps
+                float4 l0 = *reinterpret_cast<const float4*>(la_t + ro);
+                float4 l1 = *reinterpret_cast<const float4*>(la_t + ro + 4);
+                kr[i] = ld_shared_v4(kt + 2u * ro);
+                if (Q) qr[i] = ld_shared_v4(qt + 2u * ro);
+                if (!live) {
+                    l0 = l1 = make_float4(0.f, 0.f, 0.f, 0.f);
+                    kr[i] = make_uint4(0u, 0u, 0u, 0u);
+                    if (Q) qr[i] = make_uint4(0u, 0u, 0u, 0u);
+                }
+                const float la8[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    acc[j] += clamp_gate(la8[j]);
+                    g[i][j] = acc[j];
+                }
             }
-            *reinterpret_cast<float4*>(gsum + w * D + c0) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-            if (tid < C) beta_s[tid] = raw.beta;
+            // the second half-warp's tokens follow the first's: add the partner's total
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float pt = __shfl_xor_sync(0xffffffffu, acc[j], 16);
+                if (hl) {
+                    acc[j] += pt;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) g[i][j] += pt;
+                }
+            }
+            if (hl) {  // the warp's 8-token sums
+                *reinterpret_cast<float4*>(gsum + w * D + c0) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+                *reinterpret_cast<float4*>(gsum + w * D + c0 + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+            }
+            if (tid < C) beta_s[tid] = t0 + tid < te ? ld_nc_f1(a.beta + (t0 + tid) * H + h) : 0.f;
+            // every raw tile has been read: LA may take the next chunk's log alpha
+            if (bar_named_or(BAR_PREP, NPREP, !lok)) {
+                ok = false;
+                break;
+            }
         }
-        // the slot's products of chunk c-2 are done, so Q~, K_dec, P, gamma may be overwritten
-        const bool wok = wait_bar(bar + B_EMPTY + s, use ^ 1u);
-        if (bar_named_or(BAR_PREP, NPREP, !wok)) {
-            ok = false;
-            break;
+        if (tid == 0) {
+            TRACE(0, c, 1);
+            if (c + 1 < x.nc) {
+                tma_la<MODE>(sm, bar, maps, h, (int)(t0 + C));
+                la_out = true;
+                la_par = (uint32_t)((c + 1) & 1);
+            }
         }
+        if (tid == 32 && c + 3 < x.nc) prefetch_chunk<Q>(maps, h, (int)(t0 + 3 * C));
         // per-channel references from the eight warps' sums: rho_a = g_15 (end of warp
         // 1), rho_b = g_47 (end of warp 5), g_last = g_63, and this warp's offset
-        float off[4] = {0.f, 0.f, 0.f, 0.f}, ra[4] = {0.f, 0.f, 0.f, 0.f}, rb[4], gl[4];
+        float rhoL[8], rbL[8], eR[8], dRb[8];
         {
-            float run[4] = {0.f, 0.f, 0.f, 0.f};
+            float run[8], ra[8], rb[8], off[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) run[j] = off[j] = ra[j] = rb[j] = 0.f;
 #pragma unroll
             for (int ww = 0; ww < 8; ++ww) {
-                const float4 t4 = *reinterpret_cast<const float4*>(gsum + ww * D + c0);
-                if (ww == w) {
-                    off[0] = run[0];
-                    off[1] = run[1];
-                    off[2] = run[2];
-                    off[3] = run[3];
+                const float4 t0v = *reinterpret_cast<const float4*>(gsum + ww * D + c0);
+                const float4 t1v = *reinterpret_cast<const float4*>(gsum + ww * D + c0 + 4);
+                const float tv[8] = {t0v.x, t0v.y, t0v.z, t0v.w, t1v.x, t1v.y, t1v.z, t1v.w};
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    if (ww == w) off[j] = run[j];
+                    run[j] += tv[j];
+                    if (ww == 1) ra[j] = run[j];
+                    if (ww == 5) rb[j] = run[j];
                 }
-                run[0] += t4.x;
-                run[1] += t4.y;
-                run[2] += t4.z;
-                run[3] += t4.w;
-                if (ww == 1)
+            }
+            // factors per channel: eR = e^{rho_h} (this warp's half), dRb = e^{g_last - rho_b}
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) ra[j] = run[j];
-                if (ww == 5)
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) rb[j] = run[j];
+            for (int j = 0; j < 8; ++j) {
+                rhoL[j] = (half_b ? rb[j] : ra[j]) * LOG2E;
+                rbL[j] = rb[j] * LOG2E;
+                eR[j] = ex2(rhoL[j]);
+                dRb[j] = ex2((run[j] - rb[j]) * LOG2E);
             }
 #pragma unroll
-            for (int j = 0; j < 4; ++j) gl[j] = run[j];
-        }
-        // factors per channel: eR = e^{rho_h} (this warp's half), dRb = e^{g_last - rho_b}
-        float rhoL[4], rbL[4], eR[4], dRb[4];
+            for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            rhoL[j] = (half_b ? rb[j] : ra[j]) * LOG2E;
-            rbL[j] = rb[j] * LOG2E;
-            eR[j] = ex2(rhoL[j]);
-            dRb[j] = ex2((gl[j] - rb[j]) * LOG2E);
+                for (int j = 0; j < 8; ++j) g[i][j] += off[j];  // inclusive cumsum over the chunk
+            if (w == 0 && hl == 0) {
+                float4* gp = reinterpret_cast<float4*>(slot + L::S_GAM + 4 * c0);
+                gp[0] = make_float4(ex2(run[0] * LOG2E), ex2(run[1] * LOG2E), ex2(run[2] * LOG2E),
+                                    ex2(run[3] * LOG2E));
+                gp[1] = make_float4(ex2(run[4] * LOG2E), ex2(run[5] * LOG2E), ex2(run[6] * LOG2E),
+                                    ex2(run[7] * LOG2E));
+            }
         }
-        if (w == 0)
-            *reinterpret_cast<float4*>(slot + L::S_GAM + 4 * c0) =
-                make_float4(ex2(gl[0] * LOG2E), ex2(gl[1] * LOG2E), ex2(gl[2] * LOG2E), ex2(gl[3] * LOG2E));
 
-        // ============ operand images
+        // ============ operand images (one factor at a time, to keep registers few)
+        {
+            const uint32_t a_slot = smem_u32(slot) + a_r64;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int r = 8 * w + i;
-            float kf[4], qf[4];
-            unpack_bf16x4(raw.k[i], kf);
-            if (Q) unpack_bf16x4(raw.q[i], qf);
-            float e1[4], e2[4], e3[4], kd[4], kg[4];
+            for (int i = 0; i < 4; ++i) {
+                const int rr = 4 * hl + i;  // row within the warp's 8-row swizzle atom
+                const uint32_t ro = (uint32_t)rr * 128u + ((uint32_t)((cg & 7) ^ rr) << 4);
+                float kf[8], f[8], p[8];
+                unpack_bf16x8(kr[i], kf);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float gg = g[i][j] + off[j];
-                const float d2 = fmaf(gg, LOG2E, -rhoL[j]);  // (g - rho_h) log2 e
-                e1[j] = ex2(d2);
-                e2[j] = ex2(-d2);
-                // e^{rho_b - g} for the first half's keys (cross-half block, K_dec)
-                e3[j] = half_b ? 0.f : ex2(fmaf(-gg, LOG2E, rbL[j]));
-                kd[j] = (half_b ? e2[j] : e3[j]) * dRb[j];  // e^{g_last - g}
-                kg[j] = e1[j] * eR[j];                      // e^{g}
+                for (int j = 0; j < 8; ++j) f[j] = ex2(fmaf(g[i][j], LOG2E, -rhoL[j]));  // e^{g-rho_h}
+                st_prod8(a_x1 + ro, kf, f);
+                if (Q) {
+                    unpack_bf16x8(qr[i], p);
+                    st_prod8(a_x1 + 8192u + ro, p, f);
+                }
+#pragma unroll
+                for (int j = 0; j < 8; ++j) f[j] *= eR[j];  // e^{g}
+                st_prod8(a_kg + ro, kf, f);
+                if (Q) st_prod8(a_slot + L::S_QT + ro, p, f);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) f[j] = ex2(fmaf(-g[i][j], LOG2E, rhoL[j]));  // e^{rho_h-g}
+                st_prod8(a_bt + ro, kf, f);
+                if (!half_b) {  // e^{rho_b - g} for the first half's keys (cross-half block)
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) f[j] = ex2(fmaf(-g[i][j], LOG2E, rbL[j]));
+                    st_prod8(a_bt + 8192u + ro, kf, f);
+                }
+#pragma unroll
+                for (int j = 0; j < 8; ++j) f[j] *= dRb[j];  // e^{g_last - g}
+                st_prod8(a_slot + L::S_KD + ro, kf, f);
             }
-            st8(sm + L::X1, kmajor_off(r, c0, 128), kf[0] * e1[0], kf[1] * e1[1], kf[2] * e1[2],
-                kf[3] * e1[3]);
-            st8(sm + L::BT, kmajor_off(r, c0, 96), kf[0] * e2[0], kf[1] * e2[1], kf[2] * e2[2],
-                kf[3] * e2[3]);
-            if (!half_b)
-                st8(sm + L::BT, kmajor_off(64 + r, c0, 96), kf[0] * e3[0], kf[1] * e3[1],
-                    kf[2] * e3[2], kf[3] * e3[3]);
-            st8(sm + L::KG, mnmajor_off(r, c0, 64), kf[0] * kg[0], kf[1] * kg[1], kf[2] * kg[2],
-                kf[3] * kg[3]);
-            st8(slot + L::S_KD, mnmajor_off(r, c0, 64), kf[0] * kd[0], kf[1] * kd[1], kf[2] * kd[2],
-                kf[3] * kd[3]);
-            if (Q) {
-                st8(sm + L::X1, kmajor_off(64 + r, c0, 128), qf[0] * e1[0], qf[1] * e1[1],
-                    qf[2] * e1[2], qf[3] * e1[3]);
-                st8(slot + L::S_QT, kmajor_off(r, c0, 64), qf[0] * kg[0], qf[1] * kg[1],
-                    qf[2] * kg[2], qf[3] * kg[3]);
-            }
-        }
-        // the raw registers are free: the next chunk's inputs start loading now, and the
-        // one after that goes into L2
-        if (c + 1 < x.nc) load_raw<Q>(raw, a, h, t0 + C, te, tid);
-        if (tid == 32 && c + 2 < x.nc) {
-            const int tn = (int)(t0 + 2 * C);
-            tma_prefetch(&maps.la, 0, h, tn);
-            tma_prefetch(&maps.k, 0, h, tn);
-            if (Q) tma_prefetch(&maps.q, 0, h, tn);
-            tma_prefetch(&maps.v, 0, h, tn);
-            tma_prefetch(&maps.v, 64, h, tn);
         }
         fence_async_smem();
         tc_fence_before();
         bar_named(BAR_PREP, NPREP);
+        if (tid == 0) TRACE(0, c, 2);
 
         // ============ [A;P] = X1 . BT^T   (M=128, N=96, K=128)
         if (tid == 0) {
@@ -681,6 +736,13 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
             mma_commit(bar + B_AP);
             ap_out = true;
             ap_par = (uint32_t)(c & 1);
+            // this chunk's v tile into its slot's W piece, once chunk c-2's output tile has
+            // left it (chunk 0's was issued at the start)
+            if (c > 0 && (!Q || wait_bar(bar + B_WFREE + s, use ^ 1u))) {
+                tma_v(slot, bar, maps, h, (int)t0);
+                v_out = true;
+                v_par = (uint32_t)(c & 1);
+            }
         }
         {
             const bool aok = wait_bar(bar + B_AP, (uint32_t)(c & 1));
@@ -691,6 +753,7 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
             }
             tc_fence_after();
         }
+        if (tid == 0) TRACE(0, c, 3);
 
         // ============ A -> (I + A)^-1 -> TB; P into the slot beside the inversion
         {
@@ -706,6 +769,7 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
             });
         }
         fence_async_smem();
+        if (tid == 0) TRACE(0, c, 4);
         {
             // the chain has read U (previous chunk) and this chunk's v tile has landed
             const bool vok = wait_bar(bar + B_V, (uint32_t)(c & 1));
@@ -717,12 +781,13 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
                 break;
             }
         }
+        if (tid == 0) TRACE(0, c, 5);
 
         // ============ W^T = KG^T TB^T ; U'^T = V^T TB^T   (M=128, N=64, K=64)
         if (tid == 0) {
             tc_fence_after();
             const uint32_t kg = smem_u32(sm + L::KG), tbb = smem_u32(sm + L::TB),
-                           vv = smem_u32(sm + L::V);
+                           vv = smem_u32(slot + L::S_W);
             constexpr uint32_t id = idesc_bf16(128, 64, true, false);
 #pragma unroll
             for (int st = 0; st < 4; ++st)
@@ -733,26 +798,28 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
             mma_commit(bar + B_WU);
             wu_out = true;
             wu_par = (uint32_t)(c & 1);
+            // the next chunk's slot, once the chain's products of chunk c-1 have read it:
+            // its k (and q) tiles
+            if (c + 1 < x.nc) {
+                uint8_t* nslot = sm + (s ^ 1) * L::SLOT;
+                const uint32_t nuse = (uint32_t)(((c + 1) >> 1) & 1);
+                if (wait_bar(bar + B_EMPTY + (s ^ 1), nuse ^ 1u)) {
+                    tma_kq<MODE>(nslot, bar, maps, h, (int)(t0 + C));
+                    kq_out = true;
+                    kq_par = (uint32_t)((c + 1) & 1);
+                }
+            }
         }
         {
-            bool wuok = wait_bar(bar + B_WU, (uint32_t)(c & 1));
+            const bool wuok = wait_bar(bar + B_WU, (uint32_t)(c & 1));
             if (wuok && tid == 0) wu_out = false;
-            // the v buffer is consumed: the next chunk's tile
-            if (tid == 0 && wuok && c + 1 < x.nc) {
-                v_out = true;
-                v_par = (uint32_t)((c + 1) & 1);
-                mbar_expect_tx(bar + B_V, 16384);
-                tma_tile(sm + L::V, &maps.v, 0, h, (int)(t0 + C), bar + B_V);
-                tma_tile(sm + L::V + 8192, &maps.v, 64, h, (int)(t0 + C), bar + B_V);
-            }
-            // the slot's W area no longer holds chunk c-2's output tile
-            if (Q) wuok = wuok && wait_bar(bar + B_WFREE + s, use ^ 1u);
             if (bar_named_or(BAR_PREP, NPREP, !wuok)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
         }
+        if (tid == 0) TRACE(0, c, 6);
         // W^T (lane = channel) -> bf16 MN-major image (K rows = channels) in the slot
         {
             const int ch = (w & 3) * 32 + lane, r0 = 32 * (w >> 2);
@@ -772,13 +839,18 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
         fence_async_smem();
         tc_fence_before();
         bar_named(BAR_PREP, NPREP);
-        if (tid == 0) mbar_arrive(bar + B_FULL + s);
+        if (tid == 0) {
+            mbar_arrive(bar + B_FULL + s);
+            TRACE(0, c, 7);
+        }
     }
     // after a timeout: bounded waits for what may still be in flight
     if (!ok && tid == 0) {
         if (ap_out) wait_bar(bar + B_AP, ap_par);
         if (wu_out) wait_bar(bar + B_WU, wu_par);
         if (v_out) wait_bar(bar + B_V, v_par);
+        if (la_out) wait_bar(bar + B_LA, la_par);
+        if (kq_out) wait_bar(bar + B_KQ, kq_par);
     }
 }
 
@@ -787,8 +859,10 @@ __device__ void chain_fwd(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
     using L = Lay<FWD>;
     uint8_t* sm = x.sm;
     uint64_t* bar = x.bar;
-    const int ct = tid - NPREP, cw = ct >> 5, e = ct;  // e: row of S^T = TMEM lane
-    const uint32_t tmem = x.tmem, tq = tmem + ((uint32_t)(cw * 32) << 16);
+    // chain warp cw (0-7): TMEM lane quadrant cw % 4, column half ch = cw / 4; e = row of
+    // S^T (TMEM lane) of this thread
+    const int ct = tid - NPREP, cw = ct >> 5, ch = cw >> 2, e = (cw & 3) * 32 + (ct & 31);
+    const uint32_t tmem = x.tmem, tq = tmem + ((uint32_t)((cw & 3) * 32) << 16);
     const int h = x.h, H = a.H;
     const SegEntry& sg = x.sg;
     const bool snap_on = a.snap_pool != nullptr;
@@ -803,7 +877,7 @@ __device__ void chain_fwd(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
             s0 = a.s0 ? a.s0 + ((int64_t)sg.n * H + h) * D * D : nullptr;
         else
             sin = a.sin + ((int64_t)x.u * H + h) * D * D + (int64_t)e * D;
-        for (int cc = 0; cc < D; cc += 16) {
+        for (int cc = 64 * ch; cc < 64 * ch + 64; cc += 16) {
             float v[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i)
@@ -835,23 +909,34 @@ __device__ void chain_fwd(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
         if (bar_named_or(BAR_CHAIN, NCHAIN, !wok)) return false;
         if (ct == 0 && gate_on) gate_out = false;
         tc_fence_after();
-        float v[4][16];
+        // this thread: tokens r0 .. r0+31 of column e of O^T
+        const int r0 = 32 * ch;
+        float v[2][16];
 #pragma unroll
-        for (int b = 0; b < 4; ++b) tmem_ld16(tq + TM_O + 64 * s + 16 * b, v[b]);
+        for (int b = 0; b < 2; ++b) tmem_ld16(tq + TM_O + 64 * s + r0 + 16 * b, v[b]);
 #pragma unroll
-        for (int b = 0; b < 4; ++b) tmem_wait16(v[b]);
-        __nv_bfloat16* os = reinterpret_cast<__nv_bfloat16*>(sm + s * L::SLOT + L::S_W);
+        for (int b = 0; b < 2; ++b) tmem_wait16(v[b]);
+        uint8_t* os = sm + s * L::SLOT + L::S_W;  // [64][128] bf16 tile (row = token)
+        const uint32_t oa = smem_u32(os) + 2u * (uint32_t)e + (uint32_t)r0 * 256u;
         if (gate_on) {
 #pragma unroll
-            for (int b = 0; b < 4; ++b)
+            for (int b = 0; b < 2; ++b)
 #pragma unroll
-                for (int i = 0; i < 16; ++i) v[b][i] *= __bfloat162float(os[(16 * b + i) * D + e]);
+                for (int i = 0; i < 16; ++i) {
+                    uint16_t gb;
+                    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(gb) : "r"(oa + (uint32_t)(16 * b + i) * 256u));
+                    v[b][i] *= __uint_as_float((uint32_t)gb << 16);
+                }
         }
         if (Lc == C) {
 #pragma unroll
-            for (int b = 0; b < 4; ++b)
+            for (int b = 0; b < 2; ++b)
 #pragma unroll
-                for (int i = 0; i < 16; ++i) os[(16 * b + i) * D + e] = __float2bfloat16_rn(v[b][i]);
+                for (int i = 0; i < 16; ++i) {
+                    const uint16_t ob = __bfloat16_as_ushort(__float2bfloat16_rn(v[b][i]));
+                    asm volatile("st.shared.u16 [%0], %1;" ::"r"(oa + (uint32_t)(16 * b + i) * 256u), "h"(ob)
+                                 : "memory");
+                }
             fence_async_smem();
             bar_named(BAR_CHAIN, NCHAIN);
             if (ct == 32) {
@@ -863,10 +948,11 @@ __device__ void chain_fwd(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
         } else {
             __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out) + (int64_t)h * D + e;
 #pragma unroll
-            for (int b = 0; b < 4; ++b)
+            for (int b = 0; b < 2; ++b)
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
-                    if (16 * b + i < Lc) out[(t0 + 16 * b + i) * H * (int64_t)D] = __float2bfloat16_rn(v[b][i]);
+                    if (r0 + 16 * b + i < Lc)
+                        out[(t0 + r0 + 16 * b + i) * H * (int64_t)D] = __float2bfloat16_rn(v[b][i]);
             bar_named(BAR_CHAIN, NCHAIN);
             if (ct == 32) mbar_arrive(bar + B_WFREE + s);
         }
@@ -877,15 +963,15 @@ __device__ void chain_fwd(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
         const int s = (int)(c & 1);
         uint8_t* slot = sm + s * L::SLOT;
         const int64_t t0 = sg.t_begin + c * C;
+        if (ct == 0) TRACE(1, c, 0);
         bool wok = wait_bar(bar + B_FULL + s, (uint32_t)((c >> 1) & 1));
         if (!s_waited) wok = wok && wait_bar(bar + B_S, (uint32_t)((c - 1) & 1));
         s_waited = true;
         tc_fence_after();
+        if (ct == 0) TRACE(1, c, 1);
         if (wok) {  // bf16 S^T -> SB; S^T *= gamma (per column = key channel) in place
             const float* gam = reinterpret_cast<const float*>(slot + L::S_GAM);
-#pragma unroll 1
-            for (int cb = 0; cb < 4; ++cb)
-                stage_cols_tmem<2>(tq + TM_S + 32 * cb, tq + TM_SB + 16 * cb, 32 * cb, gam, true);
+            stage_cols_tmem<4>(tq + TM_S + 64 * ch, tq + TM_SB + 32 * ch, 64 * ch, gam, true);
             tmem_st_wait();
         }
         tc_fence_before();
@@ -894,6 +980,7 @@ __device__ void chain_fwd(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
             break;
         }
         if (ct == 0) {
+            TRACE(1, c, 2);
             tc_fence_after();
             const uint32_t wb = smem_u32(slot + L::S_W), qt = smem_u32(slot + L::S_QT);
             constexpr uint32_t id_neg = idesc_bf16(128, 64, false, true, true);
@@ -913,12 +1000,14 @@ __device__ void chain_fwd(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
         }
         // meanwhile: the previous chunk's output
         if (c > 0 && !(ok = epilogue(c - 1))) break;
+        if (ct == 0) TRACE(1, c, 3);
         wok = wait_bar(bar + B_U, (uint32_t)(c & 1));
         if (bar_named_or(BAR_CHAIN, NCHAIN, !wok)) {
             ok = false;
             break;
         }
         tc_fence_after();
+        if (ct == 0) TRACE(1, c, 4);
         if (ct == 0) {
             // the W area is read: this chunk's output-gate tile goes there
             if (gate_on) {
@@ -928,13 +1017,13 @@ __device__ void chain_fwd(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
                 tma_tile(slot + L::S_W, &maps.gate, 0, h, (int)t0, bar + B_GATE);
             }
         }
-        // bf16 U^T -> UB
-        stage_cols_tmem<2>(tq + TM_U, tq + TM_UB, 0, nullptr, false);
-        stage_cols_tmem<2>(tq + TM_U + 32, tq + TM_UB + 16, 32, nullptr, false);
+        // bf16 U^T -> UB (this thread: tokens 32 ch .. 32 ch + 31)
+        stage_cols_tmem<2>(tq + TM_U + 32 * ch, tq + TM_UB + 16 * ch, 32 * ch, nullptr, false);
         tmem_st_wait();
         tc_fence_before();
         bar_named(BAR_CHAIN, NCHAIN);
         if (ct == 0) {
+            TRACE(1, c, 5);
             mbar_arrive(bar + B_UFREE);  // the prep may write the next U'
             tc_fence_after();
             const uint32_t kd = smem_u32(slot + L::S_KD), pb = smem_u32(slot + L::S_PB);
@@ -953,6 +1042,7 @@ __device__ void chain_fwd(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
             mma_commit(bar + B_EMPTY + s);
             last_bar = B_EMPTY + s;
             last_par = (uint32_t)((c >> 1) & 1);
+            TRACE(1, c, 6);
         }
         s_waited = false;
         if (snap_on) {  // state snapshot at this chunk end, if one is requested
@@ -971,7 +1061,7 @@ __device__ void chain_fwd(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
                     if (ct == 0) atomicCAS(&g_tc_status, 0, ERR_BAD_SLOT);
                 } else if (slot_id >= 0) {
                     float* sp = a.snap_pool + ((int64_t)slot_id * H + h) * D * D;
-                    for (int cc = 0; cc < D; cc += 16) {
+                    for (int cc = 64 * ch; cc < 64 * ch + 64; cc += 16) {
                         float v[16];
                         tmem_ld16(tq + TM_S + cc, v);
                         tmem_wait16(v);
@@ -995,7 +1085,7 @@ __device__ void chain_fwd(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
     tc_fence_after();
     if (ok && sg.last && a.s_final) {
         float* sf = a.s_final + ((int64_t)sg.n * H + h) * D * D;
-        for (int cc = 0; cc < D; cc += 16) {
+        for (int cc = 64 * ch; cc < 64 * ch + 64; cc += 16) {
             float v[16];
             tmem_ld16(tq + TM_S + cc, v);
             tmem_wait16(v);
@@ -1013,11 +1103,11 @@ __device__ void chain_trans(const Ctx& x, const TcArgs& a, int tid) {
     using L = Lay<TRANS>;
     uint8_t* sm = x.sm;
     uint64_t* bar = x.bar;
-    const int ct = tid - NPREP, cw = ct >> 5, e = ct;
-    const uint32_t tmem = x.tmem, tq = tmem + ((uint32_t)(cw * 32) << 16);
+    const int ct = tid - NPREP, cw = ct >> 5, ch = cw >> 2, e = (cw & 3) * 32 + (ct & 31);
+    const uint32_t tmem = x.tmem, tq = tmem + ((uint32_t)((cw & 3) * 32) << 16);
     const int h = x.h, H = a.H;
     // B^T = 0, M^T = I
-    for (int cc = 0; cc < D; cc += 16) {
+    for (int cc = 64 * ch; cc < 64 * ch + 64; cc += 16) {
         float z[16], m[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
@@ -1041,15 +1131,15 @@ __device__ void chain_trans(const Ctx& x, const TcArgs& a, int tid) {
         uint8_t* slot = sm + s * L::SLOT;
         const uint32_t wb = smem_u32(slot + L::S_W), kd = smem_u32(slot + L::S_KD);
         const float* gam = reinterpret_cast<const float*>(slot + L::S_GAM);
+        if (ct == 0) TRACE(1, c, 0);
         bool wok = wait_bar(bar + B_FULL + s, (uint32_t)((c >> 1) & 1));
         if (c > 0) wok = wok && wait_bar(bar + B_S, (uint32_t)((c - 1) & 1));
         tc_fence_after();
+        if (ct == 0) TRACE(1, c, 1);
         for (int step = 0; step < 2 && ok; ++step) {  // 0: B, 1: M
             const uint32_t tstate = step == 0 ? TT_B : TT_M;
             if (wok) {
-#pragma unroll 1
-                for (int cb = 0; cb < 4; ++cb)
-                    stage_cols_tmem<2>(tq + tstate + 32 * cb, tq + TT_SB + 16 * cb, 32 * cb, gam, true);
+                stage_cols_tmem<4>(tq + tstate + 64 * ch, tq + TT_SB + 32 * ch, 64 * ch, gam, true);
                 tmem_st_wait();
             }
             tc_fence_before();
@@ -1058,6 +1148,7 @@ __device__ void chain_trans(const Ctx& x, const TcArgs& a, int tid) {
                 break;
             }
             if (ct == 0) {
+                TRACE(1, c, 2 + 3 * step);
                 tc_fence_after();
                 // B step: U^T -= B^T W^T on top of U'^T;  M step: U^T = -M^T W^T
 #pragma unroll
@@ -1074,12 +1165,13 @@ __device__ void chain_trans(const Ctx& x, const TcArgs& a, int tid) {
                 break;
             }
             tc_fence_after();
-            stage_cols_tmem<2>(tq + TM_U, tq + TT_UB, 0, nullptr, false);
-            stage_cols_tmem<2>(tq + TM_U + 32, tq + TT_UB + 16, 32, nullptr, false);
+            if (ct == 0) TRACE(1, c, 3 + 3 * step);
+            stage_cols_tmem<2>(tq + TM_U + 32 * ch, tq + TT_UB + 16 * ch, 32 * ch, nullptr, false);
             tmem_st_wait();
             tc_fence_before();
             bar_named(BAR_CHAIN, NCHAIN);
             if (ct == 0) {
+                TRACE(1, c, 4 + 3 * step);
                 if (step == 1) mbar_arrive(bar + B_UFREE);
                 tc_fence_after();
                 // state^T += U^T K_dec
@@ -1105,7 +1197,7 @@ __device__ void chain_trans(const Ctx& x, const TcArgs& a, int tid) {
     if (ok) {  // B^T then M^T of the segment
         float* tp = a.trans + ((int64_t)x.u * H + h) * 2 * D * D + (int64_t)e * D;
         for (int half = 0; half < 2; ++half) {
-            for (int cc = 0; cc < D; cc += 16) {
+            for (int cc = 64 * ch; cc < 64 * ch + 64; cc += 16) {
                 float v[16];
                 tmem_ld16(tq + (half ? TT_M : TT_B) + cc, v);
                 tmem_wait16(v);
@@ -1123,8 +1215,8 @@ __device__ void chain_dump(const Ctx& x, const TcArgs& a, int tid) {
     using L = Lay<DUMP>;
     uint8_t* sm = x.sm;
     uint64_t* bar = x.bar;
-    const int ct = tid - NPREP, cw = ct >> 5, e = ct;
-    const uint32_t tq = x.tmem + ((uint32_t)(cw * 32) << 16);
+    const int ct = tid - NPREP, cw = ct >> 5, ch = cw >> 2, e = (cw & 3) * 32 + (ct & 31);
+    const uint32_t tq = x.tmem + ((uint32_t)((cw & 3) * 32) << 16);
     const int h = x.h, H = a.H;
     for (int64_t c = 0; c < x.nc; ++c) {
         const int s = (int)(c & 1);
@@ -1142,15 +1234,16 @@ __device__ void chain_dump(const Ctx& x, const TcArgs& a, int tid) {
         copy(CI_QT, L::S_QT, 16384);
         copy(CI_PB, L::S_PB, 8192);
         copy(CI_GAM, L::S_GAM, 512);
-        {  // U'^T (row e) -> [128][64] bf16, 16-byte pieces XOR-swizzled by e & 7
-            float v[4][16];
+        {  // U'^T (row e, tokens 32 ch ..) -> [128][64] bf16, 16-byte pieces XOR-swizzled by e & 7
+            float v[2][16];
 #pragma unroll
-            for (int b = 0; b < 4; ++b) tmem_ld16(tq + TM_U + 16 * b, v[b]);
+            for (int b = 0; b < 2; ++b) tmem_ld16(tq + TM_U + 32 * ch + 16 * b, v[b]);
 #pragma unroll
-            for (int b = 0; b < 4; ++b) tmem_wait16(v[b]);
+            for (int b = 0; b < 2; ++b) tmem_wait16(v[b]);
 #pragma unroll
-            for (int p = 0; p < 8; ++p) {
-                const float* q = v[p >> 1] + 8 * (p & 1);
+            for (int pp = 0; pp < 4; ++pp) {
+                const int p = 4 * ch + pp;
+                const float* q = v[pp >> 1] + 8 * (pp & 1);
                 uint4 pk;
                 pk.x = pack_bf16(q[0], q[1]);
                 pk.y = pack_bf16(q[2], q[3]);
@@ -1174,8 +1267,9 @@ template <int MODE>
 __global__ void __launch_bounds__(NT, 1) chunk_kernel(TcArgs a, const __grid_constant__ TcMaps maps) {
     using L = Lay<MODE>;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+    // 1024-byte aligned base, formed by pointer arithmetic on the shared array so that the
+    // compiler keeps every access through it in the shared state space (no generic loads)
+    uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const int tid = threadIdx.x, warp = tid >> 5;
     const int u = blockIdx.x, h = blockIdx.y;
     if (u >= *a.n_units) return;
@@ -1208,8 +1302,15 @@ __global__ void __launch_bounds__(NT, 1) chunk_kernel(TcArgs a, const __grid_con
     x.u = u;
     x.sg = sg;
     x.nc = nc;
+    // Register split: the CTA is launched with 512 x 128 registers; the chain's two
+    // warpgroups give 24 per thread to the prep's two (8 x 32 x (152 + 104) = 65536).
     if (tid < NPREP) {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 152;" ::: "memory");
         prep_loop<MODE>(x, a, maps, tid);
+    } else {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 104;" ::: "memory");
+    }
+    if (tid < NPREP) {
     } else if (MODE == FWD) {
         chain_fwd(x, a, maps, tid);
     } else if (MODE == TRANS) {
@@ -1220,6 +1321,20 @@ __global__ void __launch_bounds__(NT, 1) chunk_kernel(TcArgs a, const __grid_con
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(x.tmem, 512);
+}
+
+// ---------------------------------------------------------------- bounded-wait self-test
+// One thread waits through the kernels' bounded mbarrier wait, with the given limit, on
+// a fresh mbarrier of arrival count 1.  With arrive = 1 it arrives first, so the wait
+// completes at once; otherwise nothing ever arrives, the wait gives up after timeout_ns
+// and records ERR_WAIT_TIMEOUT in the device status word, and the kernel returns.
+__global__ void wait_probe_kernel(uint64_t timeout_ns, int arrive) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x != 0) return;
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    if (arrive) mbar_arrive(&bar);
+    (void)mbar_wait(&bar, 0, &g_tc_status, ERR_WAIT_TIMEOUT, timeout_ns);
 }
 
 // ---------------------------------------------------------------- segment table
@@ -1504,6 +1619,16 @@ cudaError_t status_word(int** p) {
     return cudaSuccess;
 }
 
+#ifdef KDA_PHASE_TRACE
+extern "C" int kda_trace_read(unsigned long long* host, int n) {
+    const int total = 2 * kTraceChunks * kTraceStamps;
+    if (n > total) n = total;
+    if (cudaMemcpyFromSymbol(host, g_trace, (size_t)n * sizeof(unsigned long long)) != cudaSuccess)
+        return -1;
+    return n;
+}
+#endif
+
 cudaError_t tc_take_status(int* code) {
     int zero = 0;
     cudaError_t e = cudaMemcpyFromSymbol(code, g_tc_status, sizeof(int));
@@ -1557,6 +1682,11 @@ cudaError_t launch_transition(const TcArgs& a_in, const TcPlan& p, float* out, c
     c.out = out;
     c.compose = 1;
     return launch_chain(c, stream, launches);
+}
+
+cudaError_t launch_wait_probe(uint64_t timeout_ns, int arrive, cudaStream_t stream) {
+    wait_probe_kernel<<<1, 32, 0, stream>>>(timeout_ns, arrive);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_dump(const TcArgs& a, const TcPlan& p, cudaStream_t stream, int* launches) {

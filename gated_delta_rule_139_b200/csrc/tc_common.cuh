@@ -202,6 +202,19 @@ __device__ __forceinline__ bool mbar_try_wait(void* bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// The same test, but the thread may be suspended (issuing nothing) until the phase
+// completes or about `hint_ns` nanoseconds pass, so waiting warps leave the issue
+// slots to the warps that have work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(void* bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
 __device__ __forceinline__ uint64_t globaltimer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -215,7 +228,7 @@ __device__ __forceinline__ bool mbar_wait(void* bar, uint32_t parity, int* err, 
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (;;) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
         if (globaltimer_ns() - t0 > timeout_ns) {
             if (err) atomicCAS(err, 0, code);
             return false;

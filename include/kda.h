@@ -88,13 +88,11 @@ typedef struct {
  * and a chunk never straddles two sequences.  A zero-length sequence gives
  * final_state[n] = initial_state[n].
  *
- * Temporary device memory (segment table, segment transitions and incoming
- * states for long sequences, and for those also a cache of every chunk's
- * operands of the output pass, which the transition pass prepares: about 290
- * bytes per token and head) is taken stream-ordered (cudaMallocFromPoolAsync /
- * cudaFreeAsync on `stream`) from a memory pool the library creates once per
- * device and keeps for the life of the process; freed blocks stay reserved in
- * that pool for the next call.  Nothing else persists between calls apart from
+ * Temporary device memory (the segment table, and for long sequences the
+ * segment transitions and incoming states: 192 KiB per segment and head) is
+ * taken stream-ordered (cudaMallocFromPoolAsync / cudaFreeAsync on `stream`)
+ * from a memory pool the library creates once per device and keeps for the life
+ * of the process; freed blocks stay reserved in that pool for the next call.  Nothing else persists between calls apart from
  * cached kernel attributes and the device status word (kda_check_device).
  * Errors: see kda_status; a kernel fault surfaces at the caller's next
  * synchronisation, as with any CUDA launch.
@@ -327,24 +325,21 @@ kda_status kda_apply_transitions(const float* trans, int32_t count, int32_t B, i
  * Context-parallel spans with shared work.  A rank that holds one span of B
  * sequences first computes the span's transition (to exchange), then -- once it
  * knows its incoming state -- the span's forward pass.  Both need the same
- * per-segment transitions and per-chunk W, U' (see kda_fwd_ex), so the
- * transition call can leave them in a caller-owned workspace for the forward
- * call, which then runs only the segment scan and the output pass.
+ * per-segment transitions, so the transition call can leave them in a
+ * caller-owned workspace for the forward call, which then runs only the segment
+ * scan and the output pass.
  *
  * kda_span_workspace_bytes: bytes of that workspace for these dims (B, T, H;
  *   d_k = d_v = 128, bf16, no cu_seqlens); 0 for invalid dims.
  * kda_span_transition: kda_transition that also fills `workspace` (device,
  *   256-byte aligned, at least kda_span_workspace_bytes, not overlapping any
- *   argument).  It takes the span's q as well (same layout as k): besides the
- *   segment transitions it leaves every chunk's operands of the output pass
- *   (W, U', the decayed keys, the gated queries, the intra-chunk query-key
- *   matrix and the chunk decay) in the workspace, about 290 bytes per token
- *   and head.
+ *   argument) with the segment table and the segment transitions.  q is not
+ *   used (it may be NULL); it stays in the signature so that both span calls
+ *   take the same tensors.
  * kda_span_forward: kda_fwd on the same span (same k, v, log_alpha, beta and
  *   dims; q, initial_state, out, final_state as in kda_fwd) that takes the
- *   workspace's contents instead of recomputing them.  Where kda_fwd cuts the
- *   span into segments (long spans) it computes the same way, and the results
- *   are equal bit for bit; otherwise they agree within kda_fwd's tolerance.
+ *   workspace's transitions instead of recomputing them.  It computes exactly as
+ *   kda_fwd does on the span, so the results are equal bit for bit.
  *   If the workspace was not filled by kda_span_transition on the same inputs
  *   the results are undefined.  It reads the workspace only, so one transition
  *   may serve several forward calls (e.g. retries).
@@ -369,6 +364,36 @@ kda_status kda_span_forward_ex(const void* q, const void* k, const void* v,
                                const kda_dims* dims, const void* workspace, size_t workspace_bytes,
                                const kda_fwd_opts* opts, void* stream);
 
+/*
+ * kda_chunk_operands -- diagnostic: the chunkwise operands of the forward pass.
+ *
+ * The per-chunk quantities of the chunkwise form (section "Как распараллелили
+ * последовательное обновление" of the page named at the top: all tokens of a chunk
+ * at once, then the state handed on), exactly as the tensor-core forward pass
+ * computes them and hands them to its state products, written out so they can be
+ * checked one by one.  For B sequences of T tokens (q, k, v, log_alpha, beta as in
+ * kda_fwd; bf16, d_k = d_v = 128, no cu_seqlens), chunk c of sequence b and head h
+ * (c < ceil(T/64)) gets entry (b * ceil(T/64) + c) * H + h of `images`, 74 240 bytes
+ * of bf16 operand images in their shared-memory layouts (128-byte swizzle: in a
+ * K-major tile of R rows, element (r, k) sits at byte (k / 64) R 128 + (r / 8) 1024 +
+ * (r % 8) 128 + (((k % 64) / 8) ^ (r % 8)) 16 + (k % 8) 2; an MN-major tile of K rows
+ * is the same with (r, k) -> (k, mn)), with g the in-chunk cumulative clamped
+ * log-gate and T = (I + A)^-1 as in the chunkwise form:
+ *   [0, 16384)       W^T, W = T diag(beta) (K e^g): MN-major, K rows = channels
+ *   [16384, 32768)   U'^T, U' = T diag(beta) V: [128][64], the 16-byte piece p of
+ *                    row e at e 128 + ((p ^ (e % 8)) 16)
+ *   [32768, 49152)   K_dec = K e^(g_last - g): MN-major, K rows = tokens
+ *   [49152, 65536)   Q~ = Q e^g: K-major, 64 rows
+ *   [65536, 73728)   P = lower-inclusive (Q e^g)(K e^-g)^T: K-major 64 x 64
+ *   [73728, 74240)   gamma = e^(g_last), fp32 [128]
+ * Rows past a sequence's end are those of identity steps.  images: device,
+ * 16-byte aligned, B ceil(T/64) H 74240 bytes, not overlapping an input.
+ * Temporary memory as kda_fwd.  Only the operands; no state chain runs.
+ */
+kda_status kda_chunk_operands(const void* q, const void* k, const void* v,
+                              const float* log_alpha, const float* beta, const kda_dims* dims,
+                              void* images, void* stream);
+
 /* Static description of a status code. */
 const char* kda_status_string(kda_status s);
 
@@ -391,6 +416,22 @@ const char* kda_last_path(void);
  * state pool (both KDA_ERR_INVALID_ARG).  KDA_OK when neither happened since the last
  * check. */
 kda_status kda_check_device(void* stream);
+
+/*
+ * kda_selftest_wait -- exercises the failure path of the kernels' bounded waits.
+ *
+ * (No counterpart on the pages; a test aid of this library.)  Every wait of the
+ * tensor-core kernels on an mbarrier (a tensor-core product, a TMA copy, the other
+ * warp group's hand-off) is bounded in wall time; when the bound passes, the
+ * kernel records KDA_ERR_DEVICE_TIMEOUT in the device status word and returns
+ * instead of spinning.  This launches one thread that waits through that same
+ * code on an mbarrier of arrival count 1: with arrive != 0 it arrives first and
+ * the wait completes at once; with arrive == 0 nothing ever arrives, so the wait
+ * gives up after timeout_ns nanoseconds (1e3 .. 1e8, else KDA_ERR_INVALID_ARG)
+ * and the next kda_check_device reports KDA_ERR_DEVICE_TIMEOUT.  Nothing else is
+ * in flight in that kernel, so the context stays usable.  Asynchronous on stream.
+ */
+kda_status kda_selftest_wait(uint64_t timeout_ns, int32_t arrive, void* stream);
 
 /* Optional launch timing (off by default).  While enabled, every kda_fwd and
  * kda_decode call records a CUDA event on its stream before and after each

@@ -8,6 +8,13 @@ import numpy as np
 # the final state.
 TOL_F32_MAX_ABS = 1e-4
 TOL_BF16_REL_FRO = 2e-2
+# bf16 inputs, per (sequence, head, 64-token chunk of the sequence): relative Frobenius
+# error of o over the chunk's tokens x d_v, with the denominator floored at a quarter of
+# the head's RMS over the same number of tokens (so a chunk whose outputs are near zero
+# is judged against the head's scale).  The per-head bound averages over up to 2^20
+# tokens; this one catches a single wrong chunk (a ragged tail, a segment boundary, a
+# clamp-floor channel) that the average would hide.
+TOL_BF16_REL_FRO_CHUNK = 4e-2
 
 
 def to_device(inp, device="cuda"):
@@ -67,3 +74,28 @@ def rel_fro_per_head(o_gpu, o_ref, s_gpu, s_ref, inp, o_tokens=None):
             err = np.linalg.norm(s_gpu[n, h] - s_ref[n, h])
             worst_s = max(worst_s, err / den if den > 0 else err)
     return worst_o, worst_s
+
+
+def rel_fro_per_chunk(o_gpu, o_ref, inp, o_tokens=None, chunk=64):
+    """Worst per-chunk error of o (see TOL_BF16_REL_FRO_CHUNK) and where: (err, (seq, chunk, head))."""
+    H, dv = inp.H, inp.dv
+    og = o_gpu.reshape(-1, H, dv)
+    orf = o_ref.reshape(-1, H, dv)
+    worst, where = 0.0, None
+    for n, (lo, hi) in enumerate(seq_bounds(inp)):
+        if o_tokens is not None:
+            hi = min(hi, o_tokens)
+        if hi <= lo:
+            continue
+        L = hi - lo
+        nc = (L + chunk - 1) // chunk
+        pad = ((0, nc * chunk - L), (0, 0))
+        dd = np.pad(((og[lo:hi] - orf[lo:hi]) ** 2).sum(-1), pad).reshape(nc, chunk, H).sum(1)
+        rr = np.pad((orf[lo:hi] ** 2).sum(-1), pad).reshape(nc, chunk, H).sum(1)
+        cnt = np.minimum(chunk, L - np.arange(nc) * chunk)[:, None]
+        floor = 0.25 ** 2 * rr.sum(0, keepdims=True) / L * cnt
+        e = np.sqrt(dd / np.maximum(np.maximum(rr, floor), 1e-300))
+        i = np.unravel_index(int(np.argmax(e)), e.shape)
+        if e[i] > worst:
+            worst, where = float(e[i]), (n, int(i[0]), int(i[1]))
+    return worst, where
