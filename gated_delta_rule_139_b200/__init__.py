@@ -424,9 +424,9 @@ def span_workspace(k):
 
 
 def kda_span_transition(q, k, v, log_alpha, beta, workspace, out=None, stream=None):
-    """kda_transition that also leaves the span's segment table and segment
-    transitions in ``workspace`` (from :func:`span_workspace`) for
-    :func:`kda_span_forward`.  ``q`` is not used (it may be None)."""
+    """kda_transition that also leaves the span's segment transitions and every
+    chunk's output-pass operands (hence q) in ``workspace`` (from
+    :func:`span_workspace`) for :func:`kda_span_forward`."""
     import torch
     lib = load_library()
     d = _span_dims(k)

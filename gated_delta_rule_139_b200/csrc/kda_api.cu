@@ -213,8 +213,10 @@ kda_status run_tc(const kda::FwdArgs& a, cudaStream_t stream, int* launches) {
     const size_t b_off = ((size_t)(a.N + 1) * 4 + 4 + 255) & ~(size_t)255;
     const size_t b_trans = p.segmented ? (size_t)p.max_units * a.H * 2 * st : 0;
     const size_t b_sin = p.segmented ? (size_t)p.max_units * a.H * st : 0;
+    // chunk cache of the segmented plan: kCacheEntryBytes per chunk and head
+    const size_t b_cache = p.segmented ? (size_t)p.total_chunks * a.H * kda::kCacheEntryBytes : 0;
     char* ws = nullptr;
-    cudaError_t e = pool_alloc((void**)&ws, b_segs + b_off + b_trans + b_sin, stream);
+    cudaError_t e = pool_alloc((void**)&ws, b_segs + b_off + b_trans + b_sin + b_cache, stream);
     if (e != cudaSuccess) return cuda_fail(e, "workspace allocation");
     kda::TcArgs t{};
     t.q = a.q;
@@ -241,6 +243,11 @@ kda_status run_tc(const kda::FwdArgs& a, cudaStream_t stream, int* launches) {
     t.n_units = t.seg_off + a.N + 1;
     t.trans = p.segmented ? (float*)(ws + b_segs + b_off) : nullptr;
     t.sin = p.segmented ? (float*)(ws + b_segs + b_off + b_trans) : nullptr;
+    if (p.segmented) {  // pass 1 runs over every segment and leaves the chunk cache for pass 3
+        t.cache = (uint8_t*)(ws + b_segs + b_off + b_trans + b_sin);
+        t.total_chunks = p.total_chunks;
+        t.trans_all = 1;
+    }
     e = kda::launch_tc(t, p, stream, launches);
     cudaFreeAsync(ws, stream);
     if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
@@ -332,10 +339,10 @@ size_t tc_scratch_bytes(const kda::FwdArgs& a, const kda::TcPlan& p, size_t* b_s
 }
 
 // Workspace of a span (segment table, per-segment transitions and incoming
-// states) for the segment plan of the dims: offsets into one buffer.
+// states, chunk cache) for the segment plan of the dims: offsets into one buffer.
 struct SpanWs {
     kda::TcPlan p;
-    size_t segs, off, trans, sin, total;
+    size_t segs, off, trans, sin, cache, total;
 };
 
 SpanWs span_layout(const kda::FwdArgs& a) {
@@ -352,6 +359,7 @@ SpanWs span_layout(const kda::FwdArgs& a) {
     w.off = take((size_t)(a.N + 1) * 4 + 4);
     w.trans = take((size_t)w.p.max_units * a.H * 2 * st);
     w.sin = take((size_t)w.p.max_units * a.H * st);
+    w.cache = take((size_t)w.p.total_chunks * a.H * kda::kCacheEntryBytes);
     w.total = o;
     return w;
 }
@@ -372,6 +380,8 @@ kda::TcArgs span_args(const kda::FwdArgs& a, const SpanWs& w, char* ws) {
     t.n_units = t.seg_off + a.N + 1;
     t.trans = (float*)(ws + w.trans);
     t.sin = (float*)(ws + w.sin);
+    t.cache = (uint8_t*)(ws + w.cache);
+    t.total_chunks = w.p.total_chunks;
     t.trans_all = 1;
     return t;
 }
@@ -881,15 +891,15 @@ kda_status kda_span_transition(const void* q, const void* k, const void* v, cons
     g_last_launches = 0;
     g_last_path = "";
     kda::FwdArgs a;
-    kda_status st = validate_span_inputs(nullptr, k, v, log_alpha, beta, d, trans, false, &a);
+    kda_status st = validate_span_inputs(q, k, v, log_alpha, beta, d, trans, true, &a);
     if (st != KDA_OK) return st;
-    (void)q;  // not needed: the forward call recomputes every chunk's operands
     const SpanWs w = span_layout(a);
     st = check_workspace(workspace, workspace_bytes, w.total);
     if (st != KDA_OK) return st;
     const int64_t tokens = (int64_t)a.B * a.T, n = tokens * a.H * 128;
     const Range rw = {(uintptr_t)workspace, (uintptr_t)workspace + w.total, "workspace"};
-    const Range other[] = {{(uintptr_t)k, (uintptr_t)k + (k ? n * 2 : 0), "k"},
+    const Range other[] = {{(uintptr_t)q, (uintptr_t)q + (q ? n * 2 : 0), "q"},
+                           {(uintptr_t)k, (uintptr_t)k + (k ? n * 2 : 0), "k"},
                            {(uintptr_t)v, (uintptr_t)v + (v ? n * 2 : 0), "v"},
                            {(uintptr_t)log_alpha, (uintptr_t)log_alpha + (log_alpha ? n * 4 : 0),
                             "log_alpha"},
@@ -898,9 +908,9 @@ kda_status kda_span_transition(const void* q, const void* k, const void* v, cons
                             "trans"}};
     for (const Range& r : other)
         if (overlaps(rw, r)) return fail(KDA_ERR_ALIAS, "workspace overlaps %s", r.name);
-    const void* wp[] = {k, v, log_alpha, beta, trans, workspace};
-    const char* wn[] = {"k", "v", "log_alpha", "beta", "trans", "workspace"};
-    st = check_accessible(wp, wn, 6);
+    const void* wp[] = {q, k, v, log_alpha, beta, trans, workspace};
+    const char* wn[] = {"q", "k", "v", "log_alpha", "beta", "trans", "workspace"};
+    st = check_accessible(wp, wn, 7);
     if (st != KDA_OK) return st;
     kda::TcArgs t = span_args(a, w, (char*)workspace);
     int launches = 0;

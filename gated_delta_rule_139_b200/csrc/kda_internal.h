@@ -78,7 +78,9 @@ struct TcArgs {
     const void* gate = nullptr;  // optional output gate, as in FwdArgs
     int32_t trans_all = 0;       // pass 1 also for each sequence's last segment
     uint8_t* dump = nullptr;     // operand dump: [total_chunks][H][kChunkImageBytes] (launch_dump)
-    int64_t total_chunks = 0;    // chunks the dump holds per head
+    uint8_t* cache = nullptr;    // chunk cache: [total_chunks][H][kCacheEntryBytes] (pass 1 writes,
+                                 // pass 3 reads); nullptr: pass 3 recomputes every chunk's operands
+    int64_t total_chunks = 0;    // chunks the dump / cache holds per head
     // optional state snapshots, as in FwdArgs
     const int32_t* snap_slots = nullptr;
     float* snap_pool = nullptr;
@@ -89,11 +91,16 @@ struct TcArgs {
 // and head): the bf16 images of W^T, U'^T, K_dec, Q~ (16 KB each), P (8 KB) and
 // the fp32 chunk decay gamma (512 B).
 constexpr size_t kChunkImageBytes = 74240;
+// Bytes of one chunk's entry in the chunk cache that pass 1 leaves for pass 3 (per
+// chunk and head): W^T, K_dec, Q~ (16 KB each), P, T diag(beta) (8 KB each), gamma.
+constexpr size_t kCacheEntryBytes = 66048;
 
 // TMA descriptors of the q, k, v, out, gate (bf16) and log_alpha (fp32)
 // tensors, viewed as [T, H, 128]; passed as a grid constant.
 struct TcMaps {
     CUtensorMap q, k, v, la, out, gate;
+    CUtensorMap beta;  // [T][H] fp32, box (4 heads, 64 tokens); only when H % 4 == 0
+    int beta_tma;      // the beta map is set
 };
 
 struct TcPlan {

@@ -90,7 +90,11 @@ constexpr int NT = NPREP + NCHAIN;
 constexpr int BAR_PREP = 1, BAR_CHAIN = 2;  // named barriers of the two groups
 constexpr float LOG2E = 1.4426950408889634f;
 
-enum Mode : int { FWD = 0, TRANS = 1, DUMP = 2 };
+// FWD: forward from the true incoming state, every chunk's operands recomputed.
+// TRANS: segment transitions.  TRANS_CACHE: segment transitions that also leave every
+// chunk's operand images in the chunk cache for cached_kernel.  DUMP: operand images
+// for the test entry point.
+enum Mode : int { FWD = 0, TRANS = 1, DUMP = 2, TRANS_CACHE = 3 };
 
 // ---------------------------------------------------------------- shared memory map
 // Ring slot (two of them; chunk c uses slot c % 2), 1024-byte aligned pieces.  Each
@@ -117,7 +121,7 @@ enum Mode : int { FWD = 0, TRANS = 1, DUMP = 2 };
 //   GSUM  the gate sums when the slot has no P piece (transitions)
 template <int MODE>
 struct Lay {
-    static constexpr bool Q = MODE != TRANS;
+    static constexpr bool Q = MODE != TRANS;  // the prep builds q~ rows, Q~ and P
     static constexpr uint32_t S_W = 0, S_KD = 16384, S_QT = 32768, S_PB = 49152;
     static constexpr uint32_t S_GAM = Q ? 57344 : 32768;
     static constexpr uint32_t SLOT = Q ? 58368 : 33792;
@@ -126,7 +130,8 @@ struct Lay {
     static constexpr uint32_t KG = BT + 24576;
     static constexpr uint32_t LA = KG + 16384;
     static constexpr uint32_t AS = X1, TS = AS + 17408, YS = TS + 18432, TB = YS + 5120;
-    static constexpr uint32_t GSUM = LA + 32768;   // fp32 [8][128] (transitions only)
+    static constexpr uint32_t BTILE = LA + 32768;  // the log alpha tile's beta: fp32 [64][4 heads]
+    static constexpr uint32_t GSUM = BTILE + 1024; // fp32 [8][128] (transitions only)
     static constexpr uint32_t BETA = GSUM + (Q ? 0 : 4096);  // fp32 [64]
     static constexpr uint32_t BAR = BETA + 256;    // mbarriers
     static constexpr uint32_t TMEMP = BAR + 256;   // TMEM base address
@@ -174,6 +179,18 @@ constexpr uint32_t CI_QT = 49152;   // Q~: K-major, 64 rows x 128
 constexpr uint32_t CI_PB = 65536;   // P: K-major, 64 x 64
 constexpr uint32_t CI_GAM = 73728;  // fp32 [128] e^{g_last}
 static_assert(CI_GAM + 512 == kChunkImageBytes, "chunk image");
+
+// Chunk cache entry (kCacheEntryBytes per chunk and head), written by pass 1 with the
+// cache and read by cached_kernel: the bf16 operand images as they sit in shared memory,
+// in 1024-byte aligned pieces (one bulk copy into a 1024-byte aligned buffer keeps their
+// 128-byte swizzle), then gamma.
+constexpr uint32_t CE_W = 0;        // W^T: MN-major, K rows = channels, MN = tokens
+constexpr uint32_t CE_KD = 16384;   // K_dec: MN-major, K rows = tokens
+constexpr uint32_t CE_QT = 32768;   // Q~: K-major, 64 rows
+constexpr uint32_t CE_PB = 49152;   // P: K-major 64 x 64
+constexpr uint32_t CE_TB = 57344;   // T diag(beta): K-major [r][s] 64 x 64
+constexpr uint32_t CE_GAM = 65536;  // fp32 [128] e^{g_last}
+static_assert(CE_GAM + 512 == kCacheEntryBytes, "cache entry");
 
 __device__ __forceinline__ float clamp_gate(float x) { return fminf(fmaxf(x, -5.f), 0.f); }
 // 2^x by the SFU instruction (relative error about 2^-22, flushes results
@@ -259,6 +276,23 @@ __device__ __forceinline__ void tma_store_tile(const CUtensorMap* map, const voi
         "r"(0), "r"(h), "r"(t0), "r"(smem_u32(src))
         : "memory");
 }
+// plain bulk copies: shared -> global (bulk group), global -> shared (mbarrier)
+__device__ __forceinline__ void bulk_store(void* gdst, const void* ssrc, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst),
+                 "r"(smem_u32(ssrc)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_load(void* sdst, const void* gsrc, uint32_t bytes, void* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(sdst)),
+        "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+// all but the most recent of the issuing thread's bulk groups have read shared memory
+__device__ __forceinline__ void bulk_wait_read1() {
+    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
 __device__ __forceinline__ void bulk_commit() {
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
@@ -328,7 +362,8 @@ __device__ __forceinline__ void warp_store16x8(float* dst, int ld, const float (
 // the chunk products as bf16).
 template <typename Side>
 __device__ void invert_to_tb(float* As, float* Ts, float* Ys, const float* beta, uint32_t tbp,
-                             int tid, uint32_t tq, Side side) {
+                             int tid, uint32_t tq, Side side, int64_t chunk) {
+    (void)chunk;  // phase trace only
     const int warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t4 = lane & 3;
     if (warp < 2) {
@@ -362,6 +397,7 @@ __device__ void invert_to_tb(float* As, float* Ts, float* Ys, const float* beta,
                 }
             }
             __syncwarp();
+            if (tid == 0) TRACE(0, chunk, 8);
 #pragma unroll
             for (int m = 0; m < 16; ++m) trow[m] = m == i ? 1.f : 0.f;
 #pragma unroll
@@ -383,6 +419,7 @@ __device__ void invert_to_tb(float* As, float* Ts, float* Ys, const float* beta,
             }
         }
         __syncwarp();
+        if (tid == 0) TRACE(0, chunk, 9);
         // 1b. Y = A_21 T_11 (16 x 16 x 16), then T_21 = -T_22 Y, within the half
         float* Yh = Ys + warp * 16 * YS_LD;
 #pragma unroll
@@ -405,6 +442,7 @@ __device__ void invert_to_tb(float* As, float* Ts, float* Ys, const float* beta,
             warp_store16x8(Ts + (o + 16) * TS_LD + o + 8 * nt, TS_LD, d, -1.f, lane);
         }
         __syncwarp();
+        if (tid == 0) TRACE(0, chunk, 10);
     } else {
         if (warp < 6) {  // zero TB rows 0..31, columns 32..63: 128 chunks
             const int id = tid - 64, r = id >> 2, j8 = 4 + (id & 3);
@@ -413,6 +451,7 @@ __device__ void invert_to_tb(float* As, float* Ts, float* Ys, const float* beta,
         side(warp);
     }
     bar_named(BAR_PREP, NPREP);
+    if (tid == 0) TRACE(0, chunk, 11);
     {  // 2a. TB of the two diagonal halves: 2 x 32 rows x 4 chunks of 8 columns
         const int hf = tid >> 7, r = 32 * hf + ((tid >> 2) & 31), j8 = 4 * hf + (tid & 3);
         const float* tr = Ts + r * TS_LD + 8 * j8;
@@ -432,6 +471,7 @@ __device__ void invert_to_tb(float* As, float* Ts, float* Ys, const float* beta,
         warp_store16x8(Ys + 16 * mt * YS_LD + 8 * nt, YS_LD, d, 1.f, lane);
     }
     bar_named(BAR_PREP, NPREP);
+    if (tid == 0) TRACE(0, chunk, 12);
     // 3. T[32:64, 0:32] = -T_hi Z, scaled by beta_j, straight into TB
     {
         float d[4] = {0.f, 0.f, 0.f, 0.f};
@@ -509,8 +549,14 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
 template <int MODE>
 __device__ __forceinline__ void tma_la(uint8_t* sm, uint64_t* bar, const TcMaps& maps, int h, int t0) {
     using L = Lay<MODE>;
-    mbar_expect_tx(bar + B_LA, 32768);
+    mbar_expect_tx(bar + B_LA, maps.beta_tma ? 32768 + 1024 : 32768);
     tma_tile(sm + L::LA, &maps.la, 0, h, t0, bar + B_LA);
+    if (maps.beta_tma)  // beta of the four heads 4 (h / 4) .. + 3 for the chunk's tokens
+        asm volatile(
+            "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+            " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(sm + L::BTILE)),
+            "l"(reinterpret_cast<uint64_t>(&maps.beta)), "r"(h & ~3), "r"(t0), "r"(smem_u32(bar + B_LA))
+            : "memory");
 }
 template <int MODE>
 __device__ __forceinline__ void tma_kq(uint8_t* slot, uint64_t* bar, const TcMaps& maps, int h, int t0) {
@@ -561,6 +607,12 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
     // this thread's row of the raw [64][128] tiles: token 8w + 4hl + i, channels c0..
     const uint32_t raw_row0 = (uint32_t)(8 * w + 4 * hl) * 128u + (uint32_t)c0;
 
+    // pass 1 with the chunk cache: chunk c's entry (thread 0 bulk-stores TB after the
+    // inversion and the slot's images once the slot is full)
+    constexpr bool CACHE = MODE == TRANS_CACHE;
+    auto cache_entry = [&](int64_t cc) {
+        return a.cache + ((x.sg.c_base + cc) * H + h) * (int64_t)kCacheEntryBytes;
+    };
     // thread 0: TMA loads and products in flight, for the waits after a timeout
     bool ap_out = false, wu_out = false, v_out = false, la_out = false, kq_out = false;
     uint32_t ap_par = 0, wu_par = 0, v_par = 0, la_par = 0, kq_par = 0;
@@ -574,6 +626,9 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
         if (x.nc > 1) prefetch_chunk<Q>(maps, h, (int)(tb + C));
         if (x.nc > 2) prefetch_chunk<Q>(maps, h, (int)(tb + 2 * C));
     }
+    // beta of token tid of the next chunk (threads 0-63): from the tile that arrives with
+    // the log alpha tile, or (heads not a multiple of 4) loaded a chunk ahead
+    float beta_next = (!maps.beta_tma && tid < C && tb + tid < te) ? ld_nc_f1(a.beta + (tb + tid) * H + h) : 0.f;
     bool ok = true;
     for (int64_t c = 0; c < x.nc; ++c) {
         const int64_t t0 = tb + c * C;
@@ -590,7 +645,13 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
         {
             const bool lok = wait_bar(bar + B_LA, (uint32_t)(c & 1)) &&
                              wait_bar(bar + B_KQ, (uint32_t)(c & 1));
-            if (lok && tid == 0) la_out = kq_out = false;
+            if (lok && tid == 0) {
+                la_out = kq_out = false;
+                TRACE(0, c, 14);
+                // the previous chunk's TB store (all but the latest bulk group) has read
+                // X1/BT before this chunk's images go there
+                if (CACHE) bulk_wait_read1();
+            }
             const float* la_t = reinterpret_cast<const float*>(sm + L::LA);
             const uint32_t kt = smem_u32(slot + L::S_KD), qt = smem_u32(slot + L::S_QT);
             float acc[8];
@@ -630,13 +691,42 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
                 *reinterpret_cast<float4*>(gsum + w * D + c0) = make_float4(acc[0], acc[1], acc[2], acc[3]);
                 *reinterpret_cast<float4*>(gsum + w * D + c0 + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
             }
-            if (tid < C) beta_s[tid] = t0 + tid < te ? ld_nc_f1(a.beta + (t0 + tid) * H + h) : 0.f;
+            if (tid < C)
+                beta_s[tid] = maps.beta_tma ? (tid < Lc ? reinterpret_cast<const float*>(sm + L::BTILE)[4 * tid + (h & 3)] : 0.f)
+                                            : beta_next;
             // every raw tile has been read: LA may take the next chunk's log alpha
             if (bar_named_or(BAR_PREP, NPREP, !lok)) {
                 ok = false;
                 break;
             }
         }
+        // thread 0: the next chunk's k (and q) tiles go into the next slot as soon as the
+        // chain's products of chunk c-1 have read it, and this chunk's v tile into this
+        // slot's W piece as soon as chunk c-2's output tile has left it; polled at a few
+        // points of the chunk, waited for at the last one
+        bool kq_next = c + 1 >= x.nc, v_this = c == 0;
+        uint8_t* nslot = sm + (s ^ 1) * L::SLOT;
+        const uint32_t nuse = (uint32_t)(((c + 1) >> 1) & 1);
+        auto poll_tma = [&](bool block_kq, bool block_v) -> bool {
+            if (!kq_next && (block_kq ? wait_bar(bar + B_EMPTY + (s ^ 1), nuse ^ 1u)
+                                      : mbar_try_wait(bar + B_EMPTY + (s ^ 1), nuse ^ 1u))) {
+                if (CACHE) bulk_wait_read();  // chunk c-1's cache stores have read that slot
+                tma_kq<MODE>(nslot, bar, maps, h, (int)(t0 + C));
+                TRACE(0, c + 1, 13);
+                kq_next = kq_out = true;
+                kq_par = (uint32_t)((c + 1) & 1);
+            }
+            // (only the forward chain puts output tiles into the W piece; the dump chain
+            // arrives on B_WFREE anyway, the transition chains never do)
+            if (!v_this && (!(MODE == FWD || MODE == DUMP) ||
+                            (block_v ? wait_bar(bar + B_WFREE + s, use ^ 1u)
+                                     : mbar_try_wait(bar + B_WFREE + s, use ^ 1u)))) {
+                tma_v(slot, bar, maps, h, (int)t0);
+                v_this = v_out = true;
+                v_par = (uint32_t)(c & 1);
+            }
+            return kq_next && v_this;
+        };
         if (tid == 0) {
             TRACE(0, c, 1);
             if (c + 1 < x.nc) {
@@ -644,11 +734,12 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
                 la_out = true;
                 la_par = (uint32_t)((c + 1) & 1);
             }
+            poll_tma(false, false);
         }
         if (tid == 32 && c + 3 < x.nc) prefetch_chunk<Q>(maps, h, (int)(t0 + 3 * C));
         // per-channel references from the eight warps' sums: rho_a = g_15 (end of warp
         // 1), rho_b = g_47 (end of warp 5), g_last = g_63, and this warp's offset
-        float rhoL[8], rbL[8], eR[8], dRb[8];
+        float rhoL[8], sh[8], eR[8], dRb[8];
         {
             float run[8], ra[8], rb[8], off[8];
 #pragma unroll
@@ -666,13 +757,14 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
                     if (ww == 5) rb[j] = run[j];
                 }
             }
-            // factors per channel: eR = e^{rho_h} (this warp's half), dRb = e^{g_last - rho_b}
+            // factors per channel: eR = e^{rho_h} (this warp's half), dRb = e^{g_last - rho_b},
+            // sh = e^{(rho_b - rho_a) / 2} (>= e^-80 since rho_b - rho_a >= -160)
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 rhoL[j] = (half_b ? rb[j] : ra[j]) * LOG2E;
-                rbL[j] = rb[j] * LOG2E;
                 eR[j] = ex2(rhoL[j]);
                 dRb[j] = ex2((run[j] - rb[j]) * LOG2E);
+                sh[j] = ex2((rb[j] - ra[j]) * (0.5f * LOG2E));
             }
 #pragma unroll
             for (int i = 0; i < 4; ++i)
@@ -710,9 +802,12 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
 #pragma unroll
                 for (int j = 0; j < 8; ++j) f[j] = ex2(fmaf(-g[i][j], LOG2E, rhoL[j]));  // e^{rho_h-g}
                 st_prod8(a_bt + ro, kf, f);
-                if (!half_b) {  // e^{rho_b - g} for the first half's keys (cross-half block)
+                if (!half_b) {
+                    // e^{rho_b - g} for the first half's keys (cross-half block) as
+                    // (e^{rho_a - g} sh) sh: an intermediate below the normal range means a
+                    // true value below it, so flushing to zero is the right limit
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) f[j] = ex2(fmaf(-g[i][j], LOG2E, rbL[j]));
+                    for (int j = 0; j < 8; ++j) f[j] = (f[j] * sh[j]) * sh[j];
                     st_prod8(a_bt + 8192u + ro, kf, f);
                 }
 #pragma unroll
@@ -736,14 +831,11 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
             mma_commit(bar + B_AP);
             ap_out = true;
             ap_par = (uint32_t)(c & 1);
-            // this chunk's v tile into its slot's W piece, once chunk c-2's output tile has
-            // left it (chunk 0's was issued at the start)
-            if (c > 0 && (!Q || wait_bar(bar + B_WFREE + s, use ^ 1u))) {
-                tma_v(slot, bar, maps, h, (int)t0);
-                v_out = true;
-                v_par = (uint32_t)(c & 1);
-            }
+            poll_tma(false, false);
         }
+        // the next chunk's beta (without the tile): its load has until the proxy fence after
+        // the inversion
+        if (!maps.beta_tma && tid < C) beta_next = (t0 + C + tid < te) ? ld_nc_f1(a.beta + (t0 + C + tid) * H + h) : 0.f;
         {
             const bool aok = wait_bar(bar + B_AP, (uint32_t)(c & 1));
             if (aok && tid == 0) ap_out = false;
@@ -753,7 +845,10 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
             }
             tc_fence_after();
         }
-        if (tid == 0) TRACE(0, c, 3);
+        if (tid == 0) {
+            TRACE(0, c, 3);
+            poll_tma(false, false);
+        }
 
         // ============ A -> (I + A)^-1 -> TB; P into the slot beside the inversion
         {
@@ -766,10 +861,17 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
                     extract_p16(tq, r, j0, smem_u32(slot + L::S_PB));
                     extract_p16(tq, r, j0 + 16, smem_u32(slot + L::S_PB));
                 }
-            });
+            }, c);
         }
         fence_async_smem();
-        if (tid == 0) TRACE(0, c, 4);
+        if (tid == 0) {
+            TRACE(0, c, 4);
+            poll_tma(false, true);  // v must be on its way before the wait below
+            if (CACHE) {  // the chunk's T diag(beta) into its cache entry
+                bulk_store(cache_entry(c) + CE_TB, sm + L::TB, 8192);
+                bulk_commit();
+            }
+        }
         {
             // the chain has read U (previous chunk) and this chunk's v tile has landed
             const bool vok = wait_bar(bar + B_V, (uint32_t)(c & 1));
@@ -798,17 +900,7 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
             mma_commit(bar + B_WU);
             wu_out = true;
             wu_par = (uint32_t)(c & 1);
-            // the next chunk's slot, once the chain's products of chunk c-1 have read it:
-            // its k (and q) tiles
-            if (c + 1 < x.nc) {
-                uint8_t* nslot = sm + (s ^ 1) * L::SLOT;
-                const uint32_t nuse = (uint32_t)(((c + 1) >> 1) & 1);
-                if (wait_bar(bar + B_EMPTY + (s ^ 1), nuse ^ 1u)) {
-                    tma_kq<MODE>(nslot, bar, maps, h, (int)(t0 + C));
-                    kq_out = true;
-                    kq_par = (uint32_t)((c + 1) & 1);
-                }
-            }
+            poll_tma(true, true);  // the next chunk's k (and q) must be on their way
         }
         {
             const bool wuok = wait_bar(bar + B_WU, (uint32_t)(c & 1));
@@ -842,8 +934,18 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
         if (tid == 0) {
             mbar_arrive(bar + B_FULL + s);
             TRACE(0, c, 7);
+            if (CACHE) {  // the slot's images (read while the chain uses them) into the entry
+                uint8_t* ce = cache_entry(c);
+                bulk_store(ce + CE_W, slot + L::S_W, 16384);
+                bulk_store(ce + CE_KD, slot + L::S_KD, 16384);
+                bulk_store(ce + CE_QT, slot + L::S_QT, 16384);
+                bulk_store(ce + CE_PB, slot + L::S_PB, 8192);
+                bulk_store(ce + CE_GAM, slot + L::S_GAM, 512);
+                bulk_commit();
+            }
         }
     }
+    if (CACHE && tid == 0) bulk_wait_all();  // the cache entries are written
     // after a timeout: bounded waits for what may still be in flight
     if (!ok && tid == 0) {
         if (ap_out) wait_bar(bar + B_AP, ap_par);
@@ -908,6 +1010,7 @@ __device__ void chain_fwd(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
         if (gate_on) wok = wok && wait_bar(bar + B_GATE, (uint32_t)(cc & 1));
         if (bar_named_or(BAR_CHAIN, NCHAIN, !wok)) return false;
         if (ct == 0 && gate_on) gate_out = false;
+        if (ct == 0) TRACE(1, cc + 1, 7);
         tc_fence_after();
         // this thread: tokens r0 .. r0+31 of column e of O^T
         const int r0 = 32 * ch;
@@ -916,6 +1019,7 @@ __device__ void chain_fwd(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
         for (int b = 0; b < 2; ++b) tmem_ld16(tq + TM_O + 64 * s + r0 + 16 * b, v[b]);
 #pragma unroll
         for (int b = 0; b < 2; ++b) tmem_wait16(v[b]);
+        if (ct == 0) TRACE(1, cc + 1, 8);
         uint8_t* os = sm + s * L::SLOT + L::S_W;  // [64][128] bf16 tile (row = token)
         const uint32_t oa = smem_u32(os) + 2u * (uint32_t)e + (uint32_t)r0 * 256u;
         if (gate_on) {
@@ -937,6 +1041,7 @@ __device__ void chain_fwd(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
                     asm volatile("st.shared.u16 [%0], %1;" ::"r"(oa + (uint32_t)(16 * b + i) * 256u), "h"(ob)
                                  : "memory");
                 }
+            if (ct == 0) TRACE(1, cc + 1, 9);
             fence_async_smem();
             bar_named(BAR_CHAIN, NCHAIN);
             if (ct == 32) {
@@ -1099,8 +1204,9 @@ __device__ void chain_fwd(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
 // B from 0 and M from I through the segment's chunks: per chunk the B step
 // (U = U' - B W, B <- gamma B + K_dec^T U) and then the M step (U = -M W,
 // M <- gamma M + K_dec^T U), sharing the U, SB and UB columns.
+template <int MODE>
 __device__ void chain_trans(const Ctx& x, const TcArgs& a, int tid) {
-    using L = Lay<TRANS>;
+    using L = Lay<MODE>;
     uint8_t* sm = x.sm;
     uint64_t* bar = x.bar;
     const int ct = tid - NPREP, cw = ct >> 5, ch = cw >> 2, e = (cw & 3) * 32 + (ct & 31);
@@ -1275,9 +1381,9 @@ __global__ void __launch_bounds__(NT, 1) chunk_kernel(TcArgs a, const __grid_con
     if (u >= *a.n_units) return;
     const SegEntry sg = a.segs[u];
     // transitions only for segments with a successor, unless all are asked for
-    if (MODE == TRANS && sg.last && !a.trans_all) return;
+    if ((MODE == TRANS || MODE == TRANS_CACHE) && sg.last && !a.trans_all) return;
     const int64_t nc = sg.t_end > sg.t_begin ? (sg.t_end - sg.t_begin + C - 1) / C : 0;
-    if (MODE == DUMP && (sg.c_base < 0 || sg.c_base + nc > a.total_chunks)) {
+    if ((MODE == DUMP || MODE == TRANS_CACHE) && (sg.c_base < 0 || sg.c_base + nc > a.total_chunks)) {
         if (tid == 0) atomicCAS(&g_tc_status, 0, ERR_SEG_OVERFLOW);  // malformed cu_seqlens
         return;
     }
@@ -1313,14 +1419,294 @@ __global__ void __launch_bounds__(NT, 1) chunk_kernel(TcArgs a, const __grid_con
     if (tid < NPREP) {
     } else if (MODE == FWD) {
         chain_fwd(x, a, maps, tid);
-    } else if (MODE == TRANS) {
-        chain_trans(x, a, tid);
+    } else if (MODE == TRANS || MODE == TRANS_CACHE) {
+        chain_trans<MODE>(x, a, tid);
     } else {
         chain_dump(x, a, tid);
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(x.tmem, 512);
+}
+
+// ---------------------------------------------------------------- pass 3 from the chunk cache
+// Shared memory: two chunk images (the cache entry as pass 1 wrote it, 1024-byte
+// aligned) with their v tiles, the output tile and the output gate's tile.
+struct LayC {
+    static constexpr uint32_t IMG_STRIDE = 66560;          // kCacheEntryBytes rounded to 1 KB
+    static constexpr uint32_t V = 2 * IMG_STRIDE;          // [2] v tiles (two 64-channel boxes)
+    static constexpr uint32_t OUT = V + 2 * 16384;         // bf16 [64][128]
+    static constexpr uint32_t GATE = OUT + 16384;          // bf16 [64][128]
+    static constexpr uint32_t BAR = GATE + 16384;          // mbarriers: MMA, image 0, image 1, gate
+    static constexpr uint32_t TMEMP = BAR + 32;
+    static constexpr uint32_t BYTES = TMEMP + 16 + 1024;   // + alignment slack
+};
+static_assert(LayC::IMG_STRIDE >= kCacheEntryBytes && LayC::IMG_STRIDE % 1024 == 0, "image stride");
+static_assert(LayC::BYTES <= 232448, "shared memory");
+
+// Per (segment, head): the state chain from the true incoming state and the output, every
+// chunk's operands taken from the chunk cache (image and v tile loaded two chunks ahead):
+//   bf16 S^T -> TMEM, S^T *= gamma                                      (all threads)
+//   U^T = V^T TB^T ;  U^T -= S^T W^T ;  O^T = S^T Q~^T                 (one thread)
+//   bf16 U^T -> TMEM                                                   (all threads)
+//   O^T += U^T P^T ;  S^T += U^T K_dec                                 (one thread)
+//   O^T (x gate) -> bf16 tile -> TMA store                             (all threads)
+// Sixteen warps: lane quadrant warp % 4, column slice warp / 4.  The same products in
+// the same precision as chunk_kernel<FWD>: the two differ only in where W, TB, Q~, K_dec,
+// P and gamma come from.
+__global__ void __launch_bounds__(NT, 1) cached_kernel(TcArgs a, const __grid_constant__ TcMaps maps) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int u = blockIdx.x, h = blockIdx.y, H = a.H;
+    if (u >= *a.n_units) return;
+    const SegEntry sg = a.segs[u];
+    const bool snap_on = a.snap_pool != nullptr;
+    const bool gate_on = a.gate != nullptr;
+    const int64_t seq_lo = snap_on ? (a.cu ? (int64_t)a.cu[sg.n] : (int64_t)sg.n * a.T) : 0;
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + LayC::BAR);  // MMA completion
+    uint64_t* bar_img = bar + 1;                                  // [2] image and v loads
+    uint64_t* bar_gate = bar + 3;                                 // output-gate tile
+    uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(sm + LayC::TMEMP);
+    if (sg.c_base < 0 || sg.c_base + (sg.t_end - sg.t_begin + C - 1) / C > a.total_chunks) {
+        if (tid == 0) atomicCAS(&g_tc_status, 0, ERR_SEG_OVERFLOW);  // malformed cu_seqlens
+        return;
+    }
+    auto entry = [&](int64_t tt) {  // the chunk cache entry of the chunk at tt, head h
+        return a.cache + ((sg.c_base + (tt - sg.t_begin) / C) * H + h) * (int64_t)kCacheEntryBytes;
+    };
+    uint32_t pending = 0;  // thread 0: bit b = a load into image b in flight; bit 2 = gate tile
+    auto load_img = [&](int64_t tt, int b) {
+        pending |= 1u << b;
+        mbar_expect_tx(bar_img + b, (uint32_t)kCacheEntryBytes + 16384u);
+        bulk_load(sm + b * LayC::IMG_STRIDE, entry(tt), (uint32_t)kCacheEntryBytes, bar_img + b);
+        uint8_t* vb = sm + LayC::V + b * 16384;
+        tma_tile(vb, &maps.v, 0, h, (int)tt, bar_img + b);
+        tma_tile(vb + 8192, &maps.v, 64, h, (int)tt, bar_img + b);
+    };
+    auto load_gate = [&](int64_t tt) {
+        pending |= 4u;
+        mbar_expect_tx(bar_gate, 16384);
+        tma_tile(sm + LayC::GATE, &maps.gate, 0, h, (int)tt, bar_gate);
+    };
+
+    if (warp == 0) {
+        tmem_alloc(tmem_ptr, 512);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        mbar_init(bar_img, 1);
+        mbar_init(bar_img + 1, 1);
+        mbar_init(bar_gate, 1);
+        fence_mbar_init();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_ptr;
+    const int quad = warp & 3, wg = warp >> 2, lrow = quad * 32 + lane;
+    const uint32_t tq = tmem + ((uint32_t)(quad * 32) << 16);
+    if (tid == 0 && sg.t_begin < sg.t_end) {  // the first two chunks' images
+        load_img(sg.t_begin, 0);
+        if (sg.t_begin + C < sg.t_end) load_img(sg.t_begin + C, 1);
+        if (gate_on) load_gate(sg.t_begin);
+    }
+    // initial state: slice wg writes columns 32wg..32wg+31 of S^T
+    {
+        const int e = lrow, cb = 32 * wg;
+        for (int c0 = cb; c0 < cb + 32; c0 += 16) {
+            float v[16];
+            if (sg.j == 0 && sg.last) {  // single segment: the caller's state
+                const float* s0 = a.s0 ? a.s0 + ((int64_t)sg.n * H + h) * D * D : nullptr;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[i] = s0 ? s0[(int64_t)(c0 + i) * D + e] : 0.f;
+            } else {
+                const float* sin = a.sin + ((int64_t)u * H + h) * D * D + (int64_t)e * D;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[i] = sin[c0 + i];
+            }
+            tmem_st16(tq + TM_S + c0, v);
+        }
+    }
+    tmem_st_wait();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    uint32_t parity = 0, img_parity = 0, gate_parity = 0;  // img_parity: bit b for image b
+    bool mma_out = false;  // thread 0: a commit not yet waited for, on phase mma_par
+    uint32_t mma_par = 0;
+    // O^T of the chunk at tt (Lcc tokens) from the O accumulator at tm_o -> out: a full chunk
+    // as one [64][128] bf16 tile by TMA, a partial last chunk row by row from registers; with
+    // an output gate, each element gated first (then the next chunk's gate tile is loaded).
+    // Called by all threads; false if a wait gave up.
+    auto emit = [&](int64_t tt, int Lcc, uint32_t tm_o) -> bool {
+        const int r0 = 16 * wg;
+        float v[16];
+        tmem_ld16(tq + tm_o + r0, v);
+        tmem_wait16(v);
+        __nv_bfloat16* os = reinterpret_cast<__nv_bfloat16*>(sm + LayC::OUT);
+        if (gate_on) {
+            const __nv_bfloat16* gs = reinterpret_cast<const __nv_bfloat16*>(sm + LayC::GATE);
+            if (__syncthreads_or(!mbar_wait(bar_gate, gate_parity, &g_tc_status, ERR_WAIT_TIMEOUT)))
+                return false;
+            gate_parity ^= 1u;
+            pending &= ~4u;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] *= __bfloat162float(gs[(r0 + i) * D + lrow]);
+        }
+        if (Lcc == C) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) os[(r0 + i) * D + lrow] = __float2bfloat16_rn(v[i]);
+            fence_async_smem();
+            __syncthreads();
+            if (tid == 0) {
+                tma_store_tile(&maps.out, sm + LayC::OUT, h, (int)tt);
+                bulk_commit();
+                if (gate_on && tt + C < sg.t_end) load_gate(tt + C);  // GATE has been read
+            }
+        } else {
+            __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out) + (int64_t)h * D + lrow;
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                if (r0 + i < Lcc) out[(tt + r0 + i) * H * (int64_t)D] = __float2bfloat16_rn(v[i]);
+        }
+        return true;
+    };
+    // block-wide bounded wait on the MMA barrier; false (uniformly) if any thread gave up
+    auto wait_mma = [&]() -> bool {
+        const bool okw = mbar_wait(bar, parity, &g_tc_status, ERR_WAIT_TIMEOUT);
+        parity ^= 1u;
+        tc_fence_after();
+        return !__syncthreads_or(!okw);
+    };
+    bool ok = true;
+    int b = 0;
+    int64_t last_t0 = sg.t_begin;  // the chunk whose output is still in TMEM
+    int last_Lc = 0;
+    uint32_t last_o = TM_O;
+    for (int64_t t0 = sg.t_begin; t0 < sg.t_end && ok; t0 += C, b ^= 1) {
+        const int Lc = (int)((sg.t_end - t0) < C ? (sg.t_end - t0) : C);
+        uint8_t* img = sm + b * LayC::IMG_STRIDE;
+        // O accumulators alternate between chunks, so a chunk's output leaves TMEM while
+        // the next chunk's first products run
+        const uint32_t tm_o = TM_O + 64u * (uint32_t)(((t0 - sg.t_begin) / C) & 1);
+        if (!(ok = !__syncthreads_or(!mbar_wait(bar_img + b, (img_parity >> b) & 1u, &g_tc_status,
+                                                ERR_WAIT_TIMEOUT)))) break;
+        img_parity ^= 1u << b;
+        pending &= ~(1u << b);
+        // bf16 S^T into TMEM (A operand), S^T *= gamma in place
+        {
+            const float* gam = reinterpret_cast<const float*>(img + CE_GAM);
+            const int c0 = 32 * wg;
+            stage_cols_tmem<2>(tq + TM_S + c0, tq + TM_SB + c0 / 2, c0, gam, true);
+            tmem_st_wait();
+        }
+        tc_fence_before();
+        __syncthreads();
+        // U^T = V^T TB^T ;  U^T -= S^T W^T ;  O^T = S^T Q~^T
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t wb = smem_u32(img + CE_W), qt = smem_u32(img + CE_QT),
+                           tb = smem_u32(img + CE_TB), vv = smem_u32(sm + LayC::V + b * 16384);
+            constexpr uint32_t id_uv = idesc_bf16(128, 64, true, false);
+            constexpr uint32_t id_neg = idesc_bf16(128, 64, false, true, true);
+            constexpr uint32_t id = idesc_bf16(128, 64, false, false);
+#pragma unroll
+            for (int st = 0; st < 4; ++st)
+                mma_bf16(tmem + TM_U, mnmajor_desc(vv, 64, st), kmajor_desc(tb, 64, st), id_uv, st > 0);
+#pragma unroll
+            for (int st = 0; st < 8; ++st)
+                mma_bf16_ts(tmem + TM_U, tmem + TM_SB + 8 * st, mnmajor_desc(wb, 128, st), id_neg, 1);
+#pragma unroll
+            for (int st = 0; st < 8; ++st)
+                mma_bf16_ts(tmem + tm_o, tmem + TM_SB + 8 * st, kmajor_desc(qt, 64, st), id, st > 0);
+            mma_commit(bar);
+            mma_out = true;
+            mma_par = parity;
+        }
+        // meanwhile: the previous chunk's output (a full chunk: only a segment's last is partial)
+        if (t0 > sg.t_begin && !(ok = emit(t0 - C, C, last_o))) break;
+        if (!(ok = wait_mma())) break;
+        mma_out = false;
+        // bf16 U^T into TMEM; the last output store has left OUT by the next barrier
+        {
+            const int c0 = 16 * wg;
+            stage_cols_tmem<1>(tq + TM_U + c0, tq + TM_UB + c0 / 2, c0, nullptr, false);
+            tmem_st_wait();
+        }
+        if (tid == 0) bulk_wait_read();
+        tc_fence_before();
+        __syncthreads();
+        // O^T += U^T P^T ; S^T += U^T K_dec
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t pb = smem_u32(img + CE_PB), kd = smem_u32(img + CE_KD);
+            constexpr uint32_t id = idesc_bf16(128, 64, false, false);
+            constexpr uint32_t id_s = idesc_bf16(128, 128, false, true);
+#pragma unroll
+            for (int st = 0; st < 4; ++st)
+                mma_bf16_ts(tmem + tm_o, tmem + TM_UB + 8 * st, kmajor_desc(pb, 64, st), id, 1);
+#pragma unroll
+            for (int st = 0; st < 4; ++st)
+                mma_bf16_ts(tmem + TM_S, tmem + TM_UB + 8 * st, mnmajor_desc(kd, 64, st), id_s, 1);
+            mma_commit(bar);
+            mma_out = true;
+            mma_par = parity;
+        }
+        if (!(ok = wait_mma())) break;
+        mma_out = false;
+        // this image (and v tile) is consumed: the chunk after next may load into it
+        if (tid == 0 && t0 + 2 * C < sg.t_end) load_img(t0 + 2 * C, b);
+        last_t0 = t0;
+        last_Lc = Lc;
+        last_o = tm_o;
+        if (snap_on) {  // state snapshot at this chunk end, if one is requested
+            const int64_t pos = t0 + Lc - seq_lo;
+            if (pos % a.snap_interval == 0 && pos / a.snap_interval <= a.snap_max) {
+                const int slot = a.snap_slots[(int64_t)sg.n * a.snap_max + pos / a.snap_interval - 1];
+                if (slot >= a.snap_num_slots) {
+                    if (tid == 0) atomicCAS(&g_tc_status, 0, ERR_BAD_SLOT);
+                } else if (slot >= 0) {  // slice wg: columns 32wg..32wg+31 of S^T
+                    float* sp = a.snap_pool + ((int64_t)slot * H + h) * D * D;
+                    for (int c0 = 32 * wg; c0 < 32 * wg + 32; c0 += 16) {
+                        float v[16];
+                        tmem_ld16(tq + TM_S + c0, v);
+                        tmem_wait16(v);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) sp[(int64_t)(c0 + i) * D + lrow] = v[i];
+                    }
+                }
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    }
+
+    if (ok && last_Lc > 0) ok = emit(last_t0, last_Lc, last_o);  // the last chunk's output
+    if (!ok && tid == 0) {  // after a timeout: bounded waits for what may still be in flight
+        if (mma_out) mbar_wait(bar, mma_par, &g_tc_status, ERR_WAIT_TIMEOUT);
+        for (int bb = 0; bb < 2; ++bb)
+            if (pending & (1u << bb))
+                mbar_wait(bar_img + bb, (img_parity >> bb) & 1u, &g_tc_status, ERR_WAIT_TIMEOUT);
+        if (pending & 4u) mbar_wait(bar_gate, gate_parity, &g_tc_status, ERR_WAIT_TIMEOUT);
+    }
+    if (tid == 0) bulk_wait_all();  // output stores are complete
+    if (ok && sg.last && a.s_final) {  // slice wg: columns 32wg..32wg+31 of S^T
+        float* sf = a.s_final + ((int64_t)sg.n * H + h) * D * D;
+        for (int c0 = 32 * wg; c0 < 32 * wg + 32; c0 += 16) {
+            float v[16];
+            tmem_ld16(tq + TM_S + c0, v);
+            tmem_wait16(v);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) sf[(int64_t)(c0 + i) * D + lrow] = v[i];
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
 // ---------------------------------------------------------------- bounded-wait self-test
@@ -1551,6 +1937,19 @@ cudaError_t make_maps(const TcArgs& a, TcMaps* maps) {
         (err = tile_map(&maps->v, a.v, false, a.H, tokens, true)) != cudaSuccess ||
         (err = tile_map(&maps->la, a.log_alpha, true, a.H, tokens, false)) != cudaSuccess)
         return err;
+    if (a.H % 4 == 0) {  // beta as [T][H] fp32, box (4 heads, 64 tokens)
+        EncodeTiledFn fn = encode_tiled();
+        if (!fn) return cudaErrorNotSupported;
+        const cuuint64_t dims[2] = {(cuuint64_t)a.H, (cuuint64_t)tokens};
+        const cuuint64_t strides[1] = {(cuuint64_t)a.H * 4};
+        const cuuint32_t box[2] = {4, (cuuint32_t)C};
+        const cuuint32_t estr[2] = {1, 1};
+        if (fn(&maps->beta, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(a.beta), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+        maps->beta_tma = 1;
+    }
     if (a.q && (err = tile_map(&maps->q, a.q, false, a.H, tokens, false)) != cudaSuccess) return err;
     if (a.out && (err = tile_map(&maps->out, a.out, false, a.H, tokens, false)) != cudaSuccess)
         return err;
@@ -1574,6 +1973,10 @@ cudaError_t set_attributes() {
                                     (int)Lay<TRANS>::BYTES)) != cudaSuccess ||
         (err = cudaFuncSetAttribute(chunk_kernel<DUMP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)Lay<DUMP>::BYTES)) != cudaSuccess ||
+        (err = cudaFuncSetAttribute(chunk_kernel<TRANS_CACHE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)Lay<TRANS_CACHE>::BYTES)) != cudaSuccess ||
+        (err = cudaFuncSetAttribute(cached_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)LayC::BYTES)) != cudaSuccess ||
         (err = cudaFuncSetAttribute(seg_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     SCAN_SMEM)) != cudaSuccess)
         return err;
@@ -1593,8 +1996,11 @@ cudaError_t launch_setup(const TcArgs& a, const TcPlan& p, cudaStream_t stream, 
 cudaError_t launch_pass1(const TcArgs& a, const TcPlan& p, const TcMaps& maps, cudaStream_t stream,
                          int* launches) {
     profile_mark(SLOT_PASS1, true, stream);
-    chunk_kernel<TRANS><<<dim3((unsigned)p.max_units, (unsigned)a.H), NT, Lay<TRANS>::BYTES, stream>>>(
-        a, maps);
+    const dim3 grid((unsigned)p.max_units, (unsigned)a.H);
+    if (a.cache)
+        chunk_kernel<TRANS_CACHE><<<grid, NT, Lay<TRANS_CACHE>::BYTES, stream>>>(a, maps);
+    else
+        chunk_kernel<TRANS><<<grid, NT, Lay<TRANS>::BYTES, stream>>>(a, maps);
     profile_mark(SLOT_PASS1, false, stream);
     *launches += 1;
     return cudaGetLastError();
@@ -1654,7 +2060,11 @@ cudaError_t launch_tc(const TcArgs& a, const TcPlan& p, cudaStream_t stream, int
         if ((err = cudaGetLastError()) != cudaSuccess) return err;
     }
     profile_mark(SLOT_PASS3, true, stream);
-    chunk_kernel<FWD><<<dim3((unsigned)p.max_units, (unsigned)a.H), NT, Lay<FWD>::BYTES, stream>>>(a, maps);
+    const dim3 grid((unsigned)p.max_units, (unsigned)a.H);
+    if (p.segmented && a.cache)
+        cached_kernel<<<grid, NT, LayC::BYTES, stream>>>(a, maps);
+    else
+        chunk_kernel<FWD><<<grid, NT, Lay<FWD>::BYTES, stream>>>(a, maps);
     profile_mark(SLOT_PASS3, false, stream);
     *launches += 1;
     return cudaGetLastError();

@@ -89,10 +89,12 @@ typedef struct {
  * final_state[n] = initial_state[n].
  *
  * Temporary device memory (the segment table, and for long sequences the
- * segment transitions and incoming states: 192 KiB per segment and head) is
- * taken stream-ordered (cudaMallocFromPoolAsync / cudaFreeAsync on `stream`)
- * from a memory pool the library creates once per device and keeps for the life
- * of the process; freed blocks stay reserved in that pool for the next call.  Nothing else persists between calls apart from
+ * segment transitions and incoming states, 192 KiB per segment and head, and a
+ * cache of every chunk's operands of the output pass, which the transition pass
+ * prepares: about 1030 bytes per token and head) is taken stream-ordered
+ * (cudaMallocFromPoolAsync / cudaFreeAsync on `stream`) from a memory pool the
+ * library creates once per device and keeps for the life of the process; freed
+ * blocks stay reserved in that pool for the next call.  Nothing else persists between calls apart from
  * cached kernel attributes and the device status word (kda_check_device).
  * Errors: see kda_status; a kernel fault surfaces at the caller's next
  * synchronisation, as with any CUDA launch.
@@ -325,20 +327,22 @@ kda_status kda_apply_transitions(const float* trans, int32_t count, int32_t B, i
  * Context-parallel spans with shared work.  A rank that holds one span of B
  * sequences first computes the span's transition (to exchange), then -- once it
  * knows its incoming state -- the span's forward pass.  Both need the same
- * per-segment transitions, so the transition call can leave them in a
- * caller-owned workspace for the forward call, which then runs only the segment
- * scan and the output pass.
+ * per-segment transitions and per-chunk operands, so the transition call can
+ * leave them in a caller-owned workspace for the forward call, which then runs
+ * only the segment scan and the output pass.
  *
  * kda_span_workspace_bytes: bytes of that workspace for these dims (B, T, H;
  *   d_k = d_v = 128, bf16, no cu_seqlens); 0 for invalid dims.
  * kda_span_transition: kda_transition that also fills `workspace` (device,
  *   256-byte aligned, at least kda_span_workspace_bytes, not overlapping any
- *   argument) with the segment table and the segment transitions.  q is not
- *   used (it may be NULL); it stays in the signature so that both span calls
- *   take the same tensors.
+ *   argument) with the segment table, the segment transitions and, for a span
+ *   cut into segments, every chunk's operands of the output pass (W, the decayed
+ *   keys, the gated queries, the intra-chunk query-key matrix, T diag(beta) and
+ *   the chunk decay: about 1030 bytes per token and head).  It takes the span's q
+ *   as well (same layout as k).
  * kda_span_forward: kda_fwd on the same span (same k, v, log_alpha, beta and
  *   dims; q, initial_state, out, final_state as in kda_fwd) that takes the
- *   workspace's transitions instead of recomputing them.  It computes exactly as
+ *   workspace's contents instead of recomputing them.  It computes exactly as
  *   kda_fwd does on the span, so the results are equal bit for bit.
  *   If the workspace was not filled by kda_span_transition on the same inputs
  *   the results are undefined.  It reads the workspace only, so one transition

@@ -243,6 +243,10 @@ def test_span_workspace_size_and_bad_arguments():
                                      P(ws), nbytes, P(FAKE + (4 << 30)), None)
         return kda.STATUS[rc]
 
+    assert trans_call(q=None) == "KDA_ERR_INVALID_ARG"  # the workspace needs q
+    assert trans_call(q=FAKE + (9 << 30) + 8) == "KDA_ERR_MISALIGNED"
+    assert trans_call(ws=FAKE + (9 << 30)) == "KDA_ERR_ALIAS"  # workspace over q
+
     assert trans_call(ws=None) == "KDA_ERR_INVALID_ARG"
     assert trans_call(ws=FAKE + (8 << 30) + 16) == "KDA_ERR_MISALIGNED"
     assert trans_call(nbytes=n - 256) == "KDA_ERR_INVALID_ARG"
