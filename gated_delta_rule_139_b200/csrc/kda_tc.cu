@@ -64,19 +64,37 @@ namespace {
 __device__ int g_tc_status = 0;  // first device-side error code of this device (0 = none)
 
 // Phase trace (builds with -DKDA_PHASE_TRACE only): the SM clock at the phase
-// boundaries of the first kTraceChunks chunks of CTA (0, 0), per warp group
-// (0 prep, 1 chain), read back by kda_trace_read.
+// boundaries of kTraceChunks chunks of CTA (0, 0) from chunk g_trace_c0 on, per warp
+// group (0 prep, 1 chain), and per CTA of the transition pass its start and end
+// (global timer, ns), SM, chunk count and start and end SM clock; read back by
+// kda_trace_read / kda_trace_spans.
 #ifdef KDA_PHASE_TRACE
-constexpr int kTraceChunks = 64, kTraceStamps = 16;
+__device__ __forceinline__ unsigned long long smid_u32() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(r));
+    return r;
+}
+constexpr int kTraceChunks = 64, kTraceStamps = 16, kSpanCtas = 8192;
 __device__ unsigned long long g_trace[2][kTraceChunks][kTraceStamps];
+__device__ unsigned long long g_span[kSpanCtas][6];
+__device__ long long g_trace_c0;
 #define TRACE(grp, chunk, k)                                                                    \
     do {                                                                                        \
-        if (blockIdx.x == 0 && blockIdx.y == 0 && (chunk) < kTraceChunks)                       \
-            g_trace[grp][chunk][k] = clock64();                                                 \
+        if (blockIdx.x == 0 && blockIdx.y == 0 && (chunk) >= g_trace_c0 &&                      \
+            (chunk) - g_trace_c0 < kTraceChunks)                                                \
+            g_trace[grp][(chunk) - g_trace_c0][k] = clock64();                                  \
+    } while (0)
+#define SPAN(which, value)                                                                      \
+    do {                                                                                        \
+        const int cta_ = blockIdx.y * gridDim.x + blockIdx.x;                                   \
+        if (cta_ < kSpanCtas) g_span[cta_][which] = (value);                                    \
     } while (0)
 #else
 #define TRACE(grp, chunk, k) \
     do {                     \
+    } while (0)
+#define SPAN(which, value) \
+    do {                   \
     } while (0)
 #endif
 
@@ -339,10 +357,8 @@ __device__ __forceinline__ void warp_mma_tf32(float (&d)[4], const float* a, int
 __device__ __forceinline__ void warp_store16x8(float* dst, int ld, const float (&d)[4], float sgn,
                                                int lane) {
     const int g = lane >> 2, t = lane & 3;
-    dst[g * ld + 2 * t] = sgn * d[0];
-    dst[g * ld + 2 * t + 1] = sgn * d[1];
-    dst[(g + 8) * ld + 2 * t] = sgn * d[2];
-    dst[(g + 8) * ld + 2 * t + 1] = sgn * d[3];
+    *reinterpret_cast<float2*>(dst + g * ld + 2 * t) = make_float2(sgn * d[0], sgn * d[1]);
+    *reinterpret_cast<float2*>(dst + (g + 8) * ld + 2 * t) = make_float2(sgn * d[2], sgn * d[3]);
 }
 
 // Run by the 256 prep threads once the [A;P] product is in TMEM.  Writes TB =
@@ -350,16 +366,16 @@ __device__ __forceinline__ void warp_store16x8(float* dst, int ld, const float (
 // read from the product (rows of A in TMEM lanes 0-63; tq = the calling warp's
 // lane quadrant), using As, Ts (fp32) and Ys as scratch:
 //  1. warp h (h = 0, 1) reads rows 32h..32h+31 of A from TMEM (scaled by beta,
-//     strictly-lower mask) into As and builds the 32 x 32 diagonal half h of T:
-//     its two 16 x 16 diagonal blocks by substitution (one lane per row,
-//     eliminating one known entry at a time), then T_21 = -T_22 (A_21 T_11)
-//     inside the half with tf32 warp MMAs; warps 2-5 zero the upper-right
-//     32 x 32 block of TB; `side(warp)` runs on warps 2-7 meanwhile;
+//     strictly-lower mask) and builds the 32 x 32 diagonal half h of T: its two
+//     16 x 16 diagonal blocks in fp32 by forward substitution (one column per lane,
+//     both blocks at once), then T_21 = -T_22 (A_21 T_11) inside the half with tf32
+//     warp MMAs; warps 2-5 zero the upper-right 32 x 32 block of TB; `side(warp)`
+//     runs on warps 2-7 meanwhile;
 //  2. TB of the two diagonal halves (all threads), and Z = A[32:64, 0:32] T_lo
 //     (warps 0-7, one 16 x 8 tile each);
 //  3. T[32:64, 0:32] = -T_hi Z, scaled by beta_j, straight into TB.
-// The block products are tf32 warp MMAs with fp32 accumulation (T then enters
-// the chunk products as bf16).
+// The block products are tf32 warp MMAs with fp32 accumulation (T then enters the
+// chunk products as bf16).
 template <typename Side>
 __device__ void invert_to_tb(float* As, float* Ts, float* Ys, const float* beta, uint32_t tbp,
                              int tid, uint32_t tq, Side side, int64_t chunk) {
@@ -368,16 +384,15 @@ __device__ void invert_to_tb(float* As, float* Ts, float* Ys, const float* beta,
     const int g = lane >> 2, t4 = lane & 3;
     if (warp < 2) {
         const int o = 32 * warp;
-        {  // 1a. diagonal blocks o (lanes 0-15) and o+16 (lanes 16-31): lane i holds
-           // row i of its block; T_i = e_i - sum_{m<i} A_im T_m, rows finished in order
-           // and broadcast to the 16 lanes of the block by shuffles
-            const int i = lane & 15, ob = o + 16 * (lane >> 4), src0 = lane & 16;
-            float arow[16], trow[16];
-            const int r = o + lane;  // this lane's row of A
-            const float br = beta[r];
-            // the row's TMEM loads in 32-column batches, one wait each: rows 0-31 need
-            // columns 0-31; columns j < 32 of rows >= 32 are the cross-half product (TMEM
-            // 64 + j), columns 32-63 of those rows the second half's block
+        const int r = o + lane;                  // this lane's row of A
+        const int blk = lane >> 4, i = lane & 15, ob = o + 16 * blk;
+        const float br = beta[r];
+        // diagonal 16 x 16 block blk of this half, transposed: At[m][i] = A[ob+i][ob+m]
+        // (block 1 sixteen banks after block 0; in rows of As the products never read)
+        float* At = As + warp * 544 + blk * 272;
+        {  // 1a. rows o..o+31 of A from TMEM in 32-column batches, one wait each: rows
+           // 0-31 need columns 0-31; columns j < 32 of rows >= 32 are the cross-half
+           // product (TMEM 64 + j), columns 32-63 of those rows the second half's block
 #pragma unroll
             for (int bb = 0; bb < 2; ++bb) {
                 if (warp == 0 && bb == 1) break;
@@ -388,34 +403,54 @@ __device__ void invert_to_tb(float* As, float* Ts, float* Ys, const float* beta,
                 tmem_ld16(src + 16, v1);
                 tmem_wait16(v0);
                 tmem_wait16(v1);
+                if (j0 == o) {
+                    // the lane's row inside its diagonal block (strictly lower), transposed
 #pragma unroll
-                for (int m = 0; m < 32; ++m) {
-                    const float vm = m < 16 ? v0[m] : v1[m - 16];
-                    const float x = j0 + m < r ? br * vm : 0.f;
-                    As[r * AS_LD + j0 + m] = x;
-                    if (j0 + (m & ~15) == ob) arow[m & 15] = x;
+                    for (int m = 0; m < 16; ++m) At[m * 16 + i] = m < i ? br * (blk ? v1[m] : v0[m]) : 0.f;
+                    if (blk) {  // A_21 of the half (rows o+16.., columns o..o+15): row-major
+#pragma unroll
+                        for (int m4 = 0; m4 < 4; ++m4)
+                            *reinterpret_cast<float4*>(As + r * AS_LD + o + 4 * m4) =
+                                make_float4(br * v0[4 * m4], br * v0[4 * m4 + 1], br * v0[4 * m4 + 2],
+                                            br * v0[4 * m4 + 3]);
+                    }
+                } else {  // rows 32-63, columns 0-31 (all below the diagonal): row-major
+#pragma unroll
+                    for (int m4 = 0; m4 < 8; ++m4) {
+                        const float* vv = m4 < 4 ? v0 + 4 * m4 : v1 + 4 * (m4 - 4);
+                        *reinterpret_cast<float4*>(As + r * AS_LD + 4 * m4) =
+                            make_float4(br * vv[0], br * vv[1], br * vv[2], br * vv[3]);
+                    }
                 }
             }
             __syncwarp();
             if (tid == 0) TRACE(0, chunk, 8);
+            // forward substitution in fp32, one column per lane: lane (blk, i) solves
+            // (I + A_bb) x = e_i, updating every later row as soon as x_m is known, so
+            // the steps are chained by one FMA each
+            float xc[16];
 #pragma unroll
-            for (int m = 0; m < 16; ++m) trow[m] = m == i ? 1.f : 0.f;
+            for (int m = 0; m < 16; ++m) xc[m] = m == i ? 1.f : 0.f;
 #pragma unroll
             for (int m = 0; m < 15; ++m) {
-                const float am = arow[m];
+                const float xm = xc[m];
 #pragma unroll
-                for (int c = 0; c <= m; ++c) {  // row m has entries in columns 0..m only
-                    const float tmc = __shfl_sync(0xffffffffu, trow[c], src0 + m);
-                    trow[c] = fmaf(-am, tmc, trow[c]);
+                for (int i4 = (m + 1) >> 2; i4 < 4; ++i4) {
+                    const float4 a = *reinterpret_cast<const float4*>(At + m * 16 + 4 * i4);
+                    const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        if (4 * i4 + k > m) xc[4 * i4 + k] = fmaf(-av[k], xm, xc[4 * i4 + k]);
                 }
             }
 #pragma unroll
-            for (int c = 0; c < 16; ++c) Ts[(ob + i) * TS_LD + ob + c] = trow[c];
+            for (int m = 0; m < 16; ++m) Ts[(ob + m) * TS_LD + ob + i] = xc[m];
             // zero the upper-right 16 x 16 block of this half (rows o..o+15, cols o+16..o+31)
 #pragma unroll
-            for (int x = 0; x < 8; ++x) {
+            for (int x = 0; x < 2; ++x) {
                 const int e = lane + 32 * x;
-                Ts[(o + (e >> 4)) * TS_LD + o + 16 + (e & 15)] = 0.f;
+                *reinterpret_cast<float4*>(Ts + (o + (e >> 2)) * TS_LD + o + 16 + 4 * (e & 3)) =
+                    make_float4(0.f, 0.f, 0.f, 0.f);
             }
         }
         __syncwarp();
@@ -454,7 +489,9 @@ __device__ void invert_to_tb(float* As, float* Ts, float* Ys, const float* beta,
     if (tid == 0) TRACE(0, chunk, 11);
     {  // 2a. TB of the two diagonal halves: 2 x 32 rows x 4 chunks of 8 columns
         const int hf = tid >> 7, r = 32 * hf + ((tid >> 2) & 31), j8 = 4 * hf + (tid & 3);
-        const float* tr = Ts + r * TS_LD + 8 * j8;
+        const float4 ta = *reinterpret_cast<const float4*>(Ts + r * TS_LD + 8 * j8);
+        const float4 tb = *reinterpret_cast<const float4*>(Ts + r * TS_LD + 8 * j8 + 4);
+        const float tr[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
         const float* bj = beta + 8 * j8;
         st_shared_v4(tbp + kmajor_chunk_off(r, j8, 64), pack_bf16(tr[0] * bj[0], tr[1] * bj[1]),
                      pack_bf16(tr[2] * bj[2], tr[3] * bj[3]), pack_bf16(tr[4] * bj[4], tr[5] * bj[5]),
@@ -591,6 +628,7 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
     uint64_t* bar = x.bar;
     const int w = tid >> 5, lane = tid & 31, h = x.h, H = a.H;
     const int hl = lane >> 4, cg = lane & 15, c0 = 8 * cg;
+    const uint32_t gsw = (uint32_t)(cg >> 2) & 1u;  // bank spread of the lane's 32-byte reads
     const bool half_b = w >= 4;  // this warp's tokens lie in the chunk's second half
     const uint32_t tq = x.tmem + ((uint32_t)((w & 3) * 32) << 16);
     float* beta_s = reinterpret_cast<float*>(sm + L::BETA);
@@ -661,8 +699,11 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
             for (int i = 0; i < 4; ++i) {
                 const bool live = 8 * w + 4 * hl + i < Lc;  // rows past the segment end:
                 const uint32_t ro = raw_row0 + (uint32_t)i * 128u;  // identity steps
-                float4 l0 = *reinterpret_cast<const float4*>(la_t + ro);
-                float4 l1 = *reinterpret_cast<const float4*>(la_t + ro + 4);
+                // the two 16-byte halves of the lane's 32 bytes in an order that puts
+                // lanes 4-7 of each quarter on the banks lanes 0-3 leave free
+                const float4 la0 = *reinterpret_cast<const float4*>(la_t + ro + 4u * gsw);
+                const float4 la1 = *reinterpret_cast<const float4*>(la_t + ro + 4u * (gsw ^ 1u));
+                float4 l0 = gsw ? la1 : la0, l1 = gsw ? la0 : la1;
                 kr[i] = ld_shared_v4(kt + 2u * ro);
                 if (Q) qr[i] = ld_shared_v4(qt + 2u * ro);
                 if (!live) {
@@ -688,8 +729,10 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
                 }
             }
             if (hl) {  // the warp's 8-token sums
-                *reinterpret_cast<float4*>(gsum + w * D + c0) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-                *reinterpret_cast<float4*>(gsum + w * D + c0 + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+                *reinterpret_cast<float4*>(gsum + w * D + c0 + 4u * gsw) =
+                    make_float4(acc[0], acc[1], acc[2], acc[3]);
+                *reinterpret_cast<float4*>(gsum + w * D + c0 + 4u * (gsw ^ 1u)) =
+                    make_float4(acc[4], acc[5], acc[6], acc[7]);
             }
             if (tid < C)
                 beta_s[tid] = maps.beta_tma ? (tid < Lc ? reinterpret_cast<const float*>(sm + L::BTILE)[4 * tid + (h & 3)] : 0.f)
@@ -746,8 +789,8 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
             for (int j = 0; j < 8; ++j) run[j] = off[j] = ra[j] = rb[j] = 0.f;
 #pragma unroll
             for (int ww = 0; ww < 8; ++ww) {
-                const float4 t0v = *reinterpret_cast<const float4*>(gsum + ww * D + c0);
-                const float4 t1v = *reinterpret_cast<const float4*>(gsum + ww * D + c0 + 4);
+                const float4 t0v = *reinterpret_cast<const float4*>(gsum + ww * D + c0 + 4u * gsw);
+                const float4 t1v = *reinterpret_cast<const float4*>(gsum + ww * D + c0 + 4u * (gsw ^ 1u));
                 const float tv[8] = {t0v.x, t0v.y, t0v.z, t0v.w, t1v.x, t1v.y, t1v.z, t1v.w};
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
@@ -1387,6 +1430,12 @@ __global__ void __launch_bounds__(NT, 1) chunk_kernel(TcArgs a, const __grid_con
         if (tid == 0) atomicCAS(&g_tc_status, 0, ERR_SEG_OVERFLOW);  // malformed cu_seqlens
         return;
     }
+    if ((MODE == TRANS || MODE == TRANS_CACHE) && tid == 0) {
+        SPAN(0, globaltimer_ns());
+        SPAN(2, smid_u32());
+        SPAN(3, (unsigned long long)nc);
+        SPAN(4, clock64());
+    }
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L::BAR);
     uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(sm + L::TMEMP);
     if (warp == 0) {
@@ -1427,6 +1476,10 @@ __global__ void __launch_bounds__(NT, 1) chunk_kernel(TcArgs a, const __grid_con
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(x.tmem, 512);
+    if ((MODE == TRANS || MODE == TRANS_CACHE) && tid == 0) {
+        SPAN(1, globaltimer_ns());
+        SPAN(5, clock64());
+    }
 }
 
 // ---------------------------------------------------------------- pass 3 from the chunk cache
@@ -2032,6 +2085,16 @@ extern "C" int kda_trace_read(unsigned long long* host, int n) {
     if (cudaMemcpyFromSymbol(host, g_trace, (size_t)n * sizeof(unsigned long long)) != cudaSuccess)
         return -1;
     return n;
+}
+extern "C" int kda_trace_spans(unsigned long long* host, int n) {
+    const int total = kSpanCtas * 6;
+    if (n > total) n = total;
+    if (cudaMemcpyFromSymbol(host, g_span, (size_t)n * sizeof(unsigned long long)) != cudaSuccess)
+        return -1;
+    return n;
+}
+extern "C" int kda_trace_first_chunk(long long c0) {
+    return cudaMemcpyToSymbol(g_trace_c0, &c0, sizeof(c0)) == cudaSuccess ? 0 : -1;
 }
 #endif
 
