@@ -1,6 +1,6 @@
 """Build libkda.so in place with nvcc for sm_100a (B200).
 
-    python -m gated_delta_rule_139_b200.build [--force] [--trace]
+    python -m gated_delta_rule_139_b200.build [--force] [--trace | --debug]
 
 Each ``csrc/*.cu`` file is compiled to an object in ``_build/`` (in parallel),
 then linked into ``gated_delta_rule_139_b200/libkda.so``.  Objects are rebuilt
@@ -11,6 +11,12 @@ newer.
 compiled with ``-DKDA_PHASE_TRACE``: the tensor-core kernels record the SM clock
 at their phase boundaries for the first CTA, readable with ``kda_trace_read``.
 Load it by setting ``KDA_LIBRARY`` to its path before importing the package.
+
+``--debug`` builds ``_build/debug/libkda.so`` with ``-DKDA_DEBUG``: the kernels
+check every index they derive from device-built tables (segment entries, the
+per-sequence unit offsets) against the buffer it addresses before using it; a
+failed check records ``KDA_ERR_CUDA`` with the source line in the device status
+word (read by ``kda_check_device``) and the block returns without the access.
 """
 from __future__ import annotations
 
@@ -37,10 +43,18 @@ def _newest(paths):
     return max((os.path.getmtime(p) for p in paths), default=0.0)
 
 
-def build(force: bool = False, verbose: bool = False, trace: bool = False) -> str:
-    build_dir = os.path.join(BUILD, "trace") if trace else BUILD
-    lib_path = os.path.join(build_dir, "libkda.so") if trace else LIB
-    cflags = CFLAGS + (["-DKDA_PHASE_TRACE"] if trace else [])
+VARIANTS = {"trace": "-DKDA_PHASE_TRACE", "debug": "-DKDA_DEBUG"}
+
+
+def build(force: bool = False, verbose: bool = False, trace: bool = False,
+          variant: str | None = None) -> str:
+    """Builds the library (or, with variant "trace" / "debug", that diagnostic
+    build under _build/<variant>/) and returns the path of the .so."""
+    if trace:
+        variant = "trace"
+    build_dir = os.path.join(BUILD, variant) if variant else BUILD
+    lib_path = os.path.join(build_dir, "libkda.so") if variant else LIB
+    cflags = CFLAGS + ([VARIANTS[variant]] if variant else [])
     os.makedirs(build_dir, exist_ok=True)
     sources = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     headers = glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.cuh")) + \
@@ -73,4 +87,5 @@ def build(force: bool = False, verbose: bool = False, trace: bool = False) -> st
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose=True, trace="--trace" in sys.argv))
+    var = "trace" if "--trace" in sys.argv else "debug" if "--debug" in sys.argv else None
+    print(build(force="--force" in sys.argv, verbose=True, variant=var))

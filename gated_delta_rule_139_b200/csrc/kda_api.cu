@@ -215,9 +215,30 @@ kda_status run_tc(const kda::FwdArgs& a, cudaStream_t stream, int* launches) {
     const size_t b_sin = p.segmented ? (size_t)p.max_units * a.H * st : 0;
     // chunk cache of the segmented plan: kCacheEntryBytes per chunk and head
     const size_t b_cache = p.segmented ? (size_t)p.total_chunks * a.H * kda::kCacheEntryBytes : 0;
-    char* ws = nullptr;
-    cudaError_t e = pool_alloc((void**)&ws, b_segs + b_off + b_trans + b_sin + b_cache, stream);
+#ifdef KDA_DEBUG
+    // debug builds: a guard band before the first buffer and after every buffer
+    constexpr size_t G = kda::kGuardBytes;
+#else
+    constexpr size_t G = 0;
+#endif
+    char* base = nullptr;
+    cudaError_t e = pool_alloc((void**)&base, G + b_segs + G + b_off + G + b_trans + G + b_sin + G +
+                                                  b_cache + G, stream);
     if (e != cudaSuccess) return cuda_fail(e, "workspace allocation");
+    char* ws = base + G;
+    const size_t o_off = b_segs + G, o_trans = o_off + b_off + G, o_sin = o_trans + b_trans + G,
+                 o_cache = o_sin + b_sin + G;
+#ifdef KDA_DEBUG
+    kda::GuardBands guards{};
+    for (char* g : {base, ws + b_segs, ws + o_off + b_off, ws + o_trans + b_trans, ws + o_sin + b_sin,
+                    ws + o_cache + b_cache}) {
+        guards.band[guards.n++] = (const uint32_t*)g;
+        if ((e = cudaMemsetAsync(g, 0xA5, G, stream)) != cudaSuccess) {
+            cudaFreeAsync(base, stream);
+            return cuda_fail(e, "guard band fill");
+        }
+    }
+#endif
     kda::TcArgs t{};
     t.q = a.q;
     t.k = a.k;
@@ -239,17 +260,20 @@ kda_status run_tc(const kda::FwdArgs& a, cudaStream_t stream, int* launches) {
     t.H = a.H;
     t.N = a.N;
     t.segs = (kda::SegEntry*)ws;
-    t.seg_off = (int32_t*)(ws + b_segs);
+    t.seg_off = (int32_t*)(ws + o_off);
     t.n_units = t.seg_off + a.N + 1;
-    t.trans = p.segmented ? (float*)(ws + b_segs + b_off) : nullptr;
-    t.sin = p.segmented ? (float*)(ws + b_segs + b_off + b_trans) : nullptr;
+    t.trans = p.segmented ? (float*)(ws + o_trans) : nullptr;
+    t.sin = p.segmented ? (float*)(ws + o_sin) : nullptr;
     if (p.segmented) {  // pass 1 runs over every segment and leaves the chunk cache for pass 3
-        t.cache = (uint8_t*)(ws + b_segs + b_off + b_trans + b_sin);
+        t.cache = (uint8_t*)(ws + o_cache);
         t.total_chunks = p.total_chunks;
         t.trans_all = 1;
     }
     e = kda::launch_tc(t, p, stream, launches);
-    cudaFreeAsync(ws, stream);
+#ifdef KDA_DEBUG
+    if (e == cudaSuccess) e = kda::launch_guard_check(guards, stream);
+#endif
+    cudaFreeAsync(base, stream);
     if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
     return KDA_OK;
 }
@@ -472,6 +496,7 @@ kda_status kda_fwd(const void* q, const void* k, const void* v, const float* log
                    const float* beta, const float* initial_state, const int32_t* cu_seqlens,
                    int32_t chunk, void* out, float* final_state, const kda_dims* dims,
                    void* stream) {
+    kda::NvtxRange nvtx_range("kda_fwd");
     g_last_error[0] = 0;
     g_last_launches = 0;
     g_last_path = "";
@@ -568,6 +593,7 @@ kda_status kda_fwd_ex(const void* q, const void* k, const void* v, const float* 
                       const float* beta, const float* initial_state, const int32_t* cu_seqlens,
                       int32_t chunk, void* out, float* final_state, const kda_dims* dims,
                       const kda_fwd_opts* opts, void* stream) {
+    kda::NvtxRange nvtx_range("kda_fwd_ex");
     g_last_error[0] = 0;
     g_last_launches = 0;
     g_last_path = "";
@@ -585,6 +611,7 @@ kda_status kda_fwd_snap(const void* q, const void* k, const void* v, const float
                         const int32_t* cu_seqlens, int32_t chunk, void* out, float* final_state,
                         const kda_dims* dims, const kda_snap_spec* snap,
                         const int32_t* snap_slots, float* snap_pool, void* stream) {
+    kda::NvtxRange nvtx_range("kda_fwd_snap");
     if (!snap) {
         g_last_error[0] = 0;
         g_last_launches = 0;
@@ -613,6 +640,7 @@ kda_status kda_fwd_host(const void* q, const void* k, const void* v, const float
                         const float* beta, const float* initial_state,
                         const int32_t* cu_seqlens, int32_t chunk, void* out,
                         float* final_state, const kda_dims* dims, void* stream_) {
+    kda::NvtxRange nvtx_range("kda_fwd_host");
     g_last_error[0] = 0;
     g_last_launches = 0;
     g_last_path = "";
@@ -756,6 +784,7 @@ kda_status kda_fwd_noalloc(const void* q, const void* k, const void* v, const fl
                            const float* beta, const float* initial_state,
                            const int32_t* cu_seqlens, int32_t chunk, void* out,
                            float* final_state, const kda_dims* dims, void* stream_) {
+    kda::NvtxRange nvtx_range("kda_fwd_noalloc");
     g_last_error[0] = 0;
     g_last_launches = 0;
     g_last_path = "";
@@ -832,6 +861,7 @@ kda_status kda_fwd_noalloc(const void* q, const void* k, const void* v, const fl
 
 kda_status kda_transition(const void* k, const void* v, const float* log_alpha,
                           const float* beta, const kda_dims* d, float* trans, void* stream) {
+    kda::NvtxRange nvtx_range("kda_transition");
     g_last_error[0] = 0;
     g_last_launches = 0;
     g_last_path = "";
@@ -887,6 +917,7 @@ size_t kda_span_workspace_bytes(const kda_dims* d) {
 kda_status kda_span_transition(const void* q, const void* k, const void* v, const float* log_alpha,
                                const float* beta, const kda_dims* d, void* workspace,
                                size_t workspace_bytes, float* trans, void* stream) {
+    kda::NvtxRange nvtx_range("kda_span_transition");
     g_last_error[0] = 0;
     g_last_launches = 0;
     g_last_path = "";
@@ -926,6 +957,7 @@ kda_status kda_span_forward_ex(const void* q, const void* k, const void* v,
                                const float* initial_state, void* out, float* final_state,
                                const kda_dims* d, const void* workspace, size_t workspace_bytes,
                                const kda_fwd_opts* opts, void* stream) {
+    kda::NvtxRange nvtx_range("kda_span_forward_ex");
     g_last_error[0] = 0;
     g_last_launches = 0;
     g_last_path = "";
@@ -990,6 +1022,7 @@ kda_status kda_span_forward(const void* q, const void* k, const void* v, const f
 
 kda_status kda_chunk_operands(const void* q, const void* k, const void* v, const float* log_alpha,
                               const float* beta, const kda_dims* d, void* images, void* stream) {
+    kda::NvtxRange nvtx_range("kda_chunk_operands");
     g_last_error[0] = 0;
     g_last_launches = 0;
     g_last_path = "";
@@ -1044,6 +1077,7 @@ kda_status kda_chunk_operands(const void* q, const void* k, const void* v, const
 
 kda_status kda_apply_transitions(const float* trans, int32_t count, int32_t B, int32_t H,
                                  const float* initial_state, float* state_out, void* stream) {
+    kda::NvtxRange nvtx_range("kda_apply_transitions");
     g_last_error[0] = 0;
     g_last_launches = 0;
     g_last_path = "";
@@ -1090,6 +1124,7 @@ kda_status kda_decode(const void* q, const void* k, const void* v, const float* 
                       const float* beta, float* state, const int32_t* slots, void* out,
                       const void* out_gate, float* token_states, const kda_decode_dims* d,
                       void* stream) {
+    kda::NvtxRange nvtx_range("kda_decode");
     g_last_error[0] = 0;
     g_last_launches = 0;
     g_last_path = "";
@@ -1245,6 +1280,12 @@ kda_status kda_check_device(void* stream) {
         return fail(KDA_ERR_INVALID_ARG, "segment table overflow: malformed cu_seqlens");
     if (code == kda::ERR_BAD_SLOT)
         return fail(KDA_ERR_INVALID_ARG, "a decode slot index lies outside the state pool");
+    if ((code & 0xff) == kda::ERR_DEBUG_INDEX)
+        return fail(KDA_ERR_CUDA, "debug build: a device index check failed (kda_tc.cu line %d)",
+                    code >> 8);
+    if ((code & 0xff) == kda::ERR_DEBUG_GUARD)
+        return fail(KDA_ERR_CUDA, "debug build: guard band %d of the kda_fwd workspace was overwritten",
+                    code >> 8);
     if (code) return fail(KDA_ERR_CUDA, "device status %d", code);
     return KDA_OK;
 }

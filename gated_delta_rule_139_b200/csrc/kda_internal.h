@@ -2,6 +2,7 @@
 #pragma once
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdint.h>
 
 namespace kda {
@@ -9,12 +10,38 @@ namespace kda {
 constexpr int kChunk = 64;       // tokens per chunk
 constexpr int kMaxDevices = 64;  // size of per-device attribute caches
 
+// NVTX range over a host scope (header-only NVTX 3: a no-op unless a profiler is
+// attached), so a timeline shows which public call and which pass issued a kernel.
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
 // Kernel slots of the optional per-launch timing (kda_profile_*).
 enum KernelSlot : int { SLOT_SETUP = 0, SLOT_PASS1 = 1, SLOT_SCAN = 2, SLOT_PASS3 = 3, SLOT_FFMA = 4,
                         SLOT_DECODE = 5, SLOT_CHAIN = 6, NUM_SLOTS = 7 };
 
 // Device status codes (first error wins; read and cleared by kda_check_device).
-enum DeviceStatus : int { ERR_WAIT_TIMEOUT = 1, ERR_SEG_OVERFLOW = 2, ERR_BAD_SLOT = 3 };
+// ERR_DEBUG_INDEX (KDA_DEBUG builds only) carries the failing check's source line
+// in the bits above the low byte, ERR_DEBUG_GUARD (likewise) the overwritten guard
+// band's index.
+enum DeviceStatus : int { ERR_WAIT_TIMEOUT = 1, ERR_SEG_OVERFLOW = 2, ERR_BAD_SLOT = 3,
+                          ERR_DEBUG_INDEX = 4, ERR_DEBUG_GUARD = 5 };
+
+// Guard bands of the debug build's kda_fwd workspace: kGuardBytes of kGuardWord
+// before and after each of its buffers, checked after the launches.
+constexpr size_t kGuardBytes = 4096;
+constexpr uint32_t kGuardWord = 0xA5A5A5A5u;
+constexpr int kMaxGuards = 8;
+struct GuardBands {
+    const uint32_t* band[kMaxGuards];
+    int n;
+};
+// Checks every band (kGuardBytes each) on the device; an overwritten band i records
+// ERR_DEBUG_GUARD | (i << 8) in the status word.  Not counted as a launch.
+cudaError_t launch_guard_check(const GuardBands& g, cudaStream_t stream);
 // Device address of the current device's status word.
 cudaError_t status_word(int** p);
 // Records a CUDA event on `stream` before (begin=true) or after a launch of

@@ -63,6 +63,35 @@ namespace {
 
 __device__ int g_tc_status = 0;  // first device-side error code of this device (0 = none)
 
+// Debug builds (-DKDA_DEBUG): an index the kernel derives from a device-built table
+// is checked against the buffer it addresses before the first access through it.  A
+// failed check records ERR_DEBUG_INDEX with the source line and the whole block
+// returns; the condition is uniform over the block, and the checks sit before any
+// barrier, TMEM allocation or asynchronous copy.  Release builds compile them out.
+#ifdef KDA_DEBUG
+#define KDA_DCHECK(cond)                                                                    \
+    do {                                                                                    \
+        if (!(cond)) {                                                                      \
+            if (threadIdx.x == 0) atomicCAS(&g_tc_status, 0, ERR_DEBUG_INDEX | (__LINE__ << 8)); \
+            return;                                                                         \
+        }                                                                                   \
+    } while (0)
+#else
+#define KDA_DCHECK(cond) \
+    do {                 \
+    } while (0)
+#endif
+#ifdef KDA_DEBUG
+// The segment entry lies inside its sequence: n in [0, N), lo <= t_begin <= t_end <= hi
+// with t_begin on a chunk boundary of the sequence.
+__device__ bool seg_entry_ok(const TcArgs& a, const SegEntry& sg) {
+    if (sg.n < 0 || sg.n >= a.N) return false;
+    const int64_t lo = a.cu ? (int64_t)a.cu[sg.n] : (int64_t)sg.n * a.T;
+    const int64_t hi = a.cu ? (int64_t)a.cu[sg.n + 1] : lo + a.T;
+    return lo <= sg.t_begin && sg.t_begin <= sg.t_end && sg.t_end <= hi && (sg.t_begin - lo) % kChunk == 0;
+}
+#endif
+
 // Phase trace (builds with -DKDA_PHASE_TRACE only): the SM clock at the phase
 // boundaries of kTraceChunks chunks of CTA (0, 0) from chunk g_trace_c0 on, per warp
 // group (0 prep, 1 chain), and per CTA of the transition pass its start and end
@@ -1421,8 +1450,10 @@ __global__ void __launch_bounds__(NT, 1) chunk_kernel(TcArgs a, const __grid_con
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const int tid = threadIdx.x, warp = tid >> 5;
     const int u = blockIdx.x, h = blockIdx.y;
+    KDA_DCHECK(*a.n_units >= 0 && *a.n_units <= (int)gridDim.x);  // the table has gridDim.x entries
     if (u >= *a.n_units) return;
     const SegEntry sg = a.segs[u];
+    KDA_DCHECK(seg_entry_ok(a, sg));
     // transitions only for segments with a successor, unless all are asked for
     if ((MODE == TRANS || MODE == TRANS_CACHE) && sg.last && !a.trans_all) return;
     const int64_t nc = sg.t_end > sg.t_begin ? (sg.t_end - sg.t_begin + C - 1) / C : 0;
@@ -1512,8 +1543,10 @@ __global__ void __launch_bounds__(NT, 1) cached_kernel(TcArgs a, const __grid_co
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int u = blockIdx.x, h = blockIdx.y, H = a.H;
+    KDA_DCHECK(*a.n_units >= 0 && *a.n_units <= (int)gridDim.x);
     if (u >= *a.n_units) return;
     const SegEntry sg = a.segs[u];
+    KDA_DCHECK(seg_entry_ok(a, sg));
     const bool snap_on = a.snap_pool != nullptr;
     const bool gate_on = a.gate != nullptr;
     const int64_t seq_lo = snap_on ? (a.cu ? (int64_t)a.cu[sg.n] : (int64_t)sg.n * a.T) : 0;
@@ -1888,6 +1921,7 @@ __global__ void __launch_bounds__(256) seg_scan_kernel(TcArgs a) {
     const int tid = threadIdx.x, el = tid >> 5, cg = tid & 31;
     const int32_t u0 = a.seg_off[n], u1 = a.seg_off[n + 1];
     const int32_t nu = *a.n_units;
+    KDA_DCHECK(0 <= u0 && u0 <= u1 && nu >= 0);  // transitions and states indexed below nu
     if (u1 - u0 <= 1 || u0 >= nu) return;
     const int32_t last = (u1 < nu ? u1 : nu) - 1;  // segments u0 .. last; transitions u0 .. last-1
     // S_in of segment 0, also copied to the workspace so that pass 3 never reads
@@ -2112,16 +2146,24 @@ cudaError_t launch_tc(const TcArgs& a, const TcPlan& p, cudaStream_t stream, int
     TcMaps maps;
     if ((err = make_maps(a, &maps)) != cudaSuccess) return err;
     if (!from_span) {  // else the segment table and the transitions are in the workspace
-        if ((err = launch_setup(a, p, stream, launches)) != cudaSuccess) return err;
-        if (p.segmented && (err = launch_pass1(a, p, maps, stream, launches)) != cudaSuccess) return err;
+        {
+            NvtxRange r("kda.segment_table");
+            if ((err = launch_setup(a, p, stream, launches)) != cudaSuccess) return err;
+        }
+        if (p.segmented) {
+            NvtxRange r("kda.pass1_transitions");
+            if ((err = launch_pass1(a, p, maps, stream, launches)) != cudaSuccess) return err;
+        }
     }
     if (p.segmented) {
+        NvtxRange r("kda.segment_scan");
         profile_mark(SLOT_SCAN, true, stream);
         seg_scan_kernel<<<dim3((unsigned)a.N, (unsigned)a.H, D / SCAN_ROWS), 256, SCAN_SMEM, stream>>>(a);
         profile_mark(SLOT_SCAN, false, stream);
         *launches += 1;
         if ((err = cudaGetLastError()) != cudaSuccess) return err;
     }
+    NvtxRange r("kda.pass3_forward");
     profile_mark(SLOT_PASS3, true, stream);
     const dim3 grid((unsigned)p.max_units, (unsigned)a.H);
     if (p.segmented && a.cache)
@@ -2155,6 +2197,20 @@ cudaError_t launch_transition(const TcArgs& a_in, const TcPlan& p, float* out, c
     c.out = out;
     c.compose = 1;
     return launch_chain(c, stream, launches);
+}
+
+// Debug builds: each guard band around a workspace buffer still holds kGuardWord.
+__global__ void __launch_bounds__(256) guard_check_kernel(GuardBands g) {
+    const int b = blockIdx.x;
+    bool bad = false;
+    for (int i = threadIdx.x; i < (int)(kGuardBytes / 4); i += 256) bad |= g.band[b][i] != kGuardWord;
+    if (__syncthreads_or(bad) && threadIdx.x == 0) atomicCAS(&g_tc_status, 0, ERR_DEBUG_GUARD | (b << 8));
+}
+
+cudaError_t launch_guard_check(const GuardBands& g, cudaStream_t stream) {
+    if (g.n <= 0 || g.n > kMaxGuards) return cudaErrorInvalidValue;
+    guard_check_kernel<<<g.n, 256, 0, stream>>>(g);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_wait_probe(uint64_t timeout_ns, int arrive, cudaStream_t stream) {

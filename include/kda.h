@@ -414,11 +414,13 @@ int32_t kda_last_launch_count(void);
 const char* kda_last_path(void);
 
 /* Synchronises `stream`, then reads and clears the current device's status
- * word, which kernels set when a bounded wait gives up (KDA_ERR_DEVICE_TIMEOUT)
- * (KDA_ERR_DEVICE_TIMEOUT), the device-built segment table would overflow
- * because cu_seqlens is malformed, or a kda_decode slot index lay outside the
- * state pool (both KDA_ERR_INVALID_ARG).  KDA_OK when neither happened since the last
- * check. */
+ * word, which kernels set when a bounded wait gives up (KDA_ERR_DEVICE_TIMEOUT),
+ * the device-built segment table would overflow because cu_seqlens is malformed,
+ * or a kda_decode slot index lay outside the state pool (both KDA_ERR_INVALID_ARG).
+ * In a library built with -DKDA_DEBUG the kernels also check the indices they take
+ * from device-built tables before using them; a failed check reports KDA_ERR_CUDA
+ * with the source line in kda_last_error().  KDA_OK when none of these happened
+ * since the last check. */
 kda_status kda_check_device(void* stream);
 
 /*
