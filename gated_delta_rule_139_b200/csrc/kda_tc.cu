@@ -134,6 +134,7 @@ constexpr int D = 128;             // d_k = d_v
 constexpr int NPREP = 256;         // prep threads (warps 0-7)
 constexpr int NCHAIN = 256;        // chain threads (warps 8-15, two per TMEM lane quadrant)
 constexpr int NT = NPREP + NCHAIN;
+constexpr int TCOPY = 128;  // prep thread that issues the TMA loads and bulk stores
 constexpr int BAR_PREP = 1, BAR_CHAIN = 2;  // named barriers of the two groups
 constexpr float LOG2E = 1.4426950408889634f;
 
@@ -178,8 +179,8 @@ struct Lay {
     static constexpr uint32_t LA = KG + 16384;
     static constexpr uint32_t AS = X1, TS = AS + 17408, YS = TS + 18432, TB = YS + 5120;
     static constexpr uint32_t BTILE = LA + 32768;  // the log alpha tile's beta: fp32 [64][4 heads]
-    static constexpr uint32_t GSUM = BTILE + 1024; // fp32 [8][128] (transitions only)
-    static constexpr uint32_t BETA = GSUM + (Q ? 0 : 4096);  // fp32 [64]
+    static constexpr uint32_t GSUM = BTILE + 1024; // fp32 [14][128] (transitions only)
+    static constexpr uint32_t BETA = GSUM + (Q ? 0 : 8192);  // fp32 [64]
     static constexpr uint32_t BAR = BETA + 256;    // mbarriers
     static constexpr uint32_t TMEMP = BAR + 256;   // TMEM base address
     static constexpr uint32_t BYTES = TMEMP + 16 + 1024;  // + alignment slack
@@ -193,7 +194,7 @@ static_assert(Lay<FWD>::BYTES <= 232448 && Lay<TRANS>::BYTES <= 232448, "shared 
 enum Bars : int {
     B_AP = 0,      // prep: [A;P] product done
     B_WU = 1,      // prep: W and U' products done
-    B_V = 2,       // prep: a chunk's v tile landed in its slot (TMA; one per chunk, in order)
+    B_V = 2,       // prep: a chunk's v tile landed in slot 0 (TMA; one per use of the slot)
     B_FULL = 3,    // [2] ring slot filled (prep -> chain)
     B_EMPTY = 5,   // [2] the chain's products have read the slot (MMA commit)
     B_WFREE = 7,   // [2] the slot's W area is free again (output tile stored)
@@ -204,7 +205,8 @@ enum Bars : int {
     B_GATE = 14,   // chain: output-gate tile landed (TMA)
     B_LA = 15,     // prep: a chunk's log alpha tile landed (TMA; one per chunk)
     B_KQ = 16,     // prep: a chunk's k (and q) tiles landed in its slot (TMA; one per chunk)
-    NBARS = 17
+    B_V1 = 17,     // prep: a chunk's v tile landed in slot 1
+    NBARS = 18
 };
 
 // TMEM columns (512 allocated).
@@ -631,11 +633,14 @@ __device__ __forceinline__ void tma_kq(uint8_t* slot, uint64_t* bar, const TcMap
     tma_tile(slot + L::S_KD, &maps.k, 0, h, t0, bar + B_KQ);
     if (L::Q) tma_tile(slot + L::S_QT, &maps.q, 0, h, t0, bar + B_KQ);
 }
-__device__ __forceinline__ void tma_v(uint8_t* slot, uint64_t* bar, const TcMaps& maps, int h, int t0) {
-    mbar_expect_tx(bar + B_V, 16384);
-    tma_tile(slot, &maps.v, 0, h, t0, bar + B_V);  // the W piece is at offset 0
-    tma_tile(slot + 8192, &maps.v, 64, h, t0, bar + B_V);
+// v tile of the chunk at t0 into the slot's W piece (offset 0); vbar = the slot's B_V barrier
+__device__ __forceinline__ void tma_v(uint8_t* slot, uint64_t* vbar, const TcMaps& maps, int h, int t0) {
+    mbar_expect_tx(vbar, 16384);
+    tma_tile(slot, &maps.v, 0, h, t0, vbar);
+    tma_tile(slot + 8192, &maps.v, 64, h, t0, vbar);
 }
+// mbarrier of slot s's v tile
+__device__ __forceinline__ uint64_t* v_bar(uint64_t* bar, int s) { return bar + (s ? B_V1 : B_V); }
 template <bool Q>
 __device__ __forceinline__ void prefetch_chunk(const TcMaps& maps, int h, int t0) {
     tma_prefetch(&maps.la, 0, h, t0);
@@ -680,16 +685,21 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
     auto cache_entry = [&](int64_t cc) {
         return a.cache + ((x.sg.c_base + cc) * H + h) * (int64_t)kCacheEntryBytes;
     };
-    // thread 0: TMA loads and products in flight, for the waits after a timeout
-    bool ap_out = false, wu_out = false, v_out = false, la_out = false, kq_out = false;
-    uint32_t ap_par = 0, wu_par = 0, v_par = 0, la_par = 0, kq_par = 0;
-    if (x.nc > 0 && tid == 0) {  // chunk 0's tiles (slot 0 is free)
+    // Thread 0 issues the tensor-core products; the copy thread TCOPY (lane 0 of warp
+    // 4, whose share of the inversion is the shortest) issues every TMA load and bulk
+    // store, so that no warp with a full share of a phase also carries the copies.
+    // Each keeps what it has in flight, for the waits after a timeout.
+    bool ap_out = false, wu_out = false, v_out[2] = {false, false}, la_out = false, kq_out = false;
+    uint32_t ap_par = 0, wu_par = 0, v_par[2] = {0, 0}, la_par = 0, kq_par = 0;
+    // In the transition modes chunk c+1's v tile goes into its slot together with its k
+    // tile (the slot's W piece is free once its k piece is); the forward and dump chains
+    // put chunk c-2's output tile there, so chunk c's v waits for it in chunk c.
+    constexpr bool V_AHEAD = MODE == TRANS || MODE == TRANS_CACHE;
+    if (x.nc > 0 && tid == TCOPY) {  // chunk 0's tiles (slot 0 is free)
         tma_la<MODE>(sm, bar, maps, h, (int)tb);
         tma_kq<MODE>(sm, bar, maps, h, (int)tb);
-        tma_v(sm, bar, maps, h, (int)tb);
-        la_out = kq_out = v_out = true;
-    }
-    if (tid == 32) {
+        tma_v(sm, v_bar(bar, 0), maps, h, (int)tb);
+        la_out = kq_out = v_out[0] = true;
         if (x.nc > 1) prefetch_chunk<Q>(maps, h, (int)(tb + C));
         if (x.nc > 2) prefetch_chunk<Q>(maps, h, (int)(tb + 2 * C));
     }
@@ -712,11 +722,11 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
         {
             const bool lok = wait_bar(bar + B_LA, (uint32_t)(c & 1)) &&
                              wait_bar(bar + B_KQ, (uint32_t)(c & 1));
-            if (lok && tid == 0) {
+            if (lok && tid == 0) TRACE(0, c, 14);
+            if (lok && tid == TCOPY) {
                 la_out = kq_out = false;
-                TRACE(0, c, 14);
                 // the previous chunk's TB store (all but the latest bulk group) has read
-                // X1/BT before this chunk's images go there
+                // X1/BT before this chunk's images go there (after the gate barrier)
                 if (CACHE) bulk_wait_read1();
             }
             const float* la_t = reinterpret_cast<const float*>(sm + L::LA);
@@ -772,11 +782,12 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
                 break;
             }
         }
-        // thread 0: the next chunk's k (and q) tiles go into the next slot as soon as the
-        // chain's products of chunk c-1 have read it, and this chunk's v tile into this
-        // slot's W piece as soon as chunk c-2's output tile has left it; polled at a few
-        // points of the chunk, waited for at the last one
-        bool kq_next = c + 1 >= x.nc, v_this = c == 0;
+        // copy thread: the next chunk's k (and q, and in the transition modes v) tiles go
+        // into the next slot as soon as the chain's products of chunk c-1 (and its cache
+        // stores) have read it; in the forward and dump modes this chunk's v tile goes
+        // into this slot's W piece as soon as chunk c-2's output tile has left it; polled
+        // at a few points of the chunk, waited for at the last one
+        bool kq_next = c + 1 >= x.nc, v_this = c == 0 || V_AHEAD;
         uint8_t* nslot = sm + (s ^ 1) * L::SLOT;
         const uint32_t nuse = (uint32_t)(((c + 1) >> 1) & 1);
         auto poll_tma = [&](bool block_kq, bool block_v) -> bool {
@@ -787,68 +798,73 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
                 TRACE(0, c + 1, 13);
                 kq_next = kq_out = true;
                 kq_par = (uint32_t)((c + 1) & 1);
+                if (V_AHEAD) {
+                    tma_v(nslot, v_bar(bar, s ^ 1), maps, h, (int)(t0 + C));
+                    v_out[s ^ 1] = true;
+                    v_par[s ^ 1] = nuse;
+                }
             }
             // (only the forward chain puts output tiles into the W piece; the dump chain
-            // arrives on B_WFREE anyway, the transition chains never do)
-            if (!v_this && (!(MODE == FWD || MODE == DUMP) ||
-                            (block_v ? wait_bar(bar + B_WFREE + s, use ^ 1u)
-                                     : mbar_try_wait(bar + B_WFREE + s, use ^ 1u)))) {
-                tma_v(slot, bar, maps, h, (int)t0);
-                v_this = v_out = true;
-                v_par = (uint32_t)(c & 1);
+            // arrives on B_WFREE anyway)
+            if (!v_this && (block_v ? wait_bar(bar + B_WFREE + s, use ^ 1u)
+                                    : mbar_try_wait(bar + B_WFREE + s, use ^ 1u))) {
+                tma_v(slot, v_bar(bar, s), maps, h, (int)t0);
+                v_this = v_out[s] = true;
+                v_par[s] = use;
             }
             return kq_next && v_this;
         };
-        if (tid == 0) {
-            TRACE(0, c, 1);
-            if (c + 1 < x.nc) {
-                tma_la<MODE>(sm, bar, maps, h, (int)(t0 + C));
-                la_out = true;
-                la_par = (uint32_t)((c + 1) & 1);
-            }
-            poll_tma(false, false);
-        }
-        if (tid == 32 && c + 3 < x.nc) prefetch_chunk<Q>(maps, h, (int)(t0 + 3 * C));
-        // per-channel references from the eight warps' sums: rho_a = g_15 (end of warp
-        // 1), rho_b = g_47 (end of warp 5), g_last = g_63, and this warp's offset
-        float rhoL[8], sh[8], eR[8], dRb[8];
-        {
-            float run[8], ra[8], rb[8], off[8];
+        if (tid == 0) TRACE(0, c, 1);
+        // Per-channel references, once per channel by threads 0-127 (channel tid): the
+        // offsets of the eight 8-token groups (exclusive prefix of the warps' sums), rho_a
+        // = g_15 (end of group 1), rho_b = g_47 (end of group 5), g_last = g_63, and the
+        // factors eR = e^{rho}, dRb = e^{g_last - rho_b}, sh = e^{(rho_b - rho_a) / 2}
+        // (>= e^-80 since rho_b - rho_a >= -160) and gamma = e^{g_last}.  Rows of fac
+        // ([14][128], over the sums' rows 0-7, same column order; each thread reads its
+        // column before writing it): 0-7 offsets, 8/9 rho_a/rho_b (log2 units), 10/11
+        // e^rho_a / e^rho_b, 12 dRb, 13 sh.
+        float* fac = gsum;
+        if (tid < D) {
+            const int cgt = tid >> 3, jt = tid & 7;
+            const int p = 8 * cgt + 4 * (((jt >> 2) ^ (cgt >> 2)) & 1) + (jt & 3);  // swizzled column
+            float gs[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) run[j] = off[j] = ra[j] = rb[j] = 0.f;
+            for (int ww = 0; ww < 8; ++ww) gs[ww] = gsum[ww * D + p];
+            float run = 0.f, ra = 0.f, rb = 0.f;
 #pragma unroll
             for (int ww = 0; ww < 8; ++ww) {
-                const float4 t0v = *reinterpret_cast<const float4*>(gsum + ww * D + c0 + 4u * gsw);
-                const float4 t1v = *reinterpret_cast<const float4*>(gsum + ww * D + c0 + 4u * (gsw ^ 1u));
-                const float tv[8] = {t0v.x, t0v.y, t0v.z, t0v.w, t1v.x, t1v.y, t1v.z, t1v.w};
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    if (ww == w) off[j] = run[j];
-                    run[j] += tv[j];
-                    if (ww == 1) ra[j] = run[j];
-                    if (ww == 5) rb[j] = run[j];
-                }
+                fac[ww * D + p] = run;
+                run += gs[ww];
+                if (ww == 1) ra = run;
+                if (ww == 5) rb = run;
             }
-            // factors per channel: eR = e^{rho_h} (this warp's half), dRb = e^{g_last - rho_b},
-            // sh = e^{(rho_b - rho_a) / 2} (>= e^-80 since rho_b - rho_a >= -160)
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                rhoL[j] = (half_b ? rb[j] : ra[j]) * LOG2E;
-                eR[j] = ex2(rhoL[j]);
-                dRb[j] = ex2((run[j] - rb[j]) * LOG2E);
-                sh[j] = ex2((rb[j] - ra[j]) * (0.5f * LOG2E));
-            }
+            fac[8 * D + p] = ra * LOG2E;
+            fac[9 * D + p] = rb * LOG2E;
+            fac[10 * D + p] = ex2(ra * LOG2E);
+            fac[11 * D + p] = ex2(rb * LOG2E);
+            fac[12 * D + p] = ex2((run - rb) * LOG2E);
+            fac[13 * D + p] = ex2((rb - ra) * (0.5f * LOG2E));
+            reinterpret_cast<float*>(slot + L::S_GAM)[tid] = ex2(run * LOG2E);
+        }
+        bar_named(BAR_PREP, NPREP);
+        float rhoL[8], sh[8], eR[8], dRb[8];
+        {
+            auto row8 = [&](int row, float (&o)[8]) {  // channels c0..c0+7 of a fac row
+                const float4 u0 = *reinterpret_cast<const float4*>(fac + row * D + c0 + 4u * gsw);
+                const float4 u1 = *reinterpret_cast<const float4*>(fac + row * D + c0 + 4u * (gsw ^ 1u));
+                o[0] = u0.x, o[1] = u0.y, o[2] = u0.z, o[3] = u0.w;
+                o[4] = u1.x, o[5] = u1.y, o[6] = u1.z, o[7] = u1.w;
+            };
+            float off[8];
+            row8(w, off);
+            row8(8 + (half_b ? 1 : 0), rhoL);
+            row8(10 + (half_b ? 1 : 0), eR);
+            row8(12, dRb);
+            row8(13, sh);
 #pragma unroll
             for (int i = 0; i < 4; ++i)
 #pragma unroll
                 for (int j = 0; j < 8; ++j) g[i][j] += off[j];  // inclusive cumsum over the chunk
-            if (w == 0 && hl == 0) {
-                float4* gp = reinterpret_cast<float4*>(slot + L::S_GAM + 4 * c0);
-                gp[0] = make_float4(ex2(run[0] * LOG2E), ex2(run[1] * LOG2E), ex2(run[2] * LOG2E),
-                                    ex2(run[3] * LOG2E));
-                gp[1] = make_float4(ex2(run[4] * LOG2E), ex2(run[5] * LOG2E), ex2(run[6] * LOG2E),
-                                    ex2(run[7] * LOG2E));
-            }
         }
 
         // ============ operand images (one factor at a time, to keep registers few)
@@ -903,7 +919,6 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
             mma_commit(bar + B_AP);
             ap_out = true;
             ap_par = (uint32_t)(c & 1);
-            poll_tma(false, false);
         }
         // the next chunk's beta (without the tile): its load has until the proxy fence after
         // the inversion
@@ -917,10 +932,7 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
             }
             tc_fence_after();
         }
-        if (tid == 0) {
-            TRACE(0, c, 3);
-            poll_tma(false, false);
-        }
+        if (tid == 0) TRACE(0, c, 3);
 
         // ============ A -> (I + A)^-1 -> TB; P into the slot beside the inversion
         {
@@ -933,21 +945,24 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
                     extract_p16(tq, r, j0, smem_u32(slot + L::S_PB));
                     extract_p16(tq, r, j0 + 16, smem_u32(slot + L::S_PB));
                 }
+                if (tid == TCOPY) {  // the next chunk's copies while warps 0-1 invert
+                    if (c + 1 < x.nc) {  // LA is free since the gate barrier
+                        tma_la<MODE>(sm, bar, maps, h, (int)(t0 + C));
+                        la_out = true;
+                        la_par = (uint32_t)((c + 1) & 1);
+                    }
+                    poll_tma(false, false);
+                    if (c + 3 < x.nc) prefetch_chunk<Q>(maps, h, (int)(t0 + 3 * C));
+                }
             }, c);
         }
         fence_async_smem();
-        if (tid == 0) {
-            TRACE(0, c, 4);
-            poll_tma(false, true);  // v must be on its way before the wait below
-            if (CACHE) {  // the chunk's T diag(beta) into its cache entry
-                bulk_store(cache_entry(c) + CE_TB, sm + L::TB, 8192);
-                bulk_commit();
-            }
-        }
+        if (tid == 0) TRACE(0, c, 4);
+        if (tid == TCOPY) poll_tma(false, true);  // v must be on its way before the wait below
         {
             // the chain has read U (previous chunk) and this chunk's v tile has landed
-            const bool vok = wait_bar(bar + B_V, (uint32_t)(c & 1));
-            if (vok && tid == 0) v_out = false;
+            const bool vok = wait_bar(v_bar(bar, s), use);
+            if (vok && tid == TCOPY) v_out[s] = false;
             const bool uok = vok && wait_bar(bar + B_UFREE, (uint32_t)((c & 1) ^ 1));
             tc_fence_before();
             if (bar_named_or(BAR_PREP, NPREP, !uok)) {
@@ -956,6 +971,13 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
             }
         }
         if (tid == 0) TRACE(0, c, 5);
+        if (tid == TCOPY) {
+            if (CACHE) {  // the chunk's T diag(beta), complete since the barrier, into its entry
+                bulk_store(cache_entry(c) + CE_TB, sm + L::TB, 8192);
+                bulk_commit();
+            }
+            poll_tma(true, true);  // the next chunk's k (and q, v) must be on their way
+        }
 
         // ============ W^T = KG^T TB^T ; U'^T = V^T TB^T   (M=128, N=64, K=64)
         if (tid == 0) {
@@ -972,7 +994,6 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
             mma_commit(bar + B_WU);
             wu_out = true;
             wu_par = (uint32_t)(c & 1);
-            poll_tma(true, true);  // the next chunk's k (and q) must be on their way
         }
         {
             const bool wuok = wait_bar(bar + B_WU, (uint32_t)(c & 1));
@@ -1006,6 +1027,8 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
         if (tid == 0) {
             mbar_arrive(bar + B_FULL + s);
             TRACE(0, c, 7);
+        }
+        if (tid == TCOPY) {
             if (CACHE) {  // the slot's images (read while the chain uses them) into the entry
                 uint8_t* ce = cache_entry(c);
                 bulk_store(ce + CE_W, slot + L::S_W, 16384);
@@ -1017,12 +1040,15 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
             }
         }
     }
-    if (CACHE && tid == 0) bulk_wait_all();  // the cache entries are written
+    if (CACHE && tid == TCOPY) bulk_wait_all();  // the cache entries are written
     // after a timeout: bounded waits for what may still be in flight
     if (!ok && tid == 0) {
         if (ap_out) wait_bar(bar + B_AP, ap_par);
         if (wu_out) wait_bar(bar + B_WU, wu_par);
-        if (v_out) wait_bar(bar + B_V, v_par);
+    }
+    if (!ok && tid == TCOPY) {
+        for (int vs = 0; vs < 2; ++vs)
+            if (v_out[vs]) wait_bar(v_bar(bar, vs), v_par[vs]);
         if (la_out) wait_bar(bar + B_LA, la_par);
         if (kq_out) wait_bar(bar + B_KQ, kq_par);
     }
