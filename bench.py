@@ -307,23 +307,26 @@ def kernel_algorithmic_bytes(name, inp, path_bytes):
     """Minimum bytes one launch of kernel `name` must move for what it computes.
 
     pass 3 (forward) delivers the path's results from its inputs: the whole
-    path's algorithmic bytes.  Pass 1 (segment transitions) runs over every
-    segment that has a successor: it reads k, v, log alpha and beta of those
-    segments' tokens and writes one (B, M) pair (2 x 128 x 128 fp32) per such
-    segment and head."""
+    path's algorithmic bytes.  Pass 1 (segment transitions and chunk operands),
+    run when the plan cuts a sequence, builds every chunk's operands for pass 3
+    and the transition of every segment that has a successor: it must read q, k,
+    v, log alpha and beta of every token once and write one (B, M) pair
+    (2 x 128 x 128 fp32) per such segment and head.  The chunk cache it leaves
+    for pass 3 is an intermediate of this design and is not counted: it shows up
+    in the measured DRAM traffic instead."""
     if name != "tc_pass1_transitions":
         return path_bytes
     seg, cut = segment_plan(inp)
     if not cut:
         return 0
-    per_tok = inp.H * (inp.dk * 2 + inp.dv * 2 + inp.dk * 4 + 4)
+    per_tok = inp.H * (inp.dk * 2 * 2 + inp.dv * 2 + inp.dk * 4 + 4)
     toks = segs = 0
     for L in inp.seq_lens:
         L = int(L)
         nch = (L + 63) // 64
         g = max(1, (nch + seg - 1) // seg)
         segs += g - 1
-        toks += min(L, (g - 1) * seg * 64)
+        toks += L
     return toks * per_tok + segs * inp.H * 2 * inp.dk * inp.dv * 4
 
 

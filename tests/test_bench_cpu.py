@@ -42,10 +42,10 @@ def test_pass1_algorithmic_bytes_follow_the_segment_plan():
     seg, cut = bench.segment_plan(inp)
     assert cut and seg == 443
     segs = -(-16384 // seg)
-    # pass 1 runs on every segment but the last: k, v bf16; log alpha, beta fp32 of
-    # those segments' tokens, and one (B, M) pair per such segment and head
-    per_tok = 8 * (128 * 2 + 128 * 2 + 128 * 4 + 4)
-    want = (segs - 1) * seg * 64 * per_tok + (segs - 1) * 8 * 2 * 128 * 128 * 4
+    # pass 1 reads q, k, v (bf16), log alpha and beta (fp32) of every token once and
+    # writes one (B, M) pair per segment with a successor and head
+    per_tok = 8 * (128 * 2 * 3 + 128 * 4 + 4)
+    want = 16384 * 64 * per_tok + (segs - 1) * 8 * 2 * 128 * 128 * 4
     assert bench.kernel_algorithmic_bytes("tc_pass1_transitions", inp, 123) == want
     assert bench.kernel_algorithmic_bytes("tc_pass3_forward", inp, 123) == 123
     assert bench.kernel_algorithmic_bytes("tc_pass1_transitions", _inp(64 * 4, 8), 1) == 0
