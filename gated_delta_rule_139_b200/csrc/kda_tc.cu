@@ -206,7 +206,8 @@ enum Bars : int {
     B_LA = 15,     // prep: a chunk's log alpha tile landed (TMA; one per chunk)
     B_KQ = 16,     // prep: a chunk's k (and q) tiles landed in its slot (TMA; one per chunk)
     B_V1 = 17,     // prep: a chunk's v tile landed in slot 1
-    NBARS = 18
+    B_WREAD = 18,  // chain: the chunk's W^T has left TMEM (the prep may overwrite its columns)
+    NBARS = 19
 };
 
 // TMEM columns (512 allocated).
@@ -846,7 +847,14 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
             fac[13 * D + p] = ex2((rb - ra) * (0.5f * LOG2E));
             reinterpret_cast<float*>(slot + L::S_GAM)[tid] = ex2(run * LOG2E);
         }
-        bar_named(BAR_PREP, NPREP);
+        // thread 0: the previous chunk's W and U' products, which read KG and TB, are done
+        // before this chunk's images (after this barrier) overwrite them
+        const bool wu_ok = tid != 0 || c == 0 || wait_bar(bar + B_WU, (uint32_t)((c - 1) & 1));
+        if (wu_ok && tid == 0) wu_out = false;
+        if (bar_named_or(BAR_PREP, NPREP, !wu_ok)) {
+            ok = false;
+            break;
+        }
         float rhoL[8], sh[8], eR[8], dRb[8];
         {
             auto row8 = [&](int row, float (&o)[8]) {  // channels c0..c0+7 of a fac row
@@ -905,7 +913,13 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
         }
         fence_async_smem();
         tc_fence_before();
-        bar_named(BAR_PREP, NPREP);
+        // thread 0: the chain has taken the previous chunk's W^T out of the TMEM columns
+        // the [A;P] product is about to overwrite
+        const bool wr_ok = tid != 0 || c == 0 || wait_bar(bar + B_WREAD, (uint32_t)((c - 1) & 1));
+        if (bar_named_or(BAR_PREP, NPREP, !wr_ok)) {
+            ok = false;
+            break;
+        }
         if (tid == 0) TRACE(0, c, 2);
 
         // ============ [A;P] = X1 . BT^T   (M=128, N=96, K=128)
@@ -946,6 +960,12 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
                     extract_p16(tq, r, j0 + 16, smem_u32(slot + L::S_PB));
                 }
                 if (tid == TCOPY) {  // the next chunk's copies while warps 0-1 invert
+                    // the previous chunk's W image, written by the chain, into its cache entry
+                    // (before the next k/q/v copies, which wait for it to be read, reuse the slot)
+                    if (CACHE && c > 0 && wait_bar(bar + B_WREAD, (uint32_t)((c - 1) & 1))) {
+                        bulk_store(cache_entry(c - 1) + CE_W, sm + (s ^ 1) * L::SLOT + L::S_W, 16384);
+                        bulk_commit();
+                    }
                     if (c + 1 < x.nc) {  // LA is free since the gate barrier
                         tma_la<MODE>(sm, bar, maps, h, (int)(t0 + C));
                         la_out = true;
@@ -972,8 +992,15 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
         }
         if (tid == 0) TRACE(0, c, 5);
         if (tid == TCOPY) {
-            if (CACHE) {  // the chunk's T diag(beta), complete since the barrier, into its entry
-                bulk_store(cache_entry(c) + CE_TB, sm + L::TB, 8192);
+            if (CACHE) {  // the chunk's T diag(beta), complete since the barrier, into its entry,
+                          // then the slot's images but W (the chain writes W after the hand-off)
+                uint8_t* ce = cache_entry(c);
+                bulk_store(ce + CE_TB, sm + L::TB, 8192);
+                bulk_commit();
+                bulk_store(ce + CE_KD, slot + L::S_KD, 16384);
+                bulk_store(ce + CE_QT, slot + L::S_QT, 16384);
+                bulk_store(ce + CE_PB, slot + L::S_PB, 8192);
+                bulk_store(ce + CE_GAM, slot + L::S_GAM, 512);
                 bulk_commit();
             }
             poll_tma(true, true);  // the next chunk's k (and q, v) must be on their way
@@ -994,53 +1021,20 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
             mma_commit(bar + B_WU);
             wu_out = true;
             wu_par = (uint32_t)(c & 1);
-        }
-        {
-            const bool wuok = wait_bar(bar + B_WU, (uint32_t)(c & 1));
-            if (wuok && tid == 0) wu_out = false;
-            if (bar_named_or(BAR_PREP, NPREP, !wuok)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-        }
-        if (tid == 0) TRACE(0, c, 6);
-        // W^T (lane = channel) -> bf16 MN-major image (K rows = channels) in the slot
-        {
-            const int ch = (w & 3) * 32 + lane, r0 = 32 * (w >> 2);
-            float v0[16], v1[16];
-            tmem_ld16(tq + TM_W + r0, v0);
-            tmem_ld16(tq + TM_W + r0 + 16, v1);
-            tmem_wait16(v0);
-            tmem_wait16(v1);
-            const uint32_t wb = smem_u32(slot + L::S_W);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float* p = k < 2 ? v0 + 8 * k : v1 + 8 * (k - 2);
-                st_shared_v4(wb + mnmajor_chunk_off(ch, (r0 >> 3) + k, 128), pack_bf16(p[0], p[1]),
-                             pack_bf16(p[2], p[3]), pack_bf16(p[4], p[5]), pack_bf16(p[6], p[7]));
-            }
-        }
-        fence_async_smem();
-        tc_fence_before();
-        bar_named(BAR_PREP, NPREP);
-        if (tid == 0) {
+            // the slot is complete but for W, which the chain stages from TMEM itself once
+            // the products are done: hand it over now
             mbar_arrive(bar + B_FULL + s);
             TRACE(0, c, 7);
         }
-        if (tid == TCOPY) {
-            if (CACHE) {  // the slot's images (read while the chain uses them) into the entry
-                uint8_t* ce = cache_entry(c);
-                bulk_store(ce + CE_W, slot + L::S_W, 16384);
-                bulk_store(ce + CE_KD, slot + L::S_KD, 16384);
-                bulk_store(ce + CE_QT, slot + L::S_QT, 16384);
-                bulk_store(ce + CE_PB, slot + L::S_PB, 8192);
-                bulk_store(ce + CE_GAM, slot + L::S_GAM, 512);
-                bulk_commit();
-            }
-        }
     }
-    if (CACHE && tid == TCOPY) bulk_wait_all();  // the cache entries are written
+    if (CACHE && tid == TCOPY) {
+        // the last chunk's W image, then every cache entry is written
+        if (ok && x.nc > 0 && wait_bar(bar + B_WREAD, (uint32_t)((x.nc - 1) & 1))) {
+            bulk_store(cache_entry(x.nc - 1) + CE_W, sm + ((x.nc - 1) & 1) * L::SLOT + L::S_W, 16384);
+            bulk_commit();
+        }
+        bulk_wait_all();
+    }
     // after a timeout: bounded waits for what may still be in flight
     if (!ok && tid == 0) {
         if (ap_out) wait_bar(bar + B_AP, ap_par);
@@ -1055,6 +1049,32 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
 }
 
 // ---------------------------------------------------------------- chain: forward (warps 8-11)
+// Chain warps, at the start of chunk c (its slot full): wait for the prep's W product and
+// write W^T (TMEM, lane = channel) into the slot's W piece as the bf16 MN-major image (K rows
+// = channels) that the chain's U product reads.  The W piece held the chunk's v tile, which
+// the prep's U' product (committed with W) has read.  The caller's next named barrier makes
+// the image visible to the chain's products; ct == 0 then arrives on B_WREAD.
+__device__ bool chain_stage_w(const Ctx& x, uint8_t* slot_w, int64_t c, int ct) {
+    if (!wait_bar(x.bar + B_WU, (uint32_t)(c & 1))) return false;
+    tc_fence_after();
+    const int cw = ct >> 5, chn = (cw & 3) * 32 + (ct & 31), r0 = 32 * (cw >> 2);
+    const uint32_t tq = x.tmem + ((uint32_t)((cw & 3) * 32) << 16);
+    float v0[16], v1[16];
+    tmem_ld16(tq + TM_W + r0, v0);
+    tmem_ld16(tq + TM_W + r0 + 16, v1);
+    tmem_wait16(v0);
+    tmem_wait16(v1);
+    const uint32_t wb = smem_u32(slot_w);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const float* p = k < 2 ? v0 + 8 * k : v1 + 8 * (k - 2);
+        st_shared_v4(wb + mnmajor_chunk_off(chn, (r0 >> 3) + k, 128), pack_bf16(p[0], p[1]),
+                     pack_bf16(p[2], p[3]), pack_bf16(p[4], p[5]), pack_bf16(p[6], p[7]));
+    }
+    fence_async_smem();
+    return true;
+}
+
 __device__ void chain_fwd(const Ctx& x, const TcArgs& a, const TcMaps& maps, int tid) {
     using L = Lay<FWD>;
     uint8_t* sm = x.sm;
@@ -1172,6 +1192,7 @@ __device__ void chain_fwd(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
         s_waited = true;
         tc_fence_after();
         if (ct == 0) TRACE(1, c, 1);
+        wok = wok && chain_stage_w(x, slot + L::S_W, c, ct);
         if (wok) {  // bf16 S^T -> SB; S^T *= gamma (per column = key channel) in place
             const float* gam = reinterpret_cast<const float*>(slot + L::S_GAM);
             stage_cols_tmem<4>(tq + TM_S + 64 * ch, tq + TM_SB + 32 * ch, 64 * ch, gam, true);
@@ -1184,6 +1205,7 @@ __device__ void chain_fwd(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
         }
         if (ct == 0) {
             TRACE(1, c, 2);
+            mbar_arrive(bar + B_WREAD);
             tc_fence_after();
             const uint32_t wb = smem_u32(slot + L::S_W), qt = smem_u32(slot + L::S_QT);
             constexpr uint32_t id_neg = idesc_bf16(128, 64, false, true, true);
@@ -1340,6 +1362,7 @@ __device__ void chain_trans(const Ctx& x, const TcArgs& a, int tid) {
         if (c > 0) wok = wok && wait_bar(bar + B_S, (uint32_t)((c - 1) & 1));
         tc_fence_after();
         if (ct == 0) TRACE(1, c, 1);
+        wok = wok && chain_stage_w(x, slot + L::S_W, c, ct);
         for (int step = 0; step < 2 && ok; ++step) {  // 0: B, 1: M
             const uint32_t tstate = step == 0 ? TT_B : TT_M;
             if (wok) {
@@ -1353,6 +1376,7 @@ __device__ void chain_trans(const Ctx& x, const TcArgs& a, int tid) {
             }
             if (ct == 0) {
                 TRACE(1, c, 2 + 3 * step);
+                if (step == 0) mbar_arrive(bar + B_WREAD);
                 tc_fence_after();
                 // B step: U^T -= B^T W^T on top of U'^T;  M step: U^T = -M^T W^T
 #pragma unroll
@@ -1424,9 +1448,12 @@ __device__ void chain_dump(const Ctx& x, const TcArgs& a, int tid) {
     const int h = x.h, H = a.H;
     for (int64_t c = 0; c < x.nc; ++c) {
         const int s = (int)(c & 1);
-        const uint8_t* slot = sm + s * L::SLOT;
-        const bool wok = wait_bar(bar + B_FULL + s, (uint32_t)((c >> 1) & 1));
+        uint8_t* slot = sm + s * L::SLOT;
+        bool wok = wait_bar(bar + B_FULL + s, (uint32_t)((c >> 1) & 1));
+        wok = wok && chain_stage_w(x, slot + L::S_W, c, ct);
+        tc_fence_before();
         if (bar_named_or(BAR_CHAIN, NCHAIN, !wok)) break;
+        if (ct == 0) mbar_arrive(bar + B_WREAD);
         tc_fence_after();
         uint8_t* ent = a.dump + ((x.sg.c_base + c) * H + h) * (int64_t)kChunkImageBytes;
         auto copy = [&](uint32_t dst, uint32_t src, uint32_t bytes) {
