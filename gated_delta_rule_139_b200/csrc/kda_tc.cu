@@ -601,9 +601,29 @@ __device__ __forceinline__ void unpack_bf16x8(const uint4 raw, float (&f)[8]) {
     }
 }
 // 8 products a[i] * b[i], bf16, as one 16-byte shared store
+// Element-wise r = a * b and r = a * b + c over 8 fp32 values, two per packed f32x2
+// instruction: each element is rounded exactly as the scalar operation rounds it.
+__device__ __forceinline__ void mul8(float (&r)[8], const float (&a)[8], const float (&b)[8]) {
+#pragma unroll
+    for (int p = 0; p < 8; p += 2)
+        asm("{\n .reg .b64 x, y, z;\n mov.b64 x, {%2, %3};\n mov.b64 y, {%4, %5};\n"
+            " mul.rn.f32x2 z, x, y;\n mov.b64 {%0, %1}, z;\n}"
+            : "=f"(r[p]), "=f"(r[p + 1])
+            : "f"(a[p]), "f"(a[p + 1]), "f"(b[p]), "f"(b[p + 1]));
+}
+__device__ __forceinline__ void fma8(float (&r)[8], const float (&a)[8], float b, const float (&c)[8]) {
+#pragma unroll
+    for (int p = 0; p < 8; p += 2)
+        asm("{\n .reg .b64 x, y, z, w;\n mov.b64 x, {%2, %3};\n mov.b64 y, {%4, %4};\n"
+            " mov.b64 z, {%5, %6};\n fma.rn.f32x2 w, x, y, z;\n mov.b64 {%0, %1}, w;\n}"
+            : "=f"(r[p]), "=f"(r[p + 1])
+            : "f"(a[p]), "f"(a[p + 1]), "f"(b), "f"(c[p]), "f"(c[p + 1]));
+}
 __device__ __forceinline__ void st_prod8(uint32_t addr, const float (&a)[8], const float (&b)[8]) {
-    st_shared_v4(addr, pack_bf16(a[0] * b[0], a[1] * b[1]), pack_bf16(a[2] * b[2], a[3] * b[3]),
-                 pack_bf16(a[4] * b[4], a[5] * b[5]), pack_bf16(a[6] * b[6], a[7] * b[7]));
+    float r[8];
+    mul8(r, a, b);
+    st_shared_v4(addr, pack_bf16(r[0], r[1]), pack_bf16(r[2], r[3]), pack_bf16(r[4], r[5]),
+                 pack_bf16(r[6], r[7]));
 }
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
     uint4 v;
@@ -822,7 +842,7 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
         // factors eR = e^{rho}, dRb = e^{g_last - rho_b}, sh = e^{(rho_b - rho_a) / 2}
         // (>= e^-80 since rho_b - rho_a >= -160) and gamma = e^{g_last}.  Rows of fac
         // ([14][128], over the sums' rows 0-7, same column order; each thread reads its
-        // column before writing it): 0-7 offsets, 8/9 rho_a/rho_b (log2 units), 10/11
+        // column before writing it): 0-7 offsets, 8/9 -rho_a/-rho_b (log2 units), 10/11
         // e^rho_a / e^rho_b, 12 dRb, 13 sh.
         float* fac = gsum;
         if (tid < D) {
@@ -839,8 +859,8 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
                 if (ww == 1) ra = run;
                 if (ww == 5) rb = run;
             }
-            fac[8 * D + p] = ra * LOG2E;
-            fac[9 * D + p] = rb * LOG2E;
+            fac[8 * D + p] = -(ra * LOG2E);
+            fac[9 * D + p] = -(rb * LOG2E);
             fac[10 * D + p] = ex2(ra * LOG2E);
             fac[11 * D + p] = ex2(rb * LOG2E);
             fac[12 * D + p] = ex2((run - rb) * LOG2E);
@@ -855,7 +875,7 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
             ok = false;
             break;
         }
-        float rhoL[8], sh[8], eR[8], dRb[8];
+        float nrho[8], sh[8], eR[8], dRb[8];
         {
             auto row8 = [&](int row, float (&o)[8]) {  // channels c0..c0+7 of a fac row
                 const float4 u0 = *reinterpret_cast<const float4*>(fac + row * D + c0 + 4u * gsw);
@@ -865,7 +885,7 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
             };
             float off[8];
             row8(w, off);
-            row8(8 + (half_b ? 1 : 0), rhoL);
+            row8(8 + (half_b ? 1 : 0), nrho);
             row8(10 + (half_b ? 1 : 0), eR);
             row8(12, dRb);
             row8(13, sh);
@@ -882,32 +902,31 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
             for (int i = 0; i < 4; ++i) {
                 const int rr = 4 * hl + i;  // row within the warp's 8-row swizzle atom
                 const uint32_t ro = (uint32_t)rr * 128u + ((uint32_t)((cg & 7) ^ rr) << 4);
-                float kf[8], f[8], p[8];
+                float kf[8], f[8], p[8], t[8];
                 unpack_bf16x8(kr[i], kf);
+                fma8(t, g[i], LOG2E, nrho);  // (g - rho_h) log2 e
 #pragma unroll
-                for (int j = 0; j < 8; ++j) f[j] = ex2(fmaf(g[i][j], LOG2E, -rhoL[j]));  // e^{g-rho_h}
+                for (int j = 0; j < 8; ++j) f[j] = ex2(t[j]);  // e^{g-rho_h}
                 st_prod8(a_x1 + ro, kf, f);
                 if (Q) {
                     unpack_bf16x8(qr[i], p);
                     st_prod8(a_x1 + 8192u + ro, p, f);
                 }
-#pragma unroll
-                for (int j = 0; j < 8; ++j) f[j] *= eR[j];  // e^{g}
+                mul8(f, f, eR);  // e^{g}
                 st_prod8(a_kg + ro, kf, f);
                 if (Q) st_prod8(a_slot + L::S_QT + ro, p, f);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) f[j] = ex2(fmaf(-g[i][j], LOG2E, rhoL[j]));  // e^{rho_h-g}
+                for (int j = 0; j < 8; ++j) f[j] = ex2(-t[j]);  // e^{rho_h-g}
                 st_prod8(a_bt + ro, kf, f);
                 if (!half_b) {
                     // e^{rho_b - g} for the first half's keys (cross-half block) as
                     // (e^{rho_a - g} sh) sh: an intermediate below the normal range means a
                     // true value below it, so flushing to zero is the right limit
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) f[j] = (f[j] * sh[j]) * sh[j];
+                    mul8(f, f, sh);
+                    mul8(f, f, sh);
                     st_prod8(a_bt + 8192u + ro, kf, f);
                 }
-#pragma unroll
-                for (int j = 0; j < 8; ++j) f[j] *= dRb[j];  // e^{g_last - g}
+                mul8(f, f, dRb);  // e^{g_last - g}
                 st_prod8(a_slot + L::S_KD + ro, kf, f);
             }
         }
