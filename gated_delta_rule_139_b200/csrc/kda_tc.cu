@@ -250,6 +250,24 @@ __device__ __forceinline__ float ex2(float x) {
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
+// (r0, r1) = (a0 * b0, a1 * b1) and (a0 + b0, a1 + b1) in one packed f32x2 instruction; each
+// element is rounded exactly as the scalar operation rounds it
+__device__ __forceinline__ void mul2(float& r0, float& r1, float a0, float a1, float b0, float b1) {
+    asm("{\n .reg .b64 x, y, z;\n mov.b64 x, {%2, %3};\n mov.b64 y, {%4, %5};\n"
+        " mul.rn.f32x2 z, x, y;\n mov.b64 {%0, %1}, z;\n}"
+        : "=f"(r0), "=f"(r1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ void add2(float& r0, float& r1, float a0, float a1, float b0, float b1) {
+    asm("{\n .reg .b64 x, y, z;\n mov.b64 x, {%2, %3};\n mov.b64 y, {%4, %5};\n"
+        " add.rn.f32x2 z, x, y;\n mov.b64 {%0, %1}, z;\n}"
+        : "=f"(r0), "=f"(r1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ void add8(float (&r)[8], const float (&a)[8], const float (&b)[8]) {
+#pragma unroll
+    for (int p = 0; p < 8; p += 2) add2(r[p], r[p + 1], a[p], a[p + 1], b[p], b[p + 1]);
+}
 
 
 
@@ -285,10 +303,8 @@ __device__ __forceinline__ void stage_cols_tmem(uint32_t tm, uint32_t tb, int co
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const float4 gg = g4[i];
-                v[b][4 * i + 0] *= gg.x;
-                v[b][4 * i + 1] *= gg.y;
-                v[b][4 * i + 2] *= gg.z;
-                v[b][4 * i + 3] *= gg.w;
+                mul2(v[b][4 * i + 0], v[b][4 * i + 1], v[b][4 * i + 0], v[b][4 * i + 1], gg.x, gg.y);
+                mul2(v[b][4 * i + 2], v[b][4 * i + 3], v[b][4 * i + 2], v[b][4 * i + 3], gg.z, gg.w);
             }
             tmem_st16(tm + 16 * b, v[b]);
         }
@@ -605,11 +621,7 @@ __device__ __forceinline__ void unpack_bf16x8(const uint4 raw, float (&f)[8]) {
 // instruction: each element is rounded exactly as the scalar operation rounds it.
 __device__ __forceinline__ void mul8(float (&r)[8], const float (&a)[8], const float (&b)[8]) {
 #pragma unroll
-    for (int p = 0; p < 8; p += 2)
-        asm("{\n .reg .b64 x, y, z;\n mov.b64 x, {%2, %3};\n mov.b64 y, {%4, %5};\n"
-            " mul.rn.f32x2 z, x, y;\n mov.b64 {%0, %1}, z;\n}"
-            : "=f"(r[p]), "=f"(r[p + 1])
-            : "f"(a[p]), "f"(a[p + 1]), "f"(b[p]), "f"(b[p + 1]));
+    for (int p = 0; p < 8; p += 2) mul2(r[p], r[p + 1], a[p], a[p + 1], b[p], b[p + 1]);
 }
 __device__ __forceinline__ void fma8(float (&r)[8], const float (&a)[8], float b, const float (&c)[8]) {
 #pragma unroll
@@ -771,22 +783,20 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
                     kr[i] = make_uint4(0u, 0u, 0u, 0u);
                     if (Q) qr[i] = make_uint4(0u, 0u, 0u, 0u);
                 }
-                const float la8[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
+                const float cl[8] = {clamp_gate(l0.x), clamp_gate(l0.y), clamp_gate(l0.z), clamp_gate(l0.w),
+                                     clamp_gate(l1.x), clamp_gate(l1.y), clamp_gate(l1.z), clamp_gate(l1.w)};
+                add8(acc, acc, cl);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    acc[j] += clamp_gate(la8[j]);
-                    g[i][j] = acc[j];
-                }
+                for (int j = 0; j < 8; ++j) g[i][j] = acc[j];
             }
             // the second half-warp's tokens follow the first's: add the partner's total
+            float pt[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const float pt = __shfl_xor_sync(0xffffffffu, acc[j], 16);
-                if (hl) {
-                    acc[j] += pt;
+            for (int j = 0; j < 8; ++j) pt[j] = __shfl_xor_sync(0xffffffffu, acc[j], 16);
+            if (hl) {
+                add8(acc, acc, pt);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) g[i][j] += pt;
-                }
+                for (int i = 0; i < 4; ++i) add8(g[i], g[i], pt);
             }
             if (hl) {  // the warp's 8-token sums
                 *reinterpret_cast<float4*>(gsum + w * D + c0 + 4u * gsw) =
@@ -890,9 +900,7 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
             row8(12, dRb);
             row8(13, sh);
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 8; ++j) g[i][j] += off[j];  // inclusive cumsum over the chunk
+            for (int i = 0; i < 4; ++i) add8(g[i], g[i], off);  // inclusive cumsum over the chunk
         }
 
         // ============ operand images (one factor at a time, to keep registers few)
