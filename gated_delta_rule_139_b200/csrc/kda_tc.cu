@@ -13,16 +13,23 @@
 //
 // Kernels (one launch each, all on the caller's stream):
 //   seg_setup          : segment table from cu_seqlens (or B x T) on the device.
-//   chunk_kernel<TRANS>: "pass 1", per (segment, head) the transition (B, M) of
-//                        the segment: the chunk loop applied to B from 0 and to M
-//                        from I.
+//   chunk_kernel<TRANS_CACHE>: "pass 1" of kda_fwd's segmented plan, per (segment,
+//                        head) the transition (B, M) of the segment -- the chunk loop
+//                        applied to B from 0 and to M from I -- and every chunk's
+//                        operand images bulk-stored to the chunk cache.
+//   chunk_kernel<TRANS>: the transitions alone (kda_transition, kda_fwd_noalloc).
 //   seg_scan           : S_in(j+1) = M_j S_in(j) + B_j, sequential over the
 //                        segments of a sequence, parallel over (sequence, head,
 //                        8-row block).
-//   chunk_kernel<FWD>  : "pass 3", per (segment, head) the chunk loop from the
-//                        true incoming state, writing o and the final state.
+//   cached_kernel      : "pass 3" of the segmented plan, the state chain and the
+//                        output from the true incoming state, each chunk's operands
+//                        read back from the chunk cache.
+//   chunk_kernel<FWD>  : "pass 3" without a cache (unsegmented plans, the
+//                        no-allocation entry point): the whole chunk loop.
 //   chunk_kernel<DUMP> : test aid: every chunk's operand images (W, U', K_dec,
 //                        Q~, P, gamma) copied to global memory.
+//   wait_probe, guard_check: the bounded-wait self-test, and (debug builds) the
+//                        check of the workspace guard bands.
 //
 // Per chunk of C = 64 tokens (g = in-chunk inclusive cumsum of the clamped
 // log-gates, per key channel), everything in the transposed orientation so
@@ -40,15 +47,17 @@
 // K e^{g_last - g} are products of factors whose exact value is <= 1.
 //
 // Warp roles inside each CTA (one CTA per SM, 16 warps):
-//   warps 0-7 ("prep"): the chunk-local work of chunk c+1 -- raw inputs by
-//     128-bit loads one chunk ahead, gates, operand images, [A;P] product,
-//     inversion, W and U' products -- into a two-slot shared-memory ring
-//     (W, Q~, K_dec, P, gamma) and the U accumulator in tensor memory;
-//   warps 8-15 ("chain"): the state chain of chunk c -- bf16 copy of S,
-//     U -= S W, S += U K_dec, O = S Q~ + U P and the output epilogue; for the
-//     transitions the same two products on B and then on M.
-// The chain waits only on the ring, so one chunk's chunk-local work overlaps
-// the previous chunk's state products.
+//   warps 0-7 ("prep"): the chunk-local work of chunk c+1 -- gates, operand images,
+//     [A;P] product, inversion, W and U' products -- into a two-slot shared-memory
+//     ring (Q~, K_dec, P, gamma; the v tile in the W piece) and the W and U
+//     accumulators in tensor memory.  One prep thread (the copy thread) issues every
+//     TMA load of the raw tiles (log alpha + beta, k, q, v, a chunk ahead) and every
+//     bulk store to the chunk cache;
+//   warps 8-15 ("chain"): the state chain of chunk c -- W from tensor memory into
+//     the slot, bf16 copy of S, U -= S W, S += U K_dec, O = S Q~ + U P and the output
+//     epilogue; for the transitions the same two products on B and then on M.
+// The two groups meet only at mbarriers (slot full / empty, U and W columns free),
+// so one chunk's chunk-local work overlaps the previous chunk's state products.
 #include <cuda_bf16.h>
 #include <stdint.h>
 #include <string.h>
