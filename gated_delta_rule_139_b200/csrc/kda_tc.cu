@@ -352,10 +352,15 @@ __device__ __forceinline__ void tma_store_tile(const CUtensorMap* map, const voi
         : "memory");
 }
 // plain bulk copies: shared -> global (bulk group), global -> shared (mbarrier)
-__device__ __forceinline__ void bulk_store(void* gdst, const void* ssrc, uint32_t bytes) {
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst),
-                 "r"(smem_u32(ssrc)), "r"(bytes)
-                 : "memory");
+// Bulk copy shared -> global (bulk async-group) whose lines are the first to leave L2: the
+// chunk cache is read back only after the whole pass, so keeping it in L2 would only push
+// out the prefetched input tiles
+__device__ __forceinline__ void bulk_store_stream(void* gdst, const void* ssrc, uint32_t bytes) {
+    asm volatile(
+        "{\n .reg .b64 pol;\n createpolicy.fractional.L2::evict_first.b64 pol, 1.0;\n"
+        " cp.async.bulk.global.shared::cta.bulk_group.L2::cache_hint [%0], [%1], %2, pol;\n}" ::"l"(gdst),
+        "r"(smem_u32(ssrc)), "r"(bytes)
+        : "memory");
 }
 __device__ __forceinline__ void bulk_load(void* sdst, const void* gsrc, uint32_t bytes, void* bar) {
     asm volatile(
@@ -999,7 +1004,7 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
                     // the previous chunk's W image, written by the chain, into its cache entry
                     // (before the next k/q/v copies, which wait for it to be read, reuse the slot)
                     if (CACHE && c > 0 && wait_bar(bar + B_WREAD, (uint32_t)((c - 1) & 1))) {
-                        bulk_store(cache_entry(c - 1) + CE_W, sm + (s ^ 1) * L::SLOT + L::S_W, 16384);
+                        bulk_store_stream(cache_entry(c - 1) + CE_W, sm + (s ^ 1) * L::SLOT + L::S_W, 16384);
                         bulk_commit();
                     }
                     if (c + 1 < x.nc) {  // LA is free since the gate barrier
@@ -1031,12 +1036,12 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
             if (CACHE) {  // the chunk's T diag(beta), complete since the barrier, into its entry,
                           // then the slot's images but W (the chain writes W after the hand-off)
                 uint8_t* ce = cache_entry(c);
-                bulk_store(ce + CE_TB, sm + L::TB, 8192);
+                bulk_store_stream(ce + CE_TB, sm + L::TB, 8192);
                 bulk_commit();
-                bulk_store(ce + CE_KD, slot + L::S_KD, 16384);
-                bulk_store(ce + CE_QT, slot + L::S_QT, 16384);
-                bulk_store(ce + CE_PB, slot + L::S_PB, 8192);
-                bulk_store(ce + CE_GAM, slot + L::S_GAM, 512);
+                bulk_store_stream(ce + CE_KD, slot + L::S_KD, 16384);
+                bulk_store_stream(ce + CE_QT, slot + L::S_QT, 16384);
+                bulk_store_stream(ce + CE_PB, slot + L::S_PB, 8192);
+                bulk_store_stream(ce + CE_GAM, slot + L::S_GAM, 512);
                 bulk_commit();
             }
             poll_tma(true, true);  // the next chunk's k (and q, v) must be on their way
@@ -1066,7 +1071,7 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
     if (CACHE && tid == TCOPY) {
         // the last chunk's W image, then every cache entry is written
         if (ok && x.nc > 0 && wait_bar(bar + B_WREAD, (uint32_t)((x.nc - 1) & 1))) {
-            bulk_store(cache_entry(x.nc - 1) + CE_W, sm + ((x.nc - 1) & 1) * L::SLOT + L::S_W, 16384);
+            bulk_store_stream(cache_entry(x.nc - 1) + CE_W, sm + ((x.nc - 1) & 1) * L::SLOT + L::S_W, 16384);
             bulk_commit();
         }
         bulk_wait_all();
