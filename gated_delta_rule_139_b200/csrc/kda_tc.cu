@@ -657,7 +657,7 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
     return v;
 }
 
-// The prep warps' TMA issues for chunk index cc (tokens t0 = t_begin + 64 cc of head h):
+// The copy thread's TMA issues for chunk index cc (tokens t0 = t_begin + 64 cc of head h):
 // its log alpha tile into LA, its k (and q) tiles into its slot's K_dec (and Q~)
 // pieces, its v tile into its slot's W piece, each on its own mbarrier; and the L2
 // prefetch of a later chunk's tiles.
@@ -698,7 +698,8 @@ __device__ __forceinline__ void prefetch_chunk(const TcMaps& maps, int h, int t0
 }
 
 // Prep warps: for every chunk of the unit, in order, the chunk-local work into the
-// chunk's ring slot (and U' into the U accumulator).  Thread mapping for the
+// chunk's ring slot (and W, U' into their TMEM accumulators; the chain stages W into the
+// slot).  Thread mapping for the
 // elementwise phases: warp w, lane l = 16 hl + cg holds tokens 8w + 4hl + i (i < 4)
 // and channels 8cg .. 8cg + 7.
 template <int MODE>
@@ -726,8 +727,9 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
     // this thread's row of the raw [64][128] tiles: token 8w + 4hl + i, channels c0..
     const uint32_t raw_row0 = (uint32_t)(8 * w + 4 * hl) * 128u + (uint32_t)c0;
 
-    // pass 1 with the chunk cache: chunk c's entry (thread 0 bulk-stores TB after the
-    // inversion and the slot's images once the slot is full)
+    // pass 1 with the chunk cache: chunk c's entry (the copy thread bulk-stores TB and the
+    // slot's images but W after the barrier that follows the inversion, and W, which the
+    // chain writes into the slot, one chunk later)
     constexpr bool CACHE = MODE == TRANS_CACHE;
     auto cache_entry = [&](int64_t cc) {
         return a.cache + ((x.sg.c_base + cc) * H + h) * (int64_t)kCacheEntryBytes;
