@@ -202,12 +202,11 @@ static_assert(Lay<FWD>::BYTES <= 232448 && Lay<TRANS>::BYTES <= 232448, "shared 
 // mbarriers (index into BAR)
 enum Bars : int {
     B_AP = 0,      // prep: [A;P] product done
-    B_WU = 1,      // prep: W and U' products done
+    B_WU = 1,      // W and U' products done (issued by the chain, waited for by both groups)
     B_V = 2,       // prep: a chunk's v tile landed in slot 0 (TMA; one per use of the slot)
     B_FULL = 3,    // [2] ring slot filled (prep -> chain)
     B_EMPTY = 5,   // [2] the chain's products have read the slot (MMA commit)
     B_WFREE = 7,   // [2] the slot's W area is free again (output tile stored)
-    B_UFREE = 9,   // the chain has read U: the prep may write the next U'
     B_U = 10,      // chain: U product done
     B_S = 11,      // chain: state update done
     B_O = 12,      // [2] chain: output products of O buffer 0/1 done
@@ -734,12 +733,12 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
     auto cache_entry = [&](int64_t cc) {
         return a.cache + ((x.sg.c_base + cc) * H + h) * (int64_t)kCacheEntryBytes;
     };
-    // Thread 0 issues the tensor-core products; the copy thread TCOPY (lane 0 of warp
+    // Thread 0 issues the [A;P] product; the copy thread TCOPY (lane 0 of warp
     // 4, whose share of the inversion is the shortest) issues every TMA load and bulk
     // store, so that no warp with a full share of a phase also carries the copies.
     // Each keeps what it has in flight, for the waits after a timeout.
-    bool ap_out = false, wu_out = false, v_out[2] = {false, false}, la_out = false, kq_out = false;
-    uint32_t ap_par = 0, wu_par = 0, v_par[2] = {0, 0}, la_par = 0, kq_par = 0;
+    bool ap_out = false, v_out[2] = {false, false}, la_out = false, kq_out = false;
+    uint32_t ap_par = 0, v_par[2] = {0, 0}, la_par = 0, kq_par = 0;
     // In the transition modes chunk c+1's v tile goes into its slot together with its k
     // tile (the slot's W piece is free once its k piece is); the forward and dump chains
     // put chunk c-2's output tile there, so chunk c's v waits for it in chunk c.
@@ -896,7 +895,6 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
         // thread 0: the previous chunk's W and U' products, which read KG and TB, are done
         // before this chunk's images (after this barrier) overwrite them
         const bool wu_ok = tid != 0 || c == 0 || wait_bar(bar + B_WU, (uint32_t)((c - 1) & 1));
-        if (wu_ok && tid == 0) wu_out = false;
         if (bar_named_or(BAR_PREP, NPREP, !wu_ok)) {
             ok = false;
             break;
@@ -1021,19 +1019,15 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
         }
         fence_async_smem();
         if (tid == 0) TRACE(0, c, 4);
-        if (tid == TCOPY) poll_tma(false, true);  // v must be on its way before the wait below
-        {
-            // the chain has read U (previous chunk) and this chunk's v tile has landed
-            const bool vok = wait_bar(v_bar(bar, s), use);
-            if (vok && tid == TCOPY) v_out[s] = false;
-            const bool uok = vok && wait_bar(bar + B_UFREE, (uint32_t)((c & 1) ^ 1));
-            tc_fence_before();
-            if (bar_named_or(BAR_PREP, NPREP, !uok)) {
-                ok = false;
-                break;
-            }
+        if (tid == TCOPY) poll_tma(false, true);  // v must be on its way before the hand-off
+        tc_fence_before();
+        bar_named(BAR_PREP, NPREP);
+        // the slot is complete but for W: the chain issues the W and U' products (after the
+        // v tile has landed) and stages W itself
+        if (tid == 0) {
+            mbar_arrive(bar + B_FULL + s);
+            TRACE(0, c, 5);
         }
-        if (tid == 0) TRACE(0, c, 5);
         if (tid == TCOPY) {
             if (CACHE) {  // the chunk's T diag(beta), complete since the barrier, into its entry,
                           // then the slot's images but W (the chain writes W after the hand-off)
@@ -1049,26 +1043,6 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
             poll_tma(true, true);  // the next chunk's k (and q, v) must be on their way
         }
 
-        // ============ W^T = KG^T TB^T ; U'^T = V^T TB^T   (M=128, N=64, K=64)
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t kg = smem_u32(sm + L::KG), tbb = smem_u32(sm + L::TB),
-                           vv = smem_u32(slot + L::S_W);
-            constexpr uint32_t id = idesc_bf16(128, 64, true, false);
-#pragma unroll
-            for (int st = 0; st < 4; ++st)
-                mma_bf16(x.tmem + TM_W, mnmajor_desc(kg, 64, st), kmajor_desc(tbb, 64, st), id, st > 0);
-#pragma unroll
-            for (int st = 0; st < 4; ++st)
-                mma_bf16(x.tmem + TM_U, mnmajor_desc(vv, 64, st), kmajor_desc(tbb, 64, st), id, st > 0);
-            mma_commit(bar + B_WU);
-            wu_out = true;
-            wu_par = (uint32_t)(c & 1);
-            // the slot is complete but for W, which the chain stages from TMEM itself once
-            // the products are done: hand it over now
-            mbar_arrive(bar + B_FULL + s);
-            TRACE(0, c, 7);
-        }
     }
     if (CACHE && tid == TCOPY) {
         // the last chunk's W image, then every cache entry is written
@@ -1079,10 +1053,7 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
         bulk_wait_all();
     }
     // after a timeout: bounded waits for what may still be in flight
-    if (!ok && tid == 0) {
-        if (ap_out) wait_bar(bar + B_AP, ap_par);
-        if (wu_out) wait_bar(bar + B_WU, wu_par);
-    }
+    if (!ok && tid == 0 && ap_out) wait_bar(bar + B_AP, ap_par);
     if (!ok && tid == TCOPY) {
         for (int vs = 0; vs < 2; ++vs)
             if (v_out[vs]) wait_bar(v_bar(bar, vs), v_par[vs]);
@@ -1092,12 +1063,34 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
 }
 
 // ---------------------------------------------------------------- chain: forward (warps 8-11)
-// Chain warps, at the start of chunk c (its slot full): wait for the prep's W product and
-// write W^T (TMEM, lane = channel) into the slot's W piece as the bf16 MN-major image (K rows
-// = channels) that the chain's U product reads.  The W piece held the chunk's v tile, which
-// the prep's U' product (committed with W) has read.  The caller's next named barrier makes
-// the image visible to the chain's products; ct == 0 then arrives on B_WREAD.
-__device__ bool chain_stage_w(const Ctx& x, uint8_t* slot_w, int64_t c, int ct) {
+// Chain warps, at the start of chunk c (its slot full): thread ct == 0 waits for the chunk's
+// v tile and issues W^T = KG^T (T diag(beta))^T and U'^T = V^T (T diag(beta))^T (M=128,
+// N=64, K=64) from the prep's KG and TB buffers and the v tile in the slot's W piece (the U
+// columns are free: this chain read the previous chunk's U before it got here); then all
+// wait for the two products and write W^T (TMEM, lane = channel) into the slot's W piece as
+// the bf16 MN-major image (K rows = channels) that the chain's U product reads.  The
+// caller's next named barrier makes the image visible to the chain's products; ct == 0 then
+// arrives on B_WREAD.  last_bar / last_par: the commit ct == 0 issued, for the waits after a
+// timeout.
+template <int MODE>
+__device__ bool chain_stage_w(const Ctx& x, uint8_t* slot, int64_t c, int ct, int& last_bar,
+                              uint32_t& last_par) {
+    using L = Lay<MODE>;
+    if (ct == 0 && wait_bar(v_bar(x.bar, (int)(c & 1)), (uint32_t)((c >> 1) & 1))) {
+        tc_fence_after();
+        const uint32_t kg = smem_u32(x.sm + L::KG), tbb = smem_u32(x.sm + L::TB),
+                       vv = smem_u32(slot + L::S_W);
+        constexpr uint32_t id = idesc_bf16(128, 64, true, false);
+#pragma unroll
+        for (int st = 0; st < 4; ++st)
+            mma_bf16(x.tmem + TM_W, mnmajor_desc(kg, 64, st), kmajor_desc(tbb, 64, st), id, st > 0);
+#pragma unroll
+        for (int st = 0; st < 4; ++st)
+            mma_bf16(x.tmem + TM_U, mnmajor_desc(vv, 64, st), kmajor_desc(tbb, 64, st), id, st > 0);
+        mma_commit(x.bar + B_WU);
+        last_bar = B_WU;
+        last_par = (uint32_t)(c & 1);
+    }
     if (!wait_bar(x.bar + B_WU, (uint32_t)(c & 1))) return false;
     tc_fence_after();
     const int cw = ct >> 5, chn = (cw & 3) * 32 + (ct & 31), r0 = 32 * (cw >> 2);
@@ -1107,7 +1100,7 @@ __device__ bool chain_stage_w(const Ctx& x, uint8_t* slot_w, int64_t c, int ct) 
     tmem_ld16(tq + TM_W + r0 + 16, v1);
     tmem_wait16(v0);
     tmem_wait16(v1);
-    const uint32_t wb = smem_u32(slot_w);
+    const uint32_t wb = smem_u32(slot + L::S_W);
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
         const float* p = k < 2 ? v0 + 8 * k : v1 + 8 * (k - 2);
@@ -1235,7 +1228,7 @@ __device__ void chain_fwd(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
         s_waited = true;
         tc_fence_after();
         if (ct == 0) TRACE(1, c, 1);
-        wok = wok && chain_stage_w(x, slot + L::S_W, c, ct);
+        wok = wok && chain_stage_w<FWD>(x, slot, c, ct, last_bar, last_par);
         if (wok) {  // bf16 S^T -> SB; S^T *= gamma (per column = key channel) in place
             const float* gam = reinterpret_cast<const float*>(slot + L::S_GAM);
             stage_cols_tmem<4>(tq + TM_S + 64 * ch, tq + TM_SB + 32 * ch, 64 * ch, gam, true);
@@ -1292,7 +1285,6 @@ __device__ void chain_fwd(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
         bar_named(BAR_CHAIN, NCHAIN);
         if (ct == 0) {
             TRACE(1, c, 5);
-            mbar_arrive(bar + B_UFREE);  // the prep may write the next U'
             tc_fence_after();
             const uint32_t kd = smem_u32(slot + L::S_KD), pb = smem_u32(slot + L::S_PB);
             constexpr uint32_t id_s = idesc_bf16(128, 128, false, true);
@@ -1405,7 +1397,7 @@ __device__ void chain_trans(const Ctx& x, const TcArgs& a, int tid) {
         if (c > 0) wok = wok && wait_bar(bar + B_S, (uint32_t)((c - 1) & 1));
         tc_fence_after();
         if (ct == 0) TRACE(1, c, 1);
-        wok = wok && chain_stage_w(x, slot + L::S_W, c, ct);
+        wok = wok && chain_stage_w<MODE>(x, slot, c, ct, last_bar, last_par);
         for (int step = 0; step < 2 && ok; ++step) {  // 0: B, 1: M
             const uint32_t tstate = step == 0 ? TT_B : TT_M;
             if (wok) {
@@ -1443,7 +1435,6 @@ __device__ void chain_trans(const Ctx& x, const TcArgs& a, int tid) {
             bar_named(BAR_CHAIN, NCHAIN);
             if (ct == 0) {
                 TRACE(1, c, 4 + 3 * step);
-                if (step == 1) mbar_arrive(bar + B_UFREE);
                 tc_fence_after();
                 // state^T += U^T K_dec
 #pragma unroll
@@ -1489,13 +1480,19 @@ __device__ void chain_dump(const Ctx& x, const TcArgs& a, int tid) {
     const int ct = tid - NPREP, cw = ct >> 5, ch = cw >> 2, e = (cw & 3) * 32 + (ct & 31);
     const uint32_t tq = x.tmem + ((uint32_t)((cw & 3) * 32) << 16);
     const int h = x.h, H = a.H;
-    for (int64_t c = 0; c < x.nc; ++c) {
+    int last_bar = -1;  // thread ct == 0: the last commit issued, for the wait after a timeout
+    uint32_t last_par = 0;
+    bool ok = true;
+    for (int64_t c = 0; c < x.nc && ok; ++c) {
         const int s = (int)(c & 1);
         uint8_t* slot = sm + s * L::SLOT;
         bool wok = wait_bar(bar + B_FULL + s, (uint32_t)((c >> 1) & 1));
-        wok = wok && chain_stage_w(x, slot + L::S_W, c, ct);
+        wok = wok && chain_stage_w<DUMP>(x, slot, c, ct, last_bar, last_par);
         tc_fence_before();
-        if (bar_named_or(BAR_CHAIN, NCHAIN, !wok)) break;
+        if (bar_named_or(BAR_CHAIN, NCHAIN, !wok)) {
+            ok = false;
+            break;
+        }
         if (ct == 0) mbar_arrive(bar + B_WREAD);
         tc_fence_after();
         uint8_t* ent = a.dump + ((x.sg.c_base + c) * H + h) * (int64_t)kChunkImageBytes;
@@ -1529,11 +1526,11 @@ __device__ void chain_dump(const Ctx& x, const TcArgs& a, int tid) {
         tc_fence_before();
         bar_named(BAR_CHAIN, NCHAIN);
         if (ct == 0) {
-            mbar_arrive(bar + B_UFREE);
             mbar_arrive(bar + B_EMPTY + s);
             mbar_arrive(bar + B_WFREE + s);
         }
     }
+    if (!ok && ct == 0 && last_bar >= 0) wait_bar(bar + last_bar, last_par);
 }
 
 // ---------------------------------------------------------------- the kernel

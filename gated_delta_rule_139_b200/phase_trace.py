@@ -22,8 +22,8 @@ import numpy as np
 PREP = {14: "raw tiles landed", 1: "gate prefix sums", 2: "operand images", 3: "[A;P] product",
         8: "inv: A from TMEM", 9: "inv: diagonal blocks", 10: "inv: T_21 in halves",
         11: "inv: barrier", 12: "inv: Z = A_21 T_lo", 4: "inv: T_hi Z into TB",
-        5: "v landed, U free", 7: "W, U' issued; slot out"}
-CHAIN_TRANS = {1: "slot full", 2: "W image, B: state staged", 3: "B: U product", 4: "B: U staged",
+        5: "slot handed to the chain"}
+CHAIN_TRANS = {1: "slot full", 2: "W, U' products, W image, B staged", 3: "B: U product", 4: "B: U staged",
                5: "M: state staged", 6: "M: U product", 7: "M: U staged"}
 
 
