@@ -1012,7 +1012,13 @@ __device__ void prep_loop(const Ctx& x, const TcArgs& a, const TcMaps& maps, int
                         la_out = true;
                         la_par = (uint32_t)((c + 1) & 1);
                     }
-                    poll_tma(false, false);
+                    // the chain usually frees the next slot during this phase: keep polling
+                    // for it a bounded while (warps 0-1 have longer work before the next
+                    // barrier), so that its tiles go out now rather than after the hand-off
+                    const long long poll_end = clock64() + 1500;
+                    do {
+                        poll_tma(false, false);
+                    } while (!kq_next && clock64() < poll_end);
                     if (c + 3 < x.nc) prefetch_chunk<Q>(maps, h, (int)(t0 + 3 * C));
                 }
             }, c);
